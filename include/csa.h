@@ -1,0 +1,200 @@
+/*
+ * csa.h -- C ABI of libcsa, a B200 (sm_100a) library for the hybrid attention
+ * of DeepSeek-V4: Compressed Sparse Attention (CSA) and Heavily Compressed
+ * Attention (HCA).
+ *
+ * Method source: the DeepSeek-V4 paper summary on hyper.ai (papers/2606.19348),
+ * section "方法" (Method) -- the CSA paragraph (compression of every m tokens
+ * with learnable weights and a position bias, a "lightning indexer" selecting
+ * the top-k compressed entries, MQA with shared key and value), the HCA
+ * paragraph (m' >> m tokens per entry without overlap, dense attention, and a
+ * sliding-window branch in both), and the storage paragraph (RoPE dims in BF16,
+ * the rest in FP8).  The DeepSeek-V4-Pro model cards (Hugging Face,
+ * "Introduction", item 1 "hybrid attention architecture") state the same
+ * CSA + HCA combination.
+ *
+ * Conventions (all entry points):
+ *   - Every array argument is DEVICE memory owned by the caller, dense
+ *     row-major in the shape given, and 16-byte aligned.  Structs passed by
+ *     pointer (csa_kv_cache, csa_window) live in HOST memory; the pointers
+ *     inside them are device pointers.  The library never allocates; scratch
+ *     memory is queried with the *_workspace_size call and passed in.
+ *   - bf16 = IEEE bfloat16; e4m3 = OCP FP8 E4M3 (bias 7, max 448, no inf).
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL means
+ *     the legacy default stream).  Argument and shape errors are detected on
+ *     the host before anything is enqueued and returned synchronously; a
+ *     kernel launch failure returns CSA_ERR_CUDA.  Faults inside an enqueued
+ *     kernel surface at the caller's next synchronisation, as for any CUDA
+ *     work.  csa_last_error() gives a message for the last failing call of
+ *     the calling thread.
+ *   - Positions are 0-based.  Entry i of a compression with stride s has
+ *     nominal end e_i = (i+1)*s - 1; a query at position t sees entry i iff
+ *     e_i <= t.  The sliding window of a query at t is the raw tokens at
+ *     positions [max(0, t-win_len+1), t].  Entries and window keys share one
+ *     softmax per head.
+ *   - Fixed head geometry: qk dim 192 (128 "nope" + 64 RoPE channels), v dim
+ *     128, indexer 4 heads x 64.  Query heads H must be 16 or 64.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA_API __attribute__((visibility("default")))
+#else
+#define CSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSA_D_QK 192
+#define CSA_D_NOPE 128
+#define CSA_D_ROPE 64
+#define CSA_D_V 128
+#define CSA_H_I 4
+#define CSA_D_I 64
+
+typedef enum csa_status {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or shape   */
+  CSA_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels support   */
+  CSA_ERR_WORKSPACE = 3,     /* workspace pointer NULL or smaller than asked */
+  CSA_ERR_CUDA = 4           /* a CUDA runtime call or launch failed         */
+} csa_status;
+
+typedef enum csa_kv_layout {
+  /* k: bf16 [B, N, 192]; v: bf16 [B, N, 128], or NULL to use k[..., :128] */
+  CSA_KV_BF16 = 0,
+  /* split storage: nope e4m3 [B, N, 128], rope bf16 [B, N, 64], scale fp32
+   * [B, N]; key = (nope * scale) ++ rope, value = nope * scale (shared K/V) */
+  CSA_KV_SPLIT_FP8 = 1
+} csa_kv_layout;
+
+/* A compressed KV cache (host struct; device pointers). */
+typedef struct csa_kv_cache {
+  int32_t layout;            /* csa_kv_layout */
+  int32_t reserved;          /* must be 0 */
+  int64_t n_entries;         /* N, entries per sequence */
+  const void* k;             /* CSA_KV_BF16 */
+  const void* v;             /* CSA_KV_BF16, nullable */
+  const uint8_t* nope;       /* CSA_KV_SPLIT_FP8 */
+  const void* rope;          /* CSA_KV_SPLIT_FP8 */
+  const float* scale;        /* CSA_KV_SPLIT_FP8 */
+} csa_kv_cache;
+
+/* Raw (uncompressed) tokens for the sliding-window branch (host struct). */
+typedef struct csa_window {
+  const void* k;             /* bf16 [B, rows, 192] */
+  const void* v;             /* bf16 [B, rows, 128], or NULL to use k[..., :128] */
+  int64_t pos0;              /* position of row 0 */
+  int64_t rows;              /* rows held per sequence */
+  int32_t len;               /* window length w_s (0 disables the branch) */
+  int32_t reserved;          /* must be 0 */
+} csa_window;
+
+/* Library version string, e.g. "csa-b200 0.1.0 sm_100a". */
+CSA_API const char* csa_version(void);
+/* Name of a status code. */
+CSA_API const char* csa_status_string(int32_t status);
+/* Message for the last failing call made by this thread ("" if none). */
+CSA_API const char* csa_last_error(void);
+
+/*
+ * csa_compress -- CSA KV compression (Method section, CSA paragraph: every m
+ * tokens become one entry through learnable compression weights and a position
+ * bias; the windows overlap, in contrast to HCA's non-overlapping ones).
+ *
+ * Entry i (i < N = ceil(T/m)) covers the 2m tokens [(i-1)m, (i+1)m) clipped to
+ * [0, T); for each channel c:
+ *     alpha_j = softmax_j( w[c] * x[j,c] + b_pos[j - (i-1)m, c] )   (in-range j)
+ *     y[i,c]  = sum_j alpha_j * x[j,c]
+ *   x       bf16 [B, T, d], d a multiple of 8 in [8, 256]
+ *   w       fp32 [d];  b_pos fp32 [2m, d]
+ *   out_layout CSA_KV_BF16:      out = bf16 [B, N, d]   (out_rope, out_scale unused)
+ *   out_layout CSA_KV_SPLIT_FP8: requires d == 192; out = e4m3 [B, N, 128],
+ *       out_rope = bf16 [B, N, 64], out_scale = fp32 [B, N] with scale =
+ *       max|y[:128]| / 448 (1 if zero) and codes = RNE-satfinite(y / scale).
+ *   1 <= m <= 64.  T == 0 is a no-op.
+ */
+CSA_API csa_status csa_compress(const void* x, int64_t B, int64_t T, int32_t d, int32_t m,
+                        const float* w, const float* b_pos, int32_t out_layout,
+                        void* out, void* out_rope, float* out_scale, void* stream);
+
+/*
+ * hca_compress -- HCA KV compression (Method section, HCA paragraph: m' >> m
+ * tokens per entry, no overlap).  Entry i covers [i m', (i+1) m') clipped to
+ * [0, T) (the trailing entry may be partial); same per-channel softmax as
+ * csa_compress with b_pos fp32 [m', d].  N = ceil(T/m'), 1 <= m' <= 4096.
+ * Arguments and layouts as csa_compress.
+ */
+CSA_API csa_status hca_compress(const void* x, int64_t B, int64_t T, int32_t d, int32_t m_prime,
+                        const float* w, const float* b_pos, int32_t out_layout,
+                        void* out, void* out_rope, float* out_scale, void* stream);
+
+/* Workspace bytes csa_indexer_topk needs for these sizes. */
+CSA_API size_t csa_indexer_topk_workspace_size(int64_t B, int64_t Tq, int64_t N, int32_t k);
+
+/*
+ * csa_indexer_topk -- the lightning indexer and its top-k selection (Method
+ * section, CSA paragraph).  For query row r of sequence b at position
+ * t = q_pos0 + r and every visible entry i (e_i = (i+1)m - 1 <= t):
+ *     s[i] = sum_{h<4} relu(qI[b,r,h,:] . kIc[b,i,:]) * wI[b,r,h]
+ * and idx[b,r,:] receives the k entries with the highest scores, ties broken
+ * toward the lower index, as an ascending list padded with -1 when fewer than
+ * k entries are visible.
+ *   qI  bf16 [B, Tq, 4, 64];  wI fp32 [B, Tq, 4];  kIc bf16 [B, N, 64]
+ *   idx int32 [B, Tq, k] (output)
+ *   1 <= k <= 4096, 1 <= m, q_pos0 >= 0, N < 2^31.
+ */
+CSA_API csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc,
+                            int64_t B, int64_t Tq, int64_t N, int64_t q_pos0, int32_t m,
+                            int32_t k, int32_t* idx, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Workspace bytes csa_sparse_mqa needs for these sizes. */
+CSA_API size_t csa_sparse_mqa_workspace_size(int64_t B, int64_t Tq, int32_t H, int32_t k, int32_t win_len);
+
+/*
+ * csa_sparse_mqa -- CSA core attention (Method section, CSA paragraph: MQA with
+ * one key/value head shared by all query heads, over the selected entries; HCA
+ * paragraph: plus a sliding-window branch of raw recent tokens).  For query
+ * row r of sequence b at t = q_pos0 + r and each head h, one softmax over
+ *     { scale * q[b,r,h] . K_entry(i) : i in idx[b,r,:], 0 <= i < N, e_i <= t }
+ *   u { scale * q[b,r,h] . K_raw(p)   : p in [max(0,t-win_len+1), t] }
+ * and out = sum of probabilities times the matching values.
+ *   q     bf16 [B, Tq, H, 192]
+ *   cache compressed entries (either layout), N = cache->n_entries
+ *   idx   int32 [B, Tq, k] (slots that are -1, out of range or not visible
+ *         are skipped)
+ *   win   raw tokens; must hold every window position of every query
+ *   out   bf16 [B, Tq, H, 128];  lse fp32 [B, Tq, H] natural-log
+ *         log-sum-exp of the scaled logits (nullable).  A query with no keys
+ *         gets out = 0 and lse = -inf.
+ */
+CSA_API csa_status csa_sparse_mqa(const void* q, int64_t B, int64_t Tq, int32_t H, int64_t q_pos0,
+                          const csa_kv_cache* cache, int32_t m, const int32_t* idx, int32_t k,
+                          const csa_window* win, float scale, void* out, float* lse,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes hca_dense_mqa needs for these sizes. */
+CSA_API size_t hca_dense_mqa_workspace_size(int64_t B, int64_t Tq, int32_t H, int64_t N, int32_t win_len);
+
+/*
+ * hca_dense_mqa -- HCA core attention (Method section, HCA paragraph: dense
+ * attention over all heavily compressed entries, no selection, plus the same
+ * sliding window).  As csa_sparse_mqa with the entry set replaced by every
+ * visible entry i < N (e_i = (i+1)m' - 1 <= t).
+ */
+CSA_API csa_status hca_dense_mqa(const void* q, int64_t B, int64_t Tq, int32_t H, int64_t q_pos0,
+                         const csa_kv_cache* cache, int32_t m_prime, const csa_window* win,
+                         float scale, void* out, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H_ */

@@ -1,1 +1,213 @@
-"""B200-native CSA / HCA hybrid attention (placeholder; binding added with the library)."""
+"""B200-native Compressed Sparse Attention (CSA) and Heavily Compressed Attention (HCA).
+
+Thin Python binding over the C ABI of ``libcsa.so`` (declared in include/csa.h).
+Every function here only checks tensor metadata, allocates outputs and scratch
+with torch (device memory is torch's job here) and calls the library entry point
+of the same name; all arithmetic runs in the library's CUDA kernels.  There is
+no CPU or PyTorch fallback: a missing library raises.
+
+Shapes (B sequences, Tq query rows, N entries, H heads in {16, 64}):
+  csa_compress / hca_compress: x bf16 [B, T, d] -> bf16 [B, N, d], or with
+      ``fp8=True`` (d == 192) the split cache (nope e4m3 as uint8 [B, N, 128],
+      rope bf16 [B, N, 64], scale fp32 [B, N]).
+  csa_indexer_topk: qI bf16 [B, Tq, 4, 64], wI fp32 [B, Tq, 4], kIc bf16
+      [B, N, 64] -> idx int32 [B, Tq, k] (ascending, -1 padded).
+  csa_sparse_mqa / hca_dense_mqa: q bf16 [B, Tq, H, 192] -> (out bf16
+      [B, Tq, H, 128], lse fp32 [B, Tq, H]).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+
+import torch
+
+from . import _lib
+
+__all__ = ["CsaError", "KVCache", "Window", "csa_compress", "hca_compress", "csa_indexer_topk",
+           "csa_indexer_topk_workspace_size", "csa_sparse_mqa", "csa_sparse_mqa_workspace_size", "hca_dense_mqa",
+           "hca_dense_mqa_workspace_size", "version"]
+
+
+class CsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _lib.load()
+        msg = lib.csa_last_error().decode()
+        super().__init__(f"{where}: {lib.csa_status_string(status).decode()} ({msg})")
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != _lib.CSA_OK:
+        raise CsaError(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def version() -> str:
+    return _lib.load().csa_version().decode()
+
+
+@dataclasses.dataclass
+class KVCache:
+    """A compressed cache: bf16 (k, optional v) or split FP8 (nope, rope, scale)."""
+    k: torch.Tensor | None = None
+    v: torch.Tensor | None = None
+    nope: torch.Tensor | None = None
+    rope: torch.Tensor | None = None
+    scale: torch.Tensor | None = None
+
+    @property
+    def split(self) -> bool:
+        return self.nope is not None
+
+    @property
+    def n_entries(self) -> int:
+        return (self.nope if self.split else self.k).shape[1]
+
+    def desc(self) -> _lib.KVCacheDesc:
+        d = _lib.KVCacheDesc()
+        d.layout = _lib.CSA_KV_SPLIT_FP8 if self.split else _lib.CSA_KV_BF16
+        d.reserved = 0
+        d.n_entries = self.n_entries
+        d.k, d.v = _ptr(self.k), _ptr(self.v)
+        d.nope, d.rope, d.scale = _ptr(self.nope), _ptr(self.rope), _ptr(self.scale)
+        return d
+
+
+@dataclasses.dataclass
+class Window:
+    """Raw tokens for the sliding-window branch: rows hold positions pos0, pos0+1, ..."""
+    k: torch.Tensor | None
+    v: torch.Tensor | None = None
+    pos0: int = 0
+    length: int = 128
+
+    def desc(self) -> _lib.WindowDesc:
+        d = _lib.WindowDesc()
+        d.k, d.v = _ptr(self.k), _ptr(self.v)
+        d.pos0 = self.pos0
+        d.rows = 0 if self.k is None else self.k.shape[1]
+        d.len = self.length
+        d.reserved = 0
+        return d
+
+
+def _compress(fn_name, x, w, b_pos, stride, fp8, out, stream):
+    lib = _lib.load()
+    B, T, d = x.shape
+    N = -(-T // stride)
+    if fp8:
+        nope, rope, scale = out if out is not None else (
+            torch.empty(B, N, 128, dtype=torch.uint8, device=x.device),
+            torch.empty(B, N, 64, dtype=torch.bfloat16, device=x.device),
+            torch.empty(B, N, dtype=torch.float32, device=x.device))
+        st = getattr(lib, fn_name)(_ptr(x), B, T, d, stride, _ptr(w), _ptr(b_pos), _lib.CSA_KV_SPLIT_FP8,
+                                   _ptr(nope), _ptr(rope), _ptr(scale), _stream(stream))
+        _check(st, fn_name)
+        return nope, rope, scale
+    y = out if out is not None else torch.empty(B, N, d, dtype=torch.bfloat16, device=x.device)
+    st = getattr(lib, fn_name)(_ptr(x), B, T, d, stride, _ptr(w), _ptr(b_pos), _lib.CSA_KV_BF16, _ptr(y), None,
+                               None, _stream(stream))
+    _check(st, fn_name)
+    return y
+
+
+def csa_compress(x, w, b_pos, m, *, fp8=False, out=None, stream=None):
+    """CSA compression: overlapping 2m-token windows with stride m."""
+    return _compress("csa_compress", x, w, b_pos, m, fp8, out, stream)
+
+
+def hca_compress(x, w, b_pos, m_prime, *, fp8=False, out=None, stream=None):
+    """HCA compression: non-overlapping m'-token windows."""
+    return _compress("hca_compress", x, w, b_pos, m_prime, fp8, out, stream)
+
+
+def csa_indexer_topk_workspace_size(B, Tq, N, k) -> int:
+    return int(_lib.load().csa_indexer_topk_workspace_size(B, Tq, N, k))
+
+
+def csa_indexer_topk(qI, wI, kIc, m, k, *, q_pos0=0, idx=None, workspace=None, stream=None):
+    """Lightning-indexer scores and top-k entry ids (int32 [B, Tq, k], ascending, -1 padded)."""
+    lib = _lib.load()
+    B, Tq = qI.shape[0], qI.shape[1]
+    N = kIc.shape[1]
+    if idx is None:
+        idx = torch.empty(B, Tq, k, dtype=torch.int32, device=qI.device)
+    need = csa_indexer_topk_workspace_size(B, Tq, N, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=qI.device)
+    st = lib.csa_indexer_topk(_ptr(qI), _ptr(wI), _ptr(kIc), B, Tq, N, q_pos0, m, k, _ptr(idx), _ptr(workspace),
+                              workspace.numel(), _stream(stream))
+    _check(st, "csa_indexer_topk")
+    return idx
+
+
+def csa_sparse_mqa_workspace_size(B, Tq, H, k, win_len) -> int:
+    return int(_lib.load().csa_sparse_mqa_workspace_size(B, Tq, H, k, win_len))
+
+
+def hca_dense_mqa_workspace_size(B, Tq, H, N, win_len) -> int:
+    return int(_lib.load().hca_dense_mqa_workspace_size(B, Tq, H, N, win_len))
+
+
+def _attn_out(q, out, lse):
+    B, Tq, H, _ = q.shape
+    if out is None:
+        out = torch.empty(B, Tq, H, 128, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, Tq, H, dtype=torch.float32, device=q.device)
+    return out, lse
+
+
+def csa_sparse_mqa(q, cache: KVCache, m, idx, win: Window | None, scale, *, q_pos0=0, out=None, lse=None,
+                   workspace=None, stream=None):
+    """CSA core attention over the selected entries plus the sliding window (one softmax)."""
+    lib = _lib.load()
+    B, Tq, H, _ = q.shape
+    k = idx.shape[-1]
+    out, lse = _attn_out(q, out, lse)
+    wlen = win.length if win is not None else 0
+    need = csa_sparse_mqa_workspace_size(B, Tq, H, k, wlen)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    cd = cache.desc()
+    wd = win.desc() if win is not None else None
+    st = lib.csa_sparse_mqa(_ptr(q), B, Tq, H, q_pos0, ctypes.byref(cd), m, _ptr(idx), k,
+                            ctypes.byref(wd) if wd is not None else None, float(scale), _ptr(out), _ptr(lse),
+                            _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
+    _check(st, "csa_sparse_mqa")
+    return out, lse
+
+
+def hca_dense_mqa(q, cache: KVCache, m_prime, win: Window | None, scale, *, q_pos0=0, out=None, lse=None,
+                  workspace=None, stream=None):
+    """HCA core attention over every visible entry plus the sliding window (one softmax)."""
+    lib = _lib.load()
+    B, Tq, H, _ = q.shape
+    out, lse = _attn_out(q, out, lse)
+    wlen = win.length if win is not None else 0
+    need = hca_dense_mqa_workspace_size(B, Tq, H, cache.n_entries, wlen)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    cd = cache.desc()
+    wd = win.desc() if win is not None else None
+    st = lib.hca_dense_mqa(_ptr(q), B, Tq, H, q_pos0, ctypes.byref(cd), m_prime,
+                           ctypes.byref(wd) if wd is not None else None, float(scale), _ptr(out), _ptr(lse),
+                           _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
+    _check(st, "hca_dense_mqa")
+    return out, lse

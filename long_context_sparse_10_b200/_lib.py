@@ -1,0 +1,64 @@
+"""ctypes declarations of the libcsa C ABI (include/csa.h)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+c_i32, c_i64, c_f32, c_sz, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
+
+CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUDA = 0, 1, 2, 3, 4
+CSA_KV_BF16, CSA_KV_SPLIT_FP8 = 0, 1
+
+# every symbol include/csa.h declares, with (restype, argtypes)
+SIGNATURES = {
+    "csa_version": (ctypes.c_char_p, []),
+    "csa_status_string": (ctypes.c_char_p, [c_i32]),
+    "csa_last_error": (ctypes.c_char_p, []),
+    "csa_compress": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
+    "hca_compress": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
+    "csa_indexer_topk_workspace_size": (c_sz, [c_i64, c_i64, c_i64, c_i32]),
+    "csa_indexer_topk": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_sz,
+                                 c_vp]),
+    "csa_sparse_mqa_workspace_size": (c_sz, [c_i64, c_i64, c_i32, c_i32, c_i32]),
+    "csa_sparse_mqa": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i64, c_vp, c_i32, c_vp, c_i32, c_vp, c_f32, c_vp, c_vp,
+                               c_vp, c_sz, c_vp]),
+    "hca_dense_mqa_workspace_size": (c_sz, [c_i64, c_i64, c_i32, c_i64, c_i32]),
+    "hca_dense_mqa": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i64, c_vp, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_sz,
+                              c_vp]),
+}
+
+
+class KVCacheDesc(ctypes.Structure):
+    """csa_kv_cache."""
+    _fields_ = [("layout", c_i32), ("reserved", c_i32), ("n_entries", c_i64), ("k", c_vp), ("v", c_vp),
+                ("nope", c_vp), ("rope", c_vp), ("scale", c_vp)]
+
+
+class WindowDesc(ctypes.Structure):
+    """csa_window."""
+    _fields_ = [("k", c_vp), ("v", c_vp), ("pos0", c_i64), ("rows", c_i64), ("len", c_i32), ("reserved", c_i32)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libcsa.so (once).  Raises if it has not been built: there is no fallback."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(f"libcsa.so not found at {path}; build it with "
+                                   "`python -m long_context_sparse_10_b200.build` (nvcc, sm_100a)")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+        return _lib

@@ -1,0 +1,60 @@
+// Library-wide entry points: version, status names, per-thread error text.
+#include <cstdarg>
+#include <cstdio>
+
+#include "host_util.h"
+
+namespace {
+thread_local char g_msg[512] = "";
+int g_sms[64] = {0};
+}  // namespace
+
+namespace csa {
+
+csa_status fail(csa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+void clear_error() { g_msg[0] = '\0'; }
+
+csa_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return CSA_OK;
+}
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (g_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+}  // namespace csa
+
+extern "C" {
+
+const char* csa_version(void) { return "csa-b200 0.1.0 sm_100a"; }
+
+const char* csa_status_string(int32_t s) {
+  switch (s) {
+    case CSA_OK: return "CSA_OK";
+    case CSA_ERR_INVALID_ARG: return "CSA_ERR_INVALID_ARG";
+    case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED";
+    case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE";
+    case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
+    default: return "CSA_ERR_UNKNOWN";
+  }
+}
+
+const char* csa_last_error(void) { return g_msg; }
+
+}  // extern "C"

@@ -1,0 +1,268 @@
+// KV compression for CSA (overlapping 2m-token windows, stride m) and HCA
+// (non-overlapping m'-token windows).
+//
+// DeepSeek-V4 paper summary (hyper.ai), section "Method": CSA compresses every m
+// tokens of the KV cache into one entry using learnable compression weights and
+// a position bias; HCA merges every m' >> m tokens into one entry without
+// overlapping compression.  Per channel c of entry i with window start s:
+//   alpha_j = softmax over in-range j of (w[c] x[j,c] + b[j - s, c]),
+//   y[i,c]  = sum_j alpha_j x[j,c].
+// The softmax runs online in fp32 (running max, rescaled sum and weighted sum).
+//
+// Memory bound: each lane owns 8 channels (one 16-byte load per token row), a
+// warp covers one entry's row (d <= 256).  Short windows (CSA) use one warp
+// per entry; long windows (HCA) spread the rows of one entry over 8 warps and
+// merge their softmax states in shared memory.
+#include "common.cuh"
+#include "host_util.h"
+
+namespace csa {
+namespace {
+
+struct CompressParams {
+  const __nv_bfloat16* x;
+  const float* w;
+  const float* b;
+  int64_t B, T, N;
+  int d, G;  // channels and 8-channel groups
+  int stride, cwin;
+  int layout;
+  void* out;
+  __nv_bfloat16* out_rope;
+  float* out_scale;
+};
+
+struct Acc8 {
+  float m[8], s[8], a[8];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      m[c] = -INFINITY;
+      s[c] = 0.f;
+      a[c] = 0.f;
+    }
+  }
+  __device__ __forceinline__ void add(const float* xv, const float* wv, const float* bv) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float l = fmaf(wv[c], xv[c], bv[c]);
+      float mn = fmaxf(m[c], l);
+      float corr = __expf(m[c] - mn);
+      float p = __expf(l - mn);
+      s[c] = fmaf(s[c], corr, p);
+      a[c] = fmaf(a[c], corr, p * xv[c]);
+      m[c] = mn;
+    }
+  }
+};
+
+__device__ __forceinline__ void unpack8(uint4 r, float* f) {
+  f[0] = bf16_lo(r.x); f[1] = bf16_hi(r.x);
+  f[2] = bf16_lo(r.y); f[3] = bf16_hi(r.y);
+  f[4] = bf16_lo(r.z); f[5] = bf16_hi(r.z);
+  f[6] = bf16_lo(r.w); f[7] = bf16_hi(r.w);
+}
+
+__device__ __forceinline__ void load8f(const float* p, float* f) {
+  float4 u = __ldg(reinterpret_cast<const float4*>(p));
+  float4 v = __ldg(reinterpret_cast<const float4*>(p + 4));
+  f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+  f[4] = v.x; f[5] = v.y; f[6] = v.z; f[7] = v.w;
+}
+
+// Writes entry (b, i).  Called by all 32 lanes; lane g < G holds channels
+// [8g, 8g+8) in y.
+__device__ __forceinline__ void store_entry(const CompressParams& p, int64_t b, int64_t i, int lane,
+                                            const float* y) {
+  const int64_t e = b * p.N + i;
+  if (p.layout == CSA_KV_BF16) {
+    if (lane < p.G) {
+      uint4 o;
+      o.x = pack_bf16x2(y[0], y[1]);
+      o.y = pack_bf16x2(y[2], y[3]);
+      o.z = pack_bf16x2(y[4], y[5]);
+      o.w = pack_bf16x2(y[6], y[7]);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + e * p.d + 8 * lane) = o;
+    }
+    return;
+  }
+  // split FP8 storage (d == 192): lanes 0..15 hold the 128 nope channels,
+  // lanes 16..23 the 64 RoPE channels.
+  float am = 0.f;
+  if (lane < 16) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) am = fmaxf(am, fabsf(y[c]));
+  }
+#pragma unroll
+  for (int o = 8; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const float scale = am > 0.f ? am / 448.0f : 1.0f;
+  if (lane < 16) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int c = 0; c < 4; c += 2) {
+      __nv_fp8x2_storage_t q0 =
+          __nv_cvt_float2_to_fp8x2(make_float2(y[c] / scale, y[c + 1] / scale), __NV_SATFINITE, __NV_E4M3);
+      lo |= static_cast<uint32_t>(q0) << (8 * c);
+      __nv_fp8x2_storage_t q1 = __nv_cvt_float2_to_fp8x2(make_float2(y[c + 4] / scale, y[c + 5] / scale),
+                                                         __NV_SATFINITE, __NV_E4M3);
+      hi |= static_cast<uint32_t>(q1) << (8 * c);
+    }
+    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.out) + e * kDNope + 8 * lane) = make_uint2(lo, hi);
+    if (lane == 0) p.out_scale[e] = scale;
+  } else if (lane < 24) {
+    uint4 o;
+    o.x = pack_bf16x2(y[0], y[1]);
+    o.y = pack_bf16x2(y[2], y[3]);
+    o.z = pack_bf16x2(y[4], y[5]);
+    o.w = pack_bf16x2(y[6], y[7]);
+    *reinterpret_cast<uint4*>(p.out_rope + e * kDRope + 8 * (lane - 16)) = o;
+  }
+}
+
+// One warp per entry (short windows).
+__global__ void __launch_bounds__(256) compress_short_kernel(CompressParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+  if (e >= p.B * p.N) return;
+  const int64_t b = e / p.N, i = e % p.N;
+  const int64_t start = i * p.stride - (p.cwin - p.stride);
+  const int64_t j0 = start > 0 ? start : 0;
+  const int64_t j1 = (start + p.cwin) < p.T ? (start + p.cwin) : p.T;
+  float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (lane < p.G) {
+    float wv[8];
+    load8f(p.w + 8 * lane, wv);
+    Acc8 acc;
+    acc.init();
+    const __nv_bfloat16* xb = p.x + b * p.T * p.d + 8 * lane;
+    for (int64_t j = j0; j < j1; ++j) {
+      float xv[8], bv[8];
+      unpack8(ldg_nc16(xb + j * p.d), xv);
+      load8f(p.b + (j - start) * p.d + 8 * lane, bv);
+      acc.add(xv, wv, bv);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) y[c] = acc.a[c] / acc.s[c];
+  }
+  store_entry(p, b, i, lane, y);
+}
+
+// One CTA per entry (long windows): 8 warps take interleaved rows, then warp 0
+// merges the 8 partial softmax states.
+__global__ void __launch_bounds__(256) compress_long_kernel(CompressParams p) {
+  __shared__ float st[8][3][8][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t e = blockIdx.x;
+  const int64_t b = e / p.N, i = e % p.N;
+  const int64_t start = i * p.stride - (p.cwin - p.stride);
+  const int64_t j0 = start > 0 ? start : 0;
+  const int64_t j1 = (start + p.cwin) < p.T ? (start + p.cwin) : p.T;
+  Acc8 acc;
+  acc.init();
+  if (lane < p.G) {
+    float wv[8];
+    load8f(p.w + 8 * lane, wv);
+    const __nv_bfloat16* xb = p.x + b * p.T * p.d + 8 * lane;
+#pragma unroll 4
+    for (int64_t j = j0 + warp; j < j1; j += 8) {
+      float xv[8], bv[8];
+      unpack8(ldg_nc16(xb + j * p.d), xv);
+      load8f(p.b + (j - start) * p.d + 8 * lane, bv);
+      acc.add(xv, wv, bv);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    st[warp][0][c][lane] = acc.m[c];
+    st[warp][1][c][lane] = acc.s[c];
+    st[warp][2][c][lane] = acc.a[c];
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  float y[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) M = fmaxf(M, st[w][0][c][lane]);
+    float S = 0.f, A = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      float f = __expf(st[w][0][c][lane] - M);
+      S = fmaf(st[w][1][c][lane], f, S);
+      A = fmaf(st[w][2][c][lane], f, A);
+    }
+    y[c] = lane < p.G ? A / S : 0.f;
+  }
+  store_entry(p, b, i, lane, y);
+}
+
+csa_status compress_impl(const char* name, const void* x, int64_t B, int64_t T, int32_t d, int32_t stride,
+                         int32_t cwin, const float* w, const float* b_pos, int32_t layout, void* out,
+                         void* out_rope, float* out_scale, void* stream) {
+  clear_error();
+  CSA_REQUIRE(B >= 0 && T >= 0, "%s: B and T must be >= 0", name);
+  CSA_REQUIRE(d >= 8 && d <= 256 && d % 8 == 0, "%s: d must be a multiple of 8 in [8, 256] (got %d)", name, d);
+  CSA_REQUIRE(layout == CSA_KV_BF16 || layout == CSA_KV_SPLIT_FP8, "%s: unknown out_layout %d", name, layout);
+  if (layout == CSA_KV_SPLIT_FP8 && d != kDQK)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: split FP8 output needs d == 192 (got %d)", name, d);
+  if (B == 0 || T == 0) return CSA_OK;
+  CSA_REQUIRE_PTR(x);
+  CSA_REQUIRE_PTR(w);
+  CSA_REQUIRE_PTR(b_pos);
+  CSA_REQUIRE_PTR(out);
+  if (layout == CSA_KV_SPLIT_FP8) {
+    CSA_REQUIRE_PTR(out_rope);
+    CSA_REQUIRE_PTR(out_scale);
+  }
+  CompressParams p;
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.w = w;
+  p.b = b_pos;
+  p.B = B;
+  p.T = T;
+  p.N = (T + stride - 1) / stride;
+  p.d = d;
+  p.G = d / 8;
+  p.stride = stride;
+  p.cwin = cwin;
+  p.layout = layout;
+  p.out = out;
+  p.out_rope = static_cast<__nv_bfloat16*>(out_rope);
+  p.out_scale = out_scale;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t entries = B * p.N;
+  if (cwin <= 32) {
+    const int64_t grid = (entries + 7) / 8;
+    CSA_REQUIRE(grid < (1LL << 31), "%s: too many entries", name);
+    compress_short_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(p);
+  } else {
+    CSA_REQUIRE(entries < (1LL << 31), "%s: too many entries", name);
+    compress_long_kernel<<<static_cast<unsigned>(entries), 256, 0, s>>>(p);
+  }
+  return check_launch(name);
+}
+
+}  // namespace
+}  // namespace csa
+
+extern "C" {
+
+csa_status csa_compress(const void* x, int64_t B, int64_t T, int32_t d, int32_t m, const float* w,
+                        const float* b_pos, int32_t out_layout, void* out, void* out_rope, float* out_scale,
+                        void* stream) {
+  if (m < 1 || m > 64) return csa::fail(CSA_ERR_INVALID_ARG, "csa_compress: m must be in [1, 64] (got %d)", m);
+  return csa::compress_impl("csa_compress", x, B, T, d, m, 2 * m, w, b_pos, out_layout, out, out_rope,
+                            out_scale, stream);
+}
+
+csa_status hca_compress(const void* x, int64_t B, int64_t T, int32_t d, int32_t m_prime, const float* w,
+                        const float* b_pos, int32_t out_layout, void* out, void* out_rope, float* out_scale,
+                        void* stream) {
+  if (m_prime < 1 || m_prime > 4096)
+    return csa::fail(CSA_ERR_INVALID_ARG, "hca_compress: m' must be in [1, 4096] (got %d)", m_prime);
+  return csa::compress_impl("hca_compress", x, B, T, d, m_prime, m_prime, w, b_pos, out_layout, out, out_rope,
+                            out_scale, stream);
+}
+
+}  // extern "C"

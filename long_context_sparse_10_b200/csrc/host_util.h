@@ -1,0 +1,34 @@
+// Host-side helpers shared by the entry points: argument checks, error text.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "csa.h"
+
+namespace csa {
+
+// Records a printf-style message for csa_last_error() and returns `s`.
+csa_status fail(csa_status s, const char* fmt, ...);
+// Clears the calling thread's message.
+void clear_error();
+// Maps a pending launch error (cudaGetLastError) to CSA_ERR_CUDA.
+csa_status check_launch(const char* what);
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace csa
+
+#define CSA_REQUIRE(cond, ...)                                   \
+  do {                                                           \
+    if (!(cond)) return ::csa::fail(CSA_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+#define CSA_REQUIRE_PTR(p)                                                        \
+  do {                                                                            \
+    if ((p) == nullptr) return ::csa::fail(CSA_ERR_INVALID_ARG, "%s is NULL", #p); \
+    if (!::csa::aligned16(p))                                                     \
+      return ::csa::fail(CSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p);  \
+  } while (0)
