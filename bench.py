@@ -1,0 +1,552 @@
+#!/usr/bin/env python
+"""Throughput of the CSA / HCA hot path on B200, one JSON line on rank 0.
+
+Default workload: hybrid decode at 1,048,576-token context, batch 8 per GPU:
+one CSA layer (lightning indexer + top-2048 over 262,144 compressed entries,
+sparse MQA over an FP8/BF16 split cache + a 128-token window) then one HCA
+layer (dense MQA over 8,192 heavily compressed entries + the window), 64 query
+heads, qk dim 192, v dim 128.  A step is that whole pass for one new token of
+every sequence; value = tokens (sequences x GPUs) per second.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own 8 sequences
+(weak scaling, no collective on the data path); time = max over ranks.
+``--impl reference`` times the float64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA/HCA attention tokens/s at 128K and 1M ctx; % of HBM / tensor-core peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="hybrid_decode_l1m")
+    ap.add_argument("--cpu-sample-s", type=float, default=12.0, help="host seconds for the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-reps", type=int, default=100, help="launches of the dominant kernel to average")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def profile_traffic(kernel: str, source: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.md")
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
+    for line in open(path):
+        m = re.match(r"\|\s*(\S+)\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]+)\s*\|", line)
+        if m and m.group(1) == kernel and m.group(3) == sha:
+            return float(m.group(2))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while a region runs."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.4)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def __exit__(self, *exc):
+        self.t1 = time.time()
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [l for (t, l) in self.lines if self.t0 <= t <= self.t1 + 0.06]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            parts = [x.strip() for x in r.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# decode workloads (CSA decode, hybrid CSA + HCA decode)
+# ---------------------------------------------------------------------------
+class DecodeRun:
+    def __init__(self, wl, rank, dev):
+        import torch
+        import long_context_sparse_10_b200 as csa
+        from long_context_sparse_10_b200 import synth
+        self.torch, self.csa, self.wl, self.dev = torch, csa, wl, dev
+        from long_context_sparse_10_b200 import replicas
+        self.host = synth.decode_inputs(wl, seed=0, batch=replicas.shard(rank, wl.B))
+        h = self.host
+        d = {k: v.to(dev) for k, v in h.items()}
+        self.d = d
+        B, L, H, k, m = wl.B, wl.L, wl.H, wl.k, wl.m
+        self.scale = 1.0 / math.sqrt(192)
+        self.q_pos0 = L - 1
+        self.cache = csa.KVCache(nope=d["nope"], rope=d["rope"], scale=d["scale"])
+        self.win = csa.Window(k=d["win_k"], pos0=L - wl.win, length=wl.win)
+        self.idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
+        self.ws_idx = torch.empty(max(1, csa.csa_indexer_topk_workspace_size(B, 1, wl.N, k)), dtype=torch.uint8,
+                                  device=dev)
+        nws = csa.csa_sparse_mqa_workspace_size(B, 1, H, k, wl.win)
+        self.ws_attn = torch.empty(max(1, nws), dtype=torch.uint8, device=dev)
+        self.out = torch.empty(B, 1, H, 128, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(B, 1, H, dtype=torch.float32, device=dev)
+        self.launches = 4 + (2 if nws else 1)
+        self.hybrid = wl.kind == "hybrid"
+        if self.hybrid:
+            self.hcache = csa.KVCache(nope=d["hca_nope"], rope=d["hca_rope"], scale=d["hca_scale"])
+            self.hwin = csa.Window(k=d["hca_win_k"], pos0=L - wl.win, length=wl.win)
+            hws = csa.hca_dense_mqa_workspace_size(B, 1, H, wl.N_hca, wl.win)
+            self.ws_hca = torch.empty(max(1, hws), dtype=torch.uint8, device=dev)
+            self.hout = torch.empty(B, 1, H, 128, dtype=torch.bfloat16, device=dev)
+            self.hlse = torch.empty(B, 1, H, dtype=torch.float32, device=dev)
+            self.launches += 2 if hws else 1
+        # pinned host buffers for the end-to-end measurement
+        self.h_in = {k: h[k].pin_memory() for k in (["q", "qI", "wI"] + (["hca_q"] if self.hybrid else []))}
+        self.h_out = [torch.empty_like(self.out, device="cpu").pin_memory()]
+        if self.hybrid:
+            self.h_out.append(torch.empty_like(self.hout, device="cpu").pin_memory())
+        self.tokens = B
+
+    def indexer(self):
+        wl = self.wl
+        self.csa.csa_indexer_topk(self.d["qI"], self.d["wI"], self.d["kIc"], wl.m, wl.k, q_pos0=self.q_pos0,
+                                  idx=self.idx, workspace=self.ws_idx)
+
+    def step(self):
+        wl, csa = self.wl, self.csa
+        self.indexer()
+        csa.csa_sparse_mqa(self.d["q"], self.cache, wl.m, self.idx, self.win, self.scale, q_pos0=self.q_pos0,
+                           out=self.out, lse=self.lse, workspace=self.ws_attn)
+        if self.hybrid:
+            csa.hca_dense_mqa(self.d["hca_q"], self.hcache, wl.m_hca, self.hwin, self.scale, q_pos0=self.q_pos0,
+                              out=self.hout, lse=self.hlse, workspace=self.ws_hca)
+
+    def e2e_step(self):
+        for k, v in self.h_in.items():
+            self.d[k].copy_(v, non_blocking=True)
+        self.step()
+        self.h_out[0].copy_(self.out, non_blocking=True)
+        if self.hybrid:
+            self.h_out[1].copy_(self.hout, non_blocking=True)
+
+    def e2e_bytes(self):
+        hi = sum(v.numel() * v.element_size() for v in self.h_in.values())
+        ho = sum(v.numel() * v.element_size() for v in self.h_out)
+        return hi, ho
+
+    def dominant(self):
+        """(name, source file, algorithmic bytes per launch, callable that launches it)."""
+        wl = self.wl
+        b = wl.B * wl.N * 64 * 2 + wl.B * 4 * 64 * 2 + wl.B * 4 * 4
+        return "indexer_score_long", "long_context_sparse_10_b200/csrc/indexer.cu", b, "hbm", self.indexer
+
+    def describe(self, world):
+        wl = self.wl
+        s = (f"{wl.name}: decode at context {wl.L}, batch {wl.B} per GPU, {wl.H} query heads, qk 192 / v 128; "
+             f"CSA m={wl.m} (N={wl.N}, FP8-e4m3 nope + BF16 RoPE cache, indexer 4x64 bf16, top-k={wl.k})")
+        if self.hybrid:
+            s += f" then HCA m'={wl.m_hca} (N'={wl.N_hca}, same split cache)"
+        s += f", sliding window {wl.win}"
+        return {"workload": s, "global_batch": wl.B * world, "seq_len": wl.L, "parallelism": f"dp{world} (replicas)",
+                "l2": "inputs larger than L2 (the indexer streams 268 MB/step > 126 MB L2)",
+                "timing": "CUDA graph replay of the whole step"}
+
+    def oracle_sample(self, budget_s):
+        """Time the float64 oracle on whole sequences of this workload (host cores)."""
+        import numpy as np
+        from oracle import csa_ref as R
+        h, wl = self.host, self.wl
+        done, spent = 0, 0.0
+        for b in range(wl.B):
+            qI = h["qI"][b:b + 1].double().numpy()
+            wI = h["wI"][b:b + 1].double().numpy()
+            kI = h["kIc"][b:b + 1].double().numpy()
+            q = h["q"][b:b + 1].double().numpy()
+            wk = h["win_k"][b:b + 1].double().numpy()
+            nope, rope, sc = h["nope"][b:b + 1].numpy(), h["rope"][b:b + 1].double().numpy(), h["scale"][b:b + 1].numpy()
+            if self.hybrid:
+                hq = h["hca_q"][b:b + 1].double().numpy()
+                hwk = h["hca_win_k"][b:b + 1].double().numpy()
+                hn, hr, hs = (h["hca_nope"][b:b + 1].numpy(), h["hca_rope"][b:b + 1].double().numpy(),
+                              h["hca_scale"][b:b + 1].numpy())
+            pos = np.array([wl.L - 1])
+            t0 = time.perf_counter()
+            s = R.indexer_scores(qI, wI, kI, pos, wl.m)
+            idx = R.topk_set(s, wl.k)
+            K, V = R.dequant_split(nope, rope, sc)
+            R.csa_sparse_mqa(q, pos, K, V, idx, wl.m, wk, wk[..., :128], wl.L - wl.win, wl.win, self.scale)
+            if self.hybrid:
+                HK, HV = R.dequant_split(hn, hr, hs)
+                R.hca_dense_mqa(hq, pos, HK, HV, wl.m_hca, hwk, hwk[..., :128], wl.L - wl.win, wl.win, self.scale)
+            spent += time.perf_counter() - t0
+            done += 1
+            if spent >= budget_s:
+                break
+        return done, spent, f"{done} of {wl.B} sequences of one rank's batch, whole decode step each"
+
+
+# ---------------------------------------------------------------------------
+# prefill workloads (CSA prefill, HCA prefill)
+# ---------------------------------------------------------------------------
+class PrefillRun:
+    def __init__(self, wl, rank, dev):
+        import torch
+        import long_context_sparse_10_b200 as csa
+        from long_context_sparse_10_b200 import synth
+        self.torch, self.csa, self.wl, self.dev = torch, csa, wl, dev
+        self.host = synth.prefill_inputs(wl, seed=rank)
+        d = {k: v.to(dev) for k, v in self.host.items()}
+        self.d = d
+        B, T, H, m, N = wl.B, wl.T, wl.H, wl.m, wl.N
+        self.scale = 1.0 / math.sqrt(192)
+        self.Kc = torch.empty(B, N, 192, dtype=torch.bfloat16, device=dev)
+        self.Vc = torch.empty(B, N, 128, dtype=torch.bfloat16, device=dev)
+        self.win = csa.Window(k=d["k"], v=d["v"], pos0=0, length=wl.win)
+        self.out = torch.empty(B, T, H, 128, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(B, T, H, dtype=torch.float32, device=dev)
+        self.csa_kind = wl.kind == "csa"
+        self.launches = 2 + 1
+        if self.csa_kind:
+            self.kIc = torch.empty(B, N, 64, dtype=torch.bfloat16, device=dev)
+            self.idx = torch.empty(B, T, wl.k, dtype=torch.int32, device=dev)
+            self.ws_idx = torch.empty(max(1, csa.csa_indexer_topk_workspace_size(B, T, N, wl.k)), dtype=torch.uint8,
+                                      device=dev)
+            self.launches += 1 + 2
+        self.h_in = {k: self.host[k].pin_memory() for k in self.host}
+        self.h_out = [torch.empty_like(self.out, device="cpu").pin_memory()]
+        self.tokens = B * T
+
+    def attention(self):
+        wl, csa = self.wl, self.csa
+        if self.csa_kind:
+            csa.csa_sparse_mqa(self.d["q"], csa.KVCache(k=self.Kc, v=self.Vc), wl.m, self.idx, self.win, self.scale,
+                               out=self.out, lse=self.lse)
+        else:
+            csa.hca_dense_mqa(self.d["q"], csa.KVCache(k=self.Kc, v=self.Vc), wl.m, self.win, self.scale,
+                              out=self.out, lse=self.lse)
+
+    def step(self):
+        wl, csa, d = self.wl, self.csa, self.d
+        fn = csa.csa_compress if self.csa_kind else csa.hca_compress
+        fn(d["k"], d["w_k"], d["b_k"], wl.m, out=self.Kc)
+        fn(d["v"], d["w_v"], d["b_v"], wl.m, out=self.Vc)
+        if self.csa_kind:
+            fn(d["kI"], d["w_i"], d["b_i"], wl.m, out=self.kIc)
+            csa.csa_indexer_topk(d["qI"], d["wI"], self.kIc, wl.m, wl.k, idx=self.idx, workspace=self.ws_idx)
+        self.attention()
+
+    def e2e_step(self):
+        for k, v in self.h_in.items():
+            self.d[k].copy_(v, non_blocking=True)
+        self.step()
+        self.h_out[0].copy_(self.out, non_blocking=True)
+
+    def e2e_bytes(self):
+        return (sum(v.numel() * v.element_size() for v in self.h_in.values()),
+                sum(v.numel() * v.element_size() for v in self.h_out))
+
+    def attn_flops(self):
+        wl = self.wl
+        t = __import__("numpy").arange(wl.T)
+        ent = (t + 1) // wl.m
+        if self.csa_kind:
+            ent = __import__("numpy").minimum(ent, wl.k)
+        keys = ent + __import__("numpy").minimum(wl.win, t + 1)
+        return float(wl.B * wl.H * 2 * (192 + 128) * keys.sum())
+
+    def dominant(self):
+        return ("attention_prefill", "long_context_sparse_10_b200/csrc/attention.cu", self.attn_flops(), "tensor",
+                self.attention)
+
+    def describe(self, world):
+        wl = self.wl
+        s = (f"{wl.name}: {wl.kind.upper()} prefill, B={wl.B}, T={wl.T}, {wl.H} query heads, qk 192 / v 128, "
+             f"stride {wl.m}" + (f", indexer 4x64, top-k={wl.k}" if self.csa_kind else "") + f", window {wl.win}")
+        return {"workload": s, "global_batch": wl.B * world, "seq_len": wl.T, "parallelism": f"dp{world} (replicas)",
+                "l2": "inputs larger than L2" if wl.T * wl.H * 384 * wl.B > 126e6 else "inputs fit in L2",
+                "timing": "CUDA graph replay of the whole step"}
+
+    def oracle_sample(self, budget_s):
+        import numpy as np
+        from oracle import csa_ref as R
+        h, wl = self.host, self.wl
+        t0 = time.perf_counter()
+        cw = 2 * wl.m if self.csa_kind else wl.m
+        K = h["k"][:1].double().numpy()
+        V = h["v"][:1].double().numpy()
+        Kc = R.compress(K, h["w_k"].double().numpy(), h["b_k"].double().numpy(), wl.m, cw)
+        Vc = R.compress(V, h["w_v"].double().numpy(), h["b_v"].double().numpy(), wl.m, cw)
+        if self.csa_kind:
+            kIc = R.compress(h["kI"][:1].double().numpy(), h["w_i"].double().numpy(), h["b_i"].double().numpy(),
+                             wl.m, cw)
+        rows_done = 0
+        rng = np.random.default_rng(0)
+        order = rng.permutation(wl.T)
+        for c in range(0, wl.T, 64):
+            rows = np.sort(order[c:c + 64])
+            q = h["q"][:1, rows].double().numpy()
+            if self.csa_kind:
+                s = R.indexer_scores(h["qI"][:1, rows].double().numpy(), h["wI"][:1, rows].double().numpy(), kIc,
+                                     rows, wl.m)
+                idx = R.topk_set(s, wl.k)
+                R.csa_sparse_mqa(q, rows, Kc, Vc, idx, wl.m, K, V, 0, wl.win, self.scale)
+            else:
+                R.hca_dense_mqa(q, rows, Kc, Vc, wl.m, K, V, 0, wl.win, self.scale)
+            rows_done += len(rows)
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        spent = time.perf_counter() - t0
+        return rows_done, spent, (f"compression of sequence 0 plus {rows_done} random query rows of it "
+                                  f"(tokens/s counts those rows)")
+
+
+# ---------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def make_run(name, rank, dev):
+    from long_context_sparse_10_b200 import synth
+    wl = synth.WORKLOADS[name]
+    return (DecodeRun if isinstance(wl, synth.Decode) else PrefillRun)(wl, rank, dev)
+
+
+def reference_arm(args):
+    """The float64 CPU oracle, timed on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from long_context_sparse_10_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+
+    class HostOnly:  # the same inputs, without touching a GPU
+        pass
+
+    run = (DecodeRun if isinstance(wl, synth.Decode) else PrefillRun).__new__(
+        DecodeRun if isinstance(wl, synth.Decode) else PrefillRun)
+    run.wl = wl
+    run.scale = 1.0 / math.sqrt(192)
+    if isinstance(wl, synth.Decode):
+        run.host = synth.decode_inputs(wl, seed=0, batch=slice(0, wl.B))
+        run.hybrid = wl.kind == "hybrid"
+    else:
+        run.host = synth.prefill_inputs(wl, seed=0)
+        run.csa_kind = wl.kind == "csa"
+    budget = min(150.0, max(5.0, args.cpu_sample_s * 4))
+    per_step_budget = budget / max(1, args.steps + args.warmup)
+    n, spent, sample = run.oracle_sample(max(per_step_budget, 0.0))
+    steps_done = 1
+    total_n, total_s = n, spent
+    while total_s < budget and steps_done < args.steps:
+        n, spent, _ = run.oracle_sample(0.0)
+        total_n += n
+        total_s += spent
+        steps_done += 1
+    value = total_n / total_s
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": steps_done, "steps_requested": args.steps, "warmup": 0, "ms_per_step": 1e3 * total_s / steps_done,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "oracle": "numpy float64 (oracle/csa_ref.py)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample + f"; {steps_done} step(s) within a {budget:.0f} s budget",
+                             "host_cpus": os.cpu_count()},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import long_context_sparse_10_b200 as csa
+    from long_context_sparse_10_b200 import _lib, replicas
+    lib = _lib.load()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    run = make_run(args.workload, rank, dev)
+    torch.cuda.synchronize()
+
+    # warm-up outside the graph (per-device one-time set-up happens here), then capture the step
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            run.step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run.step()
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    # timed region: K graph replays
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        ev0.record()
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+    barrier()
+    ms = replicas.max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
+
+    # dominant kernel: average launch duration with events recorded around it by the library
+    name, src, work, bound, launch = run.dominant()
+    reps = max(1, args.profile_reps)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:          # torch creates the CUDA event on first record
+        a.record()
+        b.record()
+    torch.cuda.synchronize()
+    for i in range(reps):
+        a, b = evs[i]
+        assert lib.csa_profile_next_call(a.cuda_event, b.cuda_event) == 0
+        launch()
+    torch.cuda.synchronize()
+    kms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    pk, pk_kind = peaks()
+    if bound == "hbm":
+        achieved = work / (kms * 1e-3) / 1e9
+        peak = pk["hbm_gbs"]
+        unit = "GB/s"
+    else:
+        achieved = work / (kms * 1e-3) / 1e12
+        peak = pk["bf16_tflops"]
+        unit = "TFLOP/s"
+    traffic = profile_traffic(name, src)
+    roofline = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "peak_source": f"{pk_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+                "traffic": traffic, "algorithmic_per_launch": work, "launch_ms": kms}
+
+    # end to end through the public API, pinned host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        k2 = max(10, min(args.steps // 10, 500))
+        for _ in range(3):
+            run.e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(k2):
+            run.e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ems = replicas.max_over_ranks(e0.elapsed_time(e1) / k2, dev)
+        bi, bo = run.e2e_bytes()
+        e2e = {"value": run.tokens * world / (ems * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": ems, "steps": k2}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, spent, sample = run.oracle_sample(args.cpu_sample_s)
+        cpu = {"value": n / spent, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": sample,
+               "host_cpus": os.cpu_count(), "seconds": spent}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": run.tokens * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": run.describe(world), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": run.launches * args.steps, "clocks": clocks.summary(),
+                "library": csa.version()}
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

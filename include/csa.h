@@ -104,6 +104,18 @@ CSA_API const char* csa_status_string(int32_t status);
 CSA_API const char* csa_last_error(void);
 
 /*
+ * csa_profile_next_call -- timing hook (library infrastructure, not part of
+ * the method).  `start_event` and `stop_event` are cudaEvent_t handles created
+ * by the caller.  The next entry point that enqueues work on this thread
+ * records `start_event` on its stream immediately before its main kernel and
+ * `stop_event` immediately after it (compression: the compression kernel;
+ * indexer: the scoring kernel; attention: the attention kernel, without the
+ * split combine), then forgets both.  Passing NULLs clears a pending hook.
+ * Returns CSA_ERR_INVALID_ARG if exactly one handle is NULL.
+ */
+CSA_API csa_status csa_profile_next_call(void* start_event, void* stop_event);
+
+/*
  * csa_compress -- CSA KV compression (Method section, CSA paragraph: every m
  * tokens become one entry through learnable compression weights and a position
  * bias; the windows overlap, in contrast to HCA's non-overlapping ones).

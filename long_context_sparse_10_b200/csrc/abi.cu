@@ -6,6 +6,9 @@
 
 namespace {
 thread_local char g_msg[512] = "";
+thread_local cudaEvent_t g_prof_start = nullptr;
+thread_local cudaEvent_t g_prof_stop = nullptr;
+thread_local bool g_prof_started = false;
 int g_sms[64] = {0};
 }  // namespace
 
@@ -38,9 +41,34 @@ int num_sms() {
   return g_sms[dev];
 }
 
+void prof_begin(cudaStream_t s) {
+  if (g_prof_start && g_prof_stop) {
+    cudaEventRecord(g_prof_start, s);
+    g_prof_started = true;
+  }
+}
+
+void prof_end(cudaStream_t s) {
+  if (g_prof_started) {
+    cudaEventRecord(g_prof_stop, s);
+    g_prof_start = g_prof_stop = nullptr;
+    g_prof_started = false;
+  }
+}
+
 }  // namespace csa
 
 extern "C" {
+
+csa_status csa_profile_next_call(void* start_event, void* stop_event) {
+  if ((start_event == nullptr) != (stop_event == nullptr))
+    return csa::fail(CSA_ERR_INVALID_ARG, "csa_profile_next_call: pass both events or neither");
+  g_prof_start = static_cast<cudaEvent_t>(start_event);
+  g_prof_stop = static_cast<cudaEvent_t>(stop_event);
+  g_prof_started = false;
+  return CSA_OK;
+}
+
 
 const char* csa_version(void) { return "csa-b200 0.1.0 sm_100a"; }
 

@@ -516,10 +516,12 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(static_cast<unsigned>(R), static_cast<unsigned>(pl.nsplit));
+  prof_begin(s);
   if (H == 64)
     attn_kernel<1><<<grid, kThreads, kSmemBytes, s>>>(p);
   else
     attn_kernel<4><<<grid, kThreads, kSmemBytes, s>>>(p);
+  prof_end(s);
   if (csa_status st = check_launch(name); st != CSA_OK) return st;
   if (pl.nsplit > 1) {
     const int64_t warps = R * H;

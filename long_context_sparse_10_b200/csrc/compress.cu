@@ -232,14 +232,13 @@ csa_status compress_impl(const char* name, const void* x, int64_t B, int64_t T, 
   p.out_scale = out_scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t entries = B * p.N;
-  if (cwin <= 32) {
-    const int64_t grid = (entries + 7) / 8;
-    CSA_REQUIRE(grid < (1LL << 31), "%s: too many entries", name);
-    compress_short_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(p);
-  } else {
-    CSA_REQUIRE(entries < (1LL << 31), "%s: too many entries", name);
+  CSA_REQUIRE(entries < (1LL << 31), "%s: too many entries", name);
+  prof_begin(s);
+  if (cwin <= 32)
+    compress_short_kernel<<<static_cast<unsigned>((entries + 7) / 8), 256, 0, s>>>(p);
+  else
     compress_long_kernel<<<static_cast<unsigned>(entries), 256, 0, s>>>(p);
-  }
+  prof_end(s);
   return check_launch(name);
 }
 

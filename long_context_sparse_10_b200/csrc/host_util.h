@@ -16,6 +16,9 @@ void clear_error();
 csa_status check_launch(const char* what);
 // Streaming multiprocessors of the current device (cached per device).
 int num_sms();
+// Records the pending csa_profile_next_call start/stop event (if any) on `s`.
+void prof_begin(cudaStream_t s);
+void prof_end(cudaStream_t s);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -534,7 +534,9 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
     const int64_t groups = (Tq + QR - 1) / QR;
     dim3 grid(static_cast<unsigned>((N + p.chunk - 1) / p.chunk), static_cast<unsigned>(B * groups));
     CSA_REQUIRE(B * groups < 65536, "csa_indexer_topk: too many query rows for one launch");
+    prof_begin(s);
     score_kernel<QR, false><<<grid, kScoreThreads, tile_smem, s>>>(p);
+    prof_end(s);
     if (csa_status st = check_launch("indexer score"); st != CSA_OK) return st;
     const size_t smem = static_cast<size_t>(N) * 4;
     static bool attr_set[64] = {false};
@@ -566,7 +568,9 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
   p.hist = w.hist;
   CSA_REQUIRE(R < 65536, "csa_indexer_topk: too many query rows for the long-row path");
   dim3 grid(static_cast<unsigned>((N + p.chunk - 1) / p.chunk), static_cast<unsigned>(R));
+  prof_begin(s);
   score_kernel<1, true><<<grid, kScoreThreads, tile_smem + kHistBins * 4, s>>>(p);
+  prof_end(s);
   if (csa_status st = check_launch("indexer score (long rows)"); st != CSA_OK) return st;
   topk_threshold_kernel<<<static_cast<unsigned>(R), 1024, 0, s>>>(w, N, Tq, q_pos0, m, k);
   if (csa_status st = check_launch("indexer threshold"); st != CSA_OK) return st;
