@@ -167,6 +167,27 @@ CSA_API csa_status csa_indexer_topk(const void* qI, const float* wI, const void*
                             int32_t k, int32_t* idx, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/*
+ * csa_indexer_topk_noalloc -- csa_indexer_topk without a caller workspace.
+ * The paper has no counterpart: this is a library convenience.  Some callers
+ * cannot allocate device memory themselves (for example a plugin whose host
+ * application owns every device allocation, or code on a latency-critical
+ * path that must not call cudaMalloc); this call needs none.  Its scratch is a
+ * 32 MiB static device array inside the library, held on every GPU that loads
+ * the library until the process exits.  Sizes whose workspace
+ * (csa_indexer_topk_workspace_size) exceeds 32 MiB are rejected with
+ * CSA_ERR_UNSUPPORTED and a message; e.g. 8 decode rows over 262,144 entries
+ * fit.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and caches it; make that
+ * first call before any stream capture.  No call allocates.  Every call
+ * shares the array and it keeps the last call's contents (the call clears what
+ * must start at zero), so calls that overlap on the GPU race on it.  Other
+ * arguments, outputs and errors as csa_indexer_topk.
+ */
+CSA_API csa_status csa_indexer_topk_noalloc(const void* qI, const float* wI, const void* kIc,
+                                            int64_t B, int64_t Tq, int64_t N, int64_t q_pos0,
+                                            int32_t m, int32_t k, int32_t* idx, void* stream);
+
 /* Workspace bytes csa_sparse_mqa needs for these sizes. */
 CSA_API size_t csa_sparse_mqa_workspace_size(int64_t B, int64_t Tq, int32_t H, int32_t k, int32_t win_len);
 

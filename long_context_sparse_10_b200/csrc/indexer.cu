@@ -20,6 +20,8 @@
 //     kernel, a select kernel that emits a bitmap of the entries above the
 //     threshold bin plus a candidate list of the threshold bin, and a finalize
 //     kernel that resolves the candidates and writes the ascending list.
+#include <mutex>
+
 #include "common.cuh"
 #include "host_util.h"
 
@@ -582,3 +584,56 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// csa_indexer_topk_noalloc: the same selection with library-owned scratch.
+//
+// Some callers cannot allocate device memory themselves -- for example a plugin
+// whose host application owns every device allocation, or code on a latency-
+// critical path that must not call cudaMalloc.  This variant takes no
+// workspace: it uses a file-scope static device array of
+// kStaticScratchBytes (32 MiB), which every GPU that loads the library holds
+// until the process exits.  Host code cannot hand the array's name to a kernel
+// (on the host it is only a stand-in for the symbol), so the first call on
+// each device looks up the array's device address with cudaGetSymbolAddress
+// while that device is current and caches it; that first call should come
+// before any stream capture.  The call itself allocates nothing: it forwards
+// to csa_indexer_topk with the cached address as the workspace, and that path
+// clears the parts of the scratch that must start at zero on every call.  All
+// calls share the one array and it keeps the last call's contents, so calls
+// that overlap on the GPU (different streams, or host threads, without
+// ordering between them) race on it.
+// ---------------------------------------------------------------------------
+static constexpr size_t kStaticScratchBytes = static_cast<size_t>(32) << 20;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+static std::mutex g_static_mu;
+static void* g_static_ptr[64] = {nullptr};
+
+extern "C" csa_status csa_indexer_topk_noalloc(const void* qI, const float* wI, const void* kIc, int64_t B,
+                                               int64_t Tq, int64_t N, int64_t q_pos0, int32_t m, int32_t k,
+                                               int32_t* idx, void* stream) {
+  using namespace csa;
+  if (B < 0 || Tq < 0 || N < 0) return fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk_noalloc: negative size");
+  const size_t need = csa::workspace_bytes(B, Tq, N);
+  if (need > kStaticScratchBytes)
+    return fail(CSA_ERR_UNSUPPORTED,
+                "csa_indexer_topk_noalloc: these sizes need %zu bytes of scratch but the static scratch holds %zu; "
+                "call csa_indexer_topk with a caller workspace instead",
+                need, kStaticScratchBytes);
+  void* ptr = nullptr;
+  if (need > 0) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+      return fail(CSA_ERR_CUDA, "csa_indexer_topk_noalloc: no usable current device");
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_ptr[dev] == nullptr) {
+      const cudaError_t e = cudaGetSymbolAddress(&g_static_ptr[dev], g_static_scratch);
+      if (e != cudaSuccess) {
+        g_static_ptr[dev] = nullptr;
+        return fail(CSA_ERR_CUDA, "csa_indexer_topk_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+      }
+    }
+    ptr = g_static_ptr[dev];
+  }
+  return csa_indexer_topk(qI, wI, kIc, B, Tq, N, q_pos0, m, k, idx, ptr, ptr ? kStaticScratchBytes : 0, stream);
+}
