@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-reps", type=int, default=100, help="launches of the dominant kernel to average")
+    ap.add_argument("--breakdown", action="store_true", help="also time each library call of the step (stderr)")
     return ap.parse_args()
 
 
@@ -158,7 +159,7 @@ class DecodeRun:
         self.ws_attn = torch.empty(max(1, nws), dtype=torch.uint8, device=dev)
         self.out = torch.empty(B, 1, H, 128, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(B, 1, H, dtype=torch.float32, device=dev)
-        self.launches = 4 + (2 if nws else 1)
+        self.launches = 2 + 1          # indexer: score + select; attention: one cluster launch
         self.hybrid = wl.kind == "hybrid"
         if self.hybrid:
             self.hcache = csa.KVCache(nope=d["hca_nope"], rope=d["hca_rope"], scale=d["hca_scale"])
@@ -167,7 +168,7 @@ class DecodeRun:
             self.ws_hca = torch.empty(max(1, hws), dtype=torch.uint8, device=dev)
             self.hout = torch.empty(B, 1, H, 128, dtype=torch.bfloat16, device=dev)
             self.hlse = torch.empty(B, 1, H, dtype=torch.float32, device=dev)
-            self.launches += 2 if hws else 1
+            self.launches += 1
         # pinned host buffers for the end-to-end measurement
         self.h_in = {k: h[k].pin_memory() for k in (["q", "qI", "wI"] + (["hca_q"] if self.hybrid else []))}
         self.h_out = [torch.empty_like(self.out, device="cpu").pin_memory()]
@@ -188,6 +189,19 @@ class DecodeRun:
         if self.hybrid:
             csa.hca_dense_mqa(self.d["hca_q"], self.hcache, wl.m_hca, self.hwin, self.scale, q_pos0=self.q_pos0,
                               out=self.hout, lse=self.hlse, workspace=self.ws_hca)
+
+    def parts(self):
+        """The step's library calls, separately (for --breakdown)."""
+        wl, csa = self.wl, self.csa
+        out = [("csa_indexer_topk", self.indexer),
+               ("csa_sparse_mqa", lambda: csa.csa_sparse_mqa(self.d["q"], self.cache, wl.m, self.idx, self.win,
+                                                             self.scale, q_pos0=self.q_pos0, out=self.out,
+                                                             lse=self.lse, workspace=self.ws_attn))]
+        if self.hybrid:
+            out.append(("hca_dense_mqa", lambda: csa.hca_dense_mqa(self.d["hca_q"], self.hcache, wl.m_hca, self.hwin,
+                                                                   self.scale, q_pos0=self.q_pos0, out=self.hout,
+                                                                   lse=self.hlse, workspace=self.ws_hca)))
+        return out
 
     def e2e_step(self):
         for k, v in self.h_in.items():
@@ -273,13 +287,13 @@ class PrefillRun:
         self.out = torch.empty(B, T, H, 128, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(B, T, H, dtype=torch.float32, device=dev)
         self.csa_kind = wl.kind == "csa"
-        self.launches = 2 + 1
+        self.launches = 2 + 1          # compress K, V; attention
         if self.csa_kind:
             self.kIc = torch.empty(B, N, 64, dtype=torch.bfloat16, device=dev)
             self.idx = torch.empty(B, T, wl.k, dtype=torch.int32, device=dev)
             self.ws_idx = torch.empty(max(1, csa.csa_indexer_topk_workspace_size(B, T, N, wl.k)), dtype=torch.uint8,
                                       device=dev)
-            self.launches += 1 + 2
+            self.launches += 1 + 2     # compress kI; indexer score + top-k
         self.h_in = {k: self.host[k].pin_memory() for k in self.host}
         self.h_out = [torch.empty_like(self.out, device="cpu").pin_memory()]
         self.tokens = B * T
@@ -302,6 +316,18 @@ class PrefillRun:
             fn(d["kI"], d["w_i"], d["b_i"], wl.m, out=self.kIc)
             csa.csa_indexer_topk(d["qI"], d["wI"], self.kIc, wl.m, wl.k, idx=self.idx, workspace=self.ws_idx)
         self.attention()
+
+    def parts(self):
+        wl, csa, d = self.wl, self.csa, self.d
+        fn = csa.csa_compress if self.csa_kind else csa.hca_compress
+        out = [("compress K", lambda: fn(d["k"], d["w_k"], d["b_k"], wl.m, out=self.Kc)),
+               ("compress V", lambda: fn(d["v"], d["w_v"], d["b_v"], wl.m, out=self.Vc))]
+        if self.csa_kind:
+            out += [("compress kI", lambda: fn(d["kI"], d["w_i"], d["b_i"], wl.m, out=self.kIc)),
+                    ("csa_indexer_topk", lambda: csa.csa_indexer_topk(d["qI"], d["wI"], self.kIc, wl.m, wl.k,
+                                                                      idx=self.idx, workspace=self.ws_idx))]
+        out.append(("attention", self.attention))
+        return out
 
     def e2e_step(self):
         for k, v in self.h_in.items():
@@ -508,6 +534,18 @@ def main():
     roofline = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "peak_source": f"{pk_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
                 "traffic": traffic, "algorithmic_per_launch": work, "launch_ms": kms}
+
+    if args.breakdown and rank == 0:
+        reps = 50
+        for name_, fn_ in run.parts():
+            evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+            for a, b in evp:
+                a.record()
+                fn_()
+                b.record()
+            torch.cuda.synchronize()
+            ts = sorted(a.elapsed_time(b) * 1e3 for a, b in evp)
+            print(f"breakdown {name_:20s} median {ts[reps // 2]:8.1f} us  min {ts[0]:8.1f} us", file=sys.stderr)
 
     # end to end through the public API, pinned host buffers, copies inside the timed region
     e2e = None

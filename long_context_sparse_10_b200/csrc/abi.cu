@@ -1,6 +1,9 @@
 // Library-wide entry points: version, status names, per-thread error text.
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
+#include <map>
+#include <utility>
 
 #include "host_util.h"
 
@@ -39,6 +42,23 @@ int num_sms() {
     g_sms[dev] = n;
   }
   return g_sms[dev];
+}
+
+bool ensure_smem(const void* kernel, int bytes) {
+  // The limit is one value per kernel and device: only ever raise it.
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, int> limit;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  int& cur = limit[std::make_pair(dev, kernel)];
+  if (bytes <= cur) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  cur = bytes;
+  return true;
 }
 
 void prof_begin(cudaStream_t s) {

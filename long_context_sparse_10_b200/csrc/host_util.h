@@ -16,6 +16,9 @@ void clear_error();
 csa_status check_launch(const char* what);
 // Streaming multiprocessors of the current device (cached per device).
 int num_sms();
+// Raises a kernel's dynamic shared memory limit to `bytes` on the current
+// device (once per device and kernel).  Returns false if the runtime refuses.
+bool ensure_smem(const void* kernel, int bytes);
 // Records the pending csa_profile_next_call start/stop event (if any) on `s`.
 void prof_begin(cudaStream_t s);
 void prof_end(cudaStream_t s);

@@ -16,10 +16,11 @@
 //   * rows whose visible prefix fits in shared memory (prefill) run one CTA
 //     per row over the row held in shared memory;
 //   * long rows (decode over 10^5..10^6 entries) get a 4096-bin histogram of
-//     the key's top 12 bits fused into the scoring kernel, then a threshold
-//     kernel, a select kernel that emits a bitmap of the entries above the
-//     threshold bin plus a candidate list of the threshold bin, and a finalize
-//     kernel that resolves the candidates and writes the ascending list.
+//     the key's top 12 bits fused into the scoring kernel, whose last CTA per
+//     row derives the threshold bin; one select kernel then emits a bitmap of
+//     the entries above that bin plus a candidate list of the bin itself, and
+//     its last CTA per row resolves the candidates and writes the ascending
+//     list.  "Last CTA" is decided by an atomic counter (no CTA ever waits).
 #include <mutex>
 
 #include "common.cuh"
@@ -44,11 +45,126 @@ struct ScoreParams {
   int chunk;        // entries per CTA (multiple of kTileRows)
   float* scores;    // [R, N]
   uint32_t* hist;   // [R, kHistBins] (QR == 1 only)
+  uint32_t* done;   // [R, 2] CTA counters (QR == 1 only)
+  int32_t* thr;     // [R, 2] threshold (QR == 1 only)
+  int k;
 };
 
 __device__ __forceinline__ int64_t visible(int64_t t, int m, int64_t N) {
   int64_t v = (t + 1) / m;
   return v < N ? v : N;
+}
+
+// ---------------------------------------------------------------------------
+// block-wide helpers (blockDim.x == 1024)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* total, uint32_t* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) sh[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = lane < nw ? sh[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += t;
+    }
+    sh[lane] = w;
+  }
+  __syncthreads();
+  const uint32_t before = warp ? sh[warp - 1] : 0u;
+  *total = sh[nw - 1];
+  __syncthreads();
+  return before + incl - v;
+}
+
+// Warp 0 walks 256 bins from the top and finds the digit holding the
+// `remaining`-th largest element.  Writes digit, count strictly above, and the
+// bin's own count to out[0..2].
+__device__ __forceinline__ void find_digit_256(const uint32_t* hist, uint32_t remaining, uint32_t* out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t c[8], sum = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    c[j] = hist[255 - 8 * lane - j];
+    sum += c[j];
+  }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const uint32_t excl = incl - sum;
+  if (excl < remaining && incl >= remaining) {
+    uint32_t acc = excl;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (acc + c[j] >= remaining) {
+        out[0] = 255 - 8 * lane - j;
+        out[1] = acc;
+        out[2] = c[j];
+        break;
+      }
+      acc += c[j];
+    }
+  }
+}
+
+__device__ __forceinline__ void write_prefix_ids(int32_t* out, int64_t nv, int k) {
+  for (int j = threadIdx.x; j < k; j += blockDim.x) out[j] = j < nv ? j : -1;
+}
+
+// Threshold of one row from its global histogram, by one CTA of NT threads
+// (each owns 4096/NT consecutive bins, read as 16-byte vectors).  thr = (bin,
+// count still needed from that bin); bin -1 when every visible entry fits.
+template <int NT>
+__device__ void row_threshold(const uint32_t* gh, int64_t nv, int k, int32_t* thr, uint32_t* scan_sh) {
+  constexpr int PER = kHistBins / NT;
+  static_assert(PER % 4 == 0, "bins per thread must be a multiple of 4");
+  if (nv <= k) {
+    if (threadIdx.x == 0) {
+      thr[0] = -1;
+      thr[1] = 0;
+    }
+    return;
+  }
+  // thread t owns bins [4096 - PER(t+1), 4096 - PER t), walked from the top
+  const int lo = kHistBins - PER * (threadIdx.x + 1);
+  uint32_t c[PER];
+#pragma unroll
+  for (int j = 0; j < PER / 4; ++j) {
+    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(gh + lo) + j);
+    c[4 * j] = v.x;
+    c[4 * j + 1] = v.y;
+    c[4 * j + 2] = v.z;
+    c[4 * j + 3] = v.w;
+  }
+  uint32_t sum = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) sum += c[j];
+  uint32_t total;
+  const uint32_t excl = block_excl_scan(sum, &total, scan_sh);
+  const uint32_t kk = static_cast<uint32_t>(k);
+  if (excl < kk && excl + sum >= kk) {
+    uint32_t acc = excl;
+#pragma unroll
+    for (int j = PER - 1; j >= 0; --j) {
+      if (acc + c[j] >= kk) {
+        thr[0] = lo + j;
+        thr[1] = static_cast<int32_t>(kk - acc);
+        break;
+      }
+      acc += c[j];
+    }
+  }
 }
 
 // Scores QR consecutive query rows of one sequence against one chunk of entries.
@@ -163,80 +279,28 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
   }
   cp_async_wait<0>();
   if (HIST) {
+    // flush the CTA histogram; the row's last CTA then derives its threshold
+    __shared__ uint32_t last_s;
+    __shared__ uint32_t scan_sh[32];
     __syncthreads();
-    uint32_t* gh = p.hist + (b * p.Tq + r0) * kHistBins;
+    const int64_t row = b * p.Tq + r0;
+    uint32_t* gh = p.hist + row * kHistBins;
     for (int j = threadIdx.x; j < kHistBins; j += kScoreThreads) {
       const uint32_t c = hist_s[j];
       if (c) atomicAdd(gh + j, c);
     }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// block-wide helpers (blockDim.x == 1024)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* total, uint32_t* sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nw = blockDim.x >> 5;
-  uint32_t incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) sh[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t w = lane < nw ? sh[lane] : 0u;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += t;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const uint32_t ctas = static_cast<uint32_t>((nv_max + p.chunk - 1) / p.chunk);
+      last_s = (atomicAdd(p.done + 2 * row, 1u) == ctas - 1) ? 1u : 0u;
     }
-    sh[lane] = w;
-  }
-  __syncthreads();
-  const uint32_t before = warp ? sh[warp - 1] : 0u;
-  *total = sh[nw - 1];
-  __syncthreads();
-  return before + incl - v;
-}
-
-// Warp 0 walks 256 bins from the top and finds the digit holding the
-// `remaining`-th largest element.  Writes digit, count strictly above, and the
-// bin's own count to out[0..2].
-__device__ __forceinline__ void find_digit_256(const uint32_t* hist, uint32_t remaining, uint32_t* out) {
-  const int lane = threadIdx.x & 31;
-  uint32_t c[8], sum = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    c[j] = hist[255 - 8 * lane - j];
-    sum += c[j];
-  }
-  uint32_t incl = sum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  const uint32_t excl = incl - sum;
-  if (excl < remaining && incl >= remaining) {
-    uint32_t acc = excl;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (acc + c[j] >= remaining) {
-        out[0] = 255 - 8 * lane - j;
-        out[1] = acc;
-        out[2] = c[j];
-        break;
-      }
-      acc += c[j];
+    __syncthreads();
+    if (last_s) {
+      __threadfence();
+      row_threshold<kScoreThreads>(gh, nv_max, p.k, p.thr + 2 * row, scan_sh);
     }
   }
-}
-
-__device__ __forceinline__ void write_prefix_ids(int32_t* out, int64_t nv, int k) {
-  for (int j = threadIdx.x; j < k; j += blockDim.x) out[j] = j < nv ? j : -1;
 }
 
 // ---------------------------------------------------------------------------
@@ -292,117 +356,123 @@ __global__ void __launch_bounds__(1024) topk_rows_kernel(const float* __restrict
 }
 
 // ---------------------------------------------------------------------------
-// long-row path (histogram fused into scoring)
+// long-row path: histogram + threshold fused into scoring, then one select
+// kernel whose last CTA per row resolves the threshold bin and writes the list
 // ---------------------------------------------------------------------------
+constexpr int kSelThreads = 512;
+constexpr int kSelChunk = 4096;
+
 struct LongWs {
-  float* scores;       // [R, N]
-  uint32_t* hist;      // [R, kHistBins]
-  uint32_t* cand_cnt;  // [R]
-  int32_t* thr;        // [R, 2]: threshold bin (-1: take every visible entry), needed from it
-  uint2* cand;         // [R, N]: (key, index)
-  uint32_t* bitmap;    // [R, W]
+  float* scores;        // [R, N]
+  uint32_t* hist;       // [R, kHistBins]    (zeroed per call)
+  uint32_t* cand_cnt;   // [R]               (zeroed per call)
+  uint32_t* done;       // [R, 2]: scoring / select CTAs finished (zeroed per call)
+  int32_t* thr;         // [R, 2]
+  uint2* cand;          // [R, N]: (key, index) of the threshold bin's entries
+  uint32_t* bitmap;     // [R, W]
   int64_t W;
 };
 
-__global__ void __launch_bounds__(1024) topk_threshold_kernel(LongWs ws, int64_t N, int64_t Tq, int64_t q_pos0,
-                                                              int m, int k) {
+// Per CTA: a bitmap word for every 32 entries (entries above the threshold
+// bin), and the threshold bin's entries appended to the row's candidate list
+// (gathered in shared memory first, one global atomic per CTA).  The last CTA
+// of a row then radix-selects the `need` best candidates on the composite key
+// (score key << 32 | ~index), adds them to the bitmap and writes the row's
+// ascending index list.
+__global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, int64_t N, int64_t Tq, int64_t q_pos0,
+                                                                  int m, int k, int32_t* __restrict__ idx) {
+  __shared__ uint2 cand_s[kSelChunk];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t dig[3];
   __shared__ uint32_t scan_sh[32];
-  const int64_t row = blockIdx.x;
-  const int64_t nv = visible(q_pos0 + row % Tq, m, N);
-  if (nv <= k) {
-    if (threadIdx.x == 0) {
-      ws.thr[2 * row] = -1;
-      ws.thr[2 * row + 1] = 0;
-    }
-    return;
-  }
-  const uint32_t* h = ws.hist + row * kHistBins;
-  // thread t owns bins 4095-4t .. 4092-4t (descending)
-  uint32_t c[4], sum = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    c[j] = h[kHistBins - 1 - 4 * threadIdx.x - j];
-    sum += c[j];
-  }
-  uint32_t total;
-  const uint32_t excl = block_excl_scan(sum, &total, scan_sh);
-  const uint32_t kk = static_cast<uint32_t>(k);
-  if (excl < kk && excl + sum >= kk) {
-    uint32_t acc = excl;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (acc + c[j] >= kk) {
-        ws.thr[2 * row] = kHistBins - 1 - 4 * threadIdx.x - j;
-        ws.thr[2 * row + 1] = static_cast<int32_t>(kk - acc);
-        break;
-      }
-      acc += c[j];
-    }
-  }
-}
-
-constexpr int kSelThreads = 256;
-constexpr int kSelChunk = 8192;
-
-__global__ void __launch_bounds__(kSelThreads) topk_select_kernel(LongWs ws, int64_t N, int64_t Tq,
-                                                                  int64_t q_pos0, int m) {
+  __shared__ uint32_t n_cand, base_s, last_s;
   const int64_t row = blockIdx.y;
   const int64_t nv = visible(q_pos0 + row % Tq, m, N);
   const int64_t e_begin = static_cast<int64_t>(blockIdx.x) * kSelChunk;
   if (e_begin >= nv) return;
-  const int64_t e_end = (e_begin + kSelChunk) < nv ? (e_begin + kSelChunk) : nv;
+  int32_t* out = idx + row * k;
   const int thr_bin = ws.thr[2 * row];
-  if (thr_bin < 0) return;  // finalize takes the whole visible prefix
+  if (thr_bin < 0) {  // every visible entry is selected
+    if (blockIdx.x == 0) write_prefix_ids(out, nv, k);
+    return;
+  }
+  const int64_t e_end = (e_begin + kSelChunk) < nv ? (e_begin + kSelChunk) : nv;
   const uint32_t tb = static_cast<uint32_t>(thr_bin);
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) n_cand = 0;
+  __syncthreads();
   const float* srow = ws.scores + row * N;
-  for (int64_t base = e_begin + (threadIdx.x & ~31); base < e_end; base += kSelThreads) {
+  constexpr int kIters = kSelChunk / kSelThreads;
+  float sv[kIters];
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {  // all loads first, then the bookkeeping
+    const int64_t i = e_begin + it * kSelThreads + threadIdx.x;
+    sv[it] = i < e_end ? __ldcg(srow + i) : 0.f;
+  }
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const int64_t base = e_begin + it * kSelThreads + (threadIdx.x & ~31);
     const int64_t i = base + lane;
     const bool ok = i < e_end;
-    const uint32_t key = ok ? f2key(srow[i]) : 0u;
+    const uint32_t key = ok ? f2key(sv[it]) : 0u;
     const uint32_t bin = key >> 20;
-    const bool def = ok && bin > tb;
+    const uint32_t word = __ballot_sync(0xffffffffu, ok && bin > tb);
+    if (lane == 0 && base < e_end) ws.bitmap[row * ws.W + (base >> 5)] = word;
     const bool cnd = ok && bin == tb;
-    const uint32_t word = __ballot_sync(0xffffffffu, def);
-    if (lane == 0) ws.bitmap[row * ws.W + (base >> 5)] = word;
     const uint32_t cm = __ballot_sync(0xffffffffu, cnd);
     if (cm) {
       uint32_t pos = 0;
-      if (lane == 0) pos = atomicAdd(ws.cand_cnt + row, static_cast<uint32_t>(__popc(cm)));
+      if (lane == 0) pos = atomicAdd(&n_cand, static_cast<uint32_t>(__popc(cm)));
       pos = __shfl_sync(0xffffffffu, pos, 0);
-      if (cnd) ws.cand[row * N + pos + __popc(cm & ((1u << lane) - 1u))] = make_uint2(key, static_cast<uint32_t>(i));
+      if (cnd) cand_s[pos + __popc(cm & ((1u << lane) - 1u))] = make_uint2(key, static_cast<uint32_t>(i));
     }
   }
-}
-
-__global__ void __launch_bounds__(1024) topk_finalize_kernel(LongWs ws, int64_t N, int64_t Tq, int64_t q_pos0,
-                                                             int m, int k, int32_t* __restrict__ idx) {
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t dig[3];
-  __shared__ uint32_t scan_sh[32];
-  const int64_t row = blockIdx.x;
-  const int64_t nv = visible(q_pos0 + row % Tq, m, N);
-  int32_t* out = idx + row * k;
-  const int thr_bin = ws.thr[2 * row];
-  if (thr_bin < 0) {
-    write_prefix_ids(out, nv, k);
-    return;
+  __syncthreads();
+  const uint32_t nc = n_cand;
+  if (threadIdx.x == 0 && nc) base_s = atomicAdd(ws.cand_cnt + row, nc);
+  __syncthreads();
+  for (uint32_t c = threadIdx.x; c < nc; c += kSelThreads) ws.cand[row * N + base_s + c] = cand_s[c];
+  // last CTA of this row?
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t chunks = static_cast<uint32_t>((nv + kSelChunk - 1) / kSelChunk);
+    last_s = (atomicAdd(ws.done + 2 * row + 1, 1u) == chunks - 1) ? 1u : 0u;
   }
-  // Composite key: (score key << 32) | ~index; its top 12 bits equal thr_bin
-  // for every candidate.  Radix-select the `need`-th largest composite.
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+
+  // ---- resolve the threshold bin: radix select on the 52 low composite bits
+  const uint32_t cnt = __ldcg(ws.cand_cnt + row);
   const uint2* cand = ws.cand + row * N;
-  const uint32_t cnt = ws.cand_cnt[row];
+  if (cnt <= static_cast<uint32_t>(kSelChunk)) {  // usual case: work on a shared-memory copy
+    for (uint32_t c0 = 0; c0 < cnt; c0 += 4 * kSelThreads) {
+      uint2 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t c = c0 + u * kSelThreads + threadIdx.x;
+        v[u] = c < cnt ? __ldcg(cand + c) : make_uint2(0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t c = c0 + u * kSelThreads + threadIdx.x;
+        if (c < cnt) cand_s[c] = v[u];
+      }
+    }
+    __syncthreads();
+    cand = cand_s;
+  }
   uint32_t remaining = static_cast<uint32_t>(ws.thr[2 * row + 1]);
   uint64_t prefix = static_cast<uint64_t>(thr_bin) << 52;
   uint64_t mask = 0xfffull << 52;
   uint32_t in_bucket = cnt;
-  // 52 unresolved low bits: six 8-bit digits (bits 51..4), then one 4-bit digit.
   for (int pass = 0; pass < 7 && in_bucket != remaining; ++pass) {
     const int sh = pass < 6 ? 44 - 8 * pass : 0;
     const uint64_t dmask = pass < 6 ? 255ull : 15ull;
-    for (int j = threadIdx.x; j < 256; j += blockDim.x) hist[j] = 0;
+    for (int j = threadIdx.x; j < 256; j += kSelThreads) hist[j] = 0;
     __syncthreads();
-    for (uint32_t c = threadIdx.x; c < cnt; c += blockDim.x) {
+    for (uint32_t c = threadIdx.x; c < cnt; c += kSelThreads) {
       const uint2 kv = cand[c];
       const uint64_t x = (static_cast<uint64_t>(kv.x) << 32) | (0xffffffffu - kv.y);
       if ((x & mask) == prefix) atomicAdd(&hist[(x >> sh) & dmask], 1u);
@@ -416,29 +486,48 @@ __global__ void __launch_bounds__(1024) topk_finalize_kernel(LongWs ws, int64_t 
     in_bucket = dig[2];
     __syncthreads();
   }
-  // chosen candidates: (x & mask) >= prefix
-  for (uint32_t c = threadIdx.x; c < cnt; c += blockDim.x) {
+  for (uint32_t c = threadIdx.x; c < cnt; c += kSelThreads) {
     const uint2 kv = cand[c];
     const uint64_t x = (static_cast<uint64_t>(kv.x) << 32) | (0xffffffffu - kv.y);
     if ((x & mask) >= prefix) atomicOr(ws.bitmap + row * ws.W + (kv.y >> 5), 1u << (kv.y & 31));
   }
   __threadfence();
   __syncthreads();
-  // ascending output from the bitmap
+
+  // ---- ascending list from the bitmap: 16 consecutive words per thread per round
   const int64_t words = (nv + 31) >> 5;
   const uint32_t* bm = ws.bitmap + row * ws.W;
   uint32_t before = 0;
-  for (int64_t base = 0; base < words; base += blockDim.x) {
-    const int64_t wi = base + threadIdx.x;
-    uint32_t word = wi < words ? __ldcg(bm + wi) : 0u;
-    if (wi == words - 1 && (nv & 31)) word &= (1u << (nv & 31)) - 1u;
+  for (int64_t base = 0; base < words; base += 16 * kSelThreads) {
+    const int64_t w0 = base + 16 * threadIdx.x;
+    uint32_t wv[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = w0 + 4 * j < words ? __ldcg(reinterpret_cast<const uint4*>(bm + w0) + j) : make_uint4(0, 0, 0, 0);
+      wv[4 * j] = v.x;
+      wv[4 * j + 1] = v.y;
+      wv[4 * j + 2] = v.z;
+      wv[4 * j + 3] = v.w;
+    }
+    uint32_t cntw = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int64_t wi = w0 + j;
+      if (wi >= words) wv[j] = 0;
+      else if (wi == words - 1 && (nv & 31)) wv[j] &= (1u << (nv & 31)) - 1u;
+      cntw += __popc(wv[j]);
+    }
     uint32_t total;
-    uint32_t pos = before + block_excl_scan(static_cast<uint32_t>(__popc(word)), &total, scan_sh);
-    while (word) {
-      const int bit = __ffs(word) - 1;
-      word &= word - 1;
-      if (pos < static_cast<uint32_t>(k)) out[pos] = static_cast<int32_t>((wi << 5) + bit);
-      ++pos;
+    uint32_t pos = before + block_excl_scan(cntw, &total, scan_sh);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      uint32_t word = wv[j];
+      while (word) {
+        const int bit = __ffs(word) - 1;
+        word &= word - 1;
+        if (pos < static_cast<uint32_t>(k)) out[pos] = static_cast<int32_t>(((w0 + j) << 5) + bit);
+        ++pos;
+      }
     }
     before += total;
   }
@@ -452,17 +541,18 @@ size_t align_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 bool use_row_path(int64_t R, int64_t N) { return N <= kRowPathMaxN && R > 256; }
 
 struct LongLayout {
-  size_t scores, hist, cnt, thr, cand, bitmap, total;
+  size_t scores, hist, cnt, done, thr, cand, bitmap, total;
   int64_t W;
 };
 
 LongLayout long_layout(int64_t R, int64_t N) {
   LongLayout L;
-  L.W = (N + 31) / 32;
+  L.W = ((N + 31) / 32 + 15) / 16 * 16;  // 16-word multiple: vector reads stay in the row
   size_t off = 0;
   L.scores = off; off = align_up(off + static_cast<size_t>(R) * N * 4);
-  L.hist = off;   off += static_cast<size_t>(R) * kHistBins * 4;     // hist and cnt are zeroed together
-  L.cnt = off;    off = align_up(off + static_cast<size_t>(R) * 4);
+  L.hist = off;   off += static_cast<size_t>(R) * kHistBins * 4;     // hist, cnt and done: zeroed together
+  L.cnt = off;    off += static_cast<size_t>(R) * 4;
+  L.done = off;   off = align_up(off + static_cast<size_t>(R) * 8);
   L.thr = off;    off = align_up(off + static_cast<size_t>(R) * 8);
   L.cand = off;   off = align_up(off + static_cast<size_t>(R) * N * 8);
   L.bitmap = off; off = align_up(off + static_cast<size_t>(R) * L.W * 4);
@@ -533,6 +623,9 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
     p.chunk = 2048;
     p.scores = reinterpret_cast<float*>(ws);
     p.hist = nullptr;
+    p.done = nullptr;
+    p.thr = nullptr;
+    p.k = k;
     const int64_t groups = (Tq + QR - 1) / QR;
     dim3 grid(static_cast<unsigned>((N + p.chunk - 1) / p.chunk), static_cast<unsigned>(B * groups));
     CSA_REQUIRE(B * groups < 65536, "csa_indexer_topk: too many query rows for one launch");
@@ -541,15 +634,8 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
     prof_end(s);
     if (csa_status st = check_launch("indexer score"); st != CSA_OK) return st;
     const size_t smem = static_cast<size_t>(N) * 4;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-      if (cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowPathMaxN * 4) !=
-          cudaSuccess)
-        return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
-      if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
+    if (!ensure_smem(reinterpret_cast<const void*>(topk_rows_kernel), kRowPathMaxN * 4))
+      return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
     topk_rows_kernel<<<static_cast<unsigned>(R), 1024, smem, s>>>(p.scores, N, Tq, q_pos0, m, k, idx);
     return check_launch("indexer top-k (rows)");
   }
@@ -559,6 +645,7 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
   w.scores = reinterpret_cast<float*>(ws + L.scores);
   w.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
   w.cand_cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
+  w.done = reinterpret_cast<uint32_t*>(ws + L.done);
   w.thr = reinterpret_cast<int32_t*>(ws + L.thr);
   w.cand = reinterpret_cast<uint2*>(ws + L.cand);
   w.bitmap = reinterpret_cast<uint32_t*>(ws + L.bitmap);
@@ -568,19 +655,20 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
   p.chunk = 4096;
   p.scores = w.scores;
   p.hist = w.hist;
+  p.done = w.done;
+  p.thr = w.thr;
+  p.k = k;
   CSA_REQUIRE(R < 65536, "csa_indexer_topk: too many query rows for the long-row path");
   dim3 grid(static_cast<unsigned>((N + p.chunk - 1) / p.chunk), static_cast<unsigned>(R));
+  if (!ensure_smem(reinterpret_cast<const void*>(score_kernel<1, true>), tile_smem + kHistBins * 4))
+    return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
   prof_begin(s);
   score_kernel<1, true><<<grid, kScoreThreads, tile_smem + kHistBins * 4, s>>>(p);
   prof_end(s);
   if (csa_status st = check_launch("indexer score (long rows)"); st != CSA_OK) return st;
-  topk_threshold_kernel<<<static_cast<unsigned>(R), 1024, 0, s>>>(w, N, Tq, q_pos0, m, k);
-  if (csa_status st = check_launch("indexer threshold"); st != CSA_OK) return st;
   dim3 sgrid(static_cast<unsigned>((N + kSelChunk - 1) / kSelChunk), static_cast<unsigned>(R));
-  topk_select_kernel<<<sgrid, kSelThreads, 0, s>>>(w, N, Tq, q_pos0, m);
-  if (csa_status st = check_launch("indexer select"); st != CSA_OK) return st;
-  topk_finalize_kernel<<<static_cast<unsigned>(R), 1024, 0, s>>>(w, N, Tq, q_pos0, m, k, idx);
-  return check_launch("indexer finalize");
+  topk_select_kernel<<<sgrid, kSelThreads, 0, s>>>(w, N, Tq, q_pos0, m, k, idx);
+  return check_launch("indexer select");
 }
 
 }  // extern "C"
