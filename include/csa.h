@@ -63,7 +63,8 @@ typedef enum csa_status {
   CSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or shape   */
   CSA_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels support   */
   CSA_ERR_WORKSPACE = 3,     /* workspace pointer NULL or smaller than asked */
-  CSA_ERR_CUDA = 4           /* a CUDA runtime call or launch failed         */
+  CSA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed         */
+  CSA_ERR_DEVICE_TIMEOUT = 5 /* a kernel gave up a bounded wait (see below)  */
 } csa_status;
 
 typedef enum csa_kv_layout {
@@ -102,6 +103,16 @@ CSA_API const char* csa_version(void);
 CSA_API const char* csa_status_string(int32_t status);
 /* Message for the last failing call made by this thread ("" if none). */
 CSA_API const char* csa_last_error(void);
+
+/*
+ * csa_check_device_error -- synchronises `stream`, then reports (and clears)
+ * the device error word of the attention kernels: their waits on tensor-core
+ * completion barriers are bounded, and a wait that runs out records an error
+ * instead of hanging; the affected outputs are then not valid.  Returns
+ * CSA_OK, CSA_ERR_DEVICE_TIMEOUT, or CSA_ERR_CUDA if the synchronisation
+ * itself fails.
+ */
+CSA_API csa_status csa_check_device_error(void* stream);
 
 /*
  * csa_profile_next_call -- timing hook (library infrastructure, not part of

@@ -10,7 +10,7 @@ LIB_PATH = os.path.join(_HERE, "libcsa.so")
 
 c_i32, c_i64, c_f32, c_sz, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
 
-CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUDA = 0, 1, 2, 3, 4
+CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUDA, CSA_ERR_DEVICE_TIMEOUT = 0, 1, 2, 3, 4, 5
 CSA_KV_BF16, CSA_KV_SPLIT_FP8 = 0, 1
 
 # every symbol include/csa.h declares, with (restype, argtypes)
@@ -19,6 +19,7 @@ SIGNATURES = {
     "csa_status_string": (ctypes.c_char_p, [c_i32]),
     "csa_last_error": (ctypes.c_char_p, []),
     "csa_profile_next_call": (c_i32, [c_vp, c_vp]),
+    "csa_check_device_error": (c_i32, [c_vp]),
     "csa_compress": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "hca_compress": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "csa_indexer_topk_workspace_size": (c_sz, [c_i64, c_i64, c_i64, c_i32]),

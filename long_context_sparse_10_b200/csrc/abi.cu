@@ -99,6 +99,7 @@ const char* csa_status_string(int32_t s) {
     case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED";
     case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE";
     case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
+    case CSA_ERR_DEVICE_TIMEOUT: return "CSA_ERR_DEVICE_TIMEOUT";
     default: return "CSA_ERR_UNKNOWN";
   }
 }

@@ -34,6 +34,7 @@
 
 #include "common.cuh"
 #include "host_util.h"
+#include "tc.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -433,6 +434,471 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// H = 64: tcgen05 path.  One elected thread issues the MMAs; accumulators live
+// in tensor memory (TMEM).  A tile is 128 keys.  An M = 64 accumulator fills
+// 16 of the 32 lanes of each TMEM lane quarter (row m -> lane (m % 16) +
+// 32 (m / 16)); a second one at lane offset 16 fills the other half.  So
+//   S = Q K^T of keys 0..63   -> lanes +0,  columns [0, 64)
+//   S = Q K^T of keys 64..127 -> lanes +16, columns [0, 64)
+//   O channels 0..63          -> lanes +0,  columns [64, 128)
+//   O channels 64..127        -> lanes +16, columns [64, 128)
+// and thread (warp q, lane L) owns head 16q + L % 16 and half L / 16 of both:
+// every lane works, and the two halves of a head combine their row max with
+// one shuffle.  Operands sit in shared memory in the 128-byte-swizzled layout
+// (8 rows x 128 bytes per 1024-byte atom): Q and K K-major in three 64-dim
+// blocks, P K-major in two 64-key blocks, V read MN-major straight out of the
+// first two K blocks when key and value are shared.  O is rescaled in TMEM
+// only when a row's running max grows by more than 2^8 (probabilities stay <=
+// 256 in between).  FP8 entries are dequantised (code x scale, rounded to
+// bf16) while widening into the K tile.  Every mbarrier wait is bounded; a
+// timeout sets the device error word instead of hanging.
+// ---------------------------------------------------------------------------
+constexpr int kTcKeys = 128;
+
+constexpr int kTcThreads = 256;  // warps 0-3: softmax + MMA issue; warps 4-7: loads
+
+struct TcLayout {
+  size_t q, k, v, p, raw, sc, stype, srow, vmask, bars, idx, total;
+};
+
+__host__ __device__ inline TcLayout tc_layout(bool fp8, bool shv, int tps) {
+  TcLayout L;
+  size_t off = 0;
+  L.q = off; off += 3 * 8192;                    // Q: 64 heads x 192 dims
+  L.k = off; off += 2 * 3 * 16384;               // K: 2 stages x 128 keys x 192 dims
+  L.v = off; if (!shv) off += 2 * 2 * 16384;     // V: 2 stages x 128 keys x 128 dims
+  L.p = off; off += 2 * 2 * 8192;                // P: 2 buffers x 64 heads x 128 keys
+  L.raw = off; if (fp8) off += 2 * 16384;        // raw E4M3 nope codes: 2 stages x 128 x 128
+  L.sc = off; off += 2 * kTcKeys * sizeof(float);
+  L.stype = off; off += 2 * kTcKeys * sizeof(int);
+  L.srow = off; off += 2 * kTcKeys * sizeof(int64_t);
+  L.vmask = off; off += 2 * 4 * sizeof(uint32_t);
+  L.bars = off; off += 128;
+  L.idx = off;  // (the producer reads the selection straight from global memory)
+  (void)tps;
+  const size_t reduce = 80 * (kDV + 4) * sizeof(float);  // cluster merge records (reuse Q/K)
+  L.total = (off > reduce ? off : reduce) + 1024;          // + alignment slack
+  return L;
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <bool FP8, bool SHV>
+__global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const TcLayout L = tc_layout(FP8, SHV, p.tps);
+  uint8_t* Qs = smem + L.q;
+  uint8_t* Kst = smem + L.k;
+  uint8_t* Vst = smem + L.v;
+  uint8_t* Pst = smem + L.p;
+  uint8_t* rawst = smem + L.raw;
+  auto sc = reinterpret_cast<float(*)[kTcKeys]>(smem + L.sc);
+  auto stype = reinterpret_cast<int(*)[kTcKeys]>(smem + L.stype);
+  auto srow = reinterpret_cast<int64_t(*)[kTcKeys]>(smem + L.srow);
+  auto vmask = reinterpret_cast<uint32_t(*)[4]>(smem + L.vmask);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [2] stage loaded
+  uint64_t* empty = full + 2;                                     // [2] PV of the stage's tile done
+  uint64_t* sdone = full + 4;                                     // [2] S of the tile done
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(full + 8);
+  constexpr int kKB = 16384;  // one 64-dim block of a 128-key tile
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t row = blockIdx.x / p.cl;
+  const int split = static_cast<int>(blockIdx.x % p.cl);
+  const int64_t b = row / p.Tq;
+  const int64_t t = p.q_pos0 + row % p.Tq;
+  const bool dense = p.idx == nullptr;
+  int64_t n_ent;
+  if (dense) {
+    n_ent = (t + 1) / p.stride;
+    if (n_ent > p.N) n_ent = p.N;
+  } else {
+    n_ent = p.k;
+  }
+  const int64_t wlo = (t - p.wlen + 1) > 0 ? (t - p.wlen + 1) : 0;
+  const int64_t n_win = p.wlen > 0 ? (t - wlo + 1) : 0;
+  const int64_t n_slots = n_ent + n_win;
+  const int64_t s0 = static_cast<int64_t>(split) * p.tps * kTcKeys;
+  int64_t s1 = s0 + static_cast<int64_t>(p.tps) * kTcKeys;
+  if (s1 > n_slots) s1 = n_slots;
+  const int ntiles = s1 > s0 ? static_cast<int>((s1 - s0 + kTcKeys - 1) / kTcKeys) : 0;
+
+  if (tid == 0) {
+    for (int i = 0; i < 6; ++i) tc::bar_init(&full[i], 1);
+    tc::bar_init_fence();
+  }
+  if (warp == 0) tc::tmem_alloc(tslot, 256);
+  for (int piece = tid; piece < 64 * 24; piece += kTcThreads) {  // Q, swizzled K-major
+    const int hh = piece / 24, ch = piece % 24;
+    cp_async16(Qs + (ch >> 3) * 8192 + tc::sw128(hh, ch & 7), p.q + (row * 64 + hh) * kDQK + ch * 8);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  tc::fence_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tslot;
+  constexpr uint32_t kHalfLane = 16u << 16;
+  bool healthy = true;  // false after a barrier wait ran out: later waits are skipped
+
+  float m_ref = -INFINITY, l = 0.f;  // consumer state (head h, key/channel half)
+  const int half = lane >> 4;
+  const int h = (warp & 3) * 16 + (lane & 15);
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t tO = tmem + 128;
+
+  if (warp >= 4) {
+    // ===================== producer: gather, widen, publish =====================
+    const int pt = tid - 128;  // 0..127: one slot per thread
+    for (int tile = 0; tile < ntiles; ++tile) {
+      const int st = tile & 1;
+      if (tile >= 2 && healthy) healthy = tc::bar_wait(&empty[st], ((tile >> 1) - 1) & 1);
+      // slot -> (type, row): 0 skip, 1 compressed entry, 2 raw window token
+      {
+        const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
+        int type = 0;
+        int64_t r = 0;
+        if (sl < s1) {
+          if (sl < n_ent) {
+            const int64_t i = dense ? sl : static_cast<int64_t>(__ldg(p.idx + row * p.k + sl));
+            if (i >= 0 && i < p.N && (i + 1) * p.stride - 1 <= t) {
+              type = 1;
+              r = b * p.N + i;
+            }
+          } else {
+            type = 2;
+            r = b * p.wrows + (wlo + (sl - n_ent) - p.wpos0);
+          }
+        }
+        stype[st][pt] = type;
+        srow[st][pt] = r;
+        const uint32_t bal = __ballot_sync(0xffffffffu, type != 0);
+        if (lane == 0) vmask[st][warp - 4] = bal;
+      }
+      named_sync(1, 128);
+      uint8_t* Kt = Kst + st * 3 * kKB;
+      uint8_t* Vt = Vst + st * 2 * kKB;
+      // The tile's slots are an entry run [0, ne) then a window run [ne, ne + nw):
+      // contiguous runs are copied with consecutive lanes on consecutive 16-byte
+      // chunks (512-byte warp requests); selected entries are gathered four keys
+      // per warp instruction (8 lanes per 128-byte row).
+      const int64_t a0 = s0 + static_cast<int64_t>(tile) * kTcKeys;
+      const int64_t a1 = (a0 + kTcKeys) < s1 ? (a0 + kTcKeys) : s1;
+      const int ne = static_cast<int>(((a1 < n_ent ? a1 : n_ent) - a0) > 0 ? ((a1 < n_ent ? a1 : n_ent) - a0) : 0);
+      const int nw = static_cast<int>(a1 - a0) - ne;
+      const int pwarp = warp - 4;
+      if (ne > 0 && dense) {
+        const int64_t r0 = srow[st][0];
+        if (FP8) {
+          for (int pc = pt; pc < ne * 8; pc += 128) {
+            cp_async16(rawst + st * kKB + pc * 16, p.cnope + r0 * kDNope + pc * 16);
+            cp_async16(Kt + 2 * kKB + tc::sw128(pc >> 3, pc & 7), p.crope + r0 * kDRope + pc * 8);
+          }
+          if (pt < ne) cp_async4(&sc[st][pt], p.cscale + r0 + pt);
+        } else {
+          for (int pc = pt; pc < ne * 24; pc += 128) {
+            const int key = pc / 24, c = pc % 24;
+            cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.ck + r0 * kDQK + pc * 8);
+          }
+          if (!SHV) {
+            for (int pc = pt; pc < ne * 16; pc += 128) {
+              const int key = pc >> 4, c = pc & 15;
+              const __nv_bfloat16* src = p.cv ? p.cv + r0 * kDV + pc * 8 : p.ck + (r0 + key) * kDQK + c * 8;
+              cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), src);
+            }
+          }
+        }
+      } else if (ne > 0) {
+        const int c = lane & 7;
+        for (int kb = pwarp * 4; kb < ne; kb += 16) {
+          const int key = kb + (lane >> 3);
+          if (key >= ne) continue;
+          const int type = stype[st][key];
+          const int64_t r = srow[st][key];
+          const int bytes = type ? 16 : 0;
+          if (FP8) {
+            cp_async16(rawst + st * kKB + key * kDNope + c * 16, type ? p.cnope + r * kDNope + c * 16 : p.cnope, bytes);
+            cp_async16(Kt + 2 * kKB + tc::sw128(key, c), type ? p.crope + r * kDRope + c * 8 : p.crope, bytes);
+            if (c == 0) {
+              if (type)
+                cp_async4(&sc[st][key], p.cscale + r);
+              else
+                sc[st][key] = 1.f;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 3; ++j)
+              cp_async16(Kt + j * kKB + tc::sw128(key, c), type ? p.ck + r * kDQK + (8 * j + c) * 8 : p.ck, bytes);
+            if (!SHV) {
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const __nv_bfloat16* src = !type ? p.ck : (p.cv ? p.cv + r * kDV + (8 * j + c) * 8
+                                                                : p.ck + r * kDQK + (8 * j + c) * 8);
+                cp_async16(Vt + j * kKB + tc::sw128(key, c), src, bytes);
+              }
+            }
+          }
+        }
+      }
+      if (nw > 0) {  // raw window tokens: contiguous rows
+        const int64_t rw0 = srow[st][ne];
+        for (int pc = pt; pc < nw * 24; pc += 128) {
+          const int key = ne + pc / 24, c = pc % 24;
+          cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.wk + rw0 * kDQK + pc * 8);
+        }
+        if (!SHV) {
+          for (int pc = pt; pc < nw * 16; pc += 128) {
+            const int key = ne + (pc >> 4), c = pc & 15;
+            const __nv_bfloat16* src = p.wv ? p.wv + rw0 * kDV + pc * 8 : p.wk + (rw0 + (pc >> 4)) * kDQK + c * 8;
+            cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), src);
+          }
+        }
+        if (FP8 && pt >= ne && pt < ne + nw) sc[st][pt] = 1.f;
+      }
+      // slots past the end of the row: zero rows (their logits are masked)
+      for (int pc = pt; pc < (kTcKeys - ne - nw) * 24; pc += 128) {
+        const int key = ne + nw + pc / 24, c = pc % 24;
+        cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.q, 0);
+      }
+      if (!SHV) {
+        for (int pc = pt; pc < (kTcKeys - ne - nw) * 16; pc += 128) {
+          const int key = ne + nw + (pc >> 4), c = pc & 15;
+          cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.q, 0);
+        }
+      }
+      if (FP8 && pt >= ne + nw) sc[st][pt] = 1.f;
+      cp_async_commit();
+      cp_async_wait<0>();
+      named_sync(1, 128);
+      if (FP8) {  // code * scale -> bf16 into the swizzled K (and V) tile
+        for (int piece = pt; piece < kTcKeys * 8; piece += 128) {
+          const int key = piece >> 3, c = piece & 7;
+          if (stype[st][key] != 1) continue;
+          const uint4 codes = *reinterpret_cast<const uint4*>(rawst + st * kKB + key * kDNope + c * 16);
+          const float scl = sc[st][key];
+          const uint32_t w4[4] = {codes.x, codes.y, codes.z, codes.w};
+          uint32_t outw[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+              __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                  static_cast<__nv_fp8x2_storage_t>((w4[q] >> (16 * hlf)) & 0xffffu), __NV_E4M3);
+              const float2 f = __half22float2(*reinterpret_cast<__half2*>(&hr));
+              outw[2 * q + hlf] = pack_bf16x2(f.x * scl, f.y * scl);
+            }
+          }
+          const int blk = c >> 2;
+          const uint4 lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+          const uint4 hi = make_uint4(outw[4], outw[5], outw[6], outw[7]);
+          *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
+          *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
+          if (!SHV) {
+            uint8_t* Vt = Vst + st * 2 * kKB;
+            *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
+            *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
+          }
+        }
+      }
+      tc::fence_async_smem();
+      named_sync(1, 128);
+      if (pt == 0) bar_arrive(&full[st]);
+    }
+  } else {
+    // ===================== consumer: S MMA, softmax, PV MMA =====================
+    constexpr uint32_t kIdescS = tc::idesc_bf16(64, 64, false);
+    constexpr uint32_t kIdescO = tc::idesc_bf16(64, 64, true);
+    auto issue_s = [&](int tile) {  // thread 0 only
+      const int st = tile & 1;
+      const uint32_t tS = tmem + 64 * st;
+      const uint32_t qa = smem_u32(Qs), ka = smem_u32(Kst + st * 3 * kKB);
+      tc::fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < 12; ++kk) {
+        const uint64_t adesc = tc::desc_sw128(qa + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+        const uint32_t kb = ka + (kk >> 2) * kKB + (kk & 3) * 32;
+        tc::mma_bf16_ss(tS, adesc, tc::desc_sw128(kb, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+        tc::mma_bf16_ss(tS + kHalfLane, adesc, tc::desc_sw128(kb + 64 * 128, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(&sdone[st]);
+    };
+    if (ntiles > 0 && tid == 0) {
+      if (healthy) healthy = tc::bar_wait(&full[0], 0);
+      issue_s(0);
+    }
+    for (int tile = 0; tile < ntiles; ++tile) {
+      const int st = tile & 1;
+      if (healthy) healthy = tc::bar_wait(&sdone[st], (tile >> 1) & 1);
+      tc::fence_after_sync();
+      float sv[64];
+      tc::tmem_ld32(tmem + 64 * st + lane_base, sv);
+      tc::tmem_ld32(tmem + 64 * st + lane_base + 32, sv + 32);
+      const uint32_t vm0 = vmask[st][2 * half], vm1 = vmask[st][2 * half + 1];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        const bool ok = ((j < 32 ? vm0 : vm1) >> (j & 31)) & 1u;
+        sv[j] = ok ? sv[j] * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, sv[j]);
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m_ref, mx);
+      const bool resc = m_new > m_ref + 8.f;
+      float corr = 1.f;
+      if (resc) {
+        corr = exp2f(m_ref - m_new);
+        m_ref = m_new;
+        l *= corr;
+      }
+      const float base = m_ref == -INFINITY ? 0.f : m_ref;
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        sv[j] = exp2f(sv[j] - base);
+        sum += sv[j];
+      }
+      l += sum;
+      if (tile > 0 && __any_sync(0xffffffffu, resc)) {
+        // O must be quiet: the previous tile's PV has to be done
+        if (healthy) healthy = tc::bar_wait(&empty[(tile - 1) & 1], ((tile - 1) >> 1) & 1);
+        tc::fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float ov[32];
+          tc::tmem_ld32(tO + lane_base + 32 * c, ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= corr;
+          tc::tmem_st32(tO + lane_base + 32 * c, ov);
+        }
+        tc::tmem_wait_st();
+      }
+      {
+        uint8_t* Pb = Pst + st * 2 * 8192 + half * 8192;  // keys half*64 .. half*64+63
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = make_uint4(pack_bf16x2(sv[8 * c], sv[8 * c + 1]), pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]),
+                                     pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]),
+                                     pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]));
+          *reinterpret_cast<uint4*>(Pb + tc::sw128(h, c)) = v;
+        }
+      }
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      named_sync(2, 128);
+      if (tid == 0) {
+        tc::fence_after_sync();
+        const uint32_t pa = smem_u32(Pst + st * 2 * 8192);
+        const uint32_t va = SHV ? smem_u32(Kst + st * 3 * kKB) : smem_u32(Vst + st * 2 * kKB);
+#pragma unroll
+        for (int ks = 0; ks < kTcKeys / 16; ++ks) {
+          const uint64_t adesc = tc::desc_sw128(pa + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+          const uint32_t vb = va + ks * 2048;
+          const uint32_t acc = (tile > 0 || ks > 0) ? 1u : 0u;
+          tc::mma_bf16_ss(tO, adesc, tc::desc_sw128(vb, kKB, 1024), kIdescO, acc);
+          tc::mma_bf16_ss(tO + kHalfLane, adesc, tc::desc_sw128(vb + kKB, kKB, 1024), kIdescO, acc);
+        }
+        tc::mma_commit(&empty[st]);
+        if (tile + 1 < ntiles) {  // next tile's S right behind this PV
+          if (healthy) healthy = tc::bar_wait(&full[st ^ 1], ((tile + 1) >> 1) & 1);
+          issue_s(tile + 1);
+        }
+      }
+    }
+    if (ntiles > 0) {
+      const int last = ntiles - 1;
+      if (healthy) healthy = tc::bar_wait(&empty[last & 1], (last >> 1) & 1);
+      tc::fence_after_sync();
+    }
+  }
+  cp_async_wait<0>();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+
+  // ---- output (consumer threads): channels half*64..+63 of head h, with (m_ref, l) ----
+  cg::cluster_group cluster = cg::this_cluster();
+  if (p.cl > 1) cluster.sync();  // peers may now write merge records over our Q/K tiles
+  float* rbuf = reinterpret_cast<float*>(smem);
+  constexpr int kRec = kDV + 4;  // 128 channels, m, l, pad: 16-byte aligned records
+  if (warp < 4) {
+    const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
+    float* dst = nullptr;
+    if (p.cl > 1) {
+      const int owner = h % p.cl;
+      dst = cluster.map_shared_rank(rbuf, owner) + (static_cast<int64_t>(h / p.cl) * p.cl + split) * kRec;
+    }
+    const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      float ov[32];
+      if (ntiles > 0) {
+        tc::tmem_ld32(tO + lane_base + 32 * c, ov);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+      }
+      const int d0 = half * 64 + 32 * c;
+      if (p.cl > 1) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(dst + d0 + i) = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
+      } else {
+        __nv_bfloat16* o = p.out + (row * p.H + h) * kDV + d0;
+#pragma unroll
+        for (int i = 0; i < 32; i += 8)
+          *reinterpret_cast<uint4*>(o + i) =
+              make_uint4(pack_bf16x2(ov[i] * inv, ov[i + 1] * inv), pack_bf16x2(ov[i + 2] * inv, ov[i + 3] * inv),
+                         pack_bf16x2(ov[i + 4] * inv, ov[i + 5] * inv), pack_bf16x2(ov[i + 6] * inv, ov[i + 7] * inv));
+      }
+    }
+    if (half == 0) {
+      if (p.cl > 1) {
+        dst[kDV] = m_ref;
+        dst[kDV + 1] = l_row;
+      } else if (p.lse) {
+        p.lse[row * p.H + h] = l_row > 0.f ? (m_ref + log2f(l_row)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 256);
+  if (p.cl == 1) return;
+  cluster.sync();
+  const int sub = tid >> 5;  // 8 warps, one head at a time each
+  for (int j = sub; split + j * p.cl < p.H; j += 8) {
+    const int hh = split + j * p.cl;
+    const float* rec = rbuf + static_cast<int64_t>(j) * p.cl * kRec;
+    float M = -INFINITY;
+    for (int c = 0; c < p.cl; ++c) M = fmaxf(M, rec[c * kRec + kDV]);
+    const float bse = M == -INFINITY ? 0.f : M;
+    float Lsum = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int c = 0; c < p.cl; ++c) {
+      const float* r = rec + c * kRec;
+      const float w = exp2f(r[kDV] - bse);
+      Lsum += w * r[kDV + 1];
+      const float4 u = *reinterpret_cast<const float4*>(r + lane * 4);
+      a0 += w * u.x;
+      a1 += w * u.y;
+      a2 += w * u.z;
+      a3 += w * u.w;
+    }
+    const float iv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    *reinterpret_cast<uint2*>(p.out + (row * p.H + hh) * kDV + lane * 4) =
+        make_uint2(pack_bf16x2(a0 * iv, a1 * iv), pack_bf16x2(a2 * iv, a3 * iv));
+    if (lane == 0 && p.lse) p.lse[row * p.H + hh] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -440,8 +906,8 @@ struct Plan {
   int cl, tps;
 };
 
-Plan plan(int64_t R, int64_t max_slots) {
-  const int64_t tiles = max_slots > 0 ? (max_slots + kKeys - 1) / kKeys : 1;
+Plan plan(int64_t R, int64_t max_slots, int tile_keys) {
+  const int64_t tiles = max_slots > 0 ? (max_slots + tile_keys - 1) / tile_keys : 1;
   const int64_t target = 2LL * num_sms();
   int64_t cl = 1;
   if (R < target) {
@@ -465,8 +931,17 @@ KernelFn pick(int H, bool fp8, bool shv) {
   return shv ? attn_kernel<4, false, true> : attn_kernel<4, false, false>;
 }
 
+KernelFn pick_tc(bool fp8, bool shv) {
+  if (fp8) return shv ? attn_tc_kernel<true, true> : attn_tc_kernel<true, false>;
+  return shv ? attn_tc_kernel<false, true> : attn_tc_kernel<false, false>;
+}
+
+size_t smem_bytes(bool use_tc, bool fp8, bool shv, int tps) {
+  return use_tc ? tc_layout(fp8, shv, tps).total : smem_layout(fp8, shv, tps).total;
+}
+
 // Largest cluster size <= want that the device can co-schedule for this kernel.
-int feasible_cluster(KernelFn fn, int want, size_t smem) {
+int feasible_cluster(KernelFn fn, int want, size_t smem, int threads) {
   static std::mutex mu;
   static std::map<std::tuple<int, const void*, int, size_t>, int> cache;
   int dev = 0;
@@ -479,7 +954,7 @@ int feasible_cluster(KernelFn fn, int want, size_t smem) {
   while (cl > 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(cl));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
@@ -557,9 +1032,13 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   const bool win_shared_v = wlen == 0 || win->v == nullptr;
   const bool shv = cache_shared_v && win_shared_v;
   const int64_t max_slots = (idx ? k : N) + wlen;
-  Plan pl = plan(R, max_slots);
-  KernelFn fn = pick(H, fp8, shv);
-  size_t smem = smem_layout(fp8, shv, pl.tps).total;
+  // tcgen05 path for 64 heads; H = 16, and an FP8 cache combined with a separate
+  // raw-window V (too much shared memory for the staged tiles), use the warp-MMA kernel
+  const bool use_tc = H == 64 && !(fp8 && !shv);
+  const int tile_keys = use_tc ? kTcKeys : kKeys;
+  Plan pl = plan(R, max_slots, tile_keys);
+  KernelFn fn = use_tc ? pick_tc(fp8, shv) : pick(H, fp8, shv);
+  size_t smem = smem_bytes(use_tc, fp8, shv, pl.tps);
   if (!ensure_smem(reinterpret_cast<const void*>(fn), static_cast<int>(smem)))
     return fail(CSA_ERR_CUDA, "%s: cannot raise the shared memory limit to %zu", name, smem);
   if (pl.cl > 1) {
@@ -571,12 +1050,12 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
         pl.cl = pl.cl > 8 ? 8 : pl.cl;  // portable cluster sizes only
       }
     }
-    const int cl = feasible_cluster(fn, pl.cl, smem);
+    const int cl = feasible_cluster(fn, pl.cl, smem, use_tc ? kTcThreads : kThreads);
     if (cl != pl.cl) {  // re-plan with the co-schedulable cluster size
-      const int64_t tiles = max_slots > 0 ? (max_slots + kKeys - 1) / kKeys : 1;
+      const int64_t tiles = max_slots > 0 ? (max_slots + tile_keys - 1) / tile_keys : 1;
       pl.tps = static_cast<int>((tiles + cl - 1) / cl);
       pl.cl = static_cast<int>((tiles + pl.tps - 1) / pl.tps);
-      smem = smem_layout(fp8, shv, pl.tps).total;
+      smem = smem_bytes(use_tc, fp8, shv, pl.tps);
       if (!ensure_smem(reinterpret_cast<const void*>(fn), static_cast<int>(smem)))
         return fail(CSA_ERR_CUDA, "%s: cannot raise the shared memory limit to %zu", name, smem);
     }
@@ -609,7 +1088,7 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(R * pl.cl));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(use_tc ? kTcThreads : kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr;
@@ -630,6 +1109,21 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
 }  // namespace csa
 
 extern "C" {
+
+csa_status csa_check_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return csa::fail(CSA_ERR_CUDA, "csa_check_device_error: %s", cudaGetErrorString(e));
+  int word = 0;
+  e = cudaMemcpyFromSymbol(&word, csa::tc::g_device_error, sizeof(int));
+  if (e != cudaSuccess) return csa::fail(CSA_ERR_CUDA, "csa_check_device_error: %s", cudaGetErrorString(e));
+  if (word != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(csa::tc::g_device_error, &zero, sizeof(int));
+    return csa::fail(CSA_ERR_DEVICE_TIMEOUT, "a kernel gave up waiting on a tensor-core barrier (code %d); its "
+                     "outputs are not valid", word);
+  }
+  return CSA_OK;
+}
 
 size_t csa_sparse_mqa_workspace_size(int64_t B, int64_t Tq, int32_t H, int32_t k, int32_t win_len) {
   (void)B, (void)Tq, (void)H, (void)k, (void)win_len;
