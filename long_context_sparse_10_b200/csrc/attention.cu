@@ -940,36 +940,48 @@ size_t smem_bytes(bool use_tc, bool fp8, bool shv, int tps) {
   return use_tc ? tc_layout(fp8, shv, tps).total : smem_layout(fp8, shv, tps).total;
 }
 
-// Largest cluster size <= want that the device can co-schedule for this kernel.
-int feasible_cluster(KernelFn fn, int want, size_t smem, int threads) {
+// Clusters of this kernel (cluster size cl, given shared memory and block size)
+// the device can keep resident at once; 0 if it cannot run them at all.
+int max_active_clusters(KernelFn fn, int cl, size_t smem, int threads) {
   static std::mutex mu;
-  static std::map<std::tuple<int, const void*, int, size_t>, int> cache;
+  static std::map<std::tuple<int, const void*, int, size_t, int>, int> cache;
   int dev = 0;
   cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_tuple(dev, reinterpret_cast<const void*>(fn), want, smem);
+  const auto key = std::make_tuple(dev, reinterpret_cast<const void*>(fn), cl, smem, threads);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
-  int cl = want;
-  while (cl > 1) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(cl));
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = cl;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) == cudaSuccess && n > 0) break;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(cl));
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = cl;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
     cudaGetLastError();
-    --cl;
+    n = 0;
   }
-  cache[key] = cl;
-  return cl;
+  cache[key] = n;
+  return n;
+}
+
+// Cluster size for `rows` rows of `tiles` tiles each: the largest size <= want
+// whose clusters all fit on the device at once (one wave); if none does, the
+// largest size that runs at all.
+int choose_cluster(KernelFn fn, int want, int64_t rows, size_t smem, int threads) {
+  int fallback = 1;
+  for (int cl = want; cl > 1; --cl) {
+    const int n = max_active_clusters(fn, cl, smem, threads);
+    if (n >= rows) return cl;
+    if (n > 0 && fallback == 1) fallback = cl;
+  }
+  return fallback;
 }
 
 csa_status check_cache(const char* name, const csa_kv_cache* c) {
@@ -1050,7 +1062,7 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
         pl.cl = pl.cl > 8 ? 8 : pl.cl;  // portable cluster sizes only
       }
     }
-    const int cl = feasible_cluster(fn, pl.cl, smem, use_tc ? kTcThreads : kThreads);
+    const int cl = choose_cluster(fn, pl.cl, R, smem, use_tc ? kTcThreads : kThreads);
     if (cl != pl.cl) {  // re-plan with the co-schedulable cluster size
       const int64_t tiles = max_slots > 0 ? (max_slots + tile_keys - 1) / tile_keys : 1;
       pl.tps = static_cast<int>((tiles + cl - 1) / cl);

@@ -360,7 +360,9 @@ __global__ void __launch_bounds__(1024) topk_rows_kernel(const float* __restrict
 // kernel whose last CTA per row resolves the threshold bin and writes the list
 // ---------------------------------------------------------------------------
 constexpr int kSelThreads = 512;
-constexpr int kSelChunk = 4096;
+constexpr int kSelChunk = 8192;         // entries per select CTA
+constexpr int kCandSmem = 4096;         // threshold-bin candidates kept in shared memory
+constexpr int kBitmapSmemWords = 8192;  // rows up to 262144 entries emit from a shared-memory bitmap
 
 struct LongWs {
   float* scores;        // [R, N]
@@ -377,15 +379,18 @@ struct LongWs {
 // bin), and the threshold bin's entries appended to the row's candidate list
 // (gathered in shared memory first, one global atomic per CTA).  The last CTA
 // of a row then radix-selects the `need` best candidates on the composite key
-// (score key << 32 | ~index), adds them to the bitmap and writes the row's
-// ascending index list.
+// (score key << 32 | ~index), merges them into the row's bitmap and writes the
+// ascending index list.  Rows up to kBitmapSmemWords*32 entries keep that final
+// bitmap in shared memory.
 __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, int64_t N, int64_t Tq, int64_t q_pos0,
-                                                                  int m, int k, int32_t* __restrict__ idx) {
-  __shared__ uint2 cand_s[kSelChunk];
+                                                                     int m, int k, int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) uint8_t sel_smem[];  // candidates, then the final bitmap
+  uint2* cand_s = reinterpret_cast<uint2*>(sel_smem);
+  uint32_t* bm_s = reinterpret_cast<uint32_t*>(sel_smem + kCandSmem * sizeof(uint2));
   __shared__ uint32_t hist[256];
   __shared__ uint32_t dig[3];
   __shared__ uint32_t scan_sh[32];
-  __shared__ uint32_t n_cand, base_s, last_s;
+  __shared__ uint32_t n_cand, base_s, last_s, spill_base;
   const int64_t row = blockIdx.y;
   const int64_t nv = visible(q_pos0 + row % Tq, m, N);
   const int64_t e_begin = static_cast<int64_t>(blockIdx.x) * kSelChunk;
@@ -424,11 +429,18 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
       uint32_t pos = 0;
       if (lane == 0) pos = atomicAdd(&n_cand, static_cast<uint32_t>(__popc(cm)));
       pos = __shfl_sync(0xffffffffu, pos, 0);
-      if (cnd) cand_s[pos + __popc(cm & ((1u << lane) - 1u))] = make_uint2(key, static_cast<uint32_t>(i));
+      const uint32_t my = pos + __popc(cm & ((1u << lane) - 1u));
+      if (cnd) {
+        if (my < static_cast<uint32_t>(kCandSmem)) {
+          cand_s[my] = make_uint2(key, static_cast<uint32_t>(i));
+        } else {  // rare (many equal scores): straight to the row's list
+          ws.cand[row * N + atomicAdd(ws.cand_cnt + row, 1u)] = make_uint2(key, static_cast<uint32_t>(i));
+        }
+      }
     }
   }
   __syncthreads();
-  const uint32_t nc = n_cand;
+  const uint32_t nc = n_cand < static_cast<uint32_t>(kCandSmem) ? n_cand : static_cast<uint32_t>(kCandSmem);
   if (threadIdx.x == 0 && nc) base_s = atomicAdd(ws.cand_cnt + row, nc);
   __syncthreads();
   for (uint32_t c = threadIdx.x; c < nc; c += kSelThreads) ws.cand[row * N + base_s + c] = cand_s[c];
@@ -442,11 +454,25 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   __syncthreads();
   if (!last_s) return;
   __threadfence();
+  (void)spill_base;
 
-  // ---- resolve the threshold bin: radix select on the 52 low composite bits
+  // ---- load the row's candidates (when they fit) and bitmap (when it fits) together
+  const int64_t words = (nv + 31) >> 5;
   const uint32_t cnt = __ldcg(ws.cand_cnt + row);
   const uint2* cand = ws.cand + row * N;
-  if (cnt <= static_cast<uint32_t>(kSelChunk)) {  // usual case: work on a shared-memory copy
+  uint32_t* gbm = ws.bitmap + row * ws.W;
+  const bool bm_in_smem = words <= kBitmapSmemWords;
+  const bool cand_in_smem = cnt <= static_cast<uint32_t>(kCandSmem);
+  if (bm_in_smem) {
+    for (int64_t w0 = 4 * threadIdx.x; w0 < words; w0 += 4 * kSelThreads) {
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(gbm + w0));
+      bm_s[w0] = v.x;
+      if (w0 + 1 < words) bm_s[w0 + 1] = v.y;
+      if (w0 + 2 < words) bm_s[w0 + 2] = v.z;
+      if (w0 + 3 < words) bm_s[w0 + 3] = v.w;
+    }
+  }
+  if (cand_in_smem) {
     for (uint32_t c0 = 0; c0 < cnt; c0 += 4 * kSelThreads) {
       uint2 v[4];
 #pragma unroll
@@ -460,9 +486,11 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
         if (c < cnt) cand_s[c] = v[u];
       }
     }
-    __syncthreads();
     cand = cand_s;
   }
+  __syncthreads();
+
+  // ---- resolve the threshold bin: radix select on the 52 low composite bits
   uint32_t remaining = static_cast<uint32_t>(ws.thr[2 * row + 1]);
   uint64_t prefix = static_cast<uint64_t>(thr_bin) << 52;
   uint64_t mask = 0xfffull << 52;
@@ -473,7 +501,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
     for (int j = threadIdx.x; j < 256; j += kSelThreads) hist[j] = 0;
     __syncthreads();
     for (uint32_t c = threadIdx.x; c < cnt; c += kSelThreads) {
-      const uint2 kv = cand[c];
+      const uint2 kv = cand_in_smem ? cand[c] : __ldcg(cand + c);
       const uint64_t x = (static_cast<uint64_t>(kv.x) << 32) | (0xffffffffu - kv.y);
       if ((x & mask) == prefix) atomicAdd(&hist[(x >> sh) & dmask], 1u);
     }
@@ -486,37 +514,31 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
     in_bucket = dig[2];
     __syncthreads();
   }
+  uint32_t* bm = bm_in_smem ? bm_s : gbm;
   for (uint32_t c = threadIdx.x; c < cnt; c += kSelThreads) {
-    const uint2 kv = cand[c];
+    const uint2 kv = cand_in_smem ? cand[c] : __ldcg(cand + c);
     const uint64_t x = (static_cast<uint64_t>(kv.x) << 32) | (0xffffffffu - kv.y);
-    if ((x & mask) >= prefix) atomicOr(ws.bitmap + row * ws.W + (kv.y >> 5), 1u << (kv.y & 31));
+    if ((x & mask) >= prefix) atomicOr(bm + (kv.y >> 5), 1u << (kv.y & 31));
   }
-  __threadfence();
+  if (!bm_in_smem) __threadfence();
   __syncthreads();
 
   // ---- ascending list from the bitmap: 16 consecutive words per thread per round
-  const int64_t words = (nv + 31) >> 5;
-  const uint32_t* bm = ws.bitmap + row * ws.W;
   uint32_t before = 0;
   for (int64_t base = 0; base < words; base += 16 * kSelThreads) {
     const int64_t w0 = base + 16 * threadIdx.x;
     uint32_t wv[16];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 v = w0 + 4 * j < words ? __ldcg(reinterpret_cast<const uint4*>(bm + w0) + j) : make_uint4(0, 0, 0, 0);
-      wv[4 * j] = v.x;
-      wv[4 * j + 1] = v.y;
-      wv[4 * j + 2] = v.z;
-      wv[4 * j + 3] = v.w;
+    for (int j = 0; j < 16; ++j) {
+      const int64_t wi = w0 + j;
+      uint32_t word = 0;
+      if (wi < words) word = bm_in_smem ? bm_s[wi] : __ldcg(gbm + wi);
+      if (wi == words - 1 && (nv & 31)) word &= (1u << (nv & 31)) - 1u;
+      wv[j] = word;
     }
     uint32_t cntw = 0;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int64_t wi = w0 + j;
-      if (wi >= words) wv[j] = 0;
-      else if (wi == words - 1 && (nv & 31)) wv[j] &= (1u << (nv & 31)) - 1u;
-      cntw += __popc(wv[j]);
-    }
+    for (int j = 0; j < 16; ++j) cntw += __popc(wv[j]);
     uint32_t total;
     uint32_t pos = before + block_excl_scan(cntw, &total, scan_sh);
 #pragma unroll
@@ -667,7 +689,10 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
   prof_end(s);
   if (csa_status st = check_launch("indexer score (long rows)"); st != CSA_OK) return st;
   dim3 sgrid(static_cast<unsigned>((N + kSelChunk - 1) / kSelChunk), static_cast<unsigned>(R));
-  topk_select_kernel<<<sgrid, kSelThreads, 0, s>>>(w, N, Tq, q_pos0, m, k, idx);
+  constexpr int kSelSmem = kCandSmem * 8 + kBitmapSmemWords * 4;
+  if (!ensure_smem(reinterpret_cast<const void*>(topk_select_kernel), kSelSmem))
+    return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
+  topk_select_kernel<<<sgrid, kSelThreads, kSelSmem, s>>>(w, N, Tq, q_pos0, m, k, idx);
   return check_launch("indexer select");
 }
 
