@@ -106,9 +106,10 @@ CSA_API const char* csa_last_error(void);
 
 /*
  * csa_check_device_error -- synchronises `stream`, then reports (and clears)
- * the device error word of the attention kernels: their waits on tensor-core
- * completion barriers are bounded, and a wait that runs out records an error
- * instead of hanging; the affected outputs are then not valid.  Returns
+ * the device error words of the attention and indexer kernels: their waits on
+ * tensor-core and bulk-copy completion barriers are bounded, and a wait that
+ * runs out records an error instead of hanging; the affected outputs are then
+ * not valid.  Returns
  * CSA_OK, CSA_ERR_DEVICE_TIMEOUT, or CSA_ERR_CUDA if the synchronisation
  * itself fails.
  */

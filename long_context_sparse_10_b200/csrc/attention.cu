@@ -900,6 +900,275 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
 }
 
 // ---------------------------------------------------------------------------
+// Dense (HCA) prefill: one CTA per block of consecutive queries.  Its 128 MMA
+// rows are (query, head) pairs, QB = 128 / H queries.  Consecutive queries see
+// nearly the same keys (the same visible entries, overlapping windows), so the
+// union of the block's keys is staged once per 64-key tile and every row masks
+// what its own query may not see: entry i needs (i+1)m' - 1 <= t_q, a window
+// token p needs t_q - w_s < p <= t_q.  M = 128 puts row r in TMEM lane r, so
+// consumer thread r owns row r.  Producer warpgroup: coalesced copies of the
+// entry run and the window run; consumer warpgroup: softmax and MMA issue.
+// ---------------------------------------------------------------------------
+constexpr int kBlkKeys = 64;
+
+struct BlkLayout {
+  size_t q, k, v, p, bars, total;
+};
+
+__host__ __device__ inline BlkLayout blk_layout() {
+  BlkLayout L;
+  size_t off = 0;
+  L.q = off; off += 3 * 16384;          // Q: 128 rows x 192 dims (3 blocks of 128 x 128 B)
+  L.k = off; off += 2 * 3 * 8192;       // K: 2 stages x 64 keys x 192 dims
+  L.v = off; off += 2 * 2 * 8192;       // V: 2 stages x 64 keys x 128 dims
+  L.p = off; off += 2 * 16384;          // P: 2 buffers x 128 rows x 64 keys
+  L.bars = off; off += 128;
+  L.total = off + 1024;
+  return L;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) attn_block_kernel(AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const BlkLayout L = blk_layout();
+  uint8_t* Qs = smem + L.q;
+  uint8_t* Kst = smem + L.k;
+  uint8_t* Vst = smem + L.v;
+  uint8_t* Pst = smem + L.p;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* empty = full + 2;
+  uint64_t* sdone = full + 4;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(full + 8);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int H = p.H;
+  const int QB = 128 / H;
+  const int64_t nblk = (p.Tq + QB - 1) / QB;
+  const int64_t b = blockIdx.x / nblk;
+  const int64_t qb = blockIdx.x % nblk;
+  const int64_t r0 = qb * QB;                     // first query row of the block
+  const int nq = static_cast<int>((p.Tq - r0) < QB ? (p.Tq - r0) : QB);
+  const int64_t t0 = p.q_pos0 + r0, tl = t0 + nq - 1;
+  int64_t ent_n = (tl + 1) / p.stride;
+  if (ent_n > p.N) ent_n = p.N;
+  const int64_t wlo0 = (t0 - p.wlen + 1) > 0 ? (t0 - p.wlen + 1) : 0;
+  const int64_t nwin = p.wlen > 0 ? (tl - wlo0 + 1) : 0;
+  const int64_t n_slots = ent_n + nwin;
+  const int ntiles = static_cast<int>((n_slots + kBlkKeys - 1) / kBlkKeys);
+
+  if (tid == 0) {
+    for (int i = 0; i < 6; ++i) tc::bar_init(&full[i], 1);
+    tc::bar_init_fence();
+  }
+  if (warp == 0) tc::tmem_alloc(tslot, 256);
+  {  // Q rows (query, head), swizzled K-major; rows past the block's queries are zero
+    const __nv_bfloat16* qsrc = p.q + ((b * p.Tq + r0) * H) * kDQK;
+    const int valid_rows = nq * H;
+    for (int piece = tid; piece < 128 * 24; piece += kTcThreads) {
+      const int r = piece / 24, ch = piece % 24;
+      cp_async16(Qs + (ch >> 3) * 16384 + tc::sw128(r, ch & 7), r < valid_rows ? qsrc + piece * 8 : p.q,
+                 r < valid_rows ? 16 : 0);
+    }
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  tc::fence_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tslot;
+  const uint32_t tO = tmem + 128;
+  bool healthy = true;
+
+  if (warp >= 4) {
+    // ===================== producer =====================
+    const int pt = tid - 128;
+    for (int tile = 0; tile < ntiles; ++tile) {
+      const int st = tile & 1;
+      if (tile >= 2 && healthy) healthy = tc::bar_wait(&empty[st], ((tile >> 1) - 1) & 1);
+      uint8_t* Kt = Kst + st * 3 * 8192;
+      uint8_t* Vt = Vst + st * 2 * 8192;
+      const int64_t a0 = static_cast<int64_t>(tile) * kBlkKeys;
+      const int64_t a1 = (a0 + kBlkKeys) < n_slots ? (a0 + kBlkKeys) : n_slots;
+      const int ne = static_cast<int>(((a1 < ent_n ? a1 : ent_n) - a0) > 0 ? ((a1 < ent_n ? a1 : ent_n) - a0) : 0);
+      const int nw = static_cast<int>(a1 - a0) - ne;
+      if (ne > 0) {  // entries a0 .. a0+ne-1 of sequence b: contiguous rows
+        const int64_t er = b * p.N + a0;
+        for (int pc = pt; pc < ne * 24; pc += 128) {
+          const int key = pc / 24, c = pc % 24;
+          cp_async16(Kt + (c >> 3) * 8192 + tc::sw128(key, c & 7), p.ck + er * kDQK + pc * 8);
+        }
+        for (int pc = pt; pc < ne * 16; pc += 128) {
+          const int key = pc >> 4, c = pc & 15;
+          const __nv_bfloat16* src = p.cv ? p.cv + er * kDV + pc * 8 : p.ck + (er + key) * kDQK + c * 8;
+          cp_async16(Vt + (c >> 3) * 8192 + tc::sw128(key, c & 7), src);
+        }
+      }
+      if (nw > 0) {  // window positions from wlo0 + (max(a0, ent_n) - ent_n)
+        const int64_t rw = b * p.wrows + (wlo0 + (a0 + ne - ent_n) - p.wpos0);
+        for (int pc = pt; pc < nw * 24; pc += 128) {
+          const int key = ne + pc / 24, c = pc % 24;
+          cp_async16(Kt + (c >> 3) * 8192 + tc::sw128(key, c & 7), p.wk + rw * kDQK + pc * 8);
+        }
+        for (int pc = pt; pc < nw * 16; pc += 128) {
+          const int key = ne + (pc >> 4), c = pc & 15;
+          const __nv_bfloat16* src = p.wv ? p.wv + rw * kDV + pc * 8 : p.wk + (rw + (pc >> 4)) * kDQK + c * 8;
+          cp_async16(Vt + (c >> 3) * 8192 + tc::sw128(key, c & 7), src);
+        }
+      }
+      for (int pc = pt; pc < (kBlkKeys - ne - nw) * 24; pc += 128) {
+        const int key = ne + nw + pc / 24, c = pc % 24;
+        cp_async16(Kt + (c >> 3) * 8192 + tc::sw128(key, c & 7), p.q, 0);
+      }
+      for (int pc = pt; pc < (kBlkKeys - ne - nw) * 16; pc += 128) {
+        const int key = ne + nw + (pc >> 4), c = pc & 15;
+        cp_async16(Vt + (c >> 3) * 8192 + tc::sw128(key, c & 7), p.q, 0);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      tc::fence_async_smem();
+      named_sync(1, 128);
+      if (pt == 0) bar_arrive(&full[st]);
+    }
+  } else {
+    // ===================== consumer: thread tid owns row tid =====================
+    constexpr uint32_t kIdescS = tc::idesc_bf16(128, kBlkKeys, false);
+    constexpr uint32_t kIdescO = tc::idesc_bf16(128, kDV, true);
+    const int qr = tid / H;                       // query of this row within the block
+    const bool row_ok = qr < nq;
+    const int64_t tq = t0 + (row_ok ? qr : 0);
+    int64_t nv_q = (tq + 1) / p.stride;
+    if (nv_q > p.N) nv_q = p.N;
+    const int64_t lo_q = (tq - p.wlen + 1) > 0 ? (tq - p.wlen + 1) : 0;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float m_ref = -INFINITY, l = 0.f;
+    auto issue_s = [&](int tile) {
+      const int st = tile & 1;
+      const uint32_t qa = smem_u32(Qs), ka = smem_u32(Kst + st * 3 * 8192);
+      tc::fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < 12; ++kk)
+        tc::mma_bf16_ss(tmem + 64 * st, tc::desc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        tc::desc_sw128(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+      tc::mma_commit(&sdone[st]);
+    };
+    if (ntiles > 0 && tid == 0) {
+      if (healthy) healthy = tc::bar_wait(&full[0], 0);
+      issue_s(0);
+    }
+    for (int tile = 0; tile < ntiles; ++tile) {
+      const int st = tile & 1;
+      if (healthy) healthy = tc::bar_wait(&sdone[st], (tile >> 1) & 1);
+      tc::fence_after_sync();
+      float sv[kBlkKeys];
+      tc::tmem_ld32(tmem + 64 * st + lane_base, sv);
+      tc::tmem_ld32(tmem + 64 * st + lane_base + 32, sv + 32);
+      float mx = -INFINITY;
+      const int64_t sbase = static_cast<int64_t>(tile) * kBlkKeys;
+#pragma unroll
+      for (int j = 0; j < kBlkKeys; ++j) {
+        const int64_t sl = sbase + j;
+        bool ok;
+        if (sl < ent_n) {
+          ok = sl < nv_q;
+        } else {
+          const int64_t pos = wlo0 + (sl - ent_n);
+          ok = sl < n_slots && pos >= lo_q && pos <= tq;
+        }
+        ok = ok && row_ok;
+        sv[j] = ok ? sv[j] * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, sv[j]);
+      }
+      const float m_new = fmaxf(m_ref, mx);
+      const bool resc = m_new > m_ref + 8.f;
+      float corr = 1.f;
+      if (resc) {
+        corr = exp2f(m_ref - m_new);
+        m_ref = m_new;
+        l *= corr;
+      }
+      const float base = m_ref == -INFINITY ? 0.f : m_ref;
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < kBlkKeys; ++j) {
+        sv[j] = exp2f(sv[j] - base);
+        sum += sv[j];
+      }
+      l += sum;
+      if (tile > 0 && __any_sync(0xffffffffu, resc)) {
+        if (healthy) healthy = tc::bar_wait(&empty[(tile - 1) & 1], ((tile - 1) >> 1) & 1);
+        tc::fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float ov[32];
+          tc::tmem_ld32(tO + lane_base + 32 * c, ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= corr;
+          tc::tmem_st32(tO + lane_base + 32 * c, ov);
+        }
+        tc::tmem_wait_st();
+      }
+      {
+        uint8_t* Pb = Pst + st * 16384;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = make_uint4(pack_bf16x2(sv[8 * c], sv[8 * c + 1]), pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]),
+                                     pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]),
+                                     pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]));
+          *reinterpret_cast<uint4*>(Pb + tc::sw128(tid, c)) = v;
+        }
+      }
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      named_sync(2, 128);
+      if (tid == 0) {
+        tc::fence_after_sync();
+        const uint32_t pa = smem_u32(Pst + st * 16384);
+        const uint32_t va = smem_u32(Vst + st * 2 * 8192);
+#pragma unroll
+        for (int ks = 0; ks < kBlkKeys / 16; ++ks)
+          tc::mma_bf16_ss(tO, tc::desc_sw128(pa + ks * 32, 16, 1024), tc::desc_sw128(va + ks * 2048, 8192, 1024),
+                          kIdescO, (tile > 0 || ks > 0) ? 1u : 0u);
+        tc::mma_commit(&empty[st]);
+        if (tile + 1 < ntiles) {
+          if (healthy) healthy = tc::bar_wait(&full[st ^ 1], ((tile + 1) >> 1) & 1);
+          issue_s(tile + 1);
+        }
+      }
+    }
+    if (ntiles > 0) {
+      const int last = ntiles - 1;
+      if (healthy) healthy = tc::bar_wait(&empty[last & 1], (last >> 1) & 1);
+      tc::fence_after_sync();
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    __nv_bfloat16* o = p.out + ((b * p.Tq + r0) * H + tid) * kDV;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float ov[32];
+      if (ntiles > 0) {
+        tc::tmem_ld32(tO + lane_base + 32 * c, ov);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+      }
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8)
+          *reinterpret_cast<uint4*>(o + 32 * c + i) =
+              make_uint4(pack_bf16x2(ov[i] * inv, ov[i + 1] * inv), pack_bf16x2(ov[i + 2] * inv, ov[i + 3] * inv),
+                         pack_bf16x2(ov[i + 4] * inv, ov[i + 5] * inv), pack_bf16x2(ov[i + 6] * inv, ov[i + 7] * inv));
+      }
+    }
+    if (row_ok && p.lse) p.lse[(b * p.Tq + r0) * H + tid] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+  }
+  cp_async_wait<0>();
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 struct Plan {
@@ -1073,6 +1342,16 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
     }
   }
 
+  // dense (HCA) prefill over a bf16 cache: query-blocked tcgen05 kernel
+  const bool use_blk = idx == nullptr && !fp8 && Tq >= 128 / H && R >= 2LL * num_sms();
+  if (use_blk) {
+    fn = attn_block_kernel;
+    smem = blk_layout().total;
+    if (!ensure_smem(reinterpret_cast<const void*>(fn), static_cast<int>(smem)))
+      return fail(CSA_ERR_CUDA, "%s: cannot raise the shared memory limit to %zu", name, smem);
+    pl.cl = 1;
+  }
+
   AttnParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.Tq = Tq;
@@ -1099,8 +1378,8 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   p.lse = lse;
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(R * pl.cl));
-  cfg.blockDim = dim3(use_tc ? kTcThreads : kThreads);
+  cfg.gridDim = dim3(static_cast<unsigned>(use_blk ? B * ((Tq + (128 / H) - 1) / (128 / H)) : R * pl.cl));
+  cfg.blockDim = dim3(use_tc || use_blk ? kTcThreads : kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr;
@@ -1128,6 +1407,9 @@ csa_status csa_check_device_error(void* stream) {
   int word = 0;
   e = cudaMemcpyFromSymbol(&word, csa::tc::g_device_error, sizeof(int));
   if (e != cudaSuccess) return csa::fail(CSA_ERR_CUDA, "csa_check_device_error: %s", cudaGetErrorString(e));
+  const int iword = csa::indexer_device_error(true);
+  if (iword < 0) return csa::fail(CSA_ERR_CUDA, "csa_check_device_error: cannot read the indexer error word");
+  word |= iword;
   if (word != 0) {
     const int zero = 0;
     cudaMemcpyToSymbol(csa::tc::g_device_error, &zero, sizeof(int));

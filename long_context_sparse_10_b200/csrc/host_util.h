@@ -19,6 +19,8 @@ int num_sms();
 // Raises a kernel's dynamic shared memory limit to `bytes` on the current
 // device (once per device and kernel).  Returns false if the runtime refuses.
 bool ensure_smem(const void* kernel, int bytes);
+// The indexer unit's device error word (bounded barrier waits); -1 if unreadable.
+int indexer_device_error(bool clear);
 // Records the pending csa_profile_next_call start/stop event (if any) on `s`.
 void prof_begin(cudaStream_t s);
 void prof_end(cudaStream_t s);

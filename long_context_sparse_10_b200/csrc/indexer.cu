@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "host_util.h"
+#include "tc.cuh"
 
 namespace csa {
 namespace {
@@ -590,6 +591,19 @@ size_t workspace_bytes(int64_t B, int64_t Tq, int64_t N) {
 }
 
 }  // namespace
+}  // namespace csa
+
+namespace csa {
+// Reads (and optionally clears) this unit's device error word.
+int indexer_device_error(bool clear) {
+  int word = 0;
+  if (cudaMemcpyFromSymbol(&word, tc::g_device_error, sizeof(int)) != cudaSuccess) return -1;
+  if (word && clear) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(tc::g_device_error, &zero, sizeof(int));
+  }
+  return word;
+}
 }  // namespace csa
 
 extern "C" {
