@@ -178,8 +178,12 @@ class DecodeRun:
 
     def indexer(self):
         wl = self.wl
-        self.csa.csa_indexer_topk(self.d["qI"], self.d["wI"], self.d["kIc"], wl.m, wl.k, q_pos0=self.q_pos0,
-                                  idx=self.idx, workspace=self.ws_idx)
+        if wl.indexer_fp8:
+            self.csa.csa_indexer_topk_e4m3(self.d["qI"], self.d["wI"], self.d["kI_codes"], self.d["kI_scale"], wl.m,
+                                           wl.k, q_pos0=self.q_pos0, idx=self.idx, workspace=self.ws_idx)
+        else:
+            self.csa.csa_indexer_topk(self.d["qI"], self.d["wI"], self.d["kIc"], wl.m, wl.k, q_pos0=self.q_pos0,
+                                      idx=self.idx, workspace=self.ws_idx)
 
     def step(self):
         wl, csa = self.wl, self.csa
@@ -219,18 +223,22 @@ class DecodeRun:
     def dominant(self):
         """(name, source file, algorithmic bytes per launch, callable that launches it)."""
         wl = self.wl
-        b = wl.B * wl.N * 64 * 2 + wl.B * 4 * 64 * 2 + wl.B * 4 * 4
-        return "indexer_score_long", "long_context_sparse_10_b200/csrc/indexer.cu", b, "hbm", self.indexer
+        per_entry = (64 + 4) if wl.indexer_fp8 else 64 * 2  # E4M3 codes + scale, or bf16 keys
+        b = wl.B * wl.N * per_entry + wl.B * 4 * 64 * 2 + wl.B * 4 * 4
+        name = "indexer_score_long_e4m3" if wl.indexer_fp8 else "indexer_score_long"
+        return name, "long_context_sparse_10_b200/csrc/indexer.cu", b, "hbm", self.indexer
 
     def describe(self, world):
         wl = self.wl
         s = (f"{wl.name}: decode at context {wl.L}, batch {wl.B} per GPU, {wl.H} query heads, qk 192 / v 128; "
-             f"CSA m={wl.m} (N={wl.N}, FP8-e4m3 nope + BF16 RoPE cache, indexer 4x64 bf16, top-k={wl.k})")
+             f"CSA m={wl.m} (N={wl.N}, FP8-e4m3 nope + BF16 RoPE cache, indexer 4x64 "
+             f"{'e4m3 keys + per-entry scale' if wl.indexer_fp8 else 'bf16'}, top-k={wl.k})")
         if self.hybrid:
             s += f" then HCA m'={wl.m_hca} (N'={wl.N_hca}, same split cache)"
         s += f", sliding window {wl.win}"
         return {"workload": s, "global_batch": wl.B * world, "seq_len": wl.L, "parallelism": f"dp{world} (replicas)",
-                "l2": "inputs larger than L2 (the indexer streams 268 MB/step > 126 MB L2)",
+                "l2": f"inputs larger than L2 (the indexer streams {wl.B * wl.N * (68 if wl.indexer_fp8 else 128) / 1e6:.0f} "
+                      "MB/step > 126 MB L2)",
                 "timing": "CUDA graph replay of the whole step"}
 
     def oracle_sample(self, budget_s):
@@ -242,7 +250,10 @@ class DecodeRun:
         for b in range(wl.B):
             qI = h["qI"][b:b + 1].double().numpy()
             wI = h["wI"][b:b + 1].double().numpy()
-            kI = h["kIc"][b:b + 1].double().numpy()
+            if wl.indexer_fp8:
+                kI = R.e4m3_decode(h["kI_codes"][b:b + 1].numpy()) * h["kI_scale"][b:b + 1].double().numpy()[..., None]
+            else:
+                kI = h["kIc"][b:b + 1].double().numpy()
             q = h["q"][b:b + 1].double().numpy()
             wk = h["win_k"][b:b + 1].double().numpy()
             nope, rope, sc = h["nope"][b:b + 1].numpy(), h["rope"][b:b + 1].double().numpy(), h["scale"][b:b + 1].numpy()

@@ -180,6 +180,21 @@ CSA_API csa_status csa_indexer_topk(const void* qI, const float* wI, const void*
                             void* stream);
 
 /*
+ * csa_indexer_topk_e4m3 -- csa_indexer_topk over indexer keys stored in FP8
+ * (Method section, storage paragraph: the lightning indexer runs at low
+ * precision -- the pages give FP4; this layout stores E4M3 codes).  Entry i's
+ * key is kI_codes[b,i,:] (64 E4M3 bytes) times kI_scale[b,i] (fp32, > 0); the
+ * score is computed from those exact values (the scale factors out of the relu
+ * and head sums).  Same selection rule, output, workspace
+ * (csa_indexer_topk_workspace_size) and errors as csa_indexer_topk.
+ *   kI_codes uint8 [B, N, 64];  kI_scale fp32 [B, N]
+ */
+CSA_API csa_status csa_indexer_topk_e4m3(const void* qI, const float* wI, const uint8_t* kI_codes,
+                                         const float* kI_scale, int64_t B, int64_t Tq, int64_t N,
+                                         int64_t q_pos0, int32_t m, int32_t k, int32_t* idx,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * csa_indexer_topk_noalloc -- csa_indexer_topk without a caller workspace.
  * The paper has no counterpart: this is a library convenience.  Some callers
  * cannot allocate device memory themselves (for example a plugin whose host

@@ -24,7 +24,7 @@ import torch
 
 from . import _lib
 
-__all__ = ["CsaError", "KVCache", "Window", "csa_compress", "hca_compress", "csa_indexer_topk",
+__all__ = ["CsaError", "KVCache", "Window", "csa_compress", "hca_compress", "csa_indexer_topk", "csa_indexer_topk_e4m3",
            "csa_indexer_topk_workspace_size", "csa_sparse_mqa", "csa_sparse_mqa_workspace_size", "hca_dense_mqa",
            "hca_dense_mqa_workspace_size", "version"]
 
@@ -154,6 +154,22 @@ def csa_indexer_topk(qI, wI, kIc, m, k, *, q_pos0=0, idx=None, workspace=None, s
     st = lib.csa_indexer_topk(_ptr(qI), _ptr(wI), _ptr(kIc), B, Tq, N, q_pos0, m, k, _ptr(idx), _ptr(workspace),
                               workspace.numel(), _stream(stream))
     _check(st, "csa_indexer_topk")
+    return idx
+
+
+def csa_indexer_topk_e4m3(qI, wI, kI_codes, kI_scale, m, k, *, q_pos0=0, idx=None, workspace=None, stream=None):
+    """csa_indexer_topk over FP8 keys: kI_codes uint8 [B, N, 64] (E4M3), kI_scale fp32 [B, N]."""
+    lib = _lib.load()
+    B, Tq = qI.shape[0], qI.shape[1]
+    N = kI_codes.shape[1]
+    if idx is None:
+        idx = torch.empty(B, Tq, k, dtype=torch.int32, device=qI.device)
+    need = csa_indexer_topk_workspace_size(B, Tq, N, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=qI.device)
+    st = lib.csa_indexer_topk_e4m3(_ptr(qI), _ptr(wI), _ptr(kI_codes), _ptr(kI_scale), B, Tq, N, q_pos0, m, k,
+                                   _ptr(idx), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "csa_indexer_topk_e4m3")
     return idx
 
 

@@ -25,6 +25,8 @@ SIGNATURES = {
     "csa_indexer_topk_workspace_size": (c_sz, [c_i64, c_i64, c_i64, c_i32]),
     "csa_indexer_topk": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_sz,
                                  c_vp]),
+    "csa_indexer_topk_e4m3": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp,
+                                      c_sz, c_vp]),
     "csa_indexer_topk_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp]),
     "csa_sparse_mqa_workspace_size": (c_sz, [c_i64, c_i64, c_i32, c_i32, c_i32]),
     "csa_sparse_mqa": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i64, c_vp, c_i32, c_vp, c_i32, c_vp, c_f32, c_vp, c_vp,

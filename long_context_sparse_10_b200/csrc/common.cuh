@@ -76,6 +76,28 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t codes) {
   return pack_bf16x2(f.x, f.y);
 }
 
+// Two E4M3 codes (low byte first) -> two fp16 in one register, exactly (every
+// E4M3 value, subnormals included, is an fp16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes16) {
+  uint32_t r;
+  asm("{\n.reg .b16 c;\ncvt.u16.u32 c, %1;\ncvt.rn.f16x2.e4m3x2 %0, c;\n}\n" : "=r"(r) : "r"(codes16));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void mma_f16(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Order-preserving map float -> uint32 (larger float -> larger key).  -0 is
 // folded onto +0 by the callers (s + 0.0f) so equal scores get equal keys.
 __device__ __forceinline__ uint32_t f2key(float f) {

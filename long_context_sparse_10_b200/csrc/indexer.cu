@@ -21,6 +21,9 @@
 //     the entries above that bin plus a candidate list of the bin itself, and
 //     its last CTA per row resolves the candidates and writes the ascending
 //     list.  "Last CTA" is decided by an atomic counter (no CTA ever waits).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -33,17 +36,27 @@ namespace {
 constexpr int kMaxK = 4096;
 constexpr int kRowPathMaxN = 32768;  // rows up to this many visible entries live in shared memory
 constexpr int kHistBins = 4096;      // first-level bins: top 12 bits of the key
-constexpr int kStages = 4;
-constexpr int kTileRows = 64;        // entries per pipeline stage (8 KB)
-constexpr int kScoreThreads = 128;
+// Scoring pipeline shape (compile-time tunables): stages of kTileRows entries
+// (128 B each) per CTA of kScoreThreads threads; each warp owns 16 rows of a stage.
+#ifndef CSA_SCORE_STAGES
+#define CSA_SCORE_STAGES 4
+#endif
+#ifndef CSA_SCORE_WARPS
+#define CSA_SCORE_WARPS 4
+#endif
+constexpr int kStages = CSA_SCORE_STAGES;
+constexpr int kScoreThreads = 32 * CSA_SCORE_WARPS;
+constexpr int kTileRows = 16 * CSA_SCORE_WARPS;  // entries per pipeline stage
 
 struct ScoreParams {
   const __nv_bfloat16* qI;  // [B, Tq, 4, 64]
   const float* wI;          // [B, Tq, 4]
-  const __nv_bfloat16* kI;  // [B, N, 64]
+  const __nv_bfloat16* kI;  // [B, N, 64] (bf16 keys)
+  const uint8_t* kcodes;    // [B, N, 64] E4M3 key codes (E4 variant)
+  const float* kscale;      // [B, N] per-entry scale (E4 variant)
   int64_t Tq, N, q_pos0;
   int m;
-  int chunk;        // entries per CTA (multiple of kTileRows)
+  int chunk;        // entries per CTA (multiple of 2 * kTileRows)
   float* scores;    // [R, N]
   uint32_t* hist;   // [R, kHistBins] (QR == 1 only)
   uint32_t* done;   // [R, 2] CTA counters (QR == 1 only)
@@ -169,13 +182,33 @@ __device__ void row_threshold(const uint32_t* gh, int64_t nv, int k, int32_t* th
 }
 
 // Scores QR consecutive query rows of one sequence against one chunk of entries.
-template <int QR, bool HIST>
+// Shared memory of the scoring kernel: bf16 keys: kStages swizzled tiles;
+// E4M3 keys: kStages stages of codes + scales, twice the entries per stage
+// (same bytes per stage); then the histogram (HIST).
+__host__ __device__ constexpr size_t score_tile_bytes(bool e4) {
+  return e4 ? static_cast<size_t>(kStages) * (2 * kTileRows) * (64 + 4)
+            : static_cast<size_t>(kStages) * kTileRows * 128;
+}
+
+// E4M3 keys feed an fp16 MMA straight from registers.  The dot product over
+// the 64 dimensions may visit them in any order as long as A (keys) and B
+// (query) agree, so lane (g = lane/4, t = lane%4) takes dims 16t .. 16t+15 of
+// its key rows with one 16-byte shared load: k-step j, fragment slots
+// {2t, 2t+1, 2t+8, 2t+9} <- dims 16t + 4j + {0, 1, 2, 3}.  The query is scaled
+// per (row, head) by a power of two 2^e that brings its largest magnitude into
+// [2^14, 2^15) before the fp16 conversion (exact for every bf16 value in that
+// head down to 2^-28 of its maximum), and 2^-e moves onto the head weight:
+// relu(2^e x) 2^-e w = relu(x) w.
+template <int QR, bool E4>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
   constexpr int NCOL = QR * 4;
   constexpr int NT = (NCOL + 7) / 8;
+  constexpr int TR = E4 ? 2 * kTileRows : kTileRows;  // entries per stage
+  constexpr int MT = TR / kTileRows;                  // 16-row MMA tiles per warp and stage
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* tiles = smem;
-  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + kStages * kTileRows * 128);
+  uint8_t* tiles = smem;                                             // bf16: [kStages] swizzled tiles
+  uint8_t* codes_st = smem;                                          // E4: [kStages][TR][64]
+  float* scale_st = reinterpret_cast<float*>(smem + kStages * TR * 64);  // E4: [kStages][TR]
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t groups = (p.Tq + QR - 1) / QR;
@@ -187,22 +220,43 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
   if (e_begin >= nv_max) return;  // uniform for the CTA
   const int64_t e_end = (e_begin + p.chunk) < nv_max ? (e_begin + p.chunk) : nv_max;
 
-  if (HIST) {
-    for (int j = threadIdx.x; j < kHistBins; j += kScoreThreads) hist_s[j] = 0;
-  }
-
   // B operand (k = dim, n = row*4 + head), held in registers for the whole CTA.
   uint32_t bq[4][NT][2];
+  int qexp[NT];  // E4: exponent e of column n = nt*8 + lane/4
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int n = nt * 8 + (lane >> 2);
     const int rr = n >> 2, h = n & 3;
     const bool ok = n < NCOL && rr < nrows;
-    const __nv_bfloat16* qp = p.qI + (((b * p.Tq + r0 + (ok ? rr : 0)) * kHI + h) * kDI) + (lane & 3) * 2;
+    const __nv_bfloat16* qrow = p.qI + (((b * p.Tq + r0 + (ok ? rr : 0)) * kHI + h) * kDI);
+    if (E4) {
+      const __nv_bfloat16* qp = qrow + (lane & 3) * 16;
+      float qv[16];
+      float amax = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      bq[kk][nt][0] = ok ? *reinterpret_cast<const uint32_t*>(qp + kk * 16) : 0u;
-      bq[kk][nt][1] = ok ? *reinterpret_cast<const uint32_t*>(qp + kk * 16 + 8) : 0u;
+      for (int i = 0; i < 16; ++i) {
+        qv[i] = ok ? __bfloat162float(qp[i]) : 0.f;
+        amax = fmaxf(amax, fabsf(qv[i]));
+      }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      int e = 14 - (static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127);
+      e = amax > 0.f ? (e < -60 ? -60 : (e > 60 ? 60 : e)) : 0;
+      qexp[nt] = e;
+      const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        bq[kk][nt][0] = pack_f16x2(qv[4 * kk] * sc, qv[4 * kk + 1] * sc);
+        bq[kk][nt][1] = pack_f16x2(qv[4 * kk + 2] * sc, qv[4 * kk + 3] * sc);
+      }
+    } else {
+      const __nv_bfloat16* qp = qrow + (lane & 3) * 2;
+      qexp[nt] = 0;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        bq[kk][nt][0] = ok ? *reinterpret_cast<const uint32_t*>(qp + kk * 16) : 0u;
+        bq[kk][nt][1] = ok ? *reinterpret_cast<const uint32_t*>(qp + kk * 16 + 8) : 0u;
+      }
     }
   }
   // This lane's accumulator columns: row rr = nt*2 + ((lane&3)>>1), heads (lane&1)*2 + {0,1}.
@@ -217,14 +271,40 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
     const int h0 = (lane & 1) * 2;
     wv[nt][0] = ok ? p.wI[row * kHI + h0] : 0.f;
     wv[nt][1] = ok ? p.wI[row * kHI + h0 + 1] : 0.f;
+    if (E4) {  // columns 2t, 2t+1 of this n-tile were scaled by the lanes with g = 2t, 2t+1
+      const int e0 = __shfl_sync(0xffffffffu, qexp[nt], 4 * (2 * (lane & 3)));
+      const int e1 = __shfl_sync(0xffffffffu, qexp[nt], 4 * (2 * (lane & 3) + 1));
+      wv[nt][0] *= __uint_as_float(static_cast<uint32_t>(127 - e0) << 23);
+      wv[nt][1] *= __uint_as_float(static_cast<uint32_t>(127 - e1) << 23);
+    }
     nv_r[nt] = ok ? visible(p.q_pos0 + r0 + rr, p.m, p.N) : 0;
     srow[nt] = row;
   }
 
-  const int ntiles = static_cast<int>((e_end - e_begin + kTileRows - 1) / kTileRows);
+  const int ntiles = static_cast<int>((e_end - e_begin + TR - 1) / TR);
   const __nv_bfloat16* kbase = p.kI + b * p.N * kDI;
   auto load_tile = [&](int tile, int stage) {
-    const int64_t base = e_begin + static_cast<int64_t>(tile) * kTileRows;
+    const int64_t base = e_begin + static_cast<int64_t>(tile) * TR;
+    if (E4) {
+      // 64 code bytes per entry (4 pieces) and one 4-byte scale per entry
+      for (int piece = threadIdx.x; piece < TR * 4; piece += kScoreThreads) {
+        const int row = piece >> 2, ch = piece & 3;
+        const int64_t e = base + row;
+        const bool ok = e < e_end;
+        cp_async16(codes_st + (stage * TR + row) * 64 + ch * 16,
+                   p.kcodes + (b * p.N + (ok ? e : e_begin)) * kDI + ch * 16, ok ? 16 : 0);
+      }
+      for (int row = threadIdx.x; row < TR; row += kScoreThreads) {
+        const int64_t e = base + row;
+        if (e < e_end) {
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(scale_st + stage * TR + row)),
+                       "l"(p.kscale + b * p.N + e));
+        } else {
+          scale_st[stage * TR + row] = 0.f;
+        }
+      }
+      return;
+    }
 #pragma unroll
     for (int u = 0; u < (kTileRows * 8) / kScoreThreads; ++u) {
       const int piece = threadIdx.x + u * kScoreThreads;
@@ -250,57 +330,286 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
       if (nxt < ntiles) load_tile(nxt, nxt % kStages);
       cp_async_commit();
     }
-    const uint8_t* st = tiles + (tile % kStages) * (kTileRows * 128);
-    float acc[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    for (int mt = 0; mt < MT; ++mt) {
+      const int rbase = warp * (16 * MT) + mt * 16;  // this warp's first row of the stage
+      float acc[NT][4];
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const int row = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int ch = kk * 2 + (lane >> 4);
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(a0, a1, a2, a3, st + row * 128 + ((ch ^ (row & 7)) << 4));
+      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+      if (E4) {
+        const uint8_t* cs = codes_st + ((tile % kStages) * TR + rbase + (lane >> 2)) * 64 + (lane & 3) * 16;
+        const uint4 lo = *reinterpret_cast<const uint4*>(cs);
+        const uint4 hi = *reinterpret_cast<const uint4*>(cs + 8 * 64);
+        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt], a0, a1, a2, a3, bq[kk][nt][0], bq[kk][nt][1]);
-    }
-    const int64_t ebase = e_begin + static_cast<int64_t>(tile) * kTileRows + warp * 16 + (lane >> 2);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t a0 = e4m3x2_to_f16x2(wl[kk] & 0xffffu), a2 = e4m3x2_to_f16x2(wl[kk] >> 16);
+          const uint32_t a1 = e4m3x2_to_f16x2(wh[kk] & 0xffffu), a3 = e4m3x2_to_f16x2(wh[kk] >> 16);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+          for (int nt = 0; nt < NT; ++nt) mma_f16(acc[nt], a0, a1, a2, a3, bq[kk][nt][0], bq[kk][nt][1]);
+        }
+      } else {
+        const uint8_t* st = tiles + (tile % kStages) * (kTileRows * 128);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float part = fmaxf(acc[nt][2 * hf], 0.f) * wv[nt][0] + fmaxf(acc[nt][2 * hf + 1], 0.f) * wv[nt][1];
-        const float full = part + __shfl_xor_sync(0xffffffffu, part, 1) + 0.0f;
-        const int64_t e = ebase + hf * 8;
-        if ((lane & 1) == 0 && e < nv_r[nt]) {
-          p.scores[srow[nt] * p.N + e] = full;
-          if (HIST) atomicAdd(&hist_s[f2key(full) >> 20], 1u);
+        for (int kk = 0; kk < 4; ++kk) {
+          const int row = rbase + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int ch = kk * 2 + (lane >> 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(a0, a1, a2, a3, st + row * 128 + ((ch ^ (row & 7)) << 4));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt], a0, a1, a2, a3, bq[kk][nt][0], bq[kk][nt][1]);
+        }
+      }
+      const int64_t ebase = e_begin + static_cast<int64_t>(tile) * TR + rbase + (lane >> 2);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float part = fmaxf(acc[nt][2 * hf], 0.f) * wv[nt][0] + fmaxf(acc[nt][2 * hf + 1], 0.f) * wv[nt][1];
+          float full = part + __shfl_xor_sync(0xffffffffu, part, 1);
+          const int64_t e = ebase + hf * 8;
+          if (E4)  // scale > 0 factors out of relu: score = scale * sum_h relu(q_h . codes) w_h
+            full *= scale_st[(tile % kStages) * TR + rbase + (lane >> 2) + hf * 8];
+          full += 0.0f;
+          if ((lane & 1) == 0 && e < nv_r[nt]) {
+            p.scores[srow[nt] * p.N + e] = full;
+          }
         }
       }
     }
   }
   cp_async_wait<0>();
-  if (HIST) {
-    // flush the CTA histogram; the row's last CTA then derives its threshold
-    __shared__ uint32_t last_s;
-    __shared__ uint32_t scan_sh[32];
-    __syncthreads();
-    const int64_t row = b * p.Tq + r0;
-    uint32_t* gh = p.hist + row * kHistBins;
-    for (int j = threadIdx.x; j < kHistBins; j += kScoreThreads) {
-      const uint32_t c = hist_s[j];
-      if (c) atomicAdd(gh + j, c);
+}
+
+// ---------------------------------------------------------------------------
+// long rows: one query row per CTA row of the grid, histogram fused
+// ---------------------------------------------------------------------------
+// Each CTA scores one chunk of one row.  Stages of kLongTR entries arrive by
+// bulk copy (bf16 keys: one TMA box of a [B][N][64] tensor map with the
+// 128-byte swizzle that ldmatrix reads conflict-free; E4M3 keys: one
+// contiguous copy of the codes, plus 4-byte cp.async copies of the scales),
+// each completing on its stage's mbarrier.  Each warp owns 32 entries of a
+// stage: two 16-row MMA tiles whose 4 useful accumulator columns (the 4
+// heads) are folded so that every lane ends with one entry's score, and the
+// score store and histogram update run once per entry on all 32 lanes.
+constexpr int kLongThreads = 128;
+constexpr int kLongTR = 128;  // entries per stage (32 per warp)
+constexpr int kLongMinChunk = 1024;
+
+template <bool E4>
+struct LongShape {
+  static constexpr int kStages = E4 ? 4 : 3;
+  static constexpr int kStageBytes = kLongTR * (E4 ? 64 : 128);
+  static constexpr size_t kScaleOff = static_cast<size_t>(kStages) * kStageBytes;
+  static constexpr size_t kHistOff = kScaleOff + (E4 ? static_cast<size_t>(kStages) * kLongTR * 4 : 0);
+  static constexpr size_t kBarOff = kHistOff + kHistBins * 4;
+  static constexpr size_t kSmem = kBarOff + kStages * 8 + 1024;  // + alignment slack for the 1024-byte swizzle atoms
+};
+
+struct LongScoreParams {
+  const __nv_bfloat16* qI;  // [B, Tq, 4, 64]
+  const float* wI;          // [B, Tq, 4]
+  const uint8_t* kcodes;    // [B, N, 64] (E4)
+  const float* kscale;      // [B, N] (E4)
+  int64_t Tq, N, q_pos0;
+  int m;
+  int chunk;  // entries per CTA, a multiple of kLongTR
+  float* scores;
+  uint32_t* hist;
+  uint32_t* done;
+  int32_t* thr;
+  int k;
+};
+
+template <bool E4>
+__global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParams p,
+                                                                  const __grid_constant__ CUtensorMap kmap) {
+  using S = LongShape<E4>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  float* scale_st = reinterpret_cast<float*>(smem + S::kScaleOff);  // E4: [kStages][kLongTR]
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + S::kHistOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  __shared__ uint32_t last_s;
+  __shared__ uint32_t scan_sh[32];
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int64_t row = blockIdx.y;
+  const int64_t b = row / p.Tq;
+  const int64_t nv = visible(p.q_pos0 + row % p.Tq, p.m, p.N);
+  const int64_t e_begin = static_cast<int64_t>(blockIdx.x) * p.chunk;
+  if (e_begin >= nv) return;  // uniform for the CTA
+  const int64_t e_end = (e_begin + p.chunk) < nv ? (e_begin + p.chunk) : nv;
+  const int ntiles = static_cast<int>((e_end - e_begin + kLongTR - 1) / kLongTR);
+
+  for (int j = threadIdx.x; j < kHistBins; j += kLongThreads) hist_s[j] = 0;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < S::kStages; ++st) tc::bar_init(&bars[st], 1);
+    tc::bar_init_fence();
+  }
+
+  // B operand: column n = g (heads 0..3 valid), k = dim; the E4 variant uses
+  // the permuted dimension order and per-head power-of-two scaling described
+  // above score_kernel.
+  const bool qok = g < kHI;
+  const __nv_bfloat16* qrow = p.qI + (row * kHI + (qok ? g : 0)) * kDI;
+  uint32_t bq[4][2];
+  int qexp = 0;
+  if (E4) {
+    const __nv_bfloat16* qp = qrow + t * 16;
+    float qv[16];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      qv[i] = qok ? __bfloat162float(qp[i]) : 0.f;
+      amax = fmaxf(amax, fabsf(qv[i]));
     }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    int e = 14 - (static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127);
+    qexp = amax > 0.f ? (e < -60 ? -60 : (e > 60 ? 60 : e)) : 0;
+    const float sc = __uint_as_float(static_cast<uint32_t>(qexp + 127) << 23);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      bq[kk][0] = pack_f16x2(qv[4 * kk] * sc, qv[4 * kk + 1] * sc);
+      bq[kk][1] = pack_f16x2(qv[4 * kk + 2] * sc, qv[4 * kk + 3] * sc);
+    }
+  } else {
+    const __nv_bfloat16* qp = qrow + t * 2;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      bq[kk][0] = qok ? *reinterpret_cast<const uint32_t*>(qp + kk * 16) : 0u;
+      bq[kk][1] = qok ? *reinterpret_cast<const uint32_t*>(qp + kk * 16 + 8) : 0u;
+    }
+  }
+  // accumulator columns 2t, 2t+1 of this lane = heads 2t, 2t+1 (valid for t < 2)
+  float w0 = 0.f, w1 = 0.f;
+  {
+    const int e0 = __shfl_sync(0xffffffffu, qexp, 4 * (2 * t));
+    const int e1 = __shfl_sync(0xffffffffu, qexp, 4 * (2 * t + 1));
+    if (t < 2) {
+      w0 = p.wI[row * kHI + 2 * t] * __uint_as_float(static_cast<uint32_t>(127 - e0) << 23);
+      w1 = p.wI[row * kHI + 2 * t + 1] * __uint_as_float(static_cast<uint32_t>(127 - e1) << 23);
+    }
+  }
+
+  auto load_stage = [&](int tile) {
+    const int st = tile % S::kStages;
+    const int64_t base = e_begin + static_cast<int64_t>(tile) * kLongTR;
+    uint8_t* dst = smem + st * S::kStageBytes;
+    if (E4) {
+      const int rows = static_cast<int>((e_end - base) < kLongTR ? (e_end - base) : kLongTR);
+      if (threadIdx.x == 0) {
+        tc::bar_arrive_expect_tx(&bars[st], static_cast<uint32_t>(rows) * 64u);
+        tc::bulk_load(dst, p.kcodes + (b * p.N + base) * kDI, static_cast<uint32_t>(rows) * 64u, &bars[st]);
+      }
+      const int r = threadIdx.x;  // kLongThreads == kLongTR: one scale per thread
+      if (r < rows) {
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(scale_st + st * kLongTR + r)),
+                     "l"(p.kscale + b * p.N + base + r));
+      } else {
+        scale_st[st * kLongTR + r] = 0.f;
+      }
+      cp_async_commit();
+    } else if (threadIdx.x == 0) {
+      tc::bar_arrive_expect_tx(&bars[st], static_cast<uint32_t>(S::kStageBytes));
+      tc::tma_load_3d(dst, &kmap, 0, static_cast<int>(base), static_cast<int>(b), &bars[st]);
+    }
+  };
+
+  __syncthreads();  // barriers initialised, histogram cleared
+#pragma unroll
+  for (int i = 0; i < S::kStages - 1; ++i) {
+    if (i < ntiles) {
+      load_stage(i);
+    } else if (E4) {
+      cp_async_commit();
+    }
+  }
+  for (int tile = 0; tile < ntiles; ++tile) {
+    const int st = tile % S::kStages;
+    tc::bar_wait(&bars[st], static_cast<uint32_t>((tile / S::kStages) & 1));
+    if (E4) cp_async_wait<S::kStages - 2>();
+    __syncthreads();  // every warp is done with the stage refilled next; scales visible
+    {
+      const int nxt = tile + S::kStages - 1;
+      if (nxt < ntiles) {
+        load_stage(nxt);
+      } else if (E4) {
+        cp_async_commit();
+      }
+    }
+    float acc[2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      const int rbase = warp * 32 + mt * 16;
+      if (E4) {
+        const uint8_t* cs = smem + st * S::kStageBytes + (rbase + g) * 64 + t * 16;
+        const uint4 lo = *reinterpret_cast<const uint4*>(cs);
+        const uint4 hi = *reinterpret_cast<const uint4*>(cs + 8 * 64);
+        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t a0 = e4m3x2_to_f16x2(wl[kk] & 0xffffu), a2 = e4m3x2_to_f16x2(wl[kk] >> 16);
+          const uint32_t a1 = e4m3x2_to_f16x2(wh[kk] & 0xffffu), a3 = e4m3x2_to_f16x2(wh[kk] >> 16);
+          mma_f16(acc[mt], a0, a1, a2, a3, bq[kk][0], bq[kk][1]);
+        }
+      } else {
+        const uint8_t* stg = smem + st * S::kStageBytes;
+        const int r = rbase + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const int ch = kk * 2 + (lane >> 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(a0, a1, a2, a3, stg + r * 128 + ((ch ^ (r & 7)) << 4));
+          mma_bf16(acc[mt], a0, a1, a2, a3, bq[kk][0], bq[kk][1]);
+        }
+      }
+    }
+    // fold: lanes t = 0, 1 hold heads (0,1) and (2,3) of rows g, g+8 of both
+    // tiles; afterwards lane (g, t) owns row 16 (t >> 1) + 8 (t & 1) + g.
+    float f[2][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const float part = fmaxf(acc[mt][2 * hf], 0.f) * w0 + fmaxf(acc[mt][2 * hf + 1], 0.f) * w1;
+        f[mt][hf] = part + __shfl_xor_sync(0xffffffffu, part, 1);
+      }
+    }
+    const float y = (t & 1) ? f[1][1] : f[1][0];
+    const float z = __shfl_xor_sync(0xffffffffu, y, 2);
+    float score = t < 2 ? ((t & 1) ? f[0][1] : f[0][0]) : z;
+    const int rloc = warp * 32 + (t >> 1) * 16 + (t & 1) * 8 + g;
+    if (E4) score *= scale_st[st * kLongTR + rloc];  // scale > 0 factors out of relu
+    score += 0.0f;
+    const int64_t e = e_begin + static_cast<int64_t>(tile) * kLongTR + rloc;
+    if (e < e_end) {
+      p.scores[row * p.N + e] = score;
+      atomicAdd(&hist_s[f2key(score) >> 20], 1u);
+    }
+  }
+  if (E4) cp_async_wait<0>();
+
+  // flush the CTA histogram; the row's last CTA then derives its threshold
+  __syncthreads();
+  uint32_t* gh = p.hist + row * kHistBins;
+  for (int j = threadIdx.x; j < kHistBins; j += kLongThreads) {
+    const uint32_t c = hist_s[j];
+    if (c) atomicAdd(gh + j, c);
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t ctas = static_cast<uint32_t>((nv + p.chunk - 1) / p.chunk);
+    last_s = (atomicAdd(p.done + 2 * row, 1u) == ctas - 1) ? 1u : 0u;
+  }
+  __syncthreads();
+  if (last_s) {
     __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const uint32_t ctas = static_cast<uint32_t>((nv_max + p.chunk - 1) / p.chunk);
-      last_s = (atomicAdd(p.done + 2 * row, 1u) == ctas - 1) ? 1u : 0u;
-    }
-    __syncthreads();
-    if (last_s) {
-      __threadfence();
-      row_threshold<kScoreThreads>(gh, nv_max, p.k, p.thr + 2 * row, scan_sh);
-    }
+    row_threshold<kLongThreads>(gh, nv, p.k, p.thr + 2 * row, scan_sh);
   }
 }
 
@@ -391,12 +700,16 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   __shared__ uint32_t hist[256];
   __shared__ uint32_t dig[3];
   __shared__ uint32_t scan_sh[32];
-  __shared__ uint32_t n_cand, base_s, last_s, spill_base;
+  __shared__ uint32_t n_cand, base_s, last_s;
   const int64_t row = blockIdx.y;
   const int64_t nv = visible(q_pos0 + row % Tq, m, N);
   const int64_t e_begin = static_cast<int64_t>(blockIdx.x) * kSelChunk;
-  if (e_begin >= nv) return;
   int32_t* out = idx + row * k;
+  if (nv == 0) {  // no entry visible yet (the scoring kernel skipped the row): all padding
+    if (blockIdx.x == 0) write_prefix_ids(out, 0, k);
+    return;
+  }
+  if (e_begin >= nv) return;
   const int thr_bin = ws.thr[2 * row];
   if (thr_bin < 0) {  // every visible entry is selected
     if (blockIdx.x == 0) write_prefix_ids(out, nv, k);
@@ -455,7 +768,6 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   __syncthreads();
   if (!last_s) return;
   __threadfence();
-  (void)spill_base;
 
   // ---- load the row's candidates (when they fit) and bitmap (when it fits) together
   const int64_t words = (nv + 31) >> 5;
@@ -614,11 +926,32 @@ size_t csa_indexer_topk_workspace_size(int64_t B, int64_t Tq, int64_t N, int32_t
   return csa::workspace_bytes(B, Tq, N);
 }
 
-csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, int64_t B, int64_t Tq, int64_t N,
-                            int64_t q_pos0, int32_t m, int32_t k, int32_t* idx, void* workspace,
-                            size_t workspace_bytes, void* stream) {
-  using namespace csa;
+}  // extern "C"
+
+namespace csa {
+namespace {
+// The driver's tensor-map encoder, fetched through the runtime so that the
+// library carries no link-time dependency on the driver library.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const uint8_t* kcodes, const float* kscale,
+                        int64_t B, int64_t Tq, int64_t N, int64_t q_pos0, int32_t m, int32_t k, int32_t* idx,
+                        void* workspace, size_t workspace_bytes, void* stream) {
   clear_error();
+  const bool e4 = kcodes != nullptr;
   CSA_REQUIRE(B >= 0 && Tq >= 0 && N >= 0, "csa_indexer_topk: negative size");
   CSA_REQUIRE(N < (1LL << 31), "csa_indexer_topk: N must be < 2^31");
   CSA_REQUIRE(m >= 1, "csa_indexer_topk: m must be >= 1");
@@ -636,7 +969,13 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
   }
   CSA_REQUIRE_PTR(qI);
   CSA_REQUIRE_PTR(wI);
-  CSA_REQUIRE_PTR(kIc);
+  if (e4) {
+    CSA_REQUIRE_PTR(kcodes);
+    CSA_REQUIRE(kscale != nullptr && (reinterpret_cast<uintptr_t>(kscale) & 3u) == 0,
+                "csa_indexer_topk: key scales NULL or misaligned");
+  } else {
+    CSA_REQUIRE_PTR(kIc);
+  }
   const size_t need = csa::workspace_bytes(B, Tq, N);
   if (workspace == nullptr || workspace_bytes < need)
     return fail(CSA_ERR_WORKSPACE, "csa_indexer_topk: workspace of %zu bytes needed (got %zu)", need,
@@ -647,6 +986,8 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
   p.qI = static_cast<const __nv_bfloat16*>(qI);
   p.wI = wI;
   p.kI = static_cast<const __nv_bfloat16*>(kIc);
+  p.kcodes = kcodes;
+  p.kscale = kscale;
   p.Tq = Tq;
   p.N = N;
   p.q_pos0 = q_pos0;
@@ -666,7 +1007,12 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
     dim3 grid(static_cast<unsigned>((N + p.chunk - 1) / p.chunk), static_cast<unsigned>(B * groups));
     CSA_REQUIRE(B * groups < 65536, "csa_indexer_topk: too many query rows for one launch");
     prof_begin(s);
-    score_kernel<QR, false><<<grid, kScoreThreads, tile_smem, s>>>(p);
+    if (e4) {
+      const size_t sm = score_tile_bytes(true);
+      score_kernel<QR, true><<<grid, kScoreThreads, sm, s>>>(p);
+    } else {
+      score_kernel<QR, false><<<grid, kScoreThreads, tile_smem, s>>>(p);
+    }
     prof_end(s);
     if (csa_status st = check_launch("indexer score"); st != CSA_OK) return st;
     const size_t smem = static_cast<size_t>(N) * 4;
@@ -688,18 +1034,58 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
   w.W = L.W;
   if (cudaMemsetAsync(w.hist, 0, L.thr - L.hist, s) != cudaSuccess)
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: memset failed");
-  p.chunk = 4096;
-  p.scores = w.scores;
-  p.hist = w.hist;
-  p.done = w.done;
-  p.thr = w.thr;
-  p.k = k;
   CSA_REQUIRE(R < 65536, "csa_indexer_topk: too many query rows for the long-row path");
-  dim3 grid(static_cast<unsigned>((N + p.chunk - 1) / p.chunk), static_cast<unsigned>(R));
-  if (!ensure_smem(reinterpret_cast<const void*>(score_kernel<1, true>), tile_smem + kHistBins * 4))
+  LongScoreParams lp;
+  lp.qI = p.qI;
+  lp.wI = wI;
+  lp.kcodes = kcodes;
+  lp.kscale = kscale;
+  lp.Tq = Tq;
+  lp.N = N;
+  lp.q_pos0 = q_pos0;
+  lp.m = m;
+  lp.scores = w.scores;
+  lp.hist = w.hist;
+  lp.done = w.done;
+  lp.thr = w.thr;
+  lp.k = k;
+  CUtensorMap kmap;
+  memset(&kmap, 0, sizeof(kmap));
+  if (!e4) {
+    const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (encode == nullptr) return fail(CSA_ERR_CUDA, "csa_indexer_topk: cuTensorMapEncodeTiled unavailable");
+    CSA_REQUIRE(aligned16(kIc), "csa_indexer_topk: kIc must be 16-byte aligned");
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDI), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDI) * 2, static_cast<cuuint64_t>(N) * kDI * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kDI), static_cast<cuuint32_t>(kLongTR), 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUresult r = encode(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kIc), dims,
+                                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "csa_indexer_topk: tensor map encoding failed (%d)", int(r));
+  } else {
+    CSA_REQUIRE(aligned16(kcodes), "csa_indexer_topk: key codes must be 16-byte aligned");
+  }
+  const void* skern = e4 ? reinterpret_cast<const void*>(score_long_kernel<true>)
+                        : reinterpret_cast<const void*>(score_long_kernel<false>);
+  const size_t ssmem = e4 ? LongShape<true>::kSmem : LongShape<false>::kSmem;
+  if (!ensure_smem(skern, static_cast<int>(ssmem)))
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
+  // one wave: the row's chunks spread over every resident CTA slot
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, skern, kLongThreads, ssmem) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int64_t per_row = std::max<int64_t>(1, static_cast<int64_t>(num_sms()) * per_sm / R);
+  int64_t chunk = (N + per_row - 1) / per_row;
+  chunk = std::max<int64_t>(kLongMinChunk, (chunk + kLongTR - 1) / kLongTR * kLongTR);
+  lp.chunk = static_cast<int>(chunk);
+  dim3 grid(static_cast<unsigned>((N + chunk - 1) / chunk), static_cast<unsigned>(R));
   prof_begin(s);
-  score_kernel<1, true><<<grid, kScoreThreads, tile_smem + kHistBins * 4, s>>>(p);
+  if (e4)
+    score_long_kernel<true><<<grid, kLongThreads, ssmem, s>>>(lp, kmap);
+  else
+    score_long_kernel<false><<<grid, kLongThreads, ssmem, s>>>(lp, kmap);
   prof_end(s);
   if (csa_status st = check_launch("indexer score (long rows)"); st != CSA_OK) return st;
   dim3 sgrid(static_cast<unsigned>((N + kSelChunk - 1) / kSelChunk), static_cast<unsigned>(R));
@@ -708,6 +1094,24 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
   topk_select_kernel<<<sgrid, kSelThreads, kSelSmem, s>>>(w, N, Tq, q_pos0, m, k, idx);
   return check_launch("indexer select");
+}
+}  // namespace
+}  // namespace csa
+
+extern "C" {
+
+csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, int64_t B, int64_t Tq, int64_t N,
+                            int64_t q_pos0, int32_t m, int32_t k, int32_t* idx, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return csa::indexer_impl(qI, wI, kIc, nullptr, nullptr, B, Tq, N, q_pos0, m, k, idx, workspace, workspace_bytes,
+                           stream);
+}
+
+csa_status csa_indexer_topk_e4m3(const void* qI, const float* wI, const uint8_t* kI_codes, const float* kI_scale,
+                                 int64_t B, int64_t Tq, int64_t N, int64_t q_pos0, int32_t m, int32_t k, int32_t* idx,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  return csa::indexer_impl(qI, wI, nullptr, kI_codes, kI_scale, B, Tq, N, q_pos0, m, k, idx, workspace,
+                           workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -114,6 +114,15 @@ def split_fp8_cache(x: torch.Tensor):
     return codes, rope, scale.contiguous()
 
 
+def fp8_rows(x: torch.Tensor):
+    """Store rows [..., d] (fp32) as E4M3 codes with one scale per row (max |x| / 448, 1 if zero)."""
+    x = x.float()
+    amax = x.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax)).float()
+    qv = (x / scale[..., None]).clamp(-E4M3_MAX, E4M3_MAX)
+    return qv.to(torch.float8_e4m3fn).view(torch.uint8).contiguous(), scale.contiguous()
+
+
 @dataclasses.dataclass(frozen=True)
 class Prefill:
     """One prefill workload: B sequences of T tokens, all queries attend."""
@@ -147,6 +156,7 @@ class Decode:
     k: int
     win: int = 128
     m_hca: int = 128
+    indexer_fp8: bool = False  # indexer keys stored as E4M3 codes + per-entry scale
 
     @property
     def N(self):
@@ -163,6 +173,9 @@ WORKLOADS = {
     "csa_decode_l131072": Decode("csa_decode_l131072", "csa", B=64, L=131072, H=64, m=4, k=2048),
     "csa_prefill_t65536": Prefill("csa_prefill_t65536", "csa", B=1, T=65536, H=64, m=4, k=2048),
     "hybrid_decode_l1m": Decode("hybrid_decode_l1m", "hybrid", B=8, L=1 << 20, H=64, m=4, k=2048),
+    # the same workload with FP8 (E4M3 + per-entry scale) lightning-indexer keys
+    "hybrid_decode_l1m_fp8idx": Decode("hybrid_decode_l1m_fp8idx", "hybrid", B=8, L=1 << 20, H=64, m=4, k=2048,
+                                       indexer_fp8=True),
 }
 
 
@@ -219,9 +232,12 @@ def decode_inputs(w: Decode, seed: int = 0, batch: slice | None = None) -> dict:
         "qI": rows("qI", (1, H_I, D_I)),
         "wI": rows("wI", (1, H_I), kind="uniform"),
         "nope": nope, "rope": rope, "scale": scale,
-        "kIc": rows("kIc", (w.N, D_I)),
         "win_k": rows("win_k", (w.win, D_QK)),
     }
+    if w.indexer_fp8:
+        out["kI_codes"], out["kI_scale"] = fp8_rows(rows("kIc", (w.N, D_I), kind="normal_f32"))
+    else:
+        out["kIc"] = rows("kIc", (w.N, D_I))
     if w.kind == "hybrid":
         hc = rows("hca_cache", (w.N_hca, D_QK), kind="normal_f32")
         hn, hr, hs = split_fp8_cache(hc)

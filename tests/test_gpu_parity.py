@@ -100,6 +100,7 @@ def _indexer_case(g, B, Tq, N, tie_blocks=0, zero_q=False):
     (4, 8, 1000, 3000, 4, 100, 0, False),      # few rows: long-row path with short rows
     (2, 3, 3000, 11999, 4, 2048, 2, False),    # long-row path with ties
     (2, 2, 70, 100, 4, 40, 0, False),          # every row sees fewer than k entries
+    (1, 40, 300, 0, 4, 8, 0, False),           # long-row path; the first rows see no entry at all
     (1, 1, 40000, 4 * 40000 - 1, 4, 4096, 0, True),   # long rows, all ties, k = max
 ])
 def test_indexer_topk(B, Tq, N, q_pos0, m, k, ties, zero):
@@ -274,3 +275,27 @@ def test_no_device_timeouts_recorded():
     from long_context_sparse_10_b200 import _lib
     lib = _lib.load()
     assert lib.csa_check_device_error(torch.cuda.current_stream().cuda_stream) == 0, lib.csa_last_error()
+
+
+@pytest.mark.parametrize("B,Tq,N,q_pos0,m,k,head_scale", [
+    (3, 1, 50000, 4 * 50000 - 1, 4, 2048, None),     # long rows (decode)
+    (2, 1, 30000, 100000, 4, 512, None),             # long rows, partly visible
+    (1, 600, 150, 0, 4, 64, None),                   # prefill rows
+    # query heads far outside fp16's range in both directions (the kernel
+    # rescales each head by a power of two before its fp16 MMA)
+    (2, 1, 20000, 4 * 20000 - 1, 4, 256, (2.0 ** -40, 2.0 ** 30, 1.0, 2.0 ** -10)),
+    (1, 40, 300, 0, 4, 32, (2.0 ** 25, 2.0 ** -35, 0.0, 1.0)),
+])
+def test_indexer_topk_e4m3_keys(B, Tq, N, q_pos0, m, k, head_scale):
+    g = np.random.default_rng(N + k + 17)
+    qI = _bf16(g, (B, Tq, 4, 64))
+    if head_scale is not None:
+        qI = (qI.float() * torch.tensor(head_scale).view(1, 1, 4, 1)).to(torch.bfloat16)
+    wI = torch.from_numpy(g.random((B, Tq, 4)).astype(np.float32))
+    codes, scale = synth.fp8_rows(torch.from_numpy(g.standard_normal((B, N, 64)).astype(np.float32)))
+    idx = csa.csa_indexer_topk_e4m3(qI.to(DEV), wI.to(DEV), codes.to(DEV), scale.to(DEV), m, k, q_pos0=q_pos0)
+    torch.cuda.synchronize()
+    kI = R.e4m3_decode(codes.numpy()) * scale.double().numpy()[..., None]
+    s = R.indexer_scores(f64(qI), f64(wI), kI, q_pos0 + np.arange(Tq), m)
+    same = check_topk(idx.cpu().numpy(), s, R.topk_set(s, k), k, "indexer e4m3")
+    assert same.mean() > 0.97
