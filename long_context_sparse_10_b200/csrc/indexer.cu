@@ -414,6 +414,7 @@ struct LongScoreParams {
   int64_t Tq, N, q_pos0;
   int m;
   int chunk;  // entries per CTA, a multiple of kLongTR
+  int64_t pitch;  // row pitch of scores
   float* scores;
   uint32_t* hist;
   uint32_t* done;
@@ -587,7 +588,7 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
     score += 0.0f;
     const int64_t e = e_begin + static_cast<int64_t>(tile) * kLongTR + rloc;
     if (e < e_end) {
-      p.scores[row * p.N + e] = score;
+      p.scores[row * p.pitch + e] = score;
       atomicAdd(&hist_s[f2key(score) >> 20], 1u);
     }
   }
@@ -673,9 +674,14 @@ constexpr int kSelThreads = 512;
 constexpr int kSelChunk = 8192;         // entries per select CTA
 constexpr int kCandSmem = 4096;         // threshold-bin candidates kept in shared memory
 constexpr int kBitmapSmemWords = 8192;  // rows up to 262144 entries emit from a shared-memory bitmap
+// The shared-memory bitmap leaves 4 words free after every 16, so that lanes
+// reading their 16 consecutive words as four 16-byte vectors (the emission
+// pass) do not collide on banks.
+__host__ __device__ constexpr int bm_pad(int64_t wi) { return static_cast<int>(wi + 4 * (wi >> 4)); }
+constexpr int kBitmapSmemPadded = kBitmapSmemWords + kBitmapSmemWords / 4;
 
 struct LongWs {
-  float* scores;        // [R, N]
+  float* scores;        // [R, pitch] (pitch = N rounded up to 4: 16-byte aligned rows)
   uint32_t* hist;       // [R, kHistBins]    (zeroed per call)
   uint32_t* cand_cnt;   // [R]               (zeroed per call)
   uint32_t* done;       // [R, 2]: scoring / select CTAs finished (zeroed per call)
@@ -683,6 +689,7 @@ struct LongWs {
   uint2* cand;          // [R, N]: (key, index) of the threshold bin's entries
   uint32_t* bitmap;     // [R, W]
   int64_t W;
+  int64_t pitch;
 };
 
 // Per CTA: a bitmap word for every 32 entries (entries above the threshold
@@ -720,35 +727,60 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) n_cand = 0;
   __syncthreads();
-  const float* srow = ws.scores + row * N;
-  constexpr int kIters = kSelChunk / kSelThreads;
-  float sv[kIters];
+  // warp w scans entries [e_begin + 512 w, e_begin + 512 (w + 1)), four per
+  // lane per step (16-byte loads; rows are 16-byte aligned and padded)
+  const float* srow = ws.scores + row * ws.pitch;
+  constexpr int kSelWarps = kSelThreads / 32;
+  constexpr int kPerWarp = kSelChunk / kSelWarps;
+  constexpr int kSteps = kPerWarp / 128;
+  const int warp = threadIdx.x >> 5;
+  float4 sv[kSteps];
 #pragma unroll
-  for (int it = 0; it < kIters; ++it) {  // all loads first, then the bookkeeping
-    const int64_t i = e_begin + it * kSelThreads + threadIdx.x;
-    sv[it] = i < e_end ? __ldcg(srow + i) : 0.f;
+  for (int it = 0; it < kSteps; ++it) {  // all loads first, then the bookkeeping
+    const int64_t i = e_begin + warp * kPerWarp + it * 128 + 4 * lane;
+    sv[it] = i < e_end ? __ldcg(reinterpret_cast<const float4*>(srow + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
-  for (int it = 0; it < kIters; ++it) {
-    const int64_t base = e_begin + it * kSelThreads + (threadIdx.x & ~31);
-    const int64_t i = base + lane;
-    const bool ok = i < e_end;
-    const uint32_t key = ok ? f2key(sv[it]) : 0u;
-    const uint32_t bin = key >> 20;
-    const uint32_t word = __ballot_sync(0xffffffffu, ok && bin > tb);
-    if (lane == 0 && base < e_end) ws.bitmap[row * ws.W + (base >> 5)] = word;
-    const bool cnd = ok && bin == tb;
-    const uint32_t cm = __ballot_sync(0xffffffffu, cnd);
-    if (cm) {
+  for (int it = 0; it < kSteps; ++it) {
+    const int64_t base = e_begin + warp * kPerWarp + it * 128;  // a multiple of 32
+    if (base >= e_end) break;                                     // uniform for the warp
+    const int64_t i0 = base + 4 * lane;
+    const float v[4] = {sv[it].x, sv[it].y, sv[it].z, sv[it].w};
+    uint32_t above = 0, cand_bits = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool ok = i0 + u < e_end;
+      const uint32_t bin = f2key(v[u]) >> 20;
+      above |= (ok && bin > tb) ? (1u << u) : 0u;
+      cand_bits |= (ok && bin == tb) ? (1u << u) : 0u;
+    }
+    // bitmap word of entries [32 j, 32 j + 32): lanes 8j .. 8j+7, four bits each
+    uint32_t word = above << (4 * (lane & 7));
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+    word |= __shfl_xor_sync(0xffffffffu, word, 4);
+    if ((lane & 7) == 0 && i0 < e_end) ws.bitmap[row * ws.W + (i0 >> 5)] = word;
+    if (__any_sync(0xffffffffu, cand_bits != 0u)) {
+      const uint32_t nc = __popc(cand_bits);
+      uint32_t incl = nc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
       uint32_t pos = 0;
-      if (lane == 0) pos = atomicAdd(&n_cand, static_cast<uint32_t>(__popc(cm)));
-      pos = __shfl_sync(0xffffffffu, pos, 0);
-      const uint32_t my = pos + __popc(cm & ((1u << lane) - 1u));
-      if (cnd) {
-        if (my < static_cast<uint32_t>(kCandSmem)) {
-          cand_s[my] = make_uint2(key, static_cast<uint32_t>(i));
-        } else {  // rare (many equal scores): straight to the row's list
-          ws.cand[row * N + atomicAdd(ws.cand_cnt + row, 1u)] = make_uint2(key, static_cast<uint32_t>(i));
+      if (lane == 31) pos = atomicAdd(&n_cand, incl);
+      pos = __shfl_sync(0xffffffffu, pos, 31) + incl - nc;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (cand_bits & (1u << u)) {
+          const uint2 kv = make_uint2(f2key(v[u]), static_cast<uint32_t>(i0 + u));
+          if (pos < static_cast<uint32_t>(kCandSmem)) {
+            cand_s[pos] = kv;
+          } else {  // rare (many equal scores): straight to the row's list
+            ws.cand[row * N + atomicAdd(ws.cand_cnt + row, 1u)] = kv;
+          }
+          ++pos;
         }
       }
     }
@@ -769,35 +801,59 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   if (!last_s) return;
   __threadfence();
 
-  // ---- load the row's candidates (when they fit) and bitmap (when it fits) together
+  // ---- load the row's candidates (when they fit) and bitmap (when it fits)
+  // together.  Warp w owns the bitmap words [w * per_warp, (w + 1) * per_warp)
+  // and counts their bits as it loads them (wcnt), so the final emission
+  // needs no separate counting pass.
   const int64_t words = (nv + 31) >> 5;
   const uint32_t cnt = __ldcg(ws.cand_cnt + row);
   const uint2* cand = ws.cand + row * N;
   uint32_t* gbm = ws.bitmap + row * ws.W;
   const bool bm_in_smem = words <= kBitmapSmemWords;
   const bool cand_in_smem = cnt <= static_cast<uint32_t>(kCandSmem);
-  if (bm_in_smem) {
-    for (int64_t w0 = 4 * threadIdx.x; w0 < words; w0 += 4 * kSelThreads) {
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(gbm + w0));
-      bm_s[w0] = v.x;
-      if (w0 + 1 < words) bm_s[w0 + 1] = v.y;
-      if (w0 + 2 < words) bm_s[w0 + 2] = v.z;
-      if (w0 + 3 < words) bm_s[w0 + 3] = v.w;
+  __shared__ uint32_t wcnt[kSelWarps];
+  // a shared-memory bitmap gives every warp 512 words (16 per lane)
+  const int64_t per_warp =
+      bm_in_smem ? kBitmapSmemWords / kSelWarps : (words + 32 * kSelWarps - 1) / (32 * kSelWarps) * 32;
+  const int64_t wb = warp * per_warp;
+  const int64_t we = (wb + per_warp) < words ? (wb + per_warp) : words;
+  // candidate loads first (in flight together with the bitmap's)
+  constexpr int kCandPerThread = kCandSmem / kSelThreads;
+  uint2 cv[kCandPerThread];
+  if (cand_in_smem) {
+#pragma unroll
+    for (int u = 0; u < kCandPerThread; ++u) {
+      const uint32_t c = u * kSelThreads + threadIdx.x;
+      cv[u] = c < cnt ? __ldcg(cand + c) : make_uint2(0, 0);
     }
   }
+  {
+    // 16 words per lane in flight (a shared-memory bitmap has at most 512 words per warp)
+    uint32_t bits = 0;
+    for (int64_t w0 = wb; w0 < we; w0 += 16 * 32) {
+      uint32_t v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int64_t wi = w0 + u * 32 + lane;
+        v[u] = wi < we ? __ldcg(gbm + wi) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int64_t wi = w0 + u * 32 + lane;
+        if (wi == words - 1 && (nv & 31)) v[u] &= (1u << (nv & 31)) - 1u;
+        if (bm_in_smem && wi < we) bm_s[bm_pad(wi)] = v[u];
+        bits += __popc(v[u]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bits += __shfl_xor_sync(0xffffffffu, bits, o);
+    if (lane == 0) wcnt[warp] = bits;
+  }
   if (cand_in_smem) {
-    for (uint32_t c0 = 0; c0 < cnt; c0 += 4 * kSelThreads) {
-      uint2 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t c = c0 + u * kSelThreads + threadIdx.x;
-        v[u] = c < cnt ? __ldcg(cand + c) : make_uint2(0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t c = c0 + u * kSelThreads + threadIdx.x;
-        if (c < cnt) cand_s[c] = v[u];
-      }
+    for (int u = 0; u < kCandPerThread; ++u) {
+      const uint32_t c = u * kSelThreads + threadIdx.x;
+      if (c < cnt) cand_s[c] = cv[u];
     }
     cand = cand_s;
   }
@@ -827,44 +883,87 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
     in_bucket = dig[2];
     __syncthreads();
   }
-  uint32_t* bm = bm_in_smem ? bm_s : gbm;
   for (uint32_t c = threadIdx.x; c < cnt; c += kSelThreads) {
     const uint2 kv = cand_in_smem ? cand[c] : __ldcg(cand + c);
     const uint64_t x = (static_cast<uint64_t>(kv.x) << 32) | (0xffffffffu - kv.y);
-    if ((x & mask) >= prefix) atomicOr(bm + (kv.y >> 5), 1u << (kv.y & 31));
+    if ((x & mask) >= prefix) {  // a threshold-bin entry: its bit is not set yet
+      atomicOr(bm_in_smem ? bm_s + bm_pad(kv.y >> 5) : gbm + (kv.y >> 5), 1u << (kv.y & 31));
+      atomicAdd(&wcnt[(kv.y >> 5) / per_warp], 1u);
+    }
   }
   if (!bm_in_smem) __threadfence();
   __syncthreads();
 
-  // ---- ascending list from the bitmap: 16 consecutive words per thread per round
-  uint32_t before = 0;
-  for (int64_t base = 0; base < words; base += 16 * kSelThreads) {
-    const int64_t w0 = base + 16 * threadIdx.x;
+  // ---- ascending list from the bitmap: each warp emits its own word range
+  // at the offset of the bits before it; within the warp each lane takes
+  // per_warp / 32 consecutive words (one count pass, one scan, one emit pass).
+  uint32_t pos = 0;
+  for (int w = 0; w < warp; ++w) pos += wcnt[w];
+  const int64_t per_lane = per_warp / 32;
+  const int64_t lb = wb + lane * per_lane;
+  const int64_t le = (lb + per_lane) < we ? (lb + per_lane) : we;
+  if (bm_in_smem) {  // 16 words per lane, in registers
+    static_assert(kBitmapSmemWords / kSelWarps == 16 * 32, "16 bitmap words per lane");
     uint32_t wv[16];
+    const uint4* src = reinterpret_cast<const uint4*>(bm_s + bm_pad(lb));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = src[j];
+      wv[4 * j] = v.x;
+      wv[4 * j + 1] = v.y;
+      wv[4 * j + 2] = v.z;
+      wv[4 * j + 3] = v.w;
+    }
+    uint32_t c = 0;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const int64_t wi = w0 + j;
-      uint32_t word = 0;
-      if (wi < words) word = bm_in_smem ? bm_s[wi] : __ldcg(gbm + wi);
-      if (wi == words - 1 && (nv & 31)) word &= (1u << (nv & 31)) - 1u;
-      wv[j] = word;
+      const int64_t wi = lb + j;
+      if (wi >= words) wv[j] = 0u;
+      if (wi == words - 1 && (nv & 31)) wv[j] &= (1u << (nv & 31)) - 1u;
+      c += __popc(wv[j]);
     }
-    uint32_t cntw = 0;
+    uint32_t incl = c;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) cntw += __popc(wv[j]);
-    uint32_t total;
-    uint32_t pos = before + block_excl_scan(cntw, &total, scan_sh);
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    uint32_t p = pos + incl - c;
+    const int32_t e0 = static_cast<int32_t>(lb << 5);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       uint32_t word = wv[j];
       while (word) {
         const int bit = __ffs(word) - 1;
         word &= word - 1;
-        if (pos < static_cast<uint32_t>(k)) out[pos] = static_cast<int32_t>(((w0 + j) << 5) + bit);
-        ++pos;
+        if (p < static_cast<uint32_t>(k)) out[p] = e0 + 32 * j + bit;
+        ++p;
       }
     }
-    before += total;
+    return;
+  }
+  uint32_t c = 0;
+  for (int64_t wi = lb; wi < le; ++wi) {
+    uint32_t word = __ldcg(gbm + wi);
+    if (wi == words - 1 && (nv & 31)) word &= (1u << (nv & 31)) - 1u;
+    c += __popc(word);
+  }
+  uint32_t incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  uint32_t p = pos + incl - c;
+  for (int64_t wi = lb; wi < le && p < static_cast<uint32_t>(k); ++wi) {
+    uint32_t word = __ldcg(gbm + wi);
+    if (wi == words - 1 && (nv & 31)) word &= (1u << (nv & 31)) - 1u;
+    while (word) {
+      const int bit = __ffs(word) - 1;
+      word &= word - 1;
+      if (p < static_cast<uint32_t>(k)) out[p] = static_cast<int32_t>((wi << 5) + bit);
+      ++p;
+    }
   }
 }
 
@@ -877,14 +976,15 @@ bool use_row_path(int64_t R, int64_t N) { return N <= kRowPathMaxN && R > 256; }
 
 struct LongLayout {
   size_t scores, hist, cnt, done, thr, cand, bitmap, total;
-  int64_t W;
+  int64_t W, pitch;
 };
 
 LongLayout long_layout(int64_t R, int64_t N) {
   LongLayout L;
   L.W = ((N + 31) / 32 + 15) / 16 * 16;  // 16-word multiple: vector reads stay in the row
+  L.pitch = (N + 3) / 4 * 4;
   size_t off = 0;
-  L.scores = off; off = align_up(off + static_cast<size_t>(R) * N * 4);
+  L.scores = off; off = align_up(off + static_cast<size_t>(R) * L.pitch * 4);
   L.hist = off;   off += static_cast<size_t>(R) * kHistBins * 4;     // hist, cnt and done: zeroed together
   L.cnt = off;    off += static_cast<size_t>(R) * 4;
   L.done = off;   off = align_up(off + static_cast<size_t>(R) * 8);
@@ -1032,6 +1132,7 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   w.cand = reinterpret_cast<uint2*>(ws + L.cand);
   w.bitmap = reinterpret_cast<uint32_t*>(ws + L.bitmap);
   w.W = L.W;
+  w.pitch = L.pitch;
   if (cudaMemsetAsync(w.hist, 0, L.thr - L.hist, s) != cudaSuccess)
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: memset failed");
   CSA_REQUIRE(R < 65536, "csa_indexer_topk: too many query rows for the long-row path");
@@ -1045,6 +1146,7 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   lp.q_pos0 = q_pos0;
   lp.m = m;
   lp.scores = w.scores;
+  lp.pitch = w.pitch;
   lp.hist = w.hist;
   lp.done = w.done;
   lp.thr = w.thr;
@@ -1089,7 +1191,7 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   prof_end(s);
   if (csa_status st = check_launch("indexer score (long rows)"); st != CSA_OK) return st;
   dim3 sgrid(static_cast<unsigned>((N + kSelChunk - 1) / kSelChunk), static_cast<unsigned>(R));
-  constexpr int kSelSmem = kCandSmem * 8 + kBitmapSmemWords * 4;
+  constexpr int kSelSmem = kCandSmem * 8 + kBitmapSmemPadded * 4;
   if (!ensure_smem(reinterpret_cast<const void*>(topk_select_kernel), kSelSmem))
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
   topk_select_kernel<<<sgrid, kSelThreads, kSelSmem, s>>>(w, N, Tq, q_pos0, m, k, idx);
