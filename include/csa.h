@@ -215,7 +215,15 @@ CSA_API csa_status csa_indexer_topk_noalloc(const void* qI, const float* wI, con
                                             int64_t B, int64_t Tq, int64_t N, int64_t q_pos0,
                                             int32_t m, int32_t k, int32_t* idx, void* stream);
 
-/* Workspace bytes csa_sparse_mqa needs for these sizes. */
+/*
+ * Workspace bytes csa_sparse_mqa needs for these sizes on the current device
+ * (it depends on the device's SM count).  Nonzero when H = 64 and there are
+ * too few query rows (B * Tq) to fill the device: each row's keys are then
+ * split over several CTAs whose partial softmax states (per head: 128
+ * unnormalised output channels, running max, sum) are merged from this
+ * buffer.  Pass at least this many bytes, 16-byte aligned; otherwise the call
+ * returns CSA_ERR_WORKSPACE.  The buffer holds no state between calls.
+ */
 CSA_API size_t csa_sparse_mqa_workspace_size(int64_t B, int64_t Tq, int32_t H, int32_t k, int32_t win_len);
 
 /*
@@ -240,7 +248,8 @@ CSA_API csa_status csa_sparse_mqa(const void* q, int64_t B, int64_t Tq, int32_t 
                           const csa_window* win, float scale, void* out, float* lse,
                           void* workspace, size_t workspace_bytes, void* stream);
 
-/* Workspace bytes hca_dense_mqa needs for these sizes. */
+/* Workspace bytes hca_dense_mqa needs for these sizes on the current device
+ * (same rule as csa_sparse_mqa_workspace_size with k replaced by N). */
 CSA_API size_t hca_dense_mqa_workspace_size(int64_t B, int64_t Tq, int32_t H, int64_t N, int32_t win_len);
 
 /*

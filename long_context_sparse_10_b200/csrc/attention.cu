@@ -65,10 +65,17 @@ struct AttnParams {
   int64_t wpos0, wrows;
   int wlen;
   float scale_log2;
-  int cl, tps;  // CTAs per row (cluster size), tiles per CTA
+  int cl, tps;  // CTAs per row (the splits of its slots), tiles per CTA
   __nv_bfloat16* out;
   float* lse;
+  // Split records in global memory (tcgen05 path with several CTAs per row):
+  // [R][cl][H][kRec] floats = unnormalised O (128), running max m (log2
+  // units), sum l; merged by attn_merge_kernel.  Null: the CTAs of a row form
+  // a thread-block cluster and merge through distributed shared memory.
+  float* part;
 };
+
+constexpr int kRec = kDV + 4;  // 128 channels, m, l, pad: 16-byte aligned records
 
 struct SmemLayout {
   size_t ks, vs, raw, sc, stype, srow, idx, total;
@@ -457,7 +464,8 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
 // ---------------------------------------------------------------------------
 constexpr int kTcKeys = 128;
 
-constexpr int kTcThreads = 256;  // warps 0-3: softmax + MMA issue; warps 4-7: loads
+constexpr int kTcThreads = 256;     // query-blocked prefill kernel: warps 0-3 softmax + MMA, 4-7 loads
+constexpr int kTcDecThreads = 256;  // attn_tc_kernel: warps 0-3 softmax + MMA issue, 4-7 loads
 
 struct TcLayout {
   size_t q, k, v, p, raw, sc, stype, srow, vmask, bars, idx, total;
@@ -491,7 +499,7 @@ __device__ __forceinline__ void bar_arrive(uint64_t* bar) {
 }
 
 template <bool FP8, bool SHV>
-__global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
+__global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const TcLayout L = tc_layout(FP8, SHV, p.tps);
@@ -536,7 +544,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     tc::bar_init_fence();
   }
   if (warp == 0) tc::tmem_alloc(tslot, 256);
-  for (int piece = tid; piece < 64 * 24; piece += kTcThreads) {  // Q, swizzled K-major
+  for (int piece = tid; piece < 64 * 24; piece += kTcDecThreads) {  // Q, swizzled K-major
     const int hh = piece / 24, ch = piece % 24;
     cp_async16(Qs + (ch >> 3) * 8192 + tc::sw128(hh, ch & 7), p.q + (row * 64 + hh) * kDQK + ch * 8);
   }
@@ -825,10 +833,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
   tc::fence_after_sync();
 
   // ---- output (consumer threads): channels half*64..+63 of head h, with (m_ref, l) ----
+  if (p.part != nullptr) {  // split record in global memory, merged by attn_merge_kernel
+    if (warp < 4) {
+      const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      float* rec = p.part + ((row * p.cl + split) * 64 + h) * kRec;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float ov[32];
+        if (ntiles > 0) {
+          tc::tmem_ld32(tO + lane_base + 32 * c, ov);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+        }
+        const int d0 = half * 64 + 32 * c;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(rec + d0 + i) = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
+      }
+      if (half == 0) *reinterpret_cast<float2*>(rec + kDV) = make_float2(m_ref, l_row);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, 256);
+    return;
+  }
   cg::cluster_group cluster = cg::this_cluster();
   if (p.cl > 1) cluster.sync();  // peers may now write merge records over our Q/K tiles
   float* rbuf = reinterpret_cast<float*>(smem);
-  constexpr int kRec = kDV + 4;  // 128 channels, m, l, pad: 16-byte aligned records
   if (warp < 4) {
     const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
     float* dst = nullptr;
@@ -874,8 +906,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
   if (warp == 0) tc::tmem_dealloc(tmem, 256);
   if (p.cl == 1) return;
   cluster.sync();
-  const int sub = tid >> 5;  // 8 warps, one head at a time each
-  for (int j = sub; split + j * p.cl < p.H; j += 8) {
+  const int sub = tid >> 5;  // warps 0-7, one head at a time each
+  for (int j = sub; sub < 8 && split + j * p.cl < p.H; j += 8) {
     const int hh = split + j * p.cl;
     const float* rec = rbuf + static_cast<int64_t>(j) * p.cl * kRec;
     float M = -INFINITY;
@@ -1169,8 +1201,64 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_block_kernel(AttnParams p)
 }
 
 // ---------------------------------------------------------------------------
+// Merge of the split records of each (row, head): one warp per head, four
+// channels per lane.  out = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c with
+// M = max_c m_c; lse = ln 2 (M + log2 sum_c 2^(m_c - M) l_c).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict__ part, int nsplit, int H,
+                                                         __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rh = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);  // row * H + head
+  const int64_t row = rh / H;
+  const int hh = static_cast<int>(rh % H);
+  const float* rec0 = part + (row * nsplit * H + hh) * kRec;
+  const int64_t cstride = static_cast<int64_t>(H) * kRec;
+  float M = -INFINITY;
+  for (int c = 0; c < nsplit; ++c) M = fmaxf(M, __ldg(rec0 + c * cstride + kDV));
+  const float bse = M == -INFINITY ? 0.f : M;
+  float Lsum = 0.f;
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = 0; c < nsplit; ++c) {
+    const float* r = rec0 + c * cstride;
+    const float2 ml = __ldg(reinterpret_cast<const float2*>(r + kDV));
+    const float w = exp2f(ml.x - bse);
+    Lsum += w * ml.y;
+    const float4 u = __ldg(reinterpret_cast<const float4*>(r) + lane);
+    a.x += w * u.x;
+    a.y += w * u.y;
+    a.z += w * u.z;
+    a.w += w * u.w;
+  }
+  const float iv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+  *reinterpret_cast<uint2*>(out + rh * kDV + lane * 4) =
+      make_uint2(pack_bf16x2(a.x * iv, a.y * iv), pack_bf16x2(a.z * iv, a.w * iv));
+  if (lane == 0 && lse) lse[rh] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
+// Splits of a row's slots for the tcgen05 kernel (one CTA per SM): rows that
+// cannot fill the device by themselves are split so that all rows' CTAs run
+// in one wave; the splits then merge through global-memory records.
+struct TcSplit {
+  int nsplit, tps;
+};
+TcSplit tc_split(int64_t R, int64_t max_slots) {
+  const int64_t tiles = max_slots > 0 ? (max_slots + kTcKeys - 1) / kTcKeys : 1;
+  int64_t ns = R >= num_sms() ? 1 : num_sms() / R;
+  if (ns < 1) ns = 1;
+  if (ns > tiles) ns = tiles;
+  const int64_t tps = (tiles + ns - 1) / ns;
+  ns = (tiles + tps - 1) / tps;
+  return TcSplit{static_cast<int>(ns), static_cast<int>(tps)};
+}
+size_t tc_part_bytes(int64_t R, int H, int64_t max_slots) {
+  if (H != 64 || R <= 0) return 0;
+  const TcSplit sp = tc_split(R, max_slots);
+  return sp.nsplit > 1 ? static_cast<size_t>(R) * sp.nsplit * H * kRec * sizeof(float) : 0;
+}
+
 struct Plan {
   int cl, tps;
 };
@@ -1277,7 +1365,7 @@ csa_status check_cache(const char* name, const csa_kv_cache* c) {
 
 csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H, int64_t q_pos0,
                const csa_kv_cache* cache, int32_t stride, const int32_t* idx, int32_t k, const csa_window* win,
-               float scale, void* out, float* lse, void* stream) {
+               float scale, void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
   clear_error();
   CSA_REQUIRE(B >= 0 && Tq >= 0, "%s: negative size", name);
   CSA_REQUIRE(H == 16 || H == 64, "%s: H must be 16 or 64 (got %d)", name, H);
@@ -1318,11 +1406,56 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   const bool use_tc = H == 64 && !(fp8 && !shv);
   const int tile_keys = use_tc ? kTcKeys : kKeys;
   Plan pl = plan(R, max_slots, tile_keys);
+  float* part = nullptr;
+  bool tc_cluster = false;  // tcgen05 path: splits merged in a cluster (else through global records)
+  if (use_tc && !ensure_smem(reinterpret_cast<const void*>(pick_tc(fp8, shv)),
+                             static_cast<int>(tc_layout(fp8, shv, 0).total)))
+    return fail(CSA_ERR_CUDA, "%s: cannot raise the shared memory limit", name);
+  if (use_tc) {
+    const TcSplit sp = tc_split(R, max_slots);
+    if (sp.nsplit > 1 && pl.cl > 1) {
+      // A cluster merge (distributed shared memory, no second kernel) wins when
+      // a co-resident cluster size leaves at most two more tiles per CTA than
+      // the global split does (the merge kernel and its launch cost about
+      // that much).
+      static std::mutex mu;
+      bool nonportable = true;
+      {
+        std::lock_guard<std::mutex> lock(mu);
+        const KernelFn f = pick_tc(fp8, shv);
+        if (cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+          cudaGetLastError();
+          nonportable = false;
+        }
+      }
+      const int want = nonportable ? pl.cl : (pl.cl > 8 ? 8 : pl.cl);
+      const int cl = choose_cluster(pick_tc(fp8, shv), want, R, tc_layout(fp8, shv, 0).total, kTcDecThreads);
+      const int64_t tiles = max_slots > 0 ? (max_slots + kTcKeys - 1) / kTcKeys : 1;
+      const int64_t tps = (tiles + cl - 1) / cl;
+      if (cl > 1 && max_active_clusters(pick_tc(fp8, shv), cl, tc_layout(fp8, shv, 0).total, kTcDecThreads) >= R &&
+          tps <= sp.tps + 2) {
+        tc_cluster = true;
+        pl.tps = static_cast<int>(tps);
+        pl.cl = static_cast<int>((tiles + tps - 1) / tps);
+      }
+    }
+    if (!tc_cluster) {
+      pl.cl = sp.nsplit;
+      pl.tps = sp.tps;
+    }
+    if (!tc_cluster && sp.nsplit > 1) {
+      const size_t need = tc_part_bytes(R, H, max_slots);
+      if (workspace == nullptr || workspace_bytes < need)
+        return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed (got %zu)", name, need, workspace_bytes);
+      CSA_REQUIRE(aligned16(workspace), "%s: workspace is not 16-byte aligned", name);
+      part = static_cast<float*>(workspace);
+    }
+  }
   KernelFn fn = use_tc ? pick_tc(fp8, shv) : pick(H, fp8, shv);
   size_t smem = smem_bytes(use_tc, fp8, shv, pl.tps);
   if (!ensure_smem(reinterpret_cast<const void*>(fn), static_cast<int>(smem)))
     return fail(CSA_ERR_CUDA, "%s: cannot raise the shared memory limit to %zu", name, smem);
-  if (pl.cl > 1) {
+  if (pl.cl > 1 && !use_tc) {
     static std::mutex mu;
     {
       std::lock_guard<std::mutex> lock(mu);
@@ -1350,6 +1483,7 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
     if (!ensure_smem(reinterpret_cast<const void*>(fn), static_cast<int>(smem)))
       return fail(CSA_ERR_CUDA, "%s: cannot raise the shared memory limit to %zu", name, smem);
     pl.cl = 1;
+    part = nullptr;
   }
 
   AttnParams p;
@@ -1376,24 +1510,30 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   p.tps = pl.tps;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
+  p.part = part;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(use_blk ? B * ((Tq + (128 / H) - 1) / (128 / H)) : R * pl.cl));
-  cfg.blockDim = dim3(use_tc || use_blk ? kTcThreads : kThreads);
+  cfg.blockDim = dim3(use_blk ? kTcThreads : (use_tc ? kTcDecThreads : kThreads));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = pl.cl;
+  attr.val.clusterDim.x = (use_tc && !tc_cluster) || use_blk ? 1 : pl.cl;
   attr.val.clusterDim.y = 1;
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = attr.val.clusterDim.x > 1 ? 1 : 0;
   prof_begin(cfg.stream);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, fn, p);
   prof_end(cfg.stream);
   if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
-  return check_launch(name);
+  if (csa_status st = check_launch(name); st != CSA_OK) return st;
+  if (part != nullptr) {
+    attn_merge_kernel<<<static_cast<unsigned>(R * H / 8), 256, 0, cfg.stream>>>(part, pl.cl, H, p.out, lse);
+    return check_launch(name);
+  }
+  return CSA_OK;
 }
 
 }  // namespace
@@ -1420,29 +1560,29 @@ csa_status csa_check_device_error(void* stream) {
 }
 
 size_t csa_sparse_mqa_workspace_size(int64_t B, int64_t Tq, int32_t H, int32_t k, int32_t win_len) {
-  (void)B, (void)Tq, (void)H, (void)k, (void)win_len;
-  return 0;  // partial states are merged in distributed shared memory
+  if (B <= 0 || Tq <= 0 || k < 0 || win_len < 0) return 0;
+  return csa::tc_part_bytes(B * Tq, H, static_cast<int64_t>(k) + win_len);
 }
 
 size_t hca_dense_mqa_workspace_size(int64_t B, int64_t Tq, int32_t H, int64_t N, int32_t win_len) {
-  (void)B, (void)Tq, (void)H, (void)N, (void)win_len;
-  return 0;
+  if (B <= 0 || Tq <= 0 || N < 0 || win_len < 0) return 0;
+  return csa::tc_part_bytes(B * Tq, H, N + win_len);
 }
 
 csa_status csa_sparse_mqa(const void* q, int64_t B, int64_t Tq, int32_t H, int64_t q_pos0, const csa_kv_cache* cache,
                           int32_t m, const int32_t* idx, int32_t k, const csa_window* win, float scale, void* out,
                           float* lse, void* workspace, size_t workspace_bytes, void* stream) {
-  (void)workspace, (void)workspace_bytes;
   if (idx == nullptr && B * Tq > 0)
     return csa::fail(CSA_ERR_INVALID_ARG, "csa_sparse_mqa: idx is NULL");
-  return csa::run("csa_sparse_mqa", q, B, Tq, H, q_pos0, cache, m, idx, k, win, scale, out, lse, stream);
+  return csa::run("csa_sparse_mqa", q, B, Tq, H, q_pos0, cache, m, idx, k, win, scale, out, lse, workspace,
+                  workspace_bytes, stream);
 }
 
 csa_status hca_dense_mqa(const void* q, int64_t B, int64_t Tq, int32_t H, int64_t q_pos0, const csa_kv_cache* cache,
                          int32_t m_prime, const csa_window* win, float scale, void* out, float* lse, void* workspace,
                          size_t workspace_bytes, void* stream) {
-  (void)workspace, (void)workspace_bytes;
-  return csa::run("hca_dense_mqa", q, B, Tq, H, q_pos0, cache, m_prime, nullptr, 0, win, scale, out, lse, stream);
+  return csa::run("hca_dense_mqa", q, B, Tq, H, q_pos0, cache, m_prime, nullptr, 0, win, scale, out, lse, workspace,
+                  workspace_bytes, stream);
 }
 
 }  // extern "C"

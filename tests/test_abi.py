@@ -101,3 +101,19 @@ def test_workspace_sizes_are_monotone(lib):
     b = lib.csa_indexer_topk_workspace_size(8, 1, 131072, 2048)
     assert a > b > 0
     assert lib.csa_indexer_topk_workspace_size(0, 1, 10, 4) == 0
+
+
+def test_attention_workspace_rule(lib):
+    """H = 64 rows too few to fill the device split their keys over several
+    CTAs and need merge records; H = 16, many rows, or one tile need none."""
+    rec = (128 + 4) * 4
+    sms = 148  # the library's SM count when no device is visible
+    # decode: 8 rows x (2048 selected + 128 window) slots = 17 tiles of 128 keys
+    assert lib.csa_sparse_mqa_workspace_size(8, 1, 64, 2048, 128) == 8 * 17 * 64 * rec
+    # 8 rows x (8192 entries + 128 window) = 65 tiles over at most 148 // 8 = 18 splits
+    tps = -(-65 // (sms // 8))
+    assert lib.hca_dense_mqa_workspace_size(8, 1, 64, 8192, 128) == 8 * (-(-65 // tps)) * 64 * rec
+    assert lib.csa_sparse_mqa_workspace_size(8, 1, 16, 2048, 128) == 0
+    assert lib.csa_sparse_mqa_workspace_size(1, sms, 64, 2048, 128) == 0
+    assert lib.csa_sparse_mqa_workspace_size(4, 1, 64, 100, 0) == 0
+    assert lib.csa_sparse_mqa_workspace_size(0, 1, 64, 100, 0) == 0
