@@ -116,6 +116,15 @@ CSA_API const char* csa_last_error(void);
 CSA_API csa_status csa_check_device_error(void* stream);
 
 /*
+ * csa_launch_count -- number of kernels this library has enqueued in this
+ * process so far (library infrastructure, not part of the method).  Every
+ * successful kernel launch counts once, including one recorded into a CUDA
+ * graph capture (a replay of the graph does not count again).  Callers use
+ * the difference around a call to see how many kernels it launched.
+ */
+CSA_API uint64_t csa_launch_count(void);
+
+/*
  * csa_profile_next_call -- timing hook (library infrastructure, not part of
  * the method).  `start_event` and `stop_event` are cudaEvent_t handles created
  * by the caller.  The next entry point that enqueues work on this thread

@@ -26,7 +26,7 @@ from . import _lib
 
 __all__ = ["CsaError", "KVCache", "Window", "csa_compress", "hca_compress", "csa_indexer_topk", "csa_indexer_topk_e4m3",
            "csa_indexer_topk_workspace_size", "csa_sparse_mqa", "csa_sparse_mqa_workspace_size", "hca_dense_mqa",
-           "hca_dense_mqa_workspace_size", "version"]
+           "hca_dense_mqa_workspace_size", "launch_count", "version"]
 
 
 class CsaError(RuntimeError):
@@ -60,6 +60,11 @@ def _stream(stream):
 
 def version() -> str:
     return _lib.load().csa_version().decode()
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued in this process (graph captures count once)."""
+    return int(_lib.load().csa_launch_count())
 
 
 @dataclasses.dataclass

@@ -18,6 +18,7 @@ SIGNATURES = {
     "csa_version": (ctypes.c_char_p, []),
     "csa_status_string": (ctypes.c_char_p, [c_i32]),
     "csa_last_error": (ctypes.c_char_p, []),
+    "csa_launch_count": (ctypes.c_uint64, []),
     "csa_profile_next_call": (c_i32, [c_vp, c_vp]),
     "csa_check_device_error": (c_i32, [c_vp]),
     "csa_compress": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),

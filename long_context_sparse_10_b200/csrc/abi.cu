@@ -1,4 +1,5 @@
 // Library-wide entry points: version, status names, per-thread error text.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
@@ -27,11 +28,16 @@ csa_status fail(csa_status s, const char* fmt, ...) {
 
 void clear_error() { g_msg[0] = '\0'; }
 
+static std::atomic<uint64_t> g_launches{0};
+
 csa_status check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   return CSA_OK;
 }
+
+uint64_t launch_count() { return g_launches.load(std::memory_order_relaxed); }
 
 int num_sms() {
   int dev = 0;
@@ -79,6 +85,8 @@ void prof_end(cudaStream_t s) {
 }  // namespace csa
 
 extern "C" {
+
+uint64_t csa_launch_count(void) { return csa::launch_count(); }
 
 csa_status csa_profile_next_call(void* start_event, void* stop_event) {
   if ((start_event == nullptr) != (stop_event == nullptr))

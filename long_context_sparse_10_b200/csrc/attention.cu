@@ -1213,21 +1213,35 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict
   const int hh = static_cast<int>(rh % H);
   const float* rec0 = part + (row * nsplit * H + hh) * kRec;
   const int64_t cstride = static_cast<int64_t>(H) * kRec;
+  // the splits' maxima, one split per lane, then a warp max
   float M = -INFINITY;
-  for (int c = 0; c < nsplit; ++c) M = fmaxf(M, __ldg(rec0 + c * cstride + kDV));
+  for (int c = lane; c < nsplit; c += 32) M = fmaxf(M, __ldg(rec0 + c * cstride + kDV));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   const float bse = M == -INFINITY ? 0.f : M;
+  // weighted sums, 16 split records in flight per lane
+  constexpr int kBatch = 16;
   float Lsum = 0.f;
   float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c = 0; c < nsplit; ++c) {
-    const float* r = rec0 + c * cstride;
-    const float2 ml = __ldg(reinterpret_cast<const float2*>(r + kDV));
-    const float w = exp2f(ml.x - bse);
-    Lsum += w * ml.y;
-    const float4 u = __ldg(reinterpret_cast<const float4*>(r) + lane);
-    a.x += w * u.x;
-    a.y += w * u.y;
-    a.z += w * u.z;
-    a.w += w * u.w;
+  for (int c0 = 0; c0 < nsplit; c0 += kBatch) {
+    float2 ml[kBatch];
+    float4 u[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const bool ok = c0 + j < nsplit;
+      const float* r = rec0 + (ok ? c0 + j : 0) * cstride;
+      ml[j] = ok ? __ldg(reinterpret_cast<const float2*>(r + kDV)) : make_float2(-INFINITY, 0.f);
+      u[j] = ok ? __ldg(reinterpret_cast<const float4*>(r) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const float w = exp2f(ml[j].x - bse);
+      Lsum += w * ml[j].y;
+      a.x += w * u[j].x;
+      a.y += w * u[j].y;
+      a.z += w * u[j].z;
+      a.w += w * u[j].w;
+    }
   }
   const float iv = Lsum > 0.f ? 1.f / Lsum : 0.f;
   *reinterpret_cast<uint2*>(out + rh * kDV + lane * 4) =

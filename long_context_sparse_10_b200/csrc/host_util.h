@@ -13,7 +13,10 @@ csa_status fail(csa_status s, const char* fmt, ...);
 // Clears the calling thread's message.
 void clear_error();
 // Maps a pending launch error (cudaGetLastError) to CSA_ERR_CUDA.
+// Checks the launch just enqueued and counts it (csa_launch_count).  Called
+// exactly once after every kernel launch of the library.
 csa_status check_launch(const char* what);
+uint64_t launch_count();
 // Streaming multiprocessors of the current device (cached per device).
 int num_sms();
 // Raises a kernel's dynamic shared memory limit to `bytes` on the current

@@ -395,14 +395,21 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
 constexpr int kLongThreads = 128;
 constexpr int kLongTR = 128;  // entries per stage (32 per warp)
 constexpr int kLongMinChunk = 1024;
+constexpr int kLongMaxChunk = 65536 - kLongTR;  // per-CTA bin counts fit 16 bits
 
+#ifndef CSA_LONG_STAGES_BF16
+#define CSA_LONG_STAGES_BF16 3
+#endif
+#ifndef CSA_LONG_STAGES_E4
+#define CSA_LONG_STAGES_E4 4
+#endif
 template <bool E4>
 struct LongShape {
-  static constexpr int kStages = E4 ? 4 : 3;
+  static constexpr int kStages = E4 ? CSA_LONG_STAGES_E4 : CSA_LONG_STAGES_BF16;
   static constexpr int kStageBytes = kLongTR * (E4 ? 64 : 128);
   static constexpr size_t kScaleOff = static_cast<size_t>(kStages) * kStageBytes;
   static constexpr size_t kHistOff = kScaleOff + (E4 ? static_cast<size_t>(kStages) * kLongTR * 4 : 0);
-  static constexpr size_t kBarOff = kHistOff + kHistBins * 4;
+  static constexpr size_t kBarOff = kHistOff + kHistBins * 2;  // two 16-bit bins per word
   static constexpr size_t kSmem = kBarOff + kStages * 8 + 1024;  // + alignment slack for the 1024-byte swizzle atoms
 };
 
@@ -444,7 +451,7 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
   const int64_t e_end = (e_begin + p.chunk) < nv ? (e_begin + p.chunk) : nv;
   const int ntiles = static_cast<int>((e_end - e_begin + kLongTR - 1) / kLongTR);
 
-  for (int j = threadIdx.x; j < kHistBins; j += kLongThreads) hist_s[j] = 0;
+  for (int j = threadIdx.x; j < kHistBins / 2; j += kLongThreads) hist_s[j] = 0;
   if (threadIdx.x == 0) {
     for (int st = 0; st < S::kStages; ++st) tc::bar_init(&bars[st], 1);
     tc::bar_init_fence();
@@ -553,8 +560,9 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
         const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t a0 = e4m3x2_to_f16x2(wl[kk] & 0xffffu), a2 = e4m3x2_to_f16x2(wl[kk] >> 16);
-          const uint32_t a1 = e4m3x2_to_f16x2(wh[kk] & 0xffffu), a3 = e4m3x2_to_f16x2(wh[kk] >> 16);
+          uint32_t a0, a1, a2, a3;
+          e4m3x4_to_f16x2x2(wl[kk], a0, a2);
+          e4m3x4_to_f16x2x2(wh[kk], a1, a3);
           mma_f16(acc[mt], a0, a1, a2, a3, bq[kk][0], bq[kk][1]);
         }
       } else {
@@ -589,7 +597,8 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
     const int64_t e = e_begin + static_cast<int64_t>(tile) * kLongTR + rloc;
     if (e < e_end) {
       p.scores[row * p.pitch + e] = score;
-      atomicAdd(&hist_s[f2key(score) >> 20], 1u);
+      const uint32_t bin = f2key(score) >> 20;
+      atomicAdd(&hist_s[bin >> 1], 1u << ((bin & 1u) * 16));
     }
   }
   if (E4) cp_async_wait<0>();
@@ -597,9 +606,10 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
   // flush the CTA histogram; the row's last CTA then derives its threshold
   __syncthreads();
   uint32_t* gh = p.hist + row * kHistBins;
-  for (int j = threadIdx.x; j < kHistBins; j += kLongThreads) {
+  for (int j = threadIdx.x; j < kHistBins / 2; j += kLongThreads) {
     const uint32_t c = hist_s[j];
-    if (c) atomicAdd(gh + j, c);
+    if (c & 0xffffu) atomicAdd(gh + 2 * j, c & 0xffffu);
+    if (c >> 16) atomicAdd(gh + 2 * j + 1, c >> 16);
   }
   __threadfence();
   __syncthreads();
@@ -1181,6 +1191,7 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   const int64_t per_row = std::max<int64_t>(1, static_cast<int64_t>(num_sms()) * per_sm / R);
   int64_t chunk = (N + per_row - 1) / per_row;
   chunk = std::max<int64_t>(kLongMinChunk, (chunk + kLongTR - 1) / kLongTR * kLongTR);
+  chunk = std::min<int64_t>(chunk, kLongMaxChunk);
   lp.chunk = static_cast<int>(chunk);
   dim3 grid(static_cast<unsigned>((N + chunk - 1) / chunk), static_cast<unsigned>(R));
   prof_begin(s);
