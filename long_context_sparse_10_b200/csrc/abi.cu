@@ -37,6 +37,14 @@ csa_status check_launch(const char* what) {
   return CSA_OK;
 }
 
+csa_status check_launch(const char* what, cudaError_t e) {
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(CSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  }
+  return check_launch(what);
+}
+
 uint64_t launch_count() { return g_launches.load(std::memory_order_relaxed); }
 
 int num_sms() {

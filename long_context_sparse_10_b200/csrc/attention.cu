@@ -115,6 +115,8 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
 
 template <int KG, bool FP8, bool SHV>
 __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int HG = 4 / KG;       // head groups of 16
   constexpr int KPW = kKeys / KG;  // keys per warp per tile
   constexpr int NTS = KPW / 8;     // S n-tiles per warp
@@ -500,6 +502,7 @@ __device__ __forceinline__ void bar_arrive(uint64_t* bar) {
 
 template <bool FP8, bool SHV>
 __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p) {
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const TcLayout L = tc_layout(FP8, SHV, p.tps);
@@ -828,6 +831,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
     }
   }
   cp_async_wait<0>();
+  pdl_trigger();  // the epilogue is all that is left
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -960,6 +964,8 @@ __host__ __device__ inline BlkLayout blk_layout() {
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1) attn_block_kernel(AttnParams p) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const BlkLayout L = blk_layout();
@@ -1207,6 +1213,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_block_kernel(AttnParams p)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict__ part, int nsplit, int H,
                                                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  pdl_wait();  // (no early trigger: the next kernel is usually a long one)
   const int lane = threadIdx.x & 31;
   const int64_t rh = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);  // row * H + head
   const int64_t row = rh / H;
@@ -1526,27 +1533,17 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   p.lse = lse;
   p.part = part;
 
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(use_blk ? B * ((Tq + (128 / H) - 1) / (128 / H)) : R * pl.cl));
-  cfg.blockDim = dim3(use_blk ? kTcThreads : (use_tc ? kTcDecThreads : kThreads));
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = (use_tc && !tc_cluster) || use_blk ? 1 : pl.cl;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = attr.val.clusterDim.x > 1 ? 1 : 0;
-  prof_begin(cfg.stream);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, fn, p);
-  prof_end(cfg.stream);
-  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
-  if (csa_status st = check_launch(name); st != CSA_OK) return st;
-  if (part != nullptr) {
-    attn_merge_kernel<<<static_cast<unsigned>(R * H / 8), 256, 0, cfg.stream>>>(part, pl.cl, H, p.out, lse);
-    return check_launch(name);
-  }
+  const dim3 grid(static_cast<unsigned>(use_blk ? B * ((Tq + (128 / H) - 1) / (128 / H)) : R * pl.cl));
+  const dim3 block(use_blk ? kTcThreads : (use_tc ? kTcDecThreads : kThreads));
+  const int cluster = (use_tc && !tc_cluster) || use_blk ? 1 : pl.cl;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  prof_begin(s);
+  const cudaError_t e = launch_pdl(fn, grid, block, smem, s, cluster, p);
+  prof_end(s);
+  if (csa_status st = check_launch(name, e); st != CSA_OK) return st;
+  if (part != nullptr)
+    return check_launch(name, launch_pdl(attn_merge_kernel, dim3(static_cast<unsigned>(R * H / 8)), dim3(256), 0, s,
+                                         1, static_cast<const float*>(part), pl.cl, H, p.out, lse));
   return CSA_OK;
 }
 

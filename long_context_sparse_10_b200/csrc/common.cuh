@@ -105,6 +105,17 @@ __device__ __forceinline__ void mma_f16(float* c, uint32_t a0, uint32_t a1, uint
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Programmatic dependent launch.  Every kernel of the library starts with
+// pdl_wait() (returns once the previous kernel on the stream has completed and
+// its memory is visible; a no-op when the launch carries no programmatic
+// dependency), and each CTA calls pdl_trigger() once the rest of its work is
+// short (at its start for small or multi-wave kernels, before the epilogue
+// for the long single-wave ones), letting the next kernel's CTAs be scheduled
+// and wait while this one finishes.  No global memory is touched before
+// pdl_wait(), so the overlap never changes a result.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // Order-preserving map float -> uint32 (larger float -> larger key).  -0 is
 // folded onto +0 by the callers (s + 0.0f) so equal scores get equal keys.
 __device__ __forceinline__ uint32_t f2key(float f) {

@@ -121,6 +121,8 @@ __device__ __forceinline__ void store_entry(const CompressParams& p, int64_t b, 
 
 // One warp per entry (short windows).
 __global__ void __launch_bounds__(256) compress_short_kernel(CompressParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t e = static_cast<int64_t>(blockIdx.x) * 8 + warp;
   if (e >= p.B * p.N) return;
@@ -150,6 +152,8 @@ __global__ void __launch_bounds__(256) compress_short_kernel(CompressParams p) {
 // One CTA per entry (long windows): 8 warps take interleaved rows, then warp 0
 // merges the 8 partial softmax states.
 __global__ void __launch_bounds__(256) compress_long_kernel(CompressParams p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float st[8][3][8][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t e = blockIdx.x;
@@ -234,12 +238,11 @@ csa_status compress_impl(const char* name, const void* x, int64_t B, int64_t T, 
   const int64_t entries = B * p.N;
   CSA_REQUIRE(entries < (1LL << 31), "%s: too many entries", name);
   prof_begin(s);
-  if (cwin <= 32)
-    compress_short_kernel<<<static_cast<unsigned>((entries + 7) / 8), 256, 0, s>>>(p);
-  else
-    compress_long_kernel<<<static_cast<unsigned>(entries), 256, 0, s>>>(p);
+  const cudaError_t e =
+      cwin <= 32 ? launch_pdl(compress_short_kernel, dim3(static_cast<unsigned>((entries + 7) / 8)), dim3(256), 0, s, 1, p)
+                 : launch_pdl(compress_long_kernel, dim3(static_cast<unsigned>(entries)), dim3(256), 0, s, 1, p);
   prof_end(s);
-  return check_launch(name);
+  return check_launch(name, e);
 }
 
 }  // namespace

@@ -13,9 +13,38 @@ csa_status fail(csa_status s, const char* fmt, ...);
 // Clears the calling thread's message.
 void clear_error();
 // Maps a pending launch error (cudaGetLastError) to CSA_ERR_CUDA.
+// Launches `kernel` with programmatic stream serialization allowed (the kernel
+// calls pdl_wait() before touching global memory), plus an optional cluster
+// dimension (> 1).
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // Checks the launch just enqueued and counts it (csa_launch_count).  Called
 // exactly once after every kernel launch of the library.
 csa_status check_launch(const char* what);
+// The same for a launch whose own return code is `e` (cudaLaunchKernelEx).
+csa_status check_launch(const char* what, cudaError_t e);
 uint64_t launch_count();
 // Streaming multiprocessors of the current device (cached per device).
 int num_sms();

@@ -201,6 +201,8 @@ __host__ __device__ constexpr size_t score_tile_bytes(bool e4) {
 // relu(2^e x) 2^-e w = relu(x) w.
 template <int QR, bool E4>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int NCOL = QR * 4;
   constexpr int NT = (NCOL + 7) / 8;
   constexpr int TR = E4 ? 2 * kTileRows : kTileRows;  // entries per stage
@@ -432,6 +434,7 @@ struct LongScoreParams {
 template <bool E4>
 __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParams p,
                                                                   const __grid_constant__ CUtensorMap kmap) {
+  pdl_wait();
   using S = LongShape<E4>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -602,6 +605,7 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
     }
   }
   if (E4) cp_async_wait<0>();
+  pdl_trigger();  // the next kernel may be scheduled while the histograms merge
 
   // flush the CTA histogram; the row's last CTA then derives its threshold
   __syncthreads();
@@ -629,6 +633,8 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) topk_rows_kernel(const float* __restrict__ scores, int64_t N, int64_t Tq,
                                                          int64_t q_pos0, int m, int k, int32_t* __restrict__ idx) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint32_t keys[];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t dig[3];
@@ -711,6 +717,7 @@ struct LongWs {
 // bitmap in shared memory.
 __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, int64_t N, int64_t Tq, int64_t q_pos0,
                                                                      int m, int k, int32_t* __restrict__ idx) {
+  pdl_wait();
   extern __shared__ __align__(16) uint8_t sel_smem[];  // candidates, then the final bitmap
   uint2* cand_s = reinterpret_cast<uint2*>(sel_smem);
   uint32_t* bm_s = reinterpret_cast<uint32_t*>(sel_smem + kCandSmem * sizeof(uint2));
@@ -800,6 +807,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   if (threadIdx.x == 0 && nc) base_s = atomicAdd(ws.cand_cnt + row, nc);
   __syncthreads();
   for (uint32_t c = threadIdx.x; c < nc; c += kSelThreads) ws.cand[row * N + base_s + c] = cand_s[c];
+  pdl_trigger();  // only the rows' last CTAs still have work
   // last CTA of this row?
   __threadfence();
   __syncthreads();
@@ -1117,19 +1125,16 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
     dim3 grid(static_cast<unsigned>((N + p.chunk - 1) / p.chunk), static_cast<unsigned>(B * groups));
     CSA_REQUIRE(B * groups < 65536, "csa_indexer_topk: too many query rows for one launch");
     prof_begin(s);
-    if (e4) {
-      const size_t sm = score_tile_bytes(true);
-      score_kernel<QR, true><<<grid, kScoreThreads, sm, s>>>(p);
-    } else {
-      score_kernel<QR, false><<<grid, kScoreThreads, tile_smem, s>>>(p);
-    }
+    const cudaError_t e = e4 ? launch_pdl(score_kernel<QR, true>, grid, dim3(kScoreThreads), score_tile_bytes(true), s, 1, p)
+                             : launch_pdl(score_kernel<QR, false>, grid, dim3(kScoreThreads), tile_smem, s, 1, p);
     prof_end(s);
-    if (csa_status st = check_launch("indexer score"); st != CSA_OK) return st;
+    if (csa_status st = check_launch("indexer score", e); st != CSA_OK) return st;
     const size_t smem = static_cast<size_t>(N) * 4;
     if (!ensure_smem(reinterpret_cast<const void*>(topk_rows_kernel), kRowPathMaxN * 4))
       return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
-    topk_rows_kernel<<<static_cast<unsigned>(R), 1024, smem, s>>>(p.scores, N, Tq, q_pos0, m, k, idx);
-    return check_launch("indexer top-k (rows)");
+    return check_launch("indexer top-k (rows)",
+                        launch_pdl(topk_rows_kernel, dim3(static_cast<unsigned>(R)), dim3(1024), smem, s, 1,
+                                   static_cast<const float*>(p.scores), N, Tq, q_pos0, m, k, idx));
   }
 
   const LongLayout L = long_layout(R, N);
@@ -1195,18 +1200,16 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   lp.chunk = static_cast<int>(chunk);
   dim3 grid(static_cast<unsigned>((N + chunk - 1) / chunk), static_cast<unsigned>(R));
   prof_begin(s);
-  if (e4)
-    score_long_kernel<true><<<grid, kLongThreads, ssmem, s>>>(lp, kmap);
-  else
-    score_long_kernel<false><<<grid, kLongThreads, ssmem, s>>>(lp, kmap);
+  const cudaError_t e = e4 ? launch_pdl(score_long_kernel<true>, grid, dim3(kLongThreads), ssmem, s, 1, lp, kmap)
+                           : launch_pdl(score_long_kernel<false>, grid, dim3(kLongThreads), ssmem, s, 1, lp, kmap);
   prof_end(s);
-  if (csa_status st = check_launch("indexer score (long rows)"); st != CSA_OK) return st;
+  if (csa_status st = check_launch("indexer score (long rows)", e); st != CSA_OK) return st;
   dim3 sgrid(static_cast<unsigned>((N + kSelChunk - 1) / kSelChunk), static_cast<unsigned>(R));
   constexpr int kSelSmem = kCandSmem * 8 + kBitmapSmemPadded * 4;
   if (!ensure_smem(reinterpret_cast<const void*>(topk_select_kernel), kSelSmem))
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
-  topk_select_kernel<<<sgrid, kSelThreads, kSelSmem, s>>>(w, N, Tq, q_pos0, m, k, idx);
-  return check_launch("indexer select");
+  return check_launch("indexer select",
+                      launch_pdl(topk_select_kernel, sgrid, dim3(kSelThreads), kSelSmem, s, 1, w, N, Tq, q_pos0, m, k, idx));
 }
 }  // namespace
 }  // namespace csa
