@@ -445,7 +445,8 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
 
 
 // ---------------------------------------------------------------------------
-// H = 64: tcgen05 path.  One elected thread issues the MMAs; accumulators live
+// H = 64: tcgen05 path.  Warps 0-3 run the online softmax, warps 4-7 gather
+// and widen key tiles, one thread of warp 8 issues every MMA; accumulators live
 // in tensor memory (TMEM).  A tile is 128 keys.  An M = 64 accumulator fills
 // 16 of the 32 lanes of each TMEM lane quarter (row m -> lane (m % 16) +
 // 32 (m / 16)); a second one at lane offset 16 fills the other half.  So
@@ -461,33 +462,38 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
 // first two K blocks when key and value are shared.  O is rescaled in TMEM
 // only when a row's running max grows by more than 2^8 (probabilities stay <=
 // 256 in between).  FP8 entries are dequantised (code x scale, rounded to
-// bf16) while widening into the K tile.  Every mbarrier wait is bounded; a
-// timeout sets the device error word instead of hanging.
+// bf16) from registers into the K tile.  When key and value are shared the K
+// tile has three stages, so the gather runs up to two tiles ahead and the
+// next tile's S = Q K^T is computed while the softmax works on this one
+// (issue order S(0), S(1), then PV(t), S(t+2)); with a separate V tile there
+// is room for two.  Every mbarrier wait is bounded; a timeout sets the device
+// error word instead of hanging.
 // ---------------------------------------------------------------------------
 constexpr int kTcKeys = 128;
 
 constexpr int kTcThreads = 256;     // query-blocked prefill kernel: warps 0-3 softmax + MMA, 4-7 loads
-constexpr int kTcDecThreads = 256;  // attn_tc_kernel: warps 0-3 softmax + MMA issue, 4-7 loads
+constexpr int kTcDecThreads = 288;  // attn_tc_kernel: warps 0-3 softmax, 4-7 loads, 8 MMA issue
 
 struct TcLayout {
-  size_t q, k, v, p, raw, sc, stype, srow, vmask, bars, idx, total;
+  size_t q, k, v, p, stype, srow, vmask, bars, total;
 };
+
+// K-tile stages: three when the V tile is the K tile, two otherwise.
+__host__ __device__ constexpr int tc_stages(bool shv) { return shv ? 3 : 2; }
 
 __host__ __device__ inline TcLayout tc_layout(bool fp8, bool shv, int tps) {
   TcLayout L;
+  const int ns = tc_stages(shv);
   size_t off = 0;
   L.q = off; off += 3 * 8192;                    // Q: 64 heads x 192 dims
-  L.k = off; off += 2 * 3 * 16384;               // K: 2 stages x 128 keys x 192 dims
-  L.v = off; if (!shv) off += 2 * 2 * 16384;     // V: 2 stages x 128 keys x 128 dims
+  L.k = off; off += ns * 3 * 16384;              // K: stages x 128 keys x 192 dims
+  L.v = off; if (!shv) off += ns * 2 * 16384;    // V: stages x 128 keys x 128 dims
   L.p = off; off += 2 * 2 * 8192;                // P: 2 buffers x 64 heads x 128 keys
-  L.raw = off; if (fp8) off += 2 * 16384;        // raw E4M3 nope codes: 2 stages x 128 x 128
-  L.sc = off; off += 2 * kTcKeys * sizeof(float);
-  L.stype = off; off += 2 * kTcKeys * sizeof(int);
-  L.srow = off; off += 2 * kTcKeys * sizeof(int64_t);
-  L.vmask = off; off += 2 * 4 * sizeof(uint32_t);
+  L.stype = off; off += ns * kTcKeys * sizeof(int);
+  L.srow = off; off += ns * kTcKeys * sizeof(int64_t);
+  L.vmask = off; off += ns * 4 * sizeof(uint32_t);
   L.bars = off; off += 128;
-  L.idx = off;  // (the producer reads the selection straight from global memory)
-  (void)tps;
+  (void)fp8, (void)tps;
   const size_t reduce = 80 * (kDV + 4) * sizeof(float);  // cluster merge records (reuse Q/K)
   L.total = (off > reduce ? off : reduce) + 1024;          // + alignment slack
   return L;
@@ -510,15 +516,15 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   uint8_t* Kst = smem + L.k;
   uint8_t* Vst = smem + L.v;
   uint8_t* Pst = smem + L.p;
-  uint8_t* rawst = smem + L.raw;
-  auto sc = reinterpret_cast<float(*)[kTcKeys]>(smem + L.sc);
+  constexpr int NS = tc_stages(SHV);
   auto stype = reinterpret_cast<int(*)[kTcKeys]>(smem + L.stype);
   auto srow = reinterpret_cast<int64_t(*)[kTcKeys]>(smem + L.srow);
   auto vmask = reinterpret_cast<uint32_t(*)[4]>(smem + L.vmask);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [2] stage loaded
-  uint64_t* empty = full + 2;                                     // [2] PV of the stage's tile done
-  uint64_t* sdone = full + 4;                                     // [2] S of the tile done
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(full + 8);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NS] K stage loaded
+  uint64_t* empty = full + NS;                                    // [NS] PV of the stage's tile done
+  uint64_t* sdone = empty + NS;                                   // [2] S of the tile done (TMEM buffer)
+  uint64_t* pready = sdone + 2;                                   // [2] P of the tile written (smem buffer)
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(pready + 2);
   constexpr int kKB = 16384;  // one 64-dim block of a 128-key tile
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -543,7 +549,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   const int ntiles = s1 > s0 ? static_cast<int>((s1 - s0 + kTcKeys - 1) / kTcKeys) : 0;
 
   if (tid == 0) {
-    for (int i = 0; i < 6; ++i) tc::bar_init(&full[i], 1);
+    for (int i = 0; i < 2 * NS + 4; ++i) tc::bar_init(&full[i], 1);
     tc::bar_init_fence();
   }
   if (warp == 0) tc::tmem_alloc(tslot, 256);
@@ -567,12 +573,60 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const uint32_t tO = tmem + 128;
 
-  if (warp >= 4) {
+  constexpr uint32_t kIdescS = tc::idesc_bf16(64, 64, false);
+  constexpr uint32_t kIdescO = tc::idesc_bf16(64, 64, true);
+  if (warp == 8) {
+    // ===================== MMA issue (one thread) =====================
+    // S(0), S(1), then per tile t: PV(t) once P(t) is written, S(t+2) into the
+    // TMEM buffer P(t)'s softmax has drained.  A commit tracks every earlier
+    // MMA of this thread, so S(t+2) done implies PV(t) done, which frees P
+    // buffer t % 2 for tile t+2.
+    auto issue_s = [&](int tile) {
+      const int kst = tile % NS;
+      const uint32_t tS = tmem + 64 * (tile & 1);
+      const uint32_t qa = smem_u32(Qs), ka = smem_u32(Kst + kst * 3 * kKB);
+      tc::fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < 12; ++kk) {
+        const uint64_t adesc = tc::desc_sw128(qa + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+        const uint32_t kb = ka + (kk >> 2) * kKB + (kk & 3) * 32;
+        tc::mma_bf16_ss(tS, adesc, tc::desc_sw128(kb, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+        tc::mma_bf16_ss(tS + kHalfLane, adesc, tc::desc_sw128(kb + 64 * 128, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(&sdone[tile & 1]);
+    };
+    if (lane == 0 && ntiles > 0) {
+      for (int t0 = 0; t0 < 2 && t0 < ntiles; ++t0) {
+        if (healthy) healthy = tc::bar_wait(&full[t0 % NS], (t0 / NS) & 1);
+        issue_s(t0);
+      }
+      for (int tile = 0; tile < ntiles; ++tile) {
+        const int kst = tile % NS, pb = tile & 1;
+        if (healthy) healthy = tc::bar_wait(&pready[pb], (tile >> 1) & 1);
+        tc::fence_after_sync();
+        const uint32_t pa = smem_u32(Pst + pb * 2 * 8192);
+        const uint32_t va = SHV ? smem_u32(Kst + kst * 3 * kKB) : smem_u32(Vst + kst * 2 * kKB);
+#pragma unroll
+        for (int ks = 0; ks < kTcKeys / 16; ++ks) {
+          const uint64_t adesc = tc::desc_sw128(pa + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+          const uint32_t vb = va + ks * 2048;
+          const uint32_t acc = (tile > 0 || ks > 0) ? 1u : 0u;
+          tc::mma_bf16_ss(tO, adesc, tc::desc_sw128(vb, kKB, 1024), kIdescO, acc);
+          tc::mma_bf16_ss(tO + kHalfLane, adesc, tc::desc_sw128(vb + kKB, kKB, 1024), kIdescO, acc);
+        }
+        tc::mma_commit(&empty[kst]);
+        if (tile + 2 < ntiles) {
+          if (healthy) healthy = tc::bar_wait(&full[(tile + 2) % NS], ((tile + 2) / NS) & 1);
+          issue_s(tile + 2);
+        }
+      }
+    }
+  } else if (warp >= 4) {
     // ===================== producer: gather, widen, publish =====================
     const int pt = tid - 128;  // 0..127: one slot per thread
     for (int tile = 0; tile < ntiles; ++tile) {
-      const int st = tile & 1;
-      if (tile >= 2 && healthy) healthy = tc::bar_wait(&empty[st], ((tile >> 1) - 1) & 1);
+      const int st = tile % NS;
+      if (tile >= NS && healthy) healthy = tc::bar_wait(&empty[st], ((tile / NS) - 1) & 1);
       // slot -> (type, row): 0 skip, 1 compressed entry, 2 raw window token
       {
         const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
@@ -598,23 +652,36 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       named_sync(1, 128);
       uint8_t* Kt = Kst + st * 3 * kKB;
       uint8_t* Vt = Vst + st * 2 * kKB;
-      // The tile's slots are an entry run [0, ne) then a window run [ne, ne + nw):
-      // contiguous runs are copied with consecutive lanes on consecutive 16-byte
-      // chunks (512-byte warp requests); selected entries are gathered four keys
-      // per warp instruction (8 lanes per 128-byte row).
+      // The tile's slots are an entry run [0, ne) then a window run [ne, ne + nw).
       const int64_t a0 = s0 + static_cast<int64_t>(tile) * kTcKeys;
       const int64_t a1 = (a0 + kTcKeys) < s1 ? (a0 + kTcKeys) : s1;
       const int ne = static_cast<int>(((a1 < n_ent ? a1 : n_ent) - a0) > 0 ? ((a1 < n_ent ? a1 : n_ent) - a0) : 0);
       const int nw = static_cast<int>(a1 - a0) - ne;
       const int pwarp = warp - 4;
+      // FP8 entries: thread pt owns 16-code chunk c = pt % 8 of keys pt / 8 + 16 j
+      // (eight lanes per 128-byte row, four rows per warp instruction); the
+      // codes and scales go to registers here and are widened after the
+      // asynchronous copies below are issued.
+      uint4 codes[8];
+      float scl[8];
+      if (FP8) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int key = (pt >> 3) + 16 * j;
+          const bool ok = key < ne && stype[st][key] == 1;
+          const int64_t r = ok ? srow[st][key] : 0;
+          codes[j] = ok ? ldg_nc16(p.cnope + r * kDNope + (pt & 7) * 16) : make_uint4(0u, 0u, 0u, 0u);
+          scl[j] = ok ? __ldg(p.cscale + r) : 0.f;
+        }
+      }
+      // Contiguous runs are copied with consecutive lanes on consecutive 16-byte
+      // chunks (512-byte warp requests); selected entries are gathered four keys
+      // per warp instruction (8 lanes per 128-byte row).
       if (ne > 0 && dense) {
         const int64_t r0 = srow[st][0];
         if (FP8) {
-          for (int pc = pt; pc < ne * 8; pc += 128) {
-            cp_async16(rawst + st * kKB + pc * 16, p.cnope + r0 * kDNope + pc * 16);
+          for (int pc = pt; pc < ne * 8; pc += 128)
             cp_async16(Kt + 2 * kKB + tc::sw128(pc >> 3, pc & 7), p.crope + r0 * kDRope + pc * 8);
-          }
-          if (pt < ne) cp_async4(&sc[st][pt], p.cscale + r0 + pt);
         } else {
           for (int pc = pt; pc < ne * 24; pc += 128) {
             const int key = pc / 24, c = pc % 24;
@@ -637,14 +704,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
           const int64_t r = srow[st][key];
           const int bytes = type ? 16 : 0;
           if (FP8) {
-            cp_async16(rawst + st * kKB + key * kDNope + c * 16, type ? p.cnope + r * kDNope + c * 16 : p.cnope, bytes);
             cp_async16(Kt + 2 * kKB + tc::sw128(key, c), type ? p.crope + r * kDRope + c * 8 : p.crope, bytes);
-            if (c == 0) {
-              if (type)
-                cp_async4(&sc[st][key], p.cscale + r);
-              else
-                sc[st][key] = 1.f;
-            }
           } else {
 #pragma unroll
             for (int j = 0; j < 3; ++j)
@@ -673,7 +733,6 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
             cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), src);
           }
         }
-        if (FP8 && pt >= ne && pt < ne + nw) sc[st][pt] = 1.f;
       }
       // slots past the end of the row: zero rows (their logits are masked)
       for (int pc = pt; pc < (kTcKeys - ne - nw) * 24; pc += 128) {
@@ -686,27 +745,22 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
           cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.q, 0);
         }
       }
-      if (FP8 && pt >= ne + nw) sc[st][pt] = 1.f;
       cp_async_commit();
-      cp_async_wait<0>();
-      named_sync(1, 128);
-      if (FP8) {  // code * scale -> bf16 into the swizzled K (and V) tile
-        for (int piece = pt; piece < kTcKeys * 8; piece += 128) {
-          const int key = piece >> 3, c = piece & 7;
-          if (stype[st][key] != 1) continue;
-          const uint4 codes = *reinterpret_cast<const uint4*>(rawst + st * kKB + key * kDNope + c * 16);
-          const float scl = sc[st][key];
-          const uint32_t w4[4] = {codes.x, codes.y, codes.z, codes.w};
+      if (FP8) {  // code * scale -> bf16 into the swizzled K (and V) tile; skipped slots get zeros
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int key = (pt >> 3) + 16 * j, c = pt & 7;
+          if (key >= ne) continue;
+          const uint32_t w4[4] = {codes[j].x, codes[j].y, codes[j].z, codes[j].w};
           uint32_t outw[8];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-#pragma unroll
-            for (int hlf = 0; hlf < 2; ++hlf) {
-              __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
-                  static_cast<__nv_fp8x2_storage_t>((w4[q] >> (16 * hlf)) & 0xffffu), __NV_E4M3);
-              const float2 f = __half22float2(*reinterpret_cast<__half2*>(&hr));
-              outw[2 * q + hlf] = pack_bf16x2(f.x * scl, f.y * scl);
-            }
+            uint32_t h01, h23;
+            e4m3x4_to_f16x2x2(w4[q], h01, h23);
+            const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+            const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+            outw[2 * q] = pack_bf16x2(f01.x * scl[j], f01.y * scl[j]);
+            outw[2 * q + 1] = pack_bf16x2(f23.x * scl[j], f23.y * scl[j]);
           }
           const int blk = c >> 2;
           const uint4 lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
@@ -714,46 +768,26 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
           *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
           *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
           if (!SHV) {
-            uint8_t* Vt = Vst + st * 2 * kKB;
             *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
             *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
           }
         }
       }
+      cp_async_wait<0>();
       tc::fence_async_smem();
       named_sync(1, 128);
       if (pt == 0) bar_arrive(&full[st]);
     }
   } else {
-    // ===================== consumer: S MMA, softmax, PV MMA =====================
-    constexpr uint32_t kIdescS = tc::idesc_bf16(64, 64, false);
-    constexpr uint32_t kIdescO = tc::idesc_bf16(64, 64, true);
-    auto issue_s = [&](int tile) {  // thread 0 only
-      const int st = tile & 1;
-      const uint32_t tS = tmem + 64 * st;
-      const uint32_t qa = smem_u32(Qs), ka = smem_u32(Kst + st * 3 * kKB);
-      tc::fence_after_sync();
-#pragma unroll
-      for (int kk = 0; kk < 12; ++kk) {
-        const uint64_t adesc = tc::desc_sw128(qa + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-        const uint32_t kb = ka + (kk >> 2) * kKB + (kk & 3) * 32;
-        tc::mma_bf16_ss(tS, adesc, tc::desc_sw128(kb, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-        tc::mma_bf16_ss(tS + kHalfLane, adesc, tc::desc_sw128(kb + 64 * 128, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-      }
-      tc::mma_commit(&sdone[st]);
-    };
-    if (ntiles > 0 && tid == 0) {
-      if (healthy) healthy = tc::bar_wait(&full[0], 0);
-      issue_s(0);
-    }
+    // ===================== consumer: softmax =====================
     for (int tile = 0; tile < ntiles; ++tile) {
-      const int st = tile & 1;
-      if (healthy) healthy = tc::bar_wait(&sdone[st], (tile >> 1) & 1);
+      const int kst = tile % NS, pb = tile & 1;
+      if (healthy) healthy = tc::bar_wait(&sdone[pb], (tile >> 1) & 1);
       tc::fence_after_sync();
       float sv[64];
-      tc::tmem_ld32(tmem + 64 * st + lane_base, sv);
-      tc::tmem_ld32(tmem + 64 * st + lane_base + 32, sv + 32);
-      const uint32_t vm0 = vmask[st][2 * half], vm1 = vmask[st][2 * half + 1];
+      tc::tmem_ld32(tmem + 64 * pb + lane_base, sv);
+      tc::tmem_ld32(tmem + 64 * pb + lane_base + 32, sv + 32);
+      const uint32_t vm0 = vmask[kst][2 * half], vm1 = vmask[kst][2 * half + 1];
       float mx = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
@@ -780,7 +814,8 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       l += sum;
       if (tile > 0 && __any_sync(0xffffffffu, resc)) {
         // O must be quiet: the previous tile's PV has to be done
-        if (healthy) healthy = tc::bar_wait(&empty[(tile - 1) & 1], ((tile - 1) >> 1) & 1);
+        const int prev = tile - 1;
+        if (healthy) healthy = tc::bar_wait(&empty[prev % NS], (prev / NS) & 1);
         tc::fence_after_sync();
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -793,7 +828,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         tc::tmem_wait_st();
       }
       {
-        uint8_t* Pb = Pst + st * 2 * 8192 + half * 8192;  // keys half*64 .. half*64+63
+        uint8_t* Pb = Pst + pb * 2 * 8192 + half * 8192;  // keys half*64 .. half*64+63
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const uint4 v = make_uint4(pack_bf16x2(sv[8 * c], sv[8 * c + 1]), pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]),
@@ -805,28 +840,11 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       tc::fence_async_smem();
       tc::fence_before_sync();
       named_sync(2, 128);
-      if (tid == 0) {
-        tc::fence_after_sync();
-        const uint32_t pa = smem_u32(Pst + st * 2 * 8192);
-        const uint32_t va = SHV ? smem_u32(Kst + st * 3 * kKB) : smem_u32(Vst + st * 2 * kKB);
-#pragma unroll
-        for (int ks = 0; ks < kTcKeys / 16; ++ks) {
-          const uint64_t adesc = tc::desc_sw128(pa + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-          const uint32_t vb = va + ks * 2048;
-          const uint32_t acc = (tile > 0 || ks > 0) ? 1u : 0u;
-          tc::mma_bf16_ss(tO, adesc, tc::desc_sw128(vb, kKB, 1024), kIdescO, acc);
-          tc::mma_bf16_ss(tO + kHalfLane, adesc, tc::desc_sw128(vb + kKB, kKB, 1024), kIdescO, acc);
-        }
-        tc::mma_commit(&empty[st]);
-        if (tile + 1 < ntiles) {  // next tile's S right behind this PV
-          if (healthy) healthy = tc::bar_wait(&full[st ^ 1], ((tile + 1) >> 1) & 1);
-          issue_s(tile + 1);
-        }
-      }
+      if (tid == 0) bar_arrive(&pready[pb]);
     }
     if (ntiles > 0) {
       const int last = ntiles - 1;
-      if (healthy) healthy = tc::bar_wait(&empty[last & 1], (last >> 1) & 1);
+      if (healthy) healthy = tc::bar_wait(&empty[last % NS], (last / NS) & 1);
       tc::fence_after_sync();
     }
   }
