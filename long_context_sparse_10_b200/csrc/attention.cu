@@ -445,37 +445,41 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
 
 
 // ---------------------------------------------------------------------------
-// H = 64: tcgen05 path.  Warps 0-3 run the online softmax, warps 4-7 gather
-// and widen key tiles, one thread of warp 8 issues every MMA; accumulators live
-// in tensor memory (TMEM).  A tile is 128 keys.  An M = 64 accumulator fills
-// 16 of the 32 lanes of each TMEM lane quarter (row m -> lane (m % 16) +
-// 32 (m / 16)); a second one at lane offset 16 fills the other half.  So
-//   S = Q K^T of keys 0..63   -> lanes +0,  columns [0, 64)
-//   S = Q K^T of keys 64..127 -> lanes +16, columns [0, 64)
-//   O channels 0..63          -> lanes +0,  columns [64, 128)
-//   O channels 64..127        -> lanes +16, columns [64, 128)
-// and thread (warp q, lane L) owns head 16q + L % 16 and half L / 16 of both:
-// every lane works, and the two halves of a head combine their row max with
-// one shuffle.  Operands sit in shared memory in the 128-byte-swizzled layout
-// (8 rows x 128 bytes per 1024-byte atom): Q and K K-major in three 64-dim
-// blocks, P K-major in two 64-key blocks, V read MN-major straight out of the
-// first two K blocks when key and value are shared.  O is rescaled in TMEM
-// only when a row's running max grows by more than 2^8 (probabilities stay <=
-// 256 in between).  FP8 entries are dequantised (code x scale, rounded to
-// bf16) from registers into the K tile.  When key and value are shared the K
-// tile has three stages, so the gather runs up to two tiles ahead and the
-// next tile's S = Q K^T is computed while the softmax works on this one
-// (issue order S(0), S(1), then PV(t), S(t+2)); with a separate V tile there
-// is room for two.  Every mbarrier wait is bounded; a timeout sets the device
-// error word instead of hanging.
+// H = 64: tcgen05 path, with the keys as the MMA's M dimension.  One query's
+// 64 heads share every key (MQA), so instead of S = Q K^T (M = 64 heads, a
+// half-rate shape) the tensor cores compute
+//   S^T = K Q^T     M = 128 keys,     N = 64 heads, K = 192 dims  (12 MMAs)
+//   O^T += V^T P^T  M = 128 channels, N = 64 heads, K = 128 keys  (8 MMAs)
+//   l^T += 1 P^T    M = 128 (all rows equal), N = 64 heads        (8 MMAs)
+// all at M = 128, with fp32 accumulators in tensor memory: S^T double-buffered
+// in columns [0, 128), O^T in [128, 192), the running sums l in [192, 256).
+// Softmax thread t (warps 0-3) owns TMEM lane t, i.e. key t of the tile: it
+// reads its 64 head logits, and writes its row of P^T (128 bytes, the B
+// operand's MN-major layout) to shared memory.  The running max per head
+// (m_ref, shared memory) changes only when some logit exceeds it by more
+// than 2^20 (log2 units) -- always on a CTA's first tile, rarely after; then
+// the tile's per-head maxima are reduced across the 128 keys (a halving
+// shuffle per warp), O and l are rescaled in TMEM, and the tile continues.
+// Operands sit in shared memory in the 128-byte-swizzled layout: K K-major
+// (three 64-dim blocks), Q K-major, V^T read MN-major straight out of the
+// first two K blocks when key and value are shared, P^T MN-major, and the
+// all-ones A operand of the l update is one 1 KB swizzle atom read with a
+// zero row-group stride.  Warps 4-7 gather and widen key tiles (FP8 entries
+// dequantised, code x scale rounded to bf16, from registers into the K
+// tile); one thread of warp 8 issues every MMA in the order S(0), S(1), then
+// per tile t: PV(t) and the l update once P(t) is written, S(t+2) into the
+// TMEM buffer P(t)'s softmax has drained.  When key and value are shared the
+// K tile has three stages (two with a separate V tile).  Every mbarrier wait
+// is bounded; a timeout sets the device error word instead of hanging.
 // ---------------------------------------------------------------------------
 constexpr int kTcKeys = 128;
 
 constexpr int kTcThreads = 256;     // query-blocked prefill kernel: warps 0-3 softmax + MMA, 4-7 loads
-constexpr int kTcDecThreads = 288;  // attn_tc_kernel: warps 0-3 softmax, 4-7 loads, 8 MMA issue
+constexpr int kTcDecThreads = 544;  // attn_tc_kernel: warps 0-7 softmax, 8-15 loads, 16 MMA issue
+constexpr float kRescaleLog2 = 20.f;  // rescale O and l when a logit tops m_ref by more than 2^20
 
 struct TcLayout {
-  size_t q, k, v, p, stype, srow, vmask, bars, total;
+  size_t q, k, v, p, ones, stype, srow, vmask, mref, corr, wmax, bars, total;
 };
 
 // K-tile stages: three when the V tile is the K tile, two otherwise.
@@ -488,10 +492,14 @@ __host__ __device__ inline TcLayout tc_layout(bool fp8, bool shv, int tps) {
   L.q = off; off += 3 * 8192;                    // Q: 64 heads x 192 dims
   L.k = off; off += ns * 3 * 16384;              // K: stages x 128 keys x 192 dims
   L.v = off; if (!shv) off += ns * 2 * 16384;    // V: stages x 128 keys x 128 dims
-  L.p = off; off += 2 * 2 * 8192;                // P: 2 buffers x 64 heads x 128 keys
+  L.p = off; off += 2 * 16384;                   // P^T: 2 buffers x 128 keys x 64 heads (epilogue: O^T transpose)
+  L.ones = off; off += 1024;                     // all-ones swizzle atom
   L.stype = off; off += ns * kTcKeys * sizeof(int);
   L.srow = off; off += ns * kTcKeys * sizeof(int64_t);
   L.vmask = off; off += ns * 4 * sizeof(uint32_t);
+  L.mref = off; off += 64 * sizeof(float);
+  L.corr = off; off += 64 * sizeof(float);
+  L.wmax = off; off += 4 * 64 * sizeof(float);
   L.bars = off; off += 128;
   (void)fp8, (void)tps;
   const size_t reduce = 80 * (kDV + 4) * sizeof(float);  // cluster merge records (reuse Q/K)
@@ -502,8 +510,62 @@ __host__ __device__ inline TcLayout tc_layout(bool fp8, bool shv, int tps) {
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
 }
+// Named barrier that also ORs a predicate over the participating threads.
+__device__ __forceinline__ bool named_sync_or(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n.reg .pred pi, po;\nsetp.ne.u32 pi, %1, 0;\nbarrier.red.or.pred po, %2, %3, pi;\nselp.u32 %0, 1, 0, po;\n}\n"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ void bar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Per-head maximum over the 32 lanes of a warp, each lane holding v[0..63]
+// (one key, 64 heads): five halving exchange steps (62 shuffles).  Returns in
+// v[0], v[1] the maxima of heads h0 and h0 + 1, h0 = 2 * bitrev5(lane) laid
+// out as below.
+__device__ __forceinline__ int warp_head_max64(float* v, int lane) {
+#pragma unroll
+  for (int w = 32, o = 16; o >= 1; w >>= 1, o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float keep = up ? v[i + w] : v[i];
+      const float send = up ? v[i] : v[i + w];
+      v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+    }
+  }
+  return ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 + ((lane >> 1) & 1) * 4 +
+         (lane & 1) * 2;
+}
+
+// Per-head maximum over the 32 lanes of a warp, each lane holding v[0..31]
+// (one key, 32 heads): five halving exchange steps (31 shuffles); returns in
+// v[0] the maximum of head bitrev-ordered h0 below.
+__device__ __forceinline__ int warp_head_max32(float* v, int lane) {
+#pragma unroll
+  for (int w = 16, o = 16; o >= 1; w >>= 1, o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float keep = up ? v[i + w] : v[i];
+      const float send = up ? v[i] : v[i + w];
+      v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+    }
+  }
+  return ((lane >> 4) & 1) * 16 + ((lane >> 3) & 1) * 8 + ((lane >> 2) & 1) * 4 + ((lane >> 1) & 1) * 2 + (lane & 1);
+}
+
+// 2^x by the hardware approximation (relative error ~2^-22, far below the
+// bf16 rounding of the probabilities it feeds); 0 for x = -inf.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 template <bool FP8, bool SHV>
@@ -516,10 +578,14 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   uint8_t* Kst = smem + L.k;
   uint8_t* Vst = smem + L.v;
   uint8_t* Pst = smem + L.p;
+  uint8_t* ones = smem + L.ones;
   constexpr int NS = tc_stages(SHV);
   auto stype = reinterpret_cast<int(*)[kTcKeys]>(smem + L.stype);
   auto srow = reinterpret_cast<int64_t(*)[kTcKeys]>(smem + L.srow);
   auto vmask = reinterpret_cast<uint32_t(*)[4]>(smem + L.vmask);
+  float* mref = reinterpret_cast<float*>(smem + L.mref);
+  float* corr_s = reinterpret_cast<float*>(smem + L.corr);
+  auto wmax = reinterpret_cast<float(*)[64]>(smem + L.wmax);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NS] K stage loaded
   uint64_t* empty = full + NS;                                    // [NS] PV of the stage's tile done
   uint64_t* sdone = empty + NS;                                   // [2] S of the tile done (TMEM buffer)
@@ -558,29 +624,27 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
     cp_async16(Qs + (ch >> 3) * 8192 + tc::sw128(hh, ch & 7), p.q + (row * 64 + hh) * kDQK + ch * 8);
   }
   cp_async_commit();
+  if (tid < 64) {
+    reinterpret_cast<uint4*>(ones)[tid] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    mref[tid] = -INFINITY;
+  }
   cp_async_wait<0>();
   tc::fence_async_smem();
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
-  constexpr uint32_t kHalfLane = 16u << 16;
   bool healthy = true;  // false after a barrier wait ran out: later waits are skipped
-
-  float m_ref = -INFINITY, l = 0.f;  // consumer state (head h, key/channel half)
-  const int half = lane >> 4;
-  const int h = (warp & 3) * 16 + (lane & 15);
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const uint32_t tO = tmem + 128;
+  const uint32_t tO = tmem + 128, tL = tmem + 192;
 
-  constexpr uint32_t kIdescS = tc::idesc_bf16(64, 64, false);
-  constexpr uint32_t kIdescO = tc::idesc_bf16(64, 64, true);
-  if (warp == 8) {
+  constexpr uint32_t kIdescS = tc::idesc_bf16(128, 64, false, false);  // A = K (K-major), B = Q (K-major)
+  constexpr uint32_t kIdescO = tc::idesc_bf16(128, 64, true, true);    // A = V^T (MN-major), B = P^T (MN-major)
+  constexpr uint32_t kIdescL = tc::idesc_bf16(128, 64, true, false);   // A = ones, B = P^T (MN-major)
+  if (warp == 16) {
     // ===================== MMA issue (one thread) =====================
-    // S(0), S(1), then per tile t: PV(t) once P(t) is written, S(t+2) into the
-    // TMEM buffer P(t)'s softmax has drained.  A commit tracks every earlier
-    // MMA of this thread, so S(t+2) done implies PV(t) done, which frees P
-    // buffer t % 2 for tile t+2.
+    // A commit tracks every earlier MMA of this thread: S(t+2) done implies
+    // PV(t) done, which frees P buffer t % 2 for tile t+2.
     auto issue_s = [&](int tile) {
       const int kst = tile % NS;
       const uint32_t tS = tmem + 64 * (tile & 1);
@@ -588,10 +652,9 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       tc::fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < 12; ++kk) {
-        const uint64_t adesc = tc::desc_sw128(qa + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-        const uint32_t kb = ka + (kk >> 2) * kKB + (kk & 3) * 32;
-        tc::mma_bf16_ss(tS, adesc, tc::desc_sw128(kb, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-        tc::mma_bf16_ss(tS + kHalfLane, adesc, tc::desc_sw128(kb + 64 * 128, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+        const uint64_t adesc = tc::desc_sw128(ka + (kk >> 2) * kKB + (kk & 3) * 32, 16, 1024);
+        const uint64_t bdesc = tc::desc_sw128(qa + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+        tc::mma_bf16_ss(tS, adesc, bdesc, kIdescS, kk > 0 ? 1u : 0u);
       }
       tc::mma_commit(&sdone[tile & 1]);
     };
@@ -600,19 +663,19 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         if (healthy) healthy = tc::bar_wait(&full[t0 % NS], (t0 / NS) & 1);
         issue_s(t0);
       }
+      const uint64_t onesdesc = tc::desc_sw128(smem_u32(ones), 16, 0);
       for (int tile = 0; tile < ntiles; ++tile) {
         const int kst = tile % NS, pb = tile & 1;
         if (healthy) healthy = tc::bar_wait(&pready[pb], (tile >> 1) & 1);
         tc::fence_after_sync();
-        const uint32_t pa = smem_u32(Pst + pb * 2 * 8192);
+        const uint32_t pa = smem_u32(Pst + pb * 16384);
         const uint32_t va = SHV ? smem_u32(Kst + kst * 3 * kKB) : smem_u32(Vst + kst * 2 * kKB);
 #pragma unroll
         for (int ks = 0; ks < kTcKeys / 16; ++ks) {
-          const uint64_t adesc = tc::desc_sw128(pa + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-          const uint32_t vb = va + ks * 2048;
+          const uint64_t pdesc = tc::desc_sw128(pa + ks * 2048, 8192, 1024);
           const uint32_t acc = (tile > 0 || ks > 0) ? 1u : 0u;
-          tc::mma_bf16_ss(tO, adesc, tc::desc_sw128(vb, kKB, 1024), kIdescO, acc);
-          tc::mma_bf16_ss(tO + kHalfLane, adesc, tc::desc_sw128(vb + kKB, kKB, 1024), kIdescO, acc);
+          tc::mma_bf16_ss(tO, tc::desc_sw128(va + ks * 2048, kKB, 1024), pdesc, kIdescO, acc);
+          tc::mma_bf16_ss(tL, onesdesc, pdesc, kIdescL, acc);
         }
         tc::mma_commit(&empty[kst]);
         if (tile + 2 < ntiles) {
@@ -621,14 +684,14 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         }
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 8) {
     // ===================== producer: gather, widen, publish =====================
-    const int pt = tid - 128;  // 0..127: one slot per thread
+    const int pt = tid - 256;  // 0..255; threads 0..127 also own one slot each
     for (int tile = 0; tile < ntiles; ++tile) {
       const int st = tile % NS;
       if (tile >= NS && healthy) healthy = tc::bar_wait(&empty[st], ((tile / NS) - 1) & 1);
       // slot -> (type, row): 0 skip, 1 compressed entry, 2 raw window token
-      {
+      if (pt < kTcKeys) {
         const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
         int type = 0;
         int64_t r = 0;
@@ -647,9 +710,9 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         stype[st][pt] = type;
         srow[st][pt] = r;
         const uint32_t bal = __ballot_sync(0xffffffffu, type != 0);
-        if (lane == 0) vmask[st][warp - 4] = bal;
+        if (lane == 0) vmask[st][warp - 8] = bal;
       }
-      named_sync(1, 128);
+      named_sync(1, 256);
       uint8_t* Kt = Kst + st * 3 * kKB;
       uint8_t* Vt = Vst + st * 2 * kKB;
       // The tile's slots are an entry run [0, ne) then a window run [ne, ne + nw).
@@ -657,17 +720,17 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       const int64_t a1 = (a0 + kTcKeys) < s1 ? (a0 + kTcKeys) : s1;
       const int ne = static_cast<int>(((a1 < n_ent ? a1 : n_ent) - a0) > 0 ? ((a1 < n_ent ? a1 : n_ent) - a0) : 0);
       const int nw = static_cast<int>(a1 - a0) - ne;
-      const int pwarp = warp - 4;
-      // FP8 entries: thread pt owns 16-code chunk c = pt % 8 of keys pt / 8 + 16 j
+      const int pwarp = warp - 8;
+      // FP8 entries: thread pt owns 16-code chunk c = pt % 8 of keys pt / 8 + 32 j
       // (eight lanes per 128-byte row, four rows per warp instruction); the
       // codes and scales go to registers here and are widened after the
       // asynchronous copies below are issued.
-      uint4 codes[8];
-      float scl[8];
+      uint4 codes[4];
+      float scl[4];
       if (FP8) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int key = (pt >> 3) + 16 * j;
+        for (int j = 0; j < 4; ++j) {
+          const int key = (pt >> 3) + 32 * j;
           const bool ok = key < ne && stype[st][key] == 1;
           const int64_t r = ok ? srow[st][key] : 0;
           codes[j] = ok ? ldg_nc16(p.cnope + r * kDNope + (pt & 7) * 16) : make_uint4(0u, 0u, 0u, 0u);
@@ -680,15 +743,15 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       if (ne > 0 && dense) {
         const int64_t r0 = srow[st][0];
         if (FP8) {
-          for (int pc = pt; pc < ne * 8; pc += 128)
+          for (int pc = pt; pc < ne * 8; pc += 256)
             cp_async16(Kt + 2 * kKB + tc::sw128(pc >> 3, pc & 7), p.crope + r0 * kDRope + pc * 8);
         } else {
-          for (int pc = pt; pc < ne * 24; pc += 128) {
+          for (int pc = pt; pc < ne * 24; pc += 256) {
             const int key = pc / 24, c = pc % 24;
             cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.ck + r0 * kDQK + pc * 8);
           }
           if (!SHV) {
-            for (int pc = pt; pc < ne * 16; pc += 128) {
+            for (int pc = pt; pc < ne * 16; pc += 256) {
               const int key = pc >> 4, c = pc & 15;
               const __nv_bfloat16* src = p.cv ? p.cv + r0 * kDV + pc * 8 : p.ck + (r0 + key) * kDQK + c * 8;
               cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), src);
@@ -697,7 +760,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         }
       } else if (ne > 0) {
         const int c = lane & 7;
-        for (int kb = pwarp * 4; kb < ne; kb += 16) {
+        for (int kb = pwarp * 4; kb < ne; kb += 32) {
           const int key = kb + (lane >> 3);
           if (key >= ne) continue;
           const int type = stype[st][key];
@@ -722,12 +785,12 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       }
       if (nw > 0) {  // raw window tokens: contiguous rows
         const int64_t rw0 = srow[st][ne];
-        for (int pc = pt; pc < nw * 24; pc += 128) {
+        for (int pc = pt; pc < nw * 24; pc += 256) {
           const int key = ne + pc / 24, c = pc % 24;
           cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.wk + rw0 * kDQK + pc * 8);
         }
         if (!SHV) {
-          for (int pc = pt; pc < nw * 16; pc += 128) {
+          for (int pc = pt; pc < nw * 16; pc += 256) {
             const int key = ne + (pc >> 4), c = pc & 15;
             const __nv_bfloat16* src = p.wv ? p.wv + rw0 * kDV + pc * 8 : p.wk + (rw0 + (pc >> 4)) * kDQK + c * 8;
             cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), src);
@@ -735,12 +798,12 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         }
       }
       // slots past the end of the row: zero rows (their logits are masked)
-      for (int pc = pt; pc < (kTcKeys - ne - nw) * 24; pc += 128) {
+      for (int pc = pt; pc < (kTcKeys - ne - nw) * 24; pc += 256) {
         const int key = ne + nw + pc / 24, c = pc % 24;
         cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.q, 0);
       }
       if (!SHV) {
-        for (int pc = pt; pc < (kTcKeys - ne - nw) * 16; pc += 128) {
+        for (int pc = pt; pc < (kTcKeys - ne - nw) * 16; pc += 256) {
           const int key = ne + nw + (pc >> 4), c = pc & 15;
           cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.q, 0);
         }
@@ -748,8 +811,8 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       cp_async_commit();
       if (FP8) {  // code * scale -> bf16 into the swizzled K (and V) tile; skipped slots get zeros
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int key = (pt >> 3) + 16 * j, c = pt & 7;
+        for (int j = 0; j < 4; ++j) {
+          const int key = (pt >> 3) + 32 * j, c = pt & 7;
           if (key >= ne) continue;
           const uint32_t w4[4] = {codes[j].x, codes[j].y, codes[j].z, codes[j].w};
           uint32_t outw[8];
@@ -775,71 +838,84 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       }
       cp_async_wait<0>();
       tc::fence_async_smem();
-      named_sync(1, 128);
+      named_sync(1, 256);
       if (pt == 0) bar_arrive(&full[st]);
     }
   } else {
-    // ===================== consumer: softmax =====================
+    // ===================== softmax: thread = key of the tile, 32 heads =====================
+    // warp w: keys 32 (w % 4) .. +31 (its TMEM lane quarter), heads 32 (w / 4) .. +31
+    const int key = (warp & 3) * 32 + lane;
+    const int hb = (warp >> 2) * 32;
     for (int tile = 0; tile < ntiles; ++tile) {
       const int kst = tile % NS, pb = tile & 1;
       if (healthy) healthy = tc::bar_wait(&sdone[pb], (tile >> 1) & 1);
       tc::fence_after_sync();
-      float sv[64];
-      tc::tmem_ld32(tmem + 64 * pb + lane_base, sv);
-      tc::tmem_ld32(tmem + 64 * pb + lane_base + 32, sv + 32);
-      const uint32_t vm0 = vmask[kst][2 * half], vm1 = vmask[kst][2 * half + 1];
-      float mx = -INFINITY;
+      float sv[32];
+      tc::tmem_ld32(tmem + 64 * pb + lane_base + hb, sv);
+      const bool valid = stype[kst][key] != 0;
+      bool over = false;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const bool ok = ((j < 32 ? vm0 : vm1) >> (j & 31)) & 1u;
-        sv[j] = ok ? sv[j] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, sv[j]);
-      }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      const float m_new = fmaxf(m_ref, mx);
-      const bool resc = m_new > m_ref + 8.f;
-      float corr = 1.f;
-      if (resc) {
-        corr = exp2f(m_ref - m_new);
-        m_ref = m_new;
-        l *= corr;
-      }
-      const float base = m_ref == -INFINITY ? 0.f : m_ref;
-      float sum = 0.f;
+      for (int j = 0; j < 32; j += 4) {
+        const float4 m4 = *reinterpret_cast<const float4*>(mref + hb + j);
+        const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        sv[j] = exp2f(sv[j] - base);
-        sum += sv[j];
-      }
-      l += sum;
-      if (tile > 0 && __any_sync(0xffffffffu, resc)) {
-        // O must be quiet: the previous tile's PV has to be done
-        const int prev = tile - 1;
-        if (healthy) healthy = tc::bar_wait(&empty[prev % NS], (prev / NS) & 1);
-        tc::fence_after_sync();
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float ov[32];
-          tc::tmem_ld32(tO + lane_base + 32 * c, ov);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] *= corr;
-          tc::tmem_st32(tO + lane_base + 32 * c, ov);
+        for (int u = 0; u < 4; ++u) {
+          sv[j + u] = valid ? sv[j + u] * p.scale_log2 : -INFINITY;
+          over |= sv[j + u] - mm[u] > kRescaleLog2;
         }
-        tc::tmem_wait_st();
       }
-      {
-        uint8_t* Pb = Pst + pb * 2 * 8192 + half * 8192;  // keys half*64 .. half*64+63
+      if (named_sync_or(2, 256, over)) {
+        // new per-head maxima: this tile's maximum over its valid keys (the
+        // reduction consumes sv; the logits are read again from TMEM below)
+        const int h0 = warp_head_max32(sv, lane);
+        wmax[warp & 3][hb + h0] = sv[0];
+        named_sync(2, 256);
+        if (tid < 64) {
+          const float mo = mref[tid];
+          const float mt = fmaxf(fmaxf(wmax[0][tid], wmax[1][tid]), fmaxf(wmax[2][tid], wmax[3][tid]));
+          const float mn = fmaxf(mo, mt);
+          corr_s[tid] = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+          mref[tid] = mn;
+        }
+        named_sync(2, 256);
+        if (tile > 0) {  // O and l must be quiet: the previous tile's PV has to be done
+          const int prev = tile - 1;
+          if (healthy) healthy = tc::bar_wait(&empty[prev % NS], (prev / NS) & 1);
+          tc::fence_after_sync();
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = make_uint4(pack_bf16x2(sv[8 * c], sv[8 * c + 1]), pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]),
-                                     pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]),
-                                     pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]));
-          *reinterpret_cast<uint4*>(Pb + tc::sw128(h, c)) = v;
+          for (int c = 0; c < 2; ++c) {  // this thread's 32 columns of O^T, then of l^T
+            const uint32_t ta = (c == 0 ? tO : tL) + lane_base + hb;
+            float ov[32];
+            tc::tmem_ld32(ta, ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] *= corr_s[hb + i];
+            tc::tmem_st32(ta, ov);
+          }
+          tc::tmem_wait_st();
+        }
+        tc::tmem_ld32(tmem + 64 * pb + lane_base + hb, sv);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[j] = valid ? sv[j] * p.scale_log2 : -INFINITY;
+      }
+      // this key's P^T row, heads hb .. hb+31: four 16-byte chunks of the 128-byte swizzled row
+      {
+        uint8_t* Pb = Pst + pb * 16384;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float4 ma = *reinterpret_cast<const float4*>(mref + hb + 8 * c);
+          const float4 mb = *reinterpret_cast<const float4*>(mref + hb + 8 * c + 4);
+          const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+          float pv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) pv[u] = valid ? fast_exp2(sv[8 * c + u] - mm[u]) : 0.f;
+          const uint4 v = make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
+                                     pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
+          *reinterpret_cast<uint4*>(Pb + tc::sw128(key, (hb >> 3) + c)) = v;
         }
       }
       tc::fence_async_smem();
       tc::fence_before_sync();
-      named_sync(2, 128);
+      named_sync(2, 256);
       if (tid == 0) bar_arrive(&pready[pb]);
     }
     if (ntiles > 0) {
@@ -850,83 +926,81 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   }
   cp_async_wait<0>();
   pdl_trigger();  // the epilogue is all that is left
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
 
-  // ---- output (consumer threads): channels half*64..+63 of head h, with (m_ref, l) ----
-  if (p.part != nullptr) {  // split record in global memory, merged by attn_merge_kernel
-    if (warp < 4) {
-      const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
-      float* rec = p.part + ((row * p.cl + split) * 64 + h) * kRec;
+  // ---- O^T (lane = channel) -> shared-memory transpose T[h][c] (fp32, in the P buffers), l per head ----
+  float* T = reinterpret_cast<float*>(Pst);
+  float* lrow = corr_s;  // l per head
+  if (warp < 8) {
+    const int c = (warp & 3) * 32 + lane, hb = (warp >> 2) * 32;
+    float ov[32];
+    if (ntiles > 0) {
+      tc::tmem_ld32(tO + lane_base + hb, ov);
+    } else {
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float ov[32];
-        if (ntiles > 0) {
-          tc::tmem_ld32(tO + lane_base + 32 * c, ov);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = 0.f;
-        }
-        const int d0 = half * 64 + 32 * c;
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(rec + d0 + i) = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
-      }
-      if (half == 0) *reinterpret_cast<float2*>(rec + kDV) = make_float2(m_ref, l_row);
+      for (int i = 0; i < 32; ++i) ov[i] = 0.f;
     }
-    tc::fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, 256);
-    return;
-  }
-  cg::cluster_group cluster = cg::this_cluster();
-  if (p.cl > 1) cluster.sync();  // peers may now write merge records over our Q/K tiles
-  float* rbuf = reinterpret_cast<float*>(smem);
-  if (warp < 4) {
-    const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
-    float* dst = nullptr;
-    if (p.cl > 1) {
-      const int owner = h % p.cl;
-      dst = cluster.map_shared_rank(rbuf, owner) + (static_cast<int64_t>(h / p.cl) * p.cl + split) * kRec;
-    }
-    const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      float ov[32];
+    for (int i = 0; i < 32; ++i) T[(hb + i) * kDV + c] = ov[i];
+    if ((warp & 3) == 0) {  // every lane of l^T holds all 64 sums; lane 0 publishes this warp's 32
+      float lv[32];
       if (ntiles > 0) {
-        tc::tmem_ld32(tO + lane_base + 32 * c, ov);
+        tc::tmem_ld32(tL + lane_base + hb, lv);
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+        for (int i = 0; i < 32; ++i) lv[i] = 0.f;
       }
-      const int d0 = half * 64 + 32 * c;
-      if (p.cl > 1) {
+      if (lane == 0) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(dst + d0 + i) = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
-      } else {
-        __nv_bfloat16* o = p.out + (row * p.H + h) * kDV + d0;
-#pragma unroll
-        for (int i = 0; i < 32; i += 8)
-          *reinterpret_cast<uint4*>(o + i) =
-              make_uint4(pack_bf16x2(ov[i] * inv, ov[i + 1] * inv), pack_bf16x2(ov[i + 2] * inv, ov[i + 3] * inv),
-                         pack_bf16x2(ov[i + 4] * inv, ov[i + 5] * inv), pack_bf16x2(ov[i + 6] * inv, ov[i + 7] * inv));
-      }
-    }
-    if (half == 0) {
-      if (p.cl > 1) {
-        dst[kDV] = m_ref;
-        dst[kDV + 1] = l_row;
-      } else if (p.lse) {
-        p.lse[row * p.H + h] = l_row > 0.f ? (m_ref + log2f(l_row)) * kLn2 : -INFINITY;
+        for (int i = 0; i < 32; ++i) lrow[hb + i] = lv[i];
       }
     }
   }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, 256);
-  if (p.cl == 1) return;
+
+  if (p.part != nullptr) {  // split record in global memory, merged by attn_merge_kernel
+    for (int piece = tid; piece < 64 * 32; piece += kTcDecThreads) {
+      const int hh = piece >> 5, q4 = piece & 31;
+      float* rec = p.part + ((row * p.cl + split) * 64 + hh) * kRec;
+      *reinterpret_cast<float4*>(rec + 4 * q4) = *reinterpret_cast<const float4*>(T + hh * kDV + 4 * q4);
+    }
+    if (tid < 64) {
+      float* rec = p.part + ((row * p.cl + split) * 64 + tid) * kRec;
+      *reinterpret_cast<float2*>(rec + kDV) = make_float2(mref[tid], lrow[tid]);
+    }
+    return;
+  }
+  if (p.cl == 1) {
+    for (int piece = tid; piece < 64 * 16; piece += kTcDecThreads) {
+      const int hh = piece >> 4, q8 = piece & 15;
+      const float lh = lrow[hh];
+      const float inv = lh > 0.f ? 1.f / lh : 0.f;
+      const float* src = T + hh * kDV + 8 * q8;
+      *reinterpret_cast<uint4*>(p.out + (row * p.H + hh) * kDV + 8 * q8) =
+          make_uint4(pack_bf16x2(src[0] * inv, src[1] * inv), pack_bf16x2(src[2] * inv, src[3] * inv),
+                     pack_bf16x2(src[4] * inv, src[5] * inv), pack_bf16x2(src[6] * inv, src[7] * inv));
+    }
+    if (tid < 64 && p.lse) {
+      const float lh = lrow[tid];
+      p.lse[row * p.H + tid] = lh > 0.f ? (mref[tid] + log2f(lh)) * kLn2 : -INFINITY;
+    }
+    return;
+  }
+  // cluster: records into the owner CTA's shared memory (head h is owned by rank h % cl)
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();  // peers may now write merge records over our Q/K tiles
+  float* rbuf = reinterpret_cast<float*>(smem);
+  for (int piece = tid; piece < 64 * 32; piece += kTcDecThreads) {
+    const int hh = piece >> 5, q4 = piece & 31;
+    float* dst = cluster.map_shared_rank(rbuf, hh % p.cl) + (static_cast<int64_t>(hh / p.cl) * p.cl + split) * kRec;
+    *reinterpret_cast<float4*>(dst + 4 * q4) = *reinterpret_cast<const float4*>(T + hh * kDV + 4 * q4);
+  }
+  if (tid < 64) {
+    float* dst = cluster.map_shared_rank(rbuf, tid % p.cl) + (static_cast<int64_t>(tid / p.cl) * p.cl + split) * kRec;
+    dst[kDV] = mref[tid];
+    dst[kDV + 1] = lrow[tid];
+  }
   cluster.sync();
   const int sub = tid >> 5;  // warps 0-7, one head at a time each
   for (int j = sub; sub < 8 && split + j * p.cl < p.H; j += 8) {

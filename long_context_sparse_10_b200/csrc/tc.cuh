@@ -32,11 +32,12 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uin
 }
 
 // Instruction descriptor, kind::f16 with bf16 inputs and fp32 accumulation.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major, bool a_mn_major = false) {
   return (1u << 4)                                  // D = f32
          | (1u << 7)                                // A = bf16
          | (1u << 10)                               // B = bf16
-         | (b_mn_major ? (1u << 16) : 0u)           // B major-ness (A is K-major)
+         | (a_mn_major ? (1u << 15) : 0u)           // A major-ness
+         | (b_mn_major ? (1u << 16) : 0u)           // B major-ness
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
