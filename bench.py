@@ -60,15 +60,16 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def profile_traffic(kernel: str, source: str):
-    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel source."""
+def profile_traffic(kernel: str, source: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was captured on this workload and the
+    kernel source has not changed since."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.md")
     if not os.path.exists(path):
         return None
     sha = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
     for line in open(path):
-        m = re.match(r"\|\s*(\S+)\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]+)\s*\|", line)
-        if m and m.group(1) == kernel and m.group(3) == sha:
+        m = re.match(r"\|\s*(\S+)\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]+)\s*\|\s*([A-Za-z0-9_]+)", line)
+        if m and m.group(1) == kernel and m.group(3) == sha and m.group(4) == workload:
             return float(m.group(2))
     return None
 
@@ -539,7 +540,7 @@ def main():
         achieved = work / (kms * 1e-3) / 1e12
         peak = pk["bf16_tflops"]
         unit = "TFLOP/s"
-    traffic = profile_traffic(name, src)
+    traffic = profile_traffic(name, src, args.workload)
     roofline = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "peak_source": f"{pk_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
                 "traffic": traffic, "algorithmic_per_launch": work, "launch_ms": kms}
