@@ -178,6 +178,10 @@ def _split_cache(g, B, N):
 @pytest.mark.parametrize("kind,H,B,N,k,win,Tq", [
     ("csa", 64, 3, 5000, 512, 128, 1), ("csa", 16, 2, 3000, 2048, 128, 1), ("hca", 64, 2, 3000, 0, 128, 1),
     ("hca", 16, 3, 700, 0, 64, 1), ("csa", 64, 2, 4000, 256, 128, 4),
+    # rows split over many CTAs whose partial states merge through global records
+    ("hca", 64, 8, 8192, 0, 128, 1),   # the 1M-context decode's HCA shape: 17 CTAs per row
+    ("hca", 64, 2, 30000, 0, 128, 1),  # 59 CTAs per row, last split ragged
+    ("csa", 64, 8, 40000, 2048, 128, 1),  # the 1M-context decode's CSA shape (cluster merge)
 ])
 def test_decode_split_fp8(kind, H, B, N, k, win, Tq):
     g = np.random.default_rng(N + H + k)
