@@ -1,6 +1,8 @@
 // Host-side helpers shared by the entry points: argument checks, error text.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -39,6 +41,11 @@ cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStre
   cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
+
+// The driver's tensor-map encoder, fetched through the runtime so that the
+// library carries no link-time dependency on the driver library (null if the
+// driver does not provide it).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // Checks the launch just enqueued and counts it (csa_launch_count).  Called
 // exactly once after every kernel launch of the library.

@@ -1048,23 +1048,6 @@ size_t csa_indexer_topk_workspace_size(int64_t B, int64_t Tq, int64_t N, int32_t
 
 namespace csa {
 namespace {
-// The driver's tensor-map encoder, fetched through the runtime so that the
-// library carries no link-time dependency on the driver library.
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    else
-      cudaGetLastError();
-  });
-  return fn;
-}
-
 csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const uint8_t* kcodes, const float* kscale,
                         int64_t B, int64_t Tq, int64_t N, int64_t q_pos0, int32_t m, int32_t k, int32_t* idx,
                         void* workspace, size_t workspace_bytes, void* stream) {
