@@ -513,7 +513,8 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
       const int rows = static_cast<int>((e_end - base) < kLongTR ? (e_end - base) : kLongTR);
       if (threadIdx.x == 0) {
         tc::bar_arrive_expect_tx(&bars[st], static_cast<uint32_t>(rows) * 64u);
-        tc::bulk_load(dst, p.kcodes + (b * p.N + base) * kDI, static_cast<uint32_t>(rows) * 64u, &bars[st]);
+        tc::bulk_load_stream(dst, p.kcodes + (b * p.N + base) * kDI, static_cast<uint32_t>(rows) * 64u, &bars[st],
+                             tc::l2_evict_first_policy());
       }
       const int r = threadIdx.x;  // kLongThreads == kLongTR: one scale per thread
       if (r < rows) {
@@ -525,7 +526,8 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
       cp_async_commit();
     } else if (threadIdx.x == 0) {
       tc::bar_arrive_expect_tx(&bars[st], static_cast<uint32_t>(S::kStageBytes));
-      tc::tma_load_3d(dst, &kmap, 0, static_cast<int>(base), static_cast<int>(b), &bars[st]);
+      tc::tma_load_3d_stream(dst, &kmap, 0, static_cast<int>(base), static_cast<int>(b), &bars[st],
+                             tc::l2_evict_first_policy());
     }
   };
 
