@@ -137,6 +137,21 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # decode workloads (CSA decode, hybrid CSA + HCA decode)
 # ---------------------------------------------------------------------------
+def packed(torch, tensors, device, pin=False):
+    """One contiguous byte buffer holding copies of `tensors` in 256-byte aligned slots, and the views."""
+    offs, total = [], 0
+    for t in tensors:
+        offs.append(total)
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    buf = torch.empty(total, dtype=torch.uint8, device=device, pin_memory=pin)
+    views = []
+    for t, o in zip(tensors, offs):
+        v = buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        views.append(v)
+    return buf, views
+
+
 class DecodeRun:
     def __init__(self, wl, rank, dev):
         import torch
@@ -168,11 +183,19 @@ class DecodeRun:
             self.ws_hca = torch.empty(max(1, hws), dtype=torch.uint8, device=dev)
             self.hout = torch.empty(B, 1, H, 128, dtype=torch.bfloat16, device=dev)
             self.hlse = torch.empty(B, 1, H, dtype=torch.float32, device=dev)
-        # pinned host buffers for the end-to-end measurement
-        self.h_in = {k: h[k].pin_memory() for k in (["q", "qI", "wI"] + (["hca_q"] if self.hybrid else []))}
-        self.h_out = [torch.empty_like(self.out, device="cpu").pin_memory()]
+        # end-to-end buffers: the per-step inputs (queries, indexer queries and head weights) live in one
+        # device buffer filled by one copy from one pinned host buffer; the outputs likewise
+        keys = ["q", "qI", "wI"] + (["hca_q"] if self.hybrid else [])
+        self.dev_in, views = packed(torch, [d[k] for k in keys], dev)
+        for k_, v in zip(keys, views):
+            d[k_] = v
+        self.host_in, _ = packed(torch, [h[k_] for k_ in keys], "cpu", pin=True)
+        outs = [self.out] + ([self.hout] if self.hybrid else [])
+        self.dev_out, views = packed(torch, outs, dev)
+        self.out = views[0]
         if self.hybrid:
-            self.h_out.append(torch.empty_like(self.hout, device="cpu").pin_memory())
+            self.hout = views[1]
+        self.host_out = torch.empty(self.dev_out.numel(), dtype=torch.uint8, pin_memory=True)
         self.tokens = B
 
     def indexer(self):
@@ -207,17 +230,12 @@ class DecodeRun:
         return out
 
     def e2e_step(self):
-        for k, v in self.h_in.items():
-            self.d[k].copy_(v, non_blocking=True)
+        self.dev_in.copy_(self.host_in, non_blocking=True)
         self.step()
-        self.h_out[0].copy_(self.out, non_blocking=True)
-        if self.hybrid:
-            self.h_out[1].copy_(self.hout, non_blocking=True)
+        self.host_out.copy_(self.dev_out, non_blocking=True)
 
     def e2e_bytes(self):
-        hi = sum(v.numel() * v.element_size() for v in self.h_in.values())
-        ho = sum(v.numel() * v.element_size() for v in self.h_out)
-        return hi, ho
+        return self.host_in.numel(), self.host_out.numel()
 
     def dominant(self):
         """(name, source file, algorithmic bytes per launch, callable that launches it)."""
