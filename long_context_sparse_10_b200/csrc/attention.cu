@@ -524,25 +524,6 @@ __device__ __forceinline__ void bar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Per-head maximum over the 32 lanes of a warp, each lane holding v[0..63]
-// (one key, 64 heads): five halving exchange steps (62 shuffles).  Returns in
-// v[0], v[1] the maxima of heads h0 and h0 + 1, h0 = 2 * bitrev5(lane) laid
-// out as below.
-__device__ __forceinline__ int warp_head_max64(float* v, int lane) {
-#pragma unroll
-  for (int w = 32, o = 16; o >= 1; w >>= 1, o >>= 1) {
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < w; ++i) {
-      const float keep = up ? v[i + w] : v[i];
-      const float send = up ? v[i] : v[i + w];
-      v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
-    }
-  }
-  return ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 + ((lane >> 1) & 1) * 4 +
-         (lane & 1) * 2;
-}
-
 // Per-head maximum over the 32 lanes of a warp, each lane holding v[0..31]
 // (one key, 32 heads): five halving exchange steps (31 shuffles); returns in
 // v[0] the maximum of head bitrev-ordered h0 below.
@@ -1070,7 +1051,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_block_kernel(AttnParams p)
   uint64_t* sdone = full + 4;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(full + 8);
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int H = p.H;
   const int QB = 128 / H;
   const int64_t nblk = (p.Tq + QB - 1) / QB;

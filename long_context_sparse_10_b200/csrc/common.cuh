@@ -76,15 +76,8 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t codes) {
   return pack_bf16x2(f.x, f.y);
 }
 
-// Two E4M3 codes (low byte first) -> two fp16 in one register, exactly (every
-// E4M3 value, subnormals included, is an fp16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes16) {
-  uint32_t r;
-  asm("{\n.reg .b16 c;\ncvt.u16.u32 c, %1;\ncvt.rn.f16x2.e4m3x2 %0, c;\n}\n" : "=r"(r) : "r"(codes16));
-  return r;
-}
-
-// Four E4M3 codes (bytes 0..3) -> fp16 pairs (bytes 0,1) and (bytes 2,3), exactly.
+// Four E4M3 codes (bytes 0..3) -> fp16 pairs (bytes 0,1) and (bytes 2,3),
+// exactly (every E4M3 value, subnormals included, is an fp16 value).
 __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, uint32_t& hi) {
   asm("{\n.reg .b16 l, h;\nmov.b32 {l, h}, %2;\ncvt.rn.f16x2.e4m3x2 %0, l;\ncvt.rn.f16x2.e4m3x2 %1, h;\n}\n"
       : "=r"(lo), "=r"(hi)

@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
   const __nv_bfloat16* kbase = p.kI + b * p.N * kDI;
   auto load_tile = [&](int tile, int stage) {
     const int64_t base = e_begin + static_cast<int64_t>(tile) * TR;
-    if (E4) {
+    if constexpr (E4) {
       // 64 code bytes per entry (4 pieces) and one 4-byte scale per entry
       for (int piece = threadIdx.x; piece < TR * 4; piece += kScoreThreads) {
         const int row = piece >> 2, ch = piece & 3;
@@ -305,17 +305,17 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
           scale_st[stage * TR + row] = 0.f;
         }
       }
-      return;
-    }
+    } else {
 #pragma unroll
-    for (int u = 0; u < (kTileRows * 8) / kScoreThreads; ++u) {
-      const int piece = threadIdx.x + u * kScoreThreads;
-      const int row = piece >> 3, ch = piece & 7;
-      const int64_t e = base + row;
-      const bool ok = e < e_end;
-      const __nv_bfloat16* src = kbase + (ok ? e : e_begin) * kDI + ch * 8;
-      uint8_t* dst = tiles + stage * (kTileRows * 128) + row * 128 + ((ch ^ (row & 7)) << 4);
-      cp_async16(dst, src, ok ? 16 : 0);
+      for (int u = 0; u < (kTileRows * 8) / kScoreThreads; ++u) {
+        const int piece = threadIdx.x + u * kScoreThreads;
+        const int row = piece >> 3, ch = piece & 7;
+        const int64_t e = base + row;
+        const bool ok = e < e_end;
+        const __nv_bfloat16* src = kbase + (ok ? e : e_begin) * kDI + ch * 8;
+        uint8_t* dst = tiles + stage * (kTileRows * 128) + row * 128 + ((ch ^ (row & 7)) << 4);
+        cp_async16(dst, src, ok ? 16 : 0);
+      }
     }
   };
 
@@ -345,8 +345,9 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
         const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t a0 = e4m3x2_to_f16x2(wl[kk] & 0xffffu), a2 = e4m3x2_to_f16x2(wl[kk] >> 16);
-          const uint32_t a1 = e4m3x2_to_f16x2(wh[kk] & 0xffffu), a3 = e4m3x2_to_f16x2(wh[kk] >> 16);
+          uint32_t a0, a1, a2, a3;
+          e4m3x4_to_f16x2x2(wl[kk], a0, a2);
+          e4m3x4_to_f16x2x2(wh[kk], a1, a3);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) mma_f16(acc[nt], a0, a1, a2, a3, bq[kk][nt][0], bq[kk][nt][1]);
         }
@@ -725,7 +726,6 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   uint32_t* bm_s = reinterpret_cast<uint32_t*>(sel_smem + kCandSmem * sizeof(uint2));
   __shared__ uint32_t hist[256];
   __shared__ uint32_t dig[3];
-  __shared__ uint32_t scan_sh[32];
   __shared__ uint32_t n_cand, base_s, last_s;
   const int64_t row = blockIdx.y;
   const int64_t nv = visible(q_pos0 + row % Tq, m, N);
