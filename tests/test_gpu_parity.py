@@ -182,6 +182,7 @@ def _split_cache(g, B, N):
     ("hca", 64, 8, 8192, 0, 128, 1),   # the 1M-context decode's HCA shape: 17 CTAs per row
     ("hca", 64, 2, 30000, 0, 128, 1),  # 59 CTAs per row, last split ragged
     ("csa", 64, 8, 40000, 2048, 128, 1),  # the 1M-context decode's CSA shape (cluster merge)
+    ("hca", 64, 1, 30000, 0, 128, 4),  # several query rows of one sequence, each split over CTAs
 ])
 def test_decode_split_fp8(kind, H, B, N, k, win, Tq):
     g = np.random.default_rng(N + H + k)
@@ -289,6 +290,7 @@ def test_no_device_timeouts_recorded():
     # rescales each head by a power of two before its fp16 MMA)
     (2, 1, 20000, 4 * 20000 - 1, 4, 256, (2.0 ** -40, 2.0 ** 30, 1.0, 2.0 ** -10)),
     (1, 40, 300, 0, 4, 32, (2.0 ** 25, 2.0 ** -35, 0.0, 1.0)),
+    (3, 1, 20001, 4 * 20001 - 1, 4, 4096, None),     # odd N, k at its maximum
 ])
 def test_indexer_topk_e4m3_keys(B, Tq, N, q_pos0, m, k, head_scale):
     g = np.random.default_rng(N + k + 17)
@@ -303,3 +305,20 @@ def test_indexer_topk_e4m3_keys(B, Tq, N, q_pos0, m, k, head_scale):
     s = R.indexer_scores(f64(qI), f64(wI), kI, q_pos0 + np.arange(Tq), m)
     same = check_topk(idx.cpu().numpy(), s, R.topk_set(s, k), k, "indexer e4m3")
     assert same.mean() > 0.97
+
+
+def test_empty_calls_return_without_work():
+    """No query rows (Tq = 0): the calls return empty outputs and launch nothing."""
+    lib = csa._lib.load()
+    before = lib.csa_launch_count()
+    q = torch.empty(1, 0, 64, 192, dtype=torch.bfloat16, device=DEV)
+    nope = torch.zeros(1, 4, 128, dtype=torch.uint8, device=DEV)
+    rope = torch.zeros(1, 4, 64, dtype=torch.bfloat16, device=DEV)
+    scale = torch.ones(1, 4, dtype=torch.float32, device=DEV)
+    out, lse = csa.hca_dense_mqa(q, csa.KVCache(nope=nope, rope=rope, scale=scale), 128, None, 0.1)
+    idx = csa.csa_indexer_topk(torch.empty(2, 0, 4, 64, dtype=torch.bfloat16, device=DEV),
+                               torch.empty(2, 0, 4, device=DEV), torch.zeros(2, 8, 64, dtype=torch.bfloat16, device=DEV),
+                               4, 4)
+    torch.cuda.synchronize()
+    assert out.numel() == 0 and lse.numel() == 0 and idx.shape == (2, 0, 4)
+    assert lib.csa_launch_count() == before
