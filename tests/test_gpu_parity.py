@@ -102,6 +102,7 @@ def _indexer_case(g, B, Tq, N, tie_blocks=0, zero_q=False):
     (2, 2, 70, 100, 4, 40, 0, False),          # every row sees fewer than k entries
     (1, 40, 300, 0, 4, 8, 0, False),           # long-row path; the first rows see no entry at all
     (1, 1, 40000, 4 * 40000 - 1, 4, 4096, 0, True),   # long rows, all ties, k = max
+    (2, 1, 300001, 4 * 300001 - 1, 4, 2048, 0, False),  # rows past 262144 entries: bitmap in global memory
 ])
 def test_indexer_topk(B, Tq, N, q_pos0, m, k, ties, zero):
     g = np.random.default_rng(B * 1000 + N + k)
