@@ -323,3 +323,34 @@ def test_empty_calls_return_without_work():
     torch.cuda.synchronize()
     assert out.numel() == 0 and lse.numel() == 0 and idx.shape == (2, 0, 4)
     assert lib.csa_launch_count() == before
+
+
+@pytest.mark.parametrize("kind", ["csa", "hca"])
+def test_decode_split_fp8_separate_window_values(kind):
+    """FP8 cache with a raw window that carries its own values (the warp-MMA kernel's case)."""
+    g = np.random.default_rng(41)
+    H, B, N, win = 64, 2, 2000, 128
+    m = 4 if kind == "csa" else 128
+    k = 256
+    L = N * m
+    q_pos0 = L - 1
+    nope, rope, scale = _split_cache(g, B, N)
+    q = _bf16(g, (B, 1, H, 192))
+    Wk = _bf16(g, (B, win + 1, 192))
+    Wv = _bf16(g, (B, win + 1, 128))
+    wpos0 = L - 1 - win
+    cache = csa.KVCache(nope=nope.to(DEV), rope=rope.to(DEV), scale=scale.to(DEV))
+    w = csa.Window(k=Wk.to(DEV), v=Wv.to(DEV), pos0=wpos0, length=win)
+    sc = 1 / math.sqrt(192)
+    K64, V64 = R.dequant_split(nope.numpy(), f64(rope), scale.numpy())
+    if kind == "csa":
+        idx = _oracle_idx(g, B, 1, N, m, k, q_pos0)
+        out, lse = csa.csa_sparse_mqa(q.to(DEV), cache, m, torch.from_numpy(idx.astype(np.int32)).to(DEV), w, sc,
+                                      q_pos0=q_pos0)
+        O, Ls = R.csa_sparse_mqa(f64(q), q_pos0 + np.arange(1), K64, V64, idx, m, f64(Wk), f64(Wv), wpos0, win, sc)
+    else:
+        out, lse = csa.hca_dense_mqa(q.to(DEV), cache, m, w, sc, q_pos0=q_pos0)
+        O, Ls = R.hca_dense_mqa(f64(q), q_pos0 + np.arange(1), K64, V64, m, f64(Wk), f64(Wv), wpos0, win, sc)
+    torch.cuda.synchronize()
+    assert_close(f64(out), O, f"{kind} decode fp8, separate window V")
+    assert_lse(f64(lse), Ls, f"{kind} decode lse, separate window V")
