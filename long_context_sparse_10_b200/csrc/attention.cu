@@ -453,9 +453,10 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
 //   l^T += 1 P^T    M = 128 (all rows equal), N = 64 heads        (8 MMAs)
 // all at M = 128, with fp32 accumulators in tensor memory: S^T double-buffered
 // in columns [0, 128), O^T in [128, 192), the running sums l in [192, 256).
-// Softmax thread t (warps 0-3) owns TMEM lane t, i.e. key t of the tile: it
-// reads its 64 head logits, and writes its row of P^T (128 bytes, the B
-// operand's MN-major layout) to shared memory.  The running max per head
+// Softmax warps 0-7: thread (warp w, lane l) owns TMEM lane 32 (w % 4) + l,
+// i.e. that key of the tile, and heads 32 (w / 4) .. +31: it reads those
+// logits and writes its half of the key's P^T row (the row is 128 bytes, the
+// B operand's MN-major layout) to shared memory.  The running max per head
 // (m_ref, shared memory) changes only when some logit exceeds it by more
 // than 2^20 (log2 units) -- always on a CTA's first tile, rarely after; then
 // the tile's per-head maxima are reduced across the 128 keys (a halving
@@ -464,9 +465,9 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
 // (three 64-dim blocks), Q K-major, V^T read MN-major straight out of the
 // first two K blocks when key and value are shared, P^T MN-major, and the
 // all-ones A operand of the l update is one 1 KB swizzle atom read with a
-// zero row-group stride.  Warps 4-7 gather and widen key tiles (FP8 entries
+// zero row-group stride.  Warps 8-15 gather and widen key tiles (FP8 entries
 // dequantised, code x scale rounded to bf16, from registers into the K
-// tile); one thread of warp 8 issues every MMA in the order S(0), S(1), then
+// tile); one thread of warp 16 issues every MMA in the order S(0), S(1), then
 // per tile t: PV(t) and the l update once P(t) is written, S(t+2) into the
 // TMEM buffer P(t)'s softmax has drained.  When key and value are shared the
 // K tile has three stages (two with a separate V tile).  Every mbarrier wait
