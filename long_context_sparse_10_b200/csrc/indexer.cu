@@ -8,9 +8,11 @@
 // an ascending list (-1 padded when fewer than k entries are visible).
 //
 // Scoring is a skinny GEMM (entries x (rows*4 heads) x 64) that streams kIc
-// from HBM: 16-byte cp.async copies into a 128-byte XOR-swizzled shared tile
-// (4-stage pipeline), ldmatrix + bf16 tensor-core MMA (fp32 accumulate), and
-// the relu/weight reduction over the 4 heads in registers.  Selection is an
+// from HBM into 128-byte XOR-swizzled shared tiles -- by TMA with an L2
+// evict-first policy for long rows (score_long_kernel), by 16-byte cp.async
+// copies for prefill rows (score_kernel) -- then ldmatrix + bf16 tensor-core
+// MMA (fp32 accumulate) and the relu/weight reduction over the 4 heads in
+// registers; E4M3 keys are widened to fp16 in registers.  Selection is an
 // exact radix select on an order-preserving key of the fp32 score extended by
 // the inverted entry index, so ties resolve to the lower index by construction:
 //   * rows whose visible prefix fits in shared memory (prefill) run one CTA
