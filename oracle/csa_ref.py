@@ -192,14 +192,6 @@ def topk_set(s: np.ndarray, k: int) -> np.ndarray:
     return out.reshape(*lead, k)
 
 
-def kth_gap(s_row: np.ndarray, k: int):
-    """(k-th, (k+1)-th) best visible score of one row (None where absent)."""
-    v = np.sort(s_row[np.isfinite(s_row)])[::-1]
-    a = v[k - 1] if len(v) >= k else None
-    b = v[k] if len(v) > k else None
-    return a, b
-
-
 # ----------------------------------------------------------------------------
 # core attention: MQA over entries + sliding window, one joint softmax (R5, R6, R11)
 # ----------------------------------------------------------------------------
