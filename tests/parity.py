@@ -59,6 +59,11 @@ def check_topk(got_idx: np.ndarray, scores: np.ndarray, ref_idx: np.ndarray, k: 
     """Checks GPU index lists against the oracle; returns a bool mask of rows with identical sets.
 
     got_idx, ref_idx: [..., k]; scores: oracle float64 scores [..., N] (-inf = not visible).
+    A row may differ from the oracle's only where its k-th and (k+1)-th best
+    scores lie within the tie band; there the GPU list must still be a top-k of
+    the oracle's scores up to that band: k distinct visible entries in ascending
+    order, none scoring below s_k - band, and every entry scoring above
+    s_k + band among them.
     """
     got = np.asarray(got_idx).reshape(-1, k)
     ref = np.asarray(ref_idx).reshape(-1, k)
@@ -76,7 +81,11 @@ def check_topk(got_idx: np.ndarray, scores: np.ndarray, ref_idx: np.ndarray, k: 
             f"{what}: row {r} differs outside the tie band (s_k={sk}, s_k+1={sk1}); "
             f"extra={sorted(set(got[r]) - set(ref[r]))[:8]} missing={sorted(set(ref[r]) - set(got[r]))[:8]}")
         g = got[r]
+        assert np.all(g >= 0) and np.all(g < row.shape[0]), f"{what}: row {r} has padding or out-of-range ids"
         assert np.all(np.diff(g) > 0), f"{what}: row {r} not ascending/unique"
         assert np.all(vis[g]), f"{what}: row {r} selects an invisible entry"
         assert row[g].min() >= sk - band, f"{what}: row {r} selects an entry below the band"
+        must = np.flatnonzero(vis & (row > sk + band))
+        missing = np.setdiff1d(must, g)
+        assert missing.size == 0, f"{what}: row {r} drops entries above the band: {missing[:8].tolist()}"
     return same
