@@ -22,7 +22,6 @@ import hashlib
 import json
 import math
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -31,6 +30,7 @@ import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
+sys.path.insert(1, os.path.join(ROOT, "tests"))  # parity.py: the comparison rules of the GPU tests
 
 METRIC = "CSA/HCA attention tokens/s at 128K and 1M ctx; % of HBM / tensor-core peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -61,16 +61,18 @@ def peaks():
 
 
 def profile_traffic(kernel: str, source: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was captured on this workload and the
-    kernel source has not changed since."""
-    path = os.path.join(ROOT, "profiles", "ncu_traffic.md")
+    """DRAM bytes per launch from the committed ncu data table (profiles/ncu_traffic.tsv), if it was captured on
+    this workload and the kernel source has not changed since."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.tsv")
     if not os.path.exists(path):
         return None
     sha = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
     for line in open(path):
-        m = re.match(r"\|\s*(\S+)\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]+)\s*\|\s*([A-Za-z0-9_]+)", line)
-        if m and m.group(1) == kernel and m.group(3) == sha and m.group(4) == workload:
-            return float(m.group(2))
+        if line.startswith("#") or not line.strip():
+            continue
+        f = line.rstrip("\n").split("\t")
+        if len(f) >= 4 and f[0] == kernel and f[2] == sha and f[3] == workload:
+            return float(f[1])
     return None
 
 
@@ -313,41 +315,69 @@ class DecodeRun:
                       "MB/step > 126 MB L2)",
                 "timing": "CUDA graph replay of the whole step"}
 
-    def oracle_sample(self, budget_s):
-        """Time the float64 oracle on whole sequences of this workload (host cores)."""
+    def _oracle_seq(self, b):
+        """Float64 oracle of sequence b's whole decode step: (scores, idx, csa (O, lse), hca (O, lse) or None)."""
         import numpy as np
         from oracle import csa_ref as R
         h, wl = self.host, self.wl
+        qI = h["qI"][b:b + 1].double().numpy()
+        wI = h["wI"][b:b + 1].double().numpy()
+        if wl.indexer_fp8:
+            kI = R.e4m3_decode(h["kI_codes"][b:b + 1].numpy()) * h["kI_scale"][b:b + 1].double().numpy()[..., None]
+        else:
+            kI = h["kIc"][b:b + 1].double().numpy()
+        q = h["q"][b:b + 1].double().numpy()
+        wk = h["win_k"][b:b + 1].double().numpy()
+        nope, rope, sc = h["nope"][b:b + 1].numpy(), h["rope"][b:b + 1].double().numpy(), h["scale"][b:b + 1].numpy()
+        pos = np.array([wl.L - 1])
+        s = R.indexer_scores(qI, wI, kI, pos, wl.m)
+        idx = R.topk_set(s, wl.k)
+        K, V = R.dequant_split(nope, rope, sc)
+        csa_out = R.csa_sparse_mqa(q, pos, K, V, idx, wl.m, wk, wk[..., :128], wl.L - wl.win, wl.win, self.scale)
+        hca_out = None
+        if self.hybrid:
+            hq = h["hca_q"][b:b + 1].double().numpy()
+            hwk = h["hca_win_k"][b:b + 1].double().numpy()
+            HK, HV = R.dequant_split(h["hca_nope"][b:b + 1].numpy(), h["hca_rope"][b:b + 1].double().numpy(),
+                                     h["hca_scale"][b:b + 1].numpy())
+            hca_out = R.hca_dense_mqa(hq, pos, HK, HV, wl.m_hca, hwk, hwk[..., :128], wl.L - wl.win, wl.win,
+                                      self.scale)
+        return s, idx, csa_out, hca_out, (q, pos, K, V, wk)
+
+    def self_check(self):
+        """Sequence 0 of the last step against the float64 oracle (parity rules of the GPU tests)."""
+        import numpy as np
+        from oracle import csa_ref as R
+        from parity import assert_close, assert_lse, check_topk
+        torch, wl = self.torch, self.wl
+        torch.cuda.synchronize()
+        got_idx = self.idx[0:1].cpu().numpy()
+        got_o, got_l = self.out[0:1].double().cpu().numpy(), self.lse[0:1].double().cpu().numpy()
+        s, idx, (O, L), hca, (q, pos, K, V, wk) = self._oracle_seq(0)
+        same = check_topk(got_idx, s, idx, wl.k, "bench self-check: indexer")
+        if not same.all():  # tie-band row: attention is compared on the GPU's own selection
+            O, L = R.csa_sparse_mqa(q, pos, K, V, got_idx.astype(np.int64), wl.m, wk, wk[..., :128], wl.L - wl.win,
+                                    wl.win, self.scale)
+        ma, rl = assert_close(got_o, O, "bench self-check: csa attention")
+        assert_lse(got_l, L, "bench self-check: csa lse")
+        res = {"rows": 1, "topk_identical": float(same.mean()), "max_abs": ma, "rel_l2": rl}
+        if hca is not None:
+            hma, hrl = assert_close(self.hout[0:1].double().cpu().numpy(), hca[0], "bench self-check: hca attention")
+            assert_lse(self.hlse[0:1].double().cpu().numpy(), hca[1], "bench self-check: hca lse")
+            res.update(hca_max_abs=hma, hca_rel_l2=hrl)
+        return res
+
+    def oracle_sample(self, budget_s):
+        """Time the float64 oracle on whole sequences of this workload (host cores)."""
         done, spent = 0, 0.0
-        for b in range(wl.B):
-            qI = h["qI"][b:b + 1].double().numpy()
-            wI = h["wI"][b:b + 1].double().numpy()
-            if wl.indexer_fp8:
-                kI = R.e4m3_decode(h["kI_codes"][b:b + 1].numpy()) * h["kI_scale"][b:b + 1].double().numpy()[..., None]
-            else:
-                kI = h["kIc"][b:b + 1].double().numpy()
-            q = h["q"][b:b + 1].double().numpy()
-            wk = h["win_k"][b:b + 1].double().numpy()
-            nope, rope, sc = h["nope"][b:b + 1].numpy(), h["rope"][b:b + 1].double().numpy(), h["scale"][b:b + 1].numpy()
-            if self.hybrid:
-                hq = h["hca_q"][b:b + 1].double().numpy()
-                hwk = h["hca_win_k"][b:b + 1].double().numpy()
-                hn, hr, hs = (h["hca_nope"][b:b + 1].numpy(), h["hca_rope"][b:b + 1].double().numpy(),
-                              h["hca_scale"][b:b + 1].numpy())
-            pos = np.array([wl.L - 1])
+        for b in range(self.wl.B):
             t0 = time.perf_counter()
-            s = R.indexer_scores(qI, wI, kI, pos, wl.m)
-            idx = R.topk_set(s, wl.k)
-            K, V = R.dequant_split(nope, rope, sc)
-            R.csa_sparse_mqa(q, pos, K, V, idx, wl.m, wk, wk[..., :128], wl.L - wl.win, wl.win, self.scale)
-            if self.hybrid:
-                HK, HV = R.dequant_split(hn, hr, hs)
-                R.hca_dense_mqa(hq, pos, HK, HV, wl.m_hca, hwk, hwk[..., :128], wl.L - wl.win, wl.win, self.scale)
+            self._oracle_seq(b)
             spent += time.perf_counter() - t0
             done += 1
             if spent >= budget_s:
                 break
-        return done, spent, f"{done} of {wl.B} sequences of one rank's batch, whole decode step each"
+        return done, spent, f"{done} of {self.wl.B} sequences of one rank's batch, whole decode step each"
 
 
 # ---------------------------------------------------------------------------
@@ -440,6 +470,45 @@ class PrefillRun:
         return {"workload": s, "global_batch": wl.B * world, "seq_len": wl.T, "parallelism": f"dp{world} (replicas)",
                 "l2": "inputs larger than L2" if wl.T * wl.H * 384 * wl.B > 126e6 else "inputs fit in L2",
                 "timing": "CUDA graph replay of the whole step"}
+
+    def self_check(self):
+        """Sampled query rows of sequence 0 of the last step against the float64 oracle: rows before the window
+        fills and before top-k selection becomes partial, and a stride over the rest."""
+        import numpy as np
+        from oracle import csa_ref as R
+        from parity import assert_close, assert_lse, check_topk
+        torch, wl, h = self.torch, self.wl, self.host
+        torch.cuda.synchronize()
+        cw = 2 * wl.m if self.csa_kind else wl.m
+
+        def bf16_cache(x, w, b):   # the oracle's entries, stored as bf16 like the GPU cache
+            y = R.compress(x[:1].double().numpy(), w.double().numpy(), b.double().numpy(), wl.m, cw)
+            return torch.from_numpy(y.astype(np.float32)).to(torch.bfloat16).double().numpy()
+
+        Kc, Vc = bf16_cache(h["k"], h["w_k"], h["b_k"]), bf16_cache(h["v"], h["w_v"], h["b_v"])
+        res = {}
+        ma, _ = assert_close(self.Kc[0:1].double().cpu().numpy(), Kc, "bench self-check: compressed K", max_abs=1.6e-2)
+        T = wl.T
+        rows = np.unique(np.concatenate([np.arange(0, min(T, 40), 3), np.linspace(0, T - 1, 24).astype(np.int64),
+                                         [T - 1]]))
+        q = h["q"][:1, rows].double().numpy()
+        K, V = h["k"][:1].double().numpy(), h["v"][:1].double().numpy()
+        if self.csa_kind:
+            kIc = bf16_cache(h["kI"], h["w_i"], h["b_i"])
+            s = R.indexer_scores(h["qI"][:1, rows].double().numpy(), h["wI"][:1, rows].double().numpy(), kIc, rows,
+                                 wl.m)
+            idx = R.topk_set(s, wl.k)
+            got_idx = self.idx[0:1, rows].cpu().numpy()
+            same = check_topk(got_idx, s, idx, wl.k, "bench self-check: indexer")
+            use = np.where(same[None, :, None], idx, got_idx.astype(np.int64))
+            O, L = R.csa_sparse_mqa(q, rows, Kc, Vc, use, wl.m, K, V, 0, wl.win, self.scale)
+            res["topk_identical"] = float(same.mean())
+        else:
+            O, L = R.hca_dense_mqa(q, rows, Kc, Vc, wl.m, K, V, 0, wl.win, self.scale)
+        ma, rl = assert_close(self.out[0:1, rows].double().cpu().numpy(), O, "bench self-check: attention")
+        assert_lse(self.lse[0:1, rows].double().cpu().numpy(), L, "bench self-check: lse")
+        res.update(rows=int(len(rows)), max_abs=ma, rel_l2=rl)
+        return res
 
     def oracle_sample(self, budget_s):
         import numpy as np
@@ -539,10 +608,19 @@ def main():
     if args.impl == "reference":
         reference_arm(args)
         return
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one rank per GPU: relaunch this command under torchrun with --gpus ranks
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr", "127.0.0.1", "--master-port", str(29500 + os.getpid() % 1000), os.path.abspath(__file__),
+               *sys.argv[1:]]
+        sys.exit(subprocess.call(cmd))
     import torch
     import torch.distributed as dist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but the launcher started {world} rank(s)", file=sys.stderr)
+        sys.exit(2)
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
@@ -568,6 +646,22 @@ def main():
             run.step()
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
+    # the outputs of the last warm-up step against the oracle (rank 0): no line is printed for a wrong result
+    check, ok = None, 1
+    if rank == 0:
+        try:
+            check = run.self_check()
+        except AssertionError as exc:
+            print(f"bench.py: self-check against the oracle failed: {exc}", file=sys.stderr)
+            ok = 0
+    if world > 1:
+        flag = torch.tensor([ok], dtype=torch.int32, device=dev)
+        dist.all_reduce(flag, op=dist.ReduceOp.MIN)
+        ok = int(flag.item())
+    if not ok:
+        if world > 1:
+            dist.destroy_process_group()
+        sys.exit(3)
     graph = torch.cuda.CUDAGraph()
     n0 = csa.launch_count()
     with torch.cuda.graph(graph):
@@ -694,7 +788,7 @@ def main():
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": run.describe(world), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(),
-                "library": csa.version()}
+                "self_check": check, "library": csa.version()}
         print(json.dumps(line), flush=True)
     del graph
     if world > 1:

@@ -116,6 +116,18 @@ CSA_API const char* csa_last_error(void);
 CSA_API csa_status csa_check_device_error(void* stream);
 
 /*
+ * csa_debug_expire_wait -- failure-detection check (library infrastructure,
+ * not part of the method).  Enqueues one small kernel on `stream` whose single
+ * bounded wait -- the same wait the attention and indexer kernels use on their
+ * barriers -- is on a barrier nothing ever arrives at, so it runs out (2^14
+ * rounds) and records a timeout.  The next csa_check_device_error on that
+ * stream then returns CSA_ERR_DEVICE_TIMEOUT and clears the record; the
+ * context stays usable.  Nothing faults, traps or hangs.  Returns CSA_OK or
+ * CSA_ERR_CUDA (launch failure).
+ */
+CSA_API csa_status csa_debug_expire_wait(void* stream);
+
+/*
  * csa_launch_count -- number of kernels this library has enqueued in this
  * process so far (library infrastructure, not part of the method).  Every
  * successful kernel launch counts once, including one recorded into a CUDA
@@ -181,7 +193,7 @@ CSA_API size_t csa_indexer_topk_workspace_size(int64_t B, int64_t Tq, int64_t N,
  * k entries are visible.
  *   qI  bf16 [B, Tq, 4, 64];  wI fp32 [B, Tq, 4];  kIc bf16 [B, N, 64]
  *   idx int32 [B, Tq, k] (output)
- *   1 <= k <= 4096, 1 <= m, q_pos0 >= 0, N < 2^31.
+ *   1 <= k <= 4096, 1 <= m, 0 <= q_pos0 < 2^50, N < 2^31, B * Tq < 2^31.
  */
 CSA_API csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc,
                             int64_t B, int64_t Tq, int64_t N, int64_t q_pos0, int32_t m,
@@ -213,9 +225,10 @@ CSA_API csa_status csa_indexer_topk_e4m3(const void* qI, const float* wI, const 
  * the library until the process exits.  Sizes whose workspace
  * (csa_indexer_topk_workspace_size) exceeds 32 MiB are rejected with
  * CSA_ERR_UNSUPPORTED and a message; e.g. 8 decode rows over 262,144 entries
- * fit.  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current and caches it; make that
- * first call before any stream capture.  No call allocates.  Every call
+ * fit.  Every call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress, which allocates nothing); the first call on a device
+ * may also load the library's device code there, so make it before any
+ * stream capture.  No call allocates.  Every call
  * shares the array and it keeps the last call's contents (the call clears what
  * must start at zero), so calls that overlap on the GPU race on it.  Other
  * arguments, outputs and errors as csa_indexer_topk.

@@ -21,6 +21,7 @@ SIGNATURES = {
     "csa_launch_count": (ctypes.c_uint64, []),
     "csa_profile_next_call": (c_i32, [c_vp, c_vp]),
     "csa_check_device_error": (c_i32, [c_vp]),
+    "csa_debug_expire_wait": (c_i32, [c_vp]),
     "csa_compress": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "hca_compress": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "csa_indexer_topk_workspace_size": (c_sz, [c_i64, c_i64, c_i64, c_i32]),

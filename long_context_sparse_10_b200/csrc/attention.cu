@@ -22,10 +22,12 @@
 // side, so no rounding is added to cache values.  QK^T and PV are bf16
 // tensor-core MMAs (fp32 accumulate) with an online softmax in the exp2 domain.
 //
-// Rows that are few (decode) split their tiles over a thread-block cluster of
-// up to 16 CTAs; the partial softmax states (m, l, O) are merged through
-// distributed shared memory inside the cluster, so there is no global
-// scratch and no second launch.
+// Rows that are few (decode) split their tiles over several CTAs, merged in
+// one of two ways: a thread-block cluster of up to 16 CTAs whose partial
+// softmax states (m, l, O) meet in distributed shared memory (no global
+// scratch, no second launch), or, on the tcgen05 path when that leaves fewer
+// tiles per CTA, one CTA per split writing 16-byte partial records to the
+// caller's workspace, combined by attn_merge_kernel.
 #include <cooperative_groups.h>
 
 #include <map>
@@ -1331,6 +1333,22 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict
 }
 
 // ---------------------------------------------------------------------------
+// Expiring wait (failure-detection check): one thread waits, through the same
+// bounded wait every kernel of the library uses, on an mbarrier that nothing
+// arrives at.  The wait runs out after `limit` rounds and records the timeout
+// in this unit's error word.  No copy, MMA or TMEM allocation is involved.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) wait_expire_kernel(uint32_t limit) {
+  pdl_wait();
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    tc::bar_init(&bar, 1);
+    tc::bar_init_fence();
+    tc::bar_wait_bounded(&bar, 0, limit);  // phase 0 never completes: no arrival
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 // Splits of a row's slots for the tcgen05 kernel (one CTA per SM): rows that
@@ -1468,9 +1486,13 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   CSA_REQUIRE(q_pos0 >= 0, "%s: q_pos0 must be >= 0", name);
   CSA_REQUIRE(scale == scale && scale > -3.0e38f && scale < 3.0e38f, "%s: scale must be finite", name);
   if (csa_status st = check_cache(name, cache); st != CSA_OK) return st;
+  CSA_REQUIRE(q_pos0 < (int64_t(1) << 50), "%s: q_pos0 must be below 2^50", name);
+  // bound both factors before multiplying so that B * Tq cannot overflow
+  constexpr int64_t kRowLim = (int64_t(1) << 31) / kMaxCluster;
+  CSA_REQUIRE(B < kRowLim && Tq < kRowLim && (Tq == 0 || B <= (kRowLim - 1) / Tq), "%s: too many query rows",
+              name);
   const int64_t R = B * Tq;
   if (R == 0) return CSA_OK;
-  CSA_REQUIRE(R < (1LL << 31) / kMaxCluster, "%s: too many query rows", name);
   CSA_REQUIRE_PTR(q);
   CSA_REQUIRE_PTR(out);
   CSA_REQUIRE(lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u) == 0, "%s: lse misaligned", name);
@@ -1644,13 +1666,24 @@ csa_status csa_check_device_error(void* stream) {
   return CSA_OK;
 }
 
+csa_status csa_debug_expire_wait(void* stream) {
+  csa::clear_error();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return csa::check_launch("csa_debug_expire_wait",
+                           csa::launch_pdl(csa::wait_expire_kernel, dim3(1), dim3(32), 0, s, 1, uint32_t(1) << 14));
+}
+
 size_t csa_sparse_mqa_workspace_size(int64_t B, int64_t Tq, int32_t H, int32_t k, int32_t win_len) {
-  if (B <= 0 || Tq <= 0 || k < 0 || win_len < 0) return 0;
+  if (B <= 0 || Tq <= 0 || k < 0 || win_len < 0 || B >= (1LL << 31) || Tq >= (1LL << 31) ||
+      B > ((1LL << 31) - 1) / Tq)
+    return 0;
   return csa::tc_part_bytes(B * Tq, H, static_cast<int64_t>(k) + win_len);
 }
 
 size_t hca_dense_mqa_workspace_size(int64_t B, int64_t Tq, int32_t H, int64_t N, int32_t win_len) {
-  if (B <= 0 || Tq <= 0 || N < 0 || win_len < 0) return 0;
+  if (B <= 0 || Tq <= 0 || N < 0 || N >= (1LL << 31) || win_len < 0 || B >= (1LL << 31) || Tq >= (1LL << 31) ||
+      B > ((1LL << 31) - 1) / Tq)
+    return 0;
   return csa::tc_part_bytes(B * Tq, H, N + win_len);
 }
 

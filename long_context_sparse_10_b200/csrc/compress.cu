@@ -205,7 +205,8 @@ csa_status compress_impl(const char* name, const void* x, int64_t B, int64_t T, 
                          int32_t cwin, const float* w, const float* b_pos, int32_t layout, void* out,
                          void* out_rope, float* out_scale, void* stream) {
   clear_error();
-  CSA_REQUIRE(B >= 0 && T >= 0, "%s: B and T must be >= 0", name);
+  CSA_REQUIRE(B >= 0 && T >= 0 && B < (1LL << 31) && T < (1LL << 40), "%s: B must be in [0, 2^31), T in [0, 2^40)",
+              name);
   CSA_REQUIRE(d >= 8 && d <= 256 && d % 8 == 0, "%s: d must be a multiple of 8 in [8, 256] (got %d)", name, d);
   CSA_REQUIRE(layout == CSA_KV_BF16 || layout == CSA_KV_SPLIT_FP8, "%s: unknown out_layout %d", name, layout);
   if (layout == CSA_KV_SPLIT_FP8 && d != kDQK)
@@ -235,8 +236,8 @@ csa_status compress_impl(const char* name, const void* x, int64_t B, int64_t T, 
   p.out_rope = static_cast<__nv_bfloat16*>(out_rope);
   p.out_scale = out_scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CSA_REQUIRE(p.N < (1LL << 31) && B <= ((1LL << 31) - 1) / p.N, "%s: too many entries", name);
   const int64_t entries = B * p.N;
-  CSA_REQUIRE(entries < (1LL << 31), "%s: too many entries", name);
   prof_begin(s);
   const cudaError_t e =
       cwin <= 32 ? launch_pdl(compress_short_kernel, dim3(static_cast<unsigned>((entries + 7) / 8)), dim3(256), 0, s, 1, p)

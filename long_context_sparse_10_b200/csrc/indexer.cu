@@ -543,11 +543,18 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
       cp_async_commit();
     }
   }
-  for (int tile = 0; tile < ntiles; ++tile) {
+  // A stage wait that runs out (recorded in the device error word) ends the
+  // loop for the whole CTA: no further loads are issued, and the stages still
+  // in flight are waited for (again with a bound) before the CTA moves on.
+  bool healthy = true;
+  int tile = 0;
+  for (; tile < ntiles; ++tile) {
     const int st = tile % S::kStages;
-    tc::bar_wait(&bars[st], static_cast<uint32_t>((tile / S::kStages) & 1));
+    const bool ok = tc::bar_wait(&bars[st], static_cast<uint32_t>((tile / S::kStages) & 1));
     if (E4) cp_async_wait<S::kStages - 2>();
-    __syncthreads();  // every warp is done with the stage refilled next; scales visible
+    // every warp is done with the stage refilled next; scales visible
+    healthy = __syncthreads_and(ok) != 0;
+    if (!healthy) break;
     {
       const int nxt = tile + S::kStages - 1;
       if (nxt < ntiles) {
@@ -608,6 +615,12 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
       const uint32_t bin = f2key(score) >> 20;
       atomicAdd(&hist_s[bin >> 1], 1u << ((bin & 1u) * 16));
     }
+  }
+  if (!healthy && threadIdx.x == 0) {
+    // stages of tiles [tile, min(ntiles, tile + kStages - 1)) were issued and not consumed
+    const int issued_end = (tile + S::kStages - 1) < ntiles ? (tile + S::kStages - 1) : ntiles;
+    for (int d = tile; d < issued_end; ++d)
+      tc::bar_wait(&bars[d % S::kStages], static_cast<uint32_t>((d / S::kStages) & 1));
   }
   if (E4) cp_async_wait<0>();
   pdl_trigger();  // the next kernel may be scheduled while the histograms merge
@@ -1017,9 +1030,18 @@ LongLayout long_layout(int64_t R, int64_t N) {
   return L;
 }
 
+// Query rows B * Tq, or -1 when B or Tq is negative or the product is not
+// below 2^31 (checked before multiplying, so it cannot overflow).
+int64_t query_rows(int64_t B, int64_t Tq) {
+  constexpr int64_t kLim = int64_t(1) << 31;
+  if (B < 0 || Tq < 0 || B >= kLim || Tq >= kLim) return -1;
+  if (Tq > 0 && B > (kLim - 1) / Tq) return -1;
+  return B * Tq;
+}
+
 size_t workspace_bytes(int64_t B, int64_t Tq, int64_t N) {
-  const int64_t R = B * Tq;
-  if (R <= 0 || N <= 0) return 0;
+  const int64_t R = query_rows(B, Tq);
+  if (R <= 0 || N <= 0 || N >= (int64_t(1) << 31)) return 0;
   if (use_row_path(R, N)) return align_up(static_cast<size_t>(R) * N * 4);
   return long_layout(R, N).total;
 }
@@ -1061,10 +1083,10 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   CSA_REQUIRE(N < (1LL << 31), "csa_indexer_topk: N must be < 2^31");
   CSA_REQUIRE(m >= 1, "csa_indexer_topk: m must be >= 1");
   CSA_REQUIRE(k >= 1 && k <= kMaxK, "csa_indexer_topk: k must be in [1, %d] (got %d)", kMaxK, k);
-  CSA_REQUIRE(q_pos0 >= 0, "csa_indexer_topk: q_pos0 must be >= 0");
-  const int64_t R = B * Tq;
+  CSA_REQUIRE(q_pos0 >= 0 && q_pos0 < (int64_t(1) << 50), "csa_indexer_topk: q_pos0 must be in [0, 2^50)");
+  const int64_t R = query_rows(B, Tq);
+  CSA_REQUIRE(R >= 0, "csa_indexer_topk: B * Tq must be below 2^31");
   if (R == 0) return CSA_OK;
-  CSA_REQUIRE(R < (1LL << 31), "csa_indexer_topk: too many query rows");
   CSA_REQUIRE_PTR(idx);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (N == 0) {
@@ -1228,10 +1250,11 @@ csa_status csa_indexer_topk_e4m3(const void* qI, const float* wI, const uint8_t*
 // workspace: it uses a file-scope static device array of
 // kStaticScratchBytes (32 MiB), which every GPU that loads the library holds
 // until the process exits.  Host code cannot hand the array's name to a kernel
-// (on the host it is only a stand-in for the symbol), so the first call on
-// each device looks up the array's device address with cudaGetSymbolAddress
-// while that device is current and caches it; that first call should come
-// before any stream capture.  The call itself allocates nothing: it forwards
+// (on the host it is only a stand-in for the symbol), so every call looks up
+// the array's device address with cudaGetSymbolAddress on the current device;
+// the first call on a device may also load the library's device code there,
+// so make that first call before any stream capture.  The call itself
+// allocates nothing: it forwards
 // to csa_indexer_topk with the cached address as the workspace, and that path
 // clears the parts of the scratch that must start at zero on every call.  All
 // calls share the one array and it keeps the last call's contents, so calls
@@ -1240,14 +1263,14 @@ csa_status csa_indexer_topk_e4m3(const void* qI, const float* wI, const uint8_t*
 // ---------------------------------------------------------------------------
 static constexpr size_t kStaticScratchBytes = static_cast<size_t>(32) << 20;
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
-static std::mutex g_static_mu;
-static void* g_static_ptr[64] = {nullptr};
 
 extern "C" csa_status csa_indexer_topk_noalloc(const void* qI, const float* wI, const void* kIc, int64_t B,
                                                int64_t Tq, int64_t N, int64_t q_pos0, int32_t m, int32_t k,
                                                int32_t* idx, void* stream) {
   using namespace csa;
   if (B < 0 || Tq < 0 || N < 0) return fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk_noalloc: negative size");
+  if (query_rows(B, Tq) < 0 || N >= (int64_t(1) << 31))
+    return fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk_noalloc: B * Tq and N must be below 2^31");
   const size_t need = csa::workspace_bytes(B, Tq, N);
   if (need > kStaticScratchBytes)
     return fail(CSA_ERR_UNSUPPORTED,
@@ -1256,18 +1279,11 @@ extern "C" csa_status csa_indexer_topk_noalloc(const void* qI, const float* wI, 
                 need, kStaticScratchBytes);
   void* ptr = nullptr;
   if (need > 0) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-      return fail(CSA_ERR_CUDA, "csa_indexer_topk_noalloc: no usable current device");
-    std::lock_guard<std::mutex> lock(g_static_mu);
-    if (g_static_ptr[dev] == nullptr) {
-      const cudaError_t e = cudaGetSymbolAddress(&g_static_ptr[dev], g_static_scratch);
-      if (e != cudaSuccess) {
-        g_static_ptr[dev] = nullptr;
-        return fail(CSA_ERR_CUDA, "csa_indexer_topk_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
-      }
-    }
-    ptr = g_static_ptr[dev];
+    // looked up on every call (a host-side query that allocates nothing), so a
+    // device reset or a new primary context never leaves a stale address behind
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess)
+      return fail(CSA_ERR_CUDA, "csa_indexer_topk_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
   }
   return csa_indexer_topk(qI, wI, kIc, B, Tq, N, q_pos0, m, k, idx, ptr, ptr ? kStaticScratchBytes : 0, stream);
 }

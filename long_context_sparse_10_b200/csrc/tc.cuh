@@ -74,11 +74,12 @@ __device__ __forceinline__ void bar_init_fence() {
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
 
-// Waits for the mbarrier phase with parity `parity`; gives up after
-// kWaitLimit rounds, records kErrWaitTimeout and returns false.
-__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
+// Waits for the mbarrier phase with parity `parity`; gives up after `limit`
+// try_wait rounds, records kErrWaitTimeout in the unit's error word and
+// returns false.
+__device__ __forceinline__ bool bar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t it = 0; it < kWaitLimit; ++it) {
+  for (uint32_t it = 0; it < limit; ++it) {
     uint32_t ok;
     asm volatile(
         "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
@@ -89,6 +90,9 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
   }
   atomicExch(&g_device_error, kErrWaitTimeout);
   return false;
+}
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
+  return bar_wait_bounded(bar, parity, kWaitLimit);
 }
 
 // Arrives once on `bar` and raises its expected transaction count by `bytes`

@@ -103,6 +103,9 @@ def _indexer_case(g, B, Tq, N, tie_blocks=0, zero_q=False):
     (1, 40, 300, 0, 4, 8, 0, False),           # long-row path; the first rows see no entry at all
     (1, 1, 40000, 4 * 40000 - 1, 4, 4096, 0, True),   # long rows, all ties, k = max
     (2, 1, 300001, 4 * 300001 - 1, 4, 2048, 0, False),  # rows past 262144 entries: bitmap in global memory
+    # prefill rows at k = 2048 (row path): visible counts crossing k, and near 16384
+    (1, 300, 16384, 8000, 4, 2048, 0, False),
+    (1, 300, 16384, 65536 - 300, 4, 2048, 0, False),
 ])
 def test_indexer_topk(B, Tq, N, q_pos0, m, k, ties, zero):
     g = np.random.default_rng(B * 1000 + N + k)
@@ -130,6 +133,9 @@ def _oracle_idx(g, B, Tq, N, m, k, q_pos0):
 @pytest.mark.parametrize("H,B,T,m,k,win,sep_v", [
     (16, 2, 300, 4, 16, 32, True), (64, 1, 200, 4, 64, 128, True), (16, 1, 2048, 4, 64, 128, True),
     (64, 2, 150, 4, 8, 7, False),
+    # 64 heads, 5 tiles of 128 slots per late row: the K/V stage rings wrap and their barrier phases flip
+    (64, 1, 2000, 4, 512, 128, True),    # separate V: 2 stages
+    (64, 1, 2000, 4, 512, 128, False),   # V = K[:, :128]: 3 stages
 ])
 def test_csa_sparse_mqa_prefill_bf16(H, B, T, m, k, win, sep_v):
     g = np.random.default_rng(H + T + k)
@@ -354,3 +360,42 @@ def test_decode_split_fp8_separate_window_values(kind):
     torch.cuda.synchronize()
     assert_close(f64(out), O, f"{kind} decode fp8, separate window V")
     assert_lse(f64(lse), Ls, f"{kind} decode lse, separate window V")
+
+
+def test_csa_prefill_pipeline_t65536_sampled_rows():
+    """The 65,536-token CSA prefill (64 heads, k = 2048, separate V) through the whole GPU pipeline, at full
+    size, checked on sampled query rows: rows that see fewer than k entries, rows around the point where
+    selection becomes partial (t = 8191), and a stride over the rest (up to 17 key tiles per row)."""
+    wl = synth.WORKLOADS["csa_prefill_t65536"]
+    x = synth.prefill_inputs(wl, seed=0)
+    m, k, win, T = wl.m, wl.k, wl.win, wl.T
+    sc = 1 / math.sqrt(192)
+    d = {kk: v.to(DEV) for kk, v in x.items()}
+    Kc = csa.csa_compress(d["k"], d["w_k"], d["b_k"], m)
+    Vc = csa.csa_compress(d["v"], d["w_v"], d["b_v"], m)
+    kIc = csa.csa_compress(d["kI"], d["w_i"], d["b_i"], m)
+    idx = csa.csa_indexer_topk(d["qI"], d["wI"], kIc, m, k)
+    out, lse = csa.csa_sparse_mqa(d["q"], csa.KVCache(k=Kc, v=Vc), m, idx,
+                                  csa.Window(k=d["k"], v=d["v"], pos0=0, length=win), sc)
+    torch.cuda.synchronize()
+    Kc_o = f64(_round_bf16(R.compress(f64(x["k"]), f64(x["w_k"]), f64(x["b_k"]), m, 2 * m)))
+    Vc_o = f64(_round_bf16(R.compress(f64(x["v"]), f64(x["w_v"]), f64(x["b_v"]), m, 2 * m)))
+    kI_o = f64(_round_bf16(R.compress(f64(x["kI"]), f64(x["w_i"]), f64(x["b_i"]), m, 2 * m)))
+    assert_close(f64(Kc), Kc_o, "Kc", max_abs=1.6e-2)
+    assert_close(f64(Vc), Vc_o, "Vc", max_abs=1.6e-2)
+    assert_close(f64(kIc), kI_o, "kIc", max_abs=1.6e-2)
+    g = np.random.default_rng(65536)
+    rows = np.unique(np.concatenate([
+        np.arange(0, 130, 7),                                   # window still filling, few entries
+        g.choice(np.arange(130, 8100), 60, replace=False),      # every visible entry selected
+        np.arange(8180, 8200),                                  # selection turns partial at t = 8191
+        g.choice(np.arange(8200, T), 200, replace=False), [T - 1]]))
+    s = R.indexer_scores(f64(x["qI"][:, rows]), f64(x["wI"][:, rows]), kI_o, rows, m)
+    ref_idx = R.topk_set(s, k)
+    got_idx = idx[:, rows].cpu().numpy()
+    same = check_topk(got_idx, s, ref_idx, k, "t65536 indexer")
+    assert same.mean() > 0.9
+    use = np.where(same.reshape(1, -1)[..., None], ref_idx, got_idx.astype(np.int64))
+    O, L = R.csa_sparse_mqa(f64(x["q"][:, rows]), rows, Kc_o, Vc_o, use, m, f64(x["k"]), f64(x["v"]), 0, win, sc)
+    assert_close(f64(out[:, rows]), O, "t65536 attention")
+    assert_lse(f64(lse[:, rows]), L, "t65536 lse")
