@@ -40,6 +40,11 @@ choice of this project, stated once here and applied everywhere below):
       saturating to +-448.
   R11 the attention also skips selected entries that are out of range or not
       visible (R4), and a query with no keys at all outputs 0 with LSE = -inf.
+  R17 grouped output projection: the H heads form G groups of H/G consecutive
+      heads; group g's outputs, concatenated head after head, are multiplied
+      by the group's own weight W[g] (d_g x (H/G) d_v), giving d_g channels per
+      group.  A dense layer that mixes the G groups afterwards is an ordinary
+      linear layer outside this method step.
 """
 from __future__ import annotations
 
@@ -276,6 +281,30 @@ def hca_dense_mqa(q, q_pos, Kc, Vc, stride, win_k, win_v, win_pos0, win_len, sca
 
     return _mqa(q, q_pos, Kc, Vc, lists, np.asarray(win_k, np.float64), np.asarray(win_v, np.float64),
                 win_pos0, win_len, scale, want_p)
+
+
+# ----------------------------------------------------------------------------
+# grouped output projection (CSA paragraph: the MQA is followed by a grouped
+# output projection that keeps its cost down; R17)
+# ----------------------------------------------------------------------------
+def grouped_out_proj(o: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """y[.., g, :] = concat_{h in group g} o[.., h, :]  @  W[g]^T   (float64).
+
+    o [.., H, dv]: attention outputs; W [G, d_g, (H/G) * dv]: row j of W[g] holds the
+    weights of group g's output channel j.  Returns y [.., G, d_g].
+    """
+    o = np.asarray(o, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    G, dg, K = W.shape
+    H, dv = o.shape[-2], o.shape[-1]
+    hg = H // G
+    assert H % G == 0 and K == hg * dv, "W must be [G, d_g, (H/G) * dv]"
+    lead = o.shape[:-2]
+    y = np.empty(lead + (G, dg), dtype=np.float64)
+    for g in range(G):
+        x = o[..., g * hg:(g + 1) * hg, :].reshape(lead + (K,))   # head g*hg first, then the next
+        y[..., g, :] = x @ W[g].T
+    return y
 
 
 def default_scale(d_qk: int = D_QK) -> float:

@@ -477,3 +477,41 @@ def test_split_cache_dequant_shares_k_and_v():
     assert np.array_equal(K[..., :128], V)
     assert np.array_equal(K[..., 128:], rope)
     np.testing.assert_allclose(V[1, 2, 3], R.e4m3_decode(codes[1, 2, 3]) * scale[1, 2], rtol=0)
+
+
+# ---------------------------------------------------------------------------
+# grouped output projection (R17)
+# ---------------------------------------------------------------------------
+def test_grouped_out_proj_is_block_diagonal_dense_projection():
+    """The grouped projection equals one dense projection of the flattened heads by the
+    block-diagonal matrix whose diagonal blocks are the groups' weights (scipy builds it)."""
+    from scipy.linalg import block_diag
+    R_, H, dv, G, dg = 5, 8, 6, 4, 7
+    o = rng.standard_normal((R_, H, dv))
+    W = rng.standard_normal((G, dg, (H // G) * dv))
+    y = R.grouped_out_proj(o, W)
+    dense = block_diag(*[W[g].T for g in range(G)])          # [(H*dv), (G*dg)]
+    assert dense.shape == (H * dv, G * dg)
+    np.testing.assert_allclose(y.reshape(R_, G * dg), o.reshape(R_, H * dv) @ dense, rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_out_proj_selector_weights_pick_channels():
+    """Weights that select one channel: output j of group g reads head g*hg + (j % hg), channel j."""
+    H, dv, G, dg = 6, 5, 3, 4
+    hg = H // G
+    W = np.zeros((G, dg, hg * dv))
+    for g in range(G):
+        for j in range(dg):
+            W[g, j, (j % hg) * dv + j] = 1.0
+    o = rng.standard_normal((2, 3, H, dv))
+    y = R.grouped_out_proj(o, W)
+    for g in range(G):
+        for j in range(dg):
+            assert np.array_equal(y[..., g, j], o[..., g * hg + j % hg, j])
+
+
+def test_grouped_out_proj_one_head_per_group_identity():
+    H, dv = 4, 3
+    o = rng.standard_normal((7, H, dv))
+    W = np.stack([np.eye(dv)] * H)                            # G = H groups of one head, W_g = I
+    assert np.array_equal(R.grouped_out_proj(o, W), o)
