@@ -4,7 +4,11 @@ Tolerances:
   * attention outputs and compressed values (bf16 results of fp32 arithmetic on
     bf16/e4m3 inputs): max-abs error <= 2e-2 and relative L2 error <= 5e-3
     against the float64 oracle;
-  * log-sum-exp: max-abs error <= 2e-3 (fp32 accumulation of bf16 products);
+  * log-sum-exp: max-abs error <= 4e-3.  The tensor-core kernels sum the
+    probabilities after rounding them to bf16 (the same values weight V), and a
+    round to nearest moves a value by at most half an ulp, 2^-8 relative; so the
+    sum is off by at most 2^-8 relative and ln of it by at most
+    -ln(1 - 2^-8) = 3.92e-3 (fp32 accumulation and exp2 add ~1e-6);
   * E4M3 codes written by the compression epilogue: within one code step of the
     oracle's round-to-nearest-even code of its float64 value; scales rel 1e-5;
   * top-k index sets: identical, except rows where the oracle's k-th and
@@ -18,7 +22,7 @@ import torch
 
 MAX_ABS = 2e-2
 REL_L2 = 5e-3
-LSE_ABS = 2e-3
+LSE_ABS = 4e-3
 TIE_REL = 1e-3
 
 
