@@ -40,6 +40,11 @@ choice of this project, stated once here and applied everywhere below):
       saturating to +-448.
   R11 the attention also skips selected entries that are out of range or not
       visible (R4), and a query with no keys at all outputs 0 with LSE = -inf.
+  R18 FP4 indexer keys (storage paragraph: the lightning indexer in FP4):
+      OCP MX E2M1 codes (sign, 2 exponent bits with bias 1, 1 mantissa bit;
+      values 0, 0.5, 1, 1.5, 2, 3, 4, 6), two per byte -- dimension 2j in the
+      low nibble of byte j, 2j+1 in the high nibble -- and one fp32 scale per
+      entry (max|k| / 6, 1 when zero); key = decode(code) * scale.
   R17 grouped output projection: the H heads form G groups of H/G consecutive
       heads; group g's outputs, concatenated head after head, are multiplied
       by the group's own weight W[g] (d_g x (H/G) d_v), giving d_g channels per
@@ -138,6 +143,26 @@ def e4m3_encode(x: np.ndarray) -> np.ndarray:
     code = np.where(_E4M3_POS[hi] == a, hi, code)
     sign = np.signbit(x).astype(np.int64) << 7          # the sign survives rounding to zero
     return (code | sign).astype(np.uint8)
+
+
+def e2m1_decode(code4: np.ndarray) -> np.ndarray:
+    """Value of each 4-bit E2M1 code S EE M (OCP MX): bias 1; E = 0 subnormal (M * 0.5)."""
+    c = np.asarray(code4, dtype=np.int64) & 0xF
+    s = np.where(c & 0x8, -1.0, 1.0)
+    e = (c >> 1) & 0x3
+    mant = (c & 0x1).astype(np.float64)
+    normal = np.ldexp(1.0 + mant / 2.0, (e - 1).astype(np.int64))
+    sub = mant * 0.5
+    return s * np.where(e == 0, sub, normal)
+
+
+def e2m1_unpack(packed: np.ndarray) -> np.ndarray:
+    """Bytes [.., d/2] holding two E2M1 codes each -> values [.., d] (dim 2j = low nibble of byte j) (R18)."""
+    b = np.asarray(packed, dtype=np.int64)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.float64)
+    out[..., 0::2] = e2m1_decode(b & 0xF)
+    out[..., 1::2] = e2m1_decode(b >> 4)
+    return out
 
 
 def quantize_entries(y_nope: np.ndarray):

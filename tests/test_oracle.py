@@ -515,3 +515,33 @@ def test_grouped_out_proj_one_head_per_group_identity():
     o = rng.standard_normal((7, H, dv))
     W = np.stack([np.eye(dv)] * H)                            # G = H groups of one head, W_g = I
     assert np.array_equal(R.grouped_out_proj(o, W), o)
+
+
+# ---------------------------------------------------------------------------
+# FP4 E2M1 indexer keys (R18)
+# ---------------------------------------------------------------------------
+def test_e2m1_golden_values():
+    rows = []
+    for line in open(os.path.join(GOLDEN, "e2m1_ocp_values.txt")):
+        if line.strip() and not line.startswith("#"):
+            c, v = line.split()
+            rows.append((int(c, 16), float(v)))
+    assert len(rows) == 16
+    codes = np.array([c for c, _ in rows])
+    vals = R.e2m1_decode(codes)
+    for (c, v), got in zip(rows, vals):
+        assert got == v and np.signbit(got) == np.signbit(v), (hex(c), got, v)
+
+
+def test_e2m1_unpack_nibble_order():
+    """Dimension 2j sits in the low nibble of byte j: the byte 0x72 holds (1.0, 6.0) in that order."""
+    packed = np.array([[0x72, 0xA9, 0x0F]], dtype=np.uint8)
+    assert R.e2m1_unpack(packed).tolist() == [[1.0, 6.0, -0.5, -1.0, -6.0, 0.0]]
+
+
+def test_e2m1_values_are_the_grid_between_adjacent_powers():
+    """Every nonzero magnitude is 2^e * (1 + m/2) for e in {0, 1, 2} or the subnormal 0.5, and the set
+    {0, 0.5, 1, 1.5, 2, 3, 4, 6} is symmetric under the sign bit."""
+    v = R.e2m1_decode(np.arange(16))
+    assert sorted(set(np.abs(v).tolist())) == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert np.array_equal(v[8:], -v[:8])
