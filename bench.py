@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-reps", type=int, default=100, help="launches of the dominant kernel to average")
     ap.add_argument("--breakdown", action="store_true", help="also time each library call of the step (stderr)")
+    ap.add_argument("--no-extras", action="store_true", help="skip timing the rows beyond the headline step")
     return ap.parse_args()
 
 
@@ -216,6 +217,9 @@ class DecodeRun:
         if wl.indexer_fp8:
             self.csa.csa_indexer_topk_e4m3(self.d["qI"], self.d["wI"], self.d["kI_codes"], self.d["kI_scale"], wl.m,
                                            wl.k, q_pos0=self.q_pos0, idx=self.idx, workspace=self.ws_idx)
+        elif wl.indexer_fp4:
+            self.csa.csa_indexer_topk_e2m1(self.d["qI"], self.d["wI"], self.d["kI_codes"], self.d["kI_scale"], wl.m,
+                                           wl.k, q_pos0=self.q_pos0, idx=self.idx, workspace=self.ws_idx)
         else:
             self.csa.csa_indexer_topk(self.d["qI"], self.d["wI"], self.d["kIc"], wl.m, wl.k, q_pos0=self.q_pos0,
                                       idx=self.idx, workspace=self.ws_idx)
@@ -297,22 +301,45 @@ class DecodeRun:
     def dominant(self):
         """(name, source file, algorithmic bytes per launch, callable that launches it)."""
         wl = self.wl
-        per_entry = (64 + 4) if wl.indexer_fp8 else 64 * 2  # E4M3 codes + scale, or bf16 keys
+        per_entry = self.key_bytes()
         b = wl.B * wl.N * per_entry + wl.B * 4 * 64 * 2 + wl.B * 4 * 4
-        name = "indexer_score_long_e4m3" if wl.indexer_fp8 else "indexer_score_long"
+        name = ("indexer_score_long_e4m3" if wl.indexer_fp8 else
+                "indexer_score_long_e2m1" if wl.indexer_fp4 else "indexer_score_long")
         return name, "long_context_sparse_10_b200/csrc/indexer.cu", b, "hbm", self.indexer
+
+    def step_bytes(self):
+        """Algorithmic HBM bytes of one decode step: the indexer keys and queries, the gathered split-cache
+        entries (128 e4m3 + 64 bf16 + fp32 scale = 260 B), the window keys, the queries, the selection and the
+        outputs; plus, for the hybrid step, the HCA layer's whole cache, window, query and output."""
+        wl = self.wl
+        B, H, k = wl.B, wl.H, wl.k
+        b = B * wl.N * self.key_bytes() + B * (4 * 64 * 2 + 4 * 4)
+        b += B * k * 260 + B * wl.win * 192 * 2 + B * H * 192 * 2 + B * H * 128 * 2 + B * k * 4
+        if self.hybrid:
+            b += B * wl.N_hca * 260 + B * wl.win * 192 * 2 + B * H * 192 * 2 + B * H * 128 * 2
+        return b
+
+    def step_roofline(self, ms, pk):
+        b = self.step_bytes()
+        return {"bound": "hbm", "algorithmic_bytes": b, "achieved": b / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": b / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+
+    def key_bytes(self):
+        """Indexer key bytes per entry: E4M3 codes + scale, E2M1 codes + scale, or bf16."""
+        wl = self.wl
+        return (64 + 4) if wl.indexer_fp8 else (32 + 4) if wl.indexer_fp4 else 64 * 2
 
     def describe(self, world):
         wl = self.wl
+        keys = ("e4m3 keys + per-entry scale" if wl.indexer_fp8 else
+                "e2m1 (FP4) keys + per-entry scale" if wl.indexer_fp4 else "bf16")
         s = (f"{wl.name}: decode at context {wl.L}, batch {wl.B} per GPU, {wl.H} query heads, qk 192 / v 128; "
-             f"CSA m={wl.m} (N={wl.N}, FP8-e4m3 nope + BF16 RoPE cache, indexer 4x64 "
-             f"{'e4m3 keys + per-entry scale' if wl.indexer_fp8 else 'bf16'}, top-k={wl.k})")
+             f"CSA m={wl.m} (N={wl.N}, FP8-e4m3 nope + BF16 RoPE cache, indexer 4x64 {keys}, top-k={wl.k})")
         if self.hybrid:
             s += f" then HCA m'={wl.m_hca} (N'={wl.N_hca}, same split cache)"
         s += f", sliding window {wl.win}"
         return {"workload": s, "global_batch": wl.B * world, "seq_len": wl.L, "parallelism": f"dp{world} (replicas)",
-                "l2": f"inputs larger than L2 (the indexer streams {wl.B * wl.N * (68 if wl.indexer_fp8 else 128) / 1e6:.0f} "
-                      "MB/step > 126 MB L2)",
+                "l2": f"inputs larger than L2 (the step streams {self.step_bytes() / 1e6:.0f} MB > 126 MB L2)",
                 "timing": "CUDA graph replay of the whole step"}
 
     def _oracle_seq(self, b):
@@ -324,6 +351,8 @@ class DecodeRun:
         wI = h["wI"][b:b + 1].double().numpy()
         if wl.indexer_fp8:
             kI = R.e4m3_decode(h["kI_codes"][b:b + 1].numpy()) * h["kI_scale"][b:b + 1].double().numpy()[..., None]
+        elif wl.indexer_fp4:
+            kI = R.e2m1_unpack(h["kI_codes"][b:b + 1].numpy()) * h["kI_scale"][b:b + 1].double().numpy()[..., None]
         else:
             kI = h["kIc"][b:b + 1].double().numpy()
         q = h["q"][b:b + 1].double().numpy()
@@ -459,6 +488,18 @@ class PrefillRun:
         keys = ent + __import__("numpy").minimum(wl.win, t + 1)
         return float(wl.B * wl.H * 2 * (192 + 128) * keys.sum())
 
+    def step_roofline(self, ms, pk):
+        """Tensor work of the whole prefill step (attention + indexer scores, algorithmic) against bf16 peak."""
+        import numpy as np
+        wl = self.wl
+        f = self.attn_flops()
+        if self.csa_kind:
+            t = np.arange(wl.T)
+            f += float(wl.B * 2 * 4 * 64 * np.minimum((t + 1) // wl.m, wl.N).sum())
+        return {"bound": "tensor", "algorithmic_flops": f, "achieved": f / (ms * 1e-3) / 1e12,
+                "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": f / (ms * 1e-3) / 1e12 / pk["bf16_tflops_sustained"]}
+
     def dominant(self):
         return ("attention_prefill", "long_context_sparse_10_b200/csrc/attention.cu", self.attn_flops(), "tensor",
                 self.attention)
@@ -545,6 +586,133 @@ class PrefillRun:
 
 
 # ---------------------------------------------------------------------------
+# the rows beyond the headline step, each timed on its own (CUDA events around
+# graph replays of the library call) against its roofline
+# ---------------------------------------------------------------------------
+def _time_graph(torch, fn, reps=20, iters=5):
+    """Median per-call milliseconds of `fn` captured `reps` times in one CUDA graph.  `fn` may be a list of
+    callables over distinct buffers, used in turn, so that consecutive calls do not find their inputs in L2."""
+    fns = fn if isinstance(fn, (list, tuple)) else [fn]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for f in fns:
+            f()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for r in range(reps):
+            fns[r % len(fns)]()
+    g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(iters):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) / reps)
+    del g
+    return statistics.median(ts)
+
+
+def extras(dev, pk):
+    """Grouped output projection, decode-time cache append, packed prefill and the context-parallel merges."""
+    import numpy as np
+    import torch
+    import long_context_sparse_10_b200 as csa
+    from long_context_sparse_10_b200 import context_parallel as cp
+    g = np.random.default_rng(0)
+    res = {}
+
+    def bf16(shape, std=1.0):
+        return torch.from_numpy((g.standard_normal(shape) * std).astype(np.float32)).to(torch.bfloat16).to(dev)
+
+    # compression of the 65,536-token prefill (CSA m = 4: K 192, V 128, indexer key 64) and of the HCA
+    # prefill (m' = 128): algorithmic bytes = raw tokens read once + entries written
+    for name, (T, d, m, kind) in {"csa_compress_k_t65536": (65536, 192, 4, "csa"),
+                                  "csa_compress_ki_t65536": (65536, 64, 4, "csa"),
+                                  "hca_compress_k_b2_t8192": (16384, 192, 128, "hca")}.items():
+        B = 2 if kind == "hca" else 1
+        cw = 2 * m if kind == "csa" else m
+        wc = torch.from_numpy((g.standard_normal(d) * 0.02).astype(np.float32)).to(dev)
+        bc = torch.from_numpy((g.standard_normal((cw, d)) * 0.1).astype(np.float32)).to(dev)
+        fn = csa.csa_compress if kind == "csa" else csa.hca_compress
+        nbuf = max(2, int(300e6 // (T * d * 2)))   # inputs of consecutive calls together exceed the 126 MB L2
+        xs_ = [bf16((B, T // B, d)) for _ in range(nbuf)]
+        ys_ = [torch.empty(B, -(-(T // B) // m), d, dtype=torch.bfloat16, device=dev) for _ in range(nbuf)]
+        ms = _time_graph(torch, [lambda x=x, y=y: fn(x, wc, bc, m, out=y) for x, y in zip(xs_, ys_)])
+        byts = xs_[0].numel() * 2 + ys_[0].numel() * 2
+        del xs_, ys_
+        res[name] = {"us": ms * 1e3, "bound": "hbm", "algorithmic_bytes": byts,
+                     "achieved_gbs": byts / (ms * 1e-3) / 1e9, "frac": byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    # grouped output projection (64 heads in 8 groups of 8, d_g = 1024)
+    ws_ = [bf16((8, 1024, 1024), 0.02) for _ in range(12)]   # 12 x 16 MiB of weights: more than L2
+    w = ws_[0]
+    for name, rows in (("decode_rows8", 8), ("prefill_rows16384", 16384)):
+        o = bf16((rows, 64, 128), 0.5)
+        if rows <= 128:
+            ms = _time_graph(torch, [lambda w_=w_: csa.grouped_out_proj(o, w_) for w_ in ws_], reps=24)
+        else:
+            ms = _time_graph(torch, lambda: csa.grouped_out_proj(o, w))
+        flops = 2.0 * rows * 64 * 128 * 1024
+        byts = w.numel() * 2 + o.numel() * 2 + rows * 8 * 1024 * 2
+        if rows <= 128:
+            res[f"grouped_out_proj_{name}"] = {"us": ms * 1e3, "bound": "hbm", "algorithmic_bytes": byts,
+                                               "achieved_gbs": byts / (ms * 1e-3) / 1e9,
+                                               "frac": byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+        else:
+            res[f"grouped_out_proj_{name}"] = {"us": ms * 1e3, "bound": "tensor", "algorithmic_flops": flops,
+                                               "achieved_tflops": flops / (ms * 1e-3) / 1e12,
+                                               "frac": flops / (ms * 1e-3) / 1e12 / pk["bf16_tflops"]}
+    # decode-time append of the entry the newest token completes (8 sequences, split FP8 cache, d 192)
+    B, rows = 8, 256
+    xs = bf16((B, rows, 192))
+    ww = torch.from_numpy((g.standard_normal(192) * 0.02).astype(np.float32)).to(dev)
+    bb = torch.from_numpy((g.standard_normal((8, 192)) * 0.1).astype(np.float32)).to(dev)
+    cache = csa.KVCache(nope=torch.zeros(B, 4096, 128, dtype=torch.uint8, device=dev),
+                        rope=torch.zeros(B, 4096, 64, dtype=torch.bfloat16, device=dev),
+                        scale=torch.zeros(B, 4096, device=dev))
+    t = 4 * 4000 + 3
+    ms = _time_graph(torch, lambda: csa.csa_compress_append(xs, t + 1 - rows, t, ww, bb, 4, cache))
+    res["csa_compress_append_b8"] = {"us": ms * 1e3, "bound": "latency", "note": "one entry per sequence"}
+    # packed CSA prefill: 16 documents, 16,384 tokens, H 64, k 512
+    lens = [int(x) for x in g.integers(64, 2048, 16)]
+    lens[-1] += 16384 - sum(lens)
+    pkd = csa.Packed(lens, 4)
+    TT = pkd.total_tokens
+    q, K, V, qI, kI = bf16((TT, 64, 192)), bf16((TT, 192)), bf16((TT, 128)), bf16((TT, 4, 64)), bf16((TT, 64))
+    wI = torch.from_numpy(g.random((TT, 4)).astype(np.float32)).to(dev)
+    wk, bk = ww, bb
+    wv = torch.from_numpy((g.standard_normal(128) * 0.02).astype(np.float32)).to(dev)
+    bv = torch.from_numpy((g.standard_normal((8, 128)) * 0.1).astype(np.float32)).to(dev)
+    wi = torch.from_numpy((g.standard_normal(64) * 0.02).astype(np.float32)).to(dev)
+    bi = torch.from_numpy((g.standard_normal((8, 64)) * 0.1).astype(np.float32)).to(dev)
+
+    def packed_step():
+        Kc = csa.csa_compress_packed(K, pkd, wk, bk, 4)
+        Vc = csa.csa_compress_packed(V, pkd, wv, bv, 4)
+        kIc = csa.csa_compress_packed(kI, pkd, wi, bi, 4)
+        idx = csa.csa_indexer_topk_packed(qI, wI, kIc, pkd, 4, 512)
+        csa.csa_sparse_mqa_packed(q, pkd, csa.KVCache(k=Kc, v=Vc), 4, idx, K, V, 128, 1 / math.sqrt(192))
+    ms = _time_graph(torch, packed_step, reps=3, iters=3)
+    res["packed_csa_prefill_16docs_t16384"] = {"us": ms * 1e3, "tokens_per_s": TT / (ms * 1e-3),
+                                               "documents": len(lens)}
+    # context-parallel merges for 8 ranks, 8 decode rows, k 2048, 64 heads
+    ops = cp.KernelOps()
+    cs = torch.from_numpy(g.standard_normal((8, 1, 8 * 2048)).astype(np.float32)).to(dev)
+    ci = torch.arange(8 * 2048, dtype=torch.int32, device=dev).repeat(8, 1).reshape(8, 1, 8 * 2048).contiguous()
+    ms = _time_graph(torch, lambda: ops.topk_merge(cs, ci, 2048))
+    res["cp_topk_merge_g8_rows8_k2048"] = {"us": ms * 1e3, "bound": "latency"}
+    outs = bf16((8, 8, 1, 64, 128))
+    lses = torch.from_numpy(g.standard_normal((8, 8, 1, 64)).astype(np.float32)).to(dev)
+    ms = _time_graph(torch, lambda: ops.attn_merge(outs, lses))
+    res["cp_attn_merge_g8_rows8"] = {"us": ms * 1e3, "bound": "latency"}
+    return res
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -776,6 +944,10 @@ def main():
         e2e = {"value": run.tokens * world / (ems * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": ems, "steps": k2}
 
+    extra = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        extra = extras(dev, pk)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n, spent, sample = run.oracle_sample(args.cpu_sample_s)
@@ -786,9 +958,10 @@ def main():
         line = {"metric": METRIC, "value": run.tokens * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": run.describe(world), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "config": run.describe(world), "roofline": roofline, "step_roofline": run.step_roofline(ms, pk),
+                "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(),
-                "self_check": check, "library": csa.version()}
+                "self_check": check, "extras": extra, "library": csa.version()}
         print(json.dumps(line), flush=True)
     del graph
     if world > 1:

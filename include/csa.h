@@ -97,6 +97,27 @@ typedef struct csa_window {
   int32_t reserved;          /* must be 0 */
 } csa_window;
 
+/*
+ * Packed sequences (host struct; device pointers): several independent
+ * sequences stored back to back in one buffer, e.g. the documents of a packed
+ * pre-training batch.  The pages (DeepSeek-V4 summary, section "Datasets")
+ * train on packed documents with sample-level attention masks: no compression
+ * window, indexer score, sliding window or attention crosses from one sequence
+ * into another.  Sequence s owns packed tokens [cu_tokens[s], cu_tokens[s+1])
+ * (positions 0 .. len_s - 1 within the sequence) and compressed entries
+ * [cu_entries[s], cu_entries[s+1]), ceil(len_s / stride) of them -- so a CSA
+ * cache and an HCA cache of the same sequences need descriptors with their own
+ * cu_entries.  Offsets are ascending int32 with cu_*[0] = 0.
+ */
+typedef struct csa_packed {
+  const int32_t* cu_tokens;   /* device int32 [n_seqs + 1] */
+  const int32_t* cu_entries;  /* device int32 [n_seqs + 1] */
+  int32_t n_seqs;
+  int32_t max_tokens;         /* length of the longest sequence (sizes launches and scratch) */
+  int64_t total_tokens;       /* cu_tokens[n_seqs], < 2^31 */
+  int64_t total_entries;      /* cu_entries[n_seqs], < 2^31 */
+} csa_packed;
+
 /* Library version string, e.g. "csa-b200 0.1.0 sm_100a". */
 CSA_API const char* csa_version(void);
 /* Name of a status code. */
@@ -180,8 +201,53 @@ CSA_API csa_status hca_compress(const void* x, int64_t B, int64_t T, int32_t d, 
                         const float* w, const float* b_pos, int32_t out_layout,
                         void* out, void* out_rope, float* out_scale, void* stream);
 
-/* Workspace bytes csa_indexer_topk needs for these sizes. */
+/*
+ * csa_compress_append / hca_compress_append -- incremental cache append at
+ * decode time (same entry rule as csa_compress / hca_compress).  Every
+ * sequence of the call has just received the token at position t.  When t + 1
+ * is a multiple of the stride (m, or m' for HCA), entry i = (t+1)/stride - 1
+ * has just become complete; it is computed from the sequence's recent raw
+ * tokens and written into slot i of a resident cache that holds n_cap entries
+ * per sequence.  Otherwise nothing completes and the call returns CSA_OK
+ * without enqueueing work.
+ *   x       bf16 [B, rows, d]: row j of a sequence holds its token at
+ *           position x_pos0 + j; the rows must hold the entry's window
+ *           [max(0, i m - (window - stride)), t]
+ *   out...  the cache planes, as csa_compress with N replaced by n_cap
+ *           (bf16 [B, n_cap, d], or the split FP8 planes for d == 192)
+ *   i < n_cap.  Other arguments and errors as csa_compress.
+ */
+CSA_API csa_status csa_compress_append(const void* x, int64_t B, int64_t rows, int64_t x_pos0, int64_t t,
+                                       int32_t d, int32_t m, const float* w, const float* b_pos,
+                                       int32_t out_layout, void* out, void* out_rope, float* out_scale,
+                                       int64_t n_cap, void* stream);
+CSA_API csa_status hca_compress_append(const void* x, int64_t B, int64_t rows, int64_t x_pos0, int64_t t,
+                                       int32_t d, int32_t m_prime, const float* w, const float* b_pos,
+                                       int32_t out_layout, void* out, void* out_rope, float* out_scale,
+                                       int64_t n_cap, void* stream);
+
+/*
+ * csa_compress_packed / hca_compress_packed -- compression of packed
+ * sequences: each sequence is compressed on its own (its windows never reach
+ * into a neighbour), its entries landing in rows [cu_entries[s],
+ * cu_entries[s+1]) of out.
+ *   x    bf16 [total_tokens, d];  out: as csa_compress with B*N replaced by
+ *        total_entries.  packed->cu_entries must use this call's stride.
+ */
+CSA_API csa_status csa_compress_packed(const void* x, const csa_packed* packed, int32_t d, int32_t m,
+                                       const float* w, const float* b_pos, int32_t out_layout, void* out,
+                                       void* out_rope, float* out_scale, void* stream);
+CSA_API csa_status hca_compress_packed(const void* x, const csa_packed* packed, int32_t d, int32_t m_prime,
+                                       const float* w, const float* b_pos, int32_t out_layout, void* out,
+                                       void* out_rope, float* out_scale, void* stream);
+
+/* Workspace bytes csa_indexer_topk needs for these sizes (0 for prefill rows,
+ * whose scores stay on chip; nonzero for the long decode rows). */
 CSA_API size_t csa_indexer_topk_workspace_size(int64_t B, int64_t Tq, int64_t N, int32_t k);
+/* Workspace bytes csa_indexer_topk_e4m3, csa_indexer_topk_e2m1 and
+ * csa_indexer_topk_with_scores need (their prefill rows keep a score row per
+ * query in the workspace). */
+CSA_API size_t csa_indexer_topk_coded_workspace_size(int64_t B, int64_t Tq, int64_t N, int32_t k);
 
 /*
  * csa_indexer_topk -- the lightning indexer and its top-k selection (Method
@@ -201,16 +267,46 @@ CSA_API csa_status csa_indexer_topk(const void* qI, const float* wI, const void*
                             void* stream);
 
 /*
+ * csa_indexer_topk_with_scores -- csa_indexer_topk that also returns, in
+ * scores fp32 [B, Tq, k], the score of each selected entry (-inf in padded
+ * slots).  Workspace: csa_indexer_topk_coded_workspace_size.  Errors as
+ * csa_indexer_topk.  The
+ * context-parallel decode uses it: each rank selects a local top-k over its
+ * range of entries and the ranks' (score, index) candidates are merged by
+ * csa_cp_topk_merge.
+ */
+CSA_API csa_status csa_indexer_topk_with_scores(const void* qI, const float* wI, const void* kIc, int64_t B,
+                                                int64_t Tq, int64_t N, int64_t q_pos0, int32_t m, int32_t k,
+                                                int32_t* idx, float* scores, void* workspace,
+                                                size_t workspace_bytes, void* stream);
+
+/*
  * csa_indexer_topk_e4m3 -- csa_indexer_topk over indexer keys stored in FP8
  * (Method section, storage paragraph: the lightning indexer runs at low
  * precision -- the pages give FP4; this layout stores E4M3 codes).  Entry i's
  * key is kI_codes[b,i,:] (64 E4M3 bytes) times kI_scale[b,i] (fp32, > 0); the
  * score is computed from those exact values (the scale factors out of the relu
- * and head sums).  Same selection rule, output, workspace
- * (csa_indexer_topk_workspace_size) and errors as csa_indexer_topk.
+ * and head sums).  Workspace: csa_indexer_topk_coded_workspace_size.  Same
+ * selection rule, output and errors as csa_indexer_topk.
  *   kI_codes uint8 [B, N, 64];  kI_scale fp32 [B, N]
  */
 CSA_API csa_status csa_indexer_topk_e4m3(const void* qI, const float* wI, const uint8_t* kI_codes,
+                                         const float* kI_scale, int64_t B, int64_t Tq, int64_t N,
+                                         int64_t q_pos0, int32_t m, int32_t k, int32_t* idx,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * csa_indexer_topk_e2m1 -- csa_indexer_topk over FP4 indexer keys (Method
+ * section, storage paragraph: FP4 precision for the lightning indexer).  Each
+ * key is 64 OCP MX E2M1 codes (sign, 2 exponent bits with bias 1, 1 mantissa
+ * bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), two per byte -- dimension 2j in
+ * the low nibble of byte j, 2j+1 in the high nibble -- times one fp32 scale
+ * per entry (> 0; max|k| / 6 is the natural choice).  Scores are computed from
+ * those exact values.  Workspace: csa_indexer_topk_coded_workspace_size.
+ * Same selection rule, output and errors as csa_indexer_topk.
+ *   kI_codes uint8 [B, N, 32];  kI_scale fp32 [B, N]
+ */
+CSA_API csa_status csa_indexer_topk_e2m1(const void* qI, const float* wI, const uint8_t* kI_codes,
                                          const float* kI_scale, int64_t B, int64_t Tq, int64_t N,
                                          int64_t q_pos0, int32_t m, int32_t k, int32_t* idx,
                                          void* workspace, size_t workspace_bytes, void* stream);
@@ -236,6 +332,26 @@ CSA_API csa_status csa_indexer_topk_e4m3(const void* qI, const float* wI, const 
 CSA_API csa_status csa_indexer_topk_noalloc(const void* qI, const float* wI, const void* kIc,
                                             int64_t B, int64_t Tq, int64_t N, int64_t q_pos0,
                                             int32_t m, int32_t k, int32_t* idx, void* stream);
+
+/* Workspace bytes csa_indexer_topk_packed needs for these packed sequences. */
+CSA_API size_t csa_indexer_topk_packed_workspace_size(const csa_packed* packed, int32_t m, int32_t k);
+
+/*
+ * csa_indexer_topk_packed -- csa_indexer_topk over packed sequences: every
+ * token of every sequence is a query row (prefill), sequence s's row at
+ * position t (t = 0 at the sequence's first token) sees that sequence's
+ * entries i with (i+1)m - 1 <= t only.  Output indices are entry indices
+ * within the sequence (0 = its first entry), ascending, -1 padded.
+ *   qI  bf16 [total_tokens, 4, 64];  wI fp32 [total_tokens, 4]
+ *   kIc bf16 [total_entries, 64] (e.g. csa_compress_packed's output)
+ *   idx int32 [total_tokens, k] (output)
+ *   packed->cu_entries must use stride m.  Sequences of up to 32768 entries
+ *   (ceil(max_tokens / m)); longer ones return CSA_ERR_UNSUPPORTED.  Other
+ *   limits and errors as csa_indexer_topk.
+ */
+CSA_API csa_status csa_indexer_topk_packed(const void* qI, const float* wI, const void* kIc,
+                                           const csa_packed* packed, int32_t m, int32_t k, int32_t* idx,
+                                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Workspace bytes csa_sparse_mqa needs for these sizes on the current device
@@ -284,6 +400,86 @@ CSA_API csa_status hca_dense_mqa(const void* q, int64_t B, int64_t Tq, int32_t H
                          const csa_kv_cache* cache, int32_t m_prime, const csa_window* win,
                          float scale, void* out, float* lse, void* workspace,
                          size_t workspace_bytes, void* stream);
+
+/*
+ * csa_sparse_mqa_packed / hca_dense_mqa_packed -- the core attention over
+ * packed sequences (sample-level masks): query row r is packed token r, at
+ * position t within its sequence s; its entry set is drawn from s's entries
+ * only (cache rows cu_entries[s] + i, visibility (i+1)*stride - 1 <= t) and
+ * its sliding window from s's own tokens [max(0, t - len + 1), t].
+ *   q     bf16 [total_tokens, H, 192]
+ *   cache n_entries == total_entries (e.g. csa_compress_packed's output)
+ *   idx   int32 [total_tokens, k] of entry indices within the sequence
+ *         (csa_indexer_topk_packed's output)
+ *   win   the packed raw tokens: k bf16 [total_tokens, 192], v nullable,
+ *         pos0 = 0, rows = total_tokens
+ *   out   bf16 [total_tokens, H, 128];  lse fp32 [total_tokens, H] (nullable)
+ *   workspace: csa_sparse_mqa_workspace_size(1, total_tokens, H, k, len), or
+ *   for HCA hca_dense_mqa_workspace_size(1, total_tokens, H,
+ *   ceil(max_tokens / m'), len).  Other rules as csa_sparse_mqa.
+ */
+CSA_API csa_status csa_sparse_mqa_packed(const void* q, int32_t H, const csa_packed* packed,
+                                         const csa_kv_cache* cache, int32_t m, const int32_t* idx, int32_t k,
+                                         const csa_window* win, float scale, void* out, float* lse,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+CSA_API csa_status hca_dense_mqa_packed(const void* q, int32_t H, const csa_packed* packed,
+                                        const csa_kv_cache* cache, int32_t m_prime, const csa_window* win,
+                                        float scale, void* out, float* lse, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/*
+ * Context-parallel decode of one long sequence over G ranks (one process per
+ * GPU).  The pages name no parallel scheme for the attention; this split is
+ * exact: rank r holds the contiguous entry range [lo_r, lo_{r+1}) (lo
+ * ascending with r) of the compressed caches and scores it with
+ * csa_indexer_topk_with_scores (q_pos0 shifted by -lo_r * m so that
+ * visibility is unchanged); the G candidate lists, all-gathered in rank order
+ * and made global (local index + lo_r), are merged here into the global top-k,
+ * which is exactly the top-k of the whole sequence; each rank attends over the
+ * selected entries it holds (indices minus lo_r; the others fall outside its
+ * range and are skipped) and one rank also over the window; the partial
+ * (out, lse) of all ranks are merged by csa_cp_attn_merge.
+ *
+ * csa_cp_topk_merge -- per row, the k best of n_cand candidates.
+ *   cand_scores fp32 [R, n_cand], cand_idx int32 [R, n_cand] (-1 = no
+ *   candidate): the concatenation, in rank order, of each rank's ascending
+ *   list, so that positions ascend with the global index.
+ *   idx int32 [R, k]: the selected global indices, ascending, ties to the
+ *   lower index, -1 padded.  1 <= k <= 4096, 1 <= n_cand <= 32768.
+ */
+CSA_API csa_status csa_cp_topk_merge(const float* cand_scores, const int32_t* cand_idx, int64_t R,
+                                     int32_t n_cand, int32_t k, int32_t* idx, void* stream);
+
+/*
+ * csa_cp_attn_merge -- combines G partial attentions of the same query rows
+ * over disjoint key sets (each with its own softmax) into the attention over
+ * their union:  out = sum_g w_g out_g / sum_g w_g,  w_g = exp(lse_g - max lse),
+ * lse = max lse + ln sum_g w_g.  A part with lse = -inf (no keys) has weight 0;
+ * rows where every part is empty get out = 0, lse = -inf.
+ *   outs bf16 [G, R, H, 128], lses fp32 [G, R, H] -> out bf16 [R, H, 128],
+ *   lse fp32 [R, H] (nullable).
+ */
+CSA_API csa_status csa_cp_attn_merge(const void* outs, const float* lses, int32_t G, int64_t R, int32_t H,
+                                     void* out, float* lse, void* stream);
+
+/*
+ * csa_grouped_out_proj -- grouped output projection after the core attention
+ * (Method section, CSA paragraph: the MQA is followed by a grouped output
+ * projection that keeps its compute cost down).  The H heads form G groups of
+ * H/G consecutive heads; group g's outputs, concatenated head after head
+ * (K = (H/G) * 128 values per row), are multiplied by the group's own weight:
+ *     y[r, g, j] = sum_{c<K} o[r, g*H/G + c/128, c%128] * w[g, j, c]
+ *   o  bf16 [R, H, 128]   (the attention output, e.g. csa_sparse_mqa's out with
+ *                          R = B * Tq)
+ *   w  bf16 [G, d_g, K]   (row j of w[g]: the weights of output channel j, the
+ *                          layout of a linear layer's [out, in] weight)
+ *   y  bf16 [R, G, d_g]   (output; fp32 accumulation)
+ *   1 <= G, G divides H (H <= 256), d_g a multiple of 64.  R == 0 is a no-op.
+ * A layer that mixes the G groups afterwards is an ordinary dense linear layer
+ * outside this call.  Needs no workspace.
+ */
+CSA_API csa_status csa_grouped_out_proj(const void* o, int64_t R, int32_t H, int32_t G, int32_t d_g,
+                                        const void* w, void* y, void* stream);
 
 #ifdef __cplusplus
 }

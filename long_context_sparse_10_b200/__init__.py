@@ -14,6 +14,8 @@ Shapes (B sequences, Tq query rows, N entries, H heads in {16, 64}):
       [B, N, 64] -> idx int32 [B, Tq, k] (ascending, -1 padded).
   csa_sparse_mqa / hca_dense_mqa: q bf16 [B, Tq, H, 192] -> (out bf16
       [B, Tq, H, 128], lse fp32 [B, Tq, H]).
+  grouped_out_proj: out bf16 [..., H, 128], w bf16 [G, d_g, (H/G)*128] ->
+      y bf16 [..., G, d_g].
 """
 from __future__ import annotations
 
@@ -26,7 +28,9 @@ from . import _lib
 
 __all__ = ["CsaError", "KVCache", "Window", "csa_compress", "hca_compress", "csa_indexer_topk", "csa_indexer_topk_e4m3",
            "csa_indexer_topk_workspace_size", "csa_sparse_mqa", "csa_sparse_mqa_workspace_size", "hca_dense_mqa",
-           "hca_dense_mqa_workspace_size", "launch_count", "version"]
+           "hca_dense_mqa_workspace_size", "grouped_out_proj", "launch_count", "version", "Packed", "csa_compress_append",
+           "hca_compress_append", "csa_compress_packed", "hca_compress_packed", "csa_indexer_topk_packed",
+           "csa_sparse_mqa_packed", "hca_dense_mqa_packed", "csa_indexer_topk_e2m1"]
 
 
 class CsaError(RuntimeError):
@@ -146,6 +150,11 @@ def csa_indexer_topk_workspace_size(B, Tq, N, k) -> int:
     return int(_lib.load().csa_indexer_topk_workspace_size(B, Tq, N, k))
 
 
+def csa_indexer_topk_coded_workspace_size(B, Tq, N, k) -> int:
+    """Workspace of the E4M3 / E2M1 key calls and of csa_indexer_topk_with_scores."""
+    return int(_lib.load().csa_indexer_topk_coded_workspace_size(B, Tq, N, k))
+
+
 def csa_indexer_topk(qI, wI, kIc, m, k, *, q_pos0=0, idx=None, workspace=None, stream=None):
     """Lightning-indexer scores and top-k entry ids (int32 [B, Tq, k], ascending, -1 padded)."""
     lib = _lib.load()
@@ -169,12 +178,29 @@ def csa_indexer_topk_e4m3(qI, wI, kI_codes, kI_scale, m, k, *, q_pos0=0, idx=Non
     N = kI_codes.shape[1]
     if idx is None:
         idx = torch.empty(B, Tq, k, dtype=torch.int32, device=qI.device)
-    need = csa_indexer_topk_workspace_size(B, Tq, N, k)
+    need = csa_indexer_topk_coded_workspace_size(B, Tq, N, k)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=qI.device)
     st = lib.csa_indexer_topk_e4m3(_ptr(qI), _ptr(wI), _ptr(kI_codes), _ptr(kI_scale), B, Tq, N, q_pos0, m, k,
                                    _ptr(idx), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "csa_indexer_topk_e4m3")
+    return idx
+
+
+def csa_indexer_topk_e2m1(qI, wI, kI_codes, kI_scale, m, k, *, q_pos0=0, idx=None, workspace=None, stream=None):
+    """csa_indexer_topk over FP4 keys: kI_codes uint8 [B, N, 32] (E2M1, two per byte, low nibble = even
+    dimension), kI_scale fp32 [B, N]."""
+    lib = _lib.load()
+    B, Tq = qI.shape[0], qI.shape[1]
+    N = kI_codes.shape[1]
+    if idx is None:
+        idx = torch.empty(B, Tq, k, dtype=torch.int32, device=qI.device)
+    need = csa_indexer_topk_coded_workspace_size(B, Tq, N, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=qI.device)
+    st = lib.csa_indexer_topk_e2m1(_ptr(qI), _ptr(wI), _ptr(kI_codes), _ptr(kI_scale), B, Tq, N, q_pos0, m, k,
+                                   _ptr(idx), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "csa_indexer_topk_e2m1")
     return idx
 
 
@@ -231,4 +257,176 @@ def hca_dense_mqa(q, cache: KVCache, m_prime, win: Window | None, scale, *, q_po
                            ctypes.byref(wd) if wd is not None else None, float(scale), _ptr(out), _ptr(lse),
                            _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "hca_dense_mqa")
+    return out, lse
+
+
+def grouped_out_proj(o, w, *, y=None, stream=None):
+    """Grouped output projection: heads in G groups of H/G, group g's outputs times w[g]^T.
+
+    o bf16 [..., H, 128] (attention output), w bf16 [G, d_g, (H/G)*128] -> y bf16 [..., G, d_g].
+    """
+    lib = _lib.load()
+    H = o.shape[-2]
+    G, dg = w.shape[0], w.shape[1]
+    lead = tuple(o.shape[:-2])
+    R = 1
+    for n in lead:
+        R *= n
+    if y is None:
+        y = torch.empty(*lead, G, dg, dtype=torch.bfloat16, device=o.device)
+    st = lib.csa_grouped_out_proj(_ptr(o), R, H, G, dg, _ptr(w), _ptr(y), _stream(stream))
+    _check(st, "csa_grouped_out_proj")
+    return y
+
+
+class Packed:
+    """Packed sequences (e.g. the documents of a packed pre-training batch) for one stride.
+
+    Built from the host-side sequence lengths: sequence s owns packed tokens [cu_tokens[s], cu_tokens[s+1])
+    and entries [cu_entries[s], cu_entries[s+1]) (ceil(len / stride) of them).  The offsets are uploaded once.
+    """
+
+    def __init__(self, lengths, stride, device="cuda"):
+        lens = [int(n) for n in lengths]
+        if any(n < 0 for n in lens):
+            raise ValueError("sequence lengths must be >= 0")
+        ent = [-(-n // stride) for n in lens]
+        cu_t, cu_e = [0], [0]
+        for n, e in zip(lens, ent):
+            cu_t.append(cu_t[-1] + n)
+            cu_e.append(cu_e[-1] + e)
+        self.lengths, self.stride = lens, stride
+        self.cu_tokens_host, self.cu_entries_host = cu_t, cu_e
+        self.cu_tokens = torch.tensor(cu_t, dtype=torch.int32, device=device)
+        self.cu_entries = torch.tensor(cu_e, dtype=torch.int32, device=device)
+        self.total_tokens, self.total_entries = cu_t[-1], cu_e[-1]
+        self.max_tokens = max(lens) if lens else 0
+
+    def desc(self) -> _lib.PackedDesc:
+        d = _lib.PackedDesc()
+        d.cu_tokens, d.cu_entries = _ptr(self.cu_tokens), _ptr(self.cu_entries)
+        d.n_seqs = len(self.lengths)
+        d.max_tokens = self.max_tokens
+        d.total_tokens, d.total_entries = self.total_tokens, self.total_entries
+        return d
+
+
+def _compress_append(fn_name, x, x_pos0, t, w, b_pos, stride, cache, stream):
+    lib = _lib.load()
+    B, rows, d = x.shape
+    if isinstance(cache, KVCache) and cache.split:
+        st = getattr(lib, fn_name)(_ptr(x), B, rows, x_pos0, t, d, stride, _ptr(w), _ptr(b_pos),
+                                   _lib.CSA_KV_SPLIT_FP8, _ptr(cache.nope), _ptr(cache.rope), _ptr(cache.scale),
+                                   cache.nope.shape[1], _stream(stream))
+    else:
+        k = cache.k if isinstance(cache, KVCache) else cache
+        st = getattr(lib, fn_name)(_ptr(x), B, rows, x_pos0, t, d, stride, _ptr(w), _ptr(b_pos), _lib.CSA_KV_BF16,
+                                   _ptr(k), None, None, k.shape[1], _stream(stream))
+    _check(st, fn_name)
+
+
+def csa_compress_append(x, x_pos0, t, w, b_pos, m, cache, *, stream=None):
+    """Decode-time append: if token t completes CSA entry i = (t+1)/m - 1, write it into cache slot i.
+
+    x bf16 [B, rows, d] holds raw tokens at positions x_pos0 ..; cache is a bf16 tensor [B, n_cap, d] or a split
+    FP8 KVCache (nope [B, n_cap, 128], rope, scale)."""
+    _compress_append("csa_compress_append", x, x_pos0, t, w, b_pos, m, cache, stream)
+
+
+def hca_compress_append(x, x_pos0, t, w, b_pos, m_prime, cache, *, stream=None):
+    """Decode-time append of the HCA entry that token t completes (t + 1 a multiple of m')."""
+    _compress_append("hca_compress_append", x, x_pos0, t, w, b_pos, m_prime, cache, stream)
+
+
+def _compress_packed(fn_name, x, packed: Packed, w, b_pos, stride, fp8, stream):
+    lib = _lib.load()
+    d = x.shape[-1]
+    E = packed.total_entries
+    pd = packed.desc()
+    if fp8:
+        nope = torch.empty(E, 128, dtype=torch.uint8, device=x.device)
+        rope = torch.empty(E, 64, dtype=torch.bfloat16, device=x.device)
+        scale = torch.empty(E, dtype=torch.float32, device=x.device)
+        st = getattr(lib, fn_name)(_ptr(x), ctypes.byref(pd), d, stride, _ptr(w), _ptr(b_pos), _lib.CSA_KV_SPLIT_FP8,
+                                   _ptr(nope), _ptr(rope), _ptr(scale), _stream(stream))
+        _check(st, fn_name)
+        return nope, rope, scale
+    y = torch.empty(E, d, dtype=torch.bfloat16, device=x.device)
+    st = getattr(lib, fn_name)(_ptr(x), ctypes.byref(pd), d, stride, _ptr(w), _ptr(b_pos), _lib.CSA_KV_BF16, _ptr(y),
+                               None, None, _stream(stream))
+    _check(st, fn_name)
+    return y
+
+
+def csa_compress_packed(x, packed: Packed, w, b_pos, m, *, fp8=False, stream=None):
+    """CSA compression of packed sequences x bf16 [total_tokens, d] -> entries [total_entries, d]."""
+    if packed.stride != m:
+        raise ValueError("packed descriptor was built for another stride")
+    return _compress_packed("csa_compress_packed", x, packed, w, b_pos, m, fp8, stream)
+
+
+def hca_compress_packed(x, packed: Packed, w, b_pos, m_prime, *, fp8=False, stream=None):
+    """HCA compression of packed sequences x bf16 [total_tokens, d] -> entries [total_entries, d]."""
+    if packed.stride != m_prime:
+        raise ValueError("packed descriptor was built for another stride")
+    return _compress_packed("hca_compress_packed", x, packed, w, b_pos, m_prime, fp8, stream)
+
+
+def csa_indexer_topk_packed(qI, wI, kIc, packed: Packed, m, k, *, idx=None, workspace=None, stream=None):
+    """Indexer top-k over packed sequences: qI [total_tokens, 4, 64] -> idx int32 [total_tokens, k] of entry
+    indices within each row's own sequence (ascending, -1 padded)."""
+    lib = _lib.load()
+    if packed.stride != m:
+        raise ValueError("packed descriptor was built for another stride")
+    pd = packed.desc()
+    if idx is None:
+        idx = torch.empty(packed.total_tokens, k, dtype=torch.int32, device=qI.device)
+    need = int(lib.csa_indexer_topk_packed_workspace_size(ctypes.byref(pd), m, k))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=qI.device)
+    st = lib.csa_indexer_topk_packed(_ptr(qI), _ptr(wI), _ptr(kIc), ctypes.byref(pd), m, k, _ptr(idx),
+                                     _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "csa_indexer_topk_packed")
+    return idx
+
+
+def _packed_window(k, v, packed, length):
+    return Window(k=k, v=v, pos0=0, length=length)
+
+
+def csa_sparse_mqa_packed(q, packed: Packed, cache: KVCache, m, idx, win_k, win_v, win_len, scale, *, out=None,
+                          lse=None, workspace=None, stream=None):
+    """CSA attention over packed sequences: q [total_tokens, H, 192]; the window is read from the packed raw
+    tokens win_k [total_tokens, 192] (win_v [total_tokens, 128] or None)."""
+    lib = _lib.load()
+    TT, H = q.shape[0], q.shape[1]
+    k = idx.shape[-1]
+    out = out if out is not None else torch.empty(TT, H, 128, dtype=torch.bfloat16, device=q.device)
+    lse = lse if lse is not None else torch.empty(TT, H, dtype=torch.float32, device=q.device)
+    need = csa_sparse_mqa_workspace_size(1, TT, H, k, win_len)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    pd, cd, wd = packed.desc(), cache.desc(), _packed_window(win_k, win_v, packed, win_len).desc()
+    st = lib.csa_sparse_mqa_packed(_ptr(q), H, ctypes.byref(pd), ctypes.byref(cd), m, _ptr(idx), k, ctypes.byref(wd),
+                                   float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                   0 if workspace is None else workspace.numel(), _stream(stream))
+    _check(st, "csa_sparse_mqa_packed")
+    return out, lse
+
+
+def hca_dense_mqa_packed(q, packed: Packed, cache: KVCache, m_prime, win_k, win_v, win_len, scale, *, out=None,
+                         lse=None, workspace=None, stream=None):
+    """HCA attention over packed sequences (every visible entry of the row's own sequence + its window)."""
+    lib = _lib.load()
+    TT, H = q.shape[0], q.shape[1]
+    out = out if out is not None else torch.empty(TT, H, 128, dtype=torch.bfloat16, device=q.device)
+    lse = lse if lse is not None else torch.empty(TT, H, dtype=torch.float32, device=q.device)
+    need = hca_dense_mqa_workspace_size(1, TT, H, -(-packed.max_tokens // m_prime), win_len)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    pd, cd, wd = packed.desc(), cache.desc(), _packed_window(win_k, win_v, packed, win_len).desc()
+    st = lib.hca_dense_mqa_packed(_ptr(q), H, ctypes.byref(pd), ctypes.byref(cd), m_prime, ctypes.byref(wd),
+                                  float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                  0 if workspace is None else workspace.numel(), _stream(stream))
+    _check(st, "hca_dense_mqa_packed")
     return out, lse

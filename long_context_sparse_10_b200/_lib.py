@@ -24,10 +24,23 @@ SIGNATURES = {
     "csa_debug_expire_wait": (c_i32, [c_vp]),
     "csa_compress": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "hca_compress": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
+    "csa_compress_append": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp,
+                                    c_vp, c_i64, c_vp]),
+    "hca_compress_append": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp,
+                                    c_vp, c_i64, c_vp]),
+    "csa_compress_packed": (c_i32, [c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
+    "hca_compress_packed": (c_i32, [c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "csa_indexer_topk_workspace_size": (c_sz, [c_i64, c_i64, c_i64, c_i32]),
+    "csa_indexer_topk_coded_workspace_size": (c_sz, [c_i64, c_i64, c_i64, c_i32]),
     "csa_indexer_topk": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp, c_sz,
                                  c_vp]),
     "csa_indexer_topk_e4m3": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp,
+                                      c_sz, c_vp]),
+    "csa_indexer_topk_with_scores": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp,
+                                             c_vp, c_sz, c_vp]),
+    "csa_cp_topk_merge": (c_i32, [c_vp, c_vp, c_i64, c_i32, c_i32, c_vp, c_vp]),
+    "csa_cp_attn_merge": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp]),
+    "csa_indexer_topk_e2m1": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp,
                                       c_sz, c_vp]),
     "csa_indexer_topk_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i32, c_i32, c_vp, c_vp]),
     "csa_sparse_mqa_workspace_size": (c_sz, [c_i64, c_i64, c_i32, c_i32, c_i32]),
@@ -36,6 +49,12 @@ SIGNATURES = {
     "hca_dense_mqa_workspace_size": (c_sz, [c_i64, c_i64, c_i32, c_i64, c_i32]),
     "hca_dense_mqa": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i64, c_vp, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_sz,
                               c_vp]),
+    "csa_grouped_out_proj": (c_i32, [c_vp, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]),
+    "csa_indexer_topk_packed_workspace_size": (c_sz, [c_vp, c_i32, c_i32]),
+    "csa_indexer_topk_packed": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_sz, c_vp]),
+    "csa_sparse_mqa_packed": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_i32, c_vp, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp,
+                                      c_sz, c_vp]),
+    "hca_dense_mqa_packed": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_sz, c_vp]),
 }
 
 
@@ -43,6 +62,12 @@ class KVCacheDesc(ctypes.Structure):
     """csa_kv_cache."""
     _fields_ = [("layout", c_i32), ("reserved", c_i32), ("n_entries", c_i64), ("k", c_vp), ("v", c_vp),
                 ("nope", c_vp), ("rope", c_vp), ("scale", c_vp)]
+
+
+class PackedDesc(ctypes.Structure):
+    """csa_packed."""
+    _fields_ = [("cu_tokens", c_vp), ("cu_entries", c_vp), ("n_seqs", c_i32), ("max_tokens", c_i32),
+                ("total_tokens", c_i64), ("total_entries", c_i64)]
 
 
 class WindowDesc(ctypes.Structure):

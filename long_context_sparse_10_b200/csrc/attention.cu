@@ -75,7 +75,38 @@ struct AttnParams {
   // units), sum l; merged by attn_merge_kernel.  Null: the CTAs of a row form
   // a thread-block cluster and merge through distributed shared memory.
   float* part;
+  // Packed sequences (nullable): query row r belongs to the sequence s that
+  // owns packed token r (cu_tok); its position is r - cu_tok[s], its entries
+  // are cache rows [cu_ent[s], cu_ent[s+1]) and its window tokens are rows
+  // cu_tok[s] + position of the raw-token buffer.
+  const int32_t* cu_tok;
+  const int32_t* cu_ent;
+  int n_seqs;
 };
+
+// Where one query row's keys live: its position t, the cache row of its entry
+// 0 (ebase) and its entry count N, and the raw-buffer row of position 0 (wbase).
+struct RowGeo {
+  int64_t t, ebase, N, wbase;
+};
+__device__ __forceinline__ RowGeo row_geo(const AttnParams& p, int64_t row) {
+  RowGeo g;
+  if (p.cu_tok != nullptr) {
+    const int s = seq_of(p.cu_tok, p.n_seqs, row);
+    const int64_t t0 = __ldg(p.cu_tok + s);
+    g.t = row - t0;
+    g.ebase = __ldg(p.cu_ent + s);
+    g.N = __ldg(p.cu_ent + s + 1) - g.ebase;
+    g.wbase = t0;
+  } else {
+    const int64_t b = row / p.Tq;
+    g.t = p.q_pos0 + row % p.Tq;
+    g.ebase = b * p.N;
+    g.N = p.N;
+    g.wbase = b * p.wrows - p.wpos0;
+  }
+  return g;
+}
 
 constexpr int kRec = kDV + 4;  // 128 channels, m, l, pad: 16-byte aligned records
 
@@ -137,13 +168,13 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
   const int hg = warp % HG, kg = warp / HG;
   const int64_t row = blockIdx.x / p.cl;
   const int split = static_cast<int>(blockIdx.x % p.cl);
-  const int64_t b = row / p.Tq;
-  const int64_t t = p.q_pos0 + row % p.Tq;
+  const RowGeo geo = row_geo(p, row);
+  const int64_t t = geo.t;
   const bool dense = p.idx == nullptr;
   int64_t n_ent;
   if (dense) {
     n_ent = (t + 1) / p.stride;
-    if (n_ent > p.N) n_ent = p.N;
+    if (n_ent > geo.N) n_ent = geo.N;
   } else {
     n_ent = p.k;
   }
@@ -184,13 +215,13 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
     if (s < s1) {
       if (s < n_ent) {
         const int64_t i = dense ? s : static_cast<int64_t>(idx_s[s - s0]);
-        if (i >= 0 && i < p.N && (i + 1) * p.stride - 1 <= t) {
+        if (i >= 0 && i < geo.N && (i + 1) * p.stride - 1 <= t) {
           type = 1;
-          r = b * p.N + i;
+          r = geo.ebase + i;
         }
       } else {
         type = 2;
-        r = b * p.wrows + (wlo + (s - n_ent) - p.wpos0);
+        r = geo.wbase + (wlo + (s - n_ent));
       }
     }
     stype[st][tid] = type;
@@ -580,13 +611,13 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t row = blockIdx.x / p.cl;
   const int split = static_cast<int>(blockIdx.x % p.cl);
-  const int64_t b = row / p.Tq;
-  const int64_t t = p.q_pos0 + row % p.Tq;
+  const RowGeo geo = row_geo(p, row);
+  const int64_t t = geo.t;
   const bool dense = p.idx == nullptr;
   int64_t n_ent;
   if (dense) {
     n_ent = (t + 1) / p.stride;
-    if (n_ent > p.N) n_ent = p.N;
+    if (n_ent > geo.N) n_ent = geo.N;
   } else {
     n_ent = p.k;
   }
@@ -671,8 +702,16 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   } else if (warp >= 8) {
     // ===================== producer: gather, widen, publish =====================
     const int pt = tid - 256;  // 0..255; threads 0..127 also own one slot each
+    // selected entry of this thread's slot in the next tile, loaded one tile
+    // ahead so that its latency overlaps the current tile's gathers
+    auto load_sel = [&](int tile) -> int32_t {
+      const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
+      return (!dense && pt < kTcKeys && tile < ntiles && sl < s1 && sl < n_ent) ? __ldg(p.idx + row * p.k + sl) : -1;
+    };
+    int32_t sel_next = load_sel(0);
     for (int tile = 0; tile < ntiles; ++tile) {
       const int st = tile % NS;
+      const int32_t sel_cur = sel_next;
       if (tile >= NS && healthy) healthy = tc::bar_wait(&empty[st], ((tile / NS) - 1) & 1);
       // slot -> (type, row): 0 skip, 1 compressed entry, 2 raw window token
       if (pt < kTcKeys) {
@@ -681,14 +720,14 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         int64_t r = 0;
         if (sl < s1) {
           if (sl < n_ent) {
-            const int64_t i = dense ? sl : static_cast<int64_t>(__ldg(p.idx + row * p.k + sl));
-            if (i >= 0 && i < p.N && (i + 1) * p.stride - 1 <= t) {
+            const int64_t i = dense ? sl : static_cast<int64_t>(sel_cur);
+            if (i >= 0 && i < geo.N && (i + 1) * p.stride - 1 <= t) {
               type = 1;
-              r = b * p.N + i;
+              r = geo.ebase + i;
             }
           } else {
             type = 2;
-            r = b * p.wrows + (wlo + (sl - n_ent) - p.wpos0);
+            r = geo.wbase + (wlo + (sl - n_ent));
           }
         }
         stype[st][pt] = type;
@@ -793,6 +832,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         }
       }
       cp_async_commit();
+      sel_next = load_sel(tile + 1);
       if (FP8) {  // code * scale -> bf16 into the swizzled K (and V) tile; skipped slots get zeros
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -1478,7 +1518,8 @@ csa_status check_cache(const char* name, const csa_kv_cache* c) {
 
 csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H, int64_t q_pos0,
                const csa_kv_cache* cache, int32_t stride, const int32_t* idx, int32_t k, const csa_window* win,
-               float scale, void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+               float scale, void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream,
+               const csa_packed* pk = nullptr) {
   clear_error();
   CSA_REQUIRE(B >= 0 && Tq >= 0, "%s: negative size", name);
   CSA_REQUIRE(H == 16 || H == 64, "%s: H must be 16 or 64 (got %d)", name, H);
@@ -1502,9 +1543,20 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
     CSA_REQUIRE(win->reserved == 0 && win->len >= 0, "%s: bad window descriptor", name);
     wlen = win->len;
   }
+  if (pk != nullptr) {
+    CSA_REQUIRE(pk->cu_tokens != nullptr && pk->cu_entries != nullptr && pk->n_seqs > 0,
+                "%s: packed offsets NULL or no sequences", name);
+    CSA_REQUIRE(cache->n_entries == pk->total_entries, "%s: cache->n_entries must equal packed->total_entries",
+                name);
+    CSA_REQUIRE(wlen == 0 || (win->pos0 == 0 && win->rows == pk->total_tokens),
+                "%s: with packed sequences the window buffer is the packed tokens (pos0 0, rows total_tokens)",
+                name);
+  }
   if (wlen > 0) {
     CSA_REQUIRE(win->k && aligned16(win->k), "%s: win->k NULL or misaligned", name);
     CSA_REQUIRE(!win->v || aligned16(win->v), "%s: win->v misaligned", name);
+  }
+  if (wlen > 0 && pk == nullptr) {
     const int64_t lo = (q_pos0 - wlen + 1) > 0 ? (q_pos0 - wlen + 1) : 0;
     const int64_t hi = q_pos0 + Tq - 1;
     CSA_REQUIRE(win->pos0 >= 0 && win->pos0 <= lo && hi < win->pos0 + win->rows,
@@ -1517,7 +1569,9 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   const bool cache_shared_v = fp8 || cache->v == nullptr;
   const bool win_shared_v = wlen == 0 || win->v == nullptr;
   const bool shv = cache_shared_v && win_shared_v;
-  const int64_t max_slots = (idx ? k : N) + wlen;
+  // slots of the longest row: k + window for CSA; for HCA every entry of the (longest) sequence + window
+  const int64_t n_dense = pk != nullptr ? (static_cast<int64_t>(pk->max_tokens) + stride - 1) / stride : N;
+  const int64_t max_slots = (idx ? k : n_dense) + wlen;
   // tcgen05 path for 64 heads; H = 16, and an FP8 cache combined with a separate
   // raw-window V (too much shared memory for the staged tiles), use the warp-MMA kernel
   const bool use_tc = H == 64 && !(fp8 && !shv);
@@ -1593,7 +1647,7 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   }
 
   // dense (HCA) prefill over a bf16 cache: query-blocked tcgen05 kernel
-  const bool use_blk = idx == nullptr && !fp8 && Tq >= 128 / H && R >= 2LL * num_sms();
+  const bool use_blk = idx == nullptr && !fp8 && Tq >= 128 / H && R >= 2LL * num_sms() && pk == nullptr;
   if (use_blk) {
     fn = attn_block_kernel;
     smem = blk_layout().total;
@@ -1628,6 +1682,9 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.part = part;
+  p.cu_tok = pk ? pk->cu_tokens : nullptr;
+  p.cu_ent = pk ? pk->cu_entries : nullptr;
+  p.n_seqs = pk ? pk->n_seqs : 0;
 
   const dim3 grid(static_cast<unsigned>(use_blk ? B * ((Tq + (128 / H) - 1) / (128 / H)) : R * pl.cl));
   const dim3 block(use_blk ? kTcThreads : (use_tc ? kTcDecThreads : kThreads));
@@ -1660,8 +1717,9 @@ csa_status csa_check_device_error(void* stream) {
   if (word != 0) {
     const int zero = 0;
     cudaMemcpyToSymbol(csa::tc::g_device_error, &zero, sizeof(int));
-    return csa::fail(CSA_ERR_DEVICE_TIMEOUT, "a kernel gave up waiting on a tensor-core barrier (code %d); its "
-                     "outputs are not valid", word);
+    return csa::fail(CSA_ERR_DEVICE_TIMEOUT, "a kernel gave up waiting on a barrier, or skipped work it could "
+                     "not do in bounds (code %d: 1 = a bounded wait ran out, 2 = a row longer than the row path "
+                     "holds); its outputs are not valid", word);
   }
   return CSA_OK;
 }
@@ -1694,6 +1752,24 @@ csa_status csa_sparse_mqa(const void* q, int64_t B, int64_t Tq, int32_t H, int64
     return csa::fail(CSA_ERR_INVALID_ARG, "csa_sparse_mqa: idx is NULL");
   return csa::run("csa_sparse_mqa", q, B, Tq, H, q_pos0, cache, m, idx, k, win, scale, out, lse, workspace,
                   workspace_bytes, stream);
+}
+
+csa_status csa_sparse_mqa_packed(const void* q, int32_t H, const csa_packed* packed, const csa_kv_cache* cache,
+                                 int32_t m, const int32_t* idx, int32_t k, const csa_window* win, float scale,
+                                 void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  if (packed == nullptr) return csa::fail(CSA_ERR_INVALID_ARG, "csa_sparse_mqa_packed: packed is NULL");
+  if (idx == nullptr && packed->total_tokens > 0)
+    return csa::fail(CSA_ERR_INVALID_ARG, "csa_sparse_mqa_packed: idx is NULL");
+  return csa::run("csa_sparse_mqa_packed", q, 1, packed->total_tokens, H, 0, cache, m, idx, k, win, scale, out, lse,
+                  workspace, workspace_bytes, stream, packed);
+}
+
+csa_status hca_dense_mqa_packed(const void* q, int32_t H, const csa_packed* packed, const csa_kv_cache* cache,
+                                int32_t m_prime, const csa_window* win, float scale, void* out, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (packed == nullptr) return csa::fail(CSA_ERR_INVALID_ARG, "hca_dense_mqa_packed: packed is NULL");
+  return csa::run("hca_dense_mqa_packed", q, 1, packed->total_tokens, H, 0, cache, m_prime, nullptr, 0, win, scale,
+                  out, lse, workspace, workspace_bytes, stream, packed);
 }
 
 csa_status hca_dense_mqa(const void* q, int64_t B, int64_t Tq, int32_t H, int64_t q_pos0, const csa_kv_cache* cache,

@@ -84,6 +84,14 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, 
       : "r"(codes));
 }
 
+// Two bytes of E2M1 codes (OCP MX FP4, two per byte, the low nibble first)
+// -> fp16 pairs (byte 0's two values) and (byte 1's two values), exactly.
+__device__ __forceinline__ void e2m1x4_to_f16x2x2(uint16_t two_bytes, uint32_t& lo, uint32_t& hi) {
+  asm("{\n.reg .b8 b0, b1;\nmov.b16 {b0, b1}, %2;\ncvt.rn.f16x2.e2m1x2 %0, b0;\ncvt.rn.f16x2.e2m1x2 %1, b1;\n}\n"
+      : "=r"(lo), "=r"(hi)
+      : "h"(two_bytes));
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -125,6 +133,18 @@ __device__ __forceinline__ int warp_sum_i(int v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+
+// Packed sequences: the largest s in [0, n) with cu[s] <= v (cu ascending,
+// cu[0] <= v), i.e. the sequence that owns packed row v of offsets cu.  Empty
+// sequences (equal consecutive offsets) are skipped over.
+__device__ __forceinline__ int seq_of(const int32_t* cu, int n, int64_t v) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= v) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 __device__ __forceinline__ uint4 ldg_nc16(const void* p) {

@@ -20,10 +20,18 @@ namespace csa {
 namespace {
 
 struct CompressParams {
-  const __nv_bfloat16* x;
+  const __nv_bfloat16* x;  // [B, xrows, d]: row j holds the token at position xpos0 + j
   const float* w;
   const float* b;
-  int64_t B, T, N;
+  int64_t B, T, N;  // tokens at positions < T exist; N entries computed per sequence
+  int64_t i0;       // index of the first entry computed
+  int64_t xpos0, xrows;
+  int64_t n_out;    // entries per sequence in the output (its row pitch)
+  // packed documents (nullable): sequence s = tokens [cu_tok[s], cu_tok[s+1]) of
+  // x (xrows = total tokens, B = 1) whose entries are out rows [cu_ent[s], cu_ent[s+1])
+  const int32_t* cu_tok;
+  const int32_t* cu_ent;
+  int n_seqs;
   int d, G;  // channels and 8-channel groups
   int stride, cwin;
   int layout;
@@ -31,6 +39,31 @@ struct CompressParams {
   __nv_bfloat16* out_rope;
   float* out_scale;
 };
+
+// Entry e of the launch -> (output row, entry index i in its sequence, x base
+// pointer at position 0 of the sequence, tokens T of the sequence).
+struct EntryRef {
+  int64_t out_row, i, T;
+  const __nv_bfloat16* x0;
+};
+__device__ __forceinline__ EntryRef entry_ref(const CompressParams& p, int64_t e) {
+  EntryRef r;
+  if (p.cu_tok != nullptr) {
+    const int s = seq_of(p.cu_ent, p.n_seqs, e);
+    const int64_t t0 = __ldg(p.cu_tok + s);
+    r.out_row = e;
+    r.i = e - __ldg(p.cu_ent + s);
+    r.T = __ldg(p.cu_tok + s + 1) - t0;
+    r.x0 = p.x + t0 * p.d;
+    return r;
+  }
+  const int64_t b = e / p.N;
+  r.i = p.i0 + e % p.N;
+  r.out_row = b * p.n_out + r.i;
+  r.T = p.T;
+  r.x0 = p.x + (b * p.xrows - p.xpos0) * p.d;
+  return r;
+}
 
 struct Acc8 {
   float m[8], s[8], a[8];
@@ -70,11 +103,9 @@ __device__ __forceinline__ void load8f(const float* p, float* f) {
   f[4] = v.x; f[5] = v.y; f[6] = v.z; f[7] = v.w;
 }
 
-// Writes entry (b, i).  Called by all 32 lanes; lane g < G holds channels
+// Writes output row e.  Called by all 32 lanes; lane g < G holds channels
 // [8g, 8g+8) in y.
-__device__ __forceinline__ void store_entry(const CompressParams& p, int64_t b, int64_t i, int lane,
-                                            const float* y) {
-  const int64_t e = b * p.N + i;
+__device__ __forceinline__ void store_entry(const CompressParams& p, int64_t e, int lane, const float* y) {
   if (p.layout == CSA_KV_BF16) {
     if (lane < p.G) {
       uint4 o;
@@ -126,17 +157,17 @@ __global__ void __launch_bounds__(256) compress_short_kernel(CompressParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t e = static_cast<int64_t>(blockIdx.x) * 8 + warp;
   if (e >= p.B * p.N) return;
-  const int64_t b = e / p.N, i = e % p.N;
-  const int64_t start = i * p.stride - (p.cwin - p.stride);
+  const EntryRef er = entry_ref(p, e);
+  const int64_t start = er.i * p.stride - (p.cwin - p.stride);
   const int64_t j0 = start > 0 ? start : 0;
-  const int64_t j1 = (start + p.cwin) < p.T ? (start + p.cwin) : p.T;
+  const int64_t j1 = (start + p.cwin) < er.T ? (start + p.cwin) : er.T;
   float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (lane < p.G) {
     float wv[8];
     load8f(p.w + 8 * lane, wv);
     Acc8 acc;
     acc.init();
-    const __nv_bfloat16* xb = p.x + b * p.T * p.d + 8 * lane;
+    const __nv_bfloat16* xb = er.x0 + 8 * lane;
     for (int64_t j = j0; j < j1; ++j) {
       float xv[8], bv[8];
       unpack8(ldg_nc16(xb + j * p.d), xv);
@@ -146,7 +177,49 @@ __global__ void __launch_bounds__(256) compress_short_kernel(CompressParams p) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) y[c] = acc.a[c] / acc.s[c];
   }
-  store_entry(p, b, i, lane, y);
+  store_entry(p, er.out_row, lane, y);
+}
+
+// bf16 output, windows of CW rows known at compile time: one thread per
+// (entry, 8-channel group), so every lane of every warp works whatever d is,
+// and the CW row loads of a thread are all issued before the softmax runs.
+// Consecutive threads read consecutive 16-byte chunks of a row.
+template <int CW>
+__global__ void __launch_bounds__(256) compress_flat_kernel(CompressParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t gidx = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  const int64_t e = gidx / p.G;
+  const int g = static_cast<int>(gidx % p.G);
+  if (e >= p.B * p.N) return;
+  const EntryRef er = entry_ref(p, e);
+  const int64_t start = er.i * p.stride - (CW - p.stride);
+  float wv[8];
+  load8f(p.w + 8 * g, wv);
+  const __nv_bfloat16* xb = er.x0 + 8 * g;
+  uint4 raw[CW];
+#pragma unroll
+  for (int r = 0; r < CW; ++r) {
+    const int64_t j = start + r;
+    raw[r] = (j >= 0 && j < er.T) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  Acc8 acc;
+  acc.init();
+#pragma unroll
+  for (int r = 0; r < CW; ++r) {
+    const int64_t j = start + r;
+    if (j < 0 || j >= er.T) continue;  // positions outside the sequence take no part
+    float xv[8], bv[8];
+    unpack8(raw[r], xv);
+    load8f(p.b + r * p.d + 8 * g, bv);
+    acc.add(xv, wv, bv);
+  }
+  uint4 o;
+  o.x = pack_bf16x2(acc.a[0] / acc.s[0], acc.a[1] / acc.s[1]);
+  o.y = pack_bf16x2(acc.a[2] / acc.s[2], acc.a[3] / acc.s[3]);
+  o.z = pack_bf16x2(acc.a[4] / acc.s[4], acc.a[5] / acc.s[5]);
+  o.w = pack_bf16x2(acc.a[6] / acc.s[6], acc.a[7] / acc.s[7]);
+  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + er.out_row * p.d + 8 * g) = o;
 }
 
 // One CTA per entry (long windows): 8 warps take interleaved rows, then warp 0
@@ -156,17 +229,16 @@ __global__ void __launch_bounds__(256) compress_long_kernel(CompressParams p) {
   pdl_trigger();
   __shared__ float st[8][3][8][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t e = blockIdx.x;
-  const int64_t b = e / p.N, i = e % p.N;
-  const int64_t start = i * p.stride - (p.cwin - p.stride);
+  const EntryRef er = entry_ref(p, blockIdx.x);
+  const int64_t start = er.i * p.stride - (p.cwin - p.stride);
   const int64_t j0 = start > 0 ? start : 0;
-  const int64_t j1 = (start + p.cwin) < p.T ? (start + p.cwin) : p.T;
+  const int64_t j1 = (start + p.cwin) < er.T ? (start + p.cwin) : er.T;
   Acc8 acc;
   acc.init();
   if (lane < p.G) {
     float wv[8];
     load8f(p.w + 8 * lane, wv);
-    const __nv_bfloat16* xb = p.x + b * p.T * p.d + 8 * lane;
+    const __nv_bfloat16* xb = er.x0 + 8 * lane;
 #pragma unroll 4
     for (int64_t j = j0 + warp; j < j1; j += 8) {
       float xv[8], bv[8];
@@ -198,20 +270,15 @@ __global__ void __launch_bounds__(256) compress_long_kernel(CompressParams p) {
     }
     y[c] = lane < p.G ? A / S : 0.f;
   }
-  store_entry(p, b, i, lane, y);
+  store_entry(p, er.out_row, lane, y);
 }
 
-csa_status compress_impl(const char* name, const void* x, int64_t B, int64_t T, int32_t d, int32_t stride,
-                         int32_t cwin, const float* w, const float* b_pos, int32_t layout, void* out,
-                         void* out_rope, float* out_scale, void* stream) {
-  clear_error();
-  CSA_REQUIRE(B >= 0 && T >= 0 && B < (1LL << 31) && T < (1LL << 40), "%s: B must be in [0, 2^31), T in [0, 2^40)",
-              name);
+csa_status check_args(const char* name, int32_t d, int32_t layout, const void* x, const float* w,
+                      const float* b_pos, const void* out, const void* out_rope, const float* out_scale) {
   CSA_REQUIRE(d >= 8 && d <= 256 && d % 8 == 0, "%s: d must be a multiple of 8 in [8, 256] (got %d)", name, d);
   CSA_REQUIRE(layout == CSA_KV_BF16 || layout == CSA_KV_SPLIT_FP8, "%s: unknown out_layout %d", name, layout);
   if (layout == CSA_KV_SPLIT_FP8 && d != kDQK)
     return fail(CSA_ERR_UNSUPPORTED, "%s: split FP8 output needs d == 192 (got %d)", name, d);
-  if (B == 0 || T == 0) return CSA_OK;
   CSA_REQUIRE_PTR(x);
   CSA_REQUIRE_PTR(w);
   CSA_REQUIRE_PTR(b_pos);
@@ -220,13 +287,20 @@ csa_status compress_impl(const char* name, const void* x, int64_t B, int64_t T, 
     CSA_REQUIRE_PTR(out_rope);
     CSA_REQUIRE_PTR(out_scale);
   }
+  return CSA_OK;
+}
+
+CompressParams base_params(const void* x, int32_t d, int32_t stride, int32_t cwin, const float* w,
+                           const float* b_pos, int32_t layout, void* out, void* out_rope, float* out_scale) {
   CompressParams p;
   p.x = static_cast<const __nv_bfloat16*>(x);
   p.w = w;
   p.b = b_pos;
-  p.B = B;
-  p.T = T;
-  p.N = (T + stride - 1) / stride;
+  p.i0 = 0;
+  p.xpos0 = 0;
+  p.cu_tok = nullptr;
+  p.cu_ent = nullptr;
+  p.n_seqs = 0;
   p.d = d;
   p.G = d / 8;
   p.stride = stride;
@@ -235,15 +309,98 @@ csa_status compress_impl(const char* name, const void* x, int64_t B, int64_t T, 
   p.out = out;
   p.out_rope = static_cast<__nv_bfloat16*>(out_rope);
   p.out_scale = out_scale;
+  return p;
+}
+
+csa_status launch(const char* name, const CompressParams& p, int64_t entries, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  CSA_REQUIRE(p.N < (1LL << 31) && B <= ((1LL << 31) - 1) / p.N, "%s: too many entries", name);
-  const int64_t entries = B * p.N;
   prof_begin(s);
-  const cudaError_t e =
-      cwin <= 32 ? launch_pdl(compress_short_kernel, dim3(static_cast<unsigned>((entries + 7) / 8)), dim3(256), 0, s, 1, p)
-                 : launch_pdl(compress_long_kernel, dim3(static_cast<unsigned>(entries)), dim3(256), 0, s, 1, p);
+  cudaError_t e;
+  if (p.layout == CSA_KV_BF16 && p.cwin == 8) {  // CSA with m = 4
+    const int64_t threads = entries * p.G;
+    e = launch_pdl(compress_flat_kernel<8>, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, s, 1,
+                   p);
+  } else if (p.cwin <= 32) {
+    e = launch_pdl(compress_short_kernel, dim3(static_cast<unsigned>((entries + 7) / 8)), dim3(256), 0, s, 1, p);
+  } else {
+    e = launch_pdl(compress_long_kernel, dim3(static_cast<unsigned>(entries)), dim3(256), 0, s, 1, p);
+  }
   prof_end(s);
   return check_launch(name, e);
+}
+
+csa_status compress_impl(const char* name, const void* x, int64_t B, int64_t T, int32_t d, int32_t stride,
+                         int32_t cwin, const float* w, const float* b_pos, int32_t layout, void* out,
+                         void* out_rope, float* out_scale, void* stream) {
+  clear_error();
+  CSA_REQUIRE(B >= 0 && T >= 0 && B < (1LL << 31) && T < (1LL << 40), "%s: B must be in [0, 2^31), T in [0, 2^40)",
+              name);
+  if (B == 0 || T == 0) return CSA_OK;
+  if (csa_status st = check_args(name, d, layout, x, w, b_pos, out, out_rope, out_scale); st != CSA_OK) return st;
+  CompressParams p = base_params(x, d, stride, cwin, w, b_pos, layout, out, out_rope, out_scale);
+  p.B = B;
+  p.T = T;
+  p.N = (T + stride - 1) / stride;
+  p.xrows = T;
+  p.n_out = p.N;
+  CSA_REQUIRE(p.N < (1LL << 31) && B <= ((1LL << 31) - 1) / p.N, "%s: too many entries", name);
+  return launch(name, p, B * p.N, stream);
+}
+
+// The entry completed by the token at position t (same t for every sequence of
+// the call), from a buffer of recent raw tokens, written into a resident cache.
+csa_status append_impl(const char* name, const void* x, int64_t B, int64_t rows, int64_t x_pos0, int64_t t,
+                       int32_t d, int32_t stride, int32_t cwin, const float* w, const float* b_pos, int32_t layout,
+                       void* out, void* out_rope, float* out_scale, int64_t n_cap, void* stream) {
+  clear_error();
+  CSA_REQUIRE(B >= 0 && B < (1LL << 31) && rows >= 0 && rows < (1LL << 40), "%s: bad B or rows", name);
+  CSA_REQUIRE(t >= 0 && t < (1LL << 50) && x_pos0 >= 0, "%s: t and x_pos0 must be >= 0", name);
+  CSA_REQUIRE(n_cap >= 0 && n_cap < (1LL << 31) && (B == 0 || n_cap <= ((1LL << 31) - 1) / B),
+              "%s: bad cache capacity", name);
+  if (B == 0 || (t + 1) % stride != 0) return CSA_OK;  // no entry completes at this token
+  const int64_t i = (t + 1) / stride - 1;
+  CSA_REQUIRE(i < n_cap, "%s: entry %lld does not fit a cache of %lld entries", name, static_cast<long long>(i),
+              static_cast<long long>(n_cap));
+  const int64_t start = i * stride - (cwin - stride);
+  const int64_t lo = start > 0 ? start : 0;
+  CSA_REQUIRE(x_pos0 <= lo && t - x_pos0 < rows,
+              "%s: raw rows [%lld, %lld) do not hold the entry's tokens [%lld, %lld]", name,
+              static_cast<long long>(x_pos0), static_cast<long long>(x_pos0 + rows), static_cast<long long>(lo),
+              static_cast<long long>(t));
+  if (csa_status st = check_args(name, d, layout, x, w, b_pos, out, out_rope, out_scale); st != CSA_OK) return st;
+  CompressParams p = base_params(x, d, stride, cwin, w, b_pos, layout, out, out_rope, out_scale);
+  p.B = B;
+  p.T = t + 1;
+  p.N = 1;
+  p.i0 = i;
+  p.xpos0 = x_pos0;
+  p.xrows = rows;
+  p.n_out = n_cap;
+  return launch(name, p, B, stream);
+}
+
+// Packed sequences: each sequence of the packed buffer is compressed on its own.
+csa_status packed_impl(const char* name, const void* x, const csa_packed* pk, int32_t d, int32_t stride,
+                       int32_t cwin, const float* w, const float* b_pos, int32_t layout, void* out, void* out_rope,
+                       float* out_scale, void* stream) {
+  clear_error();
+  CSA_REQUIRE(pk != nullptr, "%s: packed descriptor is NULL", name);
+  CSA_REQUIRE(pk->n_seqs >= 0 && pk->total_tokens >= 0 && pk->total_tokens < (1LL << 31) &&
+                  pk->total_entries >= 0 && pk->total_entries < (1LL << 31),
+              "%s: bad packed descriptor sizes", name);
+  if (pk->n_seqs == 0 || pk->total_entries == 0) return CSA_OK;
+  CSA_REQUIRE(pk->cu_tokens != nullptr && pk->cu_entries != nullptr, "%s: packed offsets are NULL", name);
+  if (csa_status st = check_args(name, d, layout, x, w, b_pos, out, out_rope, out_scale); st != CSA_OK) return st;
+  CompressParams p = base_params(x, d, stride, cwin, w, b_pos, layout, out, out_rope, out_scale);
+  p.B = 1;
+  p.T = pk->total_tokens;
+  p.N = pk->total_entries;
+  p.xrows = pk->total_tokens;
+  p.n_out = pk->total_entries;
+  p.cu_tok = pk->cu_tokens;
+  p.cu_ent = pk->cu_entries;
+  p.n_seqs = pk->n_seqs;
+  return launch(name, p, pk->total_entries, stream);
 }
 
 }  // namespace
@@ -266,6 +423,44 @@ csa_status hca_compress(const void* x, int64_t B, int64_t T, int32_t d, int32_t 
     return csa::fail(CSA_ERR_INVALID_ARG, "hca_compress: m' must be in [1, 4096] (got %d)", m_prime);
   return csa::compress_impl("hca_compress", x, B, T, d, m_prime, m_prime, w, b_pos, out_layout, out, out_rope,
                             out_scale, stream);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+csa_status csa_compress_append(const void* x, int64_t B, int64_t rows, int64_t x_pos0, int64_t t, int32_t d,
+                               int32_t m, const float* w, const float* b_pos, int32_t out_layout, void* out,
+                               void* out_rope, float* out_scale, int64_t n_cap, void* stream) {
+  if (m < 1 || m > 64) return csa::fail(CSA_ERR_INVALID_ARG, "csa_compress_append: m must be in [1, 64] (got %d)", m);
+  return csa::append_impl("csa_compress_append", x, B, rows, x_pos0, t, d, m, 2 * m, w, b_pos, out_layout, out,
+                          out_rope, out_scale, n_cap, stream);
+}
+
+csa_status hca_compress_append(const void* x, int64_t B, int64_t rows, int64_t x_pos0, int64_t t, int32_t d,
+                               int32_t m_prime, const float* w, const float* b_pos, int32_t out_layout, void* out,
+                               void* out_rope, float* out_scale, int64_t n_cap, void* stream) {
+  if (m_prime < 1 || m_prime > 4096)
+    return csa::fail(CSA_ERR_INVALID_ARG, "hca_compress_append: m' must be in [1, 4096] (got %d)", m_prime);
+  return csa::append_impl("hca_compress_append", x, B, rows, x_pos0, t, d, m_prime, m_prime, w, b_pos, out_layout,
+                          out, out_rope, out_scale, n_cap, stream);
+}
+
+csa_status csa_compress_packed(const void* x, const csa_packed* packed, int32_t d, int32_t m, const float* w,
+                               const float* b_pos, int32_t out_layout, void* out, void* out_rope, float* out_scale,
+                               void* stream) {
+  if (m < 1 || m > 64) return csa::fail(CSA_ERR_INVALID_ARG, "csa_compress_packed: m must be in [1, 64] (got %d)", m);
+  return csa::packed_impl("csa_compress_packed", x, packed, d, m, 2 * m, w, b_pos, out_layout, out, out_rope,
+                          out_scale, stream);
+}
+
+csa_status hca_compress_packed(const void* x, const csa_packed* packed, int32_t d, int32_t m_prime, const float* w,
+                               const float* b_pos, int32_t out_layout, void* out, void* out_rope, float* out_scale,
+                               void* stream) {
+  if (m_prime < 1 || m_prime > 4096)
+    return csa::fail(CSA_ERR_INVALID_ARG, "hca_compress_packed: m' must be in [1, 4096] (got %d)", m_prime);
+  return csa::packed_impl("hca_compress_packed", x, packed, d, m_prime, m_prime, w, b_pos, out_layout, out, out_rope,
+                          out_scale, stream);
 }
 
 }  // extern "C"

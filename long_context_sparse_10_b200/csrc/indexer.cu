@@ -36,8 +36,13 @@ namespace csa {
 namespace {
 
 constexpr int kMaxK = 4096;
+// Key formats of the scoring kernels: bf16 keys, or coded keys with one fp32
+// scale per entry -- E4M3 (64 bytes per entry) or E2M1 (FP4, 32 bytes).
+constexpr int kKeyBF16 = 0, kKeyE4M3 = 1, kKeyE2M1 = 2;
+__host__ __device__ constexpr int code_bytes(int kf) { return kf == kKeyE2M1 ? 32 : 64; }
 constexpr int kRowPathMaxN = 32768;  // rows up to this many visible entries live in shared memory
 constexpr int kHistBins = 4096;      // first-level bins: top 12 bits of the key
+constexpr int kErrRowTooLong = 2;    // device error word: a row-path row longer than its shared memory
 // Scoring pipeline shape (compile-time tunables): stages of kTileRows entries
 // (128 B each) per CTA of kScoreThreads threads; each warp owns 16 rows of a stage.
 #ifndef CSA_SCORE_STAGES
@@ -64,7 +69,22 @@ struct ScoreParams {
   uint32_t* done;   // [R, 2] CTA counters (QR == 1 only)
   int32_t* thr;     // [R, 2] threshold (QR == 1 only)
   int k;
+  int64_t pitch;    // row pitch of scores (N, or the longest packed sequence's entries)
+  // packed sequences (nullable): sequence s owns query rows [cu_tok[s],
+  // cu_tok[s+1]) (positions from 0) and key rows [cu_ent[s], cu_ent[s+1]);
+  // CTA row y of the grid is the s-th sequence's group y - cu_grp[s] of QR rows
+  const int32_t* cu_tok;
+  const int32_t* cu_ent;
+  const int32_t* cu_grp;
+  int n_seqs;
 };
+
+__device__ __forceinline__ void named_sync_ix(int id, int n) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
 
 __device__ __forceinline__ int64_t visible(int64_t t, int m, int64_t N) {
   int64_t v = (t + 1) / m;
@@ -134,8 +154,14 @@ __device__ __forceinline__ void find_digit_256(const uint32_t* hist, uint32_t re
   }
 }
 
-__device__ __forceinline__ void write_prefix_ids(int32_t* out, int64_t nv, int k) {
-  for (int j = threadIdx.x; j < k; j += blockDim.x) out[j] = j < nv ? j : -1;
+// The whole visible prefix [0, nv) selected (nv <= k), -1 padded; with a
+// score output, each slot also gets the entry's score (-inf for padding).
+__device__ __forceinline__ void write_prefix_ids(int32_t* out, int64_t nv, int k, float* sout = nullptr,
+                                                 const float* srow = nullptr) {
+  for (int j = threadIdx.x; j < k; j += blockDim.x) {
+    out[j] = j < nv ? j : -1;
+    if (sout != nullptr) sout[j] = j < nv ? __ldcg(srow + j) : -INFINITY;
+  }
 }
 
 // Threshold of one row from its global histogram, by one CTA of NT threads
@@ -187,9 +213,38 @@ __device__ void row_threshold(const uint32_t* gh, int64_t nv, int k, int32_t* th
 // Shared memory of the scoring kernel: bf16 keys: kStages swizzled tiles;
 // E4M3 keys: kStages stages of codes + scales, twice the entries per stage
 // (same bytes per stage); then the histogram (HIST).
-__host__ __device__ constexpr size_t score_tile_bytes(bool e4) {
-  return e4 ? static_cast<size_t>(kStages) * (2 * kTileRows) * (64 + 4)
-            : static_cast<size_t>(kStages) * kTileRows * 128;
+__host__ __device__ constexpr size_t score_tile_bytes(int kf) {
+  return kf != kKeyBF16 ? static_cast<size_t>(kStages) * (2 * kTileRows) * (code_bytes(kf) + 4)
+                        : static_cast<size_t>(kStages) * kTileRows * 128;
+}
+
+// A fragments (fp16) of one 16-entry MMA tile of coded keys for k-step kk:
+// the lane's entry row g (codes at `row`) and g + 8, dimensions 16t + 4kk ..
+// 16t + 4kk + 3 (the permuted order described below).
+template <int KF>
+__device__ __forceinline__ void key_frags(const uint8_t* row, int t, uint32_t (&af)[4][4]) {
+  constexpr int CB = code_bytes(KF);
+  if constexpr (KF == kKeyE4M3) {  // 16 codes = dims 16t .. 16t+15, one byte each
+    const uint4 lo = *reinterpret_cast<const uint4*>(row + t * 16);
+    const uint4 hi = *reinterpret_cast<const uint4*>(row + 8 * CB + t * 16);
+    const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      e4m3x4_to_f16x2x2(wl[kk], af[kk][0], af[kk][2]);
+      e4m3x4_to_f16x2x2(wh[kk], af[kk][1], af[kk][3]);
+    }
+  } else {  // E2M1: 8 bytes = dims 16t .. 16t+15, two per byte (low nibble = even dim)
+    const uint2 lo = *reinterpret_cast<const uint2*>(row + t * 8);
+    const uint2 hi = *reinterpret_cast<const uint2*>(row + 8 * CB + t * 8);
+    const uint32_t wl[2] = {lo.x, lo.y}, wh[2] = {hi.x, hi.y};
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint16_t bl = static_cast<uint16_t>(wl[kk >> 1] >> (16 * (kk & 1)));
+      const uint16_t bh = static_cast<uint16_t>(wh[kk >> 1] >> (16 * (kk & 1)));
+      e2m1x4_to_f16x2x2(bl, af[kk][0], af[kk][2]);
+      e2m1x4_to_f16x2x2(bh, af[kk][1], af[kk][3]);
+    }
+  }
 }
 
 // E4M3 keys feed an fp16 MMA straight from registers.  The dot product over
@@ -201,25 +256,46 @@ __host__ __device__ constexpr size_t score_tile_bytes(bool e4) {
 // [2^14, 2^15) before the fp16 conversion (exact for every bf16 value in that
 // head down to 2^-28 of its maximum), and 2^-e moves onto the head weight:
 // relu(2^e x) 2^-e w = relu(x) w.
-template <int QR, bool E4>
+template <int QR, int KF>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
   pdl_wait();
   pdl_trigger();
+  constexpr bool E4 = KF != kKeyBF16;  // coded keys (E4M3 or E2M1) with a per-entry scale
+  constexpr int CB = code_bytes(KF);   // code bytes per entry
   constexpr int NCOL = QR * 4;
   constexpr int NT = (NCOL + 7) / 8;
   constexpr int TR = E4 ? 2 * kTileRows : kTileRows;  // entries per stage
   constexpr int MT = TR / kTileRows;                  // 16-row MMA tiles per warp and stage
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* tiles = smem;                                             // bf16: [kStages] swizzled tiles
-  uint8_t* codes_st = smem;                                          // E4: [kStages][TR][64]
-  float* scale_st = reinterpret_cast<float*>(smem + kStages * TR * 64);  // E4: [kStages][TR]
+  uint8_t* codes_st = smem;                                          // coded: [kStages][TR][CB]
+  float* scale_st = reinterpret_cast<float*>(smem + kStages * TR * CB);  // coded: [kStages][TR]
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t groups = (p.Tq + QR - 1) / QR;
-  const int64_t b = blockIdx.y / groups;
-  const int64_t r0 = (blockIdx.y % groups) * QR;
-  const int nrows = static_cast<int>((p.Tq - r0) < QR ? (p.Tq - r0) : QR);
-  const int64_t nv_max = visible(p.q_pos0 + r0 + nrows - 1, p.m, p.N);
+  // this CTA's QR query rows: global rows qrow0.., positions t0.., keys ebase.. (Nseq of them)
+  int64_t qrow0, t0, ebase, Nseq;
+  int nrows;
+  if (p.cu_tok != nullptr) {
+    const int64_t gy = blockIdx.y;
+    if (gy >= __ldg(p.cu_grp + p.n_seqs)) return;
+    const int sq = seq_of(p.cu_grp, p.n_seqs, gy);
+    const int64_t len = __ldg(p.cu_tok + sq + 1) - __ldg(p.cu_tok + sq);
+    t0 = (gy - __ldg(p.cu_grp + sq)) * QR;
+    qrow0 = __ldg(p.cu_tok + sq) + t0;
+    nrows = static_cast<int>((len - t0) < QR ? (len - t0) : QR);
+    ebase = __ldg(p.cu_ent + sq);
+    Nseq = __ldg(p.cu_ent + sq + 1) - ebase;
+  } else {
+    const int64_t groups = (p.Tq + QR - 1) / QR;
+    const int64_t b = blockIdx.y / groups;
+    const int64_t r0 = (blockIdx.y % groups) * QR;
+    qrow0 = b * p.Tq + r0;
+    t0 = p.q_pos0 + r0;
+    nrows = static_cast<int>((p.Tq - r0) < QR ? (p.Tq - r0) : QR);
+    ebase = b * p.N;
+    Nseq = p.N;
+  }
+  const int64_t nv_max = visible(t0 + nrows - 1, p.m, Nseq);
   const int64_t e_begin = static_cast<int64_t>(blockIdx.x) * p.chunk;
   if (e_begin >= nv_max) return;  // uniform for the CTA
   const int64_t e_end = (e_begin + p.chunk) < nv_max ? (e_begin + p.chunk) : nv_max;
@@ -232,7 +308,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
     const int n = nt * 8 + (lane >> 2);
     const int rr = n >> 2, h = n & 3;
     const bool ok = n < NCOL && rr < nrows;
-    const __nv_bfloat16* qrow = p.qI + (((b * p.Tq + r0 + (ok ? rr : 0)) * kHI + h) * kDI);
+    const __nv_bfloat16* qrow = p.qI + (((qrow0 + (ok ? rr : 0)) * kHI + h) * kDI);
     if (E4) {
       const __nv_bfloat16* qp = qrow + (lane & 3) * 16;
       float qv[16];
@@ -271,7 +347,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
   for (int nt = 0; nt < NT; ++nt) {
     const int rr = nt * 2 + ((lane & 3) >> 1);
     const bool ok = rr < nrows && nt * 8 < NCOL && (rr * 4) < NCOL;
-    const int64_t row = b * p.Tq + r0 + (ok ? rr : 0);
+    const int64_t row = qrow0 + (ok ? rr : 0);
     const int h0 = (lane & 1) * 2;
     wv[nt][0] = ok ? p.wI[row * kHI + h0] : 0.f;
     wv[nt][1] = ok ? p.wI[row * kHI + h0 + 1] : 0.f;
@@ -281,28 +357,29 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
       wv[nt][0] *= __uint_as_float(static_cast<uint32_t>(127 - e0) << 23);
       wv[nt][1] *= __uint_as_float(static_cast<uint32_t>(127 - e1) << 23);
     }
-    nv_r[nt] = ok ? visible(p.q_pos0 + r0 + rr, p.m, p.N) : 0;
+    nv_r[nt] = ok ? visible(t0 + rr, p.m, Nseq) : 0;
     srow[nt] = row;
   }
 
   const int ntiles = static_cast<int>((e_end - e_begin + TR - 1) / TR);
-  const __nv_bfloat16* kbase = p.kI + b * p.N * kDI;
+  const __nv_bfloat16* kbase = p.kI + ebase * kDI;
   auto load_tile = [&](int tile, int stage) {
     const int64_t base = e_begin + static_cast<int64_t>(tile) * TR;
     if constexpr (E4) {
-      // 64 code bytes per entry (4 pieces) and one 4-byte scale per entry
-      for (int piece = threadIdx.x; piece < TR * 4; piece += kScoreThreads) {
-        const int row = piece >> 2, ch = piece & 3;
+      // CB code bytes per entry (CB / 16 pieces) and one 4-byte scale per entry
+      constexpr int PPE = CB / 16;
+      for (int piece = threadIdx.x; piece < TR * PPE; piece += kScoreThreads) {
+        const int row = piece / PPE, ch = piece % PPE;
         const int64_t e = base + row;
         const bool ok = e < e_end;
-        cp_async16(codes_st + (stage * TR + row) * 64 + ch * 16,
-                   p.kcodes + (b * p.N + (ok ? e : e_begin)) * kDI + ch * 16, ok ? 16 : 0);
+        cp_async16(codes_st + (stage * TR + row) * CB + ch * 16,
+                   p.kcodes + (ebase + (ok ? e : e_begin)) * CB + ch * 16, ok ? 16 : 0);
       }
       for (int row = threadIdx.x; row < TR; row += kScoreThreads) {
         const int64_t e = base + row;
         if (e < e_end) {
           asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(scale_st + stage * TR + row)),
-                       "l"(p.kscale + b * p.N + e));
+                       "l"(p.kscale + ebase + e));
         } else {
           scale_st[stage * TR + row] = 0.f;
         }
@@ -341,17 +418,13 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
       if (E4) {
-        const uint8_t* cs = codes_st + ((tile % kStages) * TR + rbase + (lane >> 2)) * 64 + (lane & 3) * 16;
-        const uint4 lo = *reinterpret_cast<const uint4*>(cs);
-        const uint4 hi = *reinterpret_cast<const uint4*>(cs + 8 * 64);
-        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+        uint32_t af[4][4];
+        key_frags<KF>(codes_st + ((tile % kStages) * TR + rbase + (lane >> 2)) * CB, lane & 3, af);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          uint32_t a0, a1, a2, a3;
-          e4m3x4_to_f16x2x2(wl[kk], a0, a2);
-          e4m3x4_to_f16x2x2(wh[kk], a1, a3);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_f16(acc[nt], a0, a1, a2, a3, bq[kk][nt][0], bq[kk][nt][1]);
+          for (int nt = 0; nt < NT; ++nt)
+            mma_f16(acc[nt], af[kk][0], af[kk][1], af[kk][2], af[kk][3], bq[kk][nt][0], bq[kk][nt][1]);
         }
       } else {
         const uint8_t* st = tiles + (tile % kStages) * (kTileRows * 128);
@@ -377,7 +450,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(ScoreParams p) {
             full *= scale_st[(tile % kStages) * TR + rbase + (lane >> 2) + hf * 8];
           full += 0.0f;
           if ((lane & 1) == 0 && e < nv_r[nt]) {
-            p.scores[srow[nt] * p.N + e] = full;
+            p.scores[srow[nt] * p.pitch + e] = full;
           }
         }
       }
@@ -408,10 +481,11 @@ constexpr int kLongMaxChunk = 65536 - kLongTR;  // per-CTA bin counts fit 16 bit
 #ifndef CSA_LONG_STAGES_E4
 #define CSA_LONG_STAGES_E4 4
 #endif
-template <bool E4>
+template <int KF>
 struct LongShape {
+  static constexpr bool E4 = KF != kKeyBF16;
   static constexpr int kStages = E4 ? CSA_LONG_STAGES_E4 : CSA_LONG_STAGES_BF16;
-  static constexpr int kStageBytes = kLongTR * (E4 ? 64 : 128);
+  static constexpr int kStageBytes = kLongTR * (E4 ? code_bytes(KF) : 128);
   static constexpr size_t kScaleOff = static_cast<size_t>(kStages) * kStageBytes;
   static constexpr size_t kHistOff = kScaleOff + (E4 ? static_cast<size_t>(kStages) * kLongTR * 4 : 0);
   static constexpr size_t kBarOff = kHistOff + kHistBins * 2;  // two 16-bit bins per word
@@ -434,11 +508,13 @@ struct LongScoreParams {
   int k;
 };
 
-template <bool E4>
+template <int KF>
 __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParams p,
                                                                   const __grid_constant__ CUtensorMap kmap) {
   pdl_wait();
-  using S = LongShape<E4>;
+  using S = LongShape<KF>;
+  constexpr bool E4 = S::E4;  // coded keys (E4M3 or E2M1) with a per-entry scale
+  constexpr int CB = code_bytes(KF);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   float* scale_st = reinterpret_cast<float*>(smem + S::kScaleOff);  // E4: [kStages][kLongTR]
@@ -515,8 +591,8 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
     if (E4) {
       const int rows = static_cast<int>((e_end - base) < kLongTR ? (e_end - base) : kLongTR);
       if (threadIdx.x == 0) {
-        tc::bar_arrive_expect_tx(&bars[st], static_cast<uint32_t>(rows) * 64u);
-        tc::bulk_load_stream(dst, p.kcodes + (b * p.N + base) * kDI, static_cast<uint32_t>(rows) * 64u, &bars[st],
+        tc::bar_arrive_expect_tx(&bars[st], static_cast<uint32_t>(rows) * CB);
+        tc::bulk_load_stream(dst, p.kcodes + (b * p.N + base) * CB, static_cast<uint32_t>(rows) * CB, &bars[st],
                              tc::l2_evict_first_policy());
       }
       const int r = threadIdx.x;  // kLongThreads == kLongTR: one scale per thread
@@ -569,17 +645,10 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
       acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
       const int rbase = warp * 32 + mt * 16;
       if (E4) {
-        const uint8_t* cs = smem + st * S::kStageBytes + (rbase + g) * 64 + t * 16;
-        const uint4 lo = *reinterpret_cast<const uint4*>(cs);
-        const uint4 hi = *reinterpret_cast<const uint4*>(cs + 8 * 64);
-        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+        uint32_t af[4][4];
+        key_frags<KF>(smem + st * S::kStageBytes + (rbase + g) * CB, t, af);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          uint32_t a0, a1, a2, a3;
-          e4m3x4_to_f16x2x2(wl[kk], a0, a2);
-          e4m3x4_to_f16x2x2(wh[kk], a1, a3);
-          mma_f16(acc[mt], a0, a1, a2, a3, bq[kk][0], bq[kk][1]);
-        }
+        for (int kk = 0; kk < 4; ++kk) mma_f16(acc[mt], af[kk][0], af[kk][1], af[kk][2], af[kk][3], bq[kk][0], bq[kk][1]);
       } else {
         const uint8_t* stg = smem + st * S::kStageBytes;
         const int r = rbase + (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -649,8 +718,18 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
 // ---------------------------------------------------------------------------
 // row path: one CTA (1024 threads) per query row, row held in shared memory
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) topk_rows_kernel(const float* __restrict__ scores, int64_t N, int64_t Tq,
-                                                         int64_t q_pos0, int m, int k, int32_t* __restrict__ idx) {
+struct RowsParams {
+  const float* scores;
+  int64_t pitch, N, Tq, q_pos0;
+  int m, k;
+  int32_t* idx;
+  const int32_t* cu_tok;  // packed sequences (nullable): as ScoreParams
+  const int32_t* cu_ent;
+  int n_seqs;
+  float* sout;            // nullable: [R, k] score of each selected entry
+};
+
+__global__ void __launch_bounds__(1024) topk_rows_kernel(RowsParams p) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint32_t keys[];
@@ -658,13 +737,26 @@ __global__ void __launch_bounds__(1024) topk_rows_kernel(const float* __restrict
   __shared__ uint32_t dig[3];
   __shared__ uint32_t scan_sh[32];
   const int64_t row = blockIdx.x;
-  const int64_t nv = visible(q_pos0 + row % Tq, m, N);
-  int32_t* out = idx + row * k;
+  int64_t nv;
+  if (p.cu_tok != nullptr) {
+    const int sq = seq_of(p.cu_tok, p.n_seqs, row);
+    nv = visible(row - __ldg(p.cu_tok + sq), p.m, __ldg(p.cu_ent + sq + 1) - __ldg(p.cu_ent + sq));
+  } else {
+    nv = visible(p.q_pos0 + row % p.Tq, p.m, p.N);
+  }
+  const int k = p.k;
+  int32_t* out = p.idx + row * k;
+  float* sout = p.sout != nullptr ? p.sout + row * k : nullptr;
+  const float* srow = p.scores + row * p.pitch;
   if (nv <= k) {
-    write_prefix_ids(out, nv, k);
+    write_prefix_ids(out, nv, k, sout, srow);
     return;
   }
-  const float* srow = scores + row * N;
+  if (nv > kRowPathMaxN) {  // cannot happen for sizes the host admits; never index past the shared row
+    if (threadIdx.x == 0) atomicExch(&tc::g_device_error, kErrRowTooLong);
+    write_prefix_ids(out, 0, k, sout, srow);
+    return;
+  }
   for (int64_t i = threadIdx.x; i < nv; i += blockDim.x) keys[i] = f2key(srow[i]);
   uint32_t prefix = 0, mask = 0, remaining = static_cast<uint32_t>(k);
   for (int shift = 24; shift >= 0; shift -= 8) {
@@ -694,10 +786,344 @@ __global__ void __launch_bounds__(1024) topk_rows_kernel(const float* __restrict
     const bool sel = gt || (eq && tie_rank < remaining);
     uint32_t sel_total;
     const uint32_t pos = sel_before + block_excl_scan(sel ? 1u : 0u, &sel_total, scan_sh);
-    if (sel) out[pos] = static_cast<int32_t>(i);
+    if (sel) {
+      out[pos] = static_cast<int32_t>(i);
+      if (sout != nullptr) sout[pos] = srow[i];
+    }
     ties_before += tie_total;
     sel_before += sel_total;
   }
+}
+
+// ---------------------------------------------------------------------------
+// prefill rows with bf16 keys: tcgen05 scoring, scores kept on chip
+// ---------------------------------------------------------------------------
+// One CTA owns kPfQ consecutive query rows of one sequence.  The MMA computes
+// S^T = K Q^T with the entries as M (128 per tile, one per TMEM lane) and the
+// (query, head) pairs as N (kPfQ * 4 = 128 columns), K = 64; an epilogue
+// thread owns one entry of the tile and folds its 4 heads per query
+// (s_q = sum_h relu(S[e, 4q+h]) w[q, h]), so it holds the tile's scores of
+// every query of the CTA in registers.  The exact top-k is a radix select on
+// the order-preserving 32-bit score key, refined over passes that recompute
+// the same scores (the MMA is cheap; the scores never leave the SM):
+//   pass 0: per-query histogram of the key's top 11 bits;
+//   pass 1: 11 more bits, for entries in the query's threshold bin;
+//   pass 2: the last 10 bits, likewise;
+//   pass 3: emission -- every entry above the threshold, and the first `need`
+//           entries equal to it (ascending index, so ties go to the lower
+//           index), written as the ascending list by ordered ballots.
+// A query whose threshold bin is taken whole stops refining early; a pass
+// that no query needs only waits for its tiles.  The key tiles stream by TMA
+// (128-byte swizzle, no multicast) through a ring of stages, one thread
+// issues the MMAs into two TMEM buffers, and all waits are bounded.
+constexpr int kPfQ = 32;         // query rows per CTA (x 4 heads = 128 MMA columns)
+constexpr int kPfTile = 128;     // entries per tile (MMA M)
+constexpr int kPfStages = 4;
+constexpr int kPfThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kPfBins = 2048;    // histogram bins per query (11 bits)
+
+struct PfLayout {
+  static constexpr size_t kK = 0;                                  // [kPfStages][128 entries][128 B]
+  static constexpr size_t kQ = kK + kPfStages * 16384;             // [128 (query, head)][128 B]
+  static constexpr size_t kHist = kQ + 16384;                      // [kPfQ][kPfBins / 2] u32 (two u16 bins)
+  static constexpr size_t kW = kHist + kPfQ * (kPfBins / 2) * 4;   // [128] fp32
+  static constexpr size_t kCnt = kW + 128 * 4;                     // tie / sel counts [2][2][4][kPfQ] u32
+  static constexpr size_t kQs = kCnt + 2 * 2 * 4 * kPfQ * 4;       // per-query state, 8 x [kPfQ] u32
+  static constexpr size_t kBars = kQs + 8 * kPfQ * 4;
+  static constexpr size_t kTotal = kBars + 128 + 1024;             // + alignment slack
+};
+
+struct PfParams {
+  const __nv_bfloat16* qI;  // [B, Tq, 4, 64]
+  const float* wI;          // [B, Tq, 4]
+  int64_t Tq, N, q_pos0;
+  int m, k;
+  int64_t groups;           // CTAs: B * ceil(Tq / kPfQ)
+  int32_t* idx;             // [B, Tq, k]
+};
+
+__global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams p,
+                                                                        const __grid_constant__ CUtensorMap kmap) {
+  pdl_wait();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* Kst = smem + PfLayout::kK;
+  uint8_t* Qs = smem + PfLayout::kQ;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + PfLayout::kHist);
+  float* w_s = reinterpret_cast<float*>(smem + PfLayout::kW);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + PfLayout::kCnt);  // [par][tie/sel][q4][j]
+  uint32_t* qs = reinterpret_cast<uint32_t*>(smem + PfLayout::kQs);
+  uint32_t* nv_s = qs;                 // visible entries of query j
+  uint32_t* level_s = qs + kPfQ;       // 0..2: refining at that pass; 3: threshold known
+  uint32_t* prefix_s = qs + 2 * kPfQ;  // key bits fixed so far (levels 1, 2)
+  uint32_t* rem_s = qs + 3 * kPfQ;     // entries still to take at the current level
+  uint32_t* shift_s = qs + 4 * kPfQ;   // emission: compare key >> shift with thr, take need ties
+  uint32_t* thr_s = qs + 5 * kPfQ;
+  uint32_t* need_s = qs + 6 * kPfQ;
+  uint32_t* base_s = qs + 7 * kPfQ;    // emission: entries written so far
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + PfLayout::kBars);  // [kPfStages]
+  uint64_t* empty = full + kPfStages;                                     // [kPfStages]
+  uint64_t* tfull = empty + kPfStages;                                    // [2]
+  uint64_t* tempty = tfull + 2;                                           // [2]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
+  __shared__ uint32_t tie_base_s[kPfQ];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t gpb = (p.Tq + kPfQ - 1) / kPfQ;
+  const int64_t grp = p.groups - 1 - static_cast<int64_t>(blockIdx.x);  // late (long) rows first
+  const int64_t b = grp / gpb;
+  const int64_t r0 = (grp % gpb) * kPfQ;
+  const int nq = static_cast<int>((p.Tq - r0) < kPfQ ? (p.Tq - r0) : kPfQ);
+  const int64_t row0 = b * p.Tq + r0;  // global row of query 0
+  const int64_t nv_max = visible(p.q_pos0 + r0 + nq - 1, p.m, p.N);
+  const int k = p.k;
+
+  if (tid < kPfQ) {
+    const int j = tid;
+    const uint32_t nv = j < nq ? static_cast<uint32_t>(visible(p.q_pos0 + r0 + j, p.m, p.N)) : 0u;
+    nv_s[j] = nv;
+    const bool partial = nv > static_cast<uint32_t>(k);
+    level_s[j] = partial ? 0u : 3u;
+    prefix_s[j] = 0u;
+    rem_s[j] = static_cast<uint32_t>(k);
+    shift_s[j] = 0u;   // with thr 0 every visible key (>= 0x007fffff) is above: all visible entries
+    thr_s[j] = 0u;
+    need_s[j] = 0u;
+    base_s[j] = 0u;
+    tie_base_s[j] = 0u;
+  }
+  if (nv_max <= k) {  // every row of the CTA keeps all its visible entries: no scoring at all
+    __syncthreads();
+    for (int i = tid; i < nq * k; i += kPfThreads) {
+      const int j = i / k, c = i % k;
+      p.idx[(row0 + j) * k + c] = c < static_cast<int>(nv_s[j]) ? c : -1;
+    }
+    return;
+  }
+  const int ntiles = static_cast<int>((nv_max + kPfTile - 1) / kPfTile);
+  constexpr int kPasses = 4;
+
+  if (tid == 0) {
+    for (int i = 0; i < kPfStages; ++i) {
+      tc::bar_init(&full[i], 1);
+      tc::bar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::bar_init(&tfull[i], 1);
+      tc::bar_init(&tempty[i], 128);
+    }
+    tc::bar_init_fence();
+  }
+  if (warp == 1) tc::tmem_alloc(tslot, 256);
+  // Q: row n = (query n/4, head n%4), 64 dims = 128 B, swizzled K-major; rows past nq are zero
+  for (int piece = tid; piece < 128 * 8; piece += kPfThreads) {
+    const int n = piece >> 3, ch = piece & 7;
+    const bool ok = (n >> 2) < nq;
+    cp_async16(Qs + tc::sw128(n, ch), ok ? p.qI + ((row0 + (n >> 2)) * kHI + (n & 3)) * kDI + ch * 8 : p.qI,
+               ok ? 16 : 0);
+  }
+  cp_async_commit();
+  if (tid < 128) w_s[tid] = (tid >> 2) < nq ? p.wI[(row0 + (tid >> 2)) * kHI + (tid & 3)] : 0.f;
+  for (int i = tid; i < kPfQ * kPfBins / 2; i += kPfThreads) hist[i] = 0u;
+  cp_async_wait<0>();
+  tc::fence_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tslot;
+  const int total = kPasses * ntiles;
+
+  if (warp == 0) {
+    // ===================== TMA producer: the same tiles, once per pass =====================
+    if (lane == 0) {
+      for (int it = 0; it < total; ++it) {
+        const int st = it % kPfStages;
+        if (it >= kPfStages && !tc::bar_wait(&empty[st], static_cast<uint32_t>(((it / kPfStages) - 1) & 1))) break;
+        tc::bar_arrive_expect_tx(&full[st], 16384u);
+        tc::tma_load_3d(Kst + st * 16384, &kmap, 0, (it % ntiles) * kPfTile, static_cast<int>(b), &full[st]);
+      }
+    }
+  } else if (warp == 1) {
+    // ===================== MMA issue (one thread) =====================
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16(128, 128, false, false);
+      const uint32_t qa = smem_u32(Qs);
+      for (int it = 0; it < total; ++it) {
+        const int st = it % kPfStages, buf = it & 1;
+        if (it >= 2 && !tc::bar_wait(&tempty[buf], static_cast<uint32_t>(((it >> 1) - 1) & 1))) break;
+        if (!tc::bar_wait(&full[st], static_cast<uint32_t>((it / kPfStages) & 1))) break;
+        tc::fence_after_sync();
+        const uint32_t ka = smem_u32(Kst + st * 16384);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_bf16_ss(tmem + static_cast<uint32_t>(buf * 128), tc::desc_sw128(ka + kk * 32, 16, 1024),
+                          tc::desc_sw128(qa + kk * 32, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        tc::mma_commit(&empty[st]);
+        tc::mma_commit(&tfull[buf]);
+      }
+    }
+  } else {
+    // ===================== epilogue: thread = entry of the tile =====================
+    const int q4 = warp & 3;  // TMEM lane quarter of this warp
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    const int et = q4 * 32 + lane;  // entry within the tile
+    const int etid = tid - 64;      // 0..127
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    // A wait that runs out (recorded in the device error word) skips the later
+    // waits but keeps the loop and its named barriers, so the four warps stay
+    // in step and the CTA finishes; its output is then not valid.
+    bool healthy = true;
+    int it = 0;
+    for (int pass = 0; pass < kPasses; ++pass) {
+      // does any query refine at this pass (passes 0-2)?  pass 3 always emits
+      bool active = pass == 3;
+      if (!active) {
+        for (int j = 0; j < kPfQ; ++j) active |= level_s[j] == static_cast<uint32_t>(pass);
+      }
+      for (int tile = 0; tile < ntiles; ++tile, ++it) {
+        const int buf = it & 1;
+        if (healthy) healthy = tc::bar_wait(&tfull[buf], static_cast<uint32_t>((it >> 1) & 1));
+        tc::fence_after_sync();
+        const uint32_t e = static_cast<uint32_t>(tile * kPfTile + et);
+        uint32_t gt_m = 0u, eq_m = 0u;  // emission: per query, this entry above / at the threshold
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {  // 8 queries (32 accumulator columns) at a time
+          float v[32];
+          if (active) tc::tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 128 + c * 32), v);
+          if (c == 3) {
+            tc::fence_before_sync();
+            bar_arrive(&tempty[buf]);
+          }
+          if (!active) continue;
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int j = c * 8 + jj;
+            const float4 w4 = *reinterpret_cast<const float4*>(w_s + 4 * j);
+            const float sc = fmaxf(v[4 * jj], 0.f) * w4.x + fmaxf(v[4 * jj + 1], 0.f) * w4.y +
+                             fmaxf(v[4 * jj + 2], 0.f) * w4.z + fmaxf(v[4 * jj + 3], 0.f) * w4.w;
+            const uint32_t key = f2key(sc + 0.0f);
+            const bool vis = e < nv_s[j];
+            const uint32_t lv = level_s[j];
+            if (pass == 0) {
+              if (vis && lv == 0u) {
+                const uint32_t bin = key >> 21;
+                atomicAdd(&hist[j * (kPfBins / 2) + (bin >> 1)], 1u << ((bin & 1u) * 16));
+              }
+            } else if (pass == 1) {
+              if (vis && lv == 1u && (key >> 21) == prefix_s[j]) {
+                const uint32_t bin = (key >> 10) & 2047u;
+                atomicAdd(&hist[j * (kPfBins / 2) + (bin >> 1)], 1u << ((bin & 1u) * 16));
+              }
+            } else if (pass == 2) {
+              if (vis && lv == 2u && (key >> 10) == prefix_s[j]) {
+                const uint32_t bin = key & 1023u;
+                atomicAdd(&hist[j * (kPfBins / 2) + (bin >> 1)], 1u << ((bin & 1u) * 16));
+              }
+            } else {
+              const uint32_t kk = key >> shift_s[j];
+              const uint32_t th = thr_s[j];
+              gt_m |= (vis && kk > th) ? (1u << j) : 0u;
+              eq_m |= (vis && kk == th) ? (1u << j) : 0u;
+            }
+          }
+        }
+        if (!active || pass < 3) continue;
+        // ---- emission of this tile, in ascending entry order across the 4 warps ----
+        const int par = tile & 1;
+        uint32_t* tcnt = cnt + (par * 2 + 0) * 4 * kPfQ;
+        uint32_t* scnt = cnt + (par * 2 + 1) * 4 * kPfQ;
+        for (int j = 0; j < kPfQ; ++j) {
+          const uint32_t eb = __ballot_sync(0xffffffffu, (eq_m >> j) & 1u);
+          if (lane == 0) tcnt[q4 * kPfQ + j] = __popc(eb);
+        }
+        named_sync_ix(3, 128);
+        uint32_t sel_m = 0u;
+        for (int j = 0; j < kPfQ; ++j) {
+          const uint32_t eb = __ballot_sync(0xffffffffu, (eq_m >> j) & 1u);
+          uint32_t off = tie_base_s[j];
+          for (int w = 0; w < q4; ++w) off += tcnt[w * kPfQ + j];
+          const uint32_t rank = off + __popc(eb & lt_mask);
+          const bool eq = (eq_m >> j) & 1u;
+          const bool sel = ((gt_m >> j) & 1u) || (eq && rank < need_s[j]);
+          sel_m |= sel ? (1u << j) : 0u;
+          const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+          if (lane == 0) scnt[q4 * kPfQ + j] = __popc(sb);
+        }
+        // entries written so far per query, read before the barrier (updated after it)
+        const uint32_t my_base = lane < kPfQ ? base_s[lane] : 0u;
+        named_sync_ix(3, 128);
+        for (int j = 0; j < kPfQ; ++j) {
+          const uint32_t sb = __ballot_sync(0xffffffffu, (sel_m >> j) & 1u);
+          if (sb == 0u) continue;
+          uint32_t pos = __shfl_sync(0xffffffffu, my_base, j);
+          for (int w = 0; w < q4; ++w) pos += scnt[w * kPfQ + j];
+          pos += __popc(sb & lt_mask);
+          if (((sel_m >> j) & 1u) && pos < static_cast<uint32_t>(k)) p.idx[(row0 + j) * k + pos] = static_cast<int32_t>(e);
+        }
+        named_sync_ix(3, 128);
+        if (etid < kPfQ) {  // running totals of this tile's ties and selections
+          const int j = etid;
+          tie_base_s[j] += tcnt[j] + tcnt[kPfQ + j] + tcnt[2 * kPfQ + j] + tcnt[3 * kPfQ + j];
+          base_s[j] += scnt[j] + scnt[kPfQ + j] + scnt[2 * kPfQ + j] + scnt[3 * kPfQ + j];
+        }
+      }
+      if (pass == 3) break;
+      // ---- thresholds of the queries that refined in this pass ----
+      named_sync_ix(3, 128);
+      const int nb = pass == 2 ? 1024 : 2048;
+      const int per_lane = nb / 32;  // bins per lane, walked from the top
+      for (int j = q4; j < kPfQ; j += 4) {
+        if (level_s[j] != static_cast<uint32_t>(pass)) continue;  // uniform in the warp
+        const uint32_t* h = hist + j * (kPfBins / 2);
+        const int hi = nb - lane * per_lane;  // this lane's bins [hi - per_lane, hi)
+        uint32_t sum = 0;
+        for (int bb = hi - 1; bb >= hi - per_lane; --bb) sum += (h[bb >> 1] >> ((bb & 1) * 16)) & 0xffffu;
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const uint32_t excl = incl - sum;
+        const uint32_t rem = rem_s[j];
+        if (excl < rem && incl >= rem) {
+          uint32_t acc = excl;
+          for (int bb = hi - 1; bb >= hi - per_lane; --bb) {
+            const uint32_t c = (h[bb >> 1] >> ((bb & 1) * 16)) & 0xffffu;
+            if (acc + c >= rem) {
+              const uint32_t nrem = rem - acc;  // still needed from bin bb
+              const uint32_t pref = pass == 0 ? static_cast<uint32_t>(bb)
+                                              : (prefix_s[j] << (pass == 1 ? 11 : 10)) | static_cast<uint32_t>(bb);
+              if (c == nrem || pass == 2) {  // threshold found: ties at it are taken in index order
+                shift_s[j] = pass == 0 ? 21u : (pass == 1 ? 10u : 0u);
+                thr_s[j] = pref;
+                need_s[j] = nrem;
+                level_s[j] = 3u;
+              } else {
+                prefix_s[j] = pref;
+                rem_s[j] = nrem;
+                level_s[j] = static_cast<uint32_t>(pass + 1);
+              }
+              break;
+            }
+            acc += c;
+          }
+        }
+      }
+      named_sync_ix(3, 128);  // every warp is done reading the histograms
+      for (int i = etid; i < kPfQ * kPfBins / 2; i += 128) hist[i] = 0u;
+      named_sync_ix(3, 128);
+    }
+    named_sync_ix(3, 128);  // the last tile's running totals are in base_s
+    // padding after each query's selection
+    for (int j = 0; j < nq; ++j) {
+      const uint32_t done = base_s[j] < static_cast<uint32_t>(k) ? base_s[j] : static_cast<uint32_t>(k);
+      for (uint32_t c = done + etid; c < static_cast<uint32_t>(k); c += 128) p.idx[(row0 + j) * k + c] = -1;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) tc::tmem_dealloc(tmem, 256);
 }
 
 // ---------------------------------------------------------------------------
@@ -734,7 +1160,8 @@ struct LongWs {
 // ascending index list.  Rows up to kBitmapSmemWords*32 entries keep that final
 // bitmap in shared memory.
 __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, int64_t N, int64_t Tq, int64_t q_pos0,
-                                                                     int m, int k, int32_t* __restrict__ idx) {
+                                                                     int m, int k, int32_t* __restrict__ idx,
+                                                                     float* __restrict__ scores_out) {
   pdl_wait();
   extern __shared__ __align__(16) uint8_t sel_smem[];  // candidates, then the final bitmap
   uint2* cand_s = reinterpret_cast<uint2*>(sel_smem);
@@ -746,14 +1173,16 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   const int64_t nv = visible(q_pos0 + row % Tq, m, N);
   const int64_t e_begin = static_cast<int64_t>(blockIdx.x) * kSelChunk;
   int32_t* out = idx + row * k;
+  float* sout = scores_out != nullptr ? scores_out + row * k : nullptr;
+  const float* srow = ws.scores + row * ws.pitch;
   if (nv == 0) {  // no entry visible yet (the scoring kernel skipped the row): all padding
-    if (blockIdx.x == 0) write_prefix_ids(out, 0, k);
+    if (blockIdx.x == 0) write_prefix_ids(out, 0, k, sout, srow);
     return;
   }
   if (e_begin >= nv) return;
   const int thr_bin = ws.thr[2 * row];
   if (thr_bin < 0) {  // every visible entry is selected
-    if (blockIdx.x == 0) write_prefix_ids(out, nv, k);
+    if (blockIdx.x == 0) write_prefix_ids(out, nv, k, sout, srow);
     return;
   }
   const int64_t e_end = (e_begin + kSelChunk) < nv ? (e_begin + kSelChunk) : nv;
@@ -763,7 +1192,6 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   __syncthreads();
   // warp w scans entries [e_begin + 512 w, e_begin + 512 (w + 1)), four per
   // lane per step (16-byte loads; rows are 16-byte aligned and padded)
-  const float* srow = ws.scores + row * ws.pitch;
   constexpr int kSelWarps = kSelThreads / 32;
   constexpr int kPerWarp = kSelChunk / kSelWarps;
   constexpr int kSteps = kPerWarp / 128;
@@ -971,7 +1399,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
       while (word) {
         const int bit = __ffs(word) - 1;
         word &= word - 1;
-        if (p < static_cast<uint32_t>(k)) out[p] = e0 + 32 * j + bit;
+        if (p < static_cast<uint32_t>(k)) {
+          out[p] = e0 + 32 * j + bit;
+          if (sout != nullptr) sout[p] = __ldcg(srow + e0 + 32 * j + bit);
+        }
         ++p;
       }
     }
@@ -996,7 +1427,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
     while (word) {
       const int bit = __ffs(word) - 1;
       word &= word - 1;
-      if (p < static_cast<uint32_t>(k)) out[p] = static_cast<int32_t>((wi << 5) + bit);
+      if (p < static_cast<uint32_t>(k)) {
+        out[p] = static_cast<int32_t>((wi << 5) + bit);
+        if (sout != nullptr) sout[p] = __ldcg(srow + (wi << 5) + bit);
+      }
       ++p;
     }
   }
@@ -1039,10 +1473,12 @@ int64_t query_rows(int64_t B, int64_t Tq) {
   return B * Tq;
 }
 
-size_t workspace_bytes(int64_t B, int64_t Tq, int64_t N) {
+// Workspace of the bf16-key call (coded = false) or of the E4M3 / E2M1 calls.
+// Prefill rows with bf16 keys keep their scores on chip and need none.
+size_t workspace_bytes(int64_t B, int64_t Tq, int64_t N, bool coded = false) {
   const int64_t R = query_rows(B, Tq);
   if (R <= 0 || N <= 0 || N >= (int64_t(1) << 31)) return 0;
-  if (use_row_path(R, N)) return align_up(static_cast<size_t>(R) * N * 4);
+  if (use_row_path(R, N)) return coded ? align_up(static_cast<size_t>(R) * N * 4) : 0;
   return long_layout(R, N).total;
 }
 
@@ -1067,18 +1503,124 @@ extern "C" {
 size_t csa_indexer_topk_workspace_size(int64_t B, int64_t Tq, int64_t N, int32_t k) {
   (void)k;
   if (B < 0 || Tq < 0 || N < 0) return 0;
-  return csa::workspace_bytes(B, Tq, N);
+  return csa::workspace_bytes(B, Tq, N, false);
+}
+
+size_t csa_indexer_topk_coded_workspace_size(int64_t B, int64_t Tq, int64_t N, int32_t k) {
+  (void)k;
+  if (B < 0 || Tq < 0 || N < 0) return 0;
+  return csa::workspace_bytes(B, Tq, N, true);
 }
 
 }  // extern "C"
 
 namespace csa {
 namespace {
+constexpr int kRowGroup = 8;  // query rows per scoring CTA on the row path
+
+__global__ void fill_kernel(float* __restrict__ dst, int64_t n, float v) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = v;
+}
+
+// Scoring kernel over `groups` groups of query rows, then one top-k CTA per row.
+csa_status launch_row_path(const char* name, ScoreParams& p, const RowsParams& rp, int64_t groups, int64_t R,
+                           int64_t max_n, int kf, cudaStream_t s) {
+  p.chunk = 2048;
+  dim3 grid(static_cast<unsigned>((max_n + p.chunk - 1) / p.chunk), static_cast<unsigned>(groups));
+  const dim3 block(kScoreThreads);
+  prof_begin(s);
+  const cudaError_t e =
+      kf == kKeyE4M3   ? launch_pdl(score_kernel<kRowGroup, kKeyE4M3>, grid, block, score_tile_bytes(kf), s, 1, p)
+      : kf == kKeyE2M1 ? launch_pdl(score_kernel<kRowGroup, kKeyE2M1>, grid, block, score_tile_bytes(kf), s, 1, p)
+                       : launch_pdl(score_kernel<kRowGroup, kKeyBF16>, grid, block, score_tile_bytes(kf), s, 1, p);
+  prof_end(s);
+  if (csa_status st = check_launch(name, e); st != CSA_OK) return st;
+  const size_t smem = static_cast<size_t>(max_n) * 4;
+  if (!ensure_smem(reinterpret_cast<const void*>(topk_rows_kernel), kRowPathMaxN * 4))
+    return fail(CSA_ERR_CUDA, "%s: cannot raise shared memory limit", name);
+  return check_launch(name, launch_pdl(topk_rows_kernel, dim3(static_cast<unsigned>(R)), dim3(1024), smem, s, 1, rp));
+}
+
+// Offsets of each packed sequence's first group of kRowGroup query rows.
+__global__ void __launch_bounds__(1024) group_table_kernel(const int32_t* __restrict__ cu_tok, int n,
+                                                           int32_t* __restrict__ cu_grp) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ uint32_t scan_sh[32];
+  uint32_t carry = 0;
+  if (threadIdx.x == 0) cu_grp[0] = 0;
+  for (int base = 0; base < n; base += 1024) {
+    const int sq = base + static_cast<int>(threadIdx.x);
+    const uint32_t v = sq < n ? static_cast<uint32_t>(cu_tok[sq + 1] - cu_tok[sq] + kRowGroup - 1) / kRowGroup : 0u;
+    uint32_t total;
+    const uint32_t ex = block_excl_scan(v, &total, scan_sh);
+    if (sq < n) cu_grp[sq + 1] = static_cast<int32_t>(carry + ex + v);
+    carry += total;
+  }
+}
+
+csa_status encode_key_map(CUtensorMap* kmap, const void* kIc, int64_t B, int64_t N, const char* name) {
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return fail(CSA_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
+  CSA_REQUIRE(aligned16(kIc), "%s: kIc must be 16-byte aligned", name);
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDI), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDI) * 2, static_cast<cuuint64_t>(N) * kDI * 2};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kDI), 128u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = encode(kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kIc), dims, strides, box,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "%s: tensor map encoding failed (%d)", name, int(r));
+  return CSA_OK;
+}
+
+csa_status launch_prefill_tc(const void* qI, const float* wI, const void* kIc, int64_t B, int64_t Tq, int64_t N,
+                             int64_t q_pos0, int32_t m, int32_t k, int32_t* idx, cudaStream_t s) {
+  CUtensorMap kmap;
+  memset(&kmap, 0, sizeof(kmap));
+  if (csa_status st = encode_key_map(&kmap, kIc, B, N, "csa_indexer_topk"); st != CSA_OK) return st;
+  PfParams p;
+  p.qI = static_cast<const __nv_bfloat16*>(qI);
+  p.wI = wI;
+  p.Tq = Tq;
+  p.N = N;
+  p.q_pos0 = q_pos0;
+  p.m = m;
+  p.k = k;
+  p.groups = B * ((Tq + kPfQ - 1) / kPfQ);
+  p.idx = idx;
+  if (!ensure_smem(reinterpret_cast<const void*>(indexer_prefill_kernel), static_cast<int>(PfLayout::kTotal)))
+    return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise the shared memory limit");
+  prof_begin(s);
+  const cudaError_t e = launch_pdl(indexer_prefill_kernel, dim3(static_cast<unsigned>(p.groups)), dim3(kPfThreads),
+                                   PfLayout::kTotal, s, 1, p, kmap);
+  prof_end(s);
+  return check_launch("csa_indexer_topk (prefill, tcgen05)", e);
+}
+
+struct PackedLayout {
+  size_t scores, grp, total;
+  int64_t pitch;
+};
+PackedLayout packed_layout(const csa_packed* pk, int32_t m) {
+  PackedLayout L;
+  L.pitch = ((static_cast<int64_t>(pk->max_tokens) + m - 1) / m + 3) / 4 * 4;
+  L.scores = 0;
+  L.grp = align_up(static_cast<size_t>(pk->total_tokens) * L.pitch * 4);
+  L.total = align_up(L.grp + (static_cast<size_t>(pk->n_seqs) + 1) * 4);
+  return L;
+}
+
 csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const uint8_t* kcodes, const float* kscale,
                         int64_t B, int64_t Tq, int64_t N, int64_t q_pos0, int32_t m, int32_t k, int32_t* idx,
-                        void* workspace, size_t workspace_bytes, void* stream) {
+                        void* workspace, size_t workspace_bytes, void* stream, float* scores_out = nullptr,
+                        int kf = kKeyBF16) {
   clear_error();
-  const bool e4 = kcodes != nullptr;
+  const bool e4 = kcodes != nullptr;  // coded keys (kf: E4M3 or E2M1)
+  if (!e4) kf = kKeyBF16;
   CSA_REQUIRE(B >= 0 && Tq >= 0 && N >= 0, "csa_indexer_topk: negative size");
   CSA_REQUIRE(N < (1LL << 31), "csa_indexer_topk: N must be < 2^31");
   CSA_REQUIRE(m >= 1, "csa_indexer_topk: m must be >= 1");
@@ -1092,6 +1634,9 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   if (N == 0) {
     if (cudaMemsetAsync(idx, 0xff, static_cast<size_t>(R) * k * 4, s) != cudaSuccess)
       return fail(CSA_ERR_CUDA, "csa_indexer_topk: memset failed");
+    if (scores_out != nullptr)
+      return check_launch("csa_indexer_topk", launch_pdl(fill_kernel, dim3(static_cast<unsigned>((R * k + 255) / 256)),
+                                                         dim3(256), 0, s, 1, scores_out, R * k, -INFINITY));
     return CSA_OK;
   }
   CSA_REQUIRE_PTR(qI);
@@ -1103,11 +1648,13 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   } else {
     CSA_REQUIRE_PTR(kIc);
   }
-  const size_t need = csa::workspace_bytes(B, Tq, N);
-  if (workspace == nullptr || workspace_bytes < need)
+  const bool tc_rows = !e4 && scores_out == nullptr && use_row_path(R, N);  // tcgen05 prefill path
+  const size_t need = tc_rows ? 0 : csa::workspace_bytes(B, Tq, N, true);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
     return fail(CSA_ERR_WORKSPACE, "csa_indexer_topk: workspace of %zu bytes needed (got %zu)", need,
                 workspace_bytes);
-  CSA_REQUIRE(aligned16(workspace), "csa_indexer_topk: workspace is not 16-byte aligned");
+  CSA_REQUIRE(need == 0 || aligned16(workspace), "csa_indexer_topk: workspace is not 16-byte aligned");
+  if (tc_rows) return launch_prefill_tc(qI, wI, kIc, B, Tq, N, q_pos0, m, k, idx, s);
 
   ScoreParams p;
   p.qI = static_cast<const __nv_bfloat16*>(qI);
@@ -1119,31 +1666,22 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   p.N = N;
   p.q_pos0 = q_pos0;
   p.m = m;
+  p.pitch = N;
+  p.cu_tok = p.cu_ent = p.cu_grp = nullptr;
+  p.n_seqs = 0;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t tile_smem = static_cast<size_t>(kStages) * kTileRows * 128;
 
   if (use_row_path(R, N)) {
-    constexpr int QR = 8;
-    p.chunk = 2048;
+    constexpr int QR = kRowGroup;
     p.scores = reinterpret_cast<float*>(ws);
     p.hist = nullptr;
     p.done = nullptr;
     p.thr = nullptr;
     p.k = k;
     const int64_t groups = (Tq + QR - 1) / QR;
-    dim3 grid(static_cast<unsigned>((N + p.chunk - 1) / p.chunk), static_cast<unsigned>(B * groups));
     CSA_REQUIRE(B * groups < 65536, "csa_indexer_topk: too many query rows for one launch");
-    prof_begin(s);
-    const cudaError_t e = e4 ? launch_pdl(score_kernel<QR, true>, grid, dim3(kScoreThreads), score_tile_bytes(true), s, 1, p)
-                             : launch_pdl(score_kernel<QR, false>, grid, dim3(kScoreThreads), tile_smem, s, 1, p);
-    prof_end(s);
-    if (csa_status st = check_launch("indexer score", e); st != CSA_OK) return st;
-    const size_t smem = static_cast<size_t>(N) * 4;
-    if (!ensure_smem(reinterpret_cast<const void*>(topk_rows_kernel), kRowPathMaxN * 4))
-      return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
-    return check_launch("indexer top-k (rows)",
-                        launch_pdl(topk_rows_kernel, dim3(static_cast<unsigned>(R)), dim3(1024), smem, s, 1,
-                                   static_cast<const float*>(p.scores), N, Tq, q_pos0, m, k, idx));
+    RowsParams rp{p.scores, N, N, Tq, q_pos0, m, k, idx, nullptr, nullptr, 0, scores_out};
+    return launch_row_path("csa_indexer_topk", p, rp, B * groups, R, N, kf, s);
   }
 
   const LongLayout L = long_layout(R, N);
@@ -1193,9 +1731,12 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   } else {
     CSA_REQUIRE(aligned16(kcodes), "csa_indexer_topk: key codes must be 16-byte aligned");
   }
-  const void* skern = e4 ? reinterpret_cast<const void*>(score_long_kernel<true>)
-                        : reinterpret_cast<const void*>(score_long_kernel<false>);
-  const size_t ssmem = e4 ? LongShape<true>::kSmem : LongShape<false>::kSmem;
+  const void* skern = kf == kKeyE4M3   ? reinterpret_cast<const void*>(score_long_kernel<kKeyE4M3>)
+                      : kf == kKeyE2M1 ? reinterpret_cast<const void*>(score_long_kernel<kKeyE2M1>)
+                                       : reinterpret_cast<const void*>(score_long_kernel<kKeyBF16>);
+  const size_t ssmem = kf == kKeyE4M3   ? LongShape<kKeyE4M3>::kSmem
+                       : kf == kKeyE2M1 ? LongShape<kKeyE2M1>::kSmem
+                                        : LongShape<kKeyBF16>::kSmem;
   if (!ensure_smem(skern, static_cast<int>(ssmem)))
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
   // one wave: the row's chunks spread over every resident CTA slot
@@ -1209,8 +1750,10 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   lp.chunk = static_cast<int>(chunk);
   dim3 grid(static_cast<unsigned>((N + chunk - 1) / chunk), static_cast<unsigned>(R));
   prof_begin(s);
-  const cudaError_t e = e4 ? launch_pdl(score_long_kernel<true>, grid, dim3(kLongThreads), ssmem, s, 1, lp, kmap)
-                           : launch_pdl(score_long_kernel<false>, grid, dim3(kLongThreads), ssmem, s, 1, lp, kmap);
+  const dim3 lblock(kLongThreads);
+  const cudaError_t e = kf == kKeyE4M3   ? launch_pdl(score_long_kernel<kKeyE4M3>, grid, lblock, ssmem, s, 1, lp, kmap)
+                        : kf == kKeyE2M1 ? launch_pdl(score_long_kernel<kKeyE2M1>, grid, lblock, ssmem, s, 1, lp, kmap)
+                                         : launch_pdl(score_long_kernel<kKeyBF16>, grid, lblock, ssmem, s, 1, lp, kmap);
   prof_end(s);
   if (csa_status st = check_launch("indexer score (long rows)", e); st != CSA_OK) return st;
   dim3 sgrid(static_cast<unsigned>((N + kSelChunk - 1) / kSelChunk), static_cast<unsigned>(R));
@@ -1218,7 +1761,8 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   if (!ensure_smem(reinterpret_cast<const void*>(topk_select_kernel), kSelSmem))
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
   return check_launch("indexer select",
-                      launch_pdl(topk_select_kernel, sgrid, dim3(kSelThreads), kSelSmem, s, 1, w, N, Tq, q_pos0, m, k, idx));
+                      launch_pdl(topk_select_kernel, sgrid, dim3(kSelThreads), kSelSmem, s, 1, w, N, Tq, q_pos0, m, k, idx,
+                                 scores_out));
 }
 }  // namespace
 }  // namespace csa
@@ -1232,11 +1776,27 @@ csa_status csa_indexer_topk(const void* qI, const float* wI, const void* kIc, in
                            stream);
 }
 
+csa_status csa_indexer_topk_with_scores(const void* qI, const float* wI, const void* kIc, int64_t B, int64_t Tq,
+                                        int64_t N, int64_t q_pos0, int32_t m, int32_t k, int32_t* idx, float* scores,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (scores == nullptr || (reinterpret_cast<uintptr_t>(scores) & 3u))
+    return csa::fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk_with_scores: scores NULL or misaligned");
+  return csa::indexer_impl(qI, wI, kIc, nullptr, nullptr, B, Tq, N, q_pos0, m, k, idx, workspace, workspace_bytes,
+                           stream, scores);
+}
+
 csa_status csa_indexer_topk_e4m3(const void* qI, const float* wI, const uint8_t* kI_codes, const float* kI_scale,
                                  int64_t B, int64_t Tq, int64_t N, int64_t q_pos0, int32_t m, int32_t k, int32_t* idx,
                                  void* workspace, size_t workspace_bytes, void* stream) {
   return csa::indexer_impl(qI, wI, nullptr, kI_codes, kI_scale, B, Tq, N, q_pos0, m, k, idx, workspace,
-                           workspace_bytes, stream);
+                           workspace_bytes, stream, nullptr, csa::kKeyE4M3);
+}
+
+csa_status csa_indexer_topk_e2m1(const void* qI, const float* wI, const uint8_t* kI_codes, const float* kI_scale,
+                                 int64_t B, int64_t Tq, int64_t N, int64_t q_pos0, int32_t m, int32_t k, int32_t* idx,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  return csa::indexer_impl(qI, wI, nullptr, kI_codes, kI_scale, B, Tq, N, q_pos0, m, k, idx, workspace,
+                           workspace_bytes, stream, nullptr, csa::kKeyE2M1);
 }
 
 }  // extern "C"
@@ -1286,4 +1846,77 @@ extern "C" csa_status csa_indexer_topk_noalloc(const void* qI, const float* wI, 
       return fail(CSA_ERR_CUDA, "csa_indexer_topk_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
   }
   return csa_indexer_topk(qI, wI, kIc, B, Tq, N, q_pos0, m, k, idx, ptr, ptr ? kStaticScratchBytes : 0, stream);
+}
+
+extern "C" size_t csa_indexer_topk_packed_workspace_size(const csa_packed* packed, int32_t m, int32_t k) {
+  (void)k;
+  if (packed == nullptr || m < 1 || packed->n_seqs <= 0 || packed->max_tokens < 0 || packed->total_tokens <= 0 ||
+      packed->total_tokens >= (int64_t(1) << 31))
+    return 0;
+  return csa::packed_layout(packed, m).total;
+}
+
+extern "C" csa_status csa_indexer_topk_packed(const void* qI, const float* wI, const void* kIc,
+                                              const csa_packed* packed, int32_t m, int32_t k, int32_t* idx,
+                                              void* workspace, size_t workspace_bytes, void* stream) {
+  using namespace csa;
+  clear_error();
+  CSA_REQUIRE(packed != nullptr, "csa_indexer_topk_packed: packed is NULL");
+  CSA_REQUIRE(m >= 1, "csa_indexer_topk_packed: m must be >= 1");
+  CSA_REQUIRE(k >= 1 && k <= kMaxK, "csa_indexer_topk_packed: k must be in [1, %d] (got %d)", kMaxK, k);
+  CSA_REQUIRE(packed->n_seqs >= 0 && packed->max_tokens >= 0 && packed->total_tokens >= 0 &&
+                  packed->total_tokens < (int64_t(1) << 31) && packed->total_entries >= 0 &&
+                  packed->total_entries < (int64_t(1) << 31),
+              "csa_indexer_topk_packed: bad packed descriptor sizes");
+  if (packed->n_seqs == 0 || packed->total_tokens == 0) return CSA_OK;
+  CSA_REQUIRE(packed->cu_tokens != nullptr && packed->cu_entries != nullptr,
+              "csa_indexer_topk_packed: packed offsets are NULL");
+  const int64_t max_n = (static_cast<int64_t>(packed->max_tokens) + m - 1) / m;
+  if (max_n > kRowPathMaxN)
+    return fail(CSA_ERR_UNSUPPORTED,
+                "csa_indexer_topk_packed: sequences of up to %lld entries are supported (longest has %lld)",
+                static_cast<long long>(kRowPathMaxN), static_cast<long long>(max_n));
+  CSA_REQUIRE_PTR(qI);
+  CSA_REQUIRE_PTR(wI);
+  CSA_REQUIRE_PTR(kIc);
+  CSA_REQUIRE_PTR(idx);
+  const PackedLayout L = packed_layout(packed, m);
+  if (workspace == nullptr || workspace_bytes < L.total)
+    return fail(CSA_ERR_WORKSPACE, "csa_indexer_topk_packed: workspace of %zu bytes needed (got %zu)", L.total,
+                workspace_bytes);
+  CSA_REQUIRE(aligned16(workspace), "csa_indexer_topk_packed: workspace is not 16-byte aligned");
+  // every sequence adds at most one partial group
+  const int64_t groups = packed->total_tokens / kRowGroup + packed->n_seqs;
+  CSA_REQUIRE(groups < 65536, "csa_indexer_topk_packed: too many query rows for one launch");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* cu_grp = reinterpret_cast<int32_t*>(ws + L.grp);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (csa_status st = check_launch("csa_indexer_topk_packed",
+                                   launch_pdl(group_table_kernel, dim3(1), dim3(1024), 0, s, 1, packed->cu_tokens,
+                                              static_cast<int>(packed->n_seqs), cu_grp));
+      st != CSA_OK)
+    return st;
+  ScoreParams p;
+  p.qI = static_cast<const __nv_bfloat16*>(qI);
+  p.wI = wI;
+  p.kI = static_cast<const __nv_bfloat16*>(kIc);
+  p.kcodes = nullptr;
+  p.kscale = nullptr;
+  p.Tq = packed->total_tokens;
+  p.N = max_n;
+  p.q_pos0 = 0;
+  p.m = m;
+  p.scores = reinterpret_cast<float*>(ws + L.scores);
+  p.hist = nullptr;
+  p.done = nullptr;
+  p.thr = nullptr;
+  p.k = k;
+  p.pitch = L.pitch;
+  p.cu_tok = packed->cu_tokens;
+  p.cu_ent = packed->cu_entries;
+  p.cu_grp = cu_grp;
+  p.n_seqs = packed->n_seqs;
+  RowsParams rp{p.scores, L.pitch, max_n, p.Tq, 0, m, k, idx, packed->cu_tokens, packed->cu_entries, packed->n_seqs,
+                nullptr};
+  return launch_row_path("csa_indexer_topk_packed", p, rp, groups, packed->total_tokens, max_n, kKeyBF16, s);
 }

@@ -123,6 +123,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
+// One box of a 2-D tensor map (coordinates innermost first) into shared
+// memory, completing on `bar`.  The innermost coordinate must address a
+// 16-byte boundary.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];\n" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // L2 policy for data read exactly once (streamed keys): evict first, so that
 // the step's reused intermediates stay resident.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {

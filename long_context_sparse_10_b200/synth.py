@@ -123,6 +123,27 @@ def fp8_rows(x: torch.Tensor):
     return qv.to(torch.float8_e4m3fn).view(torch.uint8).contiguous(), scale.contiguous()
 
 
+E2M1_MAX = 6.0
+_E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])  # between adjacent E2M1 magnitudes
+
+
+def fp4_rows(x: torch.Tensor):
+    """Store rows [..., d] (fp32, d even) as OCP MX E2M1 codes, two per byte (dimension 2j in the low
+    nibble of byte j), with one scale per row (max |x| / 6, 1 if zero); magnitudes round to the nearest
+    E2M1 value, ties to the even code.  Returns (uint8 [..., d/2], fp32 [...])."""
+    x = x.float()
+    amax = x.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / E2M1_MAX, torch.ones_like(amax)).float()
+    v = (x / scale[..., None]).numpy()
+    a = np.minimum(np.abs(v), E2M1_MAX)
+    code = np.searchsorted(_E2M1_MIDS, a, side="left")            # a <= mids[code]: the lower neighbour on a tie
+    tie = (code < 7) & (a == _E2M1_MIDS[np.minimum(code, 6)])
+    code = np.where(tie & (code % 2 == 1), code + 1, code)         # ties go to the even code
+    nib = (code | (np.signbit(v).astype(np.int64) << 3)).astype(np.uint8)
+    packed = (nib[..., 0::2] | (nib[..., 1::2] << 4)).astype(np.uint8)
+    return torch.from_numpy(np.ascontiguousarray(packed)), scale.contiguous()
+
+
 @dataclasses.dataclass(frozen=True)
 class Prefill:
     """One prefill workload: B sequences of T tokens, all queries attend."""
@@ -157,6 +178,7 @@ class Decode:
     win: int = 128
     m_hca: int = 128
     indexer_fp8: bool = False  # indexer keys stored as E4M3 codes + per-entry scale
+    indexer_fp4: bool = False  # indexer keys stored as E2M1 codes (two per byte) + per-entry scale
 
     @property
     def N(self):
@@ -176,6 +198,9 @@ WORKLOADS = {
     # the same workload with FP8 (E4M3 + per-entry scale) lightning-indexer keys
     "hybrid_decode_l1m_fp8idx": Decode("hybrid_decode_l1m_fp8idx", "hybrid", B=8, L=1 << 20, H=64, m=4, k=2048,
                                        indexer_fp8=True),
+    # ... and with FP4 (E2M1 + per-entry scale) lightning-indexer keys
+    "hybrid_decode_l1m_fp4idx": Decode("hybrid_decode_l1m_fp4idx", "hybrid", B=8, L=1 << 20, H=64, m=4, k=2048,
+                                       indexer_fp4=True),
 }
 
 
@@ -236,6 +261,8 @@ def decode_inputs(w: Decode, seed: int = 0, batch: slice | None = None) -> dict:
     }
     if w.indexer_fp8:
         out["kI_codes"], out["kI_scale"] = fp8_rows(rows("kIc", (w.N, D_I), kind="normal_f32"))
+    elif w.indexer_fp4:
+        out["kI_codes"], out["kI_scale"] = fp4_rows(rows("kIc", (w.N, D_I), kind="normal_f32"))
     else:
         out["kIc"] = rows("kIc", (w.N, D_I))
     if w.kind == "hybrid":

@@ -399,3 +399,28 @@ def test_csa_prefill_pipeline_t65536_sampled_rows():
     O, L = R.csa_sparse_mqa(f64(x["q"][:, rows]), rows, Kc_o, Vc_o, use, m, f64(x["k"]), f64(x["v"]), 0, win, sc)
     assert_close(f64(out[:, rows]), O, "t65536 attention")
     assert_lse(f64(lse[:, rows]), L, "t65536 lse")
+
+
+@pytest.mark.parametrize("B,Tq,N,q_pos0,m,k,head_scale", [
+    (3, 1, 50000, 4 * 50000 - 1, 4, 2048, None),     # long rows (decode)
+    (2, 1, 30000, 100000, 4, 512, None),             # long rows, partly visible
+    (1, 600, 150, 0, 4, 64, None),                   # prefill rows (row path)
+    (2, 1, 20000, 4 * 20000 - 1, 4, 256, (2.0 ** -40, 2.0 ** 30, 1.0, 2.0 ** -10)),
+    (1, 300, 4000, 16000 - 300, 4, 2048, None),      # prefill rows at k = 2048
+    (8, 1, 262144, 4 * 262144 - 1, 4, 2048, None),   # the 1M-context decode shape
+])
+def test_indexer_topk_e2m1_keys(B, Tq, N, q_pos0, m, k, head_scale):
+    """FP4 (E2M1, two codes per byte, per-entry scale) indexer keys: scores of the decoded keys."""
+    g = np.random.default_rng(N + k + 29)
+    qI = _bf16(g, (B, Tq, 4, 64))
+    if head_scale is not None:
+        qI = (qI.float() * torch.tensor(head_scale).view(1, 1, 4, 1)).to(torch.bfloat16)
+    wI = torch.from_numpy(g.random((B, Tq, 4)).astype(np.float32))
+    codes, scale = synth.fp4_rows(torch.from_numpy(g.standard_normal((B, N, 64)).astype(np.float32)))
+    assert codes.shape == (B, N, 32)
+    idx = csa.csa_indexer_topk_e2m1(qI.to(DEV), wI.to(DEV), codes.to(DEV), scale.to(DEV), m, k, q_pos0=q_pos0)
+    torch.cuda.synchronize()
+    kI = R.e2m1_unpack(codes.numpy()) * scale.double().numpy()[..., None]
+    s = R.indexer_scores(f64(qI), f64(wI), kI, q_pos0 + np.arange(Tq), m)
+    same = check_topk(idx.cpu().numpy(), s, R.topk_set(s, k), k, "indexer e2m1")
+    assert same.mean() > 0.9
