@@ -729,18 +729,15 @@ def make_run(name, rank, dev):
 
 
 def reference_arm(args):
-    """The float64 CPU oracle, timed on the host cores (rank 0 only)."""
+    """The float64 CPU oracle, timed on the host cores (rank 0 only): W untimed then K timed steps, each step a
+    bounded sample of the workload (whole sequences for decode, sampled query rows for prefill)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     from long_context_sparse_10_b200 import synth
     wl = synth.WORKLOADS[args.workload]
-
-    class HostOnly:  # the same inputs, without touching a GPU
-        pass
-
-    run = (DecodeRun if isinstance(wl, synth.Decode) else PrefillRun).__new__(
-        DecodeRun if isinstance(wl, synth.Decode) else PrefillRun)
+    cls = DecodeRun if isinstance(wl, synth.Decode) else PrefillRun
+    run = cls.__new__(cls)   # the same inputs, without touching a GPU
     run.wl = wl
     run.scale = 1.0 / math.sqrt(192)
     if isinstance(wl, synth.Decode):
@@ -749,23 +746,22 @@ def reference_arm(args):
     else:
         run.host = synth.prefill_inputs(wl, seed=0)
         run.csa_kind = wl.kind == "csa"
-    budget = min(150.0, max(5.0, args.cpu_sample_s * 4))
-    per_step_budget = budget / max(1, args.steps + args.warmup)
-    n, spent, sample = run.oracle_sample(max(per_step_budget, 0.0))
-    steps_done = 1
-    total_n, total_s = n, spent
-    while total_s < budget and steps_done < args.steps:
-        n, spent, _ = run.oracle_sample(0.0)
+    budget = min(240.0, max(5.0, args.cpu_sample_s * 20))
+    per_step = budget / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        run.oracle_sample(per_step)
+    total_n, total_s, sample = 0, 0.0, ""
+    for _ in range(args.steps):
+        n, spent, sample = run.oracle_sample(per_step)
         total_n += n
         total_s += spent
-        steps_done += 1
     value = total_n / total_s
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": steps_done, "steps_requested": args.steps, "warmup": 0, "ms_per_step": 1e3 * total_s / steps_done,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "oracle": "numpy float64 (oracle/csa_ref.py)"},
+            "config": run.describe(args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                             "sample": sample + f"; {steps_done} step(s) within a {budget:.0f} s budget",
+                             "sample": sample + f"; each step a sample of about {per_step:.1f} s",
                              "host_cpus": os.cpu_count()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

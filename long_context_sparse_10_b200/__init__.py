@@ -86,7 +86,8 @@ class KVCache:
 
     @property
     def n_entries(self) -> int:
-        return (self.nope if self.split else self.k).shape[1]
+        # entries per sequence ([B, N, ...]), or all entries of packed sequences ([total_entries, ...])
+        return (self.nope if self.split else self.k).shape[-2]
 
     def desc(self) -> _lib.KVCacheDesc:
         d = _lib.KVCacheDesc()

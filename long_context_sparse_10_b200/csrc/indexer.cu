@@ -802,34 +802,39 @@ __global__ void __launch_bounds__(1024) topk_rows_kernel(RowsParams p) {
 // S^T = K Q^T with the entries as M (128 per tile, one per TMEM lane) and the
 // (query, head) pairs as N (kPfQ * 4 = 128 columns), K = 64; an epilogue
 // thread owns one entry of the tile and folds its 4 heads per query
-// (s_q = sum_h relu(S[e, 4q+h]) w[q, h]), so it holds the tile's scores of
-// every query of the CTA in registers.  The exact top-k is a radix select on
-// the order-preserving 32-bit score key, refined over passes that recompute
-// the same scores (the MMA is cheap; the scores never leave the SM):
-//   pass 0: per-query histogram of the key's top 11 bits;
-//   pass 1: 11 more bits, for entries in the query's threshold bin;
-//   pass 2: the last 10 bits, likewise;
-//   pass 3: emission -- every entry above the threshold, and the first `need`
-//           entries equal to it (ascending index, so ties go to the lower
-//           index), written as the ascending list by ordered ballots.
-// A query whose threshold bin is taken whole stops refining early; a pass
-// that no query needs only waits for its tiles.  The key tiles stream by TMA
-// (128-byte swizzle, no multicast) through a ring of stages, one thread
-// issues the MMAs into two TMEM buffers, and all waits are bounded.
+// (s_q = sum_h relu(S[e, 4q+h]) w[q, h]) into the order-preserving 32-bit key
+// of each query's score, which it stages in shared memory.  The keys are then
+// read back query-major: four consecutive lanes of a warp own one query and 32
+// consecutive entries of the tile each, so a query's running state lives in
+// registers of its own lanes and no two lanes of a warp share a histogram row
+// unless they share the query.  The exact top-k is a radix select on the key,
+// 8 bits per level, over passes that recompute the same scores (the MMA is
+// cheap; no score leaves the SM):
+//   passes 0-3: per-query 256-bin histogram of key byte 3, then of byte 2 for
+//               entries whose byte 3 is the query's threshold byte, and so on;
+//               a query whose threshold bin is taken whole stops refining;
+//   pass 4:     emission -- every entry above the threshold and the first
+//               `need` entries equal to it, in ascending index order (ties
+//               therefore go to the lower index), by a 4-lane scan per query.
+// A pass no query needs only waits for its tiles.  The key tiles stream by TMA
+// (128-byte swizzle, no multicast) through a ring of stages, one thread issues
+// the MMAs into two TMEM buffers, and all waits are bounded.
 constexpr int kPfQ = 32;         // query rows per CTA (x 4 heads = 128 MMA columns)
 constexpr int kPfTile = 128;     // entries per tile (MMA M)
 constexpr int kPfStages = 4;
 constexpr int kPfThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int kPfBins = 2048;    // histogram bins per query (11 bits)
+constexpr int kPfLevels = 4;     // histogram levels of 8 key bits
+constexpr int kPfHistW = 129;    // words per query histogram: 256 16-bit bins + 1 pad (bank spread)
+constexpr int kPfKeyW = 132;     // words per query row of staged keys: 4 quarters x 33 (bank spread)
 
 struct PfLayout {
   static constexpr size_t kK = 0;                                  // [kPfStages][128 entries][128 B]
   static constexpr size_t kQ = kK + kPfStages * 16384;             // [128 (query, head)][128 B]
-  static constexpr size_t kHist = kQ + 16384;                      // [kPfQ][kPfBins / 2] u32 (two u16 bins)
-  static constexpr size_t kW = kHist + kPfQ * (kPfBins / 2) * 4;   // [128] fp32
-  static constexpr size_t kCnt = kW + 128 * 4;                     // tie / sel counts [2][2][4][kPfQ] u32
-  static constexpr size_t kQs = kCnt + 2 * 2 * 4 * kPfQ * 4;       // per-query state, 8 x [kPfQ] u32
-  static constexpr size_t kBars = kQs + 8 * kPfQ * 4;
+  static constexpr size_t kHist = kQ + 16384;                      // [kPfQ][kPfHistW] u32
+  static constexpr size_t kKeys = kHist + kPfQ * kPfHistW * 4;     // [2][kPfQ][kPfKeyW] u32
+  static constexpr size_t kW = kKeys + 2 * kPfQ * kPfKeyW * 4;     // [128] fp32
+  static constexpr size_t kQs = kW + 128 * 4;                      // per-query state, 8 x [kPfQ] u32
+  static constexpr size_t kBars = (kQs + 8 * kPfQ * 4 + 7) / 8 * 8;
   static constexpr size_t kTotal = kBars + 128 + 1024;             // + alignment slack
 };
 
@@ -838,8 +843,15 @@ struct PfParams {
   const float* wI;          // [B, Tq, 4]
   int64_t Tq, N, q_pos0;
   int m, k;
-  int64_t groups;           // CTAs: B * ceil(Tq / kPfQ)
+  int64_t groups;           // CTAs: B * ceil(Tq / kPfQ), or an upper bound for packed sequences
   int32_t* idx;             // [B, Tq, k]
+  // packed sequences (nullable): sequence s owns query rows [cu_tok[s], cu_tok[s+1])
+  // (positions from 0) and key rows [cu_ent[s], cu_ent[s+1]) of a [1][total][64]
+  // key tensor; CTA g is group g - cu_grp[s] of kPfQ rows of sequence s
+  const int32_t* cu_tok;
+  const int32_t* cu_ent;
+  const int32_t* cu_grp;
+  int n_seqs;
 };
 
 __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams p,
@@ -850,47 +862,63 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
   uint8_t* Kst = smem + PfLayout::kK;
   uint8_t* Qs = smem + PfLayout::kQ;
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + PfLayout::kHist);
+  uint32_t* keys_s = reinterpret_cast<uint32_t*>(smem + PfLayout::kKeys);
   float* w_s = reinterpret_cast<float*>(smem + PfLayout::kW);
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + PfLayout::kCnt);  // [par][tie/sel][q4][j]
   uint32_t* qs = reinterpret_cast<uint32_t*>(smem + PfLayout::kQs);
   uint32_t* nv_s = qs;                 // visible entries of query j
-  uint32_t* level_s = qs + kPfQ;       // 0..2: refining at that pass; 3: threshold known
-  uint32_t* prefix_s = qs + 2 * kPfQ;  // key bits fixed so far (levels 1, 2)
+  uint32_t* level_s = qs + kPfQ;       // 0..3: refining at that level; kPfLevels: threshold known
+  uint32_t* prefix_s = qs + 2 * kPfQ;  // key bytes fixed so far
   uint32_t* rem_s = qs + 3 * kPfQ;     // entries still to take at the current level
   uint32_t* shift_s = qs + 4 * kPfQ;   // emission: compare key >> shift with thr, take need ties
   uint32_t* thr_s = qs + 5 * kPfQ;
   uint32_t* need_s = qs + 6 * kPfQ;
-  uint32_t* base_s = qs + 7 * kPfQ;    // emission: entries written so far
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + PfLayout::kBars);  // [kPfStages]
   uint64_t* empty = full + kPfStages;                                     // [kPfStages]
   uint64_t* tfull = empty + kPfStages;                                    // [2]
   uint64_t* tempty = tfull + 2;                                           // [2]
   uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
-  __shared__ uint32_t tie_base_s[kPfQ];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t gpb = (p.Tq + kPfQ - 1) / kPfQ;
   const int64_t grp = p.groups - 1 - static_cast<int64_t>(blockIdx.x);  // late (long) rows first
-  const int64_t b = grp / gpb;
-  const int64_t r0 = (grp % gpb) * kPfQ;
-  const int nq = static_cast<int>((p.Tq - r0) < kPfQ ? (p.Tq - r0) : kPfQ);
-  const int64_t row0 = b * p.Tq + r0;  // global row of query 0
-  const int64_t nv_max = visible(p.q_pos0 + r0 + nq - 1, p.m, p.N);
+  // this CTA's rows: global rows row0.., positions t0.., keys at tensor-map rows
+  // key0.. of batch kb, Nseq of them
+  int64_t row0, t0, key0, Nseq;
+  int kb, nq;
+  if (p.cu_tok != nullptr) {
+    if (grp >= __ldg(p.cu_grp + p.n_seqs)) return;  // past the last group (the grid is an upper bound)
+    const int sq = seq_of(p.cu_grp, p.n_seqs, grp);
+    const int64_t len = __ldg(p.cu_tok + sq + 1) - __ldg(p.cu_tok + sq);
+    t0 = (grp - __ldg(p.cu_grp + sq)) * kPfQ;
+    row0 = __ldg(p.cu_tok + sq) + t0;
+    nq = static_cast<int>((len - t0) < kPfQ ? (len - t0) : kPfQ);
+    key0 = __ldg(p.cu_ent + sq);
+    Nseq = __ldg(p.cu_ent + sq + 1) - key0;
+    kb = 0;
+  } else {
+    const int64_t gpb = (p.Tq + kPfQ - 1) / kPfQ;
+    const int64_t b = grp / gpb;
+    const int64_t r0 = (grp % gpb) * kPfQ;
+    nq = static_cast<int>((p.Tq - r0) < kPfQ ? (p.Tq - r0) : kPfQ);
+    row0 = b * p.Tq + r0;
+    t0 = p.q_pos0 + r0;
+    key0 = 0;
+    Nseq = p.N;
+    kb = static_cast<int>(b);
+  }
+  const int64_t nv_max = visible(t0 + nq - 1, p.m, Nseq);
   const int k = p.k;
 
   if (tid < kPfQ) {
     const int j = tid;
-    const uint32_t nv = j < nq ? static_cast<uint32_t>(visible(p.q_pos0 + r0 + j, p.m, p.N)) : 0u;
+    const uint32_t nv = j < nq ? static_cast<uint32_t>(visible(t0 + j, p.m, Nseq)) : 0u;
     nv_s[j] = nv;
     const bool partial = nv > static_cast<uint32_t>(k);
-    level_s[j] = partial ? 0u : 3u;
+    level_s[j] = partial ? 0u : static_cast<uint32_t>(kPfLevels);
     prefix_s[j] = 0u;
     rem_s[j] = static_cast<uint32_t>(k);
     shift_s[j] = 0u;   // with thr 0 every visible key (>= 0x007fffff) is above: all visible entries
     thr_s[j] = 0u;
     need_s[j] = 0u;
-    base_s[j] = 0u;
-    tie_base_s[j] = 0u;
   }
   if (nv_max <= k) {  // every row of the CTA keeps all its visible entries: no scoring at all
     __syncthreads();
@@ -901,7 +929,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
     return;
   }
   const int ntiles = static_cast<int>((nv_max + kPfTile - 1) / kPfTile);
-  constexpr int kPasses = 4;
+  constexpr int kPasses = kPfLevels + 1;
 
   if (tid == 0) {
     for (int i = 0; i < kPfStages; ++i) {
@@ -924,7 +952,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
   }
   cp_async_commit();
   if (tid < 128) w_s[tid] = (tid >> 2) < nq ? p.wI[(row0 + (tid >> 2)) * kHI + (tid & 3)] : 0.f;
-  for (int i = tid; i < kPfQ * kPfBins / 2; i += kPfThreads) hist[i] = 0u;
+  for (int i = tid; i < kPfQ * kPfHistW; i += kPfThreads) hist[i] = 0u;
   cp_async_wait<0>();
   tc::fence_async_smem();
   tc::fence_before_sync();
@@ -940,7 +968,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
         const int st = it % kPfStages;
         if (it >= kPfStages && !tc::bar_wait(&empty[st], static_cast<uint32_t>(((it / kPfStages) - 1) & 1))) break;
         tc::bar_arrive_expect_tx(&full[st], 16384u);
-        tc::tma_load_3d(Kst + st * 16384, &kmap, 0, (it % ntiles) * kPfTile, static_cast<int>(b), &full[st]);
+        tc::tma_load_3d(Kst + st * 16384, &kmap, 0, static_cast<int>(key0 + (it % ntiles) * kPfTile), kb, &full[st]);
       }
     }
   } else if (warp == 1) {
@@ -963,29 +991,36 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
       }
     }
   } else {
-    // ===================== epilogue: thread = entry of the tile =====================
+    // ===================== epilogue =====================
+    // scoring: thread = entry et of the tile (its TMEM lane); then query-major:
+    // thread = (query qj = etid / 4, quarter qq = etid % 4 of the tile's entries)
     const int q4 = warp & 3;  // TMEM lane quarter of this warp
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-    const int et = q4 * 32 + lane;  // entry within the tile
+    const int et = q4 * 32 + lane;  // entry within the tile (scoring)
     const int etid = tid - 64;      // 0..127
-    const uint32_t lt_mask = (1u << lane) - 1u;
+    const int qj = etid >> 2, qq = etid & 3;
+    const int64_t qrow = row0 + qj;
+    // key slot of entry et for query j: quarter-padded rows spread the banks
+    auto key_slot = [&](int buf, int j, int e) { return (buf * kPfQ + j) * kPfKeyW + (e >> 5) * 33 + (e & 31); };
     // A wait that runs out (recorded in the device error word) skips the later
     // waits but keeps the loop and its named barriers, so the four warps stay
     // in step and the CTA finishes; its output is then not valid.
     bool healthy = true;
     int it = 0;
+    uint32_t sel_done = 0u, ties_done = 0u;  // emission running totals of query qj (same in its 4 lanes)
     for (int pass = 0; pass < kPasses; ++pass) {
-      // does any query refine at this pass (passes 0-2)?  pass 3 always emits
-      bool active = pass == 3;
+      // does any query refine at this level (passes 0..3)?  the last pass always emits
+      bool active = pass == kPfLevels;
       if (!active) {
         for (int j = 0; j < kPfQ; ++j) active |= level_s[j] == static_cast<uint32_t>(pass);
       }
+      // this thread's query state for the pass
+      const uint32_t nv_q = nv_s[qj], lv_q = level_s[qj], pre_q = prefix_s[qj];
+      const uint32_t sh_q = shift_s[qj], thr_q = thr_s[qj], need_q = need_s[qj];
       for (int tile = 0; tile < ntiles; ++tile, ++it) {
         const int buf = it & 1;
         if (healthy) healthy = tc::bar_wait(&tfull[buf], static_cast<uint32_t>((it >> 1) & 1));
         tc::fence_after_sync();
-        const uint32_t e = static_cast<uint32_t>(tile * kPfTile + et);
-        uint32_t gt_m = 0u, eq_m = 0u;  // emission: per query, this entry above / at the threshold
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {  // 8 queries (32 accumulator columns) at a time
           float v[32];
@@ -1001,83 +1036,77 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
             const float4 w4 = *reinterpret_cast<const float4*>(w_s + 4 * j);
             const float sc = fmaxf(v[4 * jj], 0.f) * w4.x + fmaxf(v[4 * jj + 1], 0.f) * w4.y +
                              fmaxf(v[4 * jj + 2], 0.f) * w4.z + fmaxf(v[4 * jj + 3], 0.f) * w4.w;
-            const uint32_t key = f2key(sc + 0.0f);
-            const bool vis = e < nv_s[j];
-            const uint32_t lv = level_s[j];
-            if (pass == 0) {
-              if (vis && lv == 0u) {
-                const uint32_t bin = key >> 21;
-                atomicAdd(&hist[j * (kPfBins / 2) + (bin >> 1)], 1u << ((bin & 1u) * 16));
-              }
-            } else if (pass == 1) {
-              if (vis && lv == 1u && (key >> 21) == prefix_s[j]) {
-                const uint32_t bin = (key >> 10) & 2047u;
-                atomicAdd(&hist[j * (kPfBins / 2) + (bin >> 1)], 1u << ((bin & 1u) * 16));
-              }
-            } else if (pass == 2) {
-              if (vis && lv == 2u && (key >> 10) == prefix_s[j]) {
-                const uint32_t bin = key & 1023u;
-                atomicAdd(&hist[j * (kPfBins / 2) + (bin >> 1)], 1u << ((bin & 1u) * 16));
-              }
-            } else {
-              const uint32_t kk = key >> shift_s[j];
-              const uint32_t th = thr_s[j];
-              gt_m |= (vis && kk > th) ? (1u << j) : 0u;
-              eq_m |= (vis && kk == th) ? (1u << j) : 0u;
-            }
+            keys_s[key_slot(buf, j, et)] = f2key(sc + 0.0f);
           }
         }
-        if (!active || pass < 3) continue;
-        // ---- emission of this tile, in ascending entry order across the 4 warps ----
-        const int par = tile & 1;
-        uint32_t* tcnt = cnt + (par * 2 + 0) * 4 * kPfQ;
-        uint32_t* scnt = cnt + (par * 2 + 1) * 4 * kPfQ;
-        for (int j = 0; j < kPfQ; ++j) {
-          const uint32_t eb = __ballot_sync(0xffffffffu, (eq_m >> j) & 1u);
-          if (lane == 0) tcnt[q4 * kPfQ + j] = __popc(eb);
-        }
-        named_sync_ix(3, 128);
-        uint32_t sel_m = 0u;
-        for (int j = 0; j < kPfQ; ++j) {
-          const uint32_t eb = __ballot_sync(0xffffffffu, (eq_m >> j) & 1u);
-          uint32_t off = tie_base_s[j];
-          for (int w = 0; w < q4; ++w) off += tcnt[w * kPfQ + j];
-          const uint32_t rank = off + __popc(eb & lt_mask);
-          const bool eq = (eq_m >> j) & 1u;
-          const bool sel = ((gt_m >> j) & 1u) || (eq && rank < need_s[j]);
-          sel_m |= sel ? (1u << j) : 0u;
-          const uint32_t sb = __ballot_sync(0xffffffffu, sel);
-          if (lane == 0) scnt[q4 * kPfQ + j] = __popc(sb);
-        }
-        // entries written so far per query, read before the barrier (updated after it)
-        const uint32_t my_base = lane < kPfQ ? base_s[lane] : 0u;
-        named_sync_ix(3, 128);
-        for (int j = 0; j < kPfQ; ++j) {
-          const uint32_t sb = __ballot_sync(0xffffffffu, (sel_m >> j) & 1u);
-          if (sb == 0u) continue;
-          uint32_t pos = __shfl_sync(0xffffffffu, my_base, j);
-          for (int w = 0; w < q4; ++w) pos += scnt[w * kPfQ + j];
-          pos += __popc(sb & lt_mask);
-          if (((sel_m >> j) & 1u) && pos < static_cast<uint32_t>(k)) p.idx[(row0 + j) * k + pos] = static_cast<int32_t>(e);
-        }
-        named_sync_ix(3, 128);
-        if (etid < kPfQ) {  // running totals of this tile's ties and selections
-          const int j = etid;
-          tie_base_s[j] += tcnt[j] + tcnt[kPfQ + j] + tcnt[2 * kPfQ + j] + tcnt[3 * kPfQ + j];
-          base_s[j] += scnt[j] + scnt[kPfQ + j] + scnt[2 * kPfQ + j] + scnt[3 * kPfQ + j];
+        if (!active) continue;
+        named_sync_ix(3, 128);  // the tile's keys are staged (a buffer per tile parity)
+        const int e0 = qq * 32;                                  // this thread's first entry of the tile
+        const uint32_t eabs0 = static_cast<uint32_t>(tile * kPfTile + e0);
+        const int nvis = static_cast<int>(nv_q > eabs0 ? (nv_q - eabs0 < 32u ? nv_q - eabs0 : 32u) : 0u);
+        const uint32_t* kr = keys_s + key_slot(buf, qj, e0);
+        if (pass < kPfLevels) {
+          if (lv_q == static_cast<uint32_t>(pass)) {
+            const int bsh = 24 - 8 * pass;
+            uint32_t* h = hist + qj * kPfHistW;
+            for (int i = 0; i < nvis; ++i) {
+              const uint32_t key = kr[i];
+              if (pass == 0 || (key >> (bsh + 8)) == pre_q) {
+                const uint32_t bin = (key >> bsh) & 255u;
+                atomicAdd(h + (bin >> 1), 1u << ((bin & 1u) * 16));
+              }
+            }
+          }
+        } else {
+          // emission: entries above the threshold, and ties at it in index order
+          uint32_t gt = 0u, eq = 0u;
+          for (int i = 0; i < nvis; ++i) {
+            const uint32_t kk = kr[i] >> sh_q;
+            gt |= kk > thr_q ? (1u << i) : 0u;
+            eq |= kk == thr_q ? (1u << i) : 0u;
+          }
+          const uint32_t n_eq = __popc(eq);
+          uint32_t tie_incl = n_eq;  // scan over the query's 4 lanes (entries in order)
+#pragma unroll
+          for (int o = 1; o < 4; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, tie_incl, o, 4);
+            if (qq >= o) tie_incl += t;
+          }
+          const uint32_t tie0 = ties_done + tie_incl - n_eq;  // rank of this thread's first tie
+          const uint32_t take = need_q > tie0 ? (need_q - tie0 < n_eq ? need_q - tie0 : n_eq) : 0u;
+          // the first `take` tie bits (lowest entries) are selected
+          uint32_t eq_sel = eq;
+          for (uint32_t drop = n_eq - take; drop > 0; --drop) eq_sel &= ~(0x80000000u >> __clz(eq_sel));
+          const uint32_t sel = gt | eq_sel;
+          const uint32_t n_sel = __popc(sel);
+          uint32_t sel_incl = n_sel;
+#pragma unroll
+          for (int o = 1; o < 4; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, sel_incl, o, 4);
+            if (qq >= o) sel_incl += t;
+          }
+          uint32_t pos = sel_done + sel_incl - n_sel;
+          for (uint32_t m = sel; m != 0u; m &= m - 1u) {
+            if (pos < static_cast<uint32_t>(k)) p.idx[qrow * k + pos] = static_cast<int32_t>(eabs0 + __ffs(m) - 1);
+            ++pos;
+          }
+          ties_done += __shfl_sync(0xffffffffu, tie_incl, (lane & ~3) | 3);
+          sel_done += __shfl_sync(0xffffffffu, sel_incl, (lane & ~3) | 3);
         }
       }
-      if (pass == 3) break;
-      // ---- thresholds of the queries that refined in this pass ----
+      if (pass == kPfLevels) break;
+      // ---- thresholds of the queries that refined at this level ----
       named_sync_ix(3, 128);
-      const int nb = pass == 2 ? 1024 : 2048;
-      const int per_lane = nb / 32;  // bins per lane, walked from the top
       for (int j = q4; j < kPfQ; j += 4) {
         if (level_s[j] != static_cast<uint32_t>(pass)) continue;  // uniform in the warp
-        const uint32_t* h = hist + j * (kPfBins / 2);
-        const int hi = nb - lane * per_lane;  // this lane's bins [hi - per_lane, hi)
-        uint32_t sum = 0;
-        for (int bb = hi - 1; bb >= hi - per_lane; --bb) sum += (h[bb >> 1] >> ((bb & 1) * 16)) & 0xffffu;
+        const uint32_t* h = hist + j * kPfHistW;
+        uint32_t cbin[8], sum = 0;  // lane's 8 bins, walked from the top: 255 - 8 lane - i
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int bb = 255 - 8 * lane - i;
+          cbin[i] = (h[bb >> 1] >> ((bb & 1) * 16)) & 0xffffu;
+          sum += cbin[i];
+        }
         uint32_t incl = sum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -1088,17 +1117,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
         const uint32_t rem = rem_s[j];
         if (excl < rem && incl >= rem) {
           uint32_t acc = excl;
-          for (int bb = hi - 1; bb >= hi - per_lane; --bb) {
-            const uint32_t c = (h[bb >> 1] >> ((bb & 1) * 16)) & 0xffffu;
-            if (acc + c >= rem) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (acc + cbin[i] >= rem) {
+              const uint32_t bb = static_cast<uint32_t>(255 - 8 * lane - i);
               const uint32_t nrem = rem - acc;  // still needed from bin bb
-              const uint32_t pref = pass == 0 ? static_cast<uint32_t>(bb)
-                                              : (prefix_s[j] << (pass == 1 ? 11 : 10)) | static_cast<uint32_t>(bb);
-              if (c == nrem || pass == 2) {  // threshold found: ties at it are taken in index order
-                shift_s[j] = pass == 0 ? 21u : (pass == 1 ? 10u : 0u);
+              const uint32_t pref = (prefix_s[j] << 8) | bb;
+              if (cbin[i] == nrem || pass == kPfLevels - 1) {  // threshold found; its ties go in index order
+                shift_s[j] = static_cast<uint32_t>(24 - 8 * pass);
                 thr_s[j] = pref;
                 need_s[j] = nrem;
-                level_s[j] = 3u;
+                level_s[j] = static_cast<uint32_t>(kPfLevels);
               } else {
                 prefix_s[j] = pref;
                 rem_s[j] = nrem;
@@ -1106,19 +1135,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
               }
               break;
             }
-            acc += c;
+            acc += cbin[i];
           }
         }
       }
       named_sync_ix(3, 128);  // every warp is done reading the histograms
-      for (int i = etid; i < kPfQ * kPfBins / 2; i += 128) hist[i] = 0u;
+      for (int i = etid; i < kPfQ * kPfHistW; i += 128) hist[i] = 0u;
       named_sync_ix(3, 128);
     }
-    named_sync_ix(3, 128);  // the last tile's running totals are in base_s
-    // padding after each query's selection
-    for (int j = 0; j < nq; ++j) {
-      const uint32_t done = base_s[j] < static_cast<uint32_t>(k) ? base_s[j] : static_cast<uint32_t>(k);
-      for (uint32_t c = done + etid; c < static_cast<uint32_t>(k); c += 128) p.idx[(row0 + j) * k + c] = -1;
+    // padding after each query's selection (its 4 lanes hold the running total)
+    if (qj < nq) {
+      const uint32_t done = sel_done < static_cast<uint32_t>(k) ? sel_done : static_cast<uint32_t>(k);
+      for (uint32_t c = done + qq; c < static_cast<uint32_t>(k); c += 4) p.idx[qrow * k + c] = -1;
     }
   }
   tc::fence_before_sync();
@@ -1544,8 +1572,8 @@ csa_status launch_row_path(const char* name, ScoreParams& p, const RowsParams& r
   return check_launch(name, launch_pdl(topk_rows_kernel, dim3(static_cast<unsigned>(R)), dim3(1024), smem, s, 1, rp));
 }
 
-// Offsets of each packed sequence's first group of kRowGroup query rows.
-__global__ void __launch_bounds__(1024) group_table_kernel(const int32_t* __restrict__ cu_tok, int n,
+// Offsets of each packed sequence's first group of `gsize` query rows.
+__global__ void __launch_bounds__(1024) group_table_kernel(const int32_t* __restrict__ cu_tok, int n, int gsize,
                                                            int32_t* __restrict__ cu_grp) {
   pdl_wait();
   pdl_trigger();
@@ -1554,7 +1582,7 @@ __global__ void __launch_bounds__(1024) group_table_kernel(const int32_t* __rest
   if (threadIdx.x == 0) cu_grp[0] = 0;
   for (int base = 0; base < n; base += 1024) {
     const int sq = base + static_cast<int>(threadIdx.x);
-    const uint32_t v = sq < n ? static_cast<uint32_t>(cu_tok[sq + 1] - cu_tok[sq] + kRowGroup - 1) / kRowGroup : 0u;
+    const uint32_t v = sq < n ? static_cast<uint32_t>(cu_tok[sq + 1] - cu_tok[sq] + gsize - 1) / gsize : 0u;
     uint32_t total;
     const uint32_t ex = block_excl_scan(v, &total, scan_sh);
     if (sq < n) cu_grp[sq + 1] = static_cast<int32_t>(carry + ex + v);
@@ -1578,10 +1606,14 @@ csa_status encode_key_map(CUtensorMap* kmap, const void* kIc, int64_t B, int64_t
 }
 
 csa_status launch_prefill_tc(const void* qI, const float* wI, const void* kIc, int64_t B, int64_t Tq, int64_t N,
-                             int64_t q_pos0, int32_t m, int32_t k, int32_t* idx, cudaStream_t s) {
+                             int64_t q_pos0, int32_t m, int32_t k, int32_t* idx, cudaStream_t s,
+                             const csa_packed* pk = nullptr, const int32_t* cu_grp = nullptr) {
   CUtensorMap kmap;
   memset(&kmap, 0, sizeof(kmap));
-  if (csa_status st = encode_key_map(&kmap, kIc, B, N, "csa_indexer_topk"); st != CSA_OK) return st;
+  // packed sequences: one [1][total_entries][64] key tensor
+  if (csa_status st = encode_key_map(&kmap, kIc, pk ? 1 : B, pk ? pk->total_entries : N, "csa_indexer_topk");
+      st != CSA_OK)
+    return st;
   PfParams p;
   p.qI = static_cast<const __nv_bfloat16*>(qI);
   p.wI = wI;
@@ -1590,8 +1622,12 @@ csa_status launch_prefill_tc(const void* qI, const float* wI, const void* kIc, i
   p.q_pos0 = q_pos0;
   p.m = m;
   p.k = k;
-  p.groups = B * ((Tq + kPfQ - 1) / kPfQ);
+  p.groups = pk ? (pk->total_tokens / kPfQ + pk->n_seqs) : B * ((Tq + kPfQ - 1) / kPfQ);
   p.idx = idx;
+  p.cu_tok = pk ? pk->cu_tokens : nullptr;
+  p.cu_ent = pk ? pk->cu_entries : nullptr;
+  p.cu_grp = cu_grp;
+  p.n_seqs = pk ? pk->n_seqs : 0;
   if (!ensure_smem(reinterpret_cast<const void*>(indexer_prefill_kernel), static_cast<int>(PfLayout::kTotal)))
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise the shared memory limit");
   prof_begin(s);
@@ -1605,12 +1641,14 @@ struct PackedLayout {
   size_t scores, grp, total;
   int64_t pitch;
 };
+// The packed path keeps its scores on chip: the workspace holds only the
+// per-sequence group table.
 PackedLayout packed_layout(const csa_packed* pk, int32_t m) {
   PackedLayout L;
   L.pitch = ((static_cast<int64_t>(pk->max_tokens) + m - 1) / m + 3) / 4 * 4;
   L.scores = 0;
-  L.grp = align_up(static_cast<size_t>(pk->total_tokens) * L.pitch * 4);
-  L.total = align_up(L.grp + (static_cast<size_t>(pk->n_seqs) + 1) * 4);
+  L.grp = 0;
+  L.total = align_up((static_cast<size_t>(pk->n_seqs) + 1) * 4);
   return L;
 }
 
@@ -1871,11 +1909,6 @@ extern "C" csa_status csa_indexer_topk_packed(const void* qI, const float* wI, c
   if (packed->n_seqs == 0 || packed->total_tokens == 0) return CSA_OK;
   CSA_REQUIRE(packed->cu_tokens != nullptr && packed->cu_entries != nullptr,
               "csa_indexer_topk_packed: packed offsets are NULL");
-  const int64_t max_n = (static_cast<int64_t>(packed->max_tokens) + m - 1) / m;
-  if (max_n > kRowPathMaxN)
-    return fail(CSA_ERR_UNSUPPORTED,
-                "csa_indexer_topk_packed: sequences of up to %lld entries are supported (longest has %lld)",
-                static_cast<long long>(kRowPathMaxN), static_cast<long long>(max_n));
   CSA_REQUIRE_PTR(qI);
   CSA_REQUIRE_PTR(wI);
   CSA_REQUIRE_PTR(kIc);
@@ -1885,38 +1918,12 @@ extern "C" csa_status csa_indexer_topk_packed(const void* qI, const float* wI, c
     return fail(CSA_ERR_WORKSPACE, "csa_indexer_topk_packed: workspace of %zu bytes needed (got %zu)", L.total,
                 workspace_bytes);
   CSA_REQUIRE(aligned16(workspace), "csa_indexer_topk_packed: workspace is not 16-byte aligned");
-  // every sequence adds at most one partial group
-  const int64_t groups = packed->total_tokens / kRowGroup + packed->n_seqs;
-  CSA_REQUIRE(groups < 65536, "csa_indexer_topk_packed: too many query rows for one launch");
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int32_t* cu_grp = reinterpret_cast<int32_t*>(ws + L.grp);
+  int32_t* cu_grp = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + L.grp);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (csa_status st = check_launch("csa_indexer_topk_packed",
                                    launch_pdl(group_table_kernel, dim3(1), dim3(1024), 0, s, 1, packed->cu_tokens,
-                                              static_cast<int>(packed->n_seqs), cu_grp));
+                                              static_cast<int>(packed->n_seqs), kPfQ, cu_grp));
       st != CSA_OK)
     return st;
-  ScoreParams p;
-  p.qI = static_cast<const __nv_bfloat16*>(qI);
-  p.wI = wI;
-  p.kI = static_cast<const __nv_bfloat16*>(kIc);
-  p.kcodes = nullptr;
-  p.kscale = nullptr;
-  p.Tq = packed->total_tokens;
-  p.N = max_n;
-  p.q_pos0 = 0;
-  p.m = m;
-  p.scores = reinterpret_cast<float*>(ws + L.scores);
-  p.hist = nullptr;
-  p.done = nullptr;
-  p.thr = nullptr;
-  p.k = k;
-  p.pitch = L.pitch;
-  p.cu_tok = packed->cu_tokens;
-  p.cu_ent = packed->cu_entries;
-  p.cu_grp = cu_grp;
-  p.n_seqs = packed->n_seqs;
-  RowsParams rp{p.scores, L.pitch, max_n, p.Tq, 0, m, k, idx, packed->cu_tokens, packed->cu_entries, packed->n_seqs,
-                nullptr};
-  return launch_row_path("csa_indexer_topk_packed", p, rp, groups, packed->total_tokens, max_n, kKeyBF16, s);
+  return launch_prefill_tc(qI, wI, kIc, 1, packed->total_tokens, 0, 0, m, k, idx, s, packed, cu_grp);
 }
