@@ -345,9 +345,11 @@ CSA_API size_t csa_indexer_topk_packed_workspace_size(const csa_packed* packed, 
  *   qI  bf16 [total_tokens, 4, 64];  wI fp32 [total_tokens, 4]
  *   kIc bf16 [total_entries, 64] (e.g. csa_compress_packed's output)
  *   idx int32 [total_tokens, k] (output)
- *   packed->cu_entries must use stride m.  Sequences of up to 32768 entries
- *   (ceil(max_tokens / m)); longer ones return CSA_ERR_UNSUPPORTED.  Other
- *   limits and errors as csa_indexer_topk.
+ *   packed->cu_entries must use stride m.  Sequences of up to 65535 entries
+ *   (ceil(max_tokens / m)); longer ones return CSA_ERR_UNSUPPORTED.  The
+ *   scores stay on chip; the workspace (a few bytes per sequence) holds a
+ *   table of the sequences' 32-row groups.  Other limits and errors as
+ *   csa_indexer_topk.
  */
 CSA_API csa_status csa_indexer_topk_packed(const void* qI, const float* wI, const void* kIc,
                                            const csa_packed* packed, int32_t m, int32_t k, int32_t* idx,

@@ -111,7 +111,8 @@ class Window:
         d = _lib.WindowDesc()
         d.k, d.v = _ptr(self.k), _ptr(self.v)
         d.pos0 = self.pos0
-        d.rows = 0 if self.k is None else self.k.shape[1]
+        # rows per sequence ([B, rows, 192]), or all packed tokens ([total_tokens, 192])
+        d.rows = 0 if self.k is None else self.k.shape[-2]
         d.len = self.length
         d.reserved = 0
         return d

@@ -584,7 +584,7 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 template <bool FP8, bool SHV>
-__global__ void __maxnreg__(120) attn_tc_kernel(AttnParams p) {  // 17 warps x 32 x 120 <= 65536
+__global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p) {
   pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -701,44 +701,26 @@ __global__ void __maxnreg__(120) attn_tc_kernel(AttnParams p) {  // 17 warps x 3
     }
   } else if (warp >= 8) {
     // ===================== producer: gather, widen, publish =====================
-    // With three K stages the producer works one tile ahead: while tile t is
-    // widened and published, tile t+1's slots are described, its copies are in
-    // flight and its FP8 codes are being loaded, so the load latency of a tile
-    // overlaps the previous tile's work.  (The MMA order S(0), S(1), then
-    // PV(t), S(t+2) allows this with three stages: the wait for stage
-    // (t+1) % 3 is a wait for PV(t-2), which is issued before S(t).)  With two
-    // stages it would wait for PV(t-1), issued after S(t+1): the two-stage
-    // layout describes and issues each tile after publishing the previous one.
-    // The slot tables (stype, srow) are producer-private, indexed by tile
-    // parity; the softmax reads validity from the per-stage ballot words.
-    constexpr bool kAhead = NS >= 3;
     const int pt = tid - 256;  // 0..255; threads 0..127 also own one slot each
-    const int pwarp = warp - 8;
-    // selected entry of this thread's slot in a later tile, loaded ahead so
-    // that its latency overlaps the current tile's gathers
+    // selected entry of this thread's slot in the next tile, loaded one tile
+    // ahead so that its latency overlaps the current tile's gathers
     auto load_sel = [&](int tile) -> int32_t {
       const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
       return (!dense && pt < kTcKeys && tile < ntiles && sl < s1 && sl < n_ent) ? __ldg(p.idx + row * p.k + sl) : -1;
     };
-    // the tile's slots are an entry run [0, ne) then a window run [ne, ne + nw)
-    auto runs = [&](int tile, int& ne, int& nw) {
-      const int64_t a0 = s0 + static_cast<int64_t>(tile) * kTcKeys;
-      const int64_t a1 = (a0 + kTcKeys) < s1 ? (a0 + kTcKeys) : s1;
-      const int64_t ee = a1 < n_ent ? a1 : n_ent;
-      ne = static_cast<int>((ee - a0) > 0 ? (ee - a0) : 0);
-      nw = static_cast<int>(a1 - a0) - ne;
-    };
-    // slot -> (type, row): 0 skip, 1 compressed entry, 2 raw window token; the
-    // slot table goes to buffer tile & 1, the validity ballot to vmask[st]
-    auto describe = [&](int tile, int32_t sel) {
+    int32_t sel_next = load_sel(0);
+    for (int tile = 0; tile < ntiles; ++tile) {
+      const int st = tile % NS;
+      const int32_t sel_cur = sel_next;
+      if (tile >= NS && healthy) healthy = tc::bar_wait(&empty[st], ((tile / NS) - 1) & 1);
+      // slot -> (type, row): 0 skip, 1 compressed entry, 2 raw window token
       if (pt < kTcKeys) {
-        const int tb = tile & 1;
         const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
         int type = 0;
         int64_t r = 0;
         if (sl < s1) {
           if (sl < n_ent) {
-            const int64_t i = dense ? sl : static_cast<int64_t>(sel);
+            const int64_t i = dense ? sl : static_cast<int64_t>(sel_cur);
             if (i >= 0 && i < geo.N && (i + 1) * p.stride - 1 <= t) {
               type = 1;
               r = geo.ebase + i;
@@ -748,43 +730,41 @@ __global__ void __maxnreg__(120) attn_tc_kernel(AttnParams p) {  // 17 warps x 3
             r = geo.wbase + (wlo + (sl - n_ent));
           }
         }
-        stype[tb][pt] = type;
-        srow[tb][pt] = r;
+        stype[st][pt] = type;
+        srow[st][pt] = r;
         const uint32_t bal = __ballot_sync(0xffffffffu, type != 0);
-        if (lane == 0) vmask[tile % NS][warp - 8] = bal;
+        if (lane == 0) vmask[st][warp - 8] = bal;
       }
-    };
-    // FP8 entries: thread pt owns 16-code chunk c = pt % 8 of keys pt / 8 + 32 j
-    // (eight lanes per 128-byte row, four rows per warp instruction); codes and
-    // scales go to registers and are widened into the K tile later.
-    uint4 codes[4];
-    float scl[4];
-    auto load_codes = [&](int tile) {
-      if (!FP8) return;
-      int ne, nw;
-      runs(tile, ne, nw);
-      const int tb = tile & 1;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int key = (pt >> 3) + 32 * j;
-        const bool ok = key < ne && stype[tb][key] == 1;
-        const int64_t r = ok ? srow[tb][key] : 0;
-        codes[j] = ok ? ldg_nc16(p.cnope + r * kDNope + (pt & 7) * 16) : make_uint4(0u, 0u, 0u, 0u);
-        scl[j] = ok ? __ldg(p.cscale + r) : 0.f;
-      }
-    };
-    // the tile's asynchronous copies (everything but the FP8 codes), one commit group
-    auto issue = [&](int tile) {
-      const int st = tile % NS, tb = tile & 1;
+      named_sync(1, 256);
       uint8_t* Kt = Kst + st * 3 * kKB;
       uint8_t* Vt = Vst + st * 2 * kKB;
-      int ne, nw;
-      runs(tile, ne, nw);
+      // The tile's slots are an entry run [0, ne) then a window run [ne, ne + nw).
+      const int64_t a0 = s0 + static_cast<int64_t>(tile) * kTcKeys;
+      const int64_t a1 = (a0 + kTcKeys) < s1 ? (a0 + kTcKeys) : s1;
+      const int ne = static_cast<int>(((a1 < n_ent ? a1 : n_ent) - a0) > 0 ? ((a1 < n_ent ? a1 : n_ent) - a0) : 0);
+      const int nw = static_cast<int>(a1 - a0) - ne;
+      const int pwarp = warp - 8;
+      // FP8 entries: thread pt owns 16-code chunk c = pt % 8 of keys pt / 8 + 32 j
+      // (eight lanes per 128-byte row, four rows per warp instruction); the
+      // codes and scales go to registers here and are widened after the
+      // asynchronous copies below are issued.
+      uint4 codes[4];
+      float scl[4];
+      if (FP8) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int key = (pt >> 3) + 32 * j;
+          const bool ok = key < ne && stype[st][key] == 1;
+          const int64_t r = ok ? srow[st][key] : 0;
+          codes[j] = ok ? ldg_nc16(p.cnope + r * kDNope + (pt & 7) * 16) : make_uint4(0u, 0u, 0u, 0u);
+          scl[j] = ok ? __ldg(p.cscale + r) : 0.f;
+        }
+      }
       // Contiguous runs are copied with consecutive lanes on consecutive 16-byte
       // chunks (512-byte warp requests); selected entries are gathered four keys
       // per warp instruction (8 lanes per 128-byte row).
       if (ne > 0 && dense) {
-        const int64_t r0 = srow[tb][0];
+        const int64_t r0 = srow[st][0];
         if (FP8) {
           for (int pc = pt; pc < ne * 8; pc += 256)
             cp_async16(Kt + 2 * kKB + tc::sw128(pc >> 3, pc & 7), p.crope + r0 * kDRope + pc * 8);
@@ -806,8 +786,8 @@ __global__ void __maxnreg__(120) attn_tc_kernel(AttnParams p) {  // 17 warps x 3
         for (int kb = pwarp * 4; kb < ne; kb += 32) {
           const int key = kb + (lane >> 3);
           if (key >= ne) continue;
-          const int type = stype[tb][key];
-          const int64_t r = srow[tb][key];
+          const int type = stype[st][key];
+          const int64_t r = srow[st][key];
           const int bytes = type ? 16 : 0;
           if (FP8) {
             cp_async16(Kt + 2 * kKB + tc::sw128(key, c), type ? p.crope + r * kDRope + c * 8 : p.crope, bytes);
@@ -827,7 +807,7 @@ __global__ void __maxnreg__(120) attn_tc_kernel(AttnParams p) {  // 17 warps x 3
         }
       }
       if (nw > 0) {  // raw window tokens: contiguous rows
-        const int64_t rw0 = srow[tb][ne];
+        const int64_t rw0 = srow[st][ne];
         for (int pc = pt; pc < nw * 24; pc += 256) {
           const int key = ne + pc / 24, c = pc % 24;
           cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.wk + rw0 * kDQK + pc * 8);
@@ -852,80 +832,38 @@ __global__ void __maxnreg__(120) attn_tc_kernel(AttnParams p) {  // 17 warps x 3
         }
       }
       cp_async_commit();
-    };
-    // code * scale -> bf16 into the swizzled K (and V) tile of `tile`
-    auto widen = [&](int tile) {
-      if (!FP8) return;
-      const int st = tile % NS;
-      uint8_t* Kt = Kst + st * 3 * kKB;
-      uint8_t* Vt = Vst + st * 2 * kKB;
-      int ne, nw;
-      runs(tile, ne, nw);
+      sel_next = load_sel(tile + 1);
+      if (FP8) {  // code * scale -> bf16 into the swizzled K (and V) tile; skipped slots get zeros
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int key = (pt >> 3) + 32 * j, c = pt & 7;
-        if (key >= ne) continue;
-        const uint32_t w4[4] = {codes[j].x, codes[j].y, codes[j].z, codes[j].w};
-        uint32_t outw[8];
+        for (int j = 0; j < 4; ++j) {
+          const int key = (pt >> 3) + 32 * j, c = pt & 7;
+          if (key >= ne) continue;
+          const uint32_t w4[4] = {codes[j].x, codes[j].y, codes[j].z, codes[j].w};
+          uint32_t outw[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t h01, h23;
-          e4m3x4_to_f16x2x2(w4[q], h01, h23);
-          const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-          const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-          outw[2 * q] = pack_bf16x2(f01.x * scl[j], f01.y * scl[j]);
-          outw[2 * q + 1] = pack_bf16x2(f23.x * scl[j], f23.y * scl[j]);
-        }
-        const int blk = c >> 2;
-        const uint4 lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-        const uint4 hi = make_uint4(outw[4], outw[5], outw[6], outw[7]);
-        *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
-        *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
-        if (!SHV) {
-          *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
-          *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
+          for (int q = 0; q < 4; ++q) {
+            uint32_t h01, h23;
+            e4m3x4_to_f16x2x2(w4[q], h01, h23);
+            const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+            const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+            outw[2 * q] = pack_bf16x2(f01.x * scl[j], f01.y * scl[j]);
+            outw[2 * q + 1] = pack_bf16x2(f23.x * scl[j], f23.y * scl[j]);
+          }
+          const int blk = c >> 2;
+          const uint4 lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+          const uint4 hi = make_uint4(outw[4], outw[5], outw[6], outw[7]);
+          *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
+          *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
+          if (!SHV) {
+            *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
+            *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
+          }
         }
       }
-    };
-    // describe, issue and load the codes of `tile` (its stage must be free)
-    auto start_tile = [&](int tile, int32_t sel) {
-      describe(tile, sel);
-      named_sync(1, 256);
-      issue(tile);
-    };
-
-    int32_t sel_next = load_sel(0);
-    if (ntiles > 0) {
-      start_tile(0, sel_next);
-      sel_next = load_sel(1);
-      load_codes(0);
-    }
-    for (int tile = 0; tile < ntiles; ++tile) {
-      const int st = tile % NS;
-      const bool ahead = kAhead && tile + 1 < ntiles;
-      if (ahead) {  // the next tile first: its copies overlap this tile's widening
-        const int nxt = tile + 1;
-        if (nxt >= NS && healthy) healthy = tc::bar_wait(&empty[nxt % NS], ((nxt / NS) - 1) & 1);
-        start_tile(nxt, sel_next);
-        sel_next = load_sel(nxt + 1);
-      }
-      widen(tile);
-      if (ahead) {
-        load_codes(tile + 1);  // in flight until the next iteration widens it
-        cp_async_wait<1>();    // this tile's group; the next tile's may still run
-      } else {
-        cp_async_wait<0>();
-      }
+      cp_async_wait<0>();
       tc::fence_async_smem();
       named_sync(1, 256);
       if (pt == 0) bar_arrive(&full[st]);
-      if (!kAhead && tile + 1 < ntiles) {  // two stages: the next tile after this one is published
-        const int nxt = tile + 1;
-        if (nxt >= NS && healthy) healthy = tc::bar_wait(&empty[nxt % NS], ((nxt / NS) - 1) & 1);
-        start_tile(nxt, sel_next);
-        sel_next = load_sel(nxt + 1);
-        load_codes(nxt);
-      }
     }
   } else {
     // ===================== softmax: thread = key of the tile, 32 heads =====================
@@ -938,7 +876,7 @@ __global__ void __maxnreg__(120) attn_tc_kernel(AttnParams p) {  // 17 warps x 3
       tc::fence_after_sync();
       float sv[32];
       tc::tmem_ld32(tmem + 64 * pb + lane_base + hb, sv);
-      const bool valid = (vmask[kst][key >> 5] >> (key & 31)) & 1u;
+      const bool valid = stype[kst][key] != 0;
       bool over = false;
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {

@@ -85,21 +85,19 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, 
 }
 
 // One byte of E2M1 codes (OCP MX FP4: sign, 2 exponent bits with bias 1,
-// 1 mantissa bit), the low nibble first -> an fp16 pair (low nibble in the low
-// half), exactly.  Every E2M1 magnitude is an fp16 value whose low byte is 0
-// and whose high byte is one of 0x00, 0x38, 0x3C, 0x3E, 0x40, 0x42, 0x44, 0x46
-// (0, 0.5, 1, 1.5, 2, 3, 4, 6); a byte permute picks the two high bytes from
-// that table by the nibbles' 3 magnitude bits, and the nibbles' sign bits move
-// to bits 15 and 31.
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-  const uint32_t sel = ((byte & 0x70u) << 8) | ((byte & 0x07u) << 4);  // byte 3 <- hi, byte 1 <- lo, 0 <- entry 0
-  const uint32_t mag = __byte_perm(0x3E3C3800u, 0x46444240u, sel);
-  return mag | ((byte & 0x08u) << 12) | ((byte & 0x80u) << 24);
+// 1 mantissa bit), the low nibble first -> an fp16 pair, the low nibble's
+// value in the low half (every E2M1 value is an fp16 value: exact).  The byte
+// is passed in the low 8 bits of a 16-bit register and narrowed to the 8-bit
+// operand the conversion takes.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint16_t byte) {
+  uint32_t r;
+  asm("{\n.reg .b8 t;\ncvt.u8.u16 t, %1;\ncvt.rn.f16x2.e2m1x2 %0, t;\n}\n" : "=r"(r) : "h"(byte));
+  return r;
 }
 // Two bytes of E2M1 codes -> fp16 pairs (byte 0's two values) and (byte 1's).
 __device__ __forceinline__ void e2m1x4_to_f16x2x2(uint16_t two_bytes, uint32_t& lo, uint32_t& hi) {
-  lo = e2m1x2_to_f16x2(two_bytes & 0xffu);
-  hi = e2m1x2_to_f16x2(static_cast<uint32_t>(two_bytes) >> 8);
+  lo = e2m1x2_to_f16x2(static_cast<uint16_t>(two_bytes & 0xffu));
+  hi = e2m1x2_to_f16x2(static_cast<uint16_t>(two_bytes >> 8));
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {

@@ -203,8 +203,11 @@ __global__ void __launch_bounds__(256) compress_flat_kernel(CompressParams p) {
     const int64_t j = start + r;
     raw[r] = (j >= 0 && j < er.T) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
   }
-  Acc8 acc;
-  acc.init();
+  // two passes over the rows in registers: the per-channel maximum of the
+  // logits, then one exponential per (row, channel)
+  float mx[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
 #pragma unroll
   for (int r = 0; r < CW; ++r) {
     const int64_t j = start + r;
@@ -212,18 +215,39 @@ __global__ void __launch_bounds__(256) compress_flat_kernel(CompressParams p) {
     float xv[8], bv[8];
     unpack8(raw[r], xv);
     load8f(p.b + r * p.d + 8 * g, bv);
-    acc.add(xv, wv, bv);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], fmaf(wv[c], xv[c], bv[c]));
+  }
+  float sm[8], ac[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) sm[c] = ac[c] = 0.f;
+#pragma unroll
+  for (int r = 0; r < CW; ++r) {
+    const int64_t j = start + r;
+    if (j < 0 || j >= er.T) continue;
+    float xv[8], bv[8];
+    unpack8(raw[r], xv);
+    load8f(p.b + r * p.d + 8 * g, bv);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float e = __expf(fmaf(wv[c], xv[c], bv[c]) - mx[c]);
+      sm[c] += e;
+      ac[c] = fmaf(e, xv[c], ac[c]);
+    }
   }
   uint4 o;
-  o.x = pack_bf16x2(acc.a[0] / acc.s[0], acc.a[1] / acc.s[1]);
-  o.y = pack_bf16x2(acc.a[2] / acc.s[2], acc.a[3] / acc.s[3]);
-  o.z = pack_bf16x2(acc.a[4] / acc.s[4], acc.a[5] / acc.s[5]);
-  o.w = pack_bf16x2(acc.a[6] / acc.s[6], acc.a[7] / acc.s[7]);
+  o.x = pack_bf16x2(ac[0] / sm[0], ac[1] / sm[1]);
+  o.y = pack_bf16x2(ac[2] / sm[2], ac[3] / sm[3]);
+  o.z = pack_bf16x2(ac[4] / sm[4], ac[5] / sm[5]);
+  o.w = pack_bf16x2(ac[6] / sm[6], ac[7] / sm[7]);
   *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + er.out_row * p.d + 8 * g) = o;
 }
 
 // One CTA per entry (long windows): 8 warps take interleaved rows, then warp 0
-// merges the 8 partial softmax states.
+// merges the 8 partial softmax states.  RPW > 0: the window is 8 * RPW rows
+// and each warp loads its RPW rows at once, then takes the maximum and one
+// exponential per element; RPW == 0: any window, online softmax per row.
+template <int RPW>
 __global__ void __launch_bounds__(256) compress_long_kernel(CompressParams p) {
   pdl_wait();
   pdl_trigger();
@@ -239,12 +263,45 @@ __global__ void __launch_bounds__(256) compress_long_kernel(CompressParams p) {
     float wv[8];
     load8f(p.w + 8 * lane, wv);
     const __nv_bfloat16* xb = er.x0 + 8 * lane;
+    if constexpr (RPW > 0) {
+      uint4 raw[RPW];
+#pragma unroll
+      for (int i = 0; i < RPW; ++i) {  // rows start + warp + 8 i, all loads in flight together
+        const int64_t j = start + warp + 8 * i;
+        raw[i] = (j >= j0 && j < j1) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < RPW; ++i) {
+        const int64_t j = start + warp + 8 * i;
+        if (j < j0 || j >= j1) continue;
+        float xv[8], bv[8];
+        unpack8(raw[i], xv);
+        load8f(p.b + (warp + 8 * i) * p.d + 8 * lane, bv);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc.m[c] = fmaxf(acc.m[c], fmaf(wv[c], xv[c], bv[c]));
+      }
+#pragma unroll
+      for (int i = 0; i < RPW; ++i) {
+        const int64_t j = start + warp + 8 * i;
+        if (j < j0 || j >= j1) continue;
+        float xv[8], bv[8];
+        unpack8(raw[i], xv);
+        load8f(p.b + (warp + 8 * i) * p.d + 8 * lane, bv);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float e = __expf(fmaf(wv[c], xv[c], bv[c]) - acc.m[c]);
+          acc.s[c] += e;
+          acc.a[c] = fmaf(e, xv[c], acc.a[c]);
+        }
+      }
+    } else {
 #pragma unroll 4
-    for (int64_t j = j0 + warp; j < j1; j += 8) {
-      float xv[8], bv[8];
-      unpack8(ldg_nc16(xb + j * p.d), xv);
-      load8f(p.b + (j - start) * p.d + 8 * lane, bv);
-      acc.add(xv, wv, bv);
+      for (int64_t j = j0 + warp; j < j1; j += 8) {
+        float xv[8], bv[8];
+        unpack8(ldg_nc16(xb + j * p.d), xv);
+        load8f(p.b + (j - start) * p.d + 8 * lane, bv);
+        acc.add(xv, wv, bv);
+      }
     }
   }
 #pragma unroll
@@ -322,8 +379,10 @@ csa_status launch(const char* name, const CompressParams& p, int64_t entries, vo
                    p);
   } else if (p.cwin <= 32) {
     e = launch_pdl(compress_short_kernel, dim3(static_cast<unsigned>((entries + 7) / 8)), dim3(256), 0, s, 1, p);
+  } else if (p.cwin == 128) {  // HCA with m' = 128: 16 rows per warp
+    e = launch_pdl(compress_long_kernel<16>, dim3(static_cast<unsigned>(entries)), dim3(256), 0, s, 1, p);
   } else {
-    e = launch_pdl(compress_long_kernel, dim3(static_cast<unsigned>(entries)), dim3(256), 0, s, 1, p);
+    e = launch_pdl(compress_long_kernel<0>, dim3(static_cast<unsigned>(entries)), dim3(256), 0, s, 1, p);
   }
   prof_end(s);
   return check_launch(name, e);

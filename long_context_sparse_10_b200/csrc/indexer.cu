@@ -1470,6 +1470,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
 size_t align_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 bool use_row_path(int64_t R, int64_t N) { return N <= kRowPathMaxN && R > 256; }
+// Prefill rows with bf16 keys run the on-chip tcgen05 kernel, whose 16-bit
+// histogram bins hold up to 65535 entries.
+constexpr int64_t kPrefillTcMaxN = 65535;
+bool use_prefill_tc(int64_t R, int64_t N) { return N <= kPrefillTcMaxN && R > 256; }
 
 struct LongLayout {
   size_t scores, hist, cnt, done, thr, cand, bitmap, total;
@@ -1506,7 +1510,8 @@ int64_t query_rows(int64_t B, int64_t Tq) {
 size_t workspace_bytes(int64_t B, int64_t Tq, int64_t N, bool coded = false) {
   const int64_t R = query_rows(B, Tq);
   if (R <= 0 || N <= 0 || N >= (int64_t(1) << 31)) return 0;
-  if (use_row_path(R, N)) return coded ? align_up(static_cast<size_t>(R) * N * 4) : 0;
+  if (!coded && use_prefill_tc(R, N)) return 0;
+  if (coded && use_row_path(R, N)) return align_up(static_cast<size_t>(R) * N * 4);
   return long_layout(R, N).total;
 }
 
@@ -1686,7 +1691,7 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   } else {
     CSA_REQUIRE_PTR(kIc);
   }
-  const bool tc_rows = !e4 && scores_out == nullptr && use_row_path(R, N);  // tcgen05 prefill path
+  const bool tc_rows = !e4 && scores_out == nullptr && use_prefill_tc(R, N);  // tcgen05 prefill path
   const size_t need = tc_rows ? 0 : csa::workspace_bytes(B, Tq, N, true);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need))
     return fail(CSA_ERR_WORKSPACE, "csa_indexer_topk: workspace of %zu bytes needed (got %zu)", need,
@@ -1909,6 +1914,11 @@ extern "C" csa_status csa_indexer_topk_packed(const void* qI, const float* wI, c
   if (packed->n_seqs == 0 || packed->total_tokens == 0) return CSA_OK;
   CSA_REQUIRE(packed->cu_tokens != nullptr && packed->cu_entries != nullptr,
               "csa_indexer_topk_packed: packed offsets are NULL");
+  const int64_t max_n = (static_cast<int64_t>(packed->max_tokens) + m - 1) / m;
+  if (max_n > kPrefillTcMaxN)
+    return fail(CSA_ERR_UNSUPPORTED,
+                "csa_indexer_topk_packed: sequences of up to %lld entries are supported (longest has %lld)",
+                static_cast<long long>(kPrefillTcMaxN), static_cast<long long>(max_n));
   CSA_REQUIRE_PTR(qI);
   CSA_REQUIRE_PTR(wI);
   CSA_REQUIRE_PTR(kIc);

@@ -194,6 +194,8 @@ WORKLOADS = {
     "hca_prefill_t8192": Prefill("hca_prefill_t8192", "hca", B=2, T=8192, H=16, m=128),
     "csa_decode_l131072": Decode("csa_decode_l131072", "csa", B=64, L=131072, H=64, m=4, k=2048),
     "csa_prefill_t65536": Prefill("csa_prefill_t65536", "csa", B=1, T=65536, H=64, m=4, k=2048),
+    # the same shapes at a quarter of the length (for counter captures: inputs above L2, ~1 GB in all)
+    "csa_prefill_t16384": Prefill("csa_prefill_t16384", "csa", B=1, T=16384, H=64, m=4, k=2048),
     "hybrid_decode_l1m": Decode("hybrid_decode_l1m", "hybrid", B=8, L=1 << 20, H=64, m=4, k=2048),
     # the same workload with FP8 (E4M3 + per-entry scale) lightning-indexer keys
     "hybrid_decode_l1m_fp8idx": Decode("hybrid_decode_l1m_fp8idx", "hybrid", B=8, L=1 << 20, H=64, m=4, k=2048,
