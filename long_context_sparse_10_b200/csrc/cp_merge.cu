@@ -53,13 +53,21 @@ __device__ __forceinline__ uint32_t scan_excl(uint32_t v, uint32_t* total, uint3
 // index order (each rank's list is ascending and ranks hold increasing
 // ranges), so "ties to the lower index" is "ties to the lower position" and
 // an ordered compaction of the chosen positions is the ascending output.
+// One CTA per query row.  Candidate c (position in the rank-ordered list) has
+// score s[c] and global index i[c] (-1: none).  Positions are in ascending
+// index order (each rank's list is ascending and ranks hold increasing
+// ranges), so "ties to the lower index" is "ties to the lower position" and
+// an ordered compaction of the chosen positions is the ascending output.  The
+// k-th largest key is found by a radix select in levels of 11, 11 and 10 bits
+// (2048-bin shared histograms: the candidates' scores spread over far more
+// first-level bins than over the key's top byte, so the atomics collide less).
 __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(const float* __restrict__ cs,
                                                                     const int32_t* __restrict__ ci, int n, int k,
                                                                     int32_t* __restrict__ idx) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint32_t keys[];  // order-preserving score key; 0 marks an empty candidate
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[2048];
   __shared__ uint32_t scan_sh[32];
   __shared__ uint32_t dig[2];
   const int64_t row = blockIdx.x;
@@ -77,46 +85,35 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(const float* 
   scan_excl(nvalid_local, &nvalid, scan_sh);
   uint32_t prefix = 0, remaining = static_cast<uint32_t>(k);
   if (nvalid > static_cast<uint32_t>(k)) {
-    uint32_t mask = 0;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int j = threadIdx.x; j < 256; j += kMergeThreads) hist[j] = 0;
+    for (int level = 0; level < 3; ++level) {
+      const int bits = level == 2 ? 10 : 11;
+      const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
+      const uint32_t nb = 1u << bits;
+      for (uint32_t j = threadIdx.x; j < nb; j += kMergeThreads) hist[j] = 0;
       __syncthreads();
       for (int c = threadIdx.x; c < n; c += kMergeThreads) {
         const uint32_t key = keys[c];
-        if (key != 0u && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        if (key != 0u && (level == 0 || (key >> (shift + bits)) == prefix))
+          atomicAdd(&hist[(key >> shift) & (nb - 1u)], 1u);
       }
       __syncthreads();
-      if (threadIdx.x < 32) {  // walk the digits from the top for the `remaining`-th largest
-        const int lane = threadIdx.x;
-        uint32_t cnt[8], sum = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          cnt[j] = hist[255 - 8 * lane - j];
-          sum += cnt[j];
-        }
-        uint32_t incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
-        }
-        const uint32_t excl = incl - sum;
-        if (excl < remaining && incl >= remaining) {
-          uint32_t acc = excl;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (acc + cnt[j] >= remaining) {
-              dig[0] = 255 - 8 * lane - j;
-              dig[1] = acc;
-              break;
-            }
-            acc += cnt[j];
-          }
+      // thread t owns bins nb-1-2t and nb-2-2t (walked from the top)
+      const uint32_t b0 = nb - 1u - 2u * threadIdx.x, b1 = b0 - 1u;
+      const bool own = 2u * threadIdx.x < nb;
+      const uint32_t c0 = own ? hist[b0] : 0u, c1 = own ? hist[b1] : 0u;
+      uint32_t total;
+      const uint32_t excl = scan_excl(c0 + c1, &total, scan_sh);
+      if (own && excl < remaining && excl + c0 + c1 >= remaining) {
+        if (excl + c0 >= remaining) {
+          dig[0] = b0;
+          dig[1] = excl;
+        } else {
+          dig[0] = b1;
+          dig[1] = excl + c0;
         }
       }
       __syncthreads();
-      prefix |= dig[0] << shift;
-      mask |= 255u << shift;
+      prefix = (prefix << bits) | dig[0];
       remaining -= dig[1];
       __syncthreads();
     }

@@ -803,17 +803,22 @@ __global__ void __launch_bounds__(1024) topk_rows_kernel(RowsParams p) {
 // (query, head) pairs as N (kPfQ * 4 = 128 columns), K = 64; an epilogue
 // thread owns one entry of the tile and folds its 4 heads per query
 // (s_q = sum_h relu(S[e, 4q+h]) w[q, h]) into the order-preserving 32-bit key
-// of each query's score, which it stages in shared memory.  The keys are then
-// read back query-major: four consecutive lanes of a warp own one query and 32
+// of each query's score, which it stages in shared memory; eight epilogue
+// warps work in two halves of 16 queries (64 accumulator columns) each, so
+// every scheduler has two warps to interleave.  The keys are then read back
+// query-major: eight consecutive lanes of a warp own one query and 16
 // consecutive entries of the tile each, so a query's running state lives in
 // registers of its own lanes and no two lanes of a warp share a histogram row
-// unless they share the query.  The exact top-k is a radix select on the key,
-// 8 bits per level, over passes that recompute the same scores (the MMA is
+// unless they share the query; runs of equal bins are counted in a register
+// before one atomic.  The exact top-k is a radix select on the key, in
+// levels of 11, 11 and 10 bits, over passes that recompute the same scores (the MMA is
 // cheap; no score leaves the SM):
-//   passes 0-3: per-query 256-bin histogram of key byte 3, then of byte 2 for
-//               entries whose byte 3 is the query's threshold byte, and so on;
-//               a query whose threshold bin is taken whole stops refining;
-//   pass 4:     emission -- every entry above the threshold and the first
+//   passes 0-2: per-query 2048-bin histogram of key bits 31..21, then of bits
+//               20..10 for entries whose top bits are the query's threshold
+//               bin, then bits 9..0; a query whose threshold bin is taken
+//               whole stops refining, and a pass scores only the queries that
+//               still refine;
+//   pass 3:     emission -- every entry above the threshold and the first
 //               `need` entries equal to it, in ascending index order (ties
 //               therefore go to the lower index), by a 4-lane scan per query.
 // A pass no query needs only waits for its tiles.  The key tiles stream by TMA
@@ -821,22 +826,27 @@ __global__ void __launch_bounds__(1024) topk_rows_kernel(RowsParams p) {
 // the MMAs into two TMEM buffers, and all waits are bounded.
 constexpr int kPfQ = 32;         // query rows per CTA (x 4 heads = 128 MMA columns)
 constexpr int kPfTile = 128;     // entries per tile (MMA M)
-constexpr int kPfStages = 4;
-constexpr int kPfThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int kPfLevels = 4;     // histogram levels of 8 key bits
-constexpr int kPfHistW = 129;    // words per query histogram: 256 16-bit bins + 1 pad (bank spread)
+constexpr int kPfStages = 3;
+constexpr int kPfThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue (two halves of 16 queries)
+constexpr int kPfEpi = 256;      // epilogue threads
+constexpr int kPfLanesQ = 8;     // lanes per query in the query-major phase (16 entries of a tile each)
+constexpr int kPfLevels = 3;     // histogram levels: key bits 31..21, 20..10, 9..0
+constexpr int kPfHistW = 1025;   // words per query histogram: 2048 16-bit bins + 1 pad (bank spread)
 constexpr int kPfKeyW = 132;     // words per query row of staged keys: 4 quarters x 33 (bank spread)
+__host__ __device__ constexpr int pf_level_bits(int level) { return level == 2 ? 10 : 11; }
+__host__ __device__ constexpr int pf_level_shift(int level) { return level == 0 ? 21 : (level == 1 ? 10 : 0); }
 
 struct PfLayout {
   static constexpr size_t kK = 0;                                  // [kPfStages][128 entries][128 B]
   static constexpr size_t kQ = kK + kPfStages * 16384;             // [128 (query, head)][128 B]
   static constexpr size_t kHist = kQ + 16384;                      // [kPfQ][kPfHistW] u32
-  static constexpr size_t kKeys = kHist + kPfQ * kPfHistW * 4;     // [2][kPfQ][kPfKeyW] u32
-  static constexpr size_t kW = kKeys + 2 * kPfQ * kPfKeyW * 4;     // [128] fp32
-  static constexpr size_t kQs = kW + 128 * 4;                      // per-query state, 8 x [kPfQ] u32
-  static constexpr size_t kBars = (kQs + 8 * kPfQ * 4 + 7) / 8 * 8;
-  static constexpr size_t kTotal = kBars + 128 + 1024;             // + alignment slack
+  static constexpr size_t kKeys = kHist + kPfQ * kPfHistW * 4;     // [kPfQ][kPfKeyW] u32
+  static constexpr size_t kW = kKeys + kPfQ * kPfKeyW * 4;         // [128] fp32
+  static constexpr size_t kQs = kW + 128 * 4;                      // per-query state, 7 x [kPfQ] u32
+  static constexpr size_t kBars = (kQs + 7 * kPfQ * 4 + 7) / 8 * 8;
+  static constexpr size_t kTotal = kBars + 96 + 1024;              // + alignment slack
 };
+static_assert(PfLayout::kTotal <= 232448, "prefill indexer shared memory above the per-block limit");
 
 struct PfParams {
   const __nv_bfloat16* qI;  // [B, Tq, 4, 64]
@@ -871,7 +881,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
   uint32_t* rem_s = qs + 3 * kPfQ;     // entries still to take at the current level
   uint32_t* shift_s = qs + 4 * kPfQ;   // emission: compare key >> shift with thr, take need ties
   uint32_t* thr_s = qs + 5 * kPfQ;
-  uint32_t* need_s = qs + 6 * kPfQ;
+  uint32_t* need_s = qs + 6 * kPfQ;    // (7 state arrays)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + PfLayout::kBars);  // [kPfStages]
   uint64_t* empty = full + kPfStages;                                     // [kPfStages]
   uint64_t* tfull = empty + kPfStages;                                    // [2]
@@ -938,7 +948,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
     }
     for (int i = 0; i < 2; ++i) {
       tc::bar_init(&tfull[i], 1);
-      tc::bar_init(&tempty[i], 128);
+      tc::bar_init(&tempty[i], kPfEpi);
     }
     tc::bar_init_fence();
   }
@@ -992,85 +1002,115 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
     }
   } else {
     // ===================== epilogue =====================
-    // scoring: thread = entry et of the tile (its TMEM lane); then query-major:
-    // thread = (query qj = etid / 4, quarter qq = etid % 4 of the tile's entries)
-    const int q4 = warp & 3;  // TMEM lane quarter of this warp
+    // scoring: thread = entry et of the tile (its TMEM lane), queries of half
+    // hq; then query-major: thread = (query qj of the half, part qp: entries
+    // 16 qp .. 16 qp + 15 of the tile)
+    const int ew = warp - 2;            // 0..7
+    const int hq = ew >> 2;             // query half: queries 16 hq .. 16 hq + 15
+    const int q4 = warp & 3;            // TMEM lane quarter of this warp
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-    const int et = q4 * 32 + lane;  // entry within the tile (scoring)
-    const int etid = tid - 64;      // 0..127
-    const int qj = etid >> 2, qq = etid & 3;
+    const int et = q4 * 32 + lane;      // entry within the tile (scoring)
+    const int htid = (ew & 3) * 32 + lane;  // 0..127 within the half
+    const int qj = hq * 16 + (htid >> 3), qp = htid & 7;
     const int64_t qrow = row0 + qj;
-    // key slot of entry et for query j: quarter-padded rows spread the banks
-    auto key_slot = [&](int buf, int j, int e) { return (buf * kPfQ + j) * kPfKeyW + (e >> 5) * 33 + (e & 31); };
+    const int bar_half = 3 + hq;        // named barrier of this half
+    // key slot of entry e for query j: quarter-padded rows spread the banks
+    auto key_slot = [&](int j, int e) { return j * kPfKeyW + (e >> 5) * 33 + (e & 31); };
     // A wait that runs out (recorded in the device error word) skips the later
-    // waits but keeps the loop and its named barriers, so the four warps stay
-    // in step and the CTA finishes; its output is then not valid.
+    // waits but keeps the loop and its named barriers, so the warps stay in
+    // step and the CTA finishes; its output is then not valid.
     bool healthy = true;
     int it = 0;
-    uint32_t sel_done = 0u, ties_done = 0u;  // emission running totals of query qj (same in its 4 lanes)
+    uint32_t sel_done = 0u, ties_done = 0u;  // emission running totals of query qj (same in its 8 lanes)
     for (int pass = 0; pass < kPasses; ++pass) {
-      // does any query refine at this level (passes 0..3)?  the last pass always emits
-      bool active = pass == kPfLevels;
-      if (!active) {
-        for (int j = 0; j < kPfQ; ++j) active |= level_s[j] == static_cast<uint32_t>(pass);
+      const bool emit = pass == kPfLevels;
+      // queries of this half that need their scores in this pass (bit j - 16 hq)
+      uint32_t need_mask = 0u;
+      for (int j = 0; j < 16; ++j) {
+        const int jq = hq * 16 + j;
+        const bool w = emit ? nv_s[jq] > 0u : level_s[jq] == static_cast<uint32_t>(pass);
+        need_mask |= w ? (1u << j) : 0u;
       }
       // this thread's query state for the pass
       const uint32_t nv_q = nv_s[qj], lv_q = level_s[qj], pre_q = prefix_s[qj];
       const uint32_t sh_q = shift_s[qj], thr_q = thr_s[qj], need_q = need_s[qj];
+      const bool mine = (need_mask >> (qj - hq * 16)) & 1u;
       for (int tile = 0; tile < ntiles; ++tile, ++it) {
         const int buf = it & 1;
         if (healthy) healthy = tc::bar_wait(&tfull[buf], static_cast<uint32_t>((it >> 1) & 1));
         tc::fence_after_sync();
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {  // 8 queries (32 accumulator columns) at a time
+        for (int c = 0; c < 2; ++c) {  // 8 queries (32 accumulator columns) at a time
+          const uint32_t cmask = (need_mask >> (c * 8)) & 0xffu;
           float v[32];
-          if (active) tc::tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 128 + c * 32), v);
-          if (c == 3) {
+          if (cmask) tc::tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 128 + hq * 64 + c * 32), v);
+          if (c == 1) {
             tc::fence_before_sync();
             bar_arrive(&tempty[buf]);
           }
-          if (!active) continue;
+          if (!cmask) continue;
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int j = c * 8 + jj;
+          for (int jj = 0; jj < 8; ++jj) {  // all 8 queries of the chunk (unneeded keys are not read)
+            const int j = hq * 16 + c * 8 + jj;
             const float4 w4 = *reinterpret_cast<const float4*>(w_s + 4 * j);
             const float sc = fmaxf(v[4 * jj], 0.f) * w4.x + fmaxf(v[4 * jj + 1], 0.f) * w4.y +
                              fmaxf(v[4 * jj + 2], 0.f) * w4.z + fmaxf(v[4 * jj + 3], 0.f) * w4.w;
-            keys_s[key_slot(buf, j, et)] = f2key(sc + 0.0f);
+            keys_s[key_slot(j, et)] = f2key(sc + 0.0f);
           }
         }
-        if (!active) continue;
-        named_sync_ix(3, 128);  // the tile's keys are staged (a buffer per tile parity)
-        const int e0 = qq * 32;                                  // this thread's first entry of the tile
-        const uint32_t eabs0 = static_cast<uint32_t>(tile * kPfTile + e0);
-        const int nvis = static_cast<int>(nv_q > eabs0 ? (nv_q - eabs0 < 32u ? nv_q - eabs0 : 32u) : 0u);
-        const uint32_t* kr = keys_s + key_slot(buf, qj, e0);
-        if (pass < kPfLevels) {
-          if (lv_q == static_cast<uint32_t>(pass)) {
-            const int bsh = 24 - 8 * pass;
+        if (!need_mask) continue;        // uniform for the half
+        named_sync_ix(bar_half, 128);    // this half's keys of the tile are staged
+        if (mine) {
+          const int e0 = qp * 16;                                  // this thread's first entry of the tile
+          const uint32_t eabs0 = static_cast<uint32_t>(tile * kPfTile + e0);
+          const int nvis = static_cast<int>(nv_q > eabs0 ? (nv_q - eabs0 < 16u ? nv_q - eabs0 : 16u) : 0u);
+          uint32_t kv[16];
+          {
+            const uint32_t* kr = keys_s + key_slot(qj, e0);  // 16 consecutive slots in one quarter
+#pragma unroll
+            for (int i = 0; i < 16; ++i) kv[i] = kr[i];
+          }
+          if (!emit) {
+            const int bsh = pf_level_shift(pass);
+            const uint32_t bmask = (1u << pf_level_bits(pass)) - 1u;
+            const int psh = bsh + pf_level_bits(pass);  // bits above this level's
             uint32_t* h = hist + qj * kPfHistW;
-            for (int i = 0; i < nvis; ++i) {
-              const uint32_t key = kr[i];
-              if (pass == 0 || (key >> (bsh + 8)) == pre_q) {
-                const uint32_t bin = (key >> bsh) & 255u;
-                atomicAdd(h + (bin >> 1), 1u << ((bin & 1u) * 16));
+            uint32_t cur = 0xffffffffu, run = 0u;  // runs of equal bins: one atomic per run
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const uint32_t key = kv[i];
+              const bool in = i < nvis && (pass == 0 || (key >> psh) == pre_q);
+              const uint32_t bin = (key >> bsh) & bmask;
+              if (in && bin != cur) {
+                if (run) atomicAdd(h + (cur >> 1), run << ((cur & 1u) * 16));
+                cur = bin;
+                run = 0u;
               }
+              run += in ? 1u : 0u;
+            }
+            if (run) atomicAdd(h + (cur >> 1), run << ((cur & 1u) * 16));
+          }
+        }
+        if (emit) {  // every lane of the half: the scans below are warp-wide
+          uint32_t gt = 0u, eq = 0u;
+          const int e0 = qp * 16;
+          const uint32_t eabs0 = static_cast<uint32_t>(tile * kPfTile + e0);
+          if (mine) {
+            const int nvis = static_cast<int>(nv_q > eabs0 ? (nv_q - eabs0 < 16u ? nv_q - eabs0 : 16u) : 0u);
+            const uint32_t* kr = keys_s + key_slot(qj, e0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const uint32_t kk = kr[i] >> sh_q;
+              gt |= (i < nvis && kk > thr_q) ? (1u << i) : 0u;
+              eq |= (i < nvis && kk == thr_q) ? (1u << i) : 0u;
             }
           }
-        } else {
-          // emission: entries above the threshold, and ties at it in index order
-          uint32_t gt = 0u, eq = 0u;
-          for (int i = 0; i < nvis; ++i) {
-            const uint32_t kk = kr[i] >> sh_q;
-            gt |= kk > thr_q ? (1u << i) : 0u;
-            eq |= kk == thr_q ? (1u << i) : 0u;
-          }
           const uint32_t n_eq = __popc(eq);
-          uint32_t tie_incl = n_eq;  // scan over the query's 4 lanes (entries in order)
+          uint32_t tie_incl = n_eq;  // scan over the query's 8 lanes (entries in order)
 #pragma unroll
-          for (int o = 1; o < 4; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(0xffffffffu, tie_incl, o, 4);
-            if (qq >= o) tie_incl += t;
+          for (int o = 1; o < kPfLanesQ; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, tie_incl, o, kPfLanesQ);
+            if (qp >= o) tie_incl += t;
           }
           const uint32_t tie0 = ties_done + tie_incl - n_eq;  // rank of this thread's first tie
           const uint32_t take = need_q > tie0 ? (need_q - tie0 < n_eq ? need_q - tie0 : n_eq) : 0u;
@@ -1081,31 +1121,41 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
           const uint32_t n_sel = __popc(sel);
           uint32_t sel_incl = n_sel;
 #pragma unroll
-          for (int o = 1; o < 4; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(0xffffffffu, sel_incl, o, 4);
-            if (qq >= o) sel_incl += t;
+          for (int o = 1; o < kPfLanesQ; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, sel_incl, o, kPfLanesQ);
+            if (qp >= o) sel_incl += t;
           }
           uint32_t pos = sel_done + sel_incl - n_sel;
           for (uint32_t m = sel; m != 0u; m &= m - 1u) {
             if (pos < static_cast<uint32_t>(k)) p.idx[qrow * k + pos] = static_cast<int32_t>(eabs0 + __ffs(m) - 1);
             ++pos;
           }
-          ties_done += __shfl_sync(0xffffffffu, tie_incl, (lane & ~3) | 3);
-          sel_done += __shfl_sync(0xffffffffu, sel_incl, (lane & ~3) | 3);
+          const int last = (lane & ~(kPfLanesQ - 1)) | (kPfLanesQ - 1);
+          ties_done += __shfl_sync(0xffffffffu, tie_incl, last);
+          sel_done += __shfl_sync(0xffffffffu, sel_incl, last);
         }
+        named_sync_ix(bar_half, 128);  // the keys are read: the next tile may overwrite them
       }
-      if (pass == kPfLevels) break;
-      // ---- thresholds of the queries that refined at this level ----
-      named_sync_ix(3, 128);
-      for (int j = q4; j < kPfQ; j += 4) {
+      if (emit) break;
+      // ---- thresholds of the queries that refined at this level (all 8 warps) ----
+      named_sync_ix(2, kPfEpi);
+      const int nbits = pf_level_bits(pass);
+      const int per_lane = (1 << nbits) / 32;  // bins per lane, walked from the top
+      for (int j = ew; j < kPfQ; j += 8) {
         if (level_s[j] != static_cast<uint32_t>(pass)) continue;  // uniform in the warp
         const uint32_t* h = hist + j * kPfHistW;
-        uint32_t cbin[8], sum = 0;  // lane's 8 bins, walked from the top: 255 - 8 lane - i
+        const int top = (1 << nbits) - lane * per_lane;  // this lane's bins [top - per_lane, top)
+        // the lanes' bin sums, read transposed: at step c the warp reads lane c's words side by side
+        // (consecutive words, no bank conflict) and reduces them, and lane c keeps the total
+        const int wpl = per_lane / 2;  // words per lane
+        uint32_t sum = 0;
+        for (int c = 0; c < 32; ++c) {
+          const int wbase = ((1 << nbits) - (c + 1) * per_lane) / 2;
+          uint32_t v = lane < wpl ? h[wbase + lane] : 0u;
+          v = (v & 0xffffu) + (v >> 16);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int bb = 255 - 8 * lane - i;
-          cbin[i] = (h[bb >> 1] >> ((bb & 1) * 16)) & 0xffffu;
-          sum += cbin[i];
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == c) sum = v;
         }
         uint32_t incl = sum;
 #pragma unroll
@@ -1117,14 +1167,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
         const uint32_t rem = rem_s[j];
         if (excl < rem && incl >= rem) {
           uint32_t acc = excl;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (acc + cbin[i] >= rem) {
-              const uint32_t bb = static_cast<uint32_t>(255 - 8 * lane - i);
+          for (int bb = top - 1; bb >= top - per_lane; --bb) {
+            const uint32_t cb = (h[bb >> 1] >> ((bb & 1) * 16)) & 0xffffu;
+            if (acc + cb >= rem) {
               const uint32_t nrem = rem - acc;  // still needed from bin bb
-              const uint32_t pref = (prefix_s[j] << 8) | bb;
-              if (cbin[i] == nrem || pass == kPfLevels - 1) {  // threshold found; its ties go in index order
-                shift_s[j] = static_cast<uint32_t>(24 - 8 * pass);
+              const uint32_t pref = (prefix_s[j] << nbits) | static_cast<uint32_t>(bb);
+              if (cb == nrem || pass == kPfLevels - 1) {  // threshold found; its ties go in index order
+                shift_s[j] = static_cast<uint32_t>(pf_level_shift(pass));
                 thr_s[j] = pref;
                 need_s[j] = nrem;
                 level_s[j] = static_cast<uint32_t>(kPfLevels);
@@ -1135,18 +1184,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
               }
               break;
             }
-            acc += cbin[i];
+            acc += cb;
           }
         }
       }
-      named_sync_ix(3, 128);  // every warp is done reading the histograms
-      for (int i = etid; i < kPfQ * kPfHistW; i += 128) hist[i] = 0u;
-      named_sync_ix(3, 128);
+      named_sync_ix(2, kPfEpi);  // every warp is done reading the histograms
+      for (int i = ew * 32 + lane; i < kPfQ * kPfHistW; i += kPfEpi) hist[i] = 0u;
+      named_sync_ix(2, kPfEpi);
     }
-    // padding after each query's selection (its 4 lanes hold the running total)
+    // padding after each query's selection (its 8 lanes hold the running total)
     if (qj < nq) {
       const uint32_t done = sel_done < static_cast<uint32_t>(k) ? sel_done : static_cast<uint32_t>(k);
-      for (uint32_t c = done + qq; c < static_cast<uint32_t>(k); c += 4) p.idx[qrow * k + c] = -1;
+      for (uint32_t c = done + qp; c < static_cast<uint32_t>(k); c += kPfLanesQ) p.idx[qrow * k + c] = -1;
     }
   }
   tc::fence_before_sync();
