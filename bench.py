@@ -78,29 +78,86 @@ def profile_traffic(kernel: str, source: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while a region runs."""
+    """SM clock / throttle-reason samples while a region runs.
 
+    Polls NVML in a thread (every 5 ms) on the GPU that torch's device `dev` is (matched by UUID, then PCI bus
+    id), and takes one more sample when `mark()` is called after the region's work is enqueued, so that even a
+    region of a few milliseconds has a sample taken while the GPU is busy.  Without NVML it falls back to an
+    `nvidia-smi -lms 50` child.  Only reads: no clock, power or mode setting is touched."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
         self.dev = device_index
+        self.samples = []  # (sm_mhz, max_mhz, set of reasons)
+        self.nvml = None
         self.proc = None
         self.lines = []
+        self.stop = threading.Event()
+        self.source = "none"
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+        except Exception:
+            pass
+        try:
+            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def _sample_nvml(self):
+        nv, h = self.nvml
+        try:
+            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except Exception:
+            return
+        reasons = {name for name, const in self.REASONS if bits & getattr(nv, const, 0)}
+        self.samples.append((float(sm), float(mx), reasons))
+
+    def _poll(self):
+        while not self.stop.wait(0.005):
+            self._sample_nvml()
 
     def __enter__(self):
+        try:
+            self.nvml = self._nvml_handle()
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            self.source = "nvidia-smi"
             time.sleep(0.4)
         except OSError:
             self.proc = None
         self.t0 = time.time()
         return self
+
+    def mark(self):
+        """One sample now (call it after the region's work is enqueued, while the GPU runs it)."""
+        if self.nvml is not None:
+            self._sample_nvml()
 
     def _read(self):
         for line in self.proc.stdout:
@@ -108,6 +165,9 @@ class ClockSampler:
 
     def __exit__(self, *exc):
         self.t1 = time.time()
+        self.stop.set()
+        if self.nvml is not None:
+            self.thread.join(timeout=1)
         if self.proc is not None:
             time.sleep(0.1)
             self.proc.terminate()
@@ -116,25 +176,29 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
-        rows = [l for (t, l) in self.lines if self.t0 <= t <= self.t1 + 0.06]
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
+    def _smi_samples(self):
+        names = [n for n, _ in self.REASONS]
+        out = []
+        for t, r in self.lines:
+            if not (self.t0 <= t <= self.t1 + 0.06):
+                continue
             parts = [x.strip() for x in r.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                sm, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+            out.append((sm, mx, {n for n, v in zip(names, parts[5:9]) if v.lower().startswith("active")}))
+        return out
+
+    def summary(self):
+        rows = self.samples if self.nvml is not None else self._smi_samples()
+        sm = [r[0] for r in rows]
+        mx = rows[-1][1] if rows else None
+        reasons = set().union(*[r[2] for r in rows]) if rows else set()
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "source": self.source}
 
 
 # ---------------------------------------------------------------------------
@@ -844,6 +908,7 @@ def main():
         for _ in range(args.steps):
             graph.replay()
         ev1.record()
+        clocks.mark()
         torch.cuda.synchronize()
     barrier()
     ms = replicas.max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
