@@ -513,8 +513,14 @@ constexpr int kTcDecThreads = 544;  // attn_tc_kernel: warps 0-7 softmax, 8-15 l
 constexpr float kRescaleLog2 = 20.f;  // rescale O and l when a logit tops m_ref by more than 2^20
 
 struct TcLayout {
-  size_t q, k, v, p, ones, stype, srow, vmask, mref, corr, wmax, bars, total;
+  size_t q, k, v, p, ones, stype, srow, mref, corr, wmax, bars, total;
 };
+
+// Slot types of the last four tiles (ring indexed by tile % 4): 0 skipped, 1
+// compressed entry, 2 raw window token.  A tile's slot is rewritten only after
+// the softmax of the tile four back has finished with it.
+constexpr int kTypeRing = 4;
+
 
 // K-tile stages: three when the V tile is the K tile, two otherwise.
 __host__ __device__ constexpr int tc_stages(bool shv) { return shv ? 3 : 2; }
@@ -528,9 +534,8 @@ __host__ __device__ inline TcLayout tc_layout(bool fp8, bool shv, int tps) {
   L.v = off; if (!shv) off += ns * 2 * 16384;    // V: stages x 128 keys x 128 dims
   L.p = off; off += 2 * 16384;                   // P^T: 2 buffers x 128 keys x 64 heads (epilogue: O^T transpose)
   L.ones = off; off += 1024;                     // all-ones swizzle atom
-  L.stype = off; off += ns * kTcKeys * sizeof(int);
-  L.srow = off; off += ns * kTcKeys * sizeof(int64_t);
-  L.vmask = off; off += ns * 4 * sizeof(uint32_t);
+  L.stype = off; off += kTypeRing * kTcKeys * sizeof(int);
+  L.srow = off; off += kTypeRing * kTcKeys * sizeof(int64_t);
   L.mref = off; off += 64 * sizeof(float);
   L.corr = off; off += 64 * sizeof(float);
   L.wmax = off; off += 4 * 64 * sizeof(float);
@@ -553,6 +558,11 @@ __device__ __forceinline__ bool named_sync_or(int id, int n, bool pred) {
       : "r"(pred ? 1u : 0u), "r"(id), "r"(n)
       : "memory");
   return r != 0;
+}
+// Arrives on `bar` once every cp.async this thread has issued so far has
+// landed (the barrier's expected count includes this arrival).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void bar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
@@ -595,9 +605,8 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   uint8_t* Pst = smem + L.p;
   uint8_t* ones = smem + L.ones;
   constexpr int NS = tc_stages(SHV);
-  auto stype = reinterpret_cast<int(*)[kTcKeys]>(smem + L.stype);
+  auto stype = reinterpret_cast<int(*)[kTcKeys]>(smem + L.stype);  // [tile % kTypeRing][slot]
   auto srow = reinterpret_cast<int64_t(*)[kTcKeys]>(smem + L.srow);
-  auto vmask = reinterpret_cast<uint32_t(*)[4]>(smem + L.vmask);
   float* mref = reinterpret_cast<float*>(smem + L.mref);
   float* corr_s = reinterpret_cast<float*>(smem + L.corr);
   auto wmax = reinterpret_cast<float(*)[64]>(smem + L.wmax);
@@ -605,7 +614,12 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   uint64_t* empty = full + NS;                                    // [NS] PV of the stage's tile done
   uint64_t* sdone = empty + NS;                                   // [2] S of the tile done (TMEM buffer)
   uint64_t* pready = sdone + 2;                                   // [2] P of the tile written (smem buffer)
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(pready + 2);
+  uint64_t* vfull = pready + 2;                                   // [2] V stage loaded (bf16, separate V)
+  uint64_t* kfree = vfull + 2;                                    // [2] S of the K stage's tile done (same)
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(kfree + 2);
+  // bf16 cache with a separate V: K stages are released when S is done, V
+  // stages when PV is, so the next K tiles stream in while P and PV run
+  constexpr bool kSplitKV = !FP8 && !SHV;
   constexpr int kKB = 16384;  // one 64-dim block of a 128-key tile
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -630,7 +644,12 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   const int ntiles = s1 > s0 ? static_cast<int>((s1 - s0 + kTcKeys - 1) / kTcKeys) : 0;
 
   if (tid == 0) {
-    for (int i = 0; i < 2 * NS + 4; ++i) tc::bar_init(&full[i], 1);
+    // bf16 path: a loaded stage counts one arrival per producer thread, made
+    // by its copies (see the producer); the FP8 producer arrives once
+    for (int i = 0; i < 2 * NS + 8; ++i) {
+      const bool loaded = i < NS || (i >= 2 * NS + 4 && i < 2 * NS + 6);  // full[], vfull[]
+      tc::bar_init(&full[i], (!FP8 && loaded) ? 256 : 1);
+    }
     tc::bar_init_fence();
   }
   if (warp == 0) tc::tmem_alloc(tslot, 256);
@@ -664,6 +683,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       const int kst = tile % NS;
       const uint32_t tS = tmem + 64 * (tile & 1);
       const uint32_t qa = smem_u32(Qs), ka = smem_u32(Kst + kst * 3 * kKB);
+      if (!FP8) tc::fence_async_smem();  // the stage was written by cp.async
       tc::fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < 12; ++kk) {
@@ -672,6 +692,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         tc::mma_bf16_ss(tS, adesc, bdesc, kIdescS, kk > 0 ? 1u : 0u);
       }
       tc::mma_commit(&sdone[tile & 1]);
+      if (kSplitKV) tc::mma_commit(&kfree[kst]);
     };
     if (lane == 0 && ntiles > 0) {
       for (int t0 = 0; t0 < 2 && t0 < ntiles; ++t0) {
@@ -682,6 +703,8 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       for (int tile = 0; tile < ntiles; ++tile) {
         const int kst = tile % NS, pb = tile & 1;
         if (healthy) healthy = tc::bar_wait(&pready[pb], (tile >> 1) & 1);
+        if (kSplitKV && healthy) healthy = tc::bar_wait(&vfull[kst], (tile / NS) & 1);
+        if (!FP8) tc::fence_async_smem();  // the stage was written by cp.async
         tc::fence_after_sync();
         const uint32_t pa = smem_u32(Pst + pb * 16384);
         const uint32_t va = SHV ? smem_u32(Kst + kst * 3 * kKB) : smem_u32(Vst + kst * 2 * kKB);
@@ -700,170 +723,281 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       }
     }
   } else if (warp >= 8) {
-    // ===================== producer: gather, widen, publish =====================
-    const int pt = tid - 256;  // 0..255; threads 0..127 also own one slot each
-    // selected entry of this thread's slot in the next tile, loaded one tile
-    // ahead so that its latency overlaps the current tile's gathers
-    auto load_sel = [&](int tile) -> int32_t {
-      const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
-      return (!dense && pt < kTcKeys && tile < ntiles && sl < s1 && sl < n_ent) ? __ldg(p.idx + row * p.k + sl) : -1;
-    };
-    int32_t sel_next = load_sel(0);
-    for (int tile = 0; tile < ntiles; ++tile) {
-      const int st = tile % NS;
-      const int32_t sel_cur = sel_next;
-      if (tile >= NS && healthy) healthy = tc::bar_wait(&empty[st], ((tile / NS) - 1) & 1);
-      // slot -> (type, row): 0 skip, 1 compressed entry, 2 raw window token
-      if (pt < kTcKeys) {
-        const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
-        int type = 0;
-        int64_t r = 0;
-        if (sl < s1) {
-          if (sl < n_ent) {
-            const int64_t i = dense ? sl : static_cast<int64_t>(sel_cur);
-            if (i >= 0 && i < geo.N && (i + 1) * p.stride - 1 <= t) {
-              type = 1;
-              r = geo.ebase + i;
-            }
-          } else {
-            type = 2;
-            r = geo.wbase + (wlo + (sl - n_ent));
-          }
-        }
-        stype[st][pt] = type;
-        srow[st][pt] = r;
-        const uint32_t bal = __ballot_sync(0xffffffffu, type != 0);
-        if (lane == 0) vmask[st][warp - 8] = bal;
-      }
-      named_sync(1, 256);
-      uint8_t* Kt = Kst + st * 3 * kKB;
-      uint8_t* Vt = Vst + st * 2 * kKB;
-      // The tile's slots are an entry run [0, ne) then a window run [ne, ne + nw).
-      const int64_t a0 = s0 + static_cast<int64_t>(tile) * kTcKeys;
-      const int64_t a1 = (a0 + kTcKeys) < s1 ? (a0 + kTcKeys) : s1;
-      const int ne = static_cast<int>(((a1 < n_ent ? a1 : n_ent) - a0) > 0 ? ((a1 < n_ent ? a1 : n_ent) - a0) : 0);
-      const int nw = static_cast<int>(a1 - a0) - ne;
+    if constexpr (!FP8) {
+      // ===================== producer (bf16 cache): asynchronous gathers =====================
+      // 256 threads copy each tile with 16-byte cp.async and let the copies
+      // themselves arrive on the stage barrier (cp.async.mbarrier.arrive.noinc,
+      // 256 arrivals), so the producer never waits for its own data: it only
+      // waits for a stage to be free.  K(t+1) is issued before V(t): K stages
+      // are freed when S is done, V stages when PV is (separate V); with a
+      // shared V the K stage is freed by PV.
+      const int pt = tid - 256;  // 0..255; threads 0..127 also own one slot each
       const int pwarp = warp - 8;
-      // FP8 entries: thread pt owns 16-code chunk c = pt % 8 of keys pt / 8 + 32 j
-      // (eight lanes per 128-byte row, four rows per warp instruction); the
-      // codes and scales go to registers here and are widened after the
-      // asynchronous copies below are issued.
-      uint4 codes[4];
-      float scl[4];
-      if (FP8) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int key = (pt >> 3) + 32 * j;
-          const bool ok = key < ne && stype[st][key] == 1;
-          const int64_t r = ok ? srow[st][key] : 0;
-          codes[j] = ok ? ldg_nc16(p.cnope + r * kDNope + (pt & 7) * 16) : make_uint4(0u, 0u, 0u, 0u);
-          scl[j] = ok ? __ldg(p.cscale + r) : 0.f;
+      auto load_sel = [&](int tile) -> int32_t {
+        const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
+        return (!dense && pt < kTcKeys && tile < ntiles && sl < s1 && sl < n_ent) ? __ldg(p.idx + row * p.k + sl)
+                                                                                  : -1;
+      };
+      // The tile's slots are an entry run [0, ne) then a window run [ne, ne + nw).
+      auto runs = [&](int tile, int& ne, int& nw) {
+        const int64_t a0 = s0 + static_cast<int64_t>(tile) * kTcKeys;
+        const int64_t a1 = (a0 + kTcKeys) < s1 ? (a0 + kTcKeys) : s1;
+        const int64_t e1 = a1 < n_ent ? a1 : n_ent;
+        ne = static_cast<int>(e1 - a0 > 0 ? e1 - a0 : 0);
+        nw = static_cast<int>(a1 - a0) - ne;
+      };
+      // nch 16-byte chunks per key from a source row of `stride` elements:
+      // K = 24 chunks (three 64-dim blocks), V = 16 chunks (two blocks)
+      auto issue = [&](uint8_t* T, int tile, int nch, const __nv_bfloat16* esrc, int estride,
+                       const __nv_bfloat16* wsrc, int wstride) {
+        const int ring = tile & (kTypeRing - 1);
+        int ne, nw;
+        runs(tile, ne, nw);
+        if (ne > 0 && dense) {  // contiguous entry rows
+          const int64_t r0 = srow[ring][0];
+          for (int pc = pt; pc < ne * nch; pc += 256) {
+            const int key = pc / nch, c = pc % nch;
+            cp_async16(T + (c >> 3) * kKB + tc::sw128(key, c & 7), esrc + (r0 + key) * estride + c * 8);
+          }
+        } else if (ne > 0) {  // selected entries: four keys per warp instruction, 8 lanes per 128-byte row
+          const int c = lane & 7;
+          for (int kb = pwarp * 4; kb < ne; kb += 32) {
+            const int key = kb + (lane >> 3);
+            if (key >= ne) continue;
+            const int type = stype[ring][key];
+            const int64_t r = srow[ring][key];
+            for (int j = 0; j < nch / 8; ++j)
+              cp_async16(T + j * kKB + tc::sw128(key, c), type ? esrc + r * estride + (8 * j + c) * 8 : p.q,
+                         type ? 16 : 0);
+          }
+        }
+        if (nw > 0) {  // raw window tokens: contiguous rows
+          const int64_t rw0 = srow[ring][ne];
+          for (int pc = pt; pc < nw * nch; pc += 256) {
+            const int key = ne + pc / nch, c = pc % nch;
+            cp_async16(T + (c >> 3) * kKB + tc::sw128(key, c & 7), wsrc + (rw0 + pc / nch) * wstride + c * 8);
+          }
+        }
+        for (int pc = pt; pc < (kTcKeys - ne - nw) * nch; pc += 256) {  // past the row's end: zero rows
+          const int key = ne + nw + pc / nch, c = pc % nch;
+          cp_async16(T + (c >> 3) * kKB + tc::sw128(key, c & 7), p.q, 0);
+        }
+      };
+      const __nv_bfloat16* ve = p.cv ? p.cv : p.ck;
+      const int ves = p.cv ? kDV : kDQK;
+      const __nv_bfloat16* vw = p.wv ? p.wv : p.wk;
+      const int vws = p.wv ? kDV : kDQK;
+      int32_t sel_next = load_sel(0);
+      for (int it = 0; it <= ntiles; ++it) {
+        if (it < ntiles) {  // K of tile `it`
+          const int tile = it, st = tile % NS, ring = tile & (kTypeRing - 1);
+          const int32_t sel_cur = sel_next;
+          sel_next = load_sel(tile + 1);
+          if (pt < kTcKeys) {  // slot -> (type, row): 0 skip, 1 compressed entry, 2 raw window token
+            const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
+            int type = 0;
+            int64_t r = 0;
+            if (sl < s1) {
+              if (sl < n_ent) {
+                const int64_t i = dense ? sl : static_cast<int64_t>(sel_cur);
+                if (i >= 0 && i < geo.N && (i + 1) * p.stride - 1 <= t) {
+                  type = 1;
+                  r = geo.ebase + i;
+                }
+              } else {
+                type = 2;
+                r = geo.wbase + (wlo + (sl - n_ent));
+              }
+            }
+            stype[ring][pt] = type;
+            srow[ring][pt] = r;
+          }
+          bool ok = true;
+          if (tile >= NS) ok = tc::bar_wait(kSplitKV ? &kfree[st] : &empty[st], ((tile / NS) - 1) & 1);
+          if (named_sync_or(1, 256, !ok)) {  // also publishes the slot table to the 256 threads
+            healthy = false;
+            break;
+          }
+          issue(Kst + st * 3 * kKB, tile, 24, p.ck, kDQK, p.wk, kDQK);
+          cp_async_mbar_arrive_noinc(&full[st]);
+        }
+        if (kSplitKV && it >= 1) {  // V of tile `it - 1`
+          const int tile = it - 1, vs = tile % NS;
+          bool ok = true;
+          if (tile >= NS) ok = tc::bar_wait(&empty[vs], ((tile / NS) - 1) & 1);
+          if (named_sync_or(3, 256, !ok)) {
+            healthy = false;
+            break;
+          }
+          issue(Vst + vs * 2 * kKB, tile, 16, ve, ves, vw, vws);
+          cp_async_mbar_arrive_noinc(&vfull[vs]);
         }
       }
-      // Contiguous runs are copied with consecutive lanes on consecutive 16-byte
-      // chunks (512-byte warp requests); selected entries are gathered four keys
-      // per warp instruction (8 lanes per 128-byte row).
-      if (ne > 0 && dense) {
-        const int64_t r0 = srow[st][0];
-        if (FP8) {
-          for (int pc = pt; pc < ne * 8; pc += 256)
-            cp_async16(Kt + 2 * kKB + tc::sw128(pc >> 3, pc & 7), p.crope + r0 * kDRope + pc * 8);
-        } else {
-          for (int pc = pt; pc < ne * 24; pc += 256) {
-            const int key = pc / 24, c = pc % 24;
-            cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.ck + r0 * kDQK + pc * 8);
-          }
-          if (!SHV) {
-            for (int pc = pt; pc < ne * 16; pc += 256) {
-              const int key = pc >> 4, c = pc & 15;
-              const __nv_bfloat16* src = p.cv ? p.cv + r0 * kDV + pc * 8 : p.ck + (r0 + key) * kDQK + c * 8;
-              cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), src);
+      cp_async_wait<0>();  // no copy of this thread is left in flight when the CTA moves on
+    } else {
+      // ===================== producer: gather, widen, publish =====================
+      const int pt = tid - 256;  // 0..255; threads 0..127 also own one slot each
+      // selected entry of this thread's slot in the next tile, loaded one tile
+      // ahead so that its latency overlaps the current tile's gathers
+      auto load_sel = [&](int tile) -> int32_t {
+        const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
+        return (!dense && pt < kTcKeys && tile < ntiles && sl < s1 && sl < n_ent) ? __ldg(p.idx + row * p.k + sl) : -1;
+      };
+      int32_t sel_next = load_sel(0);
+      for (int tile = 0; tile < ntiles; ++tile) {
+        const int st = tile % NS;
+        const int32_t sel_cur = sel_next;
+        if (tile >= NS && healthy) healthy = tc::bar_wait(&empty[st], ((tile / NS) - 1) & 1);
+        // slot -> (type, row): 0 skip, 1 compressed entry, 2 raw window token
+        if (pt < kTcKeys) {
+          const int64_t sl = s0 + static_cast<int64_t>(tile) * kTcKeys + pt;
+          int type = 0;
+          int64_t r = 0;
+          if (sl < s1) {
+            if (sl < n_ent) {
+              const int64_t i = dense ? sl : static_cast<int64_t>(sel_cur);
+              if (i >= 0 && i < geo.N && (i + 1) * p.stride - 1 <= t) {
+                type = 1;
+                r = geo.ebase + i;
+              }
+            } else {
+              type = 2;
+              r = geo.wbase + (wlo + (sl - n_ent));
             }
           }
+          stype[tile & (kTypeRing - 1)][pt] = type;
+          srow[st][pt] = r;
         }
-      } else if (ne > 0) {
-        const int c = lane & 7;
-        for (int kb = pwarp * 4; kb < ne; kb += 32) {
-          const int key = kb + (lane >> 3);
-          if (key >= ne) continue;
-          const int type = stype[st][key];
-          const int64_t r = srow[st][key];
-          const int bytes = type ? 16 : 0;
+        named_sync(1, 256);
+        uint8_t* Kt = Kst + st * 3 * kKB;
+        uint8_t* Vt = Vst + st * 2 * kKB;
+        // The tile's slots are an entry run [0, ne) then a window run [ne, ne + nw).
+        const int64_t a0 = s0 + static_cast<int64_t>(tile) * kTcKeys;
+        const int64_t a1 = (a0 + kTcKeys) < s1 ? (a0 + kTcKeys) : s1;
+        const int ne = static_cast<int>(((a1 < n_ent ? a1 : n_ent) - a0) > 0 ? ((a1 < n_ent ? a1 : n_ent) - a0) : 0);
+        const int nw = static_cast<int>(a1 - a0) - ne;
+        const int pwarp = warp - 8;
+        // FP8 entries: thread pt owns 16-code chunk c = pt % 8 of keys pt / 8 + 32 j
+        // (eight lanes per 128-byte row, four rows per warp instruction); the
+        // codes and scales go to registers here and are widened after the
+        // asynchronous copies below are issued.
+        uint4 codes[4];
+        float scl[4];
+        if (FP8) {
+  #pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int key = (pt >> 3) + 32 * j;
+            const bool ok = key < ne && stype[tile & (kTypeRing - 1)][key] == 1;
+            const int64_t r = ok ? srow[st][key] : 0;
+            codes[j] = ok ? ldg_nc16(p.cnope + r * kDNope + (pt & 7) * 16) : make_uint4(0u, 0u, 0u, 0u);
+            scl[j] = ok ? __ldg(p.cscale + r) : 0.f;
+          }
+        }
+        // Contiguous runs are copied with consecutive lanes on consecutive 16-byte
+        // chunks (512-byte warp requests); selected entries are gathered four keys
+        // per warp instruction (8 lanes per 128-byte row).
+        if (ne > 0 && dense) {
+          const int64_t r0 = srow[st][0];
           if (FP8) {
-            cp_async16(Kt + 2 * kKB + tc::sw128(key, c), type ? p.crope + r * kDRope + c * 8 : p.crope, bytes);
+            for (int pc = pt; pc < ne * 8; pc += 256)
+              cp_async16(Kt + 2 * kKB + tc::sw128(pc >> 3, pc & 7), p.crope + r0 * kDRope + pc * 8);
           } else {
-#pragma unroll
-            for (int j = 0; j < 3; ++j)
-              cp_async16(Kt + j * kKB + tc::sw128(key, c), type ? p.ck + r * kDQK + (8 * j + c) * 8 : p.ck, bytes);
+            for (int pc = pt; pc < ne * 24; pc += 256) {
+              const int key = pc / 24, c = pc % 24;
+              cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.ck + r0 * kDQK + pc * 8);
+            }
             if (!SHV) {
-#pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                const __nv_bfloat16* src = !type ? p.ck : (p.cv ? p.cv + r * kDV + (8 * j + c) * 8
-                                                                : p.ck + r * kDQK + (8 * j + c) * 8);
-                cp_async16(Vt + j * kKB + tc::sw128(key, c), src, bytes);
+              for (int pc = pt; pc < ne * 16; pc += 256) {
+                const int key = pc >> 4, c = pc & 15;
+                const __nv_bfloat16* src = p.cv ? p.cv + r0 * kDV + pc * 8 : p.ck + (r0 + key) * kDQK + c * 8;
+                cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), src);
+              }
+            }
+          }
+        } else if (ne > 0) {
+          const int c = lane & 7;
+          for (int kb = pwarp * 4; kb < ne; kb += 32) {
+            const int key = kb + (lane >> 3);
+            if (key >= ne) continue;
+            const int type = stype[tile & (kTypeRing - 1)][key];
+            const int64_t r = srow[st][key];
+            const int bytes = type ? 16 : 0;
+            if (FP8) {
+              cp_async16(Kt + 2 * kKB + tc::sw128(key, c), type ? p.crope + r * kDRope + c * 8 : p.crope, bytes);
+            } else {
+  #pragma unroll
+              for (int j = 0; j < 3; ++j)
+                cp_async16(Kt + j * kKB + tc::sw128(key, c), type ? p.ck + r * kDQK + (8 * j + c) * 8 : p.ck, bytes);
+              if (!SHV) {
+  #pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                  const __nv_bfloat16* src = !type ? p.ck : (p.cv ? p.cv + r * kDV + (8 * j + c) * 8
+                                                                  : p.ck + r * kDQK + (8 * j + c) * 8);
+                  cp_async16(Vt + j * kKB + tc::sw128(key, c), src, bytes);
+                }
               }
             }
           }
         }
-      }
-      if (nw > 0) {  // raw window tokens: contiguous rows
-        const int64_t rw0 = srow[st][ne];
-        for (int pc = pt; pc < nw * 24; pc += 256) {
-          const int key = ne + pc / 24, c = pc % 24;
-          cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.wk + rw0 * kDQK + pc * 8);
+        if (nw > 0) {  // raw window tokens: contiguous rows
+          const int64_t rw0 = srow[st][ne];
+          for (int pc = pt; pc < nw * 24; pc += 256) {
+            const int key = ne + pc / 24, c = pc % 24;
+            cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.wk + rw0 * kDQK + pc * 8);
+          }
+          if (!SHV) {
+            for (int pc = pt; pc < nw * 16; pc += 256) {
+              const int key = ne + (pc >> 4), c = pc & 15;
+              const __nv_bfloat16* src = p.wv ? p.wv + rw0 * kDV + pc * 8 : p.wk + (rw0 + (pc >> 4)) * kDQK + c * 8;
+              cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), src);
+            }
+          }
+        }
+        // slots past the end of the row: zero rows (their logits are masked)
+        for (int pc = pt; pc < (kTcKeys - ne - nw) * 24; pc += 256) {
+          const int key = ne + nw + pc / 24, c = pc % 24;
+          cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.q, 0);
         }
         if (!SHV) {
-          for (int pc = pt; pc < nw * 16; pc += 256) {
-            const int key = ne + (pc >> 4), c = pc & 15;
-            const __nv_bfloat16* src = p.wv ? p.wv + rw0 * kDV + pc * 8 : p.wk + (rw0 + (pc >> 4)) * kDQK + c * 8;
-            cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), src);
+          for (int pc = pt; pc < (kTcKeys - ne - nw) * 16; pc += 256) {
+            const int key = ne + nw + (pc >> 4), c = pc & 15;
+            cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.q, 0);
           }
         }
-      }
-      // slots past the end of the row: zero rows (their logits are masked)
-      for (int pc = pt; pc < (kTcKeys - ne - nw) * 24; pc += 256) {
-        const int key = ne + nw + pc / 24, c = pc % 24;
-        cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.q, 0);
-      }
-      if (!SHV) {
-        for (int pc = pt; pc < (kTcKeys - ne - nw) * 16; pc += 256) {
-          const int key = ne + nw + (pc >> 4), c = pc & 15;
-          cp_async16(Vt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.q, 0);
-        }
-      }
-      cp_async_commit();
-      sel_next = load_sel(tile + 1);
-      if (FP8) {  // code * scale -> bf16 into the swizzled K (and V) tile; skipped slots get zeros
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int key = (pt >> 3) + 32 * j, c = pt & 7;
-          if (key >= ne) continue;
-          const uint32_t w4[4] = {codes[j].x, codes[j].y, codes[j].z, codes[j].w};
-          uint32_t outw[8];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t h01, h23;
-            e4m3x4_to_f16x2x2(w4[q], h01, h23);
-            const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-            const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-            outw[2 * q] = pack_bf16x2(f01.x * scl[j], f01.y * scl[j]);
-            outw[2 * q + 1] = pack_bf16x2(f23.x * scl[j], f23.y * scl[j]);
-          }
-          const int blk = c >> 2;
-          const uint4 lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-          const uint4 hi = make_uint4(outw[4], outw[5], outw[6], outw[7]);
-          *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
-          *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
-          if (!SHV) {
-            *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
-            *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
+        cp_async_commit();
+        sel_next = load_sel(tile + 1);
+        if (FP8) {  // code * scale -> bf16 into the swizzled K (and V) tile; skipped slots get zeros
+  #pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int key = (pt >> 3) + 32 * j, c = pt & 7;
+            if (key >= ne) continue;
+            const uint32_t w4[4] = {codes[j].x, codes[j].y, codes[j].z, codes[j].w};
+            uint32_t outw[8];
+  #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t h01, h23;
+              e4m3x4_to_f16x2x2(w4[q], h01, h23);
+              const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+              const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+              outw[2 * q] = pack_bf16x2(f01.x * scl[j], f01.y * scl[j]);
+              outw[2 * q + 1] = pack_bf16x2(f23.x * scl[j], f23.y * scl[j]);
+            }
+            const int blk = c >> 2;
+            const uint4 lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+            const uint4 hi = make_uint4(outw[4], outw[5], outw[6], outw[7]);
+            *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
+            *reinterpret_cast<uint4*>(Kt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
+            if (!SHV) {
+              *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c) & 7)) = lo;
+              *reinterpret_cast<uint4*>(Vt + blk * kKB + tc::sw128(key, (2 * c + 1) & 7)) = hi;
+            }
           }
         }
+        cp_async_wait<0>();
+        tc::fence_async_smem();
+        named_sync(1, 256);
+        if (pt == 0) bar_arrive(&full[st]);
       }
-      cp_async_wait<0>();
-      tc::fence_async_smem();
-      named_sync(1, 256);
-      if (pt == 0) bar_arrive(&full[st]);
     }
   } else {
     // ===================== softmax: thread = key of the tile, 32 heads =====================
@@ -871,12 +1005,12 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
     const int key = (warp & 3) * 32 + lane;
     const int hb = (warp >> 2) * 32;
     for (int tile = 0; tile < ntiles; ++tile) {
-      const int kst = tile % NS, pb = tile & 1;
+      const int pb = tile & 1;
       if (healthy) healthy = tc::bar_wait(&sdone[pb], (tile >> 1) & 1);
       tc::fence_after_sync();
       float sv[32];
       tc::tmem_ld32(tmem + 64 * pb + lane_base + hb, sv);
-      const bool valid = stype[kst][key] != 0;
+      const bool valid = stype[tile & (kTypeRing - 1)][key] != 0;
       bool over = false;
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {
@@ -1441,7 +1575,9 @@ KernelFn pick(int H, bool fp8, bool shv) {
   return shv ? attn_kernel<4, false, true> : attn_kernel<4, false, false>;
 }
 
-KernelFn pick_tc(bool fp8, bool shv) {
+using TcKernelFn = void (*)(AttnParams);
+
+TcKernelFn pick_tc(bool fp8, bool shv) {
   if (fp8) return shv ? attn_tc_kernel<true, true> : attn_tc_kernel<true, false>;
   return shv ? attn_tc_kernel<false, true> : attn_tc_kernel<false, false>;
 }
@@ -1452,7 +1588,8 @@ size_t smem_bytes(bool use_tc, bool fp8, bool shv, int tps) {
 
 // Clusters of this kernel (cluster size cl, given shared memory and block size)
 // the device can keep resident at once; 0 if it cannot run them at all.
-int max_active_clusters(KernelFn fn, int cl, size_t smem, int threads) {
+template <typename Fn>
+int max_active_clusters(Fn fn, int cl, size_t smem, int threads) {
   static std::mutex mu;
   static std::map<std::tuple<int, const void*, int, size_t, int>, int> cache;
   int dev = 0;
@@ -1484,7 +1621,8 @@ int max_active_clusters(KernelFn fn, int cl, size_t smem, int threads) {
 // Cluster size for `rows` rows of `tiles` tiles each: the largest size <= want
 // whose clusters all fit on the device at once (one wave); if none does, the
 // largest size that runs at all.
-int choose_cluster(KernelFn fn, int want, int64_t rows, size_t smem, int threads) {
+template <typename Fn>
+int choose_cluster(Fn fn, int want, int64_t rows, size_t smem, int threads) {
   int fallback = 1;
   for (int cl = want; cl > 1; --cl) {
     const int n = max_active_clusters(fn, cl, smem, threads);
@@ -1593,7 +1731,7 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
       bool nonportable = true;
       {
         std::lock_guard<std::mutex> lock(mu);
-        const KernelFn f = pick_tc(fp8, shv);
+        const TcKernelFn f = pick_tc(fp8, shv);
         if (cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
           cudaGetLastError();
           nonportable = false;
@@ -1622,9 +1760,11 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
       part = static_cast<float*>(workspace);
     }
   }
-  KernelFn fn = use_tc ? pick_tc(fp8, shv) : pick(H, fp8, shv);
+  const TcKernelFn tfn = use_tc ? pick_tc(fp8, shv) : nullptr;
+  KernelFn fn = use_tc ? nullptr : pick(H, fp8, shv);
   size_t smem = smem_bytes(use_tc, fp8, shv, pl.tps);
-  if (!ensure_smem(reinterpret_cast<const void*>(fn), static_cast<int>(smem)))
+  if (!ensure_smem(use_tc ? reinterpret_cast<const void*>(tfn) : reinterpret_cast<const void*>(fn),
+                   static_cast<int>(smem)))
     return fail(CSA_ERR_CUDA, "%s: cannot raise the shared memory limit to %zu", name, smem);
   if (pl.cl > 1 && !use_tc) {
     static std::mutex mu;
@@ -1691,7 +1831,7 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   const int cluster = (use_tc && !tc_cluster) || use_blk ? 1 : pl.cl;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   prof_begin(s);
-  const cudaError_t e = launch_pdl(fn, grid, block, smem, s, cluster, p);
+  const cudaError_t e = launch_pdl((use_tc && !use_blk) ? tfn : fn, grid, block, smem, s, cluster, p);
   prof_end(s);
   if (csa_status st = check_launch(name, e); st != CSA_OK) return st;
   if (part != nullptr)
