@@ -1011,20 +1011,27 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       float sv[32];
       tc::tmem_ld32(tmem + 64 * pb + lane_base + hb, sv);
       const bool valid = stype[tile & (kTypeRing - 1)][key] != 0;
+      // sv <- logit x scale - running max (log2 units), one FMA per logit
+      auto centre = [&]() {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(mref + hb + j);
+          sv[j] = fmaf(sv[j], p.scale_log2, -m4.x);
+          sv[j + 1] = fmaf(sv[j + 1], p.scale_log2, -m4.y);
+          sv[j + 2] = fmaf(sv[j + 2], p.scale_log2, -m4.z);
+          sv[j + 3] = fmaf(sv[j + 3], p.scale_log2, -m4.w);
+        }
+      };
+      centre();
       bool over = false;
 #pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const float4 m4 = *reinterpret_cast<const float4*>(mref + hb + j);
-        const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          sv[j + u] = valid ? sv[j + u] * p.scale_log2 : -INFINITY;
-          over |= sv[j + u] - mm[u] > kRescaleLog2;
-        }
-      }
-      if (named_sync_or(2, 256, over)) {
+      for (int j = 0; j < 32; ++j) over |= sv[j] > kRescaleLog2;
+      if (named_sync_or(2, 256, over && valid)) {
         // new per-head maxima: this tile's maximum over its valid keys (the
         // reduction consumes sv; the logits are read again from TMEM below)
+        tc::tmem_ld32(tmem + 64 * pb + lane_base + hb, sv);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[j] = valid ? sv[j] * p.scale_log2 : -INFINITY;
         const int h0 = warp_head_max32(sv, lane);
         wmax[warp & 3][hb + h0] = sv[0];
         named_sync(2, 256);
@@ -1052,20 +1059,16 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
           tc::tmem_wait_st();
         }
         tc::tmem_ld32(tmem + 64 * pb + lane_base + hb, sv);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) sv[j] = valid ? sv[j] * p.scale_log2 : -INFINITY;
+        centre();
       }
       // this key's P^T row, heads hb .. hb+31: four 16-byte chunks of the 128-byte swizzled row
       {
         uint8_t* Pb = Pst + pb * 16384;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const float4 ma = *reinterpret_cast<const float4*>(mref + hb + 8 * c);
-          const float4 mb = *reinterpret_cast<const float4*>(mref + hb + 8 * c + 4);
-          const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
           float pv[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) pv[u] = valid ? fast_exp2(sv[8 * c + u] - mm[u]) : 0.f;
+          for (int u = 0; u < 8; ++u) pv[u] = valid ? fast_exp2(sv[8 * c + u]) : 0.f;
           const uint4 v = make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
                                      pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
           *reinterpret_cast<uint4*>(Pb + tc::sw128(key, (hb >> 3) + c)) = v;
