@@ -1189,181 +1189,312 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
 }
 
 // ---------------------------------------------------------------------------
-// Dense (HCA) prefill: one CTA per block of consecutive queries.  Its 128 MMA
-// rows are (query, head) pairs, QB = 128 / H queries.  Consecutive queries see
-// nearly the same keys (the same visible entries, overlapping windows), so the
-// union of the block's keys is staged once per 64-key tile and every row masks
-// what its own query may not see: entry i needs (i+1)m' - 1 <= t_q, a window
-// token p needs t_q - w_s < p <= t_q.  M = 128 puts row r in TMEM lane r, so
-// consumer thread r owns row r.  Producer warpgroup: coalesced copies of the
-// entry run and the window run; consumer warpgroup: softmax and MMA issue.
+// Query-blocked prefill (tcgen05): one CTA per block of QB = 256 / H
+// consecutive queries, whose 256 (query, head) rows form two M = 128 MMA
+// groups that share every staged key tile.  Consecutive queries see nearly
+// the same keys, so the block's keys are staged once per 64-key tile and each
+// row masks what its own query may not see:
+//   dense (HCA): all visible entries [0, n) of the last query, then the raw
+//     window run of the block; entry i needs (i+1)m - 1 <= t_q;
+//   sparse (CSA, few heads): the union of the block's selected entries in
+//     ascending order (built in shared memory from a per-entry bit set of
+//     the queries that selected it), then the window run; a row sees an
+//     entry slot iff its query selected that entry;
+//   window token p: t_q - w_s < p <= t_q.
+// Warps 0-3 own rows 0-127 (group 0), warps 4-7 rows 128-255 (group 1): one
+// thread per row, in its TMEM lane.  Warps 8-10 copy tiles with cp.async
+// whose completions arrive on the stage barrier (the copying threads never
+// wait for their data); one thread of warp 11 issues every MMA (twelve warps:
+// three per SM sub-partition, so that each thread may hold 168 registers):
+//   S_g = Q_g K^T   (M = 128 rows, N = 64 keys, K = 192), double-buffered;
+//   O_g += P_g V    (M = 128 rows, N = 128 channels, K = 64 keys).
+// TMEM: S[g][buf] in columns 64 (2g + buf), O_g in 256 + 128 g.
 // ---------------------------------------------------------------------------
-constexpr int kBlkKeys = 64;
+constexpr int kQbKeys = 64;
+constexpr int kQbThreads = 384;
+constexpr int kQbLoaders = 96;  // warps 8-10
+constexpr int kQbMaxCand = 2048;   // sparse path: block queries x k
+constexpr int kQbMaxEnt = 16384;   // sparse path: entries per sequence (bit set in the P buffers)
 
-struct BlkLayout {
-  size_t q, k, v, p, bars, total;
+struct QbLayout {
+  size_t q, k, v, p, ulist, umask, bars, total;
 };
 
-__host__ __device__ inline BlkLayout blk_layout() {
-  BlkLayout L;
+__host__ __device__ inline QbLayout qb_layout() {
+  QbLayout L;
   size_t off = 0;
-  L.q = off; off += 3 * 16384;          // Q: 128 rows x 192 dims (3 blocks of 128 x 128 B)
+  L.q = off; off += 2 * 3 * 16384;      // Q: 2 groups x 3 blocks of 128 rows x 128 B
   L.k = off; off += 2 * 3 * 8192;       // K: 2 stages x 64 keys x 192 dims
   L.v = off; off += 2 * 2 * 8192;       // V: 2 stages x 64 keys x 128 dims
-  L.p = off; off += 2 * 16384;          // P: 2 buffers x 128 rows x 64 keys
-  L.bars = off; off += 128;
+  L.p = off; off += 2 * 16384;          // P: 2 groups x 128 rows x 64 keys (prologue: entry bit set)
+  L.ulist = off; off += kQbMaxCand * 2; // union entries (uint16)
+  L.umask = off; off += kQbMaxCand * 2; // their query bits (uint16)
+  L.bars = off; off += 256;              // 16 mbarriers + the TMEM address
   L.total = off + 1024;
   return L;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1) attn_block_kernel(AttnParams p) {
+__global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p) {
   pdl_wait();
-  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const BlkLayout L = blk_layout();
+  const QbLayout L = qb_layout();
   uint8_t* Qs = smem + L.q;
   uint8_t* Kst = smem + L.k;
   uint8_t* Vst = smem + L.v;
   uint8_t* Pst = smem + L.p;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* empty = full + 2;
-  uint64_t* sdone = full + 4;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(full + 8);
+  uint16_t* ulist = reinterpret_cast<uint16_t*>(smem + L.ulist);
+  uint16_t* umask = reinterpret_cast<uint16_t*>(smem + L.umask);
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + L.bars);  // [2] K stage loaded (one arrival per loader)
+  uint64_t* vfull = kfull + 2;                                     // [2] V stage loaded (same)
+  uint64_t* kfree = vfull + 2;                                     // [2] both S of the K stage's tile done
+  uint64_t* vfree = kfree + 2;                                     // [2] both PV of the V stage's tile done
+  uint64_t* sdone = vfree + 2;                                     // [2 groups][2 bufs] S done
+  uint64_t* pready = sdone + 4;                                    // [2 groups] P written
+  uint64_t* pvdone = pready + 2;                                   // [2 groups] PV done
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(pvdone + 2);
+  __shared__ int s_count[kQbThreads / 32];
+  __shared__ int s_union;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = p.H;
-  const int QB = 128 / H;
+  const int QB = 256 / H;
   const int64_t nblk = (p.Tq + QB - 1) / QB;
   const int64_t b = blockIdx.x / nblk;
   const int64_t qb = blockIdx.x % nblk;
-  const int64_t r0 = qb * QB;                     // first query row of the block
+  const int64_t r0 = qb * QB;  // first query row of the block within its sequence
   const int nq = static_cast<int>((p.Tq - r0) < QB ? (p.Tq - r0) : QB);
   const int64_t t0 = p.q_pos0 + r0, tl = t0 + nq - 1;
-  int64_t ent_n = (tl + 1) / p.stride;
-  if (ent_n > p.N) ent_n = p.N;
+  const bool sparse = p.idx != nullptr;
   const int64_t wlo0 = (t0 - p.wlen + 1) > 0 ? (t0 - p.wlen + 1) : 0;
   const int64_t nwin = p.wlen > 0 ? (tl - wlo0 + 1) : 0;
-  const int64_t n_slots = ent_n + nwin;
-  const int ntiles = static_cast<int>((n_slots + kBlkKeys - 1) / kBlkKeys);
 
   if (tid == 0) {
-    for (int i = 0; i < 6; ++i) tc::bar_init(&full[i], 1);
+    for (int i = 0; i < 4; ++i) tc::bar_init(&kfull[i], kQbLoaders);  // kfull, vfull
+    for (int i = 4; i < 16; ++i) tc::bar_init(&kfull[i], 1);
     tc::bar_init_fence();
   }
-  if (warp == 0) tc::tmem_alloc(tslot, 256);
-  {  // Q rows (query, head), swizzled K-major; rows past the block's queries are zero
+  if (warp == 0) tc::tmem_alloc(tslot, 512);
+  {  // Q rows (query, head) of both groups, swizzled K-major; rows past the block's queries are zero
     const __nv_bfloat16* qsrc = p.q + ((b * p.Tq + r0) * H) * kDQK;
     const int valid_rows = nq * H;
-    for (int piece = tid; piece < 128 * 24; piece += kTcThreads) {
+    for (int piece = tid; piece < 256 * 24; piece += kQbThreads) {
       const int r = piece / 24, ch = piece % 24;
-      cp_async16(Qs + (ch >> 3) * 16384 + tc::sw128(r, ch & 7), r < valid_rows ? qsrc + piece * 8 : p.q,
-                 r < valid_rows ? 16 : 0);
+      cp_async16(Qs + (r >> 7) * 49152 + (ch >> 3) * 16384 + tc::sw128(r & 127, ch & 7),
+                 r < valid_rows ? qsrc + piece * 8 : p.q, r < valid_rows ? 16 : 0);
     }
   }
   cp_async_commit();
+
+  // entry slots: the dense run [0, n_ent), or the union of the selections
+  int64_t n_ent;
+  if (!sparse) {
+    n_ent = (tl + 1) / p.stride;
+    if (n_ent > p.N) n_ent = p.N;
+  } else {
+    // per-entry bit set of the block's queries that selected it (16 bits per entry, in the P buffers)
+    uint32_t* bits = reinterpret_cast<uint32_t*>(Pst);
+    const int nwords = static_cast<int>((p.N + 1) / 2);
+    for (int w = tid; w < nwords; w += kQbThreads) bits[w] = 0u;
+    __syncthreads();
+    for (int c = tid; c < nq * p.k; c += kQbThreads) {
+      const int q = c / p.k;
+      const int64_t tq = t0 + q;
+      const int64_t i = __ldg(p.idx + (b * p.Tq + r0 + q) * p.k + (c % p.k));
+      if (i >= 0 && i < p.N && (i + 1) * p.stride - 1 <= tq)
+        atomicOr(&bits[i >> 1], 1u << (static_cast<int>(i & 1) * 16 + q));
+    }
+    __syncthreads();
+    // ascending compaction: thread chunks of words, counts, a block scan, then the writes
+    const int per = (nwords + kQbThreads - 1) / kQbThreads;
+    const int w0 = tid * per, w1 = (w0 + per) < nwords ? (w0 + per) : nwords;
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) {
+      const uint32_t v = bits[w];
+      cnt += ((v & 0xffffu) != 0u) + ((v >> 16) != 0u);
+    }
+    int incl = cnt;  // inclusive scan within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_count[warp] = incl;
+    __syncthreads();
+    if (tid == 0) {
+      int run = 0;
+      for (int w = 0; w < kQbThreads / 32; ++w) {
+        const int c2 = s_count[w];
+        s_count[w] = run;
+        run += c2;
+      }
+      s_union = run;
+    }
+    __syncthreads();
+    int pos = s_count[warp] + incl - cnt;
+    for (int w = w0; w < w1; ++w) {
+      const uint32_t v = bits[w];
+      if ((v & 0xffffu) != 0u) {
+        ulist[pos] = static_cast<uint16_t>(2 * w);
+        umask[pos++] = static_cast<uint16_t>(v & 0xffffu);
+      }
+      if ((v >> 16) != 0u) {
+        ulist[pos] = static_cast<uint16_t>(2 * w + 1);
+        umask[pos++] = static_cast<uint16_t>(v >> 16);
+      }
+    }
+    n_ent = s_union;
+  }
+  const int64_t n_slots = n_ent + nwin;
+  const int ntiles = static_cast<int>((n_slots + kQbKeys - 1) / kQbKeys);
   cp_async_wait<0>();
   tc::fence_async_smem();
   tc::fence_before_sync();
-  __syncthreads();
+  __syncthreads();  // Q, the union and the barriers are ready; the P buffers are free again
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
-  const uint32_t tO = tmem + 128;
   bool healthy = true;
 
-  if (warp >= 4) {
-    // ===================== producer =====================
-    const int pt = tid - 128;
-    for (int tile = 0; tile < ntiles; ++tile) {
-      const int st = tile & 1;
-      if (tile >= 2 && healthy) healthy = tc::bar_wait(&empty[st], ((tile >> 1) - 1) & 1);
-      uint8_t* Kt = Kst + st * 3 * 8192;
-      uint8_t* Vt = Vst + st * 2 * 8192;
-      const int64_t a0 = static_cast<int64_t>(tile) * kBlkKeys;
-      const int64_t a1 = (a0 + kBlkKeys) < n_slots ? (a0 + kBlkKeys) : n_slots;
-      const int ne = static_cast<int>(((a1 < ent_n ? a1 : ent_n) - a0) > 0 ? ((a1 < ent_n ? a1 : ent_n) - a0) : 0);
-      const int nw = static_cast<int>(a1 - a0) - ne;
-      if (ne > 0) {  // entries a0 .. a0+ne-1 of sequence b: contiguous rows
-        const int64_t er = b * p.N + a0;
-        for (int pc = pt; pc < ne * 24; pc += 128) {
-          const int key = pc / 24, c = pc % 24;
-          cp_async16(Kt + (c >> 3) * 8192 + tc::sw128(key, c & 7), p.ck + er * kDQK + pc * 8);
+  if (warp >= 8 && warp < 11) {
+    // ===================== producer: cp.async copies that arrive by themselves =====================
+    const int pt = tid - 256;
+    const int64_t ebase = b * p.N;
+    const int64_t wbase = b * p.wrows - p.wpos0 + wlo0;
+    const __nv_bfloat16* ve = p.cv ? p.cv : p.ck;
+    const int ves = p.cv ? kDV : kDQK;
+    const __nv_bfloat16* vw = p.wv ? p.wv : p.wk;
+    const int vws = p.wv ? kDV : kDQK;
+    // K (24 chunks per key) or V (16 chunks per key) of one tile
+    auto issue = [&](bool is_k, uint8_t* T, int tile) {
+      const int nch = is_k ? 24 : 16;
+      const int64_t a0 = static_cast<int64_t>(tile) * kQbKeys;
+      for (int pc = pt; pc < kQbKeys * nch; pc += kQbLoaders) {
+        const int key = pc / nch, c = pc % nch;
+        const int64_t sl = a0 + key;
+        const __nv_bfloat16* src = p.q;
+        int bytes = 0;
+        if (sl < n_ent) {
+          const int64_t e = ebase + (sparse ? static_cast<int64_t>(ulist[sl]) : sl);
+          src = is_k ? p.ck + e * kDQK + c * 8 : ve + e * ves + c * 8;
+          bytes = 16;
+        } else if (sl < n_slots) {
+          const int64_t w = wbase + (sl - n_ent);
+          src = is_k ? p.wk + w * kDQK + c * 8 : vw + w * vws + c * 8;
+          bytes = 16;
         }
-        for (int pc = pt; pc < ne * 16; pc += 128) {
-          const int key = pc >> 4, c = pc & 15;
-          const __nv_bfloat16* src = p.cv ? p.cv + er * kDV + pc * 8 : p.ck + (er + key) * kDQK + c * 8;
-          cp_async16(Vt + (c >> 3) * 8192 + tc::sw128(key, c & 7), src);
+        cp_async16(T + (c >> 3) * 8192 + tc::sw128(key, c & 7), src, bytes);
+      }
+    };
+    // K(t) is issued before V(t - 1): K stages are freed when both S are done,
+    // V stages when both PV are
+    for (int it = 0; it <= ntiles; ++it) {
+      if (it < ntiles) {
+        const int st = it & 1;
+        if (it >= 2) {
+          bool ok = true;
+          if (lane == 0) ok = tc::bar_wait(&kfree[st], ((it >> 1) - 1) & 1);
+          if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) {
+            healthy = false;
+            break;
+          }
         }
+        issue(true, Kst + st * 3 * 8192, it);
+        cp_async_mbar_arrive_noinc(&kfull[st]);
       }
-      if (nw > 0) {  // window positions from wlo0 + (max(a0, ent_n) - ent_n)
-        const int64_t rw = b * p.wrows + (wlo0 + (a0 + ne - ent_n) - p.wpos0);
-        for (int pc = pt; pc < nw * 24; pc += 128) {
-          const int key = ne + pc / 24, c = pc % 24;
-          cp_async16(Kt + (c >> 3) * 8192 + tc::sw128(key, c & 7), p.wk + rw * kDQK + pc * 8);
+      if (it >= 1) {
+        const int tile = it - 1, st = tile & 1;
+        if (tile >= 2) {
+          bool ok = true;
+          if (lane == 0) ok = tc::bar_wait(&vfree[st], ((tile >> 1) - 1) & 1);
+          if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) {
+            healthy = false;
+            break;
+          }
         }
-        for (int pc = pt; pc < nw * 16; pc += 128) {
-          const int key = ne + (pc >> 4), c = pc & 15;
-          const __nv_bfloat16* src = p.wv ? p.wv + rw * kDV + pc * 8 : p.wk + (rw + (pc >> 4)) * kDQK + c * 8;
-          cp_async16(Vt + (c >> 3) * 8192 + tc::sw128(key, c & 7), src);
-        }
+        issue(false, Vst + st * 2 * 8192, tile);
+        cp_async_mbar_arrive_noinc(&vfull[st]);
       }
-      for (int pc = pt; pc < (kBlkKeys - ne - nw) * 24; pc += 128) {
-        const int key = ne + nw + pc / 24, c = pc % 24;
-        cp_async16(Kt + (c >> 3) * 8192 + tc::sw128(key, c & 7), p.q, 0);
-      }
-      for (int pc = pt; pc < (kBlkKeys - ne - nw) * 16; pc += 128) {
-        const int key = ne + nw + (pc >> 4), c = pc & 15;
-        cp_async16(Vt + (c >> 3) * 8192 + tc::sw128(key, c & 7), p.q, 0);
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      tc::fence_async_smem();
-      named_sync(1, 128);
-      if (pt == 0) bar_arrive(&full[st]);
     }
-  } else {
-    // ===================== consumer: thread tid owns row tid =====================
-    constexpr uint32_t kIdescS = tc::idesc_bf16(128, kBlkKeys, false);
+    cp_async_wait<0>();
+  } else if (warp == 11) {
+    // ===================== MMA issue (one thread) =====================
+    constexpr uint32_t kIdescS = tc::idesc_bf16(128, kQbKeys, false);
     constexpr uint32_t kIdescO = tc::idesc_bf16(128, kDV, true);
-    const int qr = tid / H;                       // query of this row within the block
+    auto issue_s = [&](int tile) {
+      const int st = tile & 1;
+      const uint32_t ka = smem_u32(Kst + st * 3 * 8192);
+      tc::fence_async_smem();  // the stage was written by cp.async
+      tc::fence_after_sync();
+      for (int g = 0; g < 2; ++g) {
+        const uint32_t qa = smem_u32(Qs + g * 49152);
+#pragma unroll
+        for (int kk = 0; kk < 12; ++kk)
+          tc::mma_bf16_ss(tmem + 64 * (2 * g + st), tc::desc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                          tc::desc_sw128(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+        tc::mma_commit(&sdone[2 * g + st]);
+      }
+      tc::mma_commit(&kfree[st]);
+    };
+    if (lane == 0 && ntiles > 0) {
+      for (int tt = 0; tt < 2 && tt < ntiles; ++tt) {
+        if (healthy) healthy = tc::bar_wait(&kfull[tt], 0);
+        issue_s(tt);
+      }
+      for (int tile = 0; tile < ntiles; ++tile) {
+        const int st = tile & 1;
+        const uint32_t va = smem_u32(Vst + st * 2 * 8192);
+        for (int g = 0; g < 2; ++g) {
+          if (healthy) healthy = tc::bar_wait(&pready[g], tile & 1);
+          if (g == 0 && healthy) {
+            healthy = tc::bar_wait(&vfull[st], (tile >> 1) & 1);
+            tc::fence_async_smem();  // the stage was written by cp.async
+          }
+          tc::fence_after_sync();
+          const uint32_t pa = smem_u32(Pst + g * 16384);
+#pragma unroll
+          for (int ks = 0; ks < kQbKeys / 16; ++ks)
+            tc::mma_bf16_ss(tmem + 256 + 128 * g, tc::desc_sw128(pa + ks * 32, 16, 1024),
+                            tc::desc_sw128(va + ks * 2048, 8192, 1024), kIdescO, (tile > 0 || ks > 0) ? 1u : 0u);
+          tc::mma_commit(&pvdone[g]);
+        }
+        tc::mma_commit(&vfree[st]);
+        if (tile + 2 < ntiles) {
+          if (healthy) healthy = tc::bar_wait(&kfull[st], ((tile + 2) >> 1) & 1);
+          issue_s(tile + 2);
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // ===================== softmax: thread = row (query, head) of group g =====================
+    const int g = warp >> 2;
+    const int rl = tid & 127;          // TMEM lane
+    const int r = 128 * g + rl;        // row of the block
+    const int qr = r / H;              // query of this row within the block
     const bool row_ok = qr < nq;
     const int64_t tq = t0 + (row_ok ? qr : 0);
     int64_t nv_q = (tq + 1) / p.stride;
     if (nv_q > p.N) nv_q = p.N;
     const int64_t lo_q = (tq - p.wlen + 1) > 0 ? (tq - p.wlen + 1) : 0;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tO = tmem + 256 + 128 * g;
     float m_ref = -INFINITY, l = 0.f;
-    auto issue_s = [&](int tile) {
-      const int st = tile & 1;
-      const uint32_t qa = smem_u32(Qs), ka = smem_u32(Kst + st * 3 * 8192);
-      tc::fence_after_sync();
-#pragma unroll
-      for (int kk = 0; kk < 12; ++kk)
-        tc::mma_bf16_ss(tmem + 64 * st, tc::desc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                        tc::desc_sw128(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-      tc::mma_commit(&sdone[st]);
-    };
-    if (ntiles > 0 && tid == 0) {
-      if (healthy) healthy = tc::bar_wait(&full[0], 0);
-      issue_s(0);
-    }
     for (int tile = 0; tile < ntiles; ++tile) {
       const int st = tile & 1;
-      if (healthy) healthy = tc::bar_wait(&sdone[st], (tile >> 1) & 1);
+      if (healthy) healthy = tc::bar_wait(&sdone[2 * g + st], (tile >> 1) & 1);
       tc::fence_after_sync();
-      float sv[kBlkKeys];
-      tc::tmem_ld32(tmem + 64 * st + lane_base, sv);
-      tc::tmem_ld32(tmem + 64 * st + lane_base + 32, sv + 32);
+      float sv[kQbKeys];
+      tc::tmem_ld32(tmem + 64 * (2 * g + st) + lane_base, sv);
+      tc::tmem_ld32(tmem + 64 * (2 * g + st) + lane_base + 32, sv + 32);
       float mx = -INFINITY;
-      const int64_t sbase = static_cast<int64_t>(tile) * kBlkKeys;
+      const int64_t sbase = static_cast<int64_t>(tile) * kQbKeys;
 #pragma unroll
-      for (int j = 0; j < kBlkKeys; ++j) {
+      for (int j = 0; j < kQbKeys; ++j) {
         const int64_t sl = sbase + j;
         bool ok;
-        if (sl < ent_n) {
-          ok = sl < nv_q;
+        if (sl < n_ent) {
+          ok = sparse ? ((umask[sl] >> qr) & 1) != 0 : sl < nv_q;
         } else {
-          const int64_t pos = wlo0 + (sl - ent_n);
+          const int64_t pos = wlo0 + (sl - n_ent);
           ok = sl < n_slots && pos >= lo_q && pos <= tq;
         }
         ok = ok && row_ok;
@@ -1381,59 +1512,45 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_block_kernel(AttnParams p)
       const float base = m_ref == -INFINITY ? 0.f : m_ref;
       float sum = 0.f;
 #pragma unroll
-      for (int j = 0; j < kBlkKeys; ++j) {
-        sv[j] = exp2f(sv[j] - base);
+      for (int j = 0; j < kQbKeys; ++j) {
+        sv[j] = fast_exp2(sv[j] - base);
         sum += sv[j];
       }
       l += sum;
-      if (tile > 0 && __any_sync(0xffffffffu, resc)) {
-        if (healthy) healthy = tc::bar_wait(&empty[(tile - 1) & 1], ((tile - 1) >> 1) & 1);
+      if (tile > 0) {  // PV of the previous tile: the P buffer is free and O is quiet
+        if (healthy) healthy = tc::bar_wait(&pvdone[g], (tile - 1) & 1);
         tc::fence_after_sync();
+        if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float ov[32];
-          tc::tmem_ld32(tO + lane_base + 32 * c, ov);
+          for (int c = 0; c < 4; ++c) {
+            float ov[32];
+            tc::tmem_ld32(tO + lane_base + 32 * c, ov);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] *= corr;
-          tc::tmem_st32(tO + lane_base + 32 * c, ov);
+            for (int i = 0; i < 32; ++i) ov[i] *= corr;
+            tc::tmem_st32(tO + lane_base + 32 * c, ov);
+          }
+          tc::tmem_wait_st();
         }
-        tc::tmem_wait_st();
       }
       {
-        uint8_t* Pb = Pst + st * 16384;
+        uint8_t* Pb = Pst + g * 16384;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const uint4 v = make_uint4(pack_bf16x2(sv[8 * c], sv[8 * c + 1]), pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]),
                                      pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]),
                                      pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]));
-          *reinterpret_cast<uint4*>(Pb + tc::sw128(tid, c)) = v;
+          *reinterpret_cast<uint4*>(Pb + tc::sw128(rl, c)) = v;
         }
       }
       tc::fence_async_smem();
       tc::fence_before_sync();
-      named_sync(2, 128);
-      if (tid == 0) {
-        tc::fence_after_sync();
-        const uint32_t pa = smem_u32(Pst + st * 16384);
-        const uint32_t va = smem_u32(Vst + st * 2 * 8192);
-#pragma unroll
-        for (int ks = 0; ks < kBlkKeys / 16; ++ks)
-          tc::mma_bf16_ss(tO, tc::desc_sw128(pa + ks * 32, 16, 1024), tc::desc_sw128(va + ks * 2048, 8192, 1024),
-                          kIdescO, (tile > 0 || ks > 0) ? 1u : 0u);
-        tc::mma_commit(&empty[st]);
-        if (tile + 1 < ntiles) {
-          if (healthy) healthy = tc::bar_wait(&full[st ^ 1], ((tile + 1) >> 1) & 1);
-          issue_s(tile + 1);
-        }
-      }
+      named_sync(2 + g, 128);
+      if (rl == 0) bar_arrive(&pready[g]);
     }
-    if (ntiles > 0) {
-      const int last = ntiles - 1;
-      if (healthy) healthy = tc::bar_wait(&empty[last & 1], (last >> 1) & 1);
-      tc::fence_after_sync();
-    }
+    if (ntiles > 0 && healthy) healthy = tc::bar_wait(&pvdone[g], (ntiles - 1) & 1);
+    tc::fence_after_sync();
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16* o = p.out + ((b * p.Tq + r0) * H + tid) * kDV;
+    __nv_bfloat16* o = p.out + ((b * p.Tq + r0) * H + r) * kDV;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       float ov[32];
@@ -1451,12 +1568,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_block_kernel(AttnParams p)
                          pack_bf16x2(ov[i + 4] * inv, ov[i + 5] * inv), pack_bf16x2(ov[i + 6] * inv, ov[i + 7] * inv));
       }
     }
-    if (row_ok && p.lse) p.lse[(b * p.Tq + r0) * H + tid] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+    if (row_ok && p.lse) p.lse[(b * p.Tq + r0) * H + r] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
   }
-  cp_async_wait<0>();
+  pdl_trigger();
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, 256);
+  if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------------
@@ -1789,11 +1906,16 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
     }
   }
 
-  // dense (HCA) prefill over a bf16 cache: query-blocked tcgen05 kernel
-  const bool use_blk = idx == nullptr && !fp8 && Tq >= 128 / H && R >= 2LL * num_sms() && pk == nullptr;
+  // prefill over a bf16 cache with many query rows: the query-blocked tcgen05
+  // kernel, for dense (HCA) attention and for sparse attention with few heads
+  // and short selections (the block's union of selections fits on chip)
+  const int qb_rows = 256 / H;
+  const bool blk_shape = !fp8 && pk == nullptr && Tq >= qb_rows && R >= 2LL * num_sms();
+  const bool use_blk = blk_shape && (idx == nullptr || (H == 16 && static_cast<int64_t>(qb_rows) * k <= kQbMaxCand &&
+                                                        N <= kQbMaxEnt));
   if (use_blk) {
-    fn = attn_block_kernel;
-    smem = blk_layout().total;
+    fn = attn_qblock_kernel;
+    smem = qb_layout().total;
     if (!ensure_smem(reinterpret_cast<const void*>(fn), static_cast<int>(smem)))
       return fail(CSA_ERR_CUDA, "%s: cannot raise the shared memory limit to %zu", name, smem);
     pl.cl = 1;
@@ -1829,8 +1951,8 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   p.cu_ent = pk ? pk->cu_entries : nullptr;
   p.n_seqs = pk ? pk->n_seqs : 0;
 
-  const dim3 grid(static_cast<unsigned>(use_blk ? B * ((Tq + (128 / H) - 1) / (128 / H)) : R * pl.cl));
-  const dim3 block(use_blk ? kTcThreads : (use_tc ? kTcDecThreads : kThreads));
+  const dim3 grid(static_cast<unsigned>(use_blk ? B * ((Tq + qb_rows - 1) / qb_rows) : R * pl.cl));
+  const dim3 block(use_blk ? kQbThreads : (use_tc ? kTcDecThreads : kThreads));
   const int cluster = (use_tc && !tc_cluster) || use_blk ? 1 : pl.cl;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   prof_begin(s);

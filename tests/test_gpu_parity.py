@@ -136,6 +136,9 @@ def _oracle_idx(g, B, Tq, N, m, k, q_pos0):
     # 64 heads, 5 tiles of 128 slots per late row: the K/V stage rings wrap and their barrier phases flip
     (64, 1, 2000, 4, 512, 128, True),    # separate V: 2 stages
     (64, 1, 2000, 4, 512, 128, False),   # V = K[:, :128]: 3 stages
+    # 16 heads, many rows: query-blocked kernel over the union of 16 queries' selections
+    (16, 2, 333, 4, 24, 0, False),       # ragged last block, no window, V = K[:, :128]
+    (16, 1, 1500, 4, 128, 128, True),    # 16 x 128 selections per block: the largest union
 ])
 def test_csa_sparse_mqa_prefill_bf16(H, B, T, m, k, win, sep_v):
     g = np.random.default_rng(H + T + k)
