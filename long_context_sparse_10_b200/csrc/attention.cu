@@ -1217,7 +1217,7 @@ constexpr int kQbMaxCand = 2048;   // sparse path: block queries x k
 constexpr int kQbMaxEnt = 16384;   // sparse path: entries per sequence (bit set in the P buffers)
 
 struct QbLayout {
-  size_t q, k, v, p, ulist, umask, bars, total;
+  size_t q, k, v, p, ulist, qbits, bars, total;
 };
 
 __host__ __device__ inline QbLayout qb_layout() {
@@ -1228,10 +1228,19 @@ __host__ __device__ inline QbLayout qb_layout() {
   L.v = off; off += 2 * 2 * 8192;       // V: 2 stages x 64 keys x 128 dims
   L.p = off; off += 2 * 16384;          // P: 2 groups x 128 rows x 64 keys (prologue: entry bit set)
   L.ulist = off; off += kQbMaxCand * 2; // union entries (uint16)
-  L.umask = off; off += kQbMaxCand * 2; // their query bits (uint16)
+  L.qbits = off; off += 16 * kQbMaxCand / 8;  // per query: bit u = it selected union entry u
   L.bars = off; off += 256;              // 16 mbarriers + the TMEM address
   L.total = off + 1024;
   return L;
+}
+
+// Bits of the slots [lo, hi] (inclusive) within the 64-slot tile starting at sb.
+__device__ __forceinline__ uint64_t range_bits(int lo, int hi, int sb) {
+  const int a = lo - sb > 0 ? lo - sb : 0;
+  const int b = hi + 1 - sb < 64 ? hi + 1 - sb : 64;
+  if (a >= b) return 0ull;
+  const uint64_t upto = b == 64 ? ~0ull : ((1ull << b) - 1ull);
+  return upto & ~((1ull << a) - 1ull);
 }
 
 __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p) {
@@ -1244,7 +1253,7 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
   uint8_t* Vst = smem + L.v;
   uint8_t* Pst = smem + L.p;
   uint16_t* ulist = reinterpret_cast<uint16_t*>(smem + L.ulist);
-  uint16_t* umask = reinterpret_cast<uint16_t*>(smem + L.umask);
+  uint32_t* qbits = reinterpret_cast<uint32_t*>(smem + L.qbits);  // [16 queries][kQbMaxCand / 32]
   uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + L.bars);  // [2] K stage loaded (one arrival per loader)
   uint64_t* vfull = kfull + 2;                                     // [2] V stage loaded (same)
   uint64_t* kfree = vfull + 2;                                     // [2] both S of the K stage's tile done
@@ -1296,6 +1305,7 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
     uint32_t* bits = reinterpret_cast<uint32_t*>(Pst);
     const int nwords = static_cast<int>((p.N + 1) / 2);
     for (int w = tid; w < nwords; w += kQbThreads) bits[w] = 0u;
+    for (int w = tid; w < 16 * kQbMaxCand / 32; w += kQbThreads) qbits[w] = 0u;
     __syncthreads();
     for (int c = tid; c < nq * p.k; c += kQbThreads) {
       const int q = c / p.k;
@@ -1332,16 +1342,15 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
     }
     __syncthreads();
     int pos = s_count[warp] + incl - cnt;
+    auto put = [&](int e, uint32_t qm) {  // union entry `pos`: entry e, selected by the queries in qm
+      ulist[pos] = static_cast<uint16_t>(e);
+      for (; qm != 0u; qm &= qm - 1u) atomicOr(&qbits[(__ffs(qm) - 1) * (kQbMaxCand / 32) + (pos >> 5)], 1u << (pos & 31));
+      ++pos;
+    };
     for (int w = w0; w < w1; ++w) {
       const uint32_t v = bits[w];
-      if ((v & 0xffffu) != 0u) {
-        ulist[pos] = static_cast<uint16_t>(2 * w);
-        umask[pos++] = static_cast<uint16_t>(v & 0xffffu);
-      }
-      if ((v >> 16) != 0u) {
-        ulist[pos] = static_cast<uint16_t>(2 * w + 1);
-        umask[pos++] = static_cast<uint16_t>(v >> 16);
-      }
+      if ((v & 0xffffu) != 0u) put(2 * w, v & 0xffffu);
+      if ((v >> 16) != 0u) put(2 * w + 1, v >> 16);
     }
     n_ent = s_union;
   }
@@ -1357,32 +1366,33 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
 
   if (warp >= 8 && warp < 11) {
     // ===================== producer: cp.async copies that arrive by themselves =====================
-    const int pt = tid - 256;
     const int64_t ebase = b * p.N;
     const int64_t wbase = b * p.wrows - p.wpos0 + wlo0;
     const __nv_bfloat16* ve = p.cv ? p.cv : p.ck;
     const int ves = p.cv ? kDV : kDQK;
     const __nv_bfloat16* vw = p.wv ? p.wv : p.wk;
     const int vws = p.wv ? kDV : kDQK;
-    // K (24 chunks per key) or V (16 chunks per key) of one tile
+    // K (three 128-byte blocks per key) or V (two) of one tile: eight lanes per
+    // 128-byte row segment, four keys per warp instruction
+    const int pw = warp - 8, c8 = lane & 7;
     auto issue = [&](bool is_k, uint8_t* T, int tile) {
-      const int nch = is_k ? 24 : 16;
       const int64_t a0 = static_cast<int64_t>(tile) * kQbKeys;
-      for (int pc = pt; pc < kQbKeys * nch; pc += kQbLoaders) {
-        const int key = pc / nch, c = pc % nch;
+      for (int key = pw * 4 + (lane >> 3); key < kQbKeys; key += 12) {
         const int64_t sl = a0 + key;
-        const __nv_bfloat16* src = p.q;
-        int bytes = 0;
+        const __nv_bfloat16* src = nullptr;
         if (sl < n_ent) {
           const int64_t e = ebase + (sparse ? static_cast<int64_t>(ulist[sl]) : sl);
-          src = is_k ? p.ck + e * kDQK + c * 8 : ve + e * ves + c * 8;
-          bytes = 16;
+          src = is_k ? p.ck + e * kDQK : ve + e * ves;
         } else if (sl < n_slots) {
           const int64_t w = wbase + (sl - n_ent);
-          src = is_k ? p.wk + w * kDQK + c * 8 : vw + w * vws + c * 8;
-          bytes = 16;
+          src = is_k ? p.wk + w * kDQK : vw + w * vws;
         }
-        cp_async16(T + (c >> 3) * 8192 + tc::sw128(key, c & 7), src, bytes);
+        uint8_t* dst = T + tc::sw128(key, c8);
+        const __nv_bfloat16* s8 = src != nullptr ? src + c8 * 8 : p.q;
+        const int bytes = src != nullptr ? 16 : 0;
+        cp_async16(dst, s8, bytes);
+        cp_async16(dst + 8192, src != nullptr ? s8 + 64 : p.q, bytes);
+        if (is_k) cp_async16(dst + 16384, src != nullptr ? s8 + 128 : p.q, bytes);
       }
     };
     // K(t) is issued before V(t - 1): K stages are freed when both S are done,
@@ -1475,6 +1485,9 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
     int64_t nv_q = (tq + 1) / p.stride;
     if (nv_q > p.N) nv_q = p.N;
     const int64_t lo_q = (tq - p.wlen + 1) > 0 ? (tq - p.wlen + 1) : 0;
+    // slot numbers (below 2^31): the entry run, this row's visible entries and window slots
+    const int ent32 = static_cast<int>(n_ent), nv32 = static_cast<int>(nv_q);
+    const int wv_lo = static_cast<int>(n_ent + (lo_q - wlo0)), wv_hi = static_cast<int>(n_ent + (tq - wlo0));
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tmem + 256 + 128 * g;
     float m_ref = -INFINITY, l = 0.f;
@@ -1485,19 +1498,23 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
       float sv[kQbKeys];
       tc::tmem_ld32(tmem + 64 * (2 * g + st) + lane_base, sv);
       tc::tmem_ld32(tmem + 64 * (2 * g + st) + lane_base + 32, sv + 32);
+      // this row's visible slots of the tile as a bit mask: its entries, then its window run
+      const int sb = tile * kQbKeys;
+      uint64_t vm = 0;
+      if (row_ok) {
+        if (sb < ent32) {
+          vm = sparse ? (static_cast<uint64_t>(qbits[qr * (kQbMaxCand / 32) + (sb >> 5) + 1]) << 32) |
+                            qbits[qr * (kQbMaxCand / 32) + (sb >> 5)]
+                      : range_bits(0, nv32 - 1, sb);
+          vm &= range_bits(0, ent32 - 1, sb);
+        }
+        vm |= range_bits(wv_lo, wv_hi, sb);
+      }
+      const uint32_t vlo = static_cast<uint32_t>(vm), vhi = static_cast<uint32_t>(vm >> 32);
       float mx = -INFINITY;
-      const int64_t sbase = static_cast<int64_t>(tile) * kQbKeys;
 #pragma unroll
       for (int j = 0; j < kQbKeys; ++j) {
-        const int64_t sl = sbase + j;
-        bool ok;
-        if (sl < n_ent) {
-          ok = sparse ? ((umask[sl] >> qr) & 1) != 0 : sl < nv_q;
-        } else {
-          const int64_t pos = wlo0 + (sl - n_ent);
-          ok = sl < n_slots && pos >= lo_q && pos <= tq;
-        }
-        ok = ok && row_ok;
+        const bool ok = (((j < 32 ? vlo : vhi) >> (j & 31)) & 1u) != 0u;
         sv[j] = ok ? sv[j] * p.scale_log2 : -INFINITY;
         mx = fmaxf(mx, sv[j]);
       }
