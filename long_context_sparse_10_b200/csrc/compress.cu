@@ -103,6 +103,14 @@ __device__ __forceinline__ void load8f(const float* p, float* f) {
   f[4] = v.x; f[5] = v.y; f[6] = v.z; f[7] = v.w;
 }
 
+// 2^x by the hardware approximation (relative error ~2^-22, far below the
+// bf16 rounding of the entry it weights); 0 for x = -inf.
+__device__ __forceinline__ float exp2f_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Writes output row e.  Called by all 32 lanes; lane g < G holds channels
 // [8g, 8g+8) in y.
 __device__ __forceinline__ void store_entry(const CompressParams& p, int64_t e, int lane, const float* y) {
@@ -203,44 +211,136 @@ __global__ void __launch_bounds__(256) compress_flat_kernel(CompressParams p) {
     const int64_t j = start + r;
     raw[r] = (j >= 0 && j < er.T) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
   }
-  // two passes over the rows in registers: the per-channel maximum of the
-  // logits, then one exponential per (row, channel)
-  float mx[8];
+  // logits of every row kept in registers (rows outside the sequence take no
+  // part: -inf), the per-channel maximum, then one exponential per element
+  // with the subtraction folded into an FMA in the base-2 domain
+  float lg[CW][8], mx[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
 #pragma unroll
   for (int r = 0; r < CW; ++r) {
     const int64_t j = start + r;
-    if (j < 0 || j >= er.T) continue;  // positions outside the sequence take no part
-    float xv[8], bv[8];
-    unpack8(raw[r], xv);
-    load8f(p.b + r * p.d + 8 * g, bv);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], fmaf(wv[c], xv[c], bv[c]));
-  }
-  float sm[8], ac[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) sm[c] = ac[c] = 0.f;
-#pragma unroll
-  for (int r = 0; r < CW; ++r) {
-    const int64_t j = start + r;
-    if (j < 0 || j >= er.T) continue;
+    const bool in = j >= 0 && j < er.T;
     float xv[8], bv[8];
     unpack8(raw[r], xv);
     load8f(p.b + r * p.d + 8 * g, bv);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      const float e = __expf(fmaf(wv[c], xv[c], bv[c]) - mx[c]);
-      sm[c] += e;
-      ac[c] = fmaf(e, xv[c], ac[c]);
+      lg[r][c] = in ? fmaf(wv[c], xv[c], bv[c]) : -INFINITY;
+      mx[c] = fmaxf(mx[c], lg[r][c]);
+    }
+  }
+  float sm[8], ac[8], m2[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    sm[c] = ac[c] = 0.f;
+    m2[c] = mx[c] * kLog2e;
+  }
+#pragma unroll
+  for (int r = 0; r < CW; ++r) {
+    float xv[8];
+    unpack8(raw[r], xv);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float ex = exp2f_fast(fmaf(lg[r][c], kLog2e, -m2[c]));  // 0 for rows outside the sequence
+      sm[c] += ex;
+      ac[c] = fmaf(ex, xv[c], ac[c]);
     }
   }
   uint4 o;
-  o.x = pack_bf16x2(ac[0] / sm[0], ac[1] / sm[1]);
-  o.y = pack_bf16x2(ac[2] / sm[2], ac[3] / sm[3]);
-  o.z = pack_bf16x2(ac[4] / sm[4], ac[5] / sm[5]);
-  o.w = pack_bf16x2(ac[6] / sm[6], ac[7] / sm[7]);
+  o.x = pack_bf16x2(__fdividef(ac[0], sm[0]), __fdividef(ac[1], sm[1]));
+  o.y = pack_bf16x2(__fdividef(ac[2], sm[2]), __fdividef(ac[3], sm[3]));
+  o.z = pack_bf16x2(__fdividef(ac[4], sm[4]), __fdividef(ac[5], sm[5]));
+  o.w = pack_bf16x2(__fdividef(ac[6], sm[6]), __fdividef(ac[7], sm[7]));
   *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + er.out_row * p.d + 8 * g) = o;
+}
+
+// Long windows of 128 rows (HCA with m' = 128): one CTA of 16 G threads per
+// entry, thread (s, g) = 8 channels of group g over the 8 rows s, s + 16, ...;
+// the per-channel maxima meet in shared memory first, then the partial sums,
+// and warp 0 finishes the entry.  Every lane works whatever d is.
+__global__ void __launch_bounds__(512) compress_wide_kernel(CompressParams p) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float red[16][2][8][32];  // [row subset][max | sum, weighted sum][channel][group]
+  const int tid = threadIdx.x;
+  const int g = tid % p.G, rs = tid / p.G;
+  const EntryRef er = entry_ref(p, blockIdx.x);
+  const int64_t start = er.i * p.stride - (128 - p.stride);
+  float wv[8];
+  load8f(p.w + 8 * g, wv);
+  const __nv_bfloat16* xb = er.x0 + 8 * g;
+  uint4 raw[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t j = start + rs + 16 * i;
+    raw[i] = (j >= 0 && j < er.T) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float lg[8][8], mx[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = rs + 16 * i;
+    const int64_t j = start + r;
+    const bool in = j >= 0 && j < er.T;
+    float xv[8], bv[8];
+    unpack8(raw[i], xv);
+    load8f(p.b + r * p.d + 8 * g, bv);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      lg[i][c] = in ? fmaf(wv[c], xv[c], bv[c]) : -INFINITY;
+      mx[c] = fmaxf(mx[c], lg[i][c]);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) red[rs][0][c][g] = mx[c];
+  __syncthreads();
+  float m2[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2) m = fmaxf(m, red[s2][0][c][g]);
+    m2[c] = m == -INFINITY ? 0.f : m * kLog2e;
+  }
+  float sm[8], ac[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) sm[c] = ac[c] = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float xv[8];
+    unpack8(raw[i], xv);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float ex = exp2f_fast(fmaf(lg[i][c], kLog2e, -m2[c]));
+      sm[c] += ex;
+      ac[c] = fmaf(ex, xv[c], ac[c]);
+    }
+  }
+  __syncthreads();  // every thread has read the maxima
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    red[rs][0][c][g] = sm[c];
+    red[rs][1][c][g] = ac[c];
+  }
+  __syncthreads();
+  if (tid >= 32) return;
+  const int lane = tid;
+  float y[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float S = 0.f, A = 0.f;
+    if (lane < p.G) {
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2) {
+        S += red[s2][0][c][lane];
+        A += red[s2][1][c][lane];
+      }
+    }
+    y[c] = lane < p.G ? __fdividef(A, S) : 0.f;
+  }
+  store_entry(p, er.out_row, lane, y);
 }
 
 // One CTA per entry (long windows): 8 warps take interleaved rows, then warp 0
@@ -379,8 +479,9 @@ csa_status launch(const char* name, const CompressParams& p, int64_t entries, vo
                    p);
   } else if (p.cwin <= 32) {
     e = launch_pdl(compress_short_kernel, dim3(static_cast<unsigned>((entries + 7) / 8)), dim3(256), 0, s, 1, p);
-  } else if (p.cwin == 128) {  // HCA with m' = 128: 16 rows per warp
-    e = launch_pdl(compress_long_kernel<16>, dim3(static_cast<unsigned>(entries)), dim3(256), 0, s, 1, p);
+  } else if (p.cwin == 128) {  // HCA with m' = 128: 16 row subsets of 8 rows per channel group
+    e = launch_pdl(compress_wide_kernel, dim3(static_cast<unsigned>(entries)), dim3(static_cast<unsigned>(16 * p.G)), 0,
+                   s, 1, p);
   } else {
     e = launch_pdl(compress_long_kernel<0>, dim3(static_cast<unsigned>(entries)), dim3(256), 0, s, 1, p);
   }
