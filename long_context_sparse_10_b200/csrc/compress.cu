@@ -7,12 +7,15 @@
 // overlapping compression.  Per channel c of entry i with window start s:
 //   alpha_j = softmax over in-range j of (w[c] x[j,c] + b[j - s, c]),
 //   y[i,c]  = sum_j alpha_j x[j,c].
-// The softmax runs online in fp32 (running max, rescaled sum and weighted sum).
+// The softmax runs in fp32: the per-channel maximum of the logits, then one
+// exponential per element (or online, for windows of unknown length).
 //
-// Memory bound: each lane owns 8 channels (one 16-byte load per token row), a
-// warp covers one entry's row (d <= 256).  Short windows (CSA) use one warp
-// per entry; long windows (HCA) spread the rows of one entry over 8 warps and
-// merge their softmax states in shared memory.
+// A thread owns 8 channels (one 16-byte load per token row).  CSA windows of 8
+// rows (m = 4, bf16 output): one thread per (entry, channel group), its rows'
+// logits kept in registers.  Other short windows: one warp per entry.  HCA
+// windows of 128 rows: 16 row subsets per channel group in one CTA per entry,
+// their maxima and sums merged in shared memory; other long windows: 8 warps
+// per entry with online softmax states merged in shared memory.
 #include "common.cuh"
 #include "host_util.h"
 
