@@ -523,11 +523,11 @@ constexpr int kTypeRing = 4;
 
 
 // K-tile stages: three when the V tile is the K tile, two otherwise.
-__host__ __device__ constexpr int tc_stages(bool shv) { return shv ? 3 : 2; }
+__host__ __device__ constexpr int tc_stages(bool fp8, bool shv) { return (void)fp8, shv ? 3 : 2; }
 
 __host__ __device__ inline TcLayout tc_layout(bool fp8, bool shv, int tps) {
   TcLayout L;
-  const int ns = tc_stages(shv);
+  const int ns = tc_stages(fp8, shv);
   size_t off = 0;
   L.q = off; off += 3 * 8192;                    // Q: 64 heads x 192 dims
   L.k = off; off += ns * 3 * 16384;              // K: stages x 128 keys x 192 dims
@@ -604,7 +604,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   uint8_t* Vst = smem + L.v;
   uint8_t* Pst = smem + L.p;
   uint8_t* ones = smem + L.ones;
-  constexpr int NS = tc_stages(SHV);
+  constexpr int NS = tc_stages(FP8, SHV);
   auto stype = reinterpret_cast<int(*)[kTcKeys]>(smem + L.stype);  // [tile % kTypeRing][slot]
   auto srow = reinterpret_cast<int64_t(*)[kTcKeys]>(smem + L.srow);
   float* mref = reinterpret_cast<float*>(smem + L.mref);
@@ -694,31 +694,51 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
       tc::mma_commit(&sdone[tile & 1]);
       if (kSplitKV) tc::mma_commit(&kfree[kst]);
     };
+    const uint64_t onesdesc = tc::desc_sw128(smem_u32(ones), 16, 0);
+    auto issue_pv = [&](int tile) {
+      const int kst = tile % NS, pb = tile & 1;
+      if (!FP8) tc::fence_async_smem();  // the stage was written by cp.async
+      tc::fence_after_sync();
+      const uint32_t pa = smem_u32(Pst + pb * 16384);
+      const uint32_t va = SHV ? smem_u32(Kst + kst * 3 * kKB) : smem_u32(Vst + kst * 2 * kKB);
+#pragma unroll
+      for (int ks = 0; ks < kTcKeys / 16; ++ks) {
+        const uint64_t pdesc = tc::desc_sw128(pa + ks * 2048, 8192, 1024);
+        const uint32_t acc = (tile > 0 || ks > 0) ? 1u : 0u;
+        tc::mma_bf16_ss(tO, tc::desc_sw128(va + ks * 2048, kKB, 1024), pdesc, kIdescO, acc);
+        tc::mma_bf16_ss(tL, onesdesc, pdesc, kIdescL, acc);
+      }
+      tc::mma_commit(&empty[kst]);
+    };
     if (lane == 0 && ntiles > 0) {
       for (int t0 = 0; t0 < 2 && t0 < ntiles; ++t0) {
         if (healthy) healthy = tc::bar_wait(&full[t0 % NS], (t0 / NS) & 1);
         issue_s(t0);
       }
-      const uint64_t onesdesc = tc::desc_sw128(smem_u32(ones), 16, 0);
-      for (int tile = 0; tile < ntiles; ++tile) {
-        const int kst = tile % NS, pb = tile & 1;
-        if (healthy) healthy = tc::bar_wait(&pready[pb], (tile >> 1) & 1);
-        if (kSplitKV && healthy) healthy = tc::bar_wait(&vfull[kst], (tile / NS) & 1);
-        if (!FP8) tc::fence_async_smem();  // the stage was written by cp.async
-        tc::fence_after_sync();
-        const uint32_t pa = smem_u32(Pst + pb * 16384);
-        const uint32_t va = SHV ? smem_u32(Kst + kst * 3 * kKB) : smem_u32(Vst + kst * 2 * kKB);
-#pragma unroll
-        for (int ks = 0; ks < kTcKeys / 16; ++ks) {
-          const uint64_t pdesc = tc::desc_sw128(pa + ks * 2048, 8192, 1024);
-          const uint32_t acc = (tile > 0 || ks > 0) ? 1u : 0u;
-          tc::mma_bf16_ss(tO, tc::desc_sw128(va + ks * 2048, kKB, 1024), pdesc, kIdescO, acc);
-          tc::mma_bf16_ss(tL, onesdesc, pdesc, kIdescL, acc);
+      // Whichever is ready first: PV(next_pv) once its P (and V) are in, or
+      // S(next_s) once its K stage is loaded and PV(next_s - 2) has been issued
+      // (S(next_s) reuses the TMEM buffer and, through its commit, releases
+      // the P buffer of tile next_s - 2).  Neither waits behind the other.
+      int next_pv = 0, next_s = 2;
+      uint32_t idle = 0;
+      while (next_pv < ntiles && healthy) {
+        bool moved = false;
+        if (next_s < ntiles && next_s - 2 < next_pv && tc::bar_test(&full[next_s % NS], (next_s / NS) & 1)) {
+          issue_s(next_s);
+          ++next_s;
+          moved = true;
         }
-        tc::mma_commit(&empty[kst]);
-        if (tile + 2 < ntiles) {
-          if (healthy) healthy = tc::bar_wait(&full[(tile + 2) % NS], ((tile + 2) / NS) & 1);
-          issue_s(tile + 2);
+        if (tc::bar_test(&pready[next_pv & 1], (next_pv >> 1) & 1) &&
+            (!kSplitKV || tc::bar_test(&vfull[next_pv % NS], (next_pv / NS) & 1))) {
+          issue_pv(next_pv);
+          ++next_pv;
+          moved = true;
+        }
+        if (moved) {
+          idle = 0;
+        } else if (++idle > tc::kPollLimit) {
+          atomicExch(&tc::g_device_error, tc::kErrWaitTimeout);
+          healthy = false;
         }
       }
     }
@@ -1715,7 +1735,7 @@ KernelFn pick(int H, bool fp8, bool shv) {
 using TcKernelFn = void (*)(AttnParams);
 
 TcKernelFn pick_tc(bool fp8, bool shv) {
-  if (fp8) return shv ? attn_tc_kernel<true, true> : attn_tc_kernel<true, false>;
+  if (fp8) return attn_tc_kernel<true, true>;  // (an FP8 cache with a separate V never takes this path)
   return shv ? attn_tc_kernel<false, true> : attn_tc_kernel<false, false>;
 }
 

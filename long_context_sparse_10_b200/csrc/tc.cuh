@@ -95,6 +95,19 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
   return bar_wait_bounded(bar, parity, kWaitLimit);
 }
 
+// Non-blocking test of the phase with parity `parity`.  Loops that poll
+// several barriers with it give up after kPollLimit rounds without progress.
+constexpr uint32_t kPollLimit = 1u << 26;
+__device__ __forceinline__ bool bar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Arrives once on `bar` and raises its expected transaction count by `bytes`
 // (the bulk copies that complete on the barrier then count those bytes down).
 __device__ __forceinline__ void bar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
