@@ -10,17 +10,19 @@
 // the same scaled nope channels (shared key and value).
 //
 // Each query row's key list is a sequence of "slots" (entry slots first, then
-// window slots), processed in tiles of 64 keys.  A CTA of 4 warps owns one row
-// and a contiguous range of its tiles; all query heads of the row share each
-// staged key/value tile (the MQA reuse).  H = 64: each warp owns 16 heads and
-// all keys of a tile; H = 16: each warp owns the 16 heads and a quarter of the
-// tile's keys.  Tiles are double-buffered with cp.async: the next tile's rows
-// (gathered by index for CSA, contiguous for HCA) stream in while the current
-// one is multiplied.  FP8 codes are staged raw and widened to bf16 in shared
-// memory (exact: every E4M3 value is a bf16 value); the per-entry scale is
-// applied to the nope part of the logit and to the probability on the value
-// side, so no rounding is added to cache values.  QK^T and PV are bf16
-// tensor-core MMAs (fp32 accumulate) with an online softmax in the exp2 domain.
+// window slots).  Three kernels cover the shapes:
+//  - attn_tc_kernel (64 heads): one row per CTA (or a contiguous range of its
+//    128-key tiles, for few rows), tcgen05 MMAs with the keys as the M
+//    dimension; described where it is defined.
+//  - attn_qblock_kernel (prefill over a bf16 cache: dense HCA attention, and
+//    sparse CSA attention with few heads): a block of consecutive queries per
+//    CTA, 256 (query, head) rows sharing each 64-key tile of the block's keys.
+//  - attn_kernel (warp-level mma.sync, 16 heads, the remaining shapes: few
+//    rows, an FP8 cache, packed sequences): one row per CTA in tiles of 64
+//    keys, double-buffered with cp.async; FP8 codes are widened in shared
+//    memory and the per-entry scale applied to the nope part of the logit and
+//    to the probability on the value side.
+// All keep fp32 accumulators and an online softmax in the exp2 domain.
 //
 // Rows that are few (decode) split their tiles over several CTAs, merged in
 // one of two ways: a thread-block cluster of up to 16 CTAs whose partial
@@ -498,13 +500,16 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
 // (three 64-dim blocks), Q K-major, V^T read MN-major straight out of the
 // first two K blocks when key and value are shared, P^T MN-major, and the
 // all-ones A operand of the l update is one 1 KB swizzle atom read with a
-// zero row-group stride.  Warps 8-15 gather and widen key tiles (FP8 entries
-// dequantised, code x scale rounded to bf16, from registers into the K
-// tile); one thread of warp 16 issues every MMA in the order S(0), S(1), then
-// per tile t: PV(t) and the l update once P(t) is written, S(t+2) into the
-// TMEM buffer P(t)'s softmax has drained.  When key and value are shared the
-// K tile has three stages (two with a separate V tile).  Every mbarrier wait
-// is bounded; a timeout sets the device error word instead of hanging.
+// zero row-group stride.  Warps 8-15 gather key tiles: FP8 entries are
+// dequantised (code x scale rounded to bf16, from registers into the K tile);
+// bf16 rows are copied with cp.async whose completions arrive on the stage
+// barrier themselves, K stages released when S is done and V stages when PV
+// is (separate V).  One thread of warp 16 issues every MMA: S(0), S(1), then
+// whichever is ready first of PV(t) + the l update (once P(t) is written) and
+// S(t+2) (once its keys are in and PV(t) has gone out, so that S(t+2)'s
+// commit also releases P buffer t % 2).  When key and value are shared the K
+// tile has three stages (two with a separate V tile).  Every mbarrier wait is
+// bounded; a timeout sets the device error word instead of hanging.
 // ---------------------------------------------------------------------------
 constexpr int kTcKeys = 128;
 
