@@ -17,9 +17,10 @@
 //  - attn_qblock_kernel (prefill over a bf16 cache: dense HCA attention, and
 //    sparse CSA attention with few heads): a block of consecutive queries per
 //    CTA, 256 (query, head) rows sharing each 64-key tile of the block's keys.
-//  - attn_kernel (warp-level mma.sync, 16 heads, the remaining shapes: few
-//    rows, an FP8 cache, packed sequences): one row per CTA in tiles of 64
-//    keys, double-buffered with cp.async; FP8 codes are widened in shared
+//  - attn_kernel (warp-level mma.sync, the remaining shapes: 16 heads with few
+//    rows, an FP8 cache or packed sequences; 64 heads over an FP8 cache with a
+//    separate raw-window V): one row per CTA in tiles of 64 keys,
+//    double-buffered with cp.async; FP8 codes are widened in shared
 //    memory and the per-entry scale applied to the nope part of the logit and
 //    to the probability on the value side.
 // All keep fp32 accumulators and an online softmax in the exp2 domain.
