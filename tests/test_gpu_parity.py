@@ -106,6 +106,11 @@ def _indexer_case(g, B, Tq, N, tie_blocks=0, zero_q=False):
     # prefill rows at k = 2048 (row path): visible counts crossing k, and near 16384
     (1, 300, 16384, 8000, 4, 2048, 0, False),
     (1, 300, 16384, 65536 - 300, 4, 2048, 0, False),
+    # enough prefill rows (>= 32 per SM) for the on-chip tcgen05 kernel
+    (3, 1700, 425, 0, 4, 64, 0, False),        # k > visible early on, three sequences
+    (1, 5000, 5000, 0, 1, 33, 4, False),       # exact ties in blocks of 4
+    (1, 5000, 1250, 0, 4, 16, 0, True),        # all scores zero: lowest indices win
+    (1, 4800, 4096, 4000, 4, 2048, 0, False),  # k = 2048, visible counts crossing k
 ])
 def test_indexer_topk(B, Tq, N, q_pos0, m, k, ties, zero):
     g = np.random.default_rng(B * 1000 + N + k)
