@@ -795,6 +795,127 @@ __global__ void __launch_bounds__(1024) topk_rows_kernel(RowsParams p) {
   }
 }
 
+// Short rows (at most 1024 visible entries): one warp per row, 32 consecutive
+// entries per lane in registers; the same exact radix select (four levels of
+// 8 key bits, a 256-bin histogram per warp in shared memory, the threshold
+// digit found by a warp scan over the bins from the top), then an ascending
+// emission: lane order is index order, so warp scans of the per-lane counts
+// give every selected entry its position and the ties their rank.
+constexpr int kWarpRowMaxN = 1024;
+
+__global__ void __launch_bounds__(256) topk_rows_warp_kernel(RowsParams p, int64_t R) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ uint32_t hist_all[8][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+  if (row >= R) return;  // whole warps only: nothing below synchronises the block
+  uint32_t* hist = hist_all[warp];
+  int64_t nv;
+  if (p.cu_tok != nullptr) {
+    const int sq = seq_of(p.cu_tok, p.n_seqs, row);
+    nv = visible(row - __ldg(p.cu_tok + sq), p.m, __ldg(p.cu_ent + sq + 1) - __ldg(p.cu_ent + sq));
+  } else {
+    nv = visible(p.q_pos0 + row % p.Tq, p.m, p.N);
+  }
+  const int k = p.k;
+  int32_t* out = p.idx + row * k;
+  float* sout = p.sout != nullptr ? p.sout + row * k : nullptr;
+  const float* srow = p.scores + row * p.pitch;
+  if (nv <= k || nv > kWarpRowMaxN) {
+    if (nv > k && lane == 0) atomicExch(&tc::g_device_error, kErrRowTooLong);  // the host never admits this
+    const int64_t keep = nv <= k ? nv : 0;
+    for (int j = lane; j < k; j += 32) {
+      out[j] = j < keep ? j : -1;
+      if (sout != nullptr) sout[j] = j < keep ? __ldcg(srow + j) : -INFINITY;
+    }
+    return;
+  }
+  const int n = static_cast<int>(nv), base = lane * 32;
+  uint32_t key[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) key[i] = base + i < n ? f2key(__ldcg(srow + base + i)) : 0u;
+  uint32_t prefix = 0, mask = 0, remaining = static_cast<uint32_t>(k);
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int j = lane; j < 256; j += 32) hist[j] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (base + i < n && (key[i] & mask) == prefix) atomicAdd(&hist[(key[i] >> shift) & 255u], 1u);
+    __syncwarp();
+    // lane l owns bins 255 - 8l .. 248 - 8l (descending)
+    uint32_t c[8], tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      c[j] = hist[255 - 8 * lane - j];
+      tot += c[j];
+    }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t excl = incl - tot;
+    const int owner = __ffs(__ballot_sync(0xffffffffu, excl < remaining && remaining <= incl)) - 1;
+    uint32_t digit = 0, above = 0;
+    if (lane == owner) {
+      uint32_t run = excl;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (run + c[j] >= remaining) {
+          digit = static_cast<uint32_t>(255 - 8 * lane - j);
+          above = run;
+          break;
+        }
+        run += c[j];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, owner);
+    above = __shfl_sync(0xffffffffu, above, owner);
+    prefix |= digit << shift;
+    mask |= 255u << shift;
+    remaining -= above;
+    __syncwarp();
+  }
+  // the k-th key is `prefix`: take every key above it and the `remaining`
+  // lowest-index keys equal to it
+  uint32_t gt = 0, eq = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const bool in = base + i < n;
+    gt += (in && key[i] > prefix) ? 1u : 0u;
+    eq += (in && key[i] == prefix) ? 1u : 0u;
+  }
+  uint32_t eq_incl = eq;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, eq_incl, o);
+    if (lane >= o) eq_incl += y;
+  }
+  const uint32_t eq_before = eq_incl - eq;
+  const uint32_t take_eq = remaining > eq_before ? (remaining - eq_before < eq ? remaining - eq_before : eq) : 0u;
+  const uint32_t sel = gt + take_eq;
+  uint32_t sel_incl = sel;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, sel_incl, o);
+    if (lane >= o) sel_incl += y;
+  }
+  uint32_t pos = sel_incl - sel, taken = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (base + i >= n) continue;
+    const bool pick = key[i] > prefix || (key[i] == prefix && taken++ < take_eq);
+    if (pick) {
+      out[pos] = base + i;
+      if (sout != nullptr) sout[pos] = __ldcg(srow + base + i);
+      ++pos;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // prefill rows with bf16 keys: tcgen05 scoring, scores kept on chip
 // ---------------------------------------------------------------------------
@@ -1032,7 +1153,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
         need_mask |= w ? (1u << j) : 0u;
       }
       // this thread's query state for the pass
-      const uint32_t nv_q = nv_s[qj], lv_q = level_s[qj], pre_q = prefix_s[qj];
+      const uint32_t nv_q = nv_s[qj], pre_q = prefix_s[qj];
       const uint32_t sh_q = shift_s[qj], thr_q = thr_s[qj], need_q = need_s[qj];
       const bool mine = (need_mask >> (qj - hq * 16)) & 1u;
       for (int tile = 0; tile < ntiles; ++tile, ++it) {
@@ -1623,6 +1744,9 @@ csa_status launch_row_path(const char* name, ScoreParams& p, const RowsParams& r
                        : launch_pdl(score_kernel<kRowGroup, kKeyBF16>, grid, block, score_tile_bytes(kf), s, 1, p);
   prof_end(s);
   if (csa_status st = check_launch(name, e); st != CSA_OK) return st;
+  if (max_n <= kWarpRowMaxN)  // short rows: one warp per row
+    return check_launch(name, launch_pdl(topk_rows_warp_kernel, dim3(static_cast<unsigned>((R + 7) / 8)), dim3(256),
+                                         0, s, 1, rp, R));
   const size_t smem = static_cast<size_t>(max_n) * 4;
   if (!ensure_smem(reinterpret_cast<const void*>(topk_rows_kernel), kRowPathMaxN * 4))
     return fail(CSA_ERR_CUDA, "%s: cannot raise shared memory limit", name);
