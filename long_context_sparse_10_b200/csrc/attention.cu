@@ -1287,7 +1287,8 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
   uint64_t* sdone = vfree + 2;                                     // [2 groups][2 bufs] S done
   uint64_t* pready = sdone + 4;                                    // [2 groups] P written
   uint64_t* pvdone = pready + 2;                                   // [2 groups] PV done
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(pvdone + 2);
+  uint64_t* qfull = pvdone + 2;                                    // Q landed (one arrival per thread)
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(qfull + 1);
   __shared__ int s_count[kQbThreads / 32];
   __shared__ int s_union;
 
@@ -1307,8 +1308,10 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) tc::bar_init(&kfull[i], kQbLoaders);  // kfull, vfull
     for (int i = 4; i < 16; ++i) tc::bar_init(&kfull[i], 1);
+    tc::bar_init(qfull, kQbThreads);
     tc::bar_init_fence();
   }
+  __syncthreads();  // the barriers exist before any copy arrives on one
   if (warp == 0) tc::tmem_alloc(tslot, 512);
   {  // Q rows (query, head) of both groups, swizzled K-major; rows past the block's queries are zero
     const __nv_bfloat16* qsrc = p.q + ((b * p.Tq + r0) * H) * kDQK;
@@ -1320,6 +1323,7 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
     }
   }
   cp_async_commit();
+  cp_async_mbar_arrive_noinc(qfull);  // Q is waited for by the MMA thread only
 
   // entry slots: the dense run [0, n_ent), or the union of the selections
   int64_t n_ent;
@@ -1382,10 +1386,8 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
   }
   const int64_t n_slots = n_ent + nwin;
   const int ntiles = static_cast<int>((n_slots + kQbKeys - 1) / kQbKeys);
-  cp_async_wait<0>();
-  tc::fence_async_smem();
   tc::fence_before_sync();
-  __syncthreads();  // Q, the union and the barriers are ready; the P buffers are free again
+  __syncthreads();  // the union is ready and the P buffers are free again (Q may still be landing)
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
   bool healthy = true;
@@ -1472,6 +1474,7 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
       tc::mma_commit(&kfree[st]);
     };
     if (lane == 0 && ntiles > 0) {
+      if (healthy) healthy = tc::bar_wait(qfull, 0);
       for (int tt = 0; tt < 2 && tt < ntiles; ++tt) {
         if (healthy) healthy = tc::bar_wait(&kfull[tt], 0);
         issue_s(tt);
@@ -1614,6 +1617,7 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
     if (row_ok && p.lse) p.lse[(b * p.Tq + r0) * H + r] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
   }
   pdl_trigger();
+  cp_async_wait<0>();  // (the query copies landed long before; nothing of this thread stays in flight)
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, 512);
