@@ -658,22 +658,32 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
     }
     tc::bar_init_fence();
   }
-  if (warp == 0) tc::tmem_alloc(tslot, 256);
-  for (int piece = tid; piece < 64 * 24; piece += kTcDecThreads) {  // Q, swizzled K-major
-    const int hh = piece / 24, ch = piece % 24;
-    cp_async16(Qs + (ch >> 3) * 8192 + tc::sw128(hh, ch & 7), p.q + (row * 64 + hh) * kDQK + ch * 8);
+  __syncthreads();  // the barriers exist
+  // FP8 cache (decode: a few tiles per CTA): the consumers (softmax warps 0-7
+  // and the MMA warp 16) set up TMEM, Q and the running maxima while the
+  // producer gathers the first tiles.  bf16 cache (long prefill rows): every
+  // thread loads Q first (measured faster there).
+  const bool consumer = !FP8 || warp < 8 || warp == 16;
+  if (consumer) {
+    const int nct = FP8 ? 288 : kTcDecThreads;
+    const int ct = !FP8 ? tid : (warp < 8 ? tid : 256 + lane);
+    if (warp == 0) tc::tmem_alloc(tslot, 256);
+    for (int piece = ct; piece < 64 * 24; piece += nct) {  // Q, swizzled K-major
+      const int hh = piece / 24, ch = piece % 24;
+      cp_async16(Qs + (ch >> 3) * 8192 + tc::sw128(hh, ch & 7), p.q + (row * 64 + hh) * kDQK + ch * 8);
+    }
+    cp_async_commit();
+    if (tid < 64) {
+      reinterpret_cast<uint4*>(ones)[tid] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+      mref[tid] = -INFINITY;
+    }
+    cp_async_wait<0>();
+    tc::fence_async_smem();
+    tc::fence_before_sync();
+    named_sync(5, nct);
+    tc::fence_after_sync();
   }
-  cp_async_commit();
-  if (tid < 64) {
-    reinterpret_cast<uint4*>(ones)[tid] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-    mref[tid] = -INFINITY;
-  }
-  cp_async_wait<0>();
-  tc::fence_async_smem();
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = *tslot;
+  const uint32_t tmem = consumer ? *tslot : 0u;
   bool healthy = true;  // false after a barrier wait ran out: later waits are skipped
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const uint32_t tO = tmem + 128, tL = tmem + 192;
