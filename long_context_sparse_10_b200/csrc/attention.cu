@@ -1647,15 +1647,10 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict
   const int hh = static_cast<int>(rh % H);
   const float* rec0 = part + (row * nsplit * H + hh) * kRec;
   const int64_t cstride = static_cast<int64_t>(H) * kRec;
-  // the splits' maxima, one split per lane, then a warp max
-  float M = -INFINITY;
-  for (int c = lane; c < nsplit; c += 32) M = fmaxf(M, __ldg(rec0 + c * cstride + kDV));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float bse = M == -INFINITY ? 0.f : M;
-  // weighted sums, 16 split records in flight per lane
-  constexpr int kBatch = 16;
-  float Lsum = 0.f;
+  // batches of up to 24 split records, all of a batch's loads in flight at
+  // once (one batch for up to 24 splits), merged online across batches
+  constexpr int kBatch = 24;
+  float M = -INFINITY, Lsum = 0.f;
   float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int c0 = 0; c0 < nsplit; c0 += kBatch) {
     float2 ml[kBatch];
@@ -1667,6 +1662,20 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict
       ml[j] = ok ? __ldg(reinterpret_cast<const float2*>(r + kDV)) : make_float2(-INFINITY, 0.f);
       u[j] = ok ? __ldg(reinterpret_cast<const float4*>(r) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    float mb = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) mb = fmaxf(mb, ml[j].x);
+    const float mn = fmaxf(M, mb);
+    if (mn != -INFINITY && M != mn) {  // rescale what earlier batches summed
+      const float f = M == -INFINITY ? 0.f : exp2f(M - mn);
+      Lsum *= f;
+      a.x *= f;
+      a.y *= f;
+      a.z *= f;
+      a.w *= f;
+      M = mn;
+    }
+    const float bse = M == -INFINITY ? 0.f : M;
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       const float w = exp2f(ml[j].x - bse);
