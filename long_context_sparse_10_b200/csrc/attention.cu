@@ -514,7 +514,6 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
 // ---------------------------------------------------------------------------
 constexpr int kTcKeys = 128;
 
-constexpr int kTcThreads = 256;     // query-blocked prefill kernel: warps 0-3 softmax + MMA, 4-7 loads
 constexpr int kTcDecThreads = 544;  // attn_tc_kernel: warps 0-7 softmax, 8-15 loads, 16 MMA issue
 constexpr float kRescaleLog2 = 20.f;  // rescale O and l when a logit tops m_ref by more than 2^20
 
@@ -1961,7 +1960,7 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
         pl.cl = pl.cl > 8 ? 8 : pl.cl;  // portable cluster sizes only
       }
     }
-    const int cl = choose_cluster(fn, pl.cl, R, smem, use_tc ? kTcThreads : kThreads);
+    const int cl = choose_cluster(fn, pl.cl, R, smem, kThreads);
     if (cl != pl.cl) {  // re-plan with the co-schedulable cluster size
       const int64_t tiles = max_slots > 0 ? (max_slots + tile_keys - 1) / tile_keys : 1;
       pl.tps = static_cast<int>((tiles + cl - 1) / cl);
