@@ -6,7 +6,10 @@ import os
 import threading
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libcsa.so")
+# CSA_LIBRARY selects another build of the same ABI (e.g. libcsa_checked.so,
+# whose kernels bounds-check their gathers); by default the library next to
+# this file.
+LIB_PATH = os.environ.get("CSA_LIBRARY") or os.path.join(_HERE, "libcsa.so")
 
 c_i32, c_i64, c_f32, c_sz, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
 

@@ -1,10 +1,13 @@
 """Builds libcsa.so (all CUDA sources under csrc/) for sm_100a with nvcc.
 
-Usage: python -m long_context_sparse_10_b200.build [-v]
+Usage: python -m long_context_sparse_10_b200.build [-v] [-f] [--checked]
 
 Objects go to <repo>/_build/ and the shared library next to this file, so it
 travels with the source tree.  A source is recompiled when it or any header is
-newer than its object.
+newer than its object.  `--checked` builds libcsa_checked.so (objects in
+_build/checked/) with -DCSA_CHECKED: the kernels bounds-check their gather rows
+and record a failed check in the device error word that
+csa_check_device_error reports (load it with CSA_LIBRARY=<path>).
 """
 from __future__ import annotations
 
@@ -21,6 +24,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libcsa.so")
+LIB_CHECKED = os.path.join(PKG, "libcsa_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -40,15 +44,18 @@ def _newest_header() -> float:
     return max((os.path.getmtime(h) for h in hs), default=0.0)
 
 
-def build(verbose: bool = False, force: bool = False, extra_flags: list[str] | None = None) -> str:
+def build(verbose: bool = False, force: bool = False, extra_flags: list[str] | None = None,
+          checked: bool = False) -> str:
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    out_dir = os.path.join(BUILD, "checked") if checked else BUILD
+    lib = LIB_CHECKED if checked else LIB
+    os.makedirs(out_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_t = _newest_header()
-    flags = FLAGS + (extra_flags or [])
+    flags = FLAGS + (["-DCSA_CHECKED"] if checked else []) + (extra_flags or [])
 
     def compile_one(src: str) -> str:
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(out_dir, os.path.basename(src) + ".o")
         if (not force and os.path.exists(obj) and os.path.getmtime(obj) >= os.path.getmtime(src)
                 and os.path.getmtime(obj) >= hdr_t):
             return obj
@@ -64,17 +71,17 @@ def build(verbose: bool = False, force: bool = False, extra_flags: list[str] | N
 
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    if force or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [nvcc, *ARCH, "-shared", "-o", LIB + ".tmp", *objs]
+    if force or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        cmd = [nvcc, *ARCH, "-shared", "-o", lib + ".tmp", *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(LIB + ".tmp", LIB)
-    return LIB
+        os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
     v = "-v" in sys.argv
-    print(build(verbose=v, force="-f" in sys.argv))
+    print(build(verbose=v, force="-f" in sys.argv, checked="--checked" in sys.argv))

@@ -85,7 +85,16 @@ struct AttnParams {
   const int32_t* cu_tok;
   const int32_t* cu_ent;
   int n_seqs;
+  // rows of the cache planes and of the raw-token buffer (bounds of the
+  // gathers, checked in builds with CSA_CHECKED)
+  int64_t ent_rows, win_rows;
 };
+
+#ifdef CSA_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
 
 // Where one query row's keys live: its position t, the cache row of its entry
 // 0 (ebase) and its entry count N, and the raw-buffer row of position 0 (wbase).
@@ -227,6 +236,7 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(AttnParams p) {
         r = geo.wbase + (wlo + (s - n_ent));
       }
     }
+    if (type != 0 && !CSA_INBOUNDS(r >= 0 && r < (type == 1 ? p.ent_rows : p.win_rows))) type = 0;
     stype[st][tid] = type;
     srow[st][tid] = r;
   };
@@ -788,7 +798,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         const int ring = tile & (kTypeRing - 1);
         int ne, nw;
         runs(tile, ne, nw);
-        if (ne > 0 && dense) {  // contiguous entry rows
+        if (ne > 0 && dense && !kChecked) {  // contiguous entry rows
           const int64_t r0 = srow[ring][0];
           for (int pc = pt; pc < ne * nch; pc += 256) {
             const int key = pc / nch, c = pc % nch;
@@ -808,9 +818,11 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         }
         if (nw > 0) {  // raw window tokens: contiguous rows
           const int64_t rw0 = srow[ring][ne];
+          const bool inb = CSA_INBOUNDS(rw0 >= 0 && rw0 + nw <= p.win_rows);
           for (int pc = pt; pc < nw * nch; pc += 256) {
             const int key = ne + pc / nch, c = pc % nch;
-            cp_async16(T + (c >> 3) * kKB + tc::sw128(key, c & 7), wsrc + (rw0 + pc / nch) * wstride + c * 8);
+            cp_async16(T + (c >> 3) * kKB + tc::sw128(key, c & 7),
+                       inb ? wsrc + (rw0 + pc / nch) * wstride + c * 8 : p.q, inb ? 16 : 0);
           }
         }
         for (int pc = pt; pc < (kTcKeys - ne - nw) * nch; pc += 256) {  // past the row's end: zero rows
@@ -844,6 +856,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
                 r = geo.wbase + (wlo + (sl - n_ent));
               }
             }
+            if (type != 0 && !CSA_INBOUNDS(r >= 0 && r < (type == 1 ? p.ent_rows : p.win_rows))) type = 0;
             stype[ring][pt] = type;
             srow[ring][pt] = r;
           }
@@ -900,6 +913,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
               r = geo.wbase + (wlo + (sl - n_ent));
             }
           }
+          if (type != 0 && !CSA_INBOUNDS(r >= 0 && r < (type == 1 ? p.ent_rows : p.win_rows))) type = 0;
           stype[tile & (kTypeRing - 1)][pt] = type;
           srow[st][pt] = r;
         }
@@ -931,7 +945,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         // Contiguous runs are copied with consecutive lanes on consecutive 16-byte
         // chunks (512-byte warp requests); selected entries are gathered four keys
         // per warp instruction (8 lanes per 128-byte row).
-        if (ne > 0 && dense) {
+        if (ne > 0 && dense && !kChecked) {
           const int64_t r0 = srow[st][0];
           if (FP8) {
             for (int pc = pt; pc < ne * 8; pc += 256)
@@ -976,9 +990,11 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
         }
         if (nw > 0) {  // raw window tokens: contiguous rows
           const int64_t rw0 = srow[st][ne];
+          const bool inb = CSA_INBOUNDS(rw0 >= 0 && rw0 + nw <= p.win_rows);
           for (int pc = pt; pc < nw * 24; pc += 256) {
             const int key = ne + pc / 24, c = pc % 24;
-            cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), p.wk + rw0 * kDQK + pc * 8);
+            cp_async16(Kt + (c >> 3) * kKB + tc::sw128(key, c & 7), inb ? p.wk + rw0 * kDQK + pc * 8 : p.q,
+                       inb ? 16 : 0);
           }
           if (!SHV) {
             for (int pc = pt; pc < nw * 16; pc += 256) {
@@ -1419,10 +1435,10 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
         const __nv_bfloat16* src = nullptr;
         if (sl < n_ent) {
           const int64_t e = ebase + (sparse ? static_cast<int64_t>(ulist[sl]) : sl);
-          src = is_k ? p.ck + e * kDQK : ve + e * ves;
+          if (CSA_INBOUNDS(e >= 0 && e < p.ent_rows)) src = is_k ? p.ck + e * kDQK : ve + e * ves;
         } else if (sl < n_slots) {
           const int64_t w = wbase + (sl - n_ent);
-          src = is_k ? p.wk + w * kDQK : vw + w * vws;
+          if (CSA_INBOUNDS(w >= 0 && w < p.win_rows)) src = is_k ? p.wk + w * kDQK : vw + w * vws;
         }
         uint8_t* dst = T + tc::sw128(key, c8);
         const __nv_bfloat16* s8 = src != nullptr ? src + c8 * 8 : p.q;
@@ -2015,6 +2031,8 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   p.cu_tok = pk ? pk->cu_tokens : nullptr;
   p.cu_ent = pk ? pk->cu_entries : nullptr;
   p.n_seqs = pk ? pk->n_seqs : 0;
+  p.ent_rows = pk ? N : B * N;
+  p.win_rows = wlen > 0 ? (pk ? pk->total_tokens : B * win->rows) : 0;
 
   const dim3 grid(static_cast<unsigned>(use_blk ? B * ((Tq + qb_rows - 1) / qb_rows) : R * pl.cl));
   const dim3 block(use_blk ? kQbThreads : (use_tc ? kTcDecThreads : kThreads));
@@ -2041,15 +2059,19 @@ csa_status csa_check_device_error(void* stream) {
   int word = 0;
   e = cudaMemcpyFromSymbol(&word, csa::tc::g_device_error, sizeof(int));
   if (e != cudaSuccess) return csa::fail(CSA_ERR_CUDA, "csa_check_device_error: %s", cudaGetErrorString(e));
-  const int iword = csa::indexer_device_error(true);
-  if (iword < 0) return csa::fail(CSA_ERR_CUDA, "csa_check_device_error: cannot read the indexer error word");
-  word |= iword;
+  for (int (*reader)(bool) : {csa::indexer_device_error, csa::compress_device_error, csa::out_proj_device_error,
+                               csa::cp_merge_device_error}) {
+    const int uword = reader(true);
+    if (uword < 0) return csa::fail(CSA_ERR_CUDA, "csa_check_device_error: cannot read a unit's error word");
+    word |= uword;
+  }
   if (word != 0) {
     const int zero = 0;
     cudaMemcpyToSymbol(csa::tc::g_device_error, &zero, sizeof(int));
     return csa::fail(CSA_ERR_DEVICE_TIMEOUT, "a kernel gave up waiting on a barrier, or skipped work it could "
-                     "not do in bounds (code %d: 1 = a bounded wait ran out, 2 = a row longer than the row path "
-                     "holds); its outputs are not valid", word);
+                     "not do in bounds (code bits %d: 1 = a bounded wait ran out, 2 = a row longer than the row "
+                     "path holds, 4 = a checked build found an access out of bounds); its outputs are not valid",
+                     word);
   }
   return CSA_OK;
 }

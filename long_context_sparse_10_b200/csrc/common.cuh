@@ -155,6 +155,43 @@ __device__ __forceinline__ int seq_of(const int32_t* cu, int n, int64_t v) {
   return lo;
 }
 
+namespace tc {
+// Error word of the translation unit that includes this header: set when a
+// bounded wait gives up (the kernel then finishes without trusting its data
+// instead of hanging), or when a checked build finds an access out of bounds.
+// Read back by the unit's device_error reader (CSA_DEFINE_DEVICE_ERROR_READER)
+// and reported by csa_check_device_error.
+static __device__ int g_device_error;
+constexpr int kErrWaitTimeout = 1;
+constexpr int kErrBounds = 4;
+}  // namespace tc
+
+// Checked builds (compiled with -DCSA_CHECKED): CSA_INBOUNDS(cond) records
+// kErrBounds in the unit's error word when `cond` is false, and the access it
+// guards is skipped.  In the normal build it is `true` and costs nothing.
+__device__ __forceinline__ bool checked_ok(bool cond) {
+  if (!cond) atomicOr(&tc::g_device_error, tc::kErrBounds);
+  return cond;
+}
+#ifdef CSA_CHECKED
+#define CSA_INBOUNDS(cond) (::csa::checked_ok(cond))
+#else
+#define CSA_INBOUNDS(cond) (true)
+#endif
+
+// Host reader of this unit's error word (defined once per .cu file).
+#define CSA_DEFINE_DEVICE_ERROR_READER(fn)                                              \
+  int fn(bool clear) {                                                                  \
+    int word = 0;                                                                       \
+    if (cudaMemcpyFromSymbol(&word, tc::g_device_error, sizeof(int)) != cudaSuccess)    \
+      return -1;                                                                        \
+    if (word && clear) {                                                                \
+      const int zero = 0;                                                               \
+      cudaMemcpyToSymbol(tc::g_device_error, &zero, sizeof(int));                       \
+    }                                                                                   \
+    return word;                                                                        \
+  }
+
 __device__ __forceinline__ uint4 ldg_nc16(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];\n"

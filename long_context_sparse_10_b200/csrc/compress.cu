@@ -49,6 +49,13 @@ struct EntryRef {
   int64_t out_row, i, T;
   const __nv_bfloat16* x0;
 };
+
+// True when position j of the entry's sequence is a row of the raw buffer
+// (checked builds only; the host validates the buffer's coverage).
+__device__ __forceinline__ bool x_row_ok(const CompressParams& p, const EntryRef& er, int64_t j) {
+  const int64_t row = (er.x0 - p.x) / p.d + j;
+  return CSA_INBOUNDS(row >= 0 && row < p.B * p.xrows);
+}
 __device__ __forceinline__ EntryRef entry_ref(const CompressParams& p, int64_t e) {
   EntryRef r;
   if (p.cu_tok != nullptr) {
@@ -181,6 +188,7 @@ __global__ void __launch_bounds__(256) compress_short_kernel(CompressParams p) {
     const __nv_bfloat16* xb = er.x0 + 8 * lane;
     for (int64_t j = j0; j < j1; ++j) {
       float xv[8], bv[8];
+      if (!x_row_ok(p, er, j)) continue;
       unpack8(ldg_nc16(xb + j * p.d), xv);
       load8f(p.b + (j - start) * p.d + 8 * lane, bv);
       acc.add(xv, wv, bv);
@@ -212,7 +220,7 @@ __global__ void __launch_bounds__(256) compress_flat_kernel(CompressParams p) {
 #pragma unroll
   for (int r = 0; r < CW; ++r) {
     const int64_t j = start + r;
-    raw[r] = (j >= 0 && j < er.T) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
+    raw[r] = (j >= 0 && j < er.T && x_row_ok(p, er, j)) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
   }
   // logits of every row kept in registers (rows outside the sequence take no
   // part: -inf), the per-channel maximum, then one exponential per element
@@ -277,7 +285,7 @@ __global__ void __launch_bounds__(512) compress_wide_kernel(CompressParams p) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int64_t j = start + rs + 16 * i;
-    raw[i] = (j >= 0 && j < er.T) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
+    raw[i] = (j >= 0 && j < er.T && x_row_ok(p, er, j)) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
   }
   float lg[8][8], mx[8];
 #pragma unroll
@@ -371,7 +379,7 @@ __global__ void __launch_bounds__(256) compress_long_kernel(CompressParams p) {
 #pragma unroll
       for (int i = 0; i < RPW; ++i) {  // rows start + warp + 8 i, all loads in flight together
         const int64_t j = start + warp + 8 * i;
-        raw[i] = (j >= j0 && j < j1) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
+        raw[i] = (j >= j0 && j < j1 && x_row_ok(p, er, j)) ? ldg_nc16(xb + j * p.d) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int i = 0; i < RPW; ++i) {
@@ -401,6 +409,7 @@ __global__ void __launch_bounds__(256) compress_long_kernel(CompressParams p) {
 #pragma unroll 4
       for (int64_t j = j0 + warp; j < j1; j += 8) {
         float xv[8], bv[8];
+        if (!x_row_ok(p, er, j)) continue;
         unpack8(ldg_nc16(xb + j * p.d), xv);
         load8f(p.b + (j - start) * p.d + 8 * lane, bv);
         acc.add(xv, wv, bv);
@@ -589,6 +598,11 @@ csa_status hca_compress(const void* x, int64_t B, int64_t T, int32_t d, int32_t 
 }
 
 }  // extern "C"
+
+namespace csa {
+// Reads (and optionally clears) this unit's device error word.
+CSA_DEFINE_DEVICE_ERROR_READER(compress_device_error)
+}  // namespace csa
 
 extern "C" {
 

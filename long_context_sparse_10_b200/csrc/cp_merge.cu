@@ -174,6 +174,11 @@ __global__ void __launch_bounds__(256) attn_partial_merge_kernel(const __nv_bflo
 }  // namespace
 }  // namespace csa
 
+namespace csa {
+// Reads (and optionally clears) this unit's device error word.
+CSA_DEFINE_DEVICE_ERROR_READER(cp_merge_device_error)
+}  // namespace csa
+
 extern "C" {
 
 csa_status csa_cp_topk_merge(const float* cand_scores, const int32_t* cand_idx, int64_t R, int32_t n_cand, int32_t k,

@@ -10,6 +10,13 @@
 
 namespace csa {
 
+// Device error words of the units (attention.cu reads its own): -1 when the
+// word cannot be read; `clear` resets a non-zero word.
+int indexer_device_error(bool clear);
+int compress_device_error(bool clear);
+int out_proj_device_error(bool clear);
+int cp_merge_device_error(bool clear);
+
 // Records a printf-style message for csa_last_error() and returns `s`.
 csa_status fail(csa_status s, const char* fmt, ...);
 // Clears the calling thread's message.
@@ -58,8 +65,6 @@ int num_sms();
 // Raises a kernel's dynamic shared memory limit to `bytes` on the current
 // device (once per device and kernel).  Returns false if the runtime refuses.
 bool ensure_smem(const void* kernel, int bytes);
-// The indexer unit's device error word (bounded barrier waits); -1 if unreadable.
-int indexer_device_error(bool clear);
 // Records the pending csa_profile_next_call start/stop event (if any) on `s`.
 void prof_begin(cudaStream_t s);
 void prof_end(cudaStream_t s);

@@ -1693,15 +1693,7 @@ size_t workspace_bytes(int64_t B, int64_t Tq, int64_t N, bool coded = false) {
 
 namespace csa {
 // Reads (and optionally clears) this unit's device error word.
-int indexer_device_error(bool clear) {
-  int word = 0;
-  if (cudaMemcpyFromSymbol(&word, tc::g_device_error, sizeof(int)) != cudaSuccess) return -1;
-  if (word && clear) {
-    const int zero = 0;
-    cudaMemcpyToSymbol(tc::g_device_error, &zero, sizeof(int));
-  }
-  return word;
-}
+CSA_DEFINE_DEVICE_ERROR_READER(indexer_device_error)
 }  // namespace csa
 
 extern "C" {

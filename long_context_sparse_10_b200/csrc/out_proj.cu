@@ -243,3 +243,9 @@ extern "C" csa_status csa_grouped_out_proj(const void* o, int64_t R, int32_t H, 
   if (bn == 128) return launch_out_proj<128>(p, amap, bmap, s);
   return launch_out_proj<64>(p, amap, bmap, s);
 }
+
+namespace csa {
+// Reads (and optionally clears) this unit's device error word.
+CSA_DEFINE_DEVICE_ERROR_READER(out_proj_device_error)
+}  // namespace csa
+

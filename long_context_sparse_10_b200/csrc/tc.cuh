@@ -9,12 +9,6 @@
 namespace csa {
 namespace tc {
 
-// Error word of the translation unit that includes this header: set when a
-// bounded wait gives up (the kernel then finishes without trusting its data
-// instead of hanging).  Read back with cudaMemcpyFromSymbol in that unit.
-static __device__ int g_device_error;
-
-constexpr int kErrWaitTimeout = 1;
 constexpr uint32_t kWaitLimit = 1u << 22;  // try_wait rounds before giving up
 
 // Shared-memory matrix descriptor, 128-byte swizzle (the layout a TMA

@@ -117,3 +117,16 @@ def test_attention_workspace_rule(lib):
     assert lib.csa_sparse_mqa_workspace_size(1, sms, 64, 2048, 128) == 0
     assert lib.csa_sparse_mqa_workspace_size(4, 1, 64, 100, 0) == 0
     assert lib.csa_sparse_mqa_workspace_size(0, 1, 64, 100, 0) == 0
+
+
+def test_checked_build_exports_the_same_abi():
+    # libcsa_checked.so (-DCSA_CHECKED: bounds checks on the gather rows) is a drop-in
+    # replacement selected with CSA_LIBRARY; it must export exactly the declared calls too
+    from long_context_sparse_10_b200 import build
+    path = build.LIB_CHECKED
+    if not os.path.exists(path):
+        build.build(checked=True)
+    checked = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(checked, n), n
+    assert b"sm_100a" in ctypes.CFUNCTYPE(ctypes.c_char_p)(("csa_version", checked))()
