@@ -244,6 +244,7 @@ class DecodeRun:
         self.lse = torch.empty(B, 1, H, dtype=torch.float32, device=dev)
         self.hybrid = wl.kind == "hybrid"
         if self.hybrid:
+            self.side = torch.cuda.Stream(device=dev)  # the HCA branch's stream
             self.hcache = csa.KVCache(nope=d["hca_nope"], rope=d["hca_rope"], scale=d["hca_scale"])
             self.hwin = csa.Window(k=d["hca_win_k"], pos0=L - wl.win, length=wl.win)
             hws = csa.hca_dense_mqa_workspace_size(B, 1, H, wl.N_hca, wl.win)
@@ -289,13 +290,22 @@ class DecodeRun:
                                       idx=self.idx, workspace=self.ws_idx)
 
     def step(self):
-        wl, csa = self.wl, self.csa
+        """One decode step.  The HCA branch does not depend on the CSA branch's indexer, so it runs on a second
+        stream forked from (and joined back into) the caller's: its latency-bound kernels fill the SMs that the
+        top-k tail and the CSA attention leave idle."""
+        wl, csa, torch = self.wl, self.csa, self.torch
+        main = torch.cuda.current_stream()
+        if self.hybrid:
+            self.side.wait_stream(main)
         self.indexer()
+        if self.hybrid:
+            with torch.cuda.stream(self.side):
+                csa.hca_dense_mqa(self.d["hca_q"], self.hcache, wl.m_hca, self.hwin, self.scale, q_pos0=self.q_pos0,
+                                  out=self.hout, lse=self.hlse, workspace=self.ws_hca)
         csa.csa_sparse_mqa(self.d["q"], self.cache, wl.m, self.idx, self.win, self.scale, q_pos0=self.q_pos0,
                            out=self.out, lse=self.lse, workspace=self.ws_attn)
         if self.hybrid:
-            csa.hca_dense_mqa(self.d["hca_q"], self.hcache, wl.m_hca, self.hwin, self.scale, q_pos0=self.q_pos0,
-                              out=self.hout, lse=self.hlse, workspace=self.ws_hca)
+            main.wait_stream(self.side)
 
     def parts(self):
         """The step's library calls, separately (for --breakdown)."""

@@ -103,6 +103,8 @@ def _indexer_case(g, B, Tq, N, tie_blocks=0, zero_q=False):
     (1, 40, 300, 0, 4, 8, 0, False),           # long-row path; the first rows see no entry at all
     (1, 1, 40000, 4 * 40000 - 1, 4, 4096, 0, True),   # long rows, all ties, k = max
     (2, 1, 300001, 4 * 300001 - 1, 4, 2048, 0, False),  # rows past 262144 entries: bitmap in global memory
+    (1, 600, 40000, 120000, 4, 512, 0, False),  # more long rows than CTA slots: one chunk per row
+    (64, 1, 32768, 4 * 32768 - 1, 4, 2048, 0, False),  # 64 decode rows at 131072 tokens of context
     # prefill rows at k = 2048 (row path): visible counts crossing k, and near 16384
     (1, 300, 16384, 8000, 4, 2048, 0, False),
     (1, 300, 16384, 65536 - 300, 4, 2048, 0, False),
