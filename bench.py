@@ -553,6 +553,60 @@ class PrefillRun:
         return (sum(v.numel() * v.element_size() for v in self.h_in.values()),
                 sum(v.numel() * v.element_size() for v in self.h_out))
 
+    def _bind(self, st):
+        for k_, v in st["ins"].items():
+            self.d[k_] = v
+        self.out = st["out"]
+
+    def e2e_pipeline(self, n):
+        """Capture n end-to-end steps into one CUDA graph over two buffer sets: while step i computes on set
+        i % 2, one copy stream brings step i+1's inputs in from pinned host memory and another takes step i-1's
+        output out (the two directions of the link overlap).  Returns the graph."""
+        torch = self.torch
+        sets = [dict(ins={k_: self.d[k_] for k_ in self.h_in}, out=self.out, h_in=self.h_in, h_out=self.h_out[0]),
+                dict(ins={k_: torch.empty_like(self.d[k_]) for k_ in self.h_in}, out=torch.empty_like(self.out),
+                     h_in={k_: torch.empty_like(v).pin_memory().copy_(v) for k_, v in self.h_in.items()},
+                     h_out=torch.empty_like(self.h_out[0]).pin_memory())]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_done = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+
+        def copy_in(st):
+            for k_, v in st["h_in"].items():
+                st["ins"][k_].copy_(v, non_blocking=True)
+
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            main = torch.cuda.current_stream()
+            s_in.wait_stream(main)
+            s_out.wait_stream(main)
+            with torch.cuda.stream(s_in):
+                copy_in(sets[0])
+                ev_in[0].record(s_in)
+            for i in range(n):
+                cur = sets[i % 2]
+                main.wait_event(ev_in[i])
+                if i >= 2:
+                    main.wait_event(ev_out[i - 2])  # this set's previous output is on the host
+                self._bind(cur)
+                self.step()
+                ev_done[i].record(main)
+                if i + 1 < n:
+                    with torch.cuda.stream(s_in):
+                        if i >= 1:
+                            s_in.wait_event(ev_done[i - 1])  # the next set's last reader has finished
+                        copy_in(sets[(i + 1) % 2])
+                        ev_in[i + 1].record(s_in)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_done[i])
+                    cur["h_out"].copy_(cur["out"], non_blocking=True)
+                    ev_out[i].record(s_out)
+            main.wait_stream(s_in)
+            main.wait_stream(s_out)
+        self._bind(sets[0])
+        return g
+
     def attn_flops(self):
         wl = self.wl
         t = __import__("numpy").arange(wl.T)
@@ -976,7 +1030,7 @@ def main():
 
     # end to end through the public API: every step copies its inputs from pinned host memory, runs the
     # library calls and copies the outputs back; the sequence is captured once in a CUDA graph (as a
-    # serving loop would, decode steps double-buffered so one step's copies overlap the other's compute)
+    # serving loop would, steps double-buffered so one step's copies overlap the other's compute)
     # and replayed, so the copies sit inside the timed region of every step
     e2e = None
     if not args.no_e2e:
