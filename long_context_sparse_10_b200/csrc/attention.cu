@@ -88,6 +88,7 @@ struct AttnParams {
   // rows of the cache planes and of the raw-token buffer (bounds of the
   // gathers, checked in builds with CSA_CHECKED)
   int64_t ent_rows, win_rows;
+  int64_t qb_blocks;  // query-blocked kernel: B * ceil(Tq / (256 / H)) blocks
 };
 
 #ifdef CSA_CHECKED
@@ -1280,7 +1281,7 @@ __host__ __device__ inline QbLayout qb_layout() {
   L.p = off; off += 2 * 16384;          // P: 2 groups x 128 rows x 64 keys (prologue: entry bit set)
   L.ulist = off; off += kQbMaxCand * 2; // union entries (uint16)
   L.qbits = off; off += 16 * kQbMaxCand / 8;  // per query: bit u = it selected union entry u
-  L.bars = off; off += 256;              // 16 mbarriers + the TMEM address
+  L.bars = off; off += 256;              // 19 mbarriers + the TMEM address
   L.total = off + 1024;
   return L;
 }
@@ -1294,7 +1295,39 @@ __device__ __forceinline__ uint64_t range_bits(int lo, int hi, int sb) {
   return upto & ~((1ull << a) - 1ull);
 }
 
-__global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p) {
+// Geometry of one query block.
+struct QbBlock {
+  int64_t b, r0, t0, tl, wlo0, nwin;
+  int nq;
+};
+__device__ __forceinline__ QbBlock qb_block(const AttnParams& p, int64_t blk) {
+  const int QB = 256 / p.H;
+  const int64_t nblk = (p.Tq + QB - 1) / QB;
+  QbBlock k;
+  k.b = blk / nblk;
+  k.r0 = (blk % nblk) * QB;  // first query row of the block within its sequence
+  k.nq = static_cast<int>((p.Tq - k.r0) < QB ? (p.Tq - k.r0) : QB);
+  k.t0 = p.q_pos0 + k.r0;
+  k.tl = k.t0 + k.nq - 1;
+  k.wlo0 = (k.t0 - p.wlen + 1) > 0 ? (k.t0 - p.wlen + 1) : 0;
+  k.nwin = p.wlen > 0 ? (k.tl - k.wlo0 + 1) : 0;
+  return k;
+}
+// Dense entry run of a block: the entries visible to its last query.
+__device__ __forceinline__ int64_t qb_dense_entries(const AttnParams& p, const QbBlock& k) {
+  const int64_t n = (k.tl + 1) / p.stride;
+  return n < p.N ? n : p.N;
+}
+
+// Dense blocks run persistently: CTA c takes blocks c, c + gridDim.x, ...,
+// and its pipeline carries over from one block to the next (the copies of the
+// next block's key tiles start as soon as stages free up, its queries as soon
+// as the last S of the current block is done, and its first S while the
+// current block's last tile drains).  Stage and TMEM-buffer parities follow
+// a tile counter that runs across the CTA's blocks.  Sparse blocks (which
+// build their union with whole-CTA barriers) run one block per CTA.
+__global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p,
+                                                                    const __grid_constant__ CUtensorMap qmap) {
   pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -1312,60 +1345,56 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
   uint64_t* sdone = vfree + 2;                                     // [2 groups][2 bufs] S done
   uint64_t* pready = sdone + 4;                                    // [2 groups] P written
   uint64_t* pvdone = pready + 2;                                   // [2 groups] PV done
-  uint64_t* qfull = pvdone + 2;                                    // Q landed (one arrival per thread)
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(qfull + 1);
+  uint64_t* qfull = pvdone + 2;                                    // the block's queries landed
+  uint64_t* qfree = qfull + 1;                                     // the block's last S done (Q may be replaced)
+  uint64_t* ofree = qfree + 1;                                     // [2 groups] O read out by the epilogue
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(ofree + 2);
   __shared__ int s_count[kQbThreads / 32];
   __shared__ int s_union;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = p.H;
-  const int QB = 256 / H;
-  const int64_t nblk = (p.Tq + QB - 1) / QB;
-  const int64_t b = blockIdx.x / nblk;
-  const int64_t qb = blockIdx.x % nblk;
-  const int64_t r0 = qb * QB;  // first query row of the block within its sequence
-  const int nq = static_cast<int>((p.Tq - r0) < QB ? (p.Tq - r0) : QB);
-  const int64_t t0 = p.q_pos0 + r0, tl = t0 + nq - 1;
   const bool sparse = p.idx != nullptr;
-  const int64_t wlo0 = (t0 - p.wlen + 1) > 0 ? (t0 - p.wlen + 1) : 0;
-  const int64_t nwin = p.wlen > 0 ? (tl - wlo0 + 1) : 0;
+  const int64_t nblocks = p.qb_blocks;
 
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) tc::bar_init(&kfull[i], kQbLoaders);  // kfull, vfull
     for (int i = 4; i < 16; ++i) tc::bar_init(&kfull[i], 1);
-    tc::bar_init(qfull, kQbThreads);
+    tc::bar_init(qfull, 1);
+    tc::bar_init(qfree, 1);
+    tc::bar_init(&ofree[0], 1);
+    tc::bar_init(&ofree[1], 1);
     tc::bar_init_fence();
   }
   __syncthreads();  // the barriers exist before any copy arrives on one
   if (warp == 0) tc::tmem_alloc(tslot, 512);
-  {  // Q rows (query, head) of both groups, swizzled K-major; rows past the block's queries are zero
-    const __nv_bfloat16* qsrc = p.q + ((b * p.Tq + r0) * H) * kDQK;
-    const int valid_rows = nq * H;
-    for (int piece = tid; piece < 256 * 24; piece += kQbThreads) {
-      const int r = piece / 24, ch = piece % 24;
-      cp_async16(Qs + (r >> 7) * 49152 + (ch >> 3) * 16384 + tc::sw128(r & 127, ch & 7),
-                 r < valid_rows ? qsrc + piece * 8 : p.q, r < valid_rows ? 16 : 0);
-    }
-  }
-  cp_async_commit();
-  cp_async_mbar_arrive_noinc(qfull);  // Q is waited for by the MMA thread only
 
-  // entry slots: the dense run [0, n_ent), or the union of the selections
-  int64_t n_ent;
-  if (!sparse) {
-    n_ent = (tl + 1) / p.stride;
-    if (n_ent > p.N) n_ent = p.N;
-  } else {
+  // queries of a block (one thread): rows (query, head) of both groups, six
+  // TMA boxes of 128 rows x 64 dims in the 128-byte swizzle (the [B][Tq*H][192]
+  // tensor map zero-fills the rows past the sequence's last query)
+  auto load_q = [&](const QbBlock& k) {
+    tc::bar_arrive_expect_tx(qfull, 6 * 16384);
+    const int y0 = static_cast<int>(k.r0 * H);
+    for (int g = 0; g < 2; ++g)
+      for (int cb = 0; cb < 3; ++cb)
+        tc::tma_load_3d(Qs + g * 49152 + cb * 16384, &qmap, 64 * cb, y0 + 128 * g, static_cast<int>(k.b), qfull);
+  };
+
+  // sparse: the union of the block's selections (one block per CTA)
+  int64_t n_ent_sparse = 0;
+  if (sparse) {
+    const QbBlock k = qb_block(p, blockIdx.x);
+    if (tid == 8 * 32) load_q(k);  // waited for by the MMA thread only
     // per-entry bit set of the block's queries that selected it (16 bits per entry, in the P buffers)
     uint32_t* bits = reinterpret_cast<uint32_t*>(Pst);
     const int nwords = static_cast<int>((p.N + 1) / 2);
     for (int w = tid; w < nwords; w += kQbThreads) bits[w] = 0u;
     for (int w = tid; w < 16 * kQbMaxCand / 32; w += kQbThreads) qbits[w] = 0u;
     __syncthreads();
-    for (int c = tid; c < nq * p.k; c += kQbThreads) {
+    for (int c = tid; c < k.nq * p.k; c += kQbThreads) {
       const int q = c / p.k;
-      const int64_t tq = t0 + q;
-      const int64_t i = __ldg(p.idx + (b * p.Tq + r0 + q) * p.k + (c % p.k));
+      const int64_t tq = k.t0 + q;
+      const int64_t i = __ldg(p.idx + (k.b * p.Tq + k.r0 + q) * p.k + (c % p.k));
       if (i >= 0 && i < p.N && (i + 1) * p.stride - 1 <= tq)
         atomicOr(&bits[i >> 1], 1u << (static_cast<int>(i & 1) * 16 + q));
     }
@@ -1407,125 +1436,156 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
       if ((v & 0xffffu) != 0u) put(2 * w, v & 0xffffu);
       if ((v >> 16) != 0u) put(2 * w + 1, v >> 16);
     }
-    n_ent = s_union;
+    n_ent_sparse = s_union;
   }
-  const int64_t n_slots = n_ent + nwin;
-  const int ntiles = static_cast<int>((n_slots + kQbKeys - 1) / kQbKeys);
   tc::fence_before_sync();
   __syncthreads();  // the union is ready and the P buffers are free again (Q may still be landing)
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
   bool healthy = true;
+  // this CTA's blocks: one (sparse), or every gridDim.x-th (dense)
+  const int64_t blk_step = sparse ? nblocks : gridDim.x;
+  auto n_entries = [&](const QbBlock& k) { return sparse ? n_ent_sparse : qb_dense_entries(p, k); };
 
   if (warp >= 8 && warp < 11) {
     // ===================== producer: cp.async copies that arrive by themselves =====================
-    const int64_t ebase = b * p.N;
-    const int64_t wbase = b * p.wrows - p.wpos0 + wlo0;
     const __nv_bfloat16* ve = p.cv ? p.cv : p.ck;
     const int ves = p.cv ? kDV : kDQK;
     const __nv_bfloat16* vw = p.wv ? p.wv : p.wk;
     const int vws = p.wv ? kDV : kDQK;
-    // K (three 128-byte blocks per key) or V (two) of one tile: eight lanes per
-    // 128-byte row segment, four keys per warp instruction
     const int pw = warp - 8, c8 = lane & 7;
-    auto issue = [&](bool is_k, uint8_t* T, int tile) {
-      const int64_t a0 = static_cast<int64_t>(tile) * kQbKeys;
-      for (int key = pw * 4 + (lane >> 3); key < kQbKeys; key += 12) {
-        const int64_t sl = a0 + key;
-        const __nv_bfloat16* src = nullptr;
-        if (sl < n_ent) {
-          const int64_t e = ebase + (sparse ? static_cast<int64_t>(ulist[sl]) : sl);
-          if (CSA_INBOUNDS(e >= 0 && e < p.ent_rows)) src = is_k ? p.ck + e * kDQK : ve + e * ves;
-        } else if (sl < n_slots) {
-          const int64_t w = wbase + (sl - n_ent);
-          if (CSA_INBOUNDS(w >= 0 && w < p.win_rows)) src = is_k ? p.wk + w * kDQK : vw + w * vws;
+    int64_t gt = 0;  // tiles of this CTA's earlier blocks
+    int jq = 0;      // earlier blocks that had tiles (each loaded its queries once)
+    for (int64_t blk = blockIdx.x; blk < nblocks && healthy; blk += blk_step) {
+      const QbBlock k = qb_block(p, blk);
+      const int64_t n_ent = n_entries(k);
+      const int64_t n_slots = n_ent + k.nwin;
+      const int ntiles = static_cast<int>((n_slots + kQbKeys - 1) / kQbKeys);
+      if (ntiles == 0) continue;
+      const int64_t ebase = k.b * p.N;
+      const int64_t wbase = k.b * p.wrows - p.wpos0 + k.wlo0;
+      // K (three 128-byte blocks per key) or V (two) of one tile: eight lanes per
+      // 128-byte row segment, four keys per warp instruction
+      auto issue = [&](bool is_k, uint8_t* T, int tile) {
+        const int64_t a0 = static_cast<int64_t>(tile) * kQbKeys;
+        for (int key = pw * 4 + (lane >> 3); key < kQbKeys; key += 12) {
+          const int64_t sl = a0 + key;
+          const __nv_bfloat16* src = nullptr;
+          if (sl < n_ent) {
+            const int64_t e = ebase + (sparse ? static_cast<int64_t>(ulist[sl]) : sl);
+            if (CSA_INBOUNDS(e >= 0 && e < p.ent_rows)) src = is_k ? p.ck + e * kDQK : ve + e * ves;
+          } else if (sl < n_slots) {
+            const int64_t w = wbase + (sl - n_ent);
+            if (CSA_INBOUNDS(w >= 0 && w < p.win_rows)) src = is_k ? p.wk + w * kDQK : vw + w * vws;
+          }
+          uint8_t* dst = T + tc::sw128(key, c8);
+          const __nv_bfloat16* s8 = src != nullptr ? src + c8 * 8 : p.q;
+          const int bytes = src != nullptr ? 16 : 0;
+          cp_async16(dst, s8, bytes);
+          cp_async16(dst + 8192, src != nullptr ? s8 + 64 : p.q, bytes);
+          if (is_k) cp_async16(dst + 16384, src != nullptr ? s8 + 128 : p.q, bytes);
         }
-        uint8_t* dst = T + tc::sw128(key, c8);
-        const __nv_bfloat16* s8 = src != nullptr ? src + c8 * 8 : p.q;
-        const int bytes = src != nullptr ? 16 : 0;
-        cp_async16(dst, s8, bytes);
-        cp_async16(dst + 8192, src != nullptr ? s8 + 64 : p.q, bytes);
-        if (is_k) cp_async16(dst + 16384, src != nullptr ? s8 + 128 : p.q, bytes);
-      }
-    };
-    // K(t) is issued before V(t - 1): K stages are freed when both S are done,
-    // V stages when both PV are
-    for (int it = 0; it <= ntiles; ++it) {
-      if (it < ntiles) {
-        const int st = it & 1;
-        if (it >= 2) {
-          bool ok = true;
-          if (lane == 0) ok = tc::bar_wait(&kfree[st], ((it >> 1) - 1) & 1);
-          if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) {
+      };
+      auto wait_free = [&](uint64_t* bar, uint32_t parity) {  // warp-uniform outcome
+        bool ok = true;
+        if (lane == 0) ok = tc::bar_wait(bar, parity);
+        return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      };
+      // K(t) is issued before V(t - 1): K stages are freed when both S are done,
+      // V stages when both PV are (stage and parity from the CTA-wide tile count);
+      // a dense block's queries follow its first K tile, once the previous
+      // block's last S is done
+      for (int it = 0; it <= ntiles; ++it) {
+        if (it < ntiles) {
+          const int64_t G = gt + it;
+          const int st = static_cast<int>(G & 1);
+          if (G >= 2 && !wait_free(&kfree[st], static_cast<uint32_t>(((G >> 1) - 1) & 1))) {
             healthy = false;
             break;
           }
+          issue(true, Kst + st * 3 * 8192, it);
+          cp_async_mbar_arrive_noinc(&kfull[st]);
         }
-        issue(true, Kst + st * 3 * 8192, it);
-        cp_async_mbar_arrive_noinc(&kfull[st]);
-      }
-      if (it >= 1) {
-        const int tile = it - 1, st = tile & 1;
-        if (tile >= 2) {
-          bool ok = true;
-          if (lane == 0) ok = tc::bar_wait(&vfree[st], ((tile >> 1) - 1) & 1);
-          if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) {
+        if (it == 0 && !sparse) {
+          if (jq > 0 && !wait_free(qfree, (jq - 1) & 1)) {
             healthy = false;
             break;
           }
+          if (tid == 8 * 32) load_q(k);
         }
-        issue(false, Vst + st * 2 * 8192, tile);
-        cp_async_mbar_arrive_noinc(&vfull[st]);
+        if (it >= 1) {
+          const int64_t G = gt + it - 1;
+          const int st = static_cast<int>(G & 1);
+          if (G >= 2 && !wait_free(&vfree[st], static_cast<uint32_t>(((G >> 1) - 1) & 1))) {
+            healthy = false;
+            break;
+          }
+          issue(false, Vst + st * 2 * 8192, it - 1);
+          cp_async_mbar_arrive_noinc(&vfull[st]);
+        }
       }
+      gt += ntiles;
+      ++jq;
     }
     cp_async_wait<0>();
   } else if (warp == 11) {
     // ===================== MMA issue (one thread) =====================
     constexpr uint32_t kIdescS = tc::idesc_bf16(128, kQbKeys, false);
     constexpr uint32_t kIdescO = tc::idesc_bf16(128, kDV, true);
-    auto issue_s = [&](int tile) {
-      const int st = tile & 1;
-      const uint32_t ka = smem_u32(Kst + st * 3 * 8192);
-      tc::fence_async_smem();  // the stage was written by cp.async
-      tc::fence_after_sync();
-      for (int g = 0; g < 2; ++g) {
-        const uint32_t qa = smem_u32(Qs + g * 49152);
-#pragma unroll
-        for (int kk = 0; kk < 12; ++kk)
-          tc::mma_bf16_ss(tmem + 64 * (2 * g + st), tc::desc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                          tc::desc_sw128(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-        tc::mma_commit(&sdone[2 * g + st]);
-      }
-      tc::mma_commit(&kfree[st]);
-    };
-    if (lane == 0 && ntiles > 0) {
-      if (healthy) healthy = tc::bar_wait(qfull, 0);
-      for (int tt = 0; tt < 2 && tt < ntiles; ++tt) {
-        if (healthy) healthy = tc::bar_wait(&kfull[tt], 0);
-        issue_s(tt);
-      }
-      for (int tile = 0; tile < ntiles; ++tile) {
-        const int st = tile & 1;
-        const uint32_t va = smem_u32(Vst + st * 2 * 8192);
-        for (int g = 0; g < 2; ++g) {
-          if (healthy) healthy = tc::bar_wait(&pready[g], tile & 1);
-          if (g == 0 && healthy) {
-            healthy = tc::bar_wait(&vfull[st], (tile >> 1) & 1);
-            tc::fence_async_smem();  // the stage was written by cp.async
-          }
+    if (lane == 0) {
+      int64_t gt = 0;
+      int jq = 0;
+      for (int64_t blk = blockIdx.x; blk < nblocks && healthy; blk += blk_step) {
+        const QbBlock k = qb_block(p, blk);
+        const int64_t n_slots = n_entries(k) + k.nwin;
+        const int ntiles = static_cast<int>((n_slots + kQbKeys - 1) / kQbKeys);
+        if (ntiles == 0) continue;
+        auto issue_s = [&](int tile) {  // S of both groups for the block's tile; the last one frees Q
+          const int64_t G = gt + tile;
+          const int st = static_cast<int>(G & 1);
+          if (healthy) healthy = tc::bar_wait(&kfull[st], static_cast<uint32_t>((G >> 1) & 1));
+          const uint32_t ka = smem_u32(Kst + st * 3 * 8192);
+          tc::fence_async_smem();  // the stage was written by cp.async
           tc::fence_after_sync();
-          const uint32_t pa = smem_u32(Pst + g * 16384);
+          for (int g = 0; g < 2; ++g) {
+            const uint32_t qa = smem_u32(Qs + g * 49152);
 #pragma unroll
-          for (int ks = 0; ks < kQbKeys / 16; ++ks)
-            tc::mma_bf16_ss(tmem + 256 + 128 * g, tc::desc_sw128(pa + ks * 32, 16, 1024),
-                            tc::desc_sw128(va + ks * 2048, 8192, 1024), kIdescO, (tile > 0 || ks > 0) ? 1u : 0u);
-          tc::mma_commit(&pvdone[g]);
+            for (int kk = 0; kk < 12; ++kk)
+              tc::mma_bf16_ss(tmem + 64 * (2 * g + st), tc::desc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                              tc::desc_sw128(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), kIdescS,
+                              kk > 0 ? 1u : 0u);
+            tc::mma_commit(&sdone[2 * g + st]);
+          }
+          tc::mma_commit(&kfree[st]);
+          if (tile == ntiles - 1) tc::mma_commit(qfree);
+        };
+        if (healthy) healthy = tc::bar_wait(qfull, static_cast<uint32_t>(jq & 1));
+        for (int tt = 0; tt < 2 && tt < ntiles; ++tt) issue_s(tt);
+        for (int tile = 0; tile < ntiles; ++tile) {
+          const int64_t G = gt + tile;
+          const int st = static_cast<int>(G & 1);
+          const uint32_t va = smem_u32(Vst + st * 2 * 8192);
+          for (int g = 0; g < 2; ++g) {
+            if (healthy) healthy = tc::bar_wait(&pready[g], static_cast<uint32_t>(G & 1));
+            if (tile == 0 && jq > 0 && healthy)  // the previous block's O of this group has been read out
+              healthy = tc::bar_wait(&ofree[g], static_cast<uint32_t>((jq - 1) & 1));
+            if (g == 0 && healthy) {
+              healthy = tc::bar_wait(&vfull[st], static_cast<uint32_t>((G >> 1) & 1));
+              tc::fence_async_smem();  // the stage was written by cp.async
+            }
+            tc::fence_after_sync();
+            const uint32_t pa = smem_u32(Pst + g * 16384);
+#pragma unroll
+            for (int ks = 0; ks < kQbKeys / 16; ++ks)
+              tc::mma_bf16_ss(tmem + 256 + 128 * g, tc::desc_sw128(pa + ks * 32, 16, 1024),
+                              tc::desc_sw128(va + ks * 2048, 8192, 1024), kIdescO, (tile > 0 || ks > 0) ? 1u : 0u);
+            tc::mma_commit(&pvdone[g]);
+          }
+          tc::mma_commit(&vfree[st]);
+          if (tile + 2 < ntiles) issue_s(tile + 2);
         }
-        tc::mma_commit(&vfree[st]);
-        if (tile + 2 < ntiles) {
-          if (healthy) healthy = tc::bar_wait(&kfull[st], ((tile + 2) >> 1) & 1);
-          issue_s(tile + 2);
-        }
+        gt += ntiles;
+        ++jq;
       }
     }
   } else if (warp < 8) {
@@ -1534,112 +1594,132 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
     const int rl = tid & 127;          // TMEM lane
     const int r = 128 * g + rl;        // row of the block
     const int qr = r / H;              // query of this row within the block
-    const bool row_ok = qr < nq;
-    const int64_t tq = t0 + (row_ok ? qr : 0);
-    int64_t nv_q = (tq + 1) / p.stride;
-    if (nv_q > p.N) nv_q = p.N;
-    const int64_t lo_q = (tq - p.wlen + 1) > 0 ? (tq - p.wlen + 1) : 0;
-    // slot numbers (below 2^31): the entry run, this row's visible entries and window slots
-    const int ent32 = static_cast<int>(n_ent), nv32 = static_cast<int>(nv_q);
-    const int wv_lo = static_cast<int>(n_ent + (lo_q - wlo0)), wv_hi = static_cast<int>(n_ent + (tq - wlo0));
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tmem + 256 + 128 * g;
-    float m_ref = -INFINITY, l = 0.f;
-    for (int tile = 0; tile < ntiles; ++tile) {
-      const int st = tile & 1;
-      if (healthy) healthy = tc::bar_wait(&sdone[2 * g + st], (tile >> 1) & 1);
-      tc::fence_after_sync();
-      float sv[kQbKeys];
-      tc::tmem_ld32(tmem + 64 * (2 * g + st) + lane_base, sv);
-      tc::tmem_ld32(tmem + 64 * (2 * g + st) + lane_base + 32, sv + 32);
-      // this row's visible slots of the tile as a bit mask: its entries, then its window run
-      const int sb = tile * kQbKeys;
-      uint64_t vm = 0;
-      if (row_ok) {
-        if (sb < ent32) {
-          vm = sparse ? (static_cast<uint64_t>(qbits[qr * (kQbMaxCand / 32) + (sb >> 5) + 1]) << 32) |
-                            qbits[qr * (kQbMaxCand / 32) + (sb >> 5)]
-                      : range_bits(0, nv32 - 1, sb);
-          vm &= range_bits(0, ent32 - 1, sb);
-        }
-        vm |= range_bits(wv_lo, wv_hi, sb);
-      }
-      const uint32_t vlo = static_cast<uint32_t>(vm), vhi = static_cast<uint32_t>(vm >> 32);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < kQbKeys; ++j) {
-        const bool ok = (((j < 32 ? vlo : vhi) >> (j & 31)) & 1u) != 0u;
-        sv[j] = ok ? sv[j] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, sv[j]);
-      }
-      const float m_new = fmaxf(m_ref, mx);
-      const bool resc = m_new > m_ref + 8.f;
-      float corr = 1.f;
-      if (resc) {
-        corr = exp2f(m_ref - m_new);
-        m_ref = m_new;
-        l *= corr;
-      }
-      const float base = m_ref == -INFINITY ? 0.f : m_ref;
-      float sum = 0.f;
-#pragma unroll
-      for (int j = 0; j < kQbKeys; ++j) {
-        sv[j] = fast_exp2(sv[j] - base);
-        sum += sv[j];
-      }
-      l += sum;
-      if (tile > 0) {  // PV of the previous tile: the P buffer is free and O is quiet
-        if (healthy) healthy = tc::bar_wait(&pvdone[g], (tile - 1) & 1);
+    int64_t gt = 0;
+    for (int64_t blk = blockIdx.x; blk < nblocks; blk += blk_step) {
+      const QbBlock k = qb_block(p, blk);
+      const int64_t n_ent = n_entries(k);
+      const int64_t n_slots = n_ent + k.nwin;
+      const int ntiles = static_cast<int>((n_slots + kQbKeys - 1) / kQbKeys);
+      const bool row_ok = qr < k.nq;
+      // this row's output (the block geometry is not needed past this point)
+      const int64_t orow = (k.b * p.Tq + k.r0) * H + r;
+      const int64_t tq = k.t0 + (row_ok ? qr : 0);
+      int64_t nv_q = (tq + 1) / p.stride;
+      if (nv_q > p.N) nv_q = p.N;
+      const int64_t lo_q = (tq - p.wlen + 1) > 0 ? (tq - p.wlen + 1) : 0;
+      // slot numbers (below 2^31): the entry run, this row's visible entries and window slots
+      const int ent32 = static_cast<int>(n_ent), nv32 = static_cast<int>(nv_q);
+      const int wv_lo = static_cast<int>(n_ent + (lo_q - k.wlo0)), wv_hi = static_cast<int>(n_ent + (tq - k.wlo0));
+      float m_ref = -INFINITY, l = 0.f;
+      for (int tile = 0; tile < ntiles; ++tile) {
+        const int64_t G = gt + tile;
+        const int st = static_cast<int>(G & 1);
+        if (healthy) healthy = tc::bar_wait(&sdone[2 * g + st], static_cast<uint32_t>((G >> 1) & 1));
         tc::fence_after_sync();
-        if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float ov[32];
-            tc::tmem_ld32(tO + lane_base + 32 * c, ov);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] *= corr;
-            tc::tmem_st32(tO + lane_base + 32 * c, ov);
+        float sv[kQbKeys];
+        tc::tmem_ld32(tmem + 64 * (2 * g + st) + lane_base, sv);
+        tc::tmem_ld32(tmem + 64 * (2 * g + st) + lane_base + 32, sv + 32);
+        // this row's visible slots of the tile as a bit mask: its entries, then its window run
+        const int sb = tile * kQbKeys;
+        uint64_t vm = 0;
+        if (row_ok) {
+          if (sb < ent32) {
+            vm = sparse ? (static_cast<uint64_t>(qbits[qr * (kQbMaxCand / 32) + (sb >> 5) + 1]) << 32) |
+                              qbits[qr * (kQbMaxCand / 32) + (sb >> 5)]
+                        : range_bits(0, nv32 - 1, sb);
+            vm &= range_bits(0, ent32 - 1, sb);
           }
-          tc::tmem_wait_st();
+          vm |= range_bits(wv_lo, wv_hi, sb);
         }
-      }
-      {
-        uint8_t* Pb = Pst + g * 16384;
+        const uint32_t vlo = static_cast<uint32_t>(vm), vhi = static_cast<uint32_t>(vm >> 32);
+        float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = make_uint4(pack_bf16x2(sv[8 * c], sv[8 * c + 1]), pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]),
-                                     pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]),
-                                     pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]));
-          *reinterpret_cast<uint4*>(Pb + tc::sw128(rl, c)) = v;
+        for (int j = 0; j < kQbKeys; ++j) {
+          const bool ok = (((j < 32 ? vlo : vhi) >> (j & 31)) & 1u) != 0u;
+          sv[j] = ok ? sv[j] * p.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sv[j]);
         }
+        const float m_new = fmaxf(m_ref, mx);
+        const bool resc = m_new > m_ref + 8.f;
+        float corr = 1.f;
+        if (resc) {
+          corr = exp2f(m_ref - m_new);
+          m_ref = m_new;
+          l *= corr;
+        }
+        const float base = m_ref == -INFINITY ? 0.f : m_ref;
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < kQbKeys; ++j) {
+          sv[j] = fast_exp2(sv[j] - base);
+          sum += sv[j];
+        }
+        l += sum;
+        if (tile > 0) {  // PV of the previous tile: the P buffer is free and O is quiet
+          if (healthy) healthy = tc::bar_wait(&pvdone[g], static_cast<uint32_t>((G - 1) & 1));
+          tc::fence_after_sync();
+          if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float ov[32];
+              tc::tmem_ld32(tO + lane_base + 32 * c, ov);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] *= corr;
+              tc::tmem_st32(tO + lane_base + 32 * c, ov);
+            }
+            tc::tmem_wait_st();
+          }
+        }
+        {
+          uint8_t* Pb = Pst + g * 16384;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = make_uint4(pack_bf16x2(sv[8 * c], sv[8 * c + 1]), pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]),
+                                       pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]),
+                                       pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]));
+            *reinterpret_cast<uint4*>(Pb + tc::sw128(rl, c)) = v;
+          }
+        }
+        tc::fence_async_smem();
+        tc::fence_before_sync();
+        named_sync(2 + g, 128);
+        if (rl == 0) bar_arrive(&pready[g]);
       }
-      tc::fence_async_smem();
-      tc::fence_before_sync();
-      named_sync(2 + g, 128);
-      if (rl == 0) bar_arrive(&pready[g]);
-    }
-    if (ntiles > 0 && healthy) healthy = tc::bar_wait(&pvdone[g], (ntiles - 1) & 1);
-    tc::fence_after_sync();
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16* o = p.out + ((b * p.Tq + r0) * H + r) * kDV;
+      if (ntiles > 0 && healthy) healthy = tc::bar_wait(&pvdone[g], static_cast<uint32_t>((gt + ntiles - 1) & 1));
+      tc::fence_after_sync();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint32_t ob[4][16];  // the normalised row, bf16 pairs
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float ov[32];
-      if (ntiles > 0) {
-        tc::tmem_ld32(tO + lane_base + 32 * c, ov);
-      } else {
+      for (int c = 0; c < 4; ++c) {
+        float ov[32];
+        if (ntiles > 0) {
+          tc::tmem_ld32(tO + lane_base + 32 * c, ov);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+          for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ob[c][i] = pack_bf16x2(ov[2 * i] * inv, ov[2 * i + 1] * inv);
+      }
+      if (ntiles > 0) {  // O is read out: the next block's first PV may overwrite it
+        tc::fence_before_sync();
+        named_sync(2 + g, 128);
+        if (rl == 0) bar_arrive(&ofree[g]);
       }
       if (row_ok) {
+        __nv_bfloat16* o = p.out + orow * kDV;
 #pragma unroll
-        for (int i = 0; i < 32; i += 8)
-          *reinterpret_cast<uint4*>(o + 32 * c + i) =
-              make_uint4(pack_bf16x2(ov[i] * inv, ov[i + 1] * inv), pack_bf16x2(ov[i + 2] * inv, ov[i + 3] * inv),
-                         pack_bf16x2(ov[i + 4] * inv, ov[i + 5] * inv), pack_bf16x2(ov[i + 6] * inv, ov[i + 7] * inv));
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<uint4*>(o + 32 * c + 2 * i) = make_uint4(ob[c][i], ob[c][i + 1], ob[c][i + 2], ob[c][i + 3]);
+        }
+        if (p.lse) p.lse[orow] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
       }
+      gt += ntiles;
     }
-    if (row_ok && p.lse) p.lse[(b * p.Tq + r0) * H + r] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
   }
   pdl_trigger();
   cp_async_wait<0>();  // (the query copies landed long before; nothing of this thread stays in flight)
@@ -1994,10 +2074,24 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   const bool blk_shape = !fp8 && pk == nullptr && Tq >= qb_rows && R >= 2LL * num_sms();
   const bool use_blk = blk_shape && (idx == nullptr || (H == 16 && static_cast<int64_t>(qb_rows) * k <= kQbMaxCand &&
                                                         N <= kQbMaxEnt));
+  CUtensorMap qmap;  // the query-blocked kernel's queries: [B][Tq*H][192] bf16, 128 x 64 boxes
+  memset(&qmap, 0, sizeof(qmap));
   if (use_blk) {
-    fn = attn_qblock_kernel;
+    CSA_REQUIRE(Tq * H < (int64_t(1) << 31) && B < (int64_t(1) << 31), "%s: too many query rows", name);
+    CSA_REQUIRE(aligned16(q), "%s: q must be 16-byte aligned", name);
+    const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (encode == nullptr) return fail(CSA_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(Tq * H),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDQK) * 2, static_cast<cuuint64_t>(Tq * H) * kDQK * 2};
+    const cuuint32_t box[3] = {64u, 128u, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUresult r = encode(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "%s: query tensor map encoding failed (%d)", name, int(r));
     smem = qb_layout().total;
-    if (!ensure_smem(reinterpret_cast<const void*>(fn), static_cast<int>(smem)))
+    if (!ensure_smem(reinterpret_cast<const void*>(attn_qblock_kernel), static_cast<int>(smem)))
       return fail(CSA_ERR_CUDA, "%s: cannot raise the shared memory limit to %zu", name, smem);
     pl.cl = 1;
     part = nullptr;
@@ -2032,14 +2126,18 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
   p.cu_ent = pk ? pk->cu_entries : nullptr;
   p.n_seqs = pk ? pk->n_seqs : 0;
   p.ent_rows = pk ? N : B * N;
+  p.qb_blocks = use_blk ? B * ((Tq + qb_rows - 1) / qb_rows) : 0;
   p.win_rows = wlen > 0 ? (pk ? pk->total_tokens : B * win->rows) : 0;
 
-  const dim3 grid(static_cast<unsigned>(use_blk ? B * ((Tq + qb_rows - 1) / qb_rows) : R * pl.cl));
+  // dense query blocks: a persistent grid of one CTA per SM; sparse blocks: one CTA each
+  const int64_t blk_grid = idx == nullptr ? std::min<int64_t>(p.qb_blocks, num_sms()) : p.qb_blocks;
+  const dim3 grid(static_cast<unsigned>(use_blk ? blk_grid : R * pl.cl));
   const dim3 block(use_blk ? kQbThreads : (use_tc ? kTcDecThreads : kThreads));
   const int cluster = (use_tc && !tc_cluster) || use_blk ? 1 : pl.cl;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   prof_begin(s);
-  const cudaError_t e = launch_pdl((use_tc && !use_blk) ? tfn : fn, grid, block, smem, s, cluster, p);
+  const cudaError_t e = use_blk ? launch_pdl(attn_qblock_kernel, grid, block, smem, s, 1, p, qmap)
+                                : launch_pdl(use_tc ? tfn : fn, grid, block, smem, s, cluster, p);
   prof_end(s);
   if (csa_status st = check_launch(name, e); st != CSA_OK) return st;
   if (part != nullptr)
