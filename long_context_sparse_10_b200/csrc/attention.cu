@@ -2005,9 +2005,10 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
     const TcSplit sp = tc_split(R, max_slots);
     if (sp.nsplit > 1 && pl.cl > 1) {
       // A cluster merge (distributed shared memory, no second kernel) wins when
-      // a co-resident cluster size leaves at most two more tiles per CTA than
-      // the global split does (the merge kernel and its launch cost about
-      // that much).
+      // a co-resident cluster size leaves no more tiles per CTA than the global
+      // split does; with even one tile more per CTA the split and its one-round
+      // merge kernel are faster (8 CSA decode rows of 17 tiles: 9-CTA clusters
+      // of 2 tiles 12.1 us, 17 CTAs of 1 tile + merge 11.4 us, graph-replayed).
       static std::mutex mu;
       bool nonportable = true;
       {
@@ -2023,7 +2024,7 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
       const int64_t tiles = max_slots > 0 ? (max_slots + kTcKeys - 1) / kTcKeys : 1;
       const int64_t tps = (tiles + cl - 1) / cl;
       if (cl > 1 && max_active_clusters(pick_tc(fp8, shv), cl, tc_layout(fp8, shv, 0).total, kTcDecThreads) >= R &&
-          tps <= sp.tps + 2) {
+          tps <= sp.tps) {
         tc_cluster = true;
         pl.tps = static_cast<int>(tps);
         pl.cl = static_cast<int>((tiles + tps - 1) / tps);
