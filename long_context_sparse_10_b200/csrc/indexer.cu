@@ -18,11 +18,12 @@
 //   * rows whose visible prefix fits in shared memory (prefill) run one CTA
 //     per row over the row held in shared memory;
 //   * long rows (decode over 10^5..10^6 entries) get a 4096-bin histogram of
-//     the key's top 12 bits fused into the scoring kernel, whose last CTA per
-//     row derives the threshold bin; one select kernel then emits a bitmap of
-//     the entries above that bin plus a candidate list of the bin itself, and
-//     its last CTA per row resolves the candidates and writes the ascending
-//     list.  "Last CTA" is decided by an atomic counter (no CTA ever waits).
+//     the key's top 12 bits fused into the scoring kernel; one select kernel
+//     then derives each row's threshold bin from it (in every CTA), emits a
+//     bitmap of the entries above that bin plus a candidate list of the bin
+//     itself, and its last CTA per row resolves the candidates and writes the
+//     ascending list.  "Last CTA" is decided by an atomic counter (no CTA ever
+//     waits).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -502,9 +503,7 @@ struct LongScoreParams {
   int chunk;  // entries per CTA, a multiple of kLongTR
   int64_t pitch;  // row pitch of scores
   float* scores;
-  uint32_t* hist;
-  uint32_t* done;
-  int32_t* thr;
+  uint32_t* hist;  // [R, kHistBins] (zeroed per call): each CTA adds its chunk's bins
   int k;
 };
 
@@ -520,8 +519,6 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
   float* scale_st = reinterpret_cast<float*>(smem + S::kScaleOff);  // E4: [kStages][kLongTR]
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + S::kHistOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
-  __shared__ uint32_t last_s;
-  __shared__ uint32_t scan_sh[32];
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -702,17 +699,8 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
     if (c & 0xffffu) atomicAdd(gh + 2 * j, c & 0xffffu);
     if (c >> 16) atomicAdd(gh + 2 * j + 1, c >> 16);
   }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t ctas = static_cast<uint32_t>((nv + p.chunk - 1) / p.chunk);
-    last_s = (atomicAdd(p.done + 2 * row, 1u) == ctas - 1) ? 1u : 0u;
-  }
-  __syncthreads();
-  if (last_s) {
-    __threadfence();
-    row_threshold<kLongThreads>(gh, nv, p.k, p.thr + 2 * row, scan_sh);
-  }
+  // (the select kernel derives each row's threshold from the complete histogram
+  // once this grid has finished: no counter, no waiting CTA)
 }
 
 // ---------------------------------------------------------------------------
@@ -1342,17 +1330,18 @@ struct LongWs {
   float* scores;        // [R, pitch] (pitch = N rounded up to 4: 16-byte aligned rows)
   uint32_t* hist;       // [R, kHistBins]    (zeroed per call)
   uint32_t* cand_cnt;   // [R]               (zeroed per call)
-  uint32_t* done;       // [R, 2]: scoring / select CTAs finished (zeroed per call)
-  int32_t* thr;         // [R, 2]
+  uint32_t* done;       // [R]: select CTAs finished (zeroed per call)
   uint2* cand;          // [R, N]: (key, index) of the threshold bin's entries
   uint32_t* bitmap;     // [R, W]
   int64_t W;
   int64_t pitch;
 };
 
-// Per CTA: a bitmap word for every 32 entries (entries above the threshold
-// bin), and the threshold bin's entries appended to the row's candidate list
-// (gathered in shared memory first, one global atomic per CTA).  The last CTA
+// Per CTA: the row's threshold bin from its complete histogram (every CTA of
+// the row derives it, its score loads already in flight), then a bitmap word
+// for every 32 entries (entries above the threshold bin), and the threshold
+// bin's entries appended to the row's candidate list (gathered in shared
+// memory first, one global atomic per CTA).  The last CTA
 // of a row then radix-selects the `need` best candidates on the composite key
 // (score key << 32 | ~index), merges them into the row's bitmap and writes the
 // ascending index list.  Rows up to kBitmapSmemWords*32 entries keep that final
@@ -1367,6 +1356,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   __shared__ uint32_t hist[256];
   __shared__ uint32_t dig[3];
   __shared__ uint32_t n_cand, base_s, last_s;
+  __shared__ int32_t thr_s[2];
+  __shared__ uint32_t scan_sh[32];
   const int64_t row = blockIdx.y;
   const int64_t nv = visible(q_pos0 + row % Tq, m, N);
   const int64_t e_begin = static_cast<int64_t>(blockIdx.x) * kSelChunk;
@@ -1378,16 +1369,12 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
     return;
   }
   if (e_begin >= nv) return;
-  const int thr_bin = ws.thr[2 * row];
-  if (thr_bin < 0) {  // every visible entry is selected
+  if (nv <= k) {  // every visible entry is selected
     if (blockIdx.x == 0) write_prefix_ids(out, nv, k, sout, srow);
     return;
   }
   const int64_t e_end = (e_begin + kSelChunk) < nv ? (e_begin + kSelChunk) : nv;
-  const uint32_t tb = static_cast<uint32_t>(thr_bin);
   const int lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) n_cand = 0;
-  __syncthreads();
   // warp w scans entries [e_begin + 512 w, e_begin + 512 (w + 1)), four per
   // lane per step (16-byte loads; rows are 16-byte aligned and padded)
   constexpr int kSelWarps = kSelThreads / 32;
@@ -1400,6 +1387,11 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
     const int64_t i = e_begin + warp * kPerWarp + it * 128 + 4 * lane;
     sv[it] = i < e_end ? __ldcg(reinterpret_cast<const float4*>(srow + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  // the threshold bin and the count still needed from it (nv > k: a bin exists)
+  row_threshold<kSelThreads>(ws.hist + row * kHistBins, nv, k, thr_s, scan_sh);
+  if (threadIdx.x == 0) n_cand = 0;
+  __syncthreads();
+  const uint32_t tb = static_cast<uint32_t>(thr_s[0]);
 #pragma unroll
   for (int it = 0; it < kSteps; ++it) {
     const int64_t base = e_begin + warp * kPerWarp + it * 128;  // a multiple of 32
@@ -1456,7 +1448,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   __syncthreads();
   if (threadIdx.x == 0) {
     const uint32_t chunks = static_cast<uint32_t>((nv + kSelChunk - 1) / kSelChunk);
-    last_s = (atomicAdd(ws.done + 2 * row + 1, 1u) == chunks - 1) ? 1u : 0u;
+    last_s = (atomicAdd(ws.done + row, 1u) == chunks - 1) ? 1u : 0u;
   }
   __syncthreads();
   if (!last_s) return;
@@ -1521,8 +1513,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   __syncthreads();
 
   // ---- resolve the threshold bin: radix select on the 52 low composite bits
-  uint32_t remaining = static_cast<uint32_t>(ws.thr[2 * row + 1]);
-  uint64_t prefix = static_cast<uint64_t>(thr_bin) << 52;
+  uint32_t remaining = static_cast<uint32_t>(thr_s[1]);
+  uint64_t prefix = static_cast<uint64_t>(tb) << 52;
   uint64_t mask = 0xfffull << 52;
   uint32_t in_bucket = cnt;
   for (int pass = 0; pass < 7 && in_bucket != remaining; ++pass) {
@@ -1649,7 +1641,7 @@ constexpr int64_t kPrefillTcMaxN = 65535;
 bool use_prefill_tc(int64_t R, int64_t N) { return N <= kPrefillTcMaxN && R >= 32LL * num_sms(); }
 
 struct LongLayout {
-  size_t scores, hist, cnt, done, thr, cand, bitmap, total;
+  size_t scores, hist, cnt, done, zero_end, cand, bitmap, total;
   int64_t W, pitch;
 };
 
@@ -1661,8 +1653,9 @@ LongLayout long_layout(int64_t R, int64_t N) {
   L.scores = off; off = align_up(off + static_cast<size_t>(R) * L.pitch * 4);
   L.hist = off;   off += static_cast<size_t>(R) * kHistBins * 4;     // hist, cnt and done: zeroed together
   L.cnt = off;    off += static_cast<size_t>(R) * 4;
-  L.done = off;   off = align_up(off + static_cast<size_t>(R) * 8);
-  L.thr = off;    off = align_up(off + static_cast<size_t>(R) * 8);
+  L.done = off;   off += static_cast<size_t>(R) * 4;
+  L.zero_end = off;
+  off = align_up(off);
   L.cand = off;   off = align_up(off + static_cast<size_t>(R) * N * 8);
   L.bitmap = off; off = align_up(off + static_cast<size_t>(R) * L.W * 4);
   L.total = off;
@@ -1901,12 +1894,11 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   w.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
   w.cand_cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
   w.done = reinterpret_cast<uint32_t*>(ws + L.done);
-  w.thr = reinterpret_cast<int32_t*>(ws + L.thr);
   w.cand = reinterpret_cast<uint2*>(ws + L.cand);
   w.bitmap = reinterpret_cast<uint32_t*>(ws + L.bitmap);
   w.W = L.W;
   w.pitch = L.pitch;
-  if (cudaMemsetAsync(w.hist, 0, L.thr - L.hist, s) != cudaSuccess)
+  if (cudaMemsetAsync(w.hist, 0, L.zero_end - L.hist, s) != cudaSuccess)
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: memset failed");
   CSA_REQUIRE(R < 65536, "csa_indexer_topk: too many query rows for the long-row path");
   LongScoreParams lp;
@@ -1921,8 +1913,6 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   lp.scores = w.scores;
   lp.pitch = w.pitch;
   lp.hist = w.hist;
-  lp.done = w.done;
-  lp.thr = w.thr;
   lp.k = k;
   CUtensorMap kmap;
   memset(&kmap, 0, sizeof(kmap));
