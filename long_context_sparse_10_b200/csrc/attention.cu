@@ -15,8 +15,9 @@
 //    128-key tiles, for few rows), tcgen05 MMAs with the keys as the M
 //    dimension; described where it is defined.
 //  - attn_qblock_kernel (prefill over a bf16 cache: dense HCA attention, and
-//    sparse CSA attention with few heads): a block of consecutive queries per
-//    CTA, 256 (query, head) rows sharing each 64-key tile of the block's keys.
+//    sparse CSA attention with few heads): blocks of consecutive queries,
+//    256 (query, head) rows sharing each 64-key tile of the block's keys; dense
+//    blocks on a persistent grid whose pipeline runs from block to block.
 //  - attn_kernel (warp-level mma.sync, the remaining shapes: 16 heads with few
 //    rows, an FP8 cache or packed sequences; 64 heads over an FP8 cache with a
 //    separate raw-window V): one row per CTA in tiles of 64 keys,
@@ -28,9 +29,9 @@
 // Rows that are few (decode) split their tiles over several CTAs, merged in
 // one of two ways: a thread-block cluster of up to 16 CTAs whose partial
 // softmax states (m, l, O) meet in distributed shared memory (no global
-// scratch, no second launch), or, on the tcgen05 path when that leaves fewer
-// tiles per CTA, one CTA per split writing 16-byte partial records to the
-// caller's workspace, combined by attn_merge_kernel.
+// scratch, no second launch), or, on the tcgen05 path unless a cluster leaves
+// no more tiles per CTA, one CTA per split writing 16-byte partial records to
+// the caller's workspace, combined by attn_merge_kernel.
 #include <cooperative_groups.h>
 
 #include <map>

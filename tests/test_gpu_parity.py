@@ -171,7 +171,14 @@ def test_csa_sparse_mqa_prefill_bf16(H, B, T, m, k, win, sep_v):
     assert_lse(f64(lse), L, "csa prefill lse")
 
 
-@pytest.mark.parametrize("H,B,T,mp,win", [(16, 2, 700, 32, 64), (64, 1, 1000, 128, 128), (16, 1, 129, 128, 1)])
+@pytest.mark.parametrize("H,B,T,mp,win", [
+    (16, 2, 700, 32, 64), (64, 1, 1000, 128, 128), (16, 1, 129, 128, 1),
+    # more query blocks than SMs (a persistent CTA runs several): no window, so the first block of each
+    # sequence sees no key at all; the last block of each sequence holds 8 queries (its second row group
+    # lies past the sequence and is zero-filled)
+    (16, 3, 1000, 32, 0),
+    (16, 2, 2500, 64, 128),  # several blocks per CTA with a window; last block of 4 queries
+])
 def test_hca_dense_mqa_prefill_bf16(H, B, T, mp, win):
     g = np.random.default_rng(H * T + mp)
     N = -(-T // mp)
