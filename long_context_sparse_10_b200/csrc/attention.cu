@@ -1373,12 +1373,14 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
   // queries of a block (one thread): rows (query, head) of both groups, six
   // TMA boxes of 128 rows x 64 dims in the 128-byte swizzle (the [B][Tq*H][192]
   // tensor map zero-fills the rows past the sequence's last query)
-  auto load_q = [&](const QbBlock& k) {
+  auto load_q = [&](const QbBlock& k) {  // (read once: evict first, so the key rows stay in L2)
     tc::bar_arrive_expect_tx(qfull, 6 * 16384);
     const int y0 = static_cast<int>(k.r0 * H);
+    const uint64_t pol = tc::l2_evict_first_policy();
     for (int g = 0; g < 2; ++g)
       for (int cb = 0; cb < 3; ++cb)
-        tc::tma_load_3d(Qs + g * 49152 + cb * 16384, &qmap, 64 * cb, y0 + 128 * g, static_cast<int>(k.b), qfull);
+        tc::tma_load_3d_stream(Qs + g * 49152 + cb * 16384, &qmap, 64 * cb, y0 + 128 * g, static_cast<int>(k.b),
+                               qfull, pol);
   };
 
   // sparse: the union of the block's selections (one block per CTA)
@@ -1715,7 +1717,8 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
         for (int c = 0; c < 4; ++c) {
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<uint4*>(o + 32 * c + 2 * i) = make_uint4(ob[c][i], ob[c][i + 1], ob[c][i + 2], ob[c][i + 3]);
+            __stcs(reinterpret_cast<uint4*>(o + 32 * c + 2 * i),  // streamed out: not kept in L2
+                   make_uint4(ob[c][i], ob[c][i + 1], ob[c][i + 2], ob[c][i + 3]));
         }
         if (p.lse) p.lse[orow] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
       }
