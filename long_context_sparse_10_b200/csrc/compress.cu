@@ -208,10 +208,29 @@ __global__ void __launch_bounds__(256) compress_flat_kernel(CompressParams p) {
   pdl_wait();
   pdl_trigger();
   const int64_t gidx = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
-  const int64_t e = gidx / p.G;
-  const int g = static_cast<int>(gidx % p.G);
-  if (e >= p.B * p.N) return;
-  const EntryRef er = entry_ref(p, e);
+  const int64_t n_ent = p.B * p.N;
+  int64_t e;
+  int g;
+  EntryRef er;
+  if (n_ent * p.G < (int64_t(1) << 31) && p.cu_tok == nullptr) {
+    // every index below 2^31: 32-bit divisions (the 64-bit ones are emulated
+    // and cost more than the entry's arithmetic)
+    const uint32_t gi = static_cast<uint32_t>(gidx), G = static_cast<uint32_t>(p.G);
+    const uint32_t e32 = gi / G;
+    g = static_cast<int>(gi - e32 * G);
+    e = e32;
+    if (e >= n_ent) return;
+    const uint32_t N = static_cast<uint32_t>(p.N), b = e32 / N;
+    er.i = p.i0 + (e32 - b * N);
+    er.out_row = static_cast<int64_t>(b) * p.n_out + er.i;
+    er.T = p.T;
+    er.x0 = p.x + (static_cast<int64_t>(b) * p.xrows - p.xpos0) * p.d;
+  } else {
+    e = gidx / p.G;
+    g = static_cast<int>(gidx % p.G);
+    if (e >= n_ent) return;
+    er = entry_ref(p, e);
+  }
   const int64_t start = er.i * p.stride - (CW - p.stride);
   float wv[8];
   load8f(p.w + 8 * g, wv);
