@@ -107,7 +107,7 @@ def _indexer_case(g, B, Tq, N, tie_blocks=0, zero_q=False):
     (64, 1, 32768, 4 * 32768 - 1, 4, 2048, 0, False),  # 64 decode rows at 131072 tokens of context
     (2, 1, 2049, 4 * 2049 - 1, 4, 2048, 0, False),    # long rows with one entry more than k visible
     (2, 2, 2048, 4 * 2048 - 2, 4, 2048, 0, False),    # long rows with k - 1 and exactly k entries visible
-    (1, 1, 9000, 4 * 9000 - 1, 4, 1000, 8, False),    # long row, exact ties in blocks of 8 around the cut
+    (1, 1, 9000, 4 * 9000 - 1, 4, 1003, 8, False),    # long row, a block of 8 exact ties straddling the cut
     # prefill rows at k = 2048 (row path): visible counts crossing k, and near 16384
     (1, 300, 16384, 8000, 4, 2048, 0, False),
     (1, 300, 16384, 65536 - 300, 4, 2048, 0, False),
