@@ -34,3 +34,21 @@ def test_gpus_flag_must_match_the_launched_ranks():
     assert r.returncode == 2, (r.returncode, r.stderr[-2000:])
     assert "--gpus 2" in r.stderr
     assert not [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_prefill_timing_rotates_past_l2():
+    """Prefill workloads whose per-step inputs and outputs fit in the 126 MB L2 are timed over a rotation of
+    copies whose total exceeds it; larger ones use a single set.  The reference arm describes the same."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from long_context_sparse_10_b200 import synth
+    for name in ("csa_prefill_t2048", "hca_prefill_t8192"):
+        wl = synth.WORKLOADS[name]
+        run = bench.PrefillRun.__new__(bench.PrefillRun)  # host inputs only, no GPU
+        run.wl, run.host, run.csa_kind = wl, synth.prefill_inputs(wl, seed=0), wl.kind == "csa"
+        set_bytes, nsets = run.rotation()
+        host = sum(v.numel() * v.element_size() for v in run.host.values())
+        assert set_bytes == host + wl.B * wl.T * wl.H * (128 * 2 + 4)
+        assert nsets * set_bytes > 126e6 and (nsets == 1 or (nsets - 1) * set_bytes < 1.5 * 126e6)
+        l2 = run.describe(1)["l2"]
+        assert ("rotate" in l2) == (nsets > 1), l2
