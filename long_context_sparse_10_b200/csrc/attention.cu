@@ -1301,12 +1301,18 @@ struct QbBlock {
   int64_t b, r0, t0, tl, wlo0, nwin;
   int nq;
 };
+// a / b for a >= 0, b > 0: a 32-bit division when both fit (the 64-bit one is
+// emulated and costs more than the rest of a block's geometry)
+__device__ __forceinline__ int64_t qb_div(int64_t a, int64_t b) {
+  if (((a | b) >> 32) == 0) return static_cast<uint32_t>(a) / static_cast<uint32_t>(b);
+  return a / b;
+}
 __device__ __forceinline__ QbBlock qb_block(const AttnParams& p, int64_t blk) {
   const int QB = 256 / p.H;
   const int64_t nblk = (p.Tq + QB - 1) / QB;
   QbBlock k;
-  k.b = blk / nblk;
-  k.r0 = (blk % nblk) * QB;  // first query row of the block within its sequence
+  k.b = qb_div(blk, nblk);
+  k.r0 = (blk - k.b * nblk) * QB;  // first query row of the block within its sequence
   k.nq = static_cast<int>((p.Tq - k.r0) < QB ? (p.Tq - k.r0) : QB);
   k.t0 = p.q_pos0 + k.r0;
   k.tl = k.t0 + k.nq - 1;
@@ -1316,7 +1322,7 @@ __device__ __forceinline__ QbBlock qb_block(const AttnParams& p, int64_t blk) {
 }
 // Dense entry run of a block: the entries visible to its last query.
 __device__ __forceinline__ int64_t qb_dense_entries(const AttnParams& p, const QbBlock& k) {
-  const int64_t n = (k.tl + 1) / p.stride;
+  const int64_t n = qb_div(k.tl + 1, p.stride);
   return n < p.N ? n : p.N;
 }
 
@@ -1609,7 +1615,7 @@ __global__ void __launch_bounds__(kQbThreads, 1) attn_qblock_kernel(AttnParams p
       // this row's output (the block geometry is not needed past this point)
       const int64_t orow = (k.b * p.Tq + k.r0) * H + r;
       const int64_t tq = k.t0 + (row_ok ? qr : 0);
-      int64_t nv_q = (tq + 1) / p.stride;
+      int64_t nv_q = qb_div(tq + 1, p.stride);
       if (nv_q > p.N) nv_q = p.N;
       const int64_t lo_q = (tq - p.wlen + 1) > 0 ? (tq - p.wlen + 1) : 0;
       // slot numbers (below 2^31): the entry run, this row's visible entries and window slots
