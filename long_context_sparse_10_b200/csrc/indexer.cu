@@ -18,12 +18,12 @@
 //   * rows whose visible prefix fits in shared memory (prefill) run one CTA
 //     per row over the row held in shared memory;
 //   * long rows (decode over 10^5..10^6 entries) get a 4096-bin histogram of
-//     the key's top 12 bits fused into the scoring kernel; one select kernel
-//     then derives each row's threshold bin from it (in every CTA), emits a
-//     bitmap of the entries above that bin plus a candidate list of the bin
-//     itself, and its last CTA per row resolves the candidates and writes the
-//     ascending list.  "Last CTA" is decided by an atomic counter (no CTA ever
-//     waits).
+//     the key's top 12 bits fused into the scoring kernel; a classifying
+//     kernel then derives each row's threshold bin from it (in every CTA) and
+//     emits a bitmap of the entries above that bin, their count per chunk and
+//     a candidate list of the bin itself; an emitting kernel resolves the cut
+//     among the candidates (in every CTA of the row) and writes the ascending
+//     list, each CTA its own span of the row.  No CTA ever waits for another.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -691,7 +691,7 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
   if (E4) cp_async_wait<0>();
   pdl_trigger();  // the next kernel may be scheduled while the histograms merge
 
-  // flush the CTA histogram; the row's last CTA then derives its threshold
+  // flush the CTA histogram
   __syncthreads();
   uint32_t* gh = p.hist + row * kHistBins;
   for (int j = threadIdx.x; j < kHistBins / 2; j += kLongThreads) {
@@ -699,8 +699,8 @@ __global__ void __launch_bounds__(kLongThreads) score_long_kernel(LongScoreParam
     if (c & 0xffffu) atomicAdd(gh + 2 * j, c & 0xffffu);
     if (c >> 16) atomicAdd(gh + 2 * j + 1, c >> 16);
   }
-  // (the select kernel derives each row's threshold from the complete histogram
-  // once this grid has finished: no counter, no waiting CTA)
+  // (the classifying kernel derives each row's threshold from the complete
+  // histogram once this grid has finished: no counter, no waiting CTA)
 }
 
 // ---------------------------------------------------------------------------
@@ -1313,49 +1313,49 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
 }
 
 // ---------------------------------------------------------------------------
-// long-row path: histogram + threshold fused into scoring, then one select
-// kernel whose last CTA per row resolves the threshold bin and writes the list
+// long-row path: histogram fused into scoring, then two select kernels.  The
+// first classifies every entry against the row's threshold bin (bitmap words
+// for the entries above it, a candidate list of the entries in it, a count of
+// the entries above it per chunk).  The second resolves the cut inside the
+// bin and writes the ascending list: every CTA its own span of the row, at the
+// offset of the selected entries before the span.
 // ---------------------------------------------------------------------------
 constexpr int kSelThreads = 512;
-constexpr int kSelChunk = 8192;         // entries per select CTA
-constexpr int kCandSmem = 4096;         // threshold-bin candidates kept in shared memory
-constexpr int kBitmapSmemWords = 8192;  // rows up to 262144 entries emit from a shared-memory bitmap
-// The shared-memory bitmap leaves 4 words free after every 16, so that lanes
-// reading their 16 consecutive words as four 16-byte vectors (the emission
-// pass) do not collide on banks.
-__host__ __device__ constexpr int bm_pad(int64_t wi) { return static_cast<int>(wi + 4 * (wi >> 4)); }
-constexpr int kBitmapSmemPadded = kBitmapSmemWords + kBitmapSmemWords / 4;
+constexpr int kSelChunk = 8192;                 // entries per classifying CTA
+constexpr int kCandSmem = 4096;                 // threshold-bin candidates kept in shared memory
+constexpr int kEmitThreads = 512;
+constexpr int kEmitWords = 2 * kEmitThreads;    // bitmap words per emitting CTA, two per thread
+constexpr int kEmitSpan = 32 * kEmitWords;      // entries per emitting CTA
+static_assert(kEmitSpan % kSelChunk == 0, "an emitting span covers whole classifying chunks");
 
 struct LongWs {
   float* scores;        // [R, pitch] (pitch = N rounded up to 4: 16-byte aligned rows)
   uint32_t* hist;       // [R, kHistBins]    (zeroed per call)
   uint32_t* cand_cnt;   // [R]               (zeroed per call)
-  uint32_t* done;       // [R]: select CTAs finished (zeroed per call)
+  int2* rinfo;          // [R]: (threshold bin, entries still needed from it)
+  uint32_t* ccnt;       // [R, nch]: entries above the threshold bin, per chunk
   uint2* cand;          // [R, N]: (key, index) of the threshold bin's entries
-  uint32_t* bitmap;     // [R, W]
+  uint32_t* bitmap;     // [R, W]: bit e set when entry e lies above the threshold bin
   int64_t W;
   int64_t pitch;
+  int64_t nch;          // chunks per row, ceil(N / kSelChunk)
 };
 
-// Per CTA: the row's threshold bin from its complete histogram (every CTA of
-// the row derives it, its score loads already in flight), then a bitmap word
-// for every 32 entries (entries above the threshold bin), and the threshold
-// bin's entries appended to the row's candidate list (gathered in shared
-// memory first, one global atomic per CTA).  The last CTA
-// of a row then radix-selects the `need` best candidates on the composite key
-// (score key << 32 | ~index), merges them into the row's bitmap and writes the
-// ascending index list.  Rows up to kBitmapSmemWords*32 entries keep that final
-// bitmap in shared memory.
-__global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, int64_t N, int64_t Tq, int64_t q_pos0,
-                                                                     int m, int k, int32_t* __restrict__ idx,
-                                                                     float* __restrict__ scores_out) {
+// Per CTA (one chunk of a row): the row's threshold bin from its complete
+// histogram (every CTA of the row derives it, its score loads already in
+// flight), then a bitmap word for every 32 entries (entries above the
+// threshold bin), the chunk's count of such entries, and the threshold bin's
+// entries appended to the row's candidate list (gathered in shared memory
+// first, one global atomic per CTA).  Rows with no more visible entries than
+// k are written here whole.
+__global__ void __launch_bounds__(kSelThreads, 2) topk_classify_kernel(LongWs ws, int64_t N, int64_t Tq,
+                                                                       int64_t q_pos0, int m, int k,
+                                                                       int32_t* __restrict__ idx,
+                                                                       float* __restrict__ scores_out) {
   pdl_wait();
-  extern __shared__ __align__(16) uint8_t sel_smem[];  // candidates, then the final bitmap
+  extern __shared__ __align__(16) uint8_t sel_smem[];  // candidates of the chunk
   uint2* cand_s = reinterpret_cast<uint2*>(sel_smem);
-  uint32_t* bm_s = reinterpret_cast<uint32_t*>(sel_smem + kCandSmem * sizeof(uint2));
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t dig[3];
-  __shared__ uint32_t n_cand, base_s, last_s;
+  __shared__ uint32_t n_cand, n_above, base_s;
   __shared__ int32_t thr_s[2];
   __shared__ uint32_t scan_sh[32];
   const int64_t row = blockIdx.y;
@@ -1389,9 +1389,13 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
   }
   // the threshold bin and the count still needed from it (nv > k: a bin exists)
   row_threshold<kSelThreads>(ws.hist + row * kHistBins, nv, k, thr_s, scan_sh);
-  if (threadIdx.x == 0) n_cand = 0;
+  if (threadIdx.x == 0) {
+    n_cand = 0;
+    n_above = 0;
+  }
   __syncthreads();
   const uint32_t tb = static_cast<uint32_t>(thr_s[0]);
+  uint32_t n_up = 0;  // entries above the threshold bin seen by this lane
 #pragma unroll
   for (int it = 0; it < kSteps; ++it) {
     const int64_t base = e_begin + warp * kPerWarp + it * 128;  // a multiple of 32
@@ -1406,6 +1410,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
       above |= (ok && bin > tb) ? (1u << u) : 0u;
       cand_bits |= (ok && bin == tb) ? (1u << u) : 0u;
     }
+    n_up += __popc(above);
     // bitmap word of entries [32 j, 32 j + 32): lanes 8j .. 8j+7, four bits each
     uint32_t word = above << (4 * (lane & 7));
     word |= __shfl_xor_sync(0xffffffffu, word, 1);
@@ -1437,98 +1442,108 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
       }
     }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) n_up += __shfl_xor_sync(0xffffffffu, n_up, o);
+  if (lane == 0 && n_up) atomicAdd(&n_above, n_up);
   __syncthreads();
   const uint32_t nc = n_cand < static_cast<uint32_t>(kCandSmem) ? n_cand : static_cast<uint32_t>(kCandSmem);
-  if (threadIdx.x == 0 && nc) base_s = atomicAdd(ws.cand_cnt + row, nc);
+  if (threadIdx.x == 0) {
+    if (nc) base_s = atomicAdd(ws.cand_cnt + row, nc);
+    ws.ccnt[row * ws.nch + blockIdx.x] = n_above;
+    if (blockIdx.x == 0) ws.rinfo[row] = make_int2(thr_s[0], thr_s[1]);
+  }
+  pdl_trigger();  // the emitting kernel may be scheduled while the candidates are stored
   __syncthreads();
   for (uint32_t c = threadIdx.x; c < nc; c += kSelThreads) ws.cand[row * N + base_s + c] = cand_s[c];
-  pdl_trigger();  // only the rows' last CTAs still have work
-  // last CTA of this row?
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t chunks = static_cast<uint32_t>((nv + kSelChunk - 1) / kSelChunk);
-    last_s = (atomicAdd(ws.done + row, 1u) == chunks - 1) ? 1u : 0u;
-  }
-  __syncthreads();
-  if (!last_s) return;
-  __threadfence();
+}
 
-  // ---- load the row's candidates (when they fit) and bitmap (when it fits)
-  // together.  Warp w owns the bitmap words [w * per_warp, (w + 1) * per_warp)
-  // and counts their bits as it loads them (wcnt), so the final emission
-  // needs no separate counting pass.
+// Per CTA (one span of kEmitSpan entries of a row whose visible entries
+// outnumber k): radix-selects the `need` best threshold-bin candidates on the
+// composite key (score key << 32 | ~index, so equal scores go to the lower
+// index), the same cut in every CTA of the row; sets the selected candidates
+// of its span in the span's bitmap words; and writes the span's selected
+// entries in ascending order at the offset of those before it (the above-bin
+// counts of the earlier chunks plus the selected candidates before the span).
+__global__ void __launch_bounds__(kEmitThreads, 1) topk_emit_kernel(LongWs ws, int64_t N, int64_t Tq,
+                                                                    int64_t q_pos0, int m, int k,
+                                                                    int32_t* __restrict__ idx,
+                                                                    float* __restrict__ scores_out) {
+  pdl_wait();
+  extern __shared__ __align__(16) uint8_t emit_smem[];
+  uint2* cand_s = reinterpret_cast<uint2*>(emit_smem);                                  // [kCandSmem]
+  uint32_t* wsm = reinterpret_cast<uint32_t*>(emit_smem + kCandSmem * sizeof(uint2));  // [kEmitWords]
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t dig[3];
+  __shared__ uint32_t before_s;  // selected entries before the span
+  __shared__ uint32_t scan_sh[32];
+  const int64_t row = blockIdx.y;
+  const int64_t nv = visible(q_pos0 + row % Tq, m, N);
+  if (nv <= k) return;  // the classifying kernel wrote the whole list
+  const int64_t e_begin = static_cast<int64_t>(blockIdx.x) * kEmitSpan;
+  if (e_begin >= nv) return;
+  const int64_t e_end = (e_begin + kEmitSpan) < nv ? (e_begin + kEmitSpan) : nv;
   const int64_t words = (nv + 31) >> 5;
+  const int64_t w_begin = e_begin >> 5;
+  const int tid = threadIdx.x, lane = tid & 31;
+  int32_t* out = idx + row * k;
+  float* sout = scores_out != nullptr ? scores_out + row * k : nullptr;
+  const float* srow = ws.scores + row * ws.pitch;
+  const uint32_t* gbm = ws.bitmap + row * ws.W;
+
+  // ---- loads in flight together: the span's bitmap words, the candidates
+  // (when they fit in shared memory), the above-bin counts of earlier chunks
   const uint32_t cnt = __ldcg(ws.cand_cnt + row);
+  const int2 ri = __ldcg(ws.rinfo + row);
   const uint2* cand = ws.cand + row * N;
-  uint32_t* gbm = ws.bitmap + row * ws.W;
-  const bool bm_in_smem = words <= kBitmapSmemWords;
   const bool cand_in_smem = cnt <= static_cast<uint32_t>(kCandSmem);
-  __shared__ uint32_t wcnt[kSelWarps];
-  // a shared-memory bitmap gives every warp 512 words (16 per lane)
-  const int64_t per_warp =
-      bm_in_smem ? kBitmapSmemWords / kSelWarps : (words + 32 * kSelWarps - 1) / (32 * kSelWarps) * 32;
-  const int64_t wb = warp * per_warp;
-  const int64_t we = (wb + per_warp) < words ? (wb + per_warp) : words;
-  // candidate loads first (in flight together with the bitmap's)
-  constexpr int kCandPerThread = kCandSmem / kSelThreads;
+  uint32_t wv[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int64_t wi = w_begin + 2 * tid + u;
+    wv[u] = wi < words ? __ldcg(gbm + wi) : 0u;
+  }
+  constexpr int kCandPerThread = kCandSmem / kEmitThreads;
   uint2 cv[kCandPerThread];
   if (cand_in_smem) {
 #pragma unroll
     for (int u = 0; u < kCandPerThread; ++u) {
-      const uint32_t c = u * kSelThreads + threadIdx.x;
+      const uint32_t c = u * kEmitThreads + tid;
       cv[u] = c < cnt ? __ldcg(cand + c) : make_uint2(0, 0);
     }
   }
-  {
-    // 16 words per lane in flight (a shared-memory bitmap has at most 512 words per warp)
-    uint32_t bits = 0;
-    for (int64_t w0 = wb; w0 < we; w0 += 16 * 32) {
-      uint32_t v[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int64_t wi = w0 + u * 32 + lane;
-        v[u] = wi < we ? __ldcg(gbm + wi) : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int64_t wi = w0 + u * 32 + lane;
-        if (wi == words - 1 && (nv & 31)) v[u] &= (1u << (nv & 31)) - 1u;
-        if (bm_in_smem && wi < we) bm_s[bm_pad(wi)] = v[u];
-        bits += __popc(v[u]);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) bits += __shfl_xor_sync(0xffffffffu, bits, o);
-    if (lane == 0) wcnt[warp] = bits;
-  }
+  const int64_t chunks_before = e_begin / kSelChunk;
+  uint32_t before = 0;
+  for (int64_t c = tid; c < chunks_before; c += kEmitThreads) before += __ldcg(ws.ccnt + row * ws.nch + c);
+  if (tid == 0) before_s = 0;
+  wsm[2 * tid] = wv[0];
+  wsm[2 * tid + 1] = wv[1];
   if (cand_in_smem) {
 #pragma unroll
     for (int u = 0; u < kCandPerThread; ++u) {
-      const uint32_t c = u * kSelThreads + threadIdx.x;
+      const uint32_t c = u * kEmitThreads + tid;
       if (c < cnt) cand_s[c] = cv[u];
     }
     cand = cand_s;
   }
   __syncthreads();
 
-  // ---- resolve the threshold bin: radix select on the 52 low composite bits
-  uint32_t remaining = static_cast<uint32_t>(thr_s[1]);
-  uint64_t prefix = static_cast<uint64_t>(tb) << 52;
+  // ---- the cut inside the threshold bin: radix select on the 52 low composite bits
+  uint32_t remaining = static_cast<uint32_t>(ri.y);
+  uint64_t prefix = static_cast<uint64_t>(static_cast<uint32_t>(ri.x)) << 52;
   uint64_t mask = 0xfffull << 52;
   uint32_t in_bucket = cnt;
   for (int pass = 0; pass < 7 && in_bucket != remaining; ++pass) {
     const int sh = pass < 6 ? 44 - 8 * pass : 0;
     const uint64_t dmask = pass < 6 ? 255ull : 15ull;
-    for (int j = threadIdx.x; j < 256; j += kSelThreads) hist[j] = 0;
+    for (int j = tid; j < 256; j += kEmitThreads) hist[j] = 0;
     __syncthreads();
-    for (uint32_t c = threadIdx.x; c < cnt; c += kSelThreads) {
+    for (uint32_t c = tid; c < cnt; c += kEmitThreads) {
       const uint2 kv = cand_in_smem ? cand[c] : __ldcg(cand + c);
       const uint64_t x = (static_cast<uint64_t>(kv.x) << 32) | (0xffffffffu - kv.y);
       if ((x & mask) == prefix) atomicAdd(&hist[(x >> sh) & dmask], 1u);
     }
     __syncthreads();
-    if (threadIdx.x < 32) find_digit_256(hist, remaining, dig);
+    if (tid < 32) find_digit_256(hist, remaining, dig);
     __syncthreads();
     prefix |= static_cast<uint64_t>(dig[0]) << sh;
     mask |= dmask << sh;
@@ -1536,90 +1551,38 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_select_kernel(LongWs ws, 
     in_bucket = dig[2];
     __syncthreads();
   }
-  for (uint32_t c = threadIdx.x; c < cnt; c += kSelThreads) {
+  // ---- selected candidates: counted before the span, set in its words inside it
+  for (uint32_t c = tid; c < cnt; c += kEmitThreads) {
     const uint2 kv = cand_in_smem ? cand[c] : __ldcg(cand + c);
     const uint64_t x = (static_cast<uint64_t>(kv.x) << 32) | (0xffffffffu - kv.y);
-    if ((x & mask) >= prefix) {  // a threshold-bin entry: its bit is not set yet
-      atomicOr(bm_in_smem ? bm_s + bm_pad(kv.y >> 5) : gbm + (kv.y >> 5), 1u << (kv.y & 31));
-      atomicAdd(&wcnt[(kv.y >> 5) / per_warp], 1u);
-    }
-  }
-  if (!bm_in_smem) __threadfence();
-  __syncthreads();
-
-  // ---- ascending list from the bitmap: each warp emits its own word range
-  // at the offset of the bits before it; within the warp each lane takes
-  // per_warp / 32 consecutive words (one count pass, one scan, one emit pass).
-  uint32_t pos = 0;
-  for (int w = 0; w < warp; ++w) pos += wcnt[w];
-  const int64_t per_lane = per_warp / 32;
-  const int64_t lb = wb + lane * per_lane;
-  const int64_t le = (lb + per_lane) < we ? (lb + per_lane) : we;
-  if (bm_in_smem) {  // 16 words per lane, in registers
-    static_assert(kBitmapSmemWords / kSelWarps == 16 * 32, "16 bitmap words per lane");
-    uint32_t wv[16];
-    const uint4* src = reinterpret_cast<const uint4*>(bm_s + bm_pad(lb));
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 v = src[j];
-      wv[4 * j] = v.x;
-      wv[4 * j + 1] = v.y;
-      wv[4 * j + 2] = v.z;
-      wv[4 * j + 3] = v.w;
-    }
-    uint32_t c = 0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int64_t wi = lb + j;
-      if (wi >= words) wv[j] = 0u;
-      if (wi == words - 1 && (nv & 31)) wv[j] &= (1u << (nv & 31)) - 1u;
-      c += __popc(wv[j]);
-    }
-    uint32_t incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    uint32_t p = pos + incl - c;
-    const int32_t e0 = static_cast<int32_t>(lb << 5);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      uint32_t word = wv[j];
-      while (word) {
-        const int bit = __ffs(word) - 1;
-        word &= word - 1;
-        if (p < static_cast<uint32_t>(k)) {
-          out[p] = e0 + 32 * j + bit;
-          if (sout != nullptr) sout[p] = __ldcg(srow + e0 + 32 * j + bit);
-        }
-        ++p;
+    if ((x & mask) >= prefix) {
+      if (static_cast<int64_t>(kv.y) < e_begin) {
+        ++before;
+      } else if (static_cast<int64_t>(kv.y) < e_end) {
+        atomicOr(&wsm[(kv.y >> 5) - w_begin], 1u << (kv.y & 31));
       }
     }
-    return;
   }
-  uint32_t c = 0;
-  for (int64_t wi = lb; wi < le; ++wi) {
-    uint32_t word = __ldcg(gbm + wi);
-    if (wi == words - 1 && (nv & 31)) word &= (1u << (nv & 31)) - 1u;
-    c += __popc(word);
-  }
-  uint32_t incl = c;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  uint32_t p = pos + incl - c;
-  for (int64_t wi = lb; wi < le && p < static_cast<uint32_t>(k); ++wi) {
-    uint32_t word = __ldcg(gbm + wi);
-    if (wi == words - 1 && (nv & 31)) word &= (1u << (nv & 31)) - 1u;
+  for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+  if (lane == 0 && before) atomicAdd(&before_s, before);
+  __syncthreads();
+
+  // ---- ascending emission: thread t owns words 2t and 2t + 1 of the span
+  const uint32_t a = wsm[2 * tid], b = wsm[2 * tid + 1];
+  uint32_t total;
+  uint32_t p = before_s + block_excl_scan(__popc(a) + __popc(b), &total, scan_sh);
+  const int64_t e0 = (w_begin + 2 * tid) << 5;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    uint32_t word = u ? b : a;
     while (word) {
       const int bit = __ffs(word) - 1;
       word &= word - 1;
       if (p < static_cast<uint32_t>(k)) {
-        out[p] = static_cast<int32_t>((wi << 5) + bit);
-        if (sout != nullptr) sout[p] = __ldcg(srow + (wi << 5) + bit);
+        const int64_t e = e0 + 32 * u + bit;
+        out[p] = static_cast<int32_t>(e);
+        if (sout != nullptr) sout[p] = __ldcg(srow + e);
       }
       ++p;
     }
@@ -1641,21 +1604,23 @@ constexpr int64_t kPrefillTcMaxN = 65535;
 bool use_prefill_tc(int64_t R, int64_t N) { return N <= kPrefillTcMaxN && R >= 32LL * num_sms(); }
 
 struct LongLayout {
-  size_t scores, hist, cnt, done, zero_end, cand, bitmap, total;
-  int64_t W, pitch;
+  size_t scores, hist, cnt, zero_end, rinfo, ccnt, cand, bitmap, total;
+  int64_t W, pitch, nch;
 };
 
 LongLayout long_layout(int64_t R, int64_t N) {
   LongLayout L;
   L.W = ((N + 31) / 32 + 15) / 16 * 16;  // 16-word multiple: vector reads stay in the row
   L.pitch = (N + 3) / 4 * 4;
+  L.nch = (N + kSelChunk - 1) / kSelChunk;
   size_t off = 0;
   L.scores = off; off = align_up(off + static_cast<size_t>(R) * L.pitch * 4);
-  L.hist = off;   off += static_cast<size_t>(R) * kHistBins * 4;     // hist, cnt and done: zeroed together
+  L.hist = off;   off += static_cast<size_t>(R) * kHistBins * 4;     // hist and cnt: zeroed together
   L.cnt = off;    off += static_cast<size_t>(R) * 4;
-  L.done = off;   off += static_cast<size_t>(R) * 4;
   L.zero_end = off;
   off = align_up(off);
+  L.rinfo = off;  off = align_up(off + static_cast<size_t>(R) * 8);
+  L.ccnt = off;   off = align_up(off + static_cast<size_t>(R) * L.nch * 4);
   L.cand = off;   off = align_up(off + static_cast<size_t>(R) * N * 8);
   L.bitmap = off; off = align_up(off + static_cast<size_t>(R) * L.W * 4);
   L.total = off;
@@ -1893,11 +1858,13 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
   w.scores = reinterpret_cast<float*>(ws + L.scores);
   w.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
   w.cand_cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
-  w.done = reinterpret_cast<uint32_t*>(ws + L.done);
+  w.rinfo = reinterpret_cast<int2*>(ws + L.rinfo);
+  w.ccnt = reinterpret_cast<uint32_t*>(ws + L.ccnt);
   w.cand = reinterpret_cast<uint2*>(ws + L.cand);
   w.bitmap = reinterpret_cast<uint32_t*>(ws + L.bitmap);
   w.W = L.W;
   w.pitch = L.pitch;
+  w.nch = L.nch;
   if (cudaMemsetAsync(w.hist, 0, L.zero_end - L.hist, s) != cudaSuccess)
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: memset failed");
   CSA_REQUIRE(R < 65536, "csa_indexer_topk: too many query rows for the long-row path");
@@ -1957,13 +1924,20 @@ csa_status indexer_impl(const void* qI, const float* wI, const void* kIc, const 
                                          : launch_pdl(score_long_kernel<kKeyBF16>, grid, lblock, ssmem, s, 1, lp, kmap);
   prof_end(s);
   if (csa_status st = check_launch("indexer score (long rows)", e); st != CSA_OK) return st;
-  dim3 sgrid(static_cast<unsigned>((N + kSelChunk - 1) / kSelChunk), static_cast<unsigned>(R));
-  constexpr int kSelSmem = kCandSmem * 8 + kBitmapSmemPadded * 4;
-  if (!ensure_smem(reinterpret_cast<const void*>(topk_select_kernel), kSelSmem))
+  const dim3 cgrid(static_cast<unsigned>(L.nch), static_cast<unsigned>(R));
+  constexpr int kClassifySmem = kCandSmem * 8;
+  constexpr int kEmitSmem = kCandSmem * 8 + kEmitWords * 4;
+  if (!ensure_smem(reinterpret_cast<const void*>(topk_classify_kernel), kClassifySmem) ||
+      !ensure_smem(reinterpret_cast<const void*>(topk_emit_kernel), kEmitSmem))
     return fail(CSA_ERR_CUDA, "csa_indexer_topk: cannot raise shared memory limit");
-  return check_launch("indexer select",
-                      launch_pdl(topk_select_kernel, sgrid, dim3(kSelThreads), kSelSmem, s, 1, w, N, Tq, q_pos0, m, k, idx,
-                                 scores_out));
+  if (csa_status st = check_launch("indexer classify",
+                                   launch_pdl(topk_classify_kernel, cgrid, dim3(kSelThreads), kClassifySmem, s, 1, w, N,
+                                              Tq, q_pos0, m, k, idx, scores_out));
+      st != CSA_OK)
+    return st;
+  const dim3 egrid(static_cast<unsigned>((N + kEmitSpan - 1) / kEmitSpan), static_cast<unsigned>(R));
+  return check_launch("indexer emit", launch_pdl(topk_emit_kernel, egrid, dim3(kEmitThreads), kEmitSmem, s, 1, w, N,
+                                                 Tq, q_pos0, m, k, idx, scores_out));
 }
 }  // namespace
 }  // namespace csa
