@@ -225,6 +225,14 @@ class DecodeRun:
     # still runs all of its work; its inputs alone exceed L2)
     graph_steps = 8
 
+    @staticmethod
+    def hca_sms_for(wl):
+        """SMs the HCA branch keeps to while the CSA indexer streams its keys beside it (0 = all).  With bf16
+        indexer keys the scoring kernel streams for ~46 us, and a branch held to 80 SMs (10 CTAs of 7 tiles
+        per row) finishes inside that window: step 77.6 -> 73.6 us.  E4M3 and E2M1 keys score in 30-35 us, and
+        there the whole GPU is better (61.8 us against 64.8 us at 80 SMs)."""
+        return 80 if wl.kind == "hybrid" and not (wl.indexer_fp8 or wl.indexer_fp4) else 0
+
     def __init__(self, wl, rank, dev):
         import torch
         import long_context_sparse_10_b200 as csa
@@ -250,6 +258,7 @@ class DecodeRun:
         self.hybrid = wl.kind == "hybrid"
         if self.hybrid:
             self.side = torch.cuda.Stream(device=dev)  # the HCA branch's stream
+            self.hca_sms = self.hca_sms_for(wl)
             self.hcache = csa.KVCache(nope=d["hca_nope"], rope=d["hca_rope"], scale=d["hca_scale"])
             self.hwin = csa.Window(k=d["hca_win_k"], pos0=L - wl.win, length=wl.win)
             hws = csa.hca_dense_mqa_workspace_size(B, 1, H, wl.N_hca, wl.win)
@@ -309,7 +318,7 @@ class DecodeRun:
         if self.hybrid:
             with torch.cuda.stream(self.side):
                 csa.hca_dense_mqa(self.d["hca_q"], self.hcache, wl.m_hca, self.hwin, self.scale, q_pos0=self.q_pos0,
-                                  out=self.hout, lse=self.hlse, workspace=self.ws_hca)
+                                  out=self.hout, lse=self.hlse, workspace=self.ws_hca, max_sms=self.hca_sms)
         csa.csa_sparse_mqa(self.d["q"], self.cache, wl.m, self.idx, self.win, self.scale, q_pos0=self.q_pos0,
                            out=self.out, lse=self.lse, workspace=self.ws_attn)
         if self.hybrid:
@@ -420,6 +429,9 @@ class DecodeRun:
         if self.hybrid:
             s += f" then HCA m'={wl.m_hca} (N'={wl.N_hca}, same split cache)"
         s += f", sliding window {wl.win}"
+        if self.hybrid:
+            sms = self.hca_sms_for(wl)
+            s += "; HCA branch on a forked stream" + (f" held to {sms} SMs" if sms else "")
         return {"workload": s, "global_batch": wl.B * world, "seq_len": wl.L, "parallelism": f"dp{world} (replicas)",
                 "l2": f"inputs larger than L2 (the step streams {self.step_bytes() / 1e6:.0f} MB > 126 MB L2)",
                 "timing": f"CUDA graph replay, {self.graph_steps} whole steps captured per launch"}

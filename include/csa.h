@@ -404,6 +404,22 @@ CSA_API csa_status hca_dense_mqa(const void* q, int64_t B, int64_t Tq, int32_t H
                          size_t workspace_bytes, void* stream);
 
 /*
+ * hca_dense_mqa_budget -- hca_dense_mqa whose 64-head decode launch keeps to
+ * at most max_sms SMs (one CTA per SM on that path, at least one CTA per
+ * query row), so that work the caller runs beside it on another stream (the
+ * CSA branch's indexer, which does not depend on the HCA branch) keeps the
+ * other SMs.  max_sms = 0: every SM (identical to hca_dense_mqa).  The result
+ * is the same attention up to the summation order of the split merge; the
+ * workspace hca_dense_mqa_workspace_size reports is always enough.  Calls
+ * with at least as many query rows as SMs, 16 heads, or the query-blocked
+ * prefill kernel are unaffected.  max_sms < 0 returns CSA_ERR_INVALID_ARG.
+ */
+CSA_API csa_status hca_dense_mqa_budget(const void* q, int64_t B, int64_t Tq, int32_t H, int64_t q_pos0,
+                                const csa_kv_cache* cache, int32_t m_prime, const csa_window* win,
+                                float scale, void* out, float* lse, int32_t max_sms, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
  * csa_sparse_mqa_packed / hca_dense_mqa_packed -- the core attention over
  * packed sequences (sample-level masks): query row r is packed token r, at
  * position t within its sequence s; its entry set is drawn from s's entries

@@ -244,8 +244,11 @@ def csa_sparse_mqa(q, cache: KVCache, m, idx, win: Window | None, scale, *, q_po
 
 
 def hca_dense_mqa(q, cache: KVCache, m_prime, win: Window | None, scale, *, q_pos0=0, out=None, lse=None,
-                  workspace=None, stream=None):
-    """HCA core attention over every visible entry plus the sliding window (one softmax)."""
+                  workspace=None, stream=None, max_sms=0):
+    """HCA core attention over every visible entry plus the sliding window (one softmax).
+
+    ``max_sms`` > 0 keeps the 64-head decode launch to that many SMs (``hca_dense_mqa_budget``), leaving the
+    rest to work the caller runs beside it on another stream."""
     lib = _lib.load()
     B, Tq, H, _ = q.shape
     out, lse = _attn_out(q, out, lse)
@@ -255,10 +258,17 @@ def hca_dense_mqa(q, cache: KVCache, m_prime, win: Window | None, scale, *, q_po
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     cd = cache.desc()
     wd = win.desc() if win is not None else None
-    st = lib.hca_dense_mqa(_ptr(q), B, Tq, H, q_pos0, ctypes.byref(cd), m_prime,
-                           ctypes.byref(wd) if wd is not None else None, float(scale), _ptr(out), _ptr(lse),
-                           _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
-    _check(st, "hca_dense_mqa")
+    wsz = 0 if workspace is None else workspace.numel()
+    if max_sms:
+        st = lib.hca_dense_mqa_budget(_ptr(q), B, Tq, H, q_pos0, ctypes.byref(cd), m_prime,
+                                      ctypes.byref(wd) if wd is not None else None, float(scale), _ptr(out), _ptr(lse),
+                                      int(max_sms), _ptr(workspace), wsz, _stream(stream))
+        _check(st, "hca_dense_mqa_budget")
+    else:
+        st = lib.hca_dense_mqa(_ptr(q), B, Tq, H, q_pos0, ctypes.byref(cd), m_prime,
+                               ctypes.byref(wd) if wd is not None else None, float(scale), _ptr(out), _ptr(lse),
+                               _ptr(workspace), wsz, _stream(stream))
+        _check(st, "hca_dense_mqa")
     return out, lse
 
 

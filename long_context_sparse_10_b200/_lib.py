@@ -52,6 +52,8 @@ SIGNATURES = {
     "hca_dense_mqa_workspace_size": (c_sz, [c_i64, c_i64, c_i32, c_i64, c_i32]),
     "hca_dense_mqa": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i64, c_vp, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_sz,
                               c_vp]),
+    "hca_dense_mqa_budget": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_i64, c_vp, c_i32, c_vp, c_f32, c_vp, c_vp, c_i32,
+                                     c_vp, c_sz, c_vp]),
     "csa_grouped_out_proj": (c_i32, [c_vp, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]),
     "csa_indexer_topk_packed_workspace_size": (c_sz, [c_vp, c_i32, c_i32]),
     "csa_indexer_topk_packed": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_sz, c_vp]),

@@ -1817,14 +1817,14 @@ __global__ void __launch_bounds__(32) wait_expire_kernel(uint32_t limit) {
 // host side
 // ---------------------------------------------------------------------------
 // Splits of a row's slots for the tcgen05 kernel (one CTA per SM): rows that
-// cannot fill the device by themselves are split so that all rows' CTAs run
-// in one wave; the splits then merge through global-memory records.
+// cannot fill the `sms` SMs by themselves are split so that all rows' CTAs
+// run in one wave; the splits then merge through global-memory records.
 struct TcSplit {
   int nsplit, tps;
 };
-TcSplit tc_split(int64_t R, int64_t max_slots) {
+TcSplit tc_split(int64_t R, int64_t max_slots, int64_t sms) {
   const int64_t tiles = max_slots > 0 ? (max_slots + kTcKeys - 1) / kTcKeys : 1;
-  int64_t ns = R >= num_sms() ? 1 : num_sms() / R;
+  int64_t ns = R >= sms ? 1 : sms / R;
   if (ns < 1) ns = 1;
   if (ns > tiles) ns = tiles;
   const int64_t tps = (tiles + ns - 1) / ns;
@@ -1833,7 +1833,7 @@ TcSplit tc_split(int64_t R, int64_t max_slots) {
 }
 size_t tc_part_bytes(int64_t R, int H, int64_t max_slots) {
   if (H != 64 || R <= 0) return 0;
-  const TcSplit sp = tc_split(R, max_slots);
+  const TcSplit sp = tc_split(R, max_slots, num_sms());
   return sp.nsplit > 1 ? static_cast<size_t>(R) * sp.nsplit * H * kRec * sizeof(float) : 0;
 }
 
@@ -1948,7 +1948,7 @@ csa_status check_cache(const char* name, const csa_kv_cache* c) {
 csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H, int64_t q_pos0,
                const csa_kv_cache* cache, int32_t stride, const int32_t* idx, int32_t k, const csa_window* win,
                float scale, void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream,
-               const csa_packed* pk = nullptr) {
+               const csa_packed* pk = nullptr, int32_t max_sms = 0) {
   clear_error();
   CSA_REQUIRE(B >= 0 && Tq >= 0, "%s: negative size", name);
   CSA_REQUIRE(H == 16 || H == 64, "%s: H must be 16 or 64 (got %d)", name, H);
@@ -2012,8 +2012,12 @@ csa_status run(const char* name, const void* q, int64_t B, int64_t Tq, int32_t H
                              static_cast<int>(tc_layout(fp8, shv, 0).total)))
     return fail(CSA_ERR_CUDA, "%s: cannot raise the shared memory limit", name);
   if (use_tc) {
-    const TcSplit sp = tc_split(R, max_slots);
-    if (sp.nsplit > 1 && pl.cl > 1) {
+    // an SM budget (work beside this call on another stream keeps the rest)
+    // bounds the splits; it takes the global-record merge, whose split count
+    // follows the budget exactly
+    const int64_t sms = (max_sms > 0 && max_sms < num_sms()) ? max_sms : num_sms();
+    const TcSplit sp = tc_split(R, max_slots, sms);
+    if (sp.nsplit > 1 && pl.cl > 1 && max_sms <= 0) {
       // A cluster merge (distributed shared memory, no second kernel) wins when
       // a co-resident cluster size leaves no more tiles per CTA than the global
       // split does; with even one tile more per CTA the split and its one-round
@@ -2238,6 +2242,15 @@ csa_status hca_dense_mqa(const void* q, int64_t B, int64_t Tq, int32_t H, int64_
                          size_t workspace_bytes, void* stream) {
   return csa::run("hca_dense_mqa", q, B, Tq, H, q_pos0, cache, m_prime, nullptr, 0, win, scale, out, lse, workspace,
                   workspace_bytes, stream);
+}
+
+csa_status hca_dense_mqa_budget(const void* q, int64_t B, int64_t Tq, int32_t H, int64_t q_pos0,
+                                const csa_kv_cache* cache, int32_t m_prime, const csa_window* win, float scale,
+                                void* out, float* lse, int32_t max_sms, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  if (max_sms < 0) return csa::fail(CSA_ERR_INVALID_ARG, "hca_dense_mqa_budget: max_sms must be >= 0");
+  return csa::run("hca_dense_mqa_budget", q, B, Tq, H, q_pos0, cache, m_prime, nullptr, 0, win, scale, out, lse,
+                  workspace, workspace_bytes, stream, nullptr, max_sms);
 }
 
 }  // extern "C"

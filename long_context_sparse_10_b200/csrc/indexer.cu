@@ -1323,8 +1323,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) indexer_prefill_kernel(PfParams
 constexpr int kSelThreads = 512;
 constexpr int kSelChunk = 8192;                 // entries per classifying CTA
 constexpr int kCandSmem = 4096;                 // threshold-bin candidates kept in shared memory
-constexpr int kEmitThreads = 512;
-constexpr int kEmitWords = 2 * kEmitThreads;    // bitmap words per emitting CTA, two per thread
+#ifndef CSA_EMIT_THREADS
+#define CSA_EMIT_THREADS 512
+#endif
+#ifndef CSA_EMIT_WPT
+#define CSA_EMIT_WPT 2
+#endif
+constexpr int kEmitThreads = CSA_EMIT_THREADS;
+constexpr int kEmitWpt = CSA_EMIT_WPT;                // consecutive bitmap words per thread
+constexpr int kEmitWords = kEmitWpt * kEmitThreads;  // bitmap words per emitting CTA
 constexpr int kEmitSpan = 32 * kEmitWords;      // entries per emitting CTA
 static_assert(kEmitSpan % kSelChunk == 0, "an emitting span covers whole classifying chunks");
 
@@ -1496,10 +1503,10 @@ __global__ void __launch_bounds__(kEmitThreads, 1) topk_emit_kernel(LongWs ws, i
   const int2 ri = __ldcg(ws.rinfo + row);
   const uint2* cand = ws.cand + row * N;
   const bool cand_in_smem = cnt <= static_cast<uint32_t>(kCandSmem);
-  uint32_t wv[2];
+  uint32_t wv[kEmitWpt];
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int64_t wi = w_begin + 2 * tid + u;
+  for (int u = 0; u < kEmitWpt; ++u) {
+    const int64_t wi = w_begin + kEmitWpt * tid + u;
     wv[u] = wi < words ? __ldcg(gbm + wi) : 0u;
   }
   constexpr int kCandPerThread = kCandSmem / kEmitThreads;
@@ -1515,8 +1522,8 @@ __global__ void __launch_bounds__(kEmitThreads, 1) topk_emit_kernel(LongWs ws, i
   uint32_t before = 0;
   for (int64_t c = tid; c < chunks_before; c += kEmitThreads) before += __ldcg(ws.ccnt + row * ws.nch + c);
   if (tid == 0) before_s = 0;
-  wsm[2 * tid] = wv[0];
-  wsm[2 * tid + 1] = wv[1];
+#pragma unroll
+  for (int u = 0; u < kEmitWpt; ++u) wsm[kEmitWpt * tid + u] = wv[u];
   if (cand_in_smem) {
 #pragma unroll
     for (int u = 0; u < kCandPerThread; ++u) {
@@ -1568,14 +1575,19 @@ __global__ void __launch_bounds__(kEmitThreads, 1) topk_emit_kernel(LongWs ws, i
   if (lane == 0 && before) atomicAdd(&before_s, before);
   __syncthreads();
 
-  // ---- ascending emission: thread t owns words 2t and 2t + 1 of the span
-  const uint32_t a = wsm[2 * tid], b = wsm[2 * tid + 1];
-  uint32_t total;
-  uint32_t p = before_s + block_excl_scan(__popc(a) + __popc(b), &total, scan_sh);
-  const int64_t e0 = (w_begin + 2 * tid) << 5;
+  // ---- ascending emission: thread t owns words [t, t + 1) * kEmitWpt of the span
+  uint32_t nbits = 0;
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    uint32_t word = u ? b : a;
+  for (int u = 0; u < kEmitWpt; ++u) {
+    wv[u] = wsm[kEmitWpt * tid + u];
+    nbits += __popc(wv[u]);
+  }
+  uint32_t total;
+  uint32_t p = before_s + block_excl_scan(nbits, &total, scan_sh);
+  const int64_t e0 = (w_begin + kEmitWpt * tid) << 5;
+#pragma unroll
+  for (int u = 0; u < kEmitWpt; ++u) {
+    uint32_t word = wv[u];
     while (word) {
       const int bit = __ffs(word) - 1;
       word &= word - 1;

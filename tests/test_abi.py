@@ -74,6 +74,10 @@ def test_host_side_argument_errors(lib):
     # unknown cache layout
     cd.layout = 7
     assert lib.hca_dense_mqa(16, 1, 1, 64, 0, ctypes.byref(cd), 128, None, 0.1, 16, None, None, 0, None) == INV
+    # a negative SM budget
+    assert lib.hca_dense_mqa_budget(16, 1, 1, 64, 0, ctypes.byref(cd), 128, None, 0.1, 16, None, -1, None, 0,
+                                    None) == INV
+    assert b"max_sms" in lib.csa_last_error()
     # sparse attention needs idx
     cd.layout = 0
     assert lib.csa_sparse_mqa(16, 1, 1, 64, 0, ctypes.byref(cd), 4, None, 8, None, 0.1, 16, None, None, 0,

@@ -202,16 +202,18 @@ def _split_cache(g, B, N):
     return synth.split_fp8_cache(x)
 
 
-@pytest.mark.parametrize("kind,H,B,N,k,win,Tq", [
-    ("csa", 64, 3, 5000, 512, 128, 1), ("csa", 16, 2, 3000, 2048, 128, 1), ("hca", 64, 2, 3000, 0, 128, 1),
-    ("hca", 16, 3, 700, 0, 64, 1), ("csa", 64, 2, 4000, 256, 128, 4),
+@pytest.mark.parametrize("kind,H,B,N,k,win,Tq,max_sms", [
+    ("csa", 64, 3, 5000, 512, 128, 1, 0), ("csa", 16, 2, 3000, 2048, 128, 1, 0), ("hca", 64, 2, 3000, 0, 128, 1, 0),
+    ("hca", 16, 3, 700, 0, 64, 1, 0), ("csa", 64, 2, 4000, 256, 128, 4, 0),
     # rows split over many CTAs whose partial states merge through global records
-    ("hca", 64, 8, 8192, 0, 128, 1),   # the 1M-context decode's HCA shape: 17 CTAs per row
-    ("hca", 64, 2, 30000, 0, 128, 1),  # 59 CTAs per row, last split ragged
-    ("csa", 64, 8, 40000, 2048, 128, 1),  # the 1M-context decode's CSA shape (cluster merge)
-    ("hca", 64, 1, 30000, 0, 128, 4),  # several query rows of one sequence, each split over CTAs
+    ("hca", 64, 8, 8192, 0, 128, 1, 0),   # the 1M-context decode's HCA shape: 17 CTAs per row
+    ("hca", 64, 2, 30000, 0, 128, 1, 0),  # 59 CTAs per row, last split ragged
+    ("csa", 64, 8, 40000, 2048, 128, 1, 0),  # the 1M-context decode's CSA shape (cluster merge)
+    ("hca", 64, 1, 30000, 0, 128, 4, 0),  # several query rows of one sequence, each split over CTAs
+    # an SM budget: 10 CTAs of 7 tiles per row (last ragged), 2 CTAs per row, one CTA per row
+    ("hca", 64, 8, 8192, 0, 128, 1, 80), ("hca", 64, 8, 8192, 0, 128, 1, 16), ("hca", 64, 8, 8192, 0, 128, 1, 3),
 ])
-def test_decode_split_fp8(kind, H, B, N, k, win, Tq):
+def test_decode_split_fp8(kind, H, B, N, k, win, Tq, max_sms):
     g = np.random.default_rng(N + H + k)
     m = 4 if kind == "csa" else 128
     L = N * m
@@ -231,7 +233,7 @@ def test_decode_split_fp8(kind, H, B, N, k, win, Tq):
         O, Ls = R.csa_sparse_mqa(f64(q), q_pos0 + np.arange(Tq), K64, V64, idx, m, f64(Wk), f64(Wk)[..., :128],
                                  wpos0, win, sc)
     else:
-        out, lse = csa.hca_dense_mqa(q.to(DEV), cache, m, w, sc, q_pos0=q_pos0)
+        out, lse = csa.hca_dense_mqa(q.to(DEV), cache, m, w, sc, q_pos0=q_pos0, max_sms=max_sms)
         O, Ls = R.hca_dense_mqa(f64(q), q_pos0 + np.arange(Tq), K64, V64, m, f64(Wk), f64(Wk)[..., :128], wpos0,
                                 win, sc)
     torch.cuda.synchronize()
