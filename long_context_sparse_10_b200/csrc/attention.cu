@@ -528,9 +528,14 @@ constexpr int kTcKeys = 128;
 
 constexpr int kTcDecThreads = 544;  // attn_tc_kernel: warps 0-7 softmax, 8-15 loads, 16 MMA issue
 constexpr float kRescaleLog2 = 20.f;  // rescale O and l when a logit tops m_ref by more than 2^20
+// The first tile of a CTA tries the reference 0 for every head: kept when
+// every head has a valid logit of at least kFloorLog2 (so that the largest
+// probabilities are far from the fp32 / bf16 underflow) and none above
+// kRescaleLog2; otherwise the exact per-head maxima are reduced.
+constexpr float kFloorLog2 = -64.f;
 
 struct TcLayout {
-  size_t q, k, v, p, ones, stype, srow, mref, corr, wmax, bars, total;
+  size_t q, k, v, p, ones, stype, srow, mref, corr, wmax, hseen, bars, total;
 };
 
 // Slot types of the last four tiles (ring indexed by tile % 4): 0 skipped, 1
@@ -556,6 +561,7 @@ __host__ __device__ inline TcLayout tc_layout(bool fp8, bool shv, int tps) {
   L.mref = off; off += 64 * sizeof(float);
   L.corr = off; off += 64 * sizeof(float);
   L.wmax = off; off += 4 * 64 * sizeof(float);
+  L.hseen = off; off += 16;                      // 64 head flags of the first tile's trial reference
   L.bars = off; off += 128;
   (void)fp8, (void)tps;
   const size_t reduce = 80 * (kDV + 4) * sizeof(float);  // cluster merge records (reuse Q/K)
@@ -627,6 +633,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
   float* mref = reinterpret_cast<float*>(smem + L.mref);
   float* corr_s = reinterpret_cast<float*>(smem + L.corr);
   auto wmax = reinterpret_cast<float(*)[64]>(smem + L.wmax);
+  uint32_t* hseen = reinterpret_cast<uint32_t*>(smem + L.hseen);  // [2]: heads 0-31, 32-63
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // [NS] K stage loaded
   uint64_t* empty = full + NS;                                    // [NS] PV of the stage's tile done
   uint64_t* sdone = empty + NS;                                   // [2] S of the tile done (TMEM buffer)
@@ -687,6 +694,7 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
     if (tid < 64) {
       reinterpret_cast<uint4*>(ones)[tid] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
       mref[tid] = -INFINITY;
+      if (tid < 2) hseen[tid] = 0u;
     }
     cp_async_wait<0>();
     tc::fence_async_smem();
@@ -1075,11 +1083,26 @@ __global__ void __launch_bounds__(kTcDecThreads, 1) attn_tc_kernel(AttnParams p)
           sv[j + 3] = fmaf(sv[j + 3], p.scale_log2, -m4.w);
         }
       };
-      centre();
+      const bool trial = tile == 0;  // reference 0 for every head (see kFloorLog2)
+      if (trial) {
+        uint32_t seen = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          sv[j] *= p.scale_log2;
+          seen |= (valid && sv[j] >= kFloorLog2) ? (1u << j) : 0u;
+        }
+        seen = __reduce_or_sync(0xffffffffu, seen);
+        if (lane == 0 && seen) atomicOr(&hseen[hb >> 5], seen);
+      } else {
+        centre();
+      }
       bool over = false;
 #pragma unroll
       for (int j = 0; j < 32; ++j) over |= sv[j] > kRescaleLog2;
-      if (named_sync_or(2, 256, over && valid)) {
+      bool need = named_sync_or(2, 256, over && valid);
+      if (trial) need = need || (hseen[0] & hseen[1]) != 0xffffffffu;  // a head with no logit above the floor
+      if (!need && trial && tid < 64) mref[tid] = 0.f;  // read after this tile's closing barrier
+      if (need) {
         // new per-head maxima: this tile's maximum over its valid keys (the
         // reduction consumes sv; the logits are read again from TMEM below)
         tc::tmem_ld32(tmem + 64 * pb + lane_base + hb, sv);

@@ -241,6 +241,67 @@ def test_decode_split_fp8(kind, H, B, N, k, win, Tq, max_sms):
     assert_lse(f64(lse), Ls, f"{kind} decode lse")
 
 
+def _exact_split_cache(g, B, N, positive):
+    """Split cache whose widened keys are exact in bf16 (E4M3 codes times a power-of-two scale), so that
+    logits far from 1 do not magnify the key rounding of the tcgen05 path."""
+    codes = g.integers(0, 256, size=(B, N, 128)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] ^= 0x01  # no NaN codes
+    if positive:
+        codes &= 0x7F
+    rope = g.standard_normal((B, N, 64)).astype(np.float32)
+    if positive:
+        rope = np.abs(rope)
+    scale = np.full((B, N), 2.0 ** -7, np.float32)
+    return torch.from_numpy(codes), torch.from_numpy(rope).to(torch.bfloat16), torch.from_numpy(scale)
+
+
+@pytest.mark.parametrize("kind,case", [("csa", "large"), ("hca", "large"), ("csa", "negative"), ("hca", "negative"),
+                                       ("csa", "mixed"), ("hca", "mixed"), ("csa", "low"), ("hca", "low")])
+def test_decode_logit_ranges(kind, case):
+    """Logits outside the first tile's trial reference: above 2^20 for some heads (large), below 2^-64 for every
+    head (negative: positive keys, negative queries), or below it for half of the heads only (mixed); and
+    logits inside it but far below 0 for every head (low)."""
+    g = np.random.default_rng({"large": 1, "negative": 2, "mixed": 3, "low": 4}[case] + (10 if kind == "hca" else 0))
+    H, B, N, win = 64, 2, 3000, 128
+    m = 4 if kind == "csa" else 128
+    k = 512
+    L = N * m
+    q_pos0 = L - 1
+    positive = case != "large"
+    nope, rope, scale = _exact_split_cache(g, B, N, positive)
+    qf = g.standard_normal((B, 1, H, 192)).astype(np.float32)
+    wf = g.standard_normal((B, win + 1, 192)).astype(np.float32)
+    sc = 1 / math.sqrt(192)
+    if case == "large":
+        sc *= 16.0
+    elif case in ("negative", "low"):
+        wf = np.abs(wf)
+        qf = -np.abs(qf) * 2.0
+        sc *= 8.0 if case == "negative" else 4.0
+    else:
+        wf = np.abs(wf)
+        qf[:, :, :32] = -np.abs(qf[:, :, :32]) * 16.0
+    q = torch.from_numpy(qf).to(torch.bfloat16)
+    Wk = torch.from_numpy(wf).to(torch.bfloat16)
+    wpos0 = L - 1 - win
+    cache = csa.KVCache(nope=nope.to(DEV), rope=rope.to(DEV), scale=scale.to(DEV))
+    w = csa.Window(k=Wk.to(DEV), pos0=wpos0, length=win)
+    K64, V64 = R.dequant_split(nope.numpy(), f64(rope), scale.numpy())
+    if kind == "csa":
+        idx = _oracle_idx(g, B, 1, N, m, k, q_pos0)
+        out, lse = csa.csa_sparse_mqa(q.to(DEV), cache, m, torch.from_numpy(idx.astype(np.int32)).to(DEV), w, sc,
+                                      q_pos0=q_pos0)
+        O, Ls = R.csa_sparse_mqa(f64(q), q_pos0 + np.arange(1), K64, V64, idx, m, f64(Wk), f64(Wk)[..., :128],
+                                 wpos0, win, sc)
+    else:
+        out, lse = csa.hca_dense_mqa(q.to(DEV), cache, m, w, sc, q_pos0=q_pos0)
+        O, Ls = R.hca_dense_mqa(f64(q), q_pos0 + np.arange(1), K64, V64, m, f64(Wk), f64(Wk)[..., :128], wpos0,
+                                win, sc)
+    torch.cuda.synchronize()
+    assert_close(f64(out), O, f"{kind} decode logits {case}")
+    assert_lse(f64(lse), Ls, f"{kind} decode lse, logits {case}")
+
+
 def test_attention_with_no_keys_outputs_zero():
     g = np.random.default_rng(3)
     B, T, H, m = 1, 8, 16, 4
