@@ -107,6 +107,26 @@ def test_workspace_sizes_are_monotone(lib):
     assert lib.csa_indexer_topk_workspace_size(0, 1, 10, 4) == 0
 
 
+def test_long_row_indexer_workspace_layout(lib):
+    """Decode rows (long-row path): fp32 scores (rows padded to 4 entries), the 4096-bin histograms and
+    candidate counters (zeroed per call), the per-row threshold pair and per-8192-entry-chunk counts, the
+    (key, index) candidate lists and the bitmaps (rows padded to 16 words), each region 256-byte aligned."""
+    def up(x):
+        return (x + 255) // 256 * 256
+
+    for R, N in ((8, 262144), (64, 32768), (2, 300001), (3, 50000)):
+        pitch = (N + 3) // 4 * 4
+        W = ((N + 31) // 32 + 15) // 16 * 16
+        nch = -(-N // 8192)
+        off = up(R * pitch * 4)
+        off = up(off + R * 4096 * 4 + R * 4)
+        off = up(off + R * 8)
+        off = up(off + R * nch * 4)
+        off = up(off + R * N * 8)
+        off = up(off + R * W * 4)
+        assert lib.csa_indexer_topk_workspace_size(R, 1, N, 2048) == off, (R, N)
+
+
 def test_attention_workspace_rule(lib):
     """H = 64 rows too few to fill the device split their keys over several
     CTAs and need merge records; H = 16, many rows, or one tile need none."""
