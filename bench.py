@@ -920,23 +920,37 @@ def reference_arm(args):
         run.host = synth.prefill_inputs(wl, seed=0)
         run.csa_kind = wl.kind == "csa"
     budget = min(240.0, max(5.0, args.cpu_sample_s * 20))
-    per_step = budget / max(1, args.steps + args.warmup)
-    for _ in range(args.warmup):
+    warm, timed = args.warmup, max(1, args.steps)
+    # a step is at least one unit of oracle work (a whole sequence for decode, 64 query rows for prefill):
+    # the first unit (a warm-up step when W >= 1) gives its cost, and when W + K such steps would outrun
+    # the budget, fewer steps are timed (one warm-up at most), as the line states
+    _, unit_s, _ = run.oracle_sample(0.0)
+    warm = max(0, warm - 1)
+    fit = int(budget / max(unit_s, 1e-3))
+    if warm + timed > fit:
+        warm = min(warm, 1)
+        timed = max(1, min(timed, fit - warm))
+    per_step = budget / (warm + timed)
+    for _ in range(warm):
         run.oracle_sample(per_step)
     total_n, total_s, sample = 0, 0.0, ""
-    for _ in range(args.steps):
+    for _ in range(timed):
         n, spent, sample = run.oracle_sample(per_step)
         total_n += n
         total_s += spent
     value = total_n / total_s
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / max(1, args.steps),
+            "steps": timed, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / timed,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": run.describe(args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                              "sample": sample + f"; each step a sample of about {per_step:.1f} s",
                              "host_cpus": os.cpu_count()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if timed != args.steps:
+        line["steps_requested"] = args.steps
+        line["cpu_baseline"]["sample"] += (f"; {timed} of the {args.steps} requested steps timed (each step is at "
+                                           f"least one unit of {unit_s:.2f} s, the run is bounded to {budget:.0f} s)")
     print(json.dumps(line), flush=True)
 
 
