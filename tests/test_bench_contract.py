@@ -52,3 +52,21 @@ def test_prefill_timing_rotates_past_l2():
         assert nsets * set_bytes > 126e6 and (nsets == 1 or (nsets - 1) * set_bytes < 1.5 * 126e6)
         l2 = run.describe(1)["l2"]
         assert ("rotate" in l2) == (nsets > 1), l2
+
+
+def test_decode_description_states_graph_steps_and_hca_budget():
+    """The decode line names how many whole steps one graph launch holds and, for the hybrid step with bf16
+    indexer keys, the SM budget of its HCA branch (the E4M3 / E2M1 steps keep every SM for it)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from long_context_sparse_10_b200 import synth
+    expect = {"hybrid_decode_l1m": 80, "hybrid_decode_l1m_fp8idx": 0, "hybrid_decode_l1m_fp4idx": 0,
+              "csa_decode_l131072": 0}
+    for name, sms in expect.items():
+        wl = synth.WORKLOADS[name]
+        assert bench.DecodeRun.hca_sms_for(wl) == sms, name
+        run = bench.DecodeRun.__new__(bench.DecodeRun)  # no GPU
+        run.wl, run.hybrid = wl, wl.kind == "hybrid"
+        cfg = run.describe(1)
+        assert cfg["timing"] == f"CUDA graph replay, {bench.DecodeRun.graph_steps} whole steps captured per launch"
+        assert ("held to 80 SMs" in cfg["workload"]) == (sms == 80), cfg["workload"]
